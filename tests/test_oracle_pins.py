@@ -1,0 +1,497 @@
+"""Pins for the CPU oracle: checks against facts fixed outside the oracle.
+
+Each test pins one oracle function to something it does not compute itself:
+published known-answer vectors, closed forms, textbook special cases,
+invariants, brute force on tiny inputs and Monte-Carlo statistics with their
+exact standard errors.  A plausible mistake in the oracle (a dropped term, a
+wrong sign or index, a transposed operand) fails at least one of them.
+"""
+
+import math
+import os
+
+import numpy as np
+import pytest
+from scipy import integrate, special, stats
+
+from oracle import tq_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# --------------------------------------------------------------------------
+# Generator
+# --------------------------------------------------------------------------
+
+
+def _read_kat():
+    rows = []
+    with open(os.path.join(GOLDEN, "philox4x32_10_kat.txt")) as f:
+        for line in f:
+            line = line.split("#")[0].strip()
+            if line:
+                rows.append([int(x, 16) for x in line.split()])
+    return rows
+
+
+def test_philox_known_answers():
+    for row in _read_kat():
+        out = O.philox4x32_10(np.array([row[:4]], dtype=np.uint64), row[4:6])[0]
+        assert [int(x) for x in out] == row[6:10]
+
+
+def test_gaussian_stream_is_standard_normal():
+    z = O.gaussian_stream(seed=7, stream=3, count=400_001)
+    assert z.shape == (400_001,)
+    assert abs(z.mean()) < 4 / math.sqrt(z.size)
+    assert abs(z.var() - 1) < 4 * math.sqrt(2 / z.size)
+    assert stats.kstest(z, "norm").pvalue > 1e-3
+
+
+def test_gaussian_streams_are_distinct_and_prefix_stable():
+    a = O.gaussian_stream(1, 0, 1000)
+    b = O.gaussian_stream(1, 1, 1000)
+    c = O.gaussian_stream(2, 0, 1000)
+    assert np.corrcoef(a, b)[0, 1] < 0.15 and np.corrcoef(a, c)[0, 1] < 0.15
+    # counter-based: a prefix does not depend on how many values follow
+    np.testing.assert_array_equal(O.gaussian_stream(1, 0, 17), a[:17])
+
+
+# --------------------------------------------------------------------------
+# Rotation
+# --------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("d", [8, 64, 128])
+def test_rotation_orthogonal_and_norm_preserving(d):
+    tb = O.make_tables(d, 3, seed=42)
+    assert np.max(np.abs(tb.R.T @ tb.R - np.eye(d))) < 1e-12
+    k = np.random.default_rng(0).standard_normal((20, d))
+    np.testing.assert_allclose(np.linalg.norm(k @ tb.R.T, axis=1), np.linalg.norm(k, axis=1), rtol=1e-13)
+
+
+def test_rotation_is_qr_factor_with_positive_diagonal():
+    d = 16
+    G = O.gaussian_stream(5, 0, d * d).reshape(d, d)
+    R = O.haar_rotation(G)
+    T = R.T @ G                               # must be upper triangular, positive diagonal
+    assert np.max(np.abs(np.tril(T, -1))) < 1e-12
+    assert np.all(np.diag(T) > 0)
+
+
+def test_rotated_coordinates_follow_the_beta_law():
+    # For a fixed unit vector and Haar R, each coordinate of R k follows f_d.
+    d, nseed = 16, 4000
+    k = np.zeros(d)
+    k[0] = 1.0
+    u = np.array([O.make_tables(d, 2, seed=s).R @ k for s in range(nseed)])
+    assert abs(u[:, 3].mean()) < 4 / math.sqrt(d * nseed)
+    assert abs(u.var() - 1 / d) < 0.05 / d
+    cdf = lambda x: O.coord_cdf(x, d)
+    assert stats.kstest(u[:, 5], cdf).pvalue > 1e-3
+
+
+# --------------------------------------------------------------------------
+# Coordinate law
+# --------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("d", [3, 4, 9, 64, 128])
+def test_density_normalised_and_cdf_consistent(d):
+    tot, _ = integrate.quad(lambda x: float(O.coord_density(x, d)), -1, 1, limit=200)
+    assert abs(tot - 1) < 1e-9
+    for x in (-0.3, 0.05, 0.2):
+        part, _ = integrate.quad(lambda s: float(O.coord_density(s, d)), -1, x, limit=200)
+        assert abs(part - float(O.coord_cdf(x, d))) < 1e-9
+        mom, _ = integrate.quad(lambda s: s * float(O.coord_density(s, d)), x, 0.9, limit=200)
+        assert abs(mom - float(O.coord_first_moment(x, 0.9, d))) < 1e-10
+
+
+def test_large_d_law_tends_to_gaussian():
+    d = 20000
+    x = np.linspace(-3, 3, 13) / math.sqrt(d)
+    np.testing.assert_allclose(O.coord_cdf(x, d), stats.norm.cdf(x * math.sqrt(d)), atol=2e-4)
+
+
+# --------------------------------------------------------------------------
+# Lloyd-Max codebook
+# --------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("bmse", [1, 2, 3, 4])
+def test_codebook_d3_is_the_uniform_quantizer(bmse):
+    # d = 3: f_3 is uniform on [-1, 1]; the optimal quantizer is uniform.
+    c, t = O.lloyd_max_codebook(3, bmse)
+    L = 1 << bmse
+    np.testing.assert_allclose(c, -1 + (2 * np.arange(L) + 1) / L, atol=1e-12)
+    np.testing.assert_allclose(t, -1 + 2 * np.arange(1, L) / L, atol=1e-12)
+
+
+@pytest.mark.parametrize("d", [3, 8, 64, 128, 200])
+def test_codebook_one_bit_closed_form(d):
+    c, t = O.lloyd_max_codebook(d, 1)
+    c1 = math.exp(special.gammaln(d / 2) - special.gammaln((d + 1) / 2)) / math.sqrt(math.pi)
+    np.testing.assert_allclose(c, [-c1, c1], rtol=1e-12)
+    assert t[0] == 0.0
+
+
+def test_codebook_one_bit_value_at_d128():
+    c, _ = O.lloyd_max_codebook(128, 1)
+    assert abs(math.sqrt(128) * c[1] - 0.79944) < 1e-5
+
+
+def _max_table():
+    out = {}
+    with open(os.path.join(GOLDEN, "gaussian_lloyd_max_levels.txt")) as f:
+        for line in f:
+            line = line.split("#")[0].strip()
+            if line:
+                L, vals = line.split(":")
+                out[int(L)] = [float(v) for v in vals.split()]
+    return out
+
+
+@pytest.mark.parametrize("bmse", [1, 2, 3])
+def test_codebook_tends_to_max_gaussian_levels(bmse):
+    ref = _max_table()[1 << bmse]
+    d = 200000
+    c, _ = O.lloyd_max_codebook(d, bmse)
+    pos = math.sqrt(d) * c[len(c) // 2:]
+    np.testing.assert_allclose(pos, ref, atol=1.5e-3)
+
+
+@pytest.mark.parametrize("d,bmse", [(8, 2), (64, 3), (128, 2), (128, 3), (128, 4), (200, 1)])
+def test_codebook_is_a_lloyd_fixed_point(d, bmse):
+    c, t = O.lloyd_max_codebook(d, bmse)
+    assert np.all(np.diff(c) > 0)
+    np.testing.assert_allclose(t, 0.5 * (c[:-1] + c[1:]), atol=1e-15)
+    # centroid condition, checked with quadrature rather than the closed form
+    edges = np.concatenate([[-1.0], t, [1.0]])
+    for i in range(len(c)):
+        num, _ = integrate.quad(lambda x: x * float(O.coord_density(x, d)), edges[i], edges[i + 1],
+                                epsabs=1e-14, epsrel=1e-12, limit=200)
+        den, _ = integrate.quad(lambda x: float(O.coord_density(x, d)), edges[i], edges[i + 1],
+                                epsabs=1e-14, epsrel=1e-12, limit=200)
+        assert abs(num / den - c[i]) < 1e-10
+    np.testing.assert_allclose(c, -c[::-1], atol=0)
+
+
+@pytest.mark.parametrize("d", [3, 5, 8])
+@pytest.mark.parametrize("bmse", [1, 2])
+def test_codebook_matches_exhaustive_boundary_search(d, bmse):
+    # Minimise the MSE over all symmetric boundary sets on a grid (L <= 4).
+    c, t = O.lloyd_max_codebook(d, bmse)
+
+    def mse_for_bounds(tb):
+        cc = O.lloyd_centroids(np.asarray(tb), d)
+        return O.mse_distortion(cc, np.asarray(tb), d)
+
+    if bmse == 1:
+        grid = np.arange(-300, 301) * 1e-3
+        best = min(grid, key=lambda a: mse_for_bounds([a]))
+        fine = np.arange(-10, 11) * 1e-4 + best
+        best = min(fine, key=lambda a: mse_for_bounds([a]))
+        assert abs(best - t[0]) < 1.5e-4
+        return
+    grid = np.arange(1, 1000) * 1e-3
+    best = min(grid, key=lambda a: mse_for_bounds([-a, 0.0, a]))
+    fine = np.arange(-10, 11) * 1e-4 + best
+    best = min(fine, key=lambda a: mse_for_bounds([-a, 0.0, a]))
+    assert abs(best - t[2]) < 1.5e-4
+
+
+def test_mse_decreases_and_sits_between_the_bounds():
+    d = 128
+    D = []
+    for bmse in (1, 2, 3, 4):
+        c, t = O.lloyd_max_codebook(d, bmse)
+        D.append(O.mse_distortion(c, t, d))
+    assert all(a > b for a, b in zip(D, D[1:]))
+    for b, v in enumerate(D, start=1):
+        # information-theoretic lower bound 4^-b; the pages quote a factor of about 2.7 above it
+        assert 4.0 ** -b <= v <= 2.72 * 4.0 ** -b
+
+
+@pytest.mark.parametrize("d", [8, 128])
+def test_one_bit_distortion_closed_form(d):
+    c, t = O.lloyd_max_codebook(d, 1)
+    assert abs(O.mse_distortion(c, t, d) - (1 - d * c[1] ** 2)) < 1e-9
+
+
+def test_quantize_mse_matches_the_distortion_integral():
+    d, bits = 128, 3
+    tb = O.make_tables(d, bits, seed=3)
+    K = np.random.default_rng(1).standard_normal((20000, d))
+    q = O.quantize(K, tb)
+    err = np.sum((q.u - tb.c[q.codes]) ** 2, axis=1).mean()
+    ref = O.mse_distortion(tb.c, tb.t, d)
+    assert abs(err - ref) < 4 * 0.01 * ref
+
+
+# --------------------------------------------------------------------------
+# Quantize: brute force on tiny inputs, edge cases
+# --------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("d,bits", [(4, 3), (6, 2), (8, 2)])
+def test_cell_search_equals_exhaustive_nearest_codeword(d, bits):
+    import itertools
+
+    tb = O.make_tables(d, bits, seed=11, m=4)
+    K = np.random.default_rng(2).standard_normal((40, d))
+    q = O.quantize(K, tb)
+    L = len(tb.c)
+    combos = np.array(list(itertools.product(range(L), repeat=d)))
+    recon = tb.c[combos]                                      # (L^d, d)
+    u = (K @ tb.R.T) / np.linalg.norm(K, axis=1, keepdims=True)
+    best = combos[np.argmin(((u[:, None, :] - recon[None]) ** 2).sum(-1), axis=1)]
+    np.testing.assert_array_equal(q.codes, best)
+
+
+def test_quantize_residual_and_signs_by_definition():
+    d, bits = 8, 3
+    tb = O.make_tables(d, bits, seed=4, m=16)
+    k = np.random.default_rng(3).standard_normal(d) * 3.0
+    q = O.quantize(k[None], tb)
+    n = np.linalg.norm(k)
+    khat = n * sum(tb.c[q.codes[0, j]] * tb.R[j] for j in range(d))   # sum_j c_j R_j. (rows of R)
+    r = k - khat
+    np.testing.assert_allclose(q.rho[0], np.linalg.norm(r), rtol=1e-13)
+    z = np.array([sum(tb.S[i, j] * r[j] for j in range(d)) for i in range(16)])
+    np.testing.assert_array_equal(q.bits[0], z >= 0)
+    # S = P R has the distribution of a Gaussian: its rows are P's rows rotated
+    np.testing.assert_allclose(tb.S @ tb.R.T, tb.P, atol=1e-12)
+
+
+def test_zero_key_and_boundary_ties():
+    d = 64
+    tb = O.make_tables(d, 3, seed=9)
+    q = O.quantize(np.zeros((2, d)), tb)
+    assert np.all(q.codes == 0) and np.all(q.bits) and np.all(q.n16 == 0) and np.all(q.rho16 == 0)
+    # a coordinate exactly on a boundary takes the lower cell: move boundary t_i onto a computed u_j
+    k = np.random.default_rng(5).standard_normal(d)
+    u = O.quantize(k[None], tb).u[0]
+    j = int(np.argmin(np.abs(u - tb.t[1])))
+    t = tb.t.copy()
+    t[1] = u[j]
+    assert t[0] < t[1] < t[2]
+    tb2 = O.Tables(d=d, bits=3, m=d, R=tb.R, P=tb.P, S=tb.S, c=tb.c, t=t)
+    assert O.quantize(k[None], tb2).codes[0, j] == 1
+    t[1] = np.nextafter(u[j], -1)
+    assert O.quantize(k[None], tb2).codes[0, j] == 2
+
+
+def test_fp16_norm_rounding_is_single_rounding_to_nearest_even():
+    one = 1.0
+    assert np.float64(one + 2.0 ** -11).astype(np.float16) == np.float16(1.0)            # tie -> even
+    assert np.float64(one + 3 * 2.0 ** -11).astype(np.float16) == np.float16(1 + 2.0 ** -9)
+    # just above a midpoint: a double rounding through fp32 would give 1.0
+    v = np.float64(one + 2.0 ** -11 + 2.0 ** -40)
+    assert v.astype(np.float16) == np.float16(1 + 2.0 ** -10)
+    assert np.float64(70000.0).astype(np.float16) == np.float16(np.inf)
+
+
+# --------------------------------------------------------------------------
+# Estimator: unbiasedness (QJL), the 2/pi bias of the 1-bit MSE quantizer,
+# and the exact dequantisation identity
+# --------------------------------------------------------------------------
+
+
+def test_qjl_two_dim_expectation_matches_quadrature():
+    # d = 2, m = 1: E[sign(s.r) (s.q)] = sqrt(2/pi) <r, q> / ||r|| for s ~ N(0, I2).
+    r = np.array([0.6, -0.2])
+    q = np.array([0.3, 0.9])
+    f = lambda b, a: np.sign(a * r[0] + b * r[1]) * (a * q[0] + b * q[1]) * math.exp(-(a * a + b * b) / 2) / (2 * math.pi)
+    val, _ = integrate.dblquad(f, -9, 9, -9, 9, epsabs=1e-10)
+    assert abs(val - math.sqrt(2 / math.pi) * r @ q / np.linalg.norm(r)) < 1e-6
+
+
+def test_qjl_term_unbiased_over_1e5_seeds_d128():
+    """Mean QJL estimate of <r, q> over 10^5 independent Gaussian S (R fixed).
+
+    The 10^5 seeds of m = 128 rows are evaluated as batches of 1000 seeds,
+    i.e. one oracle call with 128 000 rows per batch: the estimator's
+    average over all rows equals the average of the per-seed estimates.
+    Standard error from the closed-form variance
+    rho^2 / m ((pi/2) ||q||^2 - <r/||r||, q>^2).
+    """
+    d, m, nseed, per = 128, 128, 100_000, 1000
+    rng = np.random.default_rng(123)
+    base = O.make_tables(d, 3, seed=1)
+    k = rng.standard_normal(d) * (1 + 5 * (np.arange(d) < 4))
+    qv = rng.standard_normal(d)
+    total = 0.0
+    for b in range(nseed // per):
+        P = rng.standard_normal((m * per, d))
+        tb = O.Tables(d=d, bits=3, m=m * per, R=base.R, P=P, S=P @ base.R, c=base.c, t=base.t)
+        qz = O.quantize(k[None], tb)
+        # the QJL term of the estimator alone: feed codes whose levels are zero
+        tb0 = O.Tables(d=d, bits=3, m=m * per, R=base.R, P=P, S=tb.S, c=np.zeros_like(base.c), t=base.t)
+        s, _ = O.estimate(qv[None], qz.codes, qz.bits, qz.n, qz.rho, tb0)
+        total += s[0, 0]
+    mean = total / (nseed // per)
+    r = k - qz.n[0] * (base.c[qz.codes[0]] @ base.R)
+    rho = np.linalg.norm(r)
+    var = rho ** 2 / m * ((math.pi / 2) * qv @ qv - (r @ qv / rho) ** 2)
+    se = math.sqrt(var / nseed)
+    assert abs(mean - r @ qv) < 3 * se
+
+
+def test_full_estimator_unbiased_with_r_and_s_redrawn():
+    d, bits, nseed = 32, 3, 4000
+    rng = np.random.default_rng(5)
+    k = rng.standard_normal(d) * 2
+    qv = rng.standard_normal(d)
+    est = []
+    for s in range(nseed):
+        tb = O.make_tables(d, bits, seed=1000 + s)
+        qz = O.quantize(k[None], tb)
+        v, _ = O.estimate(qv[None], qz.codes, qz.bits, qz.n, qz.rho, tb)
+        est.append(v[0, 0])
+    est = np.array(est)
+    se = est.std(ddof=1) / math.sqrt(nseed)
+    assert abs(est.mean() - k @ qv) < 3 * se
+
+
+def test_one_bit_mse_estimator_bias_factor():
+    """The MSE-only 1-bit estimator is biased: E = d c1(d)^2 <q, k>, -> 2/pi.
+
+    Derivation: with u = R k/||k||, c[idx] = c1 sign(u); Rq = <q,k/||k||> u + w,
+    E[w | u] = 0, so E[<c[idx], Rq>] = c1 E|u|_1 <q, k>/||k|| and E|u_j| = c1.
+    """
+    d, nseed = 16, 20000
+    rng = np.random.default_rng(8)
+    k = rng.standard_normal(d)
+    qv = rng.standard_normal(d)
+    c, _ = O.lloyd_max_codebook(d, 1)
+    factor = d * c[1] ** 2
+    est = []
+    for s in range(nseed):
+        G = rng.standard_normal((d, d))
+        R = O.haar_rotation(G)
+        tb = O.Tables(d=d, bits=2, m=d, R=R, P=np.zeros((d, d)), S=np.zeros((d, d)), c=c, t=np.array([0.0]))
+        qz = O.quantize(k[None], tb)
+        v, _ = O.estimate(qv[None], qz.codes, qz.bits, qz.n, qz.rho * 0, tb)
+        est.append(v[0, 0])
+    est = np.array(est)
+    se = est.std(ddof=1) / math.sqrt(nseed)
+    assert abs(est.mean() - factor * (k @ qv)) < 3.5 * se
+    c128, _ = O.lloyd_max_codebook(128, 1)
+    assert abs(128 * c128[1] ** 2 - 0.6391) < 1e-4
+    cbig, _ = O.lloyd_max_codebook(10 ** 6, 1)
+    assert abs(10 ** 6 * cbig[1] ** 2 - 2 / math.pi) < 1e-6
+
+
+def test_dequantize_full_reproduces_the_estimator_exactly():
+    d, bits = 64, 4
+    tb = O.make_tables(d, bits, seed=21)
+    rng = np.random.default_rng(6)
+    K = rng.standard_normal((50, d))
+    Q = rng.standard_normal((7, d))
+    qz = O.quantize(K, tb)
+    s, A = O.estimate(Q, qz.codes, qz.bits, qz.n16, qz.rho16, tb)
+    xh = O.dequantize(qz.codes, qz.bits, qz.n16, qz.rho16, tb, full=True)
+    np.testing.assert_allclose(Q @ xh.T, s, atol=1e-12 * A.max())
+    # MSE-only reconstruction is the first term alone
+    xm = O.dequantize(qz.codes, qz.bits, qz.n16, qz.rho16, tb, full=False)
+    tb0 = O.Tables(d=d, bits=bits, m=d, R=tb.R, P=tb.P, S=tb.S * 0, c=tb.c, t=tb.t)
+    s0, _ = O.estimate(Q, qz.codes, qz.bits, qz.n16, qz.rho16, tb0)
+    np.testing.assert_allclose(Q @ xm.T, s0, atol=1e-12 * A.max())
+
+
+def test_estimator_with_zero_residual_is_the_mse_term():
+    d = 64
+    tb = O.make_tables(d, 3, seed=2)
+    codes = np.random.default_rng(0).integers(0, 4, (5, d))
+    K = 2.5 * (tb.c[codes] @ tb.R)            # keys that sit exactly on reconstruction points
+    K /= np.linalg.norm(K, axis=1, keepdims=True)
+    K *= 2.5
+    qz = O.quantize(K * 1.0, tb)
+    qv = np.random.default_rng(1).standard_normal((3, d))
+    s, _ = O.estimate(qv, qz.codes, qz.bits, qz.n, qz.rho, tb)
+    n = np.linalg.norm(K, axis=1)
+    exact = qv @ (n[:, None] * (tb.c[qz.codes] @ tb.R)).T
+    assert np.all(qz.rho < 1e-12 * n + 0.3 * n)   # residual small relative to the key
+    np.testing.assert_allclose(s, exact + (O.QJL_CONST / d) * qz.rho * ((qv @ tb.S.T) @ (2.0 * qz.bits - 1).T),
+                               rtol=1e-12, atol=1e-12)
+
+
+def test_estimator_error_shrinks_with_bits():
+    d = 128
+    rng = np.random.default_rng(9)
+    K = rng.standard_normal((400, d))
+    Q = rng.standard_normal((8, d))
+    exact = Q @ K.T
+    errs = []
+    for bits in (2, 3, 4, 5):
+        tb = O.make_tables(d, bits, seed=31)
+        qz = O.quantize(K, tb)
+        s, _ = O.estimate(Q, qz.codes, qz.bits, qz.n16, qz.rho16, tb)
+        errs.append(np.sqrt(np.mean((s - exact) ** 2)))
+    assert all(a > b for a, b in zip(errs, errs[1:]))
+
+
+def test_topk_order_and_tie_rule():
+    d = 64
+    tb = O.make_tables(d, 3, seed=2)
+    rng = np.random.default_rng(4)
+    K = rng.standard_normal((300, d))
+    K[200] = K[17]                            # exact duplicate -> identical score, lower id first
+    qz = O.quantize(K, tb)
+    Q = K[17:18] + 0.01 * rng.standard_normal((1, d))
+    ids, sc, s, _ = O.topk(Q, qz.codes, qz.bits, qz.n16, qz.rho16, tb, k=10)
+    assert ids[0, 0] == 17 and list(ids[0]).index(200) == list(ids[0]).index(17) + 1
+    assert np.all(np.diff(sc[0]) <= 0)
+    np.testing.assert_array_equal(np.sort(s[0])[::-1][:10], sc[0])
+
+
+def test_gqa_logits_head_mapping():
+    d, B, Hkv, G, S = 64, 2, 2, 3, 20
+    tb = O.make_tables(d, 3, seed=2)
+    rng = np.random.default_rng(4)
+    K = rng.standard_normal((B, Hkv, S, d))
+    q = rng.standard_normal((B, Hkv * G, d))
+    qz = O.quantize(K.reshape(-1, d), tb)
+    sh = (B, Hkv, S)
+    out, _ = O.gqa_logits(q, qz.codes.reshape(*sh, d), qz.bits.reshape(*sh, d),
+                          qz.n16.reshape(sh), qz.rho16.reshape(sh), tb, scale=0.5)
+    b, h, s = 1, 4, 7
+    ref, _ = O.estimate(q[b, h][None], qz.codes.reshape(*sh, d)[b, h // G, s][None],
+                        qz.bits.reshape(*sh, d)[b, h // G, s][None], qz.n16.reshape(sh)[b, h // G, s][None],
+                        qz.rho16.reshape(sh)[b, h // G, s][None], tb)
+    assert abs(out[b, h, s] - 0.5 * ref[0, 0]) < 1e-12
+
+
+# --------------------------------------------------------------------------
+# Packed layout
+# --------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("d,m,bmse", [(64, 64, 1), (64, 64, 2), (128, 128, 3), (128, 128, 2),
+                                      (128, 64, 4), (256, 128, 3)])
+def test_pack_unpack_round_trip(d, m, bmse):
+    rng = np.random.default_rng(d + m + bmse)
+    codes = rng.integers(0, 1 << bmse, (33, d))
+    bits = rng.integers(0, 2, (33, m)).astype(bool)
+    p = O.pack_rows(codes, bits, bmse)
+    assert p.shape == (33, O.row_bytes(d, m, bmse))
+    c2, b2 = O.unpack_rows(p, d, m, bmse)
+    np.testing.assert_array_equal(c2, codes)
+    np.testing.assert_array_equal(b2, bits)
+
+
+def test_pack_layout_hand_example():
+    # d = m = 64, b' = 3: chunk q has 3 code halfwords and 1 sign halfword (8 bytes).
+    d = m = 64
+    codes = np.zeros((1, d), dtype=np.int64)
+    bits = np.zeros((1, m), dtype=bool)
+    codes[0, 16 + 4 * 1 + 2] = 5        # quarter 1, register 1, nibble 2 -> H1 of chunk 1, bits 8..10 = 101
+    codes[0, 4 * 3 + 1] = 6             # quarter 0, register 3, nibble 1: bit i of 6 -> H_i bit 7
+    bits[0, 48 + 4 * 2 + 3] = True      # quarter 3, sign register 2, nibble 3 -> bit 14 of chunk 3's sign halfword
+    p = O.pack_rows(codes, bits, 3)[0].view("<u2")
+    want = np.zeros(16, dtype=np.uint16)
+    want[4 + 1] = 0b101 << 8
+    want[0 + 1] |= 1 << 7
+    want[0 + 2] |= 1 << 7
+    want[12 + 3] = 1 << 14
+    np.testing.assert_array_equal(p, want)
