@@ -1,0 +1,342 @@
+"""Benchmark of the TurboQuant hot path on B200 (one JSON line on rank 0).
+
+Workload (the decode configuration the headline metric is quoted on):
+  Llama-3.1-8B-shaped decode layer: batch 8, 8 KV heads, 32 query heads
+  (GQA 4), head_dim 128, seq 32768; bf16 keys N(0,1) x per-(KV head, channel)
+  lognormal(0,1) scales with 2% of channels x20; b = 4 (3 Lloyd-Max bits + 1
+  QJL bit, m = 128); one fp32 query token per sequence.
+
+A step is one pass of the whole path over one batch: quantize all
+8 x 8 x 32768 keys into a packed cache (tq_quantize) and score the 32 query
+heads against a packed cache (tq_logits: query preparation + logits).  The
+logits of step i read the cache written in step i-1, so neither kernel reads
+data it wrote itself in the same step; the keys (537 MB) and the packed cache
+(143 MB) are larger than L2, and 680 MB of other traffic separate a cache's
+write from its read.  Per-GPU work is fixed (weak scaling): with --gpus N each
+rank runs the full workload; there is no data-path collective.
+
+--impl reference runs the CPU oracle (test infrastructure) on a bounded sample
+of the same workload on the host cores, on rank 0 only.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = json.load(open(os.path.join(ROOT, "BASELINE.json")))["metric"] if os.path.exists(
+    os.path.join(ROOT, "BASELINE.json")) else "tq_logits keys scored/s"
+
+B, HKV, HQ, D, S, BITS = 8, 8, 32, 128, 32768, 4
+SEED_KEYS, SEED_TABLES = 1001, 42
+WORKLOAD = "decode_llama31_8b_layer_b8_hkv8_hq32_d128_s32768_b4"
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        j = json.load(open(p))
+        return j["hbm_gbs"], j["bf16_tflops"], j.get("bf16_tflops_sustained"), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def bytes_per_key():
+    row = D * (BITS - 1) // 8 + D // 8
+    return {"quantize_in": 2 * D, "quantize_out": row + 4, "logits_in": row + 4, "logits_out": 4 * (HQ // HKV)}
+
+
+def cpu_baseline(budget_s: float = 12.0, max_keys: int = 1 << 19):
+    """The oracle, as it stands, on a bounded sample of the workload (host cores)."""
+    import numpy as np
+    from threadpoolctl import threadpool_info
+
+    from compressed_kv_cache_tq_b200 import workloads as W
+    from oracle import tq_oracle as O
+
+    tb = O.make_tables(D, BITS, SEED_TABLES)
+    scales = W.head_channel_scales(HKV, D, SEED_KEYS)
+    q = W.queries((B, HQ, D), seed=SEED_KEYS + 7)
+    G = HQ // HKV
+    chunk = 8192
+    done, t0 = 0, time.perf_counter()
+    for b in range(B):
+        for h in range(HKV):
+            keys = W.decode_keys_pair(b, h, S, D, scales, SEED_KEYS)
+            import torch
+
+            kb = torch.from_numpy(keys).to(torch.bfloat16).to(torch.float64).numpy()
+            for s0 in range(0, S, chunk):
+                qz = O.quantize(kb[s0:s0 + chunk], tb)
+                O.estimate(q[b, h * G:(h + 1) * G].astype(np.float64), qz.codes, qz.bits, qz.n16, qz.rho16, tb)
+                done += min(chunk, S - s0)
+                if time.perf_counter() - t0 > budget_s or done >= max_keys:
+                    break
+            if time.perf_counter() - t0 > budget_s or done >= max_keys:
+                break
+        if time.perf_counter() - t0 > budget_s or done >= max_keys:
+            break
+    dt = time.perf_counter() - t0
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    return {"value": done / dt, "unit": "keys/s", "cores": threads, "kind": "oracle",
+            "sample": f"{done} of {B * HKV * S} keys (quantize + 4-head estimates), {dt:.1f} s, fp64 numpy"}
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return 0
+    budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        cpu_baseline(budget_s=min(budget, 3.0), max_keys=8192)
+    vals = []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        vals.append(cpu_baseline(budget_s=budget, max_keys=1 << 16))
+    dt = time.perf_counter() - t0
+    v = sum(x["value"] for x in vals) / len(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "keys/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * dt / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": WORKLOAD, "sample": "bounded CPU sample per step"},
+            "cpu_baseline": {"value": v, "unit": "keys/s", "cores": vals[0]["cores"], "kind": "oracle",
+                             "sample": vals[-1]["sample"]},
+            "e2e": {"value": v, "unit": "keys/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank)
+    if args.warmup < 3:
+        args.warmup = 3
+
+    import torch
+
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    from compressed_kv_cache_tq_b200 import tq, workloads as W
+
+    dev = torch.device("cuda", local)
+    ctx = tq.tq_init(D, BITS, SEED_TABLES)
+    keys = W.decode_keys(B, HKV, S, D, SEED_KEYS, device=dev).reshape(-1, D)
+    n = keys.shape[0]
+    q = torch.from_numpy(W.queries((B, HQ, D), seed=SEED_KEYS + 7)).to(dev)
+    caches = [(torch.empty((n, ctx.row_bytes), dtype=torch.uint8, device=dev),
+               torch.empty((n, 2), dtype=torch.float16, device=dev)) for _ in range(2)]
+    out = torch.empty((B, HQ, S), dtype=torch.float32, device=dev)
+    ws = torch.empty(tq.tq_logits_workspace_bytes(ctx, B, HQ, HKV), dtype=torch.uint8, device=dev)
+    scale = 1.0 / math.sqrt(D)
+    stream = torch.cuda.current_stream()
+
+    # fill both caches once so the first logits read valid data
+    for c in caches:
+        tq.tq_quantize(ctx, keys, c[0], c[1])
+
+    ev = []
+
+    def step(i, record):
+        cw, cr = caches[i % 2], caches[(i + 1) % 2]
+        if record:
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            e[0].record(stream)
+        tq.tq_quantize(ctx, keys, cw[0], cw[1])
+        if record:
+            e[1].record(stream)
+        tq.tq_logits(ctx, q, cr[0], cr[1], HKV, scale=scale, out=out, workspace=ws)
+        if record:
+            e[2].record(stream)
+            ev.append(e)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for i in range(args.warmup):
+        step(i, False)
+    barrier()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        t_start.record(stream)
+        for i in range(args.steps):
+            step(i, True)
+        t_end.record(stream)
+        barrier()
+    ms = t_start.elapsed_time(t_end)
+    if dist is not None:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    assert tq.tq_check_device_status(ctx) == 0, "a kernel reported a device-side error"
+    ms_step = ms / args.steps
+    q_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / len(ev)
+    l_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / len(ev)
+
+    # end to end through the public API: pinned host keys in, logits out
+    host_keys = torch.empty(keys.shape, dtype=keys.dtype, pin_memory=True)
+    host_keys.copy_(keys)
+    host_q = q.cpu().pin_memory()
+    host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    dkeys = torch.empty_like(keys)
+    dq = torch.empty_like(q)
+
+    def e2e_step(i):
+        cw, cr = caches[i % 2], caches[(i + 1) % 2]
+        dkeys.copy_(host_keys, non_blocking=True)
+        dq.copy_(host_q, non_blocking=True)
+        tq.tq_quantize(ctx, dkeys, cw[0], cw[1])
+        tq.tq_logits(ctx, dq, cr[0], cr[1], HKV, scale=scale, out=out, workspace=ws)
+        host_out.copy_(out, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 10))
+    for i in range(3):
+        e2e_step(i)
+    barrier()
+    a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    b_.record(stream)
+    barrier()
+    e2e_ms = a.elapsed_time(b_) / e2e_steps
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    hbm, tf, tf_sus, src = peaks()
+    bpk = bytes_per_key()
+    q_bytes = n * (bpk["quantize_in"] + bpk["quantize_out"])
+    l_bytes = n * (bpk["logits_in"] + bpk["logits_out"])
+    kernels = {
+        "tq_quantize": {"ms": q_ms, "bytes": q_bytes, "GB/s": q_bytes / q_ms / 1e6,
+                        "vectors_per_s": n / q_ms * 1e3,
+                        "flops": n * (2 * D * D + 2 * D * D), "TFLOP/s": n * 4 * D * D / q_ms / 1e9},
+        "tq_logits": {"ms": l_ms, "bytes": l_bytes, "GB/s": l_bytes / l_ms / 1e6, "keys_per_s": n / l_ms * 1e3,
+                      "pct_of_8TBs": 100 * l_bytes / l_ms / 1e6 / 8000.0},
+    }
+    dom = "tq_quantize" if q_ms >= l_ms else "tq_logits"
+    ach = kernels[dom]["GB/s"]
+    line = {
+        "metric": METRIC,
+        "value": world * n / ms_step * 1e3,
+        "unit": "keys/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "global_batch": B * world, "seq_len": S, "kv_heads": HKV,
+                   "q_heads": HQ, "head_dim": D, "bits": BITS, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2: keys 537 MB, packed cache 143 MB; logits read the cache "
+                         "written one step earlier"},
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": hbm, "unit": "GB/s",
+                     "frac": ach / hbm, "peak_source": src, "traffic": None},
+        "kernels": kernels,
+        "logits_keys_per_s": world * n / l_ms * 1e3,
+        "quantize_vectors_per_s": world * n / q_ms * 1e3,
+        "e2e": {"value": world * n / e2e_ms * 1e3, "unit": "keys/s",
+                "h2d_bytes_per_step": int(keys.numel() * 2 + q.numel() * 4),
+                "d2h_bytes_per_step": int(out.numel() * 4)},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline()
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,244 @@
+"""Thin ctypes binding of libtq (include/tq.h): argument marshalling only.
+
+Every step of the path runs in libtq's CUDA kernels.  torch provides device
+memory and the current stream.  There is no fallback: if libtq.so is missing
+or no CUDA device is present, the calls raise.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtq.so")
+
+TQ_F32, TQ_BF16 = 0, 1
+
+_STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape or type", 3: "CUDA error",
+           4: "out of memory", 5: "workspace too small", 6: "device-side error"}
+
+
+class TQError(RuntimeError):
+    def __init__(self, status: int, what: str, detail: str = ""):
+        self.status = status
+        super().__init__(f"{what}: {_STATUS.get(status, status)} {detail}".strip())
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libtq.so (built in-tree by compressed_kv_cache_tq_b200.build)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run `python -m compressed_kv_cache_tq_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, i64, u32, u64, f32, sz = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_uint32,
+                                           ctypes.c_uint64, ctypes.c_float, ctypes.c_size_t)
+        sig = {
+            "tq_init": (i32, [i32, i32, u64, ctypes.POINTER(vp)]),
+            "tq_init_ex": (i32, [i32, i32, i32, u64, u32, ctypes.POINTER(vp)]),
+            "tq_free": (None, [vp]),
+            "tq_host_tables": (i32, [i32, i32, i32, u64, u32, vp, vp, vp, vp]),
+            "tq_info": (i32, [vp, ctypes.POINTER(i32), ctypes.POINTER(i32), ctypes.POINTER(i32),
+                              ctypes.POINTER(i32)]),
+            "tq_export_tables": (i32, [vp, vp, vp, vp, vp]),
+            "tq_quantize": (i32, [vp, vp, i32, i64, i64, vp, vp, vp]),
+            "tq_dequantize": (i32, [vp, vp, vp, i64, i32, vp, vp]),
+            "tq_logits_workspace_bytes": (sz, [vp, i32, i32, i32]),
+            "tq_logits": (i32, [vp, vp, i32, i32, i32, i64, vp, vp, f32, vp, vp, sz, vp]),
+            "tq_topk_workspace_bytes": (sz, [vp, i64, i64, i32]),
+            "tq_topk": (i32, [vp, vp, i64, vp, vp, i64, i32, vp, vp, vp, sz, vp]),
+            "tq_check_device_status": (i32, [vp, vp, ctypes.POINTER(u32)]),
+            "tq_strerror": (ctypes.c_char_p, [i32]),
+            "tq_last_cuda_error": (ctypes.c_char_p, []),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+EXPORTED = ["tq_init", "tq_init_ex", "tq_host_tables", "tq_free", "tq_info", "tq_export_tables", "tq_quantize", "tq_dequantize",
+            "tq_logits_workspace_bytes", "tq_logits", "tq_topk_workspace_bytes", "tq_topk",
+            "tq_check_device_status", "tq_strerror", "tq_last_cuda_error"]
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        detail = ""
+        if status == 3:
+            detail = lib().tq_last_cuda_error().decode()
+        raise TQError(status, what, detail)
+
+
+def _stream(stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need_cuda(t: torch.Tensor, name: str):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+class Context:
+    """A quantizer: R, S, codebook for (d, bits, m, seed) on the current device."""
+
+    def __init__(self, d: int, bits: int, seed: int, m: int | None = None, stream_base: int = 0):
+        if not torch.cuda.is_available():
+            raise RuntimeError("libtq needs a CUDA device")
+        torch.cuda.current_device()            # make the device's primary context current
+        h = ctypes.c_void_p()
+        _check(lib().tq_init_ex(d, bits, d if m is None else m, seed, stream_base, ctypes.byref(h)), "tq_init")
+        self._h = h
+        self.d, self.bits, self.m, self.row_bytes = self.info()
+        self.seed = seed
+
+    @property
+    def handle(self):
+        return self._h
+
+    def info(self):
+        d, b, m, rb = (ctypes.c_int() for _ in range(4))
+        _check(lib().tq_info(self._h, ctypes.byref(d), ctypes.byref(b), ctypes.byref(m), ctypes.byref(rb)),
+               "tq_info")
+        return d.value, b.value, m.value, rb.value
+
+    def export_tables(self):
+        import numpy as np
+
+        L = 1 << (self.bits - 1)
+        R = np.empty((self.d, self.d))
+        P = np.empty((self.m, self.d))
+        c = np.empty(L)
+        t = np.empty(L - 1)
+        _check(lib().tq_export_tables(self._h, R.ctypes.data, P.ctypes.data, c.ctypes.data, t.ctypes.data),
+               "tq_export_tables")
+        return R, P, c, t
+
+    def close(self):
+        if getattr(self, "_h", None):
+            lib().tq_free(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def tq_host_tables(d: int, bits: int, seed: int, m: int | None = None, stream_base: int = 0):
+    """fp64 (R, P, c, t) exactly as tq_init builds them; runs on the host only."""
+    import numpy as np
+
+    m = d if m is None else m
+    L = 1 << (bits - 1)
+    R, P, c, t = np.empty((d, d)), np.empty((m, d)), np.empty(L), np.empty(L - 1)
+    _check(lib().tq_host_tables(d, bits, m, seed, stream_base, R.ctypes.data, P.ctypes.data, c.ctypes.data,
+                                t.ctypes.data), "tq_host_tables")
+    return R, P, c, t
+
+
+def tq_init(d: int, bits: int, seed: int, m: int | None = None, stream_base: int = 0) -> Context:
+    return Context(d, bits, seed, m, stream_base)
+
+
+def tq_quantize(ctx: Context, keys: torch.Tensor, payload: torch.Tensor | None = None,
+                norms: torch.Tensor | None = None, stream=None):
+    """keys (n, d) fp32/bf16 on the device -> (payload uint8 (n, row_bytes), norms fp16 (n, 2))."""
+    _need_cuda(keys, "keys")
+    if keys.dim() != 2 or keys.shape[1] != ctx.d:
+        raise ValueError("keys must be (n, d)")
+    dtype = {torch.float32: TQ_F32, torch.bfloat16: TQ_BF16}.get(keys.dtype)
+    if dtype is None:
+        raise ValueError("keys must be float32 or bfloat16")
+    n = keys.shape[0]
+    if payload is None:
+        payload = torch.empty((n, ctx.row_bytes), dtype=torch.uint8, device=keys.device)
+    if norms is None:
+        norms = torch.empty((n, 2), dtype=torch.float16, device=keys.device)
+    _check(lib().tq_quantize(ctx.handle, _ptr(keys), dtype, n, keys.stride(0), _ptr(payload), _ptr(norms),
+                             ctypes.c_void_p(_stream(stream))), "tq_quantize")
+    return payload, norms
+
+
+def tq_dequantize(ctx: Context, payload: torch.Tensor, norms: torch.Tensor, full: bool = True,
+                  out: torch.Tensor | None = None, stream=None):
+    _need_cuda(payload, "payload")
+    _need_cuda(norms, "norms")
+    n = payload.shape[0]
+    if out is None:
+        out = torch.empty((n, ctx.d), dtype=torch.float32, device=payload.device)
+    _check(lib().tq_dequantize(ctx.handle, _ptr(payload), _ptr(norms), n, int(full), _ptr(out),
+                               ctypes.c_void_p(_stream(stream))), "tq_dequantize")
+    return out
+
+
+def tq_logits_workspace_bytes(ctx: Context, B: int, Hq: int, Hkv: int) -> int:
+    return int(lib().tq_logits_workspace_bytes(ctx.handle, B, Hq, Hkv))
+
+
+def tq_logits(ctx: Context, q: torch.Tensor, payload: torch.Tensor, norms: torch.Tensor, Hkv: int,
+              scale: float = 1.0, out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+              stream=None):
+    """q (B, Hq, d) fp32; payload/norms rows ordered (B, Hkv, S) -> logits (B, Hq, S) fp32."""
+    _need_cuda(q, "q")
+    _need_cuda(payload, "payload")
+    _need_cuda(norms, "norms")
+    if q.dtype != torch.float32 or q.dim() != 3 or q.shape[2] != ctx.d:
+        raise ValueError("q must be float32 (B, Hq, d)")
+    B, Hq, _ = q.shape
+    if payload.shape[0] % (B * Hkv):
+        raise ValueError("payload rows must be B * Hkv * S")
+    S = payload.shape[0] // (B * Hkv)
+    if out is None:
+        out = torch.empty((B, Hq, S), dtype=torch.float32, device=q.device)
+    ws_bytes = tq_logits_workspace_bytes(ctx, B, Hq, Hkv)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=q.device)
+    _check(lib().tq_logits(ctx.handle, _ptr(q), B, Hq, Hkv, S, _ptr(payload), _ptr(norms), float(scale), _ptr(out),
+                           _ptr(workspace), workspace.numel(), ctypes.c_void_p(_stream(stream))), "tq_logits")
+    return out
+
+
+def tq_topk_workspace_bytes(ctx: Context, nq: int, n: int, k: int) -> int:
+    return int(lib().tq_topk_workspace_bytes(ctx.handle, nq, n, k))
+
+
+def tq_topk(ctx: Context, q: torch.Tensor, payload: torch.Tensor, norms: torch.Tensor, k: int,
+            workspace: torch.Tensor | None = None, stream=None):
+    """q (nq, d) fp32 -> (ids int64 (nq, k), scores fp32 (nq, k))."""
+    _need_cuda(q, "q")
+    _need_cuda(payload, "payload")
+    _need_cuda(norms, "norms")
+    nq, n = q.shape[0], payload.shape[0]
+    ids = torch.empty((nq, k), dtype=torch.int64, device=q.device)
+    scores = torch.empty((nq, k), dtype=torch.float32, device=q.device)
+    ws_bytes = tq_topk_workspace_bytes(ctx, nq, n, k)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=q.device)
+    _check(lib().tq_topk(ctx.handle, _ptr(q), nq, _ptr(payload), _ptr(norms), n, k, _ptr(ids), _ptr(scores),
+                         _ptr(workspace), workspace.numel(), ctypes.c_void_p(_stream(stream))), "tq_topk")
+    return ids, scores
+
+
+def tq_check_device_status(ctx: Context, stream=None) -> int:
+    w = ctypes.c_uint32()
+    st = lib().tq_check_device_status(ctx.handle, ctypes.c_void_p(_stream(stream)), ctypes.byref(w))
+    if st not in (0, 6):
+        _check(st, "tq_check_device_status")
+    return w.value

@@ -1,0 +1,167 @@
+/*
+ * tq.h -- C ABI of libtq, a B200 (sm_100a) implementation of the TurboQuant
+ * hot path: online rotate -> Lloyd-Max -> 1-bit QJL quantisation of key
+ * vectors, and unbiased inner-product estimation (attention logits, top-k)
+ * against the packed codes.
+ *
+ * Sources for what each call computes (web pages on TurboQuant):
+ *   [p2]  airosetta.com, "Google TurboQuant KV compression":
+ *         section "第一階段：PolarQuant" (random rotation from the QR of a
+ *         Gaussian matrix, Beta coordinate law, per-coordinate Lloyd-Max with a
+ *         precomputed codebook, dequantise = table lookup + inverse rotation)
+ *         and section "第二階段：QJL" (1-bit sign sketch of the residual,
+ *         unbiased inner-product estimator, O(d) per vector).
+ *   [p1]  mooersco.com news article, section 1.1 (rotation preserves the L2
+ *         norm; pseudocode "rotated = key @ rotation") and 2.2 (4-bit logits on
+ *         GPU are memory-bandwidth bound).
+ *   [p5]  zhengruan.com news, "第一步 / 第二步" (precomputed codebook; one bit
+ *         for the residual direction combined with the full-precision query).
+ *
+ * Conventions (all calls):
+ *   - Device pointers are caller-owned CUDA device memory; the library never
+ *     frees them.  Host pointers are marked "host".
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Calls are asynchronous on `stream`: the returned status covers argument
+ *     validation and the launch; the kernels' own bounded waits report into a
+ *     per-context status word read by tq_check_device_status().
+ *   - A context is immutable after tq_init and may be used from several
+ *     streams at once; calls that share output buffers must be ordered by
+ *     the caller.
+ *   - Errors never abort the process.  TQ_ERR_ARG: a null pointer, a negative
+ *     or inconsistent size, a misaligned pointer.  TQ_ERR_UNSUPPORTED: a shape
+ *     the kernels do not cover.  TQ_ERR_CUDA: a CUDA runtime error (the
+ *     message is kept in tq_last_cuda_error()).
+ *
+ * Packed layout (one row per key; the pages fix no layout, only "no
+ * per-block constants"):  d and m are multiples of 64, b' = bits - 1.
+ *   payload row = 4 quarter chunks q = 0..3 of 2 (b' d/64 + m/64) bytes.
+ *   Chunk q holds rotated coordinates j = q d/4 + 4r + e (r < d/16, e < 4) as
+ *   little-endian 16-bit halfwords: the b' code halfwords of each unit
+ *   u = 0..d/64-1 (unit u = r in [4u, 4u+4)), then one sign halfword per unit
+ *   of 16 sign coordinates.  "Nibble e" of a halfword is bits 4e..4e+3.
+ *     b'=1: H0 nibble e bit i              = code(4u+i, e)
+ *     b'=2: Hi nibble e bits 0-1 / 2-3     = code(4u+2i, e) / code(4u+2i+1, e)
+ *     b'=3: Hi nibble e bits 0-2 (i<3)     = code(4u+i, e);  bit 3 = bit i of code(4u+3, e)
+ *     signs: H nibble e bit i              = [ (S r)_{q m/4 + 4(4u+i) + e} >= 0 ]
+ *   norms: two fp16 per key, (||k||, ||r||), round to nearest even.
+ *   Rows of a cache are ordered [B][Hkv][S]; row bytes = d b'/8 + m/8.
+ */
+#ifndef TQ_H_
+#define TQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct tq_ctx tq_ctx;
+
+typedef enum {
+  TQ_OK = 0,
+  TQ_ERR_ARG = 1,
+  TQ_ERR_UNSUPPORTED = 2,
+  TQ_ERR_CUDA = 3,
+  TQ_ERR_NOMEM = 4,
+  TQ_ERR_WORKSPACE = 5,
+  TQ_ERR_DEVICE = 6
+} tq_status;
+
+typedef enum { TQ_F32 = 0, TQ_BF16 = 1 } tq_dtype;
+
+/* Build the data-oblivious parameters of one quantizer and upload them to
+ * the current CUDA device ([p2] stage 1: "rotation via QR of a Gaussian
+ * matrix", "Lloyd-Max, precomputed codebook"; [p2] stage 2: Gaussian JL
+ * matrix).  R (d x d) is the orthogonal factor, with a positive triangular
+ * diagonal, of a d x d Gaussian drawn from Philox4x32-10 stream 0 of `seed`;
+ * P (m x d) is drawn from stream 1 and the JL matrix applied to the residual
+ * is S = P R; the codebook has 2^(bits-1) Lloyd-Max levels for the law of one
+ * coordinate of a random unit vector in R^d.  m = d.
+ * d: multiple of 64, 64 <= d <= 256.  bits: 2..4 (1..3 Lloyd-Max bits + 1 QJL bit).
+ * *out receives a library-owned context; release it with tq_free.
+ * Errors: TQ_ERR_ARG (out == NULL), TQ_ERR_UNSUPPORTED (d, bits), TQ_ERR_CUDA. */
+tq_status tq_init(int d, int bits, uint64_t seed, tq_ctx** out);
+
+/* As tq_init with an explicit JL row count m (multiple of 64, <= 256) and the
+ * first Philox stream used (G from stream_base, P from stream_base + 1). */
+tq_status tq_init_ex(int d, int bits, int m, uint64_t seed, uint32_t stream_base, tq_ctx** out);
+
+/* Host only, no GPU needed: the fp64 tables tq_init_ex builds for these
+ * arguments (R d*d, P m*d, c 2^(bits-1), t 2^(bits-1)-1; host pointers, any
+ * may be NULL).  Same validation as tq_init_ex. */
+tq_status tq_host_tables(int d, int bits, int m, uint64_t seed, uint32_t stream_base, double* R, double* P,
+                         double* c, double* t);
+
+/* Release a context (NULL is ignored).  Must not race with calls using it. */
+void tq_free(tq_ctx* ctx);
+
+/* Sizes: d, bits, m and the packed payload bytes per key (host out-params,
+ * any may be NULL). */
+tq_status tq_info(const tq_ctx* ctx, int* d, int* bits, int* m, int* row_bytes);
+
+/* Copy the fp64 master tables to host memory for inspection: R (d*d,
+ * row-major), P (m*d), codebook levels c (2^(bits-1)) and boundaries t
+ * (2^(bits-1) - 1), ascending, on the unit-sphere scale.  Host pointers;
+ * any may be NULL. */
+tq_status tq_export_tables(const tq_ctx* ctx, double* R, double* P, double* c, double* t);
+
+/* Quantise n keys ([p2] stages 1 and 2): per key k (row i of `keys`, leading
+ * dimension ld elements) compute n = ||k||, u = R k / n, the Lloyd-Max cell
+ * index of every u_j, the residual r = k - n R^T c[idx], the sign bits
+ * [(S r)_i >= 0] and fp16(n), fp16(||r||), and write them in the packed
+ * layout.  keys: device, dtype TQ_F32 or TQ_BF16, 16-byte aligned, ld >= d and
+ * ld a multiple of 8.  payload: device, n * row_bytes bytes.  norms: device,
+ * n * 2 fp16 values.  A zero key gets codes 0, all sign bits 1, norms 0.
+ * n == 0 is a no-op. */
+tq_status tq_quantize(const tq_ctx* ctx, const void* keys, tq_dtype dtype, int64_t n, int64_t ld,
+                      uint8_t* payload, uint16_t* norms, void* stream);
+
+/* Reconstruct n keys from the packed layout ([p2] stage 1: look up the
+ * codebook and rotate back): out[i] = n16 R^T c[idx] when full == 0, plus the
+ * QJL term sqrt(pi/2)/m rho16 S^T sigma when full != 0 (then <q, out[i]>
+ * equals the inner-product estimate).  out: device fp32, n * d. */
+tq_status tq_dequantize(const tq_ctx* ctx, const uint8_t* payload, const uint16_t* norms, int64_t n,
+                        int full, float* out, void* stream);
+
+/* Workspace bytes tq_logits needs for B*Hq query heads (prepared queries). */
+size_t tq_logits_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv);
+
+/* Decode attention logits against a packed KV cache ([p2] stage 2
+ * estimator; [p1] 2.2 memory-bound logits):
+ *   out[b, h, s] = scale * ( n16 sum_j c[idx_j] (R q)_j
+ *                            + sqrt(pi/2)/m rho16 sum_i sigma_i (S q)_i )
+ * for q = q[b, h], key row (b, h / (Hq/Hkv), s).
+ * q: device fp32 [B, Hq, d].  payload/norms: device, rows [B, Hkv, S].
+ * out: device fp32 [B, Hq, S].  Hq must be a multiple of Hkv.
+ * workspace: device, >= tq_logits_workspace_bytes, 256-byte aligned. */
+tq_status tq_logits(const tq_ctx* ctx, const float* q, int B, int Hq, int Hkv, int64_t S,
+                    const uint8_t* payload, const uint16_t* norms, float scale, float* out,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
+/* Workspace bytes tq_topk needs for nq queries against n database rows. */
+size_t tq_topk_workspace_bytes(const tq_ctx* ctx, int64_t nq, int64_t n, int k);
+
+/* Inner-product top-k over a packed database (vector search, [p2] "GloVe
+ * recall@1@k, near-zero indexing time"): for every query the k rows with the
+ * largest estimate (same estimator as tq_logits with scale 1), ordered by
+ * score descending and id ascending on ties.  Candidates are selected with
+ * the fast estimator and re-scored in fp64 before the final order.
+ * q: device fp32 [nq, d]; ids: device int64 [nq, k]; scores: device fp32
+ * [nq, k].  1 <= k <= 256, k <= n. */
+tq_status tq_topk(const tq_ctx* ctx, const float* q, int64_t nq, const uint8_t* payload,
+                  const uint16_t* norms, int64_t n, int k, int64_t* ids, float* scores,
+                  void* workspace, size_t workspace_bytes, void* stream);
+
+/* Read (and clear) the context's device status word after synchronising the
+ * stream: 0 when every kernel finished its bounded waits, otherwise a bit set
+ * per kernel that gave up.  Returns TQ_ERR_DEVICE when nonzero. */
+tq_status tq_check_device_status(const tq_ctx* ctx, void* stream, uint32_t* word);
+
+const char* tq_strerror(tq_status s);
+const char* tq_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TQ_H_ */

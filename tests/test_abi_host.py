@@ -1,0 +1,72 @@
+"""Host-side checks of libtq (no GPU): the library loads, exports every
+symbol include/tq.h declares, its host-built tables agree with the oracle's,
+and argument validation fails cleanly before any device work."""
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import tq_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from compressed_kv_cache_tq_b200 import build, tq
+
+    if not os.path.exists(tq.LIB_PATH):
+        build.build()
+    return tq
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "tq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(tq_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(L):
+    lib = L.lib()
+    names = declared_symbols()
+    assert len(names) >= 14
+    for name in names:
+        assert hasattr(lib, name), name
+    assert sorted(L.EXPORTED) == names
+
+
+@pytest.mark.parametrize("d,bits,m,seed,base", [(128, 3, 128, 42, 0), (128, 4, 128, 7, 0), (64, 2, 64, 5, 2),
+                                                (256, 3, 128, 9, 0), (64, 4, 192, 1, 4)])
+def test_host_tables_match_oracle(L, d, bits, m, seed, base):
+    R, P, c, t = L.tq_host_tables(d, bits, seed, m=m, stream_base=base)
+    tb = O.make_tables(d, bits, seed, m=m, stream_base=base)
+    assert np.max(np.abs(R - tb.R)) < 1e-12
+    assert np.max(np.abs(P - tb.P)) < 1e-13
+    np.testing.assert_allclose(c, tb.c, atol=1e-12, rtol=0)
+    np.testing.assert_allclose(t, tb.t, atol=1e-12, rtol=0)
+
+
+def test_host_tables_reject_unsupported(L):
+    lib = L.lib()
+    for d, bits, m in [(100, 3, 100), (128, 5, 128), (128, 1, 128), (512, 3, 512), (128, 3, 96)]:
+        assert lib.tq_host_tables(d, bits, m, 1, 0, None, None, None, None) == 2
+
+
+def test_argument_validation_without_device(L):
+    lib = L.lib()
+    assert lib.tq_init(128, 3, 1, None) == 1
+    assert lib.tq_quantize(None, None, 0, 10, 128, None, None, None) == 1
+    assert lib.tq_logits_workspace_bytes(None, 1, 4, 1) == 0
+    assert lib.tq_topk_workspace_bytes(None, 1, 4, 1) == 0
+    assert lib.tq_logits(None, None, 1, 4, 1, 10, None, None, 1.0, None, None, 0, None) == 1
+    assert lib.tq_info(None, None, None, None, None) == 1
+    assert lib.tq_strerror(5) == b"workspace too small"
+    lib.tq_free(None)
+
+
+def test_row_bytes_formula():
+    for d, m, b in [(128, 128, 3), (128, 128, 2), (64, 64, 1), (256, 256, 3)]:
+        assert O.row_bytes(d, m, b) == d * b // 8 + m // 8

@@ -1,0 +1,249 @@
+"""GPU parity: libtq's kernels (through the C ABI) against the CPU oracle.
+
+Small cases span several 128-key tiles with ragged tails; the full-size
+decode and long-context workloads are checked on sampled rows in the launch
+configuration bench.py times.  Bands and tolerances: tests/parity.py."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from compressed_kv_cache_tq_b200 import workloads as W
+from oracle import tq_oracle as O
+
+from tests.parity import check_close, check_quantize, oracle_estimates, tables_of
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _ctx(lib, d=128, bits=3, seed=42, m=None):
+    return lib.tq_init(d, bits, seed, m=m)
+
+
+def _status_clean(lib, ctx):
+    torch.cuda.synchronize()
+    assert lib.tq_check_device_status(ctx) == 0
+
+
+def test_device_tables_match_oracle(lib):
+    ctx = _ctx(lib, bits=4, seed=11)
+    R, P, c, t = ctx.export_tables()
+    tb = tables_of(ctx)
+    assert np.max(np.abs(R - tb.R)) < 1e-12 and np.max(np.abs(P - tb.P)) < 1e-13
+    assert np.max(np.abs(c - tb.c)) < 1e-12 and np.max(np.abs(t - tb.t)) < 1e-12
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+@pytest.mark.parametrize("n", [1, 127, 441, 4133])
+def test_quantize_bf16_tensor_core_path(lib, bits, n):
+    ctx = _ctx(lib, bits=bits, seed=7 + bits)
+    scales = W.head_channel_scales(1, 128, seed=3)
+    k32 = W.decode_keys_pair(0, 0, n, 128, scales, seed=3 + n)
+    kb = torch.from_numpy(k32).to(torch.bfloat16)
+    payload, norms = lib.tq_quantize(ctx, kb.to(DEV))
+    _status_clean(lib, ctx)
+    rep = {}
+    check_quantize(payload.cpu().numpy(), norms.cpu().numpy(), kb.to(torch.float64).numpy(), tables_of(ctx), rep)
+
+
+def test_quantize_toy_fp32(lib):
+    """toy workload: 4096 fp32 keys (+ a ragged tail), b = 3."""
+    ctx = _ctx(lib, bits=3, seed=42)
+    k = W.toy_keys(4096 + 37, 128, seed=1000)
+    payload, norms = lib.tq_quantize(ctx, torch.from_numpy(k).to(DEV))
+    _status_clean(lib, ctx)
+    check_quantize(payload.cpu().numpy(), norms.cpu().numpy(), k.astype(np.float64), tables_of(ctx))
+
+
+@pytest.mark.parametrize("d,m,bits,dtype", [(64, 64, 3, torch.bfloat16), (64, 64, 2, torch.float32),
+                                            (256, 256, 3, torch.bfloat16), (128, 64, 4, torch.float32),
+                                            (192, 128, 2, torch.bfloat16)])
+def test_quantize_other_shapes(lib, d, m, bits, dtype):
+    ctx = _ctx(lib, d=d, bits=bits, seed=5, m=m)
+    k = W.toy_keys(777, d, seed=d + m)
+    kt = torch.from_numpy(k).to(dtype)
+    payload, norms = lib.tq_quantize(ctx, kt.to(DEV))
+    _status_clean(lib, ctx)
+    check_quantize(payload.cpu().numpy(), norms.cpu().numpy(), kt.to(torch.float64).numpy(), tables_of(ctx))
+
+
+def test_quantize_edge_cases(lib):
+    ctx = _ctx(lib, bits=4, seed=3)
+    k = W.toy_keys(300, 128, seed=9)
+    k[5] = 0.0                       # zero key
+    k[17] *= 1e4                     # ||k|| above the fp16 range -> +inf norms
+    k[40] = 0.0
+    k[40][3] = 1.0                   # a basis vector
+    wide = torch.zeros((300, 256), dtype=torch.bfloat16)
+    wide[:, :128] = torch.from_numpy(k).to(torch.bfloat16)
+    keys = wide.to(DEV)[:, :128]     # leading dimension 256
+    payload = torch.empty((300, ctx.row_bytes), dtype=torch.uint8, device=DEV)
+    norms = torch.empty((300, 2), dtype=torch.float16, device=DEV)
+    import ctypes
+
+    st = lib.lib().tq_quantize(ctx.handle, ctypes.c_void_p(keys.data_ptr()), 1, 300, 256,
+                               ctypes.c_void_p(payload.data_ptr()), ctypes.c_void_p(norms.data_ptr()),
+                               ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0
+    _status_clean(lib, ctx)
+    kk = wide[:, :128].to(torch.float64).numpy()
+    nr = norms.cpu().numpy()
+    assert np.all(nr[5] == 0) and np.isinf(nr[17, 0])
+    codes, bits = O.unpack_rows(payload.cpu().numpy(), 128, 128, 3)
+    assert np.all(codes[5] == 0) and np.all(bits[5])
+    ok = np.ones(300, bool)
+    ok[17] = False
+    check_quantize(payload.cpu().numpy()[ok], nr[ok], kk[ok], tables_of(ctx))
+    # n == 0 is a no-op; bad leading dimension is rejected
+    assert lib.lib().tq_quantize(ctx.handle, ctypes.c_void_p(keys.data_ptr()), 1, 0, 256, None, None, None) == 0
+    assert lib.lib().tq_quantize(ctx.handle, ctypes.c_void_p(keys.data_ptr()), 1, 10, 100,
+                                 ctypes.c_void_p(payload.data_ptr()), ctypes.c_void_p(norms.data_ptr()),
+                                 None) == 1
+
+
+def test_quantize_is_deterministic(lib):
+    ctx = _ctx(lib, bits=3, seed=1)
+    kb = torch.from_numpy(W.toy_keys(3000, 128, seed=4)).to(torch.bfloat16).to(DEV)
+    p1, n1 = lib.tq_quantize(ctx, kb)
+    p2, n2 = lib.tq_quantize(ctx, kb)
+    assert torch.equal(p1, p2) and torch.equal(n1.view(torch.int16), n2.view(torch.int16))
+
+
+def _cache(lib, ctx, B, Hkv, S, seed):
+    scales = W.head_channel_scales(Hkv, ctx.d, seed)
+    k = np.stack([np.stack([W.decode_keys_pair(b, h, S, ctx.d, scales, seed) for h in range(Hkv)])
+                  for b in range(B)])
+    kb = torch.from_numpy(k).to(torch.bfloat16).to(DEV).reshape(-1, ctx.d)
+    return lib.tq_quantize(ctx, kb)
+
+
+@pytest.mark.parametrize("bits,B,Hkv,G,S", [(3, 2, 2, 4, 1037), (4, 1, 3, 4, 515), (4, 2, 2, 1, 200),
+                                            (3, 1, 2, 2, 333), (2, 2, 1, 8, 129), (4, 1, 1, 12, 100),
+                                            (4, 1, 2, 3, 16)])
+def test_logits_against_oracle(lib, bits, B, Hkv, G, S):
+    ctx = _ctx(lib, bits=bits, seed=21)
+    payload, norms = _cache(lib, ctx, B, Hkv, S, seed=31)
+    Hq = Hkv * G
+    q = W.queries((B, Hq, 128), seed=41)
+    scale = 1.0 / math.sqrt(128)
+    out = lib.tq_logits(ctx, torch.from_numpy(q).to(DEV), payload, norms, Hkv, scale=scale)
+    _status_clean(lib, ctx)
+    tb = tables_of(ctx)
+    pl, nr, o = payload.cpu().numpy(), norms.cpu().numpy(), out.cpu().numpy()
+    for b in range(B):
+        for hk in range(Hkv):
+            rows = slice((b * Hkv + hk) * S, (b * Hkv + hk + 1) * S)
+            s, A = oracle_estimates(pl[rows], nr[rows], q[b, hk * G:(hk + 1) * G].astype(np.float64), tb)
+            check_close(o[b, hk * G:(hk + 1) * G], scale * s, scale * A)
+
+
+def test_toy_logits_all_pairs(lib):
+    """toy workload: 64 queries x 4096 keys, all pairs (one GQA group of 64)."""
+    ctx = _ctx(lib, bits=3, seed=42)
+    k = W.toy_keys(4096, 128, seed=1000)
+    payload, norms = lib.tq_quantize(ctx, torch.from_numpy(k).to(DEV))
+    q = W.queries((1, 64, 128), seed=1001)
+    out = lib.tq_logits(ctx, torch.from_numpy(q).to(DEV), payload, norms, 1)
+    _status_clean(lib, ctx)
+    s, A = oracle_estimates(payload.cpu().numpy(), norms.cpu().numpy(), q[0].astype(np.float64), tables_of(ctx))
+    check_close(out.cpu().numpy()[0], s, A)
+
+
+@pytest.mark.parametrize("full", [True, False])
+@pytest.mark.parametrize("d,bits", [(128, 4), (64, 2)])
+def test_dequantize_against_oracle(lib, full, d, bits):
+    ctx = _ctx(lib, d=d, bits=bits, seed=13)
+    k = W.toy_keys(555, d, seed=8)
+    payload, norms = lib.tq_quantize(ctx, torch.from_numpy(k).to(DEV))
+    xh = lib.tq_dequantize(ctx, payload, norms, full=full)
+    _status_clean(lib, ctx)
+    tb = tables_of(ctx)
+    codes, bits_ = O.unpack_rows(payload.cpu().numpy(), d, d, tb.bmse)
+    nr = norms.cpu().numpy().astype(np.float64)
+    ref = O.dequantize(codes, bits_, nr[:, 0], nr[:, 1], tb, full=full)
+    # fp32 accumulation over d + m terms: bound by the sum of the magnitudes
+    v = nr[:, :1] * np.abs(tb.c[codes]).sum(1, keepdims=True)
+    if full:
+        v = v + O.QJL_CONST / tb.m * nr[:, 1:2] * np.abs(tb.P).sum()
+    err = np.abs(xh.cpu().numpy() - ref)
+    assert np.all(err <= 2e-5 * v), float(np.max(err / v))
+
+
+def test_dequantize_full_matches_logits(lib):
+    ctx = _ctx(lib, bits=3, seed=2)
+    payload, norms = _cache(lib, ctx, 1, 1, 300, seed=5)
+    xh = lib.tq_dequantize(ctx, payload, norms, full=True)
+    q = torch.from_numpy(W.queries((1, 4, 128), seed=6)).to(DEV)
+    out = lib.tq_logits(ctx, q, payload, norms, 1)
+    ref = (q[0].double() @ xh.double().T).cpu().numpy()
+    _, A = oracle_estimates(payload.cpu().numpy(), norms.cpu().numpy(), q[0].cpu().double().numpy(), tables_of(ctx))
+    check_close(out[0].cpu().numpy(), ref, A)
+
+
+@pytest.mark.parametrize("bits,n,nq,k", [(3, 5000, 16, 10), (4, 3001, 9, 1), (2, 700, 5, 64), (3, 100, 3, 10)])
+def test_topk_against_oracle(lib, bits, n, nq, k):
+    ctx = _ctx(lib, bits=bits, seed=17)
+    db = W.search_vectors(n, 128, seed=100 + bits, which=0)
+    qs = W.search_vectors(nq, 128, seed=100 + bits, which=1)
+    payload, norms = lib.tq_quantize(ctx, torch.from_numpy(db).to(DEV))
+    ids, scores = lib.tq_topk(ctx, torch.from_numpy(qs).to(DEV), payload, norms, k)
+    _status_clean(lib, ctx)
+    s, A = oracle_estimates(payload.cpu().numpy(), norms.cpu().numpy(), qs.astype(np.float64), tables_of(ctx))
+    ids = ids.cpu().numpy()
+    order = np.array([np.lexsort((np.arange(n), -s[i]))[:k + 1] for i in range(nq)])
+    near_tie = 0
+    for i in range(nq):
+        kth, nxt = s[i, order[i, k - 1]], s[i, order[i, min(k, n - 1)]] if k < n else -np.inf
+        if k < n and kth - nxt < 1e-6 * A[i].max():
+            near_tie += 1
+            assert set(ids[i][:k - 1]) <= set(order[i][:k + 1])
+            continue
+        np.testing.assert_array_equal(ids[i], order[i, :k])
+    assert near_tie <= max(1, nq // 10)
+    np.testing.assert_allclose(scores.cpu().numpy(), np.take_along_axis(s, ids, 1), rtol=1e-6,
+                               atol=1e-6 * A.max())
+
+
+def test_logits_rejects_bad_workspace(lib):
+    ctx = _ctx(lib, bits=3, seed=1)
+    payload, norms = _cache(lib, ctx, 1, 1, 64, seed=1)
+    q = torch.zeros((1, 4, 128), device=DEV)
+    small = torch.empty(256, dtype=torch.uint8, device=DEV)
+    with pytest.raises(lib.TQError) as e:
+        lib.tq_logits(ctx, q, payload, norms, 1, workspace=small)
+    assert e.value.status == 5
+
+
+# --------------------------------------------------------------------------
+# Full-size workloads, sampled (the configuration bench.py times)
+# --------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("name,B,Hkv,G,S,bits", [("decode", 8, 8, 4, 32768, 4), ("longctx", 1, 8, 4, 131072, 3)])
+def test_full_size_sampled(lib, name, B, Hkv, G, S, bits):
+    seed = 1001 if name == "decode" else 1002
+    ctx = _ctx(lib, bits=bits, seed=42)
+    keys = W.decode_keys(B, Hkv, S, 128, seed, device=DEV).reshape(-1, 128)
+    payload, norms = lib.tq_quantize(ctx, keys)
+    Hq = Hkv * G
+    q = W.queries((B, Hq, 128), seed=seed + 7)
+    out = lib.tq_logits(ctx, torch.from_numpy(q).to(DEV), payload, norms, Hkv, scale=1.0 / math.sqrt(128))
+    _status_clean(lib, ctx)
+    tb = tables_of(ctx)
+    rng = np.random.default_rng(0)
+    pairs = [(0, 0), (B - 1, Hkv - 1), (B // 2, 3)]
+    rep = {}
+    for b, h in pairs:
+        s_idx = np.sort(rng.choice(S, 1500, replace=False))
+        s_idx[-1] = S - 1
+        rows = (b * Hkv + h) * S + s_idx
+        k64 = W.decode_keys_rows(b, h, s_idx, S, 128, Hkv, seed)
+        check_quantize(payload[rows].cpu().numpy(), norms[rows].cpu().numpy(), k64, tb, rep)
+        est, A = oracle_estimates(payload[rows].cpu().numpy(), norms[rows].cpu().numpy(),
+                                  q[b, h * G:(h + 1) * G].astype(np.float64), tb)
+        got = out[b, h * G:(h + 1) * G][:, torch.from_numpy(s_idx).to(DEV)].cpu().numpy()
+        check_close(got, est / math.sqrt(128), A / math.sqrt(128))
