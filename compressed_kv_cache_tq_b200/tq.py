@@ -51,6 +51,7 @@ def lib() -> ctypes.CDLL:
             "tq_dequantize": (i32, [vp, vp, vp, i64, i32, vp, vp]),
             "tq_logits_workspace_bytes": (sz, [vp, i32, i32, i32]),
             "tq_logits": (i32, [vp, vp, i32, i32, i32, i64, vp, vp, f32, vp, vp, sz, vp]),
+            "tq_logits_noalloc": (i32, [vp, vp, i32, i32, i32, i64, vp, vp, f32, vp, vp]),
             "tq_topk_workspace_bytes": (sz, [vp, i64, i64, i32]),
             "tq_topk": (i32, [vp, vp, i64, vp, vp, i64, i32, vp, vp, vp, sz, vp]),
             "tq_check_device_status": (i32, [vp, vp, ctypes.POINTER(u32)]),
@@ -66,7 +67,7 @@ def lib() -> ctypes.CDLL:
 
 
 EXPORTED = ["tq_init", "tq_init_ex", "tq_host_tables", "tq_free", "tq_info", "tq_export_tables", "tq_quantize", "tq_dequantize",
-            "tq_logits_workspace_bytes", "tq_logits", "tq_topk_workspace_bytes", "tq_topk",
+            "tq_logits_workspace_bytes", "tq_logits", "tq_logits_noalloc", "tq_topk_workspace_bytes", "tq_topk",
             "tq_check_device_status", "tq_strerror", "tq_last_cuda_error"]
 
 
@@ -212,6 +213,23 @@ def tq_logits(ctx: Context, q: torch.Tensor, payload: torch.Tensor, norms: torch
         workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=q.device)
     _check(lib().tq_logits(ctx.handle, _ptr(q), B, Hq, Hkv, S, _ptr(payload), _ptr(norms), float(scale), _ptr(out),
                            _ptr(workspace), workspace.numel(), ctypes.c_void_p(_stream(stream))), "tq_logits")
+    return out
+
+
+def tq_logits_noalloc(ctx: Context, q: torch.Tensor, payload: torch.Tensor, norms: torch.Tensor, Hkv: int,
+                      scale: float = 1.0, out: torch.Tensor | None = None, stream=None):
+    """tq_logits with the library's static scratch array instead of a workspace."""
+    _need_cuda(q, "q")
+    _need_cuda(payload, "payload")
+    _need_cuda(norms, "norms")
+    if q.dtype != torch.float32 or q.dim() != 3 or q.shape[2] != ctx.d:
+        raise ValueError("q must be float32 (B, Hq, d)")
+    B, Hq, _ = q.shape
+    S = payload.shape[0] // (B * Hkv)
+    if out is None:
+        out = torch.empty((B, Hq, S), dtype=torch.float32, device=q.device)
+    _check(lib().tq_logits_noalloc(ctx.handle, _ptr(q), B, Hq, Hkv, S, _ptr(payload), _ptr(norms), float(scale),
+                                   _ptr(out), ctypes.c_void_p(_stream(stream))), "tq_logits_noalloc")
     return out
 
 

@@ -139,6 +139,32 @@ tq_status tq_logits(const tq_ctx* ctx, const float* q, int B, int Hq, int Hkv, i
                     const uint8_t* payload, const uint16_t* norms, float scale, float* out,
                     void* workspace, size_t workspace_bytes, void* stream);
 
+/* Size of the library-owned scratch array used by tq_logits_noalloc. */
+#define TQ_NOALLOC_SCRATCH_BYTES (1u << 20)
+
+/* tq_logits without a caller workspace and without any allocation.  The
+ * pages have no counterpart to this call: it exists for callers that cannot
+ * allocate device memory where they compute logits, for instance an engine
+ * that has handed its whole device-memory budget to its own pool, or a
+ * latency-critical decode loop in which a cudaMalloc (which may synchronise
+ * the device) is not acceptable.  It computes exactly what tq_logits
+ * computes, with the same arguments minus the workspace.
+ * Scratch: one static device array of TQ_NOALLOC_SCRATCH_BYTES bytes in
+ * libtq, present on every GPU that loads the library until the process
+ * exits.  The call allocates nothing and frees nothing.  The first call on a
+ * device looks up the array's device address (once per device, with that
+ * device current), so make that first call before any stream capture.
+ * Every call shares the array and it keeps the last call's contents; nothing
+ * in it has to start at zero (each call rewrites all it reads).  Calls whose
+ * kernels overlap on the GPU (for example on two streams) race on the array:
+ * order them.
+ * Errors: as tq_logits; TQ_ERR_WORKSPACE when tq_logits_workspace_bytes for
+ * (B, Hq, Hkv) exceeds TQ_NOALLOC_SCRATCH_BYTES (about 500 (batch, KV head)
+ * groups of up to 4 query heads each). */
+tq_status tq_logits_noalloc(const tq_ctx* ctx, const float* q, int B, int Hq, int Hkv, int64_t S,
+                            const uint8_t* payload, const uint16_t* norms, float scale, float* out,
+                            void* stream);
+
 /* Workspace bytes tq_topk needs for nq queries against n database rows. */
 size_t tq_topk_workspace_bytes(const tq_ctx* ctx, int64_t nq, int64_t n, int k);
 
