@@ -46,73 +46,105 @@ struct HeadScale {
 // ---------------------------------------------------------------------------
 // Query preparation: x = R q, y = P x (= S q), int16 fixed point per head,
 // split into two signed int8 limbs, written in MMA B-fragment order.
-// One block per (batch, kv head, head slot); slots >= G write zeros.
+// One block per (batch, kv head) group computes all 4 NT head slots; slots
+// >= G are zero.  R^T and then P^T are staged in shared memory (64 KB).
 // ---------------------------------------------------------------------------
+constexpr int kMaxSlots = 8;
+
 __global__ void __launch_bounds__(128) qprep_kernel(const float* __restrict__ q, int Hq, int Hkv, int nt_per_group,
                                                     const float* __restrict__ Rt, const float* __restrict__ Pt,
                                                     float code_inv_scale, float scale, float qjl_over_m,
                                                     uint32_t* __restrict__ frags, HeadScale* __restrict__ hscale) {
-  __shared__ float sq[D], sx[D], sy[D];
-  __shared__ int8_t limbs[2][2][D];     // [x/y][hi/lo][coordinate]
-  __shared__ float red[2][4];
+  extern __shared__ float smq[];
+  float* mat = smq;                                  // [D][D] R^T, then P^T
+  float* sq = mat + D * D;                           // [slots][D] queries, then y
+  float* sx = sq + kMaxSlots * D;                    // [slots][D] x
+  __shared__ float red[2][kMaxSlots][4];
+  __shared__ int8_t limbs[kMaxSlots][2][2][D];       // [slot][x/y][hi/lo][coordinate]
   const int G = Hq / Hkv;
   const int slots = nt_per_group * HPT;
-  const int blk = blockIdx.x;
-  const int slot = blk % slots, grp = blk / slots;      // grp = b * Hkv + hkv
-  const int b = grp / Hkv, hkv = grp % Hkv;
-  const bool live = slot < G;
-  const int h = hkv * G + slot;
-  const int tid = threadIdx.x;
-  sq[tid] = live ? q[(size_t(b) * Hq + h) * D + tid] : 0.f;
+  const int grp = blockIdx.x, b = grp / Hkv, hkv = grp % Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int i = tid; i < D * D / 4; i += 128)
+    reinterpret_cast<float4*>(mat)[i] = __ldg(reinterpret_cast<const float4*>(Rt) + i);
+  for (int h = 0; h < slots; ++h) sq[h * D + tid] = h < G ? q[(size_t(b) * Hq + hkv * G + h) * D + tid] : 0.f;
   __syncthreads();
-  float x = 0.f;
-  for (int i = 0; i < D; ++i) x = fmaf(Rt[i * D + tid], sq[i], x);
-  sx[tid] = x;
-  __syncthreads();
-  float y = 0.f;
-  for (int j = 0; j < D; ++j) y = fmaf(Pt[j * D + tid], sx[j], y);
-  sy[tid] = y;
-  float ax = fabsf(x), ay = fabsf(y);
-  for (int o = 16; o; o >>= 1) {
-    ax = fmaxf(ax, __shfl_xor_sync(0xffffffffu, ax, o));
-    ay = fmaxf(ay, __shfl_xor_sync(0xffffffffu, ay, o));
-  }
-  if ((tid & 31) == 0) {
-    red[0][tid >> 5] = ax;
-    red[1][tid >> 5] = ay;
+  float acc[kMaxSlots];
+#pragma unroll
+  for (int h = 0; h < kMaxSlots; ++h) acc[h] = 0.f;
+#pragma unroll 4
+  for (int i = 0; i < D; ++i) {
+    const float r = mat[i * D + tid];
+#pragma unroll
+    for (int h = 0; h < kMaxSlots; ++h)
+      if (h < slots) acc[h] = fmaf(r, sq[h * D + i], acc[h]);
   }
   __syncthreads();
-  const float mx = fmaxf(fmaxf(red[0][0], red[0][1]), fmaxf(red[0][2], red[0][3]));
-  const float my = fmaxf(fmaxf(red[1][0], red[1][1]), fmaxf(red[1][2], red[1][3]));
-  const float kx = mx > 0.f ? 32000.f / mx : 0.f;
-  const float ky = my > 0.f ? 32000.f / my : 0.f;
-  const int xi = __float2int_rn(sx[tid] * kx);
-  const int yi = __float2int_rn(sy[tid] * ky);
-  const int xh = (xi + 128) >> 8, yh = (yi + 128) >> 8;
-  limbs[0][0][tid] = int8_t(xh);
-  limbs[0][1][tid] = int8_t(xi - 256 * xh);
-  limbs[1][0][tid] = int8_t(yh);
-  limbs[1][1][tid] = int8_t(yi - 256 * yh);
-  if (tid == 0 && live) {
-    hscale[size_t(b) * Hq + h].code = mx > 0.f ? scale * code_inv_scale / kx : 0.f;
-    hscale[size_t(b) * Hq + h].sign = my > 0.f ? scale * qjl_over_m / ky : 0.f;
+  for (int i = tid; i < D * D / 4; i += 128)
+    reinterpret_cast<float4*>(mat)[i] = __ldg(reinterpret_cast<const float4*>(Pt) + i);
+#pragma unroll
+  for (int h = 0; h < kMaxSlots; ++h)
+    if (h < slots) sx[h * D + tid] = acc[h];
+  __syncthreads();
+  float accy[kMaxSlots];
+#pragma unroll
+  for (int h = 0; h < kMaxSlots; ++h) accy[h] = 0.f;
+#pragma unroll 4
+  for (int j = 0; j < D; ++j) {
+    const float p = mat[j * D + tid];
+#pragma unroll
+    for (int h = 0; h < kMaxSlots; ++h)
+      if (h < slots) accy[h] = fmaf(p, sx[h * D + j], accy[h]);
+  }
+  // per-slot max |x|, max |y|
+#pragma unroll
+  for (int h = 0; h < kMaxSlots; ++h) {
+    if (h >= slots) break;
+    float ax = fabsf(acc[h]), ay = fabsf(accy[h]);
+    for (int o = 16; o; o >>= 1) {
+      ax = fmaxf(ax, __shfl_xor_sync(0xffffffffu, ax, o));
+      ay = fmaxf(ay, __shfl_xor_sync(0xffffffffu, ay, o));
+    }
+    if (lane == 0) {
+      red[0][h][warp] = ax;
+      red[1][h][warp] = ay;
+    }
   }
   __syncthreads();
-  // Fragment words of this head: lanes L with L/4 = 2 (slot % 4) + limb.
-  // Word (xy, s, reg, lane) holds B[k = 16 reg + 4 tig + e][n = L/4], e = 0..3,
-  // with K position k of step s mapped to coordinate tig * D/4 + 4 (2s + reg) + e.
-  const int nt = slot / HPT, col = slot % HPT;
-  uint32_t* fr = frags + (size_t(grp) * nt_per_group + nt) * kFragWords;
-  {
-    const int w = tid;                      // 128 words per head: [xy][s][reg][limb][tig]
-    const int tig = w & 3, limb = (w >> 2) & 1, reg = (w >> 3) & 1, s = (w >> 4) & 3, xy = (w >> 6) & 1;
-    const int lane = (2 * col + limb) * 4 + tig;
+#pragma unroll
+  for (int h = 0; h < kMaxSlots; ++h) {
+    if (h >= slots) break;
+    const float mx = fmaxf(fmaxf(red[0][h][0], red[0][h][1]), fmaxf(red[0][h][2], red[0][h][3]));
+    const float my = fmaxf(fmaxf(red[1][h][0], red[1][h][1]), fmaxf(red[1][h][2], red[1][h][3]));
+    const float kx = mx > 0.f ? 32000.f / mx : 0.f;
+    const float ky = my > 0.f ? 32000.f / my : 0.f;
+    const int xi = __float2int_rn(acc[h] * kx);
+    const int yi = __float2int_rn(accy[h] * ky);
+    const int xh = (xi + 128) >> 8, yh = (yi + 128) >> 8;
+    limbs[h][0][0][tid] = int8_t(xh);
+    limbs[h][0][1][tid] = int8_t(xi - 256 * xh);
+    limbs[h][1][0][tid] = int8_t(yh);
+    limbs[h][1][1][tid] = int8_t(yi - 256 * yh);
+    if (tid == 0 && h < G) {
+      hscale[size_t(b) * Hq + hkv * G + h].code = mx > 0.f ? scale * code_inv_scale / kx : 0.f;
+      hscale[size_t(b) * Hq + hkv * G + h].sign = my > 0.f ? scale * qjl_over_m / ky : 0.f;
+    }
+  }
+  __syncthreads();
+  // Fragment word (xy, s, reg, lane) of N-tile nt holds B[k = 16 reg + 4 tig + e][n = lane / 4],
+  // e = 0..3; column n is (head slot 4 nt + n / 2, limb n % 2); K position k of step s is
+  // coordinate tig * D/4 + 4 (2s + reg) + e.
+  for (int w = tid; w < nt_per_group * kFragWords; w += 128) {
+    const int nt = w / kFragWords, rem = w - nt * kFragWords;
+    const int ln = rem & 31, reg = (rem >> 5) & 1, s = (rem >> 6) % KS, xy = (rem >> 6) / KS;
+    const int n = ln >> 2, tig = ln & 3;
+    const int slot = nt * HPT + (n >> 1), limb = n & 1;
     uint32_t word = 0;
     for (int e = 0; e < 4; ++e) {
       const int j = tig * (D / 4) + 4 * (2 * s + reg) + e;
-      word |= uint32_t(uint8_t(limbs[xy][limb][j])) << (8 * e);
+      word |= uint32_t(uint8_t(limbs[slot][xy][limb][j])) << (8 * e);
     }
-    fr[((xy * KS + s) * 2 + reg) * 32 + lane] = word;
+    frags[size_t(grp) * nt_per_group * kFragWords + w] = word;
   }
 }
 
@@ -192,14 +224,20 @@ __device__ __forceinline__ void code_selectors(const Chunk<BMSE>& c, uint32_t (&
   }
 }
 
-// Sign selectors for the 8 registers: one bit per nibble.
+// int8 {-1, +1} operands for the 8 sign registers of a quarter.  Register
+// 4u + i of unit u takes bit i of every nibble of the unit's sign halfword.
+// Masking that bit in place gives selector nibbles 0 or 2^i; the two byte
+// tables put -1 at byte 0 and +1 at byte 2^i (bit 3 is the byte-permute mode
+// bit, so register 4u + 3 shifts it down to bit 2 first).
 template <int BMSE>
-__device__ __forceinline__ void sign_selectors(const Chunk<BMSE>& c, uint32_t (&sel)[8]) {
+__device__ __forceinline__ void sign_operands(const Chunk<BMSE>& c, uint32_t (&a)[8]) {
 #pragma unroll
   for (int u = 0; u < 2; ++u) {
     const uint32_t h = chunk_half(c, 2 * BMSE + u);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) sel[4 * u + i] = (h >> i) & 0x1111u;
+    a[4 * u + 0] = prmt(0x000001FFu, 0u, h & 0x1111u);
+    a[4 * u + 1] = prmt(0x000100FFu, 0u, h & 0x2222u);
+    a[4 * u + 2] = prmt(0x000000FFu, 0x00000001u, h & 0x4444u);
+    a[4 * u + 3] = prmt(0x000000FFu, 0x00000001u, (h >> 1) & 0x4444u);
   }
 }
 
@@ -218,44 +256,57 @@ __global__ void __launch_bounds__(kLogitThreads) logits_mma_kernel(
   const int G = Hq / Hkv;
   const int64_t tpp = (S + 15) / 16;
 
+  // tile t = (group, key offset s0); advanced incrementally, no division per tile
+  int64_t grp = t_begin / tpp;
+  int64_t s0 = (t_begin - grp * tpp) * 16;
+
   uint32_t bx[NT][KS][2], by[NT][KS][2];
   float sc_code[NT], sc_sign[NT];
-  int64_t cur_grp = -1;
-
-  for (int64_t t = t_begin; t < t_end; ++t) {
-    const int64_t grp = t / tpp;
-    const int64_t s0 = (t - grp * tpp) * 16;
-    if (grp != cur_grp) {
-      cur_grp = grp;
-      const int b = int(grp / Hkv), hkv = int(grp % Hkv);
+  float* obase[NT];
+  auto load_group = [&](int64_t gi) {
+    const int b = int(gi / Hkv), hkv = int(gi - int64_t(b) * Hkv);
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const uint32_t* fr = frags + (size_t(grp) * NT + nt) * kFragWords;
+    for (int nt = 0; nt < NT; ++nt) {
+      const uint32_t* fr = frags + (size_t(gi) * NT + nt) * kFragWords;
 #pragma unroll
-        for (int s = 0; s < KS; ++s)
+      for (int s = 0; s < KS; ++s)
 #pragma unroll
-          for (int r = 0; r < 2; ++r) {
-            bx[nt][s][r] = __ldg(fr + ((0 * KS + s) * 2 + r) * 32 + lane);
-            by[nt][s][r] = __ldg(fr + ((1 * KS + s) * 2 + r) * 32 + lane);
-          }
-        const int hg = nt * HPT + tig;
-        if (hg < G) {
-          const HeadScale hs = hscale[size_t(b) * Hq + hkv * G + hg];
-          sc_code[nt] = hs.code;
-          sc_sign[nt] = hs.sign;
-        } else {
-          sc_code[nt] = 0.f;
-          sc_sign[nt] = 0.f;
+        for (int r = 0; r < 2; ++r) {
+          bx[nt][s][r] = __ldg(fr + ((0 * KS + s) * 2 + r) * 32 + lane);
+          by[nt][s][r] = __ldg(fr + ((1 * KS + s) * 2 + r) * 32 + lane);
         }
-      }
+      const int hg = nt * HPT + tig;
+      const int hh = hg < G ? hg : 0;
+      const HeadScale hs = hscale[size_t(b) * Hq + hkv * G + hh];
+      sc_code[nt] = hg < G ? hs.code : 0.f;
+      sc_sign[nt] = hg < G ? hs.sign : 0.f;
+      obase[nt] = out + (size_t(b) * Hq + hkv * G + hh) * S;
     }
-    const int64_t rowA = grp * S + s0 + g, rowB = rowA + 8;
-    const bool okA = s0 + g < S, okB = s0 + g + 8 < S;
-    Chunk<BMSE> ca, cb;
+  };
+  load_group(grp);
+
+  auto load_tile = [&](int64_t gi, int64_t so, Chunk<BMSE>& ca, Chunk<BMSE>& cb, uint32_t& na, uint32_t& nb) {
+    const int64_t rowA = gi * S + so + g, rowB = rowA + 8;
+    const bool okA = so + g < S, okB = so + g + 8 < S;
     load_chunk<BMSE>(ca, payload + rowA * kRowBytes, tig, okA);
     load_chunk<BMSE>(cb, payload + rowB * kRowBytes, tig, okB);
-    const uint32_t na = okA ? __ldg(reinterpret_cast<const uint32_t*>(norms) + rowA) : 0u;
-    const uint32_t nb = okB ? __ldg(reinterpret_cast<const uint32_t*>(norms) + rowB) : 0u;
+    na = okA ? __ldg(reinterpret_cast<const uint32_t*>(norms) + rowA) : 0u;
+    nb = okB ? __ldg(reinterpret_cast<const uint32_t*>(norms) + rowB) : 0u;
+  };
+  Chunk<BMSE> ca, cb;
+  uint32_t na, nb;
+  load_tile(grp, s0, ca, cb, na, nb);
+
+  for (int64_t t = t_begin; t < t_end; ++t) {
+    // next tile coordinates and its loads, issued before this tile's math
+    int64_t ngrp = grp, ns0 = s0 + 16;
+    if (ns0 >= S) {
+      ns0 = 0;
+      ++ngrp;
+    }
+    Chunk<BMSE> nca, ncb;
+    uint32_t nna = 0, nnb = 0;
+    if (t + 1 < t_end) load_tile(ngrp, ns0, nca, ncb, nna, nnb);
 
     uint32_t sa[8], sb[8];
     int acc_hi[NT][4], acc_lo[NT][4], acc_sg[NT][4];
@@ -280,33 +331,46 @@ __global__ void __launch_bounds__(kLogitThreads) logits_mma_kernel(
         mma_s8(acc_lo[nt], al0, al1, al2, al3, bx[nt][s][0], bx[nt][s][1]);
       }
     }
-    sign_selectors<BMSE>(ca, sa);
-    sign_selectors<BMSE>(cb, sb);
-    constexpr uint32_t kSignLut = 0x000001FFu;   // byte 0 = -1, byte 1 = +1
+    // sign registers: selectors keep one bit per nibble; the byte table maps
+    // that bit's two possible selector values to -1 and +1
+    uint32_t ga[8], gb[8];
+    sign_operands<BMSE>(ca, ga);
+    sign_operands<BMSE>(cb, gb);
 #pragma unroll
-    for (int s = 0; s < KS; ++s) {
-      const uint32_t a0 = prmt(kSignLut, 0u, sa[2 * s]), a1 = prmt(kSignLut, 0u, sb[2 * s]);
-      const uint32_t a2 = prmt(kSignLut, 0u, sa[2 * s + 1]), a3 = prmt(kSignLut, 0u, sb[2 * s + 1]);
+    for (int s = 0; s < KS; ++s)
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) mma_s8(acc_sg[nt], a0, a1, a2, a3, by[nt][s][0], by[nt][s][1]);
-    }
+      for (int nt = 0; nt < NT; ++nt)
+        mma_s8(acc_sg[nt], ga[2 * s], gb[2 * s], ga[2 * s + 1], gb[2 * s + 1], by[nt][s][0], by[nt][s][1]);
+
     // epilogue: C[row][2 tig + limb] -> head tig of each N-tile
-    const float kna = __half2float(__ushort_as_half(uint16_t(na))), kra = __half2float(__ushort_as_half(uint16_t(na >> 16)));
-    const float knb = __half2float(__ushort_as_half(uint16_t(nb))), krb = __half2float(__ushort_as_half(uint16_t(nb >> 16)));
-    const int b = int(grp / Hkv), hkv = int(grp % Hkv);
+    const float kna = __half2float(__ushort_as_half(uint16_t(na)));
+    const float kra = __half2float(__ushort_as_half(uint16_t(na >> 16)));
+    const float knb = __half2float(__ushort_as_half(uint16_t(nb)));
+    const float krb = __half2float(__ushort_as_half(uint16_t(nb >> 16)));
+    const bool okA = s0 + g < S, okB = s0 + g + 8 < S;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const int hg = nt * HPT + tig;
-      if (hg >= G) continue;
       const float codeA = float(acc_hi[nt][0]) * 65536.f + float(acc_hi[nt][1] + acc_lo[nt][0]) * 256.f +
                           float(acc_lo[nt][1]);
       const float codeB = float(acc_hi[nt][2]) * 65536.f + float(acc_hi[nt][3] + acc_lo[nt][2]) * 256.f +
                           float(acc_lo[nt][3]);
       const float signA = float(acc_sg[nt][0]) * 256.f + float(acc_sg[nt][1]);
       const float signB = float(acc_sg[nt][2]) * 256.f + float(acc_sg[nt][3]);
-      float* o = out + (size_t(b) * Hq + hkv * G + hg) * S + s0;
-      if (okA) o[g] = kna * codeA * sc_code[nt] + kra * signA * sc_sign[nt];
-      if (okB) o[g + 8] = knb * codeB * sc_code[nt] + krb * signB * sc_sign[nt];
+      float* o = obase[nt] + s0;
+      if (hg < G) {
+        if (okA) o[g] = kna * codeA * sc_code[nt] + kra * signA * sc_sign[nt];
+        if (okB) o[g + 8] = knb * codeB * sc_code[nt] + krb * signB * sc_sign[nt];
+      }
+    }
+    if (t + 1 < t_end) {
+      if (ngrp != grp) load_group(ngrp);
+      grp = ngrp;
+      s0 = ns0;
+      ca = nca;
+      cb = ncb;
+      na = nna;
+      nb = nnb;
     }
   }
 }
@@ -403,9 +467,10 @@ cudaError_t launch_logits(const tq_ctx* ctx, const float* q, int B, int Hq, int 
   uint32_t* frags = static_cast<uint32_t*>(ws);
   const size_t frag_bytes = ((size_t(groups) * nt * kFragWords * 4 + 255) / 256) * 256;
   HeadScale* hs = reinterpret_cast<HeadScale*>(static_cast<uint8_t*>(ws) + frag_bytes);
-  qprep_kernel<<<unsigned(groups * nt * HPT), 128, 0, st>>>(q, Hq, Hkv, nt, ctx->dRt, ctx->dPt,
-                                                             ctx->lut.inv_scale, scale,
-                                                             float(kQjlConst / ctx->m), frags, hs);
+  const size_t qp_smem = size_t(D * D + 2 * kMaxSlots * D) * 4;
+  cudaFuncSetAttribute(qprep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(qp_smem));
+  qprep_kernel<<<unsigned(groups), 128, qp_smem, st>>>(q, Hq, Hkv, nt, ctx->dRt, ctx->dPt, ctx->lut.inv_scale,
+                                                        scale, float(kQjlConst / ctx->m), frags, hs);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (S == 0) return cudaSuccess;

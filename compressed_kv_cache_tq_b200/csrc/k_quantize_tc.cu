@@ -13,16 +13,24 @@
 //
 // Precision: R = R_hi + R_lo in bf16 represents R to about 2^-17, so y / n is
 // within about 4e-7 of R k / ||k|| (codes differ from exact arithmetic only
-// for coordinates within that distance of a boundary); the JL product uses an
-// fp16 hi + lo split of r_rot (scaled by 2^7) and of P, dropping only lo * lo.
+// for coordinates within that distance of a boundary); n is taken from
+// ||y|| = ||R k|| (relative error about 4e-7); the JL product uses an fp16
+// hi + lo split of r_rot (scaled by 2^7) and of P, dropping only lo * lo.
 //
-// Structure (one CTA per SM, persistent over 128-key tiles):
-//   warp 4       : TMA producer (the constant B operands once, then key tiles)
-//   warp 5       : TMEM allocation and the single-thread MMA issue
-//   warps 0 .. 3 : epilogue, one thread per key row (= TMEM lane)
-// Shared memory: B operands R_hi, R_lo, P_hi, P_lo (128 KB), one key tile
-// (32 KB, TMA 128-byte swizzle) and the residual tiles r_hi, r_lo (64 KB).
-// TMEM: 256 columns, D1 = y (columns 0..127), D2 = z (columns 128..255).
+// Structure (one CTA per SM, persistent over 128-key tiles, two tiles in flight):
+//   warp 0       : TMA producer (the constant B operands once, then key tiles
+//                  into a two-deep ring)
+//   warp 1       : TMEM allocation and the single-thread MMA issue, in the
+//                  order MMA1(0), MMA1(1), MMA2(0), MMA1(2), MMA2(1), ...
+//   warps 2 .. 5 : epilogue of even local tiles (TMEM slot 0)
+//   warps 6 .. 9 : epilogue of odd local tiles (TMEM slot 1)
+//                  one thread per key row (= TMEM lane)
+// Shared memory: B operands R_hi, R_lo, P_hi, P_lo (128 KB) and two key tiles
+// (2 x 32 KB, TMA 128-byte swizzle).
+// TMEM: 512 columns, two slots of 256: y accumulates in columns 0..127 of a
+// slot; the epilogue reads it and writes the residual's fp16 hi / lo pairs
+// back over it (A operand of the JL product, read by the MMA from TMEM); z
+// accumulates in columns 128..255.
 // Every wait on an mbarrier is bounded; a wait that gives up sets the
 // context's status word, and all roles then leave their loops.
 #include <cuda.h>
@@ -37,15 +45,24 @@ namespace {
 
 constexpr int kD = 128;
 constexpr int kTile = 128;
-constexpr int kThreadsTc = 192;
+constexpr int kThreadsTc = 320;
 
 constexpr uint32_t kOffRhi = 0, kOffRlo = 32768, kOffPhi = 65536, kOffPlo = 98304;
-constexpr uint32_t kOffKey = 131072;
-constexpr uint32_t kOffAhi = 163840, kOffAlo = 196608;
-constexpr uint32_t kOffBar = 229376;
-constexpr uint32_t kSmemBytes = kOffBar + 128 + 1024;   // + slack for 1024-byte alignment
+constexpr uint32_t kOffKey = 131072;     // two 32 KB key tiles
+constexpr uint32_t kOffBar = 196608;
+constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;   // + slack for 1024-byte alignment
 
-enum Bar { kBarConst = 0, kBarKFull, kBarKEmpty, kBarD1Full, kBarD1Empty, kBarRFull, kBarD2Full, kBarD2Empty, kNumBars };
+// barriers; the per-slot ones come in pairs (slot 0, slot 1)
+enum Bar {
+  kBarConst = 0,
+  kBarKFull = 1,
+  kBarKEmpty = 3,
+  kBarD1Full = 5,
+  kBarRFull = 7,
+  kBarD2Full = 9,
+  kBarFree = 11,
+  kNumBars = 13
+};
 
 constexpr long long kWaitCycles = 4000000000LL;   // about 2 s at the boost clock
 
@@ -149,17 +166,70 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+// A operand from tensor memory, B from shared memory.
+__device__ __forceinline__ void mma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t b, uint32_t idesc,
+                                           uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+// Positive half of the symmetric codebook, scaled by 128 (the residual scale).
+struct HalfBook {
+  float T[3];   // boundaries above 0 (t_{L/2} .. t_{L-2})
+  float C[4];   // levels above 0 (c_{L/2} .. c_{L-1})
+};
+
+// Cell index and scaled residual of one rotated coordinate u (already x128).
+// The codebook is symmetric with t_{L/2-1} = 0, so idx = #{i : t_i < u} is
+// L/2 + #{boundaries above 0 below |u|} for u > 0 and L/2 - 1 - (that count)
+// otherwise (exact ties at +-t_i resolve within rounding of the boundary).
+template <int BMSE>
+__device__ __forceinline__ uint32_t cell(float u, const HalfBook& hb, float& r) {
+  const float a = fabsf(u);
+  const bool pos = u > 0.f;
+  uint32_t mag;
+  float lv;
+  if constexpr (BMSE == 3) {
+    const bool p1 = a > hb.T[0], p2 = a > hb.T[1], p3 = a > hb.T[2];
+    mag = p3 ? 3u : (p2 ? 2u : (p1 ? 1u : 0u));
+    lv = p3 ? hb.C[3] : (p2 ? hb.C[2] : (p1 ? hb.C[1] : hb.C[0]));
+    r = u - (pos ? lv : -lv);
+    return pos ? 4u + mag : 3u - mag;
+  } else if constexpr (BMSE == 2) {
+    const bool p1 = a > hb.T[0];
+    mag = p1 ? 1u : 0u;
+    lv = p1 ? hb.C[1] : hb.C[0];
+    r = u - (pos ? lv : -lv);
+    return pos ? 2u + mag : 1u - mag;
+  } else {
+    r = u - (pos ? hb.C[0] : -hb.C[0]);
+    return pos ? 1u : 0u;
+  }
+}
+
 template <int BMSE>
 __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid_constant__ CUtensorMap key_map,
                                                                    int64_t n, const uint8_t* __restrict__ bimg,
-                                                                   CodebookParams cb,
+                                                                   HalfBook book,
                                                                    uint8_t* __restrict__ payload,
                                                                    uint16_t* __restrict__ norms,
                                                                    uint32_t* __restrict__ status) {
   extern __shared__ uint8_t smem_raw[];
-  // 1024-byte aligned base (the swizzle pattern is anchored to the address)
   const uint32_t raw = smem_u32(smem_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;
+  const uint32_t base = (raw + 1023u) & ~1023u;   // the swizzle pattern is anchored to 1024-byte boundaries
   uint8_t* sbase = smem_raw + (base - raw);
   const uint32_t bar0 = base + kOffBar;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sbase + kOffBar + 8 * kNumBars);
@@ -168,205 +238,206 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t num_tiles = (n + kTile - 1) / kTile;
+  const int64_t my_tiles = num_tiles > blockIdx.x ? (num_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
 
   if (threadIdx.x == 0) {
     mbar_init(bar(kBarConst), 1);
-    mbar_init(bar(kBarKFull), 1);
-    mbar_init(bar(kBarKEmpty), 128);
-    mbar_init(bar(kBarD1Full), 1);
-    mbar_init(bar(kBarD1Empty), 128);
-    mbar_init(bar(kBarRFull), 128);
-    mbar_init(bar(kBarD2Full), 1);
-    mbar_init(bar(kBarD2Empty), 128);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(kBarKFull + s), 1);
+      mbar_init(bar(kBarKEmpty + s), 1);
+      mbar_init(bar(kBarD1Full + s), 1);
+      mbar_init(bar(kBarRFull + s), 128);
+      mbar_init(bar(kBarD2Full + s), 1);
+      mbar_init(bar(kBarFree + s), 128);
+    }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
-  if (warp == 5) {
+  if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                 "r"(256));
+                 "r"(512));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tmem_d1 = tmem, tmem_d2 = tmem + 128;
 
-  if (warp == 4) {
-    // ------------------------------------------------------------ producer
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       mbar_expect_tx(bar(kBarConst), 131072u);
       for (int c = 0; c < 8; ++c) bulk_load(base + 16384u * c, bimg + 16384 * c, 16384u, bar(kBarConst));
       int64_t i = 0;
-      for (int64_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++i) {
-        if (i > 0 && !mbar_wait(bar(kBarKEmpty), uint32_t((i - 1) & 1), abort_flag, status)) break;
-        mbar_expect_tx(bar(kBarKFull), 32768u);
-        tma_load_2d(base + kOffKey, &key_map, 0, int(tile * kTile), bar(kBarKFull));
-        tma_load_2d(base + kOffKey + 16384u, &key_map, 64, int(tile * kTile), bar(kBarKFull));
+      for (; i < my_tiles; ++i) {
+        const int kb = int(i & 1);
+        if (i >= 2 && !mbar_wait(bar(kBarKEmpty + kb), uint32_t(((i >> 1) - 1) & 1), abort_flag, status)) break;
+        const int64_t tile = blockIdx.x + i * gridDim.x;
+        const uint32_t dst = base + kOffKey + 32768u * kb;
+        mbar_expect_tx(bar(kBarKFull + kb), 32768u);
+        tma_load_2d(dst, &key_map, 0, int(tile * kTile), bar(kBarKFull + kb));
+        tma_load_2d(dst + 16384u, &key_map, 64, int(tile * kTile), bar(kBarKFull + kb));
       }
-      // do not leave with a copy in flight
-      if (i > 0) mbar_wait(bar(kBarKFull), uint32_t((i - 1) & 1), abort_flag, status);
+      // leave no copy in flight: wait for the last loads issued to each buffer
+      for (int64_t j = (i >= 2 ? i - 2 : 0); j < i; ++j)
+        mbar_wait(bar(kBarKFull + int(j & 1)), uint32_t((j >> 1) & 1), abort_flag, status);
       mbar_wait(bar(kBarConst), 0u, abort_flag, status);
     }
-  } else if (warp == 5) {
+  } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
-      bool ok = mbar_wait(bar(kBarConst), 0u, abort_flag, status);
-      int64_t i = 0;
-      for (int64_t tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++i) {
-        if (!mbar_wait(bar(kBarKFull), uint32_t(i & 1), abort_flag, status)) break;
-        if (i > 0 && !mbar_wait(bar(kBarD1Empty), uint32_t((i - 1) & 1), abort_flag, status)) break;
+      auto issue_mma1 = [&](int64_t i) -> bool {
+        const int sl = int(i & 1);
+        if (!mbar_wait(bar(kBarKFull + sl), uint32_t((i >> 1) & 1), abort_flag, status)) return false;
+        if (i >= 2 && !mbar_wait(bar(kBarFree + sl), uint32_t(((i >> 1) - 1) & 1), abort_flag, status)) return false;
         tc_fence_after();
+        const uint32_t d1 = tmem + 256u * sl;
+        const uint32_t kbase = base + kOffKey + 32768u * sl;
         uint32_t acc = 0;
         for (int pass = 0; pass < 2; ++pass)
           for (int kb = 0; kb < 2; ++kb)
             for (int ks = 0; ks < 4; ++ks) {
               const uint32_t off = 16384u * kb + 32u * ks;
-              mma_f16(tmem_d1, smem_desc(base + kOffKey + off), smem_desc(base + (pass ? kOffRlo : kOffRhi) + off),
-                      kIdescBf16, acc);
+              mma_f16(d1, smem_desc(kbase + off), smem_desc(base + (pass ? kOffRlo : kOffRhi) + off), kIdescBf16,
+                      acc);
               acc = 1;
             }
-        mma_commit(bar(kBarD1Full));
-        if (!mbar_wait(bar(kBarRFull), uint32_t(i & 1), abort_flag, status)) break;
-        if (i > 0 && !mbar_wait(bar(kBarD2Empty), uint32_t((i - 1) & 1), abort_flag, status)) break;
+        mma_commit(bar(kBarD1Full + sl));
+        mma_commit(bar(kBarKEmpty + sl));
+        return true;
+      };
+      auto issue_mma2 = [&](int64_t i) -> bool {
+        const int sl = int(i & 1);
+        if (!mbar_wait(bar(kBarRFull + sl), uint32_t((i >> 1) & 1), abort_flag, status)) return false;
         tc_fence_after();
-        acc = 0;
+        const uint32_t d1 = tmem + 256u * sl, d2 = d1 + 128u;
+        uint32_t acc = 0;
         for (int pass = 0; pass < 3; ++pass) {
-          const uint32_t a_off = pass == 2 ? kOffAlo : kOffAhi;
+          const uint32_t a_lo = pass == 2 ? 16u : 0u;
           const uint32_t b_off = pass == 1 ? kOffPlo : kOffPhi;
-          for (int kb = 0; kb < 2; ++kb)
-            for (int ks = 0; ks < 4; ++ks) {
-              const uint32_t off = 16384u * kb + 32u * ks;
-              mma_f16(tmem_d2, smem_desc(base + a_off + off), smem_desc(base + b_off + off), kIdescF16, acc);
-              acc = 1;
-            }
+          for (int k = 0; k < 8; ++k) {
+            // residual coordinates 16k .. 16k+15: chunk k/2, half k%2 (8 columns of packed pairs)
+            const uint32_t a_tmem = d1 + 32u * uint32_t(k >> 1) + 8u * uint32_t(k & 1) + a_lo;
+            const uint32_t off = 16384u * uint32_t(k >> 2) + 32u * uint32_t(k & 3);
+            mma_f16_ts(d2, a_tmem, smem_desc(base + b_off + off), kIdescF16, acc);
+            acc = 1;
+          }
         }
-        mma_commit(bar(kBarD2Full));
+        mma_commit(bar(kBarD2Full + sl));
+        return true;
+      };
+      bool ok = mbar_wait(bar(kBarConst), 0u, abort_flag, status);
+      if (ok && my_tiles > 0) ok = issue_mma1(0);
+      int64_t i = 0;
+      for (; ok && i < my_tiles; ++i) {
+        if (i + 1 < my_tiles && !issue_mma1(i + 1)) break;
+        if (!issue_mma2(i)) break;
       }
       // wait for the last MMAs before TMEM is released
-      if (i > 0) mbar_wait(bar(kBarD2Full), uint32_t((i - 1) & 1), abort_flag, status);
+      for (int64_t j = (i >= 2 ? i - 2 : 0); j < i; ++j)
+        mbar_wait(bar(kBarD2Full + int(j & 1)), uint32_t((j >> 1) & 1), abort_flag, status);
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int row = threadIdx.x;          // 0..127 = TMEM lane
-    const uint32_t lane_addr = uint32_t(warp * 32) << 16;
-    constexpr int kCodeWords = BMSE;      // per quarter: 2 units x BMSE halfwords = BMSE words
+    // warps 2..5 take local tiles 0, 2, 4, ... (TMEM slot 0); warps 6..9 the odd ones (slot 1)
+    const int grp = (warp - 2) >> 2;
+    const int row = (warp & 3) * 32 + lane;          // TMEM lane = key row within the tile
+    const uint32_t lane_addr = uint32_t((warp & 3) * 32) << 16;
+    const uint32_t d1 = tmem + 256u * grp + lane_addr, d2 = d1 + 128u;
+    constexpr int kCodeWords = BMSE;                 // per quarter: 2 units x BMSE halfwords
     constexpr int kRowBytes = kD * BMSE / 8 + kD / 8;
-    int64_t i = 0;
-    for (int64_t tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++i) {
-      const uint32_t par = uint32_t(i & 1);
-      if (!mbar_wait(bar(kBarKFull), par, abort_flag, status)) break;
-      // ||k||^2 from this row of the swizzled key tile
-      float n2 = 0.f;
-#pragma unroll
-      for (int kb = 0; kb < 2; ++kb)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 v = *reinterpret_cast<const uint4*>(sbase + kOffKey + 16384 * kb + row * 128 +
-                                                          ((c ^ (row & 7)) * 16));
-          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            const float lo = __uint_as_float(w[h] << 16), hi = __uint_as_float(w[h] & 0xFFFF0000u);
-            n2 = fmaf(lo, lo, n2);
-            n2 = fmaf(hi, hi, n2);
-          }
-        }
-      const float nk = sqrtf(n2);
-      const float inv_n = nk > 0.f ? 1.0f / nk : 0.f;
-      if (!mbar_wait(bar(kBarD1Full), par, abort_flag, status)) break;
-      mbar_arrive(bar(kBarKEmpty));
+    int64_t k = 0;
+    for (int64_t i = grp; i < my_tiles; i += 2, ++k) {
+      const uint32_t par = uint32_t(k & 1);
+      if (!mbar_wait(bar(kBarD1Full + grp), par, abort_flag, status)) break;
       tc_fence_after();
+      // ||k||^2 = ||R k||^2 from the rotated row
+      float n2 = 0.f;
+#pragma unroll 1
+      for (int q = 0; q < 4; ++q) {
+        float y[32];
+        tmem_ld32(d1 + 32u * q, y);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) n2 = fmaf(y[j], y[j], n2);
+      }
+      const float nk = sqrtf(n2);
+      const bool zero = !(n2 > 0.f);
+      const float s128 = zero ? 0.f : 128.f / nk;
+      HalfBook hb = book;
+      if (zero) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) hb.C[c] = 0.f;
+      }
       uint32_t codew[4][kCodeWords];
       float rr = 0.f;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         float y[32];
-        tmem_ld32(tmem_d1 + lane_addr + 32u * q, y);
+        tmem_ld32(d1 + 32u * q, y);
         uint32_t hw[2 * BMSE];
 #pragma unroll
         for (int h = 0; h < 2 * BMSE; ++h) hw[h] = 0;
-        uint32_t rh[16], rl[16];    // 32 fp16 values of r_hi / r_lo, packed in pairs
+        uint32_t rh[16], rl[16];
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) {
-          const float u = y[jj] * inv_n;
-          int code = 0;
-          float level = cb.c[0];
+        for (int jj = 0; jj < 32; jj += 2) {
+          float r0, r1;
+          const uint32_t c0 = cell<BMSE>(y[jj] * s128, hb, r0);
+          const uint32_t c1 = cell<BMSE>(y[jj + 1] * s128, hb, r1);
+          rr = fmaf(r0, r0, rr);
+          rr = fmaf(r1, r1, rr);
+          const __half2 hi = __floats2half2_rn(r0, r1);
+          const float2 hf = __half22float2(hi);
+          const __half2 lo = __floats2half2_rn(r0 - hf.x, r1 - hf.y);
+          rh[jj >> 1] = *reinterpret_cast<const uint32_t*>(&hi);
+          rl[jj >> 1] = *reinterpret_cast<const uint32_t*>(&lo);
 #pragma unroll
-          for (int b = 0; b < (1 << BMSE) - 1; ++b) {
-            const bool above = u > cb.t[b];
-            code += above ? 1 : 0;
-            level = above ? cb.c[b + 1] : level;
-          }
-          const float r = nk > 0.f ? u - level : 0.f;
-          if (nk == 0.f) code = 0;
-          rr = fmaf(r, r, rr);
-          const int rreg = jj >> 2, e = jj & 3, uu = rreg >> 2, ii = rreg & 3;
-          if constexpr (BMSE == 3) {
-            if (ii < 3) {
-              hw[uu * 3 + ii] |= uint32_t(code) << (4 * e);
+          for (int t2 = 0; t2 < 2; ++t2) {
+            const int j = jj + t2;
+            const uint32_t code = t2 ? c1 : c0;
+            const int rreg = j >> 2, e = j & 3, uu = rreg >> 2, ii = rreg & 3;
+            if constexpr (BMSE == 3) {
+              if (ii < 3) {
+                hw[uu * 3 + ii] |= code << (4 * e);
+              } else {
+#pragma unroll
+                for (int b = 0; b < 3; ++b) hw[uu * 3 + b] |= ((code >> b) & 1u) << (4 * e + 3);
+              }
+            } else if constexpr (BMSE == 2) {
+              hw[uu * 2 + (ii >> 1)] |= code << (4 * e + 2 * (ii & 1));
             } else {
-#pragma unroll
-              for (int b = 0; b < 3; ++b) hw[uu * 3 + b] |= uint32_t((code >> b) & 1) << (4 * e + 3);
+              hw[uu] |= code << (4 * e + ii);
             }
-          } else if constexpr (BMSE == 2) {
-            hw[uu * 2 + (ii >> 1)] |= uint32_t(code) << (4 * e + 2 * (ii & 1));
-          } else {
-            hw[uu] |= uint32_t(code) << (4 * e + ii);
-          }
-          const float rs = r * 128.f;
-          const __half hi = __float2half_rn(rs);
-          const __half lo = __float2half_rn(rs - __half2float(hi));
-          const uint32_t hb = __half_as_ushort(hi), lb = __half_as_ushort(lo);
-          if (jj & 1) {
-            rh[jj >> 1] |= hb << 16;
-            rl[jj >> 1] |= lb << 16;
-          } else {
-            rh[jj >> 1] = hb;
-            rl[jj >> 1] = lb;
           }
         }
+        // the residual overwrites the 32 columns of y just read (A operand of the JL product)
+        tmem_st16(d1 + 32u * q, rh);
+        tmem_st16(d1 + 32u * q + 16u, rl);
 #pragma unroll
-        for (int w = 0; w < kCodeWords; ++w) codew[q][w] = hw[2 * w] | (hw[2 * w + 1] << 16);
-        // residual columns 32q .. 32q+31 -> K block q/2, 16-byte chunks 4(q%2) .. 4(q%2)+3
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          const int chunk = 4 * (q & 1) + cc;
-          const uint32_t off = 16384u * uint32_t(q >> 1) + uint32_t(row) * 128u + uint32_t((chunk ^ (row & 7)) * 16);
-          *reinterpret_cast<uint4*>(sbase + kOffAhi + off) =
-              make_uint4(rh[4 * cc], rh[4 * cc + 1], rh[4 * cc + 2], rh[4 * cc + 3]);
-          *reinterpret_cast<uint4*>(sbase + kOffAlo + off) =
-              make_uint4(rl[4 * cc], rl[4 * cc + 1], rl[4 * cc + 2], rl[4 * cc + 3]);
-        }
+        for (int w = 0; w < kCodeWords; ++w) codew[q][w] = zero ? 0u : (hw[2 * w] | (hw[2 * w + 1] << 16));
       }
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       tc_fence_before();
-      mbar_arrive(bar(kBarD1Empty));
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      mbar_arrive(bar(kBarRFull));
-      const float rho = nk * sqrtf(rr);
-      if (!mbar_wait(bar(kBarD2Full), par, abort_flag, status)) break;
+      mbar_arrive(bar(kBarRFull + grp));
+      const float rho = nk * sqrtf(rr) * (1.0f / 128.f);
+      if (!mbar_wait(bar(kBarD2Full + grp), par, abort_flag, status)) break;
       tc_fence_after();
       uint32_t signw[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         float z[32];
-        tmem_ld32(tmem_d2 + lane_addr + 32u * q, z);
-        uint32_t s0 = 0, s1 = 0;
+        tmem_ld32(d2 + 32u * q, z);
+        uint32_t sw = 0;
 #pragma unroll
         for (int jj = 0; jj < 32; ++jj) {
           const int rreg = jj >> 2, e = jj & 3, uu = rreg >> 2, ii = rreg & 3;
-          const uint32_t bit = z[jj] >= 0.f ? 1u : 0u;
-          if (uu == 0)
-            s0 |= bit << (4 * e + ii);
-          else
-            s1 |= bit << (4 * e + ii);
+          sw |= (z[jj] >= 0.f ? 1u : 0u) << (16 * uu + 4 * e + ii);
         }
-        signw[q] = s0 | (s1 << 16);
+        signw[q] = sw;
       }
       tc_fence_before();
-      mbar_arrive(bar(kBarD2Empty));
-      const int64_t key = tile * kTile + row;
+      mbar_arrive(bar(kBarFree + grp));
+      const int64_t key = (blockIdx.x + i * gridDim.x) * kTile + row;
       if (key < n) {
         uint8_t* dst = payload + key * kRowBytes;
 #pragma unroll
@@ -390,9 +461,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(256));
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
   }
 }
 
@@ -441,23 +512,27 @@ cudaError_t launch_quantize_tc(const tq_ctx* ctx, const void* keys, int dtype, i
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t tiles = (n + kTile - 1) / kTile;
   const int grid = int(tiles < sms ? tiles : sms);
+  HalfBook hb{};
+  const int L = ctx->levels;
+  for (int i = 0; i < L / 2 - 1; ++i) hb.T[i] = float(128.0 * ctx->t[L / 2 + i]);
+  for (int i = 0; i < L / 2; ++i) hb.C[i] = float(128.0 * ctx->c[L / 2 + i]);
   switch (ctx->bmse) {
     case 1: {
       auto k = quantize_tc_kernel<1>;
       cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
-      k<<<grid, kThreadsTc, kSmemBytes, st>>>(map, n, ctx->dBimg, ctx->cb, payload, norms, ctx->dstatus);
+      k<<<grid, kThreadsTc, kSmemBytes, st>>>(map, n, ctx->dBimg, hb, payload, norms, ctx->dstatus);
       break;
     }
     case 2: {
       auto k = quantize_tc_kernel<2>;
       cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
-      k<<<grid, kThreadsTc, kSmemBytes, st>>>(map, n, ctx->dBimg, ctx->cb, payload, norms, ctx->dstatus);
+      k<<<grid, kThreadsTc, kSmemBytes, st>>>(map, n, ctx->dBimg, hb, payload, norms, ctx->dstatus);
       break;
     }
     default: {
       auto k = quantize_tc_kernel<3>;
       cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
-      k<<<grid, kThreadsTc, kSmemBytes, st>>>(map, n, ctx->dBimg, ctx->cb, payload, norms, ctx->dstatus);
+      k<<<grid, kThreadsTc, kSmemBytes, st>>>(map, n, ctx->dBimg, hb, payload, norms, ctx->dstatus);
       break;
     }
   }
