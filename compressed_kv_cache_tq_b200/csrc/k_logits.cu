@@ -47,7 +47,7 @@ struct HeadScale {
 // Query preparation: x = R q, y = P x (= S q), int16 fixed point per head,
 // split into two signed int8 limbs, written in MMA B-fragment order.
 // One block per (batch, kv head) group computes all 4 NT head slots; slots
-// >= G are zero.  R^T and then P^T are staged in shared memory (64 KB).
+// >= G are zero.  R^T and P^T are copied to shared memory (128 KB) at once.
 // ---------------------------------------------------------------------------
 constexpr int kMaxSlots = 8;
 
@@ -56,8 +56,9 @@ __global__ void __launch_bounds__(128) qprep_kernel(const float* __restrict__ q,
                                                     float code_inv_scale, float scale, float qjl_over_m,
                                                     uint32_t* __restrict__ frags, HeadScale* __restrict__ hscale) {
   extern __shared__ float smq[];
-  float* mat = smq;                                  // [D][D] R^T, then P^T
-  float* sq = mat + D * D;                           // [slots][D] queries, then y
+  float* matR = smq;                                 // [D][D] R^T
+  float* matP = matR + D * D;                        // [D][D] P^T
+  float* sq = matP + D * D;                          // [slots][D] queries
   float* sx = sq + kMaxSlots * D;                    // [slots][D] x
   __shared__ float red[2][kMaxSlots][4];
   __shared__ int8_t limbs[kMaxSlots][2][2][D];       // [slot][x/y][hi/lo][coordinate]
@@ -65,23 +66,28 @@ __global__ void __launch_bounds__(128) qprep_kernel(const float* __restrict__ q,
   const int slots = nt_per_group * HPT;
   const int grp = blockIdx.x, b = grp / Hkv, hkv = grp % Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (int i = tid; i < D * D / 4; i += 128)
-    reinterpret_cast<float4*>(mat)[i] = __ldg(reinterpret_cast<const float4*>(Rt) + i);
+  // both matrices in flight at once (asynchronous 16-byte copies)
+  for (int i = tid; i < D * D / 4; i += 128) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(uint32_t(__cvta_generic_to_shared(matR + 4 * i))),
+                 "l"(Rt + 4 * i)
+                 : "memory");
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(uint32_t(__cvta_generic_to_shared(matP + 4 * i))),
+                 "l"(Pt + 4 * i)
+                 : "memory");
+  }
   for (int h = 0; h < slots; ++h) sq[h * D + tid] = h < G ? q[(size_t(b) * Hq + hkv * G + h) * D + tid] : 0.f;
+  asm volatile("cp.async.wait_all;" ::: "memory");
   __syncthreads();
   float acc[kMaxSlots];
 #pragma unroll
   for (int h = 0; h < kMaxSlots; ++h) acc[h] = 0.f;
 #pragma unroll 4
   for (int i = 0; i < D; ++i) {
-    const float r = mat[i * D + tid];
+    const float r = matR[i * D + tid];
 #pragma unroll
     for (int h = 0; h < kMaxSlots; ++h)
       if (h < slots) acc[h] = fmaf(r, sq[h * D + i], acc[h]);
   }
-  __syncthreads();
-  for (int i = tid; i < D * D / 4; i += 128)
-    reinterpret_cast<float4*>(mat)[i] = __ldg(reinterpret_cast<const float4*>(Pt) + i);
 #pragma unroll
   for (int h = 0; h < kMaxSlots; ++h)
     if (h < slots) sx[h * D + tid] = acc[h];
@@ -91,7 +97,7 @@ __global__ void __launch_bounds__(128) qprep_kernel(const float* __restrict__ q,
   for (int h = 0; h < kMaxSlots; ++h) accy[h] = 0.f;
 #pragma unroll 4
   for (int j = 0; j < D; ++j) {
-    const float p = mat[j * D + tid];
+    const float p = matP[j * D + tid];
 #pragma unroll
     for (int h = 0; h < kMaxSlots; ++h)
       if (h < slots) accy[h] = fmaf(p, sx[h * D + j], accy[h]);
@@ -161,6 +167,17 @@ __device__ __forceinline__ void mma_s8(int (&c)[4], uint32_t a0, uint32_t a1, ui
       "{%0,%1,%2,%3};\n"
       : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// First k-step: D = A B with a zero accumulator input.
+__device__ __forceinline__ void mma_s8_first(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                             uint32_t b0, uint32_t b1) {
+  const int z = 0;
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%10,%10,%10,%10};\n"
+      : "=r"(c[0]), "=r"(c[1]), "=r"(c[2]), "=r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(z));
 }
 
 // Chunk of one key for one quarter: BMSE * 2 halfwords of codes (two units)
@@ -310,10 +327,6 @@ __global__ void __launch_bounds__(kLogitThreads) logits_mma_kernel(
 
     uint32_t sa[8], sb[8];
     int acc_hi[NT][4], acc_lo[NT][4], acc_sg[NT][4];
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) acc_hi[nt][i] = acc_lo[nt][i] = acc_sg[nt][i] = 0;
 
     code_selectors<BMSE>(ca, sa);
     code_selectors<BMSE>(cb, sb);
@@ -327,8 +340,13 @@ __global__ void __launch_bounds__(kLogitThreads) logits_mma_kernel(
                      al3 = prmt(lut.lo[0], lut.lo[1], sb[2 * s + 1]);
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        mma_s8(acc_hi[nt], ah0, ah1, ah2, ah3, bx[nt][s][0], bx[nt][s][1]);
-        mma_s8(acc_lo[nt], al0, al1, al2, al3, bx[nt][s][0], bx[nt][s][1]);
+        if (s == 0) {
+          mma_s8_first(acc_hi[nt], ah0, ah1, ah2, ah3, bx[nt][s][0], bx[nt][s][1]);
+          mma_s8_first(acc_lo[nt], al0, al1, al2, al3, bx[nt][s][0], bx[nt][s][1]);
+        } else {
+          mma_s8(acc_hi[nt], ah0, ah1, ah2, ah3, bx[nt][s][0], bx[nt][s][1]);
+          mma_s8(acc_lo[nt], al0, al1, al2, al3, bx[nt][s][0], bx[nt][s][1]);
+        }
       }
     }
     // sign registers: selectors keep one bit per nibble; the byte table maps
@@ -339,8 +357,12 @@ __global__ void __launch_bounds__(kLogitThreads) logits_mma_kernel(
 #pragma unroll
     for (int s = 0; s < KS; ++s)
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt)
-        mma_s8(acc_sg[nt], ga[2 * s], gb[2 * s], ga[2 * s + 1], gb[2 * s + 1], by[nt][s][0], by[nt][s][1]);
+      for (int nt = 0; nt < NT; ++nt) {
+        if (s == 0)
+          mma_s8_first(acc_sg[nt], ga[0], gb[0], ga[1], gb[1], by[nt][0][0], by[nt][0][1]);
+        else
+          mma_s8(acc_sg[nt], ga[2 * s], gb[2 * s], ga[2 * s + 1], gb[2 * s + 1], by[nt][s][0], by[nt][s][1]);
+      }
 
     // epilogue: C[row][2 tig + limb] -> head tig of each N-tile
     const float kna = __half2float(__ushort_as_half(uint16_t(na)));
@@ -351,12 +373,11 @@ __global__ void __launch_bounds__(kLogitThreads) logits_mma_kernel(
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const int hg = nt * HPT + tig;
-      const float codeA = float(acc_hi[nt][0]) * 65536.f + float(acc_hi[nt][1] + acc_lo[nt][0]) * 256.f +
-                          float(acc_lo[nt][1]);
-      const float codeB = float(acc_hi[nt][2]) * 65536.f + float(acc_hi[nt][3] + acc_lo[nt][2]) * 256.f +
-                          float(acc_lo[nt][3]);
-      const float signA = float(acc_sg[nt][0]) * 256.f + float(acc_sg[nt][1]);
-      const float signB = float(acc_sg[nt][2]) * 256.f + float(acc_sg[nt][3]);
+      // |cross terms| <= 2 * 128 * 128 * 128 and |low terms| < 2^21: the integer sums fit in 32 bits
+      const float codeA = float(acc_hi[nt][0]) * 65536.f + float((acc_hi[nt][1] + acc_lo[nt][0]) * 256 + acc_lo[nt][1]);
+      const float codeB = float(acc_hi[nt][2]) * 65536.f + float((acc_hi[nt][3] + acc_lo[nt][2]) * 256 + acc_lo[nt][3]);
+      const float signA = float(acc_sg[nt][0] * 256 + acc_sg[nt][1]);
+      const float signB = float(acc_sg[nt][2] * 256 + acc_sg[nt][3]);
       float* o = obase[nt] + s0;
       if (hg < G) {
         if (okA) o[g] = kna * codeA * sc_code[nt] + kra * signA * sc_sign[nt];
@@ -467,7 +488,7 @@ cudaError_t launch_logits(const tq_ctx* ctx, const float* q, int B, int Hq, int 
   uint32_t* frags = static_cast<uint32_t*>(ws);
   const size_t frag_bytes = ((size_t(groups) * nt * kFragWords * 4 + 255) / 256) * 256;
   HeadScale* hs = reinterpret_cast<HeadScale*>(static_cast<uint8_t*>(ws) + frag_bytes);
-  const size_t qp_smem = size_t(D * D + 2 * kMaxSlots * D) * 4;
+  const size_t qp_smem = size_t(2 * D * D + 2 * kMaxSlots * D) * 4;
   cudaFuncSetAttribute(qprep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(qp_smem));
   qprep_kernel<<<unsigned(groups), 128, qp_smem, st>>>(q, Hq, Hkv, nt, ctx->dRt, ctx->dPt, ctx->lut.inv_scale,
                                                         scale, float(kQjlConst / ctx->m), frags, hs);

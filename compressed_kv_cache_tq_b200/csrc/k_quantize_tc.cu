@@ -49,7 +49,10 @@ constexpr int kThreadsTc = 320;
 
 constexpr uint32_t kOffRhi = 0, kOffRlo = 32768, kOffPhi = 65536, kOffPlo = 98304;
 constexpr uint32_t kOffKey = 131072;     // two 32 KB key tiles
-constexpr uint32_t kOffBar = 196608;
+constexpr uint32_t kOffStage = 196608;  // packed rows of the two epilogue groups
+constexpr int kStageWords = 20;         // 64-byte row padded to 80 bytes (conflict-free 16-byte accesses)
+constexpr uint32_t kStageBytes = 128u * kStageWords * 4u;
+constexpr uint32_t kOffBar = kOffStage + 2 * kStageBytes;
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;   // + slack for 1024-byte alignment
 
 // barriers; the per-slot ones come in pairs (slot 0, slot 1)
@@ -346,7 +349,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
     const uint32_t lane_addr = uint32_t((warp & 3) * 32) << 16;
     const uint32_t d1 = tmem + 256u * grp + lane_addr, d2 = d1 + 128u;
     constexpr int kCodeWords = BMSE;                 // per quarter: 2 units x BMSE halfwords
-    constexpr int kRowBytes = kD * BMSE / 8 + kD / 8;
+    constexpr int kRowBytes = kD * BMSE / 8 + kD / 8;  // = 16 (BMSE + 1)
     int64_t k = 0;
     for (int64_t i = grp; i < my_tiles; i += 2, ++k) {
       const uint32_t par = uint32_t(k & 1);
@@ -369,9 +372,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
 #pragma unroll
         for (int c = 0; c < 4; ++c) hb.C[c] = 0.f;
       }
-      uint32_t codew[4][kCodeWords];
+      // packed row staged in shared memory: chunk q at 16 q (BMSE + 1) / 4 ... as 32-bit words
+      uint32_t* srow = reinterpret_cast<uint32_t*>(sbase + kOffStage + grp * kStageBytes) + row * kStageWords;
       float rr = 0.f;
-#pragma unroll
+#pragma unroll 1
       for (int q = 0; q < 4; ++q) {
         float y[32];
         tmem_ld32(d1 + 32u * q, y);
@@ -414,7 +418,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
         tmem_st16(d1 + 32u * q, rh);
         tmem_st16(d1 + 32u * q + 16u, rl);
 #pragma unroll
-        for (int w = 0; w < kCodeWords; ++w) codew[q][w] = zero ? 0u : (hw[2 * w] | (hw[2 * w + 1] << 16));
+        for (int w = 0; w < kCodeWords; ++w)
+          srow[q * (BMSE + 1) + w] = zero ? 0u : (hw[2 * w] | (hw[2 * w + 1] << 16));
       }
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       tc_fence_before();
@@ -422,8 +427,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
       const float rho = nk * sqrtf(rr) * (1.0f / 128.f);
       if (!mbar_wait(bar(kBarD2Full + grp), par, abort_flag, status)) break;
       tc_fence_after();
-      uint32_t signw[4];
-#pragma unroll
+#pragma unroll 1
       for (int q = 0; q < 4; ++q) {
         float z[32];
         tmem_ld32(d2 + 32u * q, z);
@@ -433,25 +437,25 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
           const int rreg = jj >> 2, e = jj & 3, uu = rreg >> 2, ii = rreg & 3;
           sw |= (z[jj] >= 0.f ? 1u : 0u) << (16 * uu + 4 * e + ii);
         }
-        signw[q] = sw;
+        srow[q * (BMSE + 1) + BMSE] = sw;
       }
       tc_fence_before();
       mbar_arrive(bar(kBarFree + grp));
       const int64_t key = (blockIdx.x + i * gridDim.x) * kTile + row;
       if (key < n) {
         uint8_t* dst = payload + key * kRowBytes;
+        if constexpr (BMSE == 3) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t* d32 = reinterpret_cast<uint32_t*>(dst + q * 4 * (BMSE + 1));
-          if constexpr (BMSE == 3) {
-            *reinterpret_cast<uint4*>(d32) = make_uint4(codew[q][0], codew[q][1], codew[q][2], signw[q]);
-          } else if constexpr (BMSE == 1) {
-            *reinterpret_cast<uint2*>(d32) = make_uint2(codew[q][0], signw[q]);
-          } else {
-            d32[0] = codew[q][0];
-            d32[1] = codew[q][1];
-            d32[2] = signw[q];
-          }
+          for (int c = 0; c < 4; ++c)
+            reinterpret_cast<uint4*>(dst)[c] = reinterpret_cast<const uint4*>(srow)[c];
+        } else if constexpr (BMSE == 1) {
+#pragma unroll
+          for (int c = 0; c < 2; ++c)
+            reinterpret_cast<uint4*>(dst)[c] = reinterpret_cast<const uint4*>(srow)[c];
+        } else {
+#pragma unroll
+          for (int c = 0; c < 3; ++c)
+            reinterpret_cast<uint4*>(dst)[c] = reinterpret_cast<const uint4*>(srow)[c];
         }
         const uint32_t nn = uint32_t(__half_as_ushort(__float2half_rn(nk))) |
                             (uint32_t(__half_as_ushort(__float2half_rn(rho))) << 16);
