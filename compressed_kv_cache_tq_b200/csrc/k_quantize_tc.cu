@@ -45,14 +45,15 @@ namespace {
 
 constexpr int kD = 128;
 constexpr int kTile = 128;
-constexpr int kThreadsTc = 320;
+constexpr int kThreadsTc = 576;   // 2 control warps + 16 epilogue warps
 
 constexpr uint32_t kOffRhi = 0, kOffRlo = 32768, kOffPhi = 65536, kOffPlo = 98304;
 constexpr uint32_t kOffKey = 131072;     // two 32 KB key tiles
 constexpr uint32_t kOffStage = 196608;  // packed rows of the two epilogue groups
 constexpr int kStageWords = 20;         // 64-byte row padded to 80 bytes (conflict-free 16-byte accesses)
 constexpr uint32_t kStageBytes = 128u * kStageWords * 4u;
-constexpr uint32_t kOffBar = kOffStage + 2 * kStageBytes;
+constexpr uint32_t kOffPart = kOffStage + 2 * kStageBytes;   // row partial sums [slot][n^2 | rr][half][row]
+constexpr uint32_t kOffBar = kOffPart + 2 * 512 * 4;
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;   // + slack for 1024-byte alignment
 
 // barriers; the per-slot ones come in pairs (slot 0, slot 1)
@@ -63,7 +64,7 @@ enum Bar {
   kBarD1Full = 5,
   kBarRFull = 7,
   kBarD2Full = 9,
-  kBarFree = 11,
+  kBarD2Free = 11,
   kNumBars = 13
 };
 
@@ -82,20 +83,23 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
+// One test of the phase with a suspend-time hint: the thread may sleep until
+// the phase completes (or about 0.5 ms pass) instead of spinning.
 __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.b32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(500000u)
       : "memory");
   return ok != 0;
 }
 // Bounded wait: false when the budget ran out or another role gave up.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           uint32_t* status) {
+  if (mbar_try(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try(bar, parity)) {
     if (*abort_flag) return false;
@@ -153,6 +157,28 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
 
+__device__ __forceinline__ void named_barrier(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// 32 consecutive TMEM columns of this thread's lane, without waiting (the
+// registers are valid after tmem_wait_ld()).
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 // 32 consecutive TMEM columns of this thread's lane.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   uint32_t r[32];
@@ -178,6 +204,12 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       : "memory");
 }
 
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
 // A operand from tensor memory, B from shared memory.
 __device__ __forceinline__ void mma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t b, uint32_t idesc,
                                            uint32_t acc) {
@@ -189,38 +221,42 @@ __device__ __forceinline__ void mma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uin
       : "memory");
 }
 
-// Positive half of the symmetric codebook, scaled by 128 (the residual scale).
+// Positive half of the symmetric codebook, scaled by 128 (the residual scale),
+// pre-arranged for the arithmetic cell search below.
 struct HalfBook {
-  float T[3];   // boundaries above 0 (t_{L/2} .. t_{L-2})
-  float C[4];   // levels above 0 (c_{L/2} .. c_{L-1})
+  float Tneg[3];   // -2^100 x boundaries above 0 (t_{L/2} .. t_{L-2})
+  float C0;        // smallest positive level
+  float dC[3];     // level steps c_{L/2+i+1} - c_{L/2+i}
 };
 
-// Cell index and scaled residual of one rotated coordinate u (already x128).
-// The codebook is symmetric with t_{L/2-1} = 0, so idx = #{i : t_i < u} is
-// L/2 + #{boundaries above 0 below |u|} for u > 0 and L/2 - 1 - (that count)
-// otherwise (exact ties at +-t_i resolve within rounding of the boundary).
+constexpr float kBig = 0x1p100f;
+
+// Cell index and scaled residual of one rotated coordinate u (already x128),
+// in fused multiply-adds only.  The codebook is symmetric with t_{L/2-1} = 0,
+// so idx = #{i : t_i < u} = L/2 + m for u > 0 and L/2 - 1 - m otherwise, where
+// m = #{boundaries above 0 that are below |u|}.  Each indicator [|u| > T] is
+// sat(2^100 |u| - 2^100 T): exact 0 or 1, because the difference of two
+// floats of this range is either 0 or far above 2^-100 (an exact tie at a
+// boundary resolves within rounding of the boundary).  The returned value
+// is the float bit pattern of 2^23 + idx.
 template <int BMSE>
-__device__ __forceinline__ uint32_t cell(float u, const HalfBook& hb, float& r) {
+__device__ __forceinline__ uint32_t cell_bits(float u, const HalfBook& hb, float& r) {
   const float a = fabsf(u);
-  const bool pos = u > 0.f;
-  uint32_t mag;
-  float lv;
-  if constexpr (BMSE == 3) {
-    const bool p1 = a > hb.T[0], p2 = a > hb.T[1], p3 = a > hb.T[2];
-    mag = p3 ? 3u : (p2 ? 2u : (p1 ? 1u : 0u));
-    lv = p3 ? hb.C[3] : (p2 ? hb.C[2] : (p1 ? hb.C[1] : hb.C[0]));
-    r = u - (pos ? lv : -lv);
-    return pos ? 4u + mag : 3u - mag;
-  } else if constexpr (BMSE == 2) {
-    const bool p1 = a > hb.T[0];
-    mag = p1 ? 1u : 0u;
-    lv = p1 ? hb.C[1] : hb.C[0];
-    r = u - (pos ? lv : -lv);
-    return pos ? 2u + mag : 1u - mag;
-  } else {
-    r = u - (pos ? hb.C[0] : -hb.C[0]);
-    return pos ? 1u : 0u;
+  const float sp = __saturatef(u * kBig);            // [u > 0]
+  const float sgn = fmaf(2.f, sp, -1.f);             // +1 for u > 0, else -1
+  float m = 0.f, lv = hb.C0;
+#pragma unroll
+  for (int i = 0; i < (1 << (BMSE - 1)) - 1; ++i) {
+    const float step = __saturatef(fmaf(a, kBig, hb.Tneg[i]));
+    m += step;
+    lv = fmaf(step, hb.dC[i], lv);
   }
+  r = fmaf(-sgn, lv, u);                              // u - sign(u) level
+  // idx = (L/2 - 1/2 + sgn/2) + sgn m, an exact small integer; adding 2^23
+  // puts it in the low mantissa bits
+  constexpr float half_l = float(1 << (BMSE - 1)) - 0.5f;
+  const float base = fmaf(sgn, 0.5f, half_l);
+  return __float_as_uint(fmaf(sgn, m, base) + 8388608.f);
 }
 
 template <int BMSE>
@@ -249,9 +285,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
       mbar_init(bar(kBarKFull + s), 1);
       mbar_init(bar(kBarKEmpty + s), 1);
       mbar_init(bar(kBarD1Full + s), 1);
-      mbar_init(bar(kBarRFull + s), 128);
+      mbar_init(bar(kBarRFull + s), 256);
       mbar_init(bar(kBarD2Full + s), 1);
-      mbar_init(bar(kBarFree + s), 128);
+      mbar_init(bar(kBarD2Free + s), 256);
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -293,7 +329,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
       auto issue_mma1 = [&](int64_t i) -> bool {
         const int sl = int(i & 1);
         if (!mbar_wait(bar(kBarKFull + sl), uint32_t((i >> 1) & 1), abort_flag, status)) return false;
-        if (i >= 2 && !mbar_wait(bar(kBarFree + sl), uint32_t(((i >> 1) - 1) & 1), abort_flag, status)) return false;
+        // the slot's y / residual columns are free once the JL MMA of tile i - 2 completed
+        if (i >= 2 && !mbar_wait(bar(kBarD2Full + sl), uint32_t(((i >> 1) - 1) & 1), abort_flag, status))
+          return false;
         tc_fence_after();
         const uint32_t d1 = tmem + 256u * sl;
         const uint32_t kbase = base + kOffKey + 32768u * sl;
@@ -313,6 +351,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
       auto issue_mma2 = [&](int64_t i) -> bool {
         const int sl = int(i & 1);
         if (!mbar_wait(bar(kBarRFull + sl), uint32_t((i >> 1) & 1), abort_flag, status)) return false;
+        // the slot's z columns are free once the epilogue of tile i - 2 read them
+        if (i >= 2 && !mbar_wait(bar(kBarD2Free + sl), uint32_t(((i >> 1) - 1) & 1), abort_flag, status))
+          return false;
         tc_fence_after();
         const uint32_t d1 = tmem + 256u * sl, d2 = d1 + 128u;
         uint32_t acc = 0;
@@ -343,123 +384,147 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    // warps 2..5 take local tiles 0, 2, 4, ... (TMEM slot 0); warps 6..9 the odd ones (slot 1)
-    const int grp = (warp - 2) >> 2;
+    // 16 warps in 4 groups: group eg serves TMEM slot eg & 1 (local tiles of
+    // that parity) and quarters 2 (eg >> 1), 2 (eg >> 1) + 1 of every row; the
+    // two groups of a slot combine their row partial sums through shared
+    // memory around a named barrier (id 1 + slot, 256 threads).
+    const int eg = (warp - 2) >> 2;
+    const int slot = eg & 1, half = eg >> 1;
     const int row = (warp & 3) * 32 + lane;          // TMEM lane = key row within the tile
     const uint32_t lane_addr = uint32_t((warp & 3) * 32) << 16;
-    const uint32_t d1 = tmem + 256u * grp + lane_addr, d2 = d1 + 128u;
-    constexpr int kCodeWords = BMSE;                 // per quarter: 2 units x BMSE halfwords
+    const uint32_t d1 = tmem + 256u * slot + lane_addr, d2 = d1 + 128u;
     constexpr int kRowBytes = kD * BMSE / 8 + kD / 8;  // = 16 (BMSE + 1)
+    float* part = reinterpret_cast<float*>(sbase + kOffPart) + slot * 512;   // [n^2 | rr][half][row]
+    uint32_t* srow = reinterpret_cast<uint32_t*>(sbase + kOffStage + slot * kStageBytes) + row * kStageWords;
+    const int q0 = 2 * half;
     int64_t k = 0;
-    for (int64_t i = grp; i < my_tiles; i += 2, ++k) {
+    for (int64_t i = slot; i < my_tiles; i += 2, ++k) {
       const uint32_t par = uint32_t(k & 1);
-      if (!mbar_wait(bar(kBarD1Full + grp), par, abort_flag, status)) break;
+      if (!mbar_wait(bar(kBarD1Full + slot), par, abort_flag, status)) break;
       tc_fence_after();
-      // ||k||^2 = ||R k||^2 from the rotated row
-      float n2 = 0.f;
-#pragma unroll 1
-      for (int q = 0; q < 4; ++q) {
-        float y[32];
-        tmem_ld32(d1 + 32u * q, y);
+      // ||k||^2 = ||R k||^2 from the rotated row, half a row per group
+      float n2p = 0.f;
+      {
+        float y0[32], y1[32];
+        tmem_ld32_nowait(d1 + 32u * q0, y0);
+        tmem_ld32_nowait(d1 + 32u * (q0 + 1), y1);
+        tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) n2 = fmaf(y[j], y[j], n2);
+        for (int j = 0; j < 32; ++j) n2p = fmaf(y0[j], y0[j], n2p);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) n2p = fmaf(y1[j], y1[j], n2p);
       }
+      part[half * 128 + row] = n2p;
+      named_barrier(1 + slot, 256);
+      const float n2 = part[row] + part[128 + row];
       const float nk = sqrtf(n2);
       const bool zero = !(n2 > 0.f);
       const float s128 = zero ? 0.f : 128.f / nk;
       HalfBook hb = book;
       if (zero) {
+        hb.C0 = 0.f;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) hb.C[c] = 0.f;
+        for (int c = 0; c < 3; ++c) hb.dC[c] = 0.f;
       }
-      // packed row staged in shared memory: chunk q at 16 q (BMSE + 1) / 4 ... as 32-bit words
-      uint32_t* srow = reinterpret_cast<uint32_t*>(sbase + kOffStage + grp * kStageBytes) + row * kStageWords;
       float rr = 0.f;
 #pragma unroll 1
-      for (int q = 0; q < 4; ++q) {
+      for (int qq = 0; qq < 2; ++qq) {
+        const int q = q0 + qq;
         float y[32];
         tmem_ld32(d1 + 32u * q, y);
         uint32_t hw[2 * BMSE];
 #pragma unroll
         for (int h = 0; h < 2 * BMSE; ++h) hw[h] = 0;
-        uint32_t rh[16], rl[16];
 #pragma unroll
-        for (int jj = 0; jj < 32; jj += 2) {
-          float r0, r1;
-          const uint32_t c0 = cell<BMSE>(y[jj] * s128, hb, r0);
-          const uint32_t c1 = cell<BMSE>(y[jj + 1] * s128, hb, r1);
-          rr = fmaf(r0, r0, rr);
-          rr = fmaf(r1, r1, rr);
-          const __half2 hi = __floats2half2_rn(r0, r1);
-          const float2 hf = __half22float2(hi);
-          const __half2 lo = __floats2half2_rn(r0 - hf.x, r1 - hf.y);
-          rh[jj >> 1] = *reinterpret_cast<const uint32_t*>(&hi);
-          rl[jj >> 1] = *reinterpret_cast<const uint32_t*>(&lo);
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t rh[8], rl[8];
 #pragma unroll
-          for (int t2 = 0; t2 < 2; ++t2) {
-            const int j = jj + t2;
-            const uint32_t code = t2 ? c1 : c0;
-            const int rreg = j >> 2, e = j & 3, uu = rreg >> 2, ii = rreg & 3;
-            if constexpr (BMSE == 3) {
-              if (ii < 3) {
-                hw[uu * 3 + ii] |= code << (4 * e);
+          for (int jp = 0; jp < 16; jp += 2) {
+            const int jj = 16 * hh + jp;
+            float r0, r1;
+            const uint32_t b0 = cell_bits<BMSE>(y[jj] * s128, hb, r0);
+            const uint32_t b1 = cell_bits<BMSE>(y[jj + 1] * s128, hb, r1);
+            rr = fmaf(r0, r0, rr);
+            rr = fmaf(r1, r1, rr);
+            const __half2 hi = __floats2half2_rn(r0, r1);
+            const float2 hf = __half22float2(hi);
+            const __half2 lo = __floats2half2_rn(r0 - hf.x, r1 - hf.y);
+            rh[jp >> 1] = *reinterpret_cast<const uint32_t*>(&hi);
+            rl[jp >> 1] = *reinterpret_cast<const uint32_t*>(&lo);
+#pragma unroll
+            for (int t2 = 0; t2 < 2; ++t2) {
+              // bits = float pattern of 2^23 + idx: idx in bits 0..2, the constant
+              // part only reaches bits >= 24 of each shifted term
+              const int j = jj + t2;
+              const uint32_t bits = t2 ? b1 : b0;
+              const int rreg = j >> 2, e = j & 3, uu = rreg >> 2, ii = rreg & 3;
+              if constexpr (BMSE == 3) {
+                if (ii < 3) {
+                  hw[uu * 3 + ii] += bits << (4 * e);
+                } else {
+#pragma unroll
+                  for (int b = 0; b < 3; ++b) hw[uu * 3 + b] |= ((bits >> b) & 1u) << (4 * e + 3);
+                }
+              } else if constexpr (BMSE == 2) {
+                hw[uu * 2 + (ii >> 1)] += bits << (4 * e + 2 * (ii & 1));
               } else {
-#pragma unroll
-                for (int b = 0; b < 3; ++b) hw[uu * 3 + b] |= ((code >> b) & 1u) << (4 * e + 3);
+                hw[uu] += bits << (4 * e + ii);
               }
-            } else if constexpr (BMSE == 2) {
-              hw[uu * 2 + (ii >> 1)] |= code << (4 * e + 2 * (ii & 1));
-            } else {
-              hw[uu] |= code << (4 * e + ii);
             }
           }
+          // the residual overwrites the columns of y just read (A operand of the JL product):
+          // coordinates 32q + 16hh .. +15 -> hi pairs at column 32q + 8hh, lo pairs 16 further
+          tmem_st8(d1 + 32u * q + 8u * hh, rh);
+          tmem_st8(d1 + 32u * q + 16u + 8u * hh, rl);
         }
-        // the residual overwrites the 32 columns of y just read (A operand of the JL product)
-        tmem_st16(d1 + 32u * q, rh);
-        tmem_st16(d1 + 32u * q + 16u, rl);
 #pragma unroll
-        for (int w = 0; w < kCodeWords; ++w)
-          srow[q * (BMSE + 1) + w] = zero ? 0u : (hw[2 * w] | (hw[2 * w + 1] << 16));
+        for (int w = 0; w < BMSE; ++w)
+          srow[q * (BMSE + 1) + w] = zero ? 0u : __byte_perm(hw[2 * w], hw[2 * w + 1], 0x5410);
       }
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       tc_fence_before();
-      mbar_arrive(bar(kBarRFull + grp));
-      const float rho = nk * sqrtf(rr) * (1.0f / 128.f);
-      if (!mbar_wait(bar(kBarD2Full + grp), par, abort_flag, status)) break;
+      mbar_arrive(bar(kBarRFull + slot));
+      part[256 + half * 128 + row] = rr;
+      if (!mbar_wait(bar(kBarD2Full + slot), par, abort_flag, status)) break;
       tc_fence_after();
-#pragma unroll 1
-      for (int q = 0; q < 4; ++q) {
-        float z[32];
-        tmem_ld32(d2 + 32u * q, z);
+      float z0[32], z1[32];
+      tmem_ld32_nowait(d2 + 32u * q0, z0);
+      tmem_ld32_nowait(d2 + 32u * (q0 + 1), z1);
+      tmem_wait_ld();
+#pragma unroll
+      for (int qq = 0; qq < 2; ++qq) {
+        const float* z = qq ? z1 : z0;
         uint32_t sw = 0;
 #pragma unroll
         for (int jj = 0; jj < 32; ++jj) {
           const int rreg = jj >> 2, e = jj & 3, uu = rreg >> 2, ii = rreg & 3;
           sw |= (z[jj] >= 0.f ? 1u : 0u) << (16 * uu + 4 * e + ii);
         }
-        srow[q * (BMSE + 1) + BMSE] = sw;
+        srow[(q0 + qq) * (BMSE + 1) + BMSE] = zero ? 0xFFFFFFFFu : sw;
       }
       tc_fence_before();
-      mbar_arrive(bar(kBarFree + grp));
+      mbar_arrive(bar(kBarD2Free + slot));
+      named_barrier(1 + slot, 256);
       const int64_t key = (blockIdx.x + i * gridDim.x) * kTile + row;
       if (key < n) {
-        uint8_t* dst = payload + key * kRowBytes;
+        // each group writes its two quarter chunks; group 0 of the slot writes the norms
+        uint8_t* dst = payload + key * kRowBytes + q0 * 4 * (BMSE + 1);
+        const uint32_t* src = srow + q0 * (BMSE + 1);
         if constexpr (BMSE == 3) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-            reinterpret_cast<uint4*>(dst)[c] = reinterpret_cast<const uint4*>(srow)[c];
+          reinterpret_cast<uint4*>(dst)[0] = reinterpret_cast<const uint4*>(src)[0];
+          reinterpret_cast<uint4*>(dst)[1] = reinterpret_cast<const uint4*>(src)[1];
         } else if constexpr (BMSE == 1) {
-#pragma unroll
-          for (int c = 0; c < 2; ++c)
-            reinterpret_cast<uint4*>(dst)[c] = reinterpret_cast<const uint4*>(srow)[c];
+          reinterpret_cast<uint4*>(dst)[0] = reinterpret_cast<const uint4*>(src)[0];
         } else {
 #pragma unroll
-          for (int c = 0; c < 3; ++c)
-            reinterpret_cast<uint4*>(dst)[c] = reinterpret_cast<const uint4*>(srow)[c];
+          for (int w = 0; w < 6; ++w) reinterpret_cast<uint32_t*>(dst)[w] = src[w];
         }
-        const uint32_t nn = uint32_t(__half_as_ushort(__float2half_rn(nk))) |
-                            (uint32_t(__half_as_ushort(__float2half_rn(rho))) << 16);
-        reinterpret_cast<uint32_t*>(norms)[key] = nn;
+        if (half == 0) {
+          const float rho = nk * sqrtf(part[256 + row] + part[384 + row]) * (1.0f / 128.f);
+          const uint32_t nn = uint32_t(__half_as_ushort(__float2half_rn(nk))) |
+                              (uint32_t(__half_as_ushort(__float2half_rn(rho))) << 16);
+          reinterpret_cast<uint32_t*>(norms)[key] = nn;
+        }
       }
     }
   }
@@ -518,8 +583,9 @@ cudaError_t launch_quantize_tc(const tq_ctx* ctx, const void* keys, int dtype, i
   const int grid = int(tiles < sms ? tiles : sms);
   HalfBook hb{};
   const int L = ctx->levels;
-  for (int i = 0; i < L / 2 - 1; ++i) hb.T[i] = float(128.0 * ctx->t[L / 2 + i]);
-  for (int i = 0; i < L / 2; ++i) hb.C[i] = float(128.0 * ctx->c[L / 2 + i]);
+  for (int i = 0; i < L / 2 - 1; ++i) hb.Tneg[i] = -float(128.0 * ctx->t[L / 2 + i]) * 0x1p100f;
+  hb.C0 = float(128.0 * ctx->c[L / 2]);
+  for (int i = 0; i + 1 < L / 2; ++i) hb.dC[i] = float(128.0 * ctx->c[L / 2 + i + 1]) - float(128.0 * ctx->c[L / 2 + i]);
   switch (ctx->bmse) {
     case 1: {
       auto k = quantize_tc_kernel<1>;
