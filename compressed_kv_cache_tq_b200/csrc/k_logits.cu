@@ -66,6 +66,8 @@ __global__ void __launch_bounds__(128) qprep_kernel(const float* __restrict__ q,
   const int slots = nt_per_group * HPT;
   const int grp = blockIdx.x, b = grp / Hkv, hkv = grp % Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // the logits grid may start streaming the cache now; it waits for this grid before reading fragments
+  asm volatile("griddepcontrol.launch_dependents;");
   // both matrices in flight at once (asynchronous 16-byte copies)
   for (int i = tid; i < D * D / 4; i += 128) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(uint32_t(__cvta_generic_to_shared(matR + 4 * i))),
@@ -258,76 +260,15 @@ __device__ __forceinline__ void sign_operands(const Chunk<BMSE>& c, uint32_t (&a
   }
 }
 
+// One 16-key MMA row tile of a 32-key tile: decode, multiply, combine, store.
 template <int BMSE, int NT>
-__global__ void __launch_bounds__(kLogitThreads) logits_mma_kernel(
-    const uint8_t* __restrict__ payload, const uint16_t* __restrict__ norms, int64_t S, int Hq, int Hkv,
-    int64_t total_tiles, const uint32_t* __restrict__ frags, const HeadScale* __restrict__ hscale, CodeLut lut,
-    float* __restrict__ out) {
-  constexpr int kRowBytes = D * BMSE / 8 + D / 8;
-  const int lane = threadIdx.x & 31;
-  const int g = lane >> 2, tig = lane & 3;
-  const int64_t nwarps = int64_t(gridDim.x) * (kLogitThreads / 32);
-  const int64_t gw = int64_t(blockIdx.x) * (kLogitThreads / 32) + (threadIdx.x >> 5);
-  const int64_t t_begin = gw * total_tiles / nwarps, t_end = (gw + 1) * total_tiles / nwarps;
-  if (t_begin >= t_end) return;
-  const int G = Hq / Hkv;
-  const int64_t tpp = (S + 15) / 16;
-
-  // tile t = (group, key offset s0); advanced incrementally, no division per tile
-  int64_t grp = t_begin / tpp;
-  int64_t s0 = (t_begin - grp * tpp) * 16;
-
-  uint32_t bx[NT][KS][2], by[NT][KS][2];
-  float sc_code[NT], sc_sign[NT];
-  float* obase[NT];
-  auto load_group = [&](int64_t gi) {
-    const int b = int(gi / Hkv), hkv = int(gi - int64_t(b) * Hkv);
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const uint32_t* fr = frags + (size_t(gi) * NT + nt) * kFragWords;
-#pragma unroll
-      for (int s = 0; s < KS; ++s)
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          bx[nt][s][r] = __ldg(fr + ((0 * KS + s) * 2 + r) * 32 + lane);
-          by[nt][s][r] = __ldg(fr + ((1 * KS + s) * 2 + r) * 32 + lane);
-        }
-      const int hg = nt * HPT + tig;
-      const int hh = hg < G ? hg : 0;
-      const HeadScale hs = hscale[size_t(b) * Hq + hkv * G + hh];
-      sc_code[nt] = hg < G ? hs.code : 0.f;
-      sc_sign[nt] = hg < G ? hs.sign : 0.f;
-      obase[nt] = out + (size_t(b) * Hq + hkv * G + hh) * S;
-    }
-  };
-  load_group(grp);
-
-  auto load_tile = [&](int64_t gi, int64_t so, Chunk<BMSE>& ca, Chunk<BMSE>& cb, uint32_t& na, uint32_t& nb) {
-    const int64_t rowA = gi * S + so + g, rowB = rowA + 8;
-    const bool okA = so + g < S, okB = so + g + 8 < S;
-    load_chunk<BMSE>(ca, payload + rowA * kRowBytes, tig, okA);
-    load_chunk<BMSE>(cb, payload + rowB * kRowBytes, tig, okB);
-    na = okA ? __ldg(reinterpret_cast<const uint32_t*>(norms) + rowA) : 0u;
-    nb = okB ? __ldg(reinterpret_cast<const uint32_t*>(norms) + rowB) : 0u;
-  };
-  Chunk<BMSE> ca, cb;
-  uint32_t na, nb;
-  load_tile(grp, s0, ca, cb, na, nb);
-
-  for (int64_t t = t_begin; t < t_end; ++t) {
-    // next tile coordinates and its loads, issued before this tile's math
-    int64_t ngrp = grp, ns0 = s0 + 16;
-    if (ns0 >= S) {
-      ns0 = 0;
-      ++ngrp;
-    }
-    Chunk<BMSE> nca, ncb;
-    uint32_t nna = 0, nnb = 0;
-    if (t + 1 < t_end) load_tile(ngrp, ns0, nca, ncb, nna, nnb);
-
+__device__ __forceinline__ void row_tile(const Chunk<BMSE>& ca, const Chunk<BMSE>& cb, uint32_t na, uint32_t nb,
+                                         bool okA, bool okB, const uint32_t (&bx)[NT][KS][2],
+                                         const uint32_t (&by)[NT][KS][2], const float (&sc_code)[NT],
+                                         const float (&sc_sign)[NT], float* const (&orow)[NT], int g, const CodeLut& lut) {
+  int acc_hi[NT][4], acc_lo[NT][4], acc_sg[NT][4];
+  {
     uint32_t sa[8], sb[8];
-    int acc_hi[NT][4], acc_lo[NT][4], acc_sg[NT][4];
-
     code_selectors<BMSE>(ca, sa);
     code_selectors<BMSE>(cb, sb);
 #pragma unroll
@@ -349,6 +290,8 @@ __global__ void __launch_bounds__(kLogitThreads) logits_mma_kernel(
         }
       }
     }
+  }
+  {
     // sign registers: selectors keep one bit per nibble; the byte table maps
     // that bit's two possible selector values to -1 and +1
     uint32_t ga[8], gb[8];
@@ -363,35 +306,116 @@ __global__ void __launch_bounds__(kLogitThreads) logits_mma_kernel(
         else
           mma_s8(acc_sg[nt], ga[2 * s], gb[2 * s], ga[2 * s + 1], gb[2 * s + 1], by[nt][s][0], by[nt][s][1]);
       }
+  }
+  // epilogue: C[row][2 tig + limb] -> head tig of each N-tile (scales are 0 for padded heads)
+  const float2 fa = __half22float2(*reinterpret_cast<const __half2*>(&na));   // (||k||, ||r||) of key g
+  const float2 fb = __half22float2(*reinterpret_cast<const __half2*>(&nb));   // of key g + 8
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    // |cross terms| <= 2 * 128 * 128 * 128 and |low terms| < 2^21: the integer sums fit in 32 bits
+    const float codeA = fmaf(float(acc_hi[nt][0]), 65536.f, float((acc_hi[nt][1] + acc_lo[nt][0]) * 256 + acc_lo[nt][1]));
+    const float codeB = fmaf(float(acc_hi[nt][2]), 65536.f, float((acc_hi[nt][3] + acc_lo[nt][2]) * 256 + acc_lo[nt][3]));
+    const float signA = float(acc_sg[nt][0] * 256 + acc_sg[nt][1]);
+    const float signB = float(acc_sg[nt][2] * 256 + acc_sg[nt][3]);
+    if (orow[nt]) {
+      if (okA) orow[nt][g] = fmaf(fa.x * sc_code[nt], codeA, fa.y * sc_sign[nt] * signA);
+      if (okB) orow[nt][g + 8] = fmaf(fb.x * sc_code[nt], codeB, fb.y * sc_sign[nt] * signB);
+    }
+  }
+}
 
-    // epilogue: C[row][2 tig + limb] -> head tig of each N-tile
-    const float kna = __half2float(__ushort_as_half(uint16_t(na)));
-    const float kra = __half2float(__ushort_as_half(uint16_t(na >> 16)));
-    const float knb = __half2float(__ushort_as_half(uint16_t(nb)));
-    const float krb = __half2float(__ushort_as_half(uint16_t(nb >> 16)));
-    const bool okA = s0 + g < S, okB = s0 + g + 8 < S;
+// Each warp streams a contiguous range of 32-key tiles (two MMA row tiles
+// sharing the query fragments of their (batch, KV head) group).
+template <int BMSE, int NT>
+__global__ void __launch_bounds__(kLogitThreads) logits_mma_kernel(
+    const uint8_t* __restrict__ payload, const uint16_t* __restrict__ norms, int64_t S, int Hq, int Hkv,
+    int64_t total_tiles, const uint32_t* __restrict__ frags, const HeadScale* __restrict__ hscale, CodeLut lut,
+    float* __restrict__ out) {
+  constexpr int kRowBytes = D * BMSE / 8 + D / 8;
+  const int lane = threadIdx.x & 31;
+  const int g = lane >> 2, tig = lane & 3;
+  const int64_t nwarps = int64_t(gridDim.x) * (kLogitThreads / 32);
+  const int64_t gw = int64_t(blockIdx.x) * (kLogitThreads / 32) + (threadIdx.x >> 5);
+  const int64_t t_begin = gw * total_tiles / nwarps, t_end = (gw + 1) * total_tiles / nwarps;
+  const int G = Hq / Hkv;
+  const int64_t tpp = (S + 31) / 32;
+
+  // tile t = (group, key offset s0); advanced incrementally, no division per tile
+  int64_t grp = t_begin / tpp;
+  int64_t s0 = (t_begin - grp * tpp) * 32;
+
+  auto load_tile = [&](int64_t gi, int64_t so, Chunk<BMSE> (&c)[4], uint32_t (&nn)[4]) {
+    const int64_t row0 = gi * S + so + g;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const bool ok = so + g + 8 * k < S;
+      load_chunk<BMSE>(c[k], payload + (row0 + 8 * k) * kRowBytes, tig, ok);
+      nn[k] = ok ? __ldg(reinterpret_cast<const uint32_t*>(norms) + row0 + 8 * k) : 0u;
+    }
+  };
+  Chunk<BMSE> cur[4];
+  uint32_t curn[4];
+  if (t_begin < t_end) load_tile(grp, s0, cur, curn);
+
+  // the query fragments are written by the preceding query-preparation grid
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (t_begin >= t_end) return;
+
+  uint32_t bx[NT][KS][2], by[NT][KS][2];
+  float sc_code[NT], sc_sign[NT];
+  float* orow[NT];
+  auto load_group = [&](int64_t gi) {
+    const int b = int(gi / Hkv), hkv = int(gi - int64_t(b) * Hkv);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
+      const uint32_t* fr = frags + (size_t(gi) * NT + nt) * kFragWords;
+#pragma unroll
+      for (int s = 0; s < KS; ++s)
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          bx[nt][s][r] = __ldg(fr + ((0 * KS + s) * 2 + r) * 32 + lane);
+          by[nt][s][r] = __ldg(fr + ((1 * KS + s) * 2 + r) * 32 + lane);
+        }
       const int hg = nt * HPT + tig;
-      // |cross terms| <= 2 * 128 * 128 * 128 and |low terms| < 2^21: the integer sums fit in 32 bits
-      const float codeA = float(acc_hi[nt][0]) * 65536.f + float((acc_hi[nt][1] + acc_lo[nt][0]) * 256 + acc_lo[nt][1]);
-      const float codeB = float(acc_hi[nt][2]) * 65536.f + float((acc_hi[nt][3] + acc_lo[nt][2]) * 256 + acc_lo[nt][3]);
-      const float signA = float(acc_sg[nt][0] * 256 + acc_sg[nt][1]);
-      const float signB = float(acc_sg[nt][2] * 256 + acc_sg[nt][3]);
-      float* o = obase[nt] + s0;
-      if (hg < G) {
-        if (okA) o[g] = kna * codeA * sc_code[nt] + kra * signA * sc_sign[nt];
-        if (okB) o[g + 8] = knb * codeB * sc_code[nt] + krb * signB * sc_sign[nt];
-      }
+      const int hh = hg < G ? hg : 0;
+      const HeadScale hs = hscale[size_t(b) * Hq + hkv * G + hh];
+      sc_code[nt] = hs.code;
+      sc_sign[nt] = hs.sign;
+      orow[nt] = hg < G ? out + (size_t(b) * Hq + hkv * G + hh) * S : nullptr;
     }
+  };
+  load_group(grp);
+
+  for (int64_t t = t_begin; t < t_end; ++t) {
+    // next tile coordinates and its loads, issued before this tile's math
+    int64_t ngrp = grp, ns0 = s0 + 32;
+    if (ns0 >= S) {
+      ns0 = 0;
+      ++ngrp;
+    }
+    Chunk<BMSE> nxt[4];
+    uint32_t nxtn[4] = {0u, 0u, 0u, 0u};
+    if (t + 1 < t_end) load_tile(ngrp, ns0, nxt, nxtn);
+
+    float* orow_t[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) orow_t[nt] = orow[nt] ? orow[nt] + s0 : nullptr;
+    row_tile<BMSE, NT>(cur[0], cur[1], curn[0], curn[1], s0 + g < S, s0 + g + 8 < S, bx, by, sc_code, sc_sign,
+                       orow_t, g, lut);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) orow_t[nt] = orow[nt] ? orow[nt] + s0 + 16 : nullptr;
+    row_tile<BMSE, NT>(cur[2], cur[3], curn[2], curn[3], s0 + g + 16 < S, s0 + g + 24 < S, bx, by, sc_code,
+                       sc_sign, orow_t, g, lut);
+
     if (t + 1 < t_end) {
       if (ngrp != grp) load_group(ngrp);
       grp = ngrp;
       s0 = ns0;
-      ca = nca;
-      cb = ncb;
-      na = nna;
-      nb = nnb;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        cur[k] = nxt[k];
+        curn[k] = nxtn[k];
+      }
     }
   }
 }
@@ -451,15 +475,24 @@ template <int BMSE, int NT>
 cudaError_t launch_mma(const tq_ctx* ctx, int B, int Hq, int Hkv, int64_t S, const uint8_t* payload,
                        const uint16_t* norms, float* out, const uint32_t* frags, const HeadScale* hs,
                        cudaStream_t st) {
-  const int64_t total = int64_t(B) * Hkv * ((S + 15) / 16);
+  const int64_t total = int64_t(B) * Hkv * ((S + 31) / 32);
   auto kern = logits_mma_kernel<BMSE, NT>;
   int per_sm = 1;
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kLogitThreads, 0);
   int64_t grid = int64_t(sm_count()) * (per_sm > 0 ? per_sm : 1);
   const int64_t needed = (total + kLogitThreads / 32 - 1) / (kLogitThreads / 32);
   if (grid > needed) grid = needed;
-  kern<<<int(grid), kLogitThreads, 0, st>>>(payload, norms, S, Hq, Hkv, total, frags, hs, ctx->lut, out);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(grid));
+  cfg.blockDim = dim3(kLogitThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // overlap with the query preparation
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, payload, norms, S, Hq, Hkv, total, frags, hs, ctx->lut, out);
 }
 
 }  // namespace
