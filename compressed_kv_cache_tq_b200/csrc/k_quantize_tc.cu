@@ -6,8 +6,8 @@
 //   n = ||k||                    (from the key tile in shared memory, fp32)
 //   idx_j = #{i : t_i < y_j / n} (Lloyd-Max cell search in registers)
 //   r_rot = y / n - c[idx]       (the residual on the unit sphere, R r / n)
-//   z = P r_rot                  (tcgen05 MMA, fp16 hi/lo split of both
-//                                 operands, three passes, fp32 in TMEM)
+//   z = P r_rot                  (tcgen05 MMA, fp16 hi/lo split of r_rot and
+//                                 the fp16 JL samples P, two passes, fp32 in TMEM)
 //   sign_i = [z_i >= 0]          (= [(S r)_i >= 0] since S r = n P r_rot)
 //   ||r|| = n ||r_rot||; both norms rounded to fp16.
 //
@@ -15,7 +15,7 @@
 // within about 4e-7 of R k / ||k|| (codes differ from exact arithmetic only
 // for coordinates within that distance of a boundary); n is taken from
 // ||y|| = ||R k|| (relative error about 4e-7); the JL product uses an fp16
-// hi + lo split of r_rot (scaled by 2^7) and of P, dropping only lo * lo.
+// hi + lo split of r_rot (scaled by 2^7) against P, which is stored exactly in fp16.
 //
 // Structure (one CTA per SM, persistent over 128-key tiles, two tiles in flight):
 //   warp 0       : TMA producer (the constant B operands once, then key tiles
@@ -25,8 +25,8 @@
 //   warps 2 .. 5 : epilogue of even local tiles (TMEM slot 0)
 //   warps 6 .. 9 : epilogue of odd local tiles (TMEM slot 1)
 //                  one thread per key row (= TMEM lane)
-// Shared memory: B operands R_hi, R_lo, P_hi, P_lo (128 KB) and two key tiles
-// (2 x 32 KB, TMA 128-byte swizzle).
+// Shared memory: B operands R_hi, R_lo, P (96 KB), two key tiles (2 x 32 KB,
+// TMA 128-byte swizzle) and the packed rows of the two slots.
 // TMEM: 512 columns, two slots of 256: y accumulates in columns 0..127 of a
 // slot; the epilogue reads it and writes the residual's fp16 hi / lo pairs
 // back over it (A operand of the JL product, read by the MMA from TMEM); z
@@ -47,9 +47,10 @@ constexpr int kD = 128;
 constexpr int kTile = 128;
 constexpr int kThreadsTc = 576;   // 2 control warps + 16 epilogue warps
 
-constexpr uint32_t kOffRhi = 0, kOffRlo = 32768, kOffPhi = 65536, kOffPlo = 98304;
-constexpr uint32_t kOffKey = 131072;     // two 32 KB key tiles
-constexpr uint32_t kOffStage = 196608;  // packed rows of the two epilogue groups
+constexpr uint32_t kOffRhi = 0, kOffRlo = 32768, kOffP = 65536;
+constexpr uint32_t kConstBytes = 98304;  // R_hi, R_lo (bf16), P (fp16)
+constexpr uint32_t kOffKey = 98304;      // two 32 KB key tiles
+constexpr uint32_t kOffStage = 163840;   // packed rows of the two slots
 constexpr int kStageWords = 20;         // 64-byte row padded to 80 bytes (conflict-free 16-byte accesses)
 constexpr uint32_t kStageBytes = 128u * kStageWords * 4u;
 constexpr uint32_t kOffPart = kOffStage + 2 * kStageBytes;   // row partial sums [slot][n^2 | rr][half][row]
@@ -231,32 +232,35 @@ struct HalfBook {
 
 constexpr float kBig = 0x1p100f;
 
-// Cell index and scaled residual of one rotated coordinate u (already x128),
-// in fused multiply-adds only.  The codebook is symmetric with t_{L/2-1} = 0,
-// so idx = #{i : t_i < u} = L/2 + m for u > 0 and L/2 - 1 - m otherwise, where
-// m = #{boundaries above 0 that are below |u|}.  Each indicator [|u| > T] is
-// sat(2^100 |u| - 2^100 T): exact 0 or 1, because the difference of two
-// floats of this range is either 0 or far above 2^-100 (an exact tie at a
-// boundary resolves within rounding of the boundary).  The returned value
-// is the float bit pattern of 2^23 + idx.
+__device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
+
+// Cell indices and scaled residuals of two rotated coordinates u = y s128
+// (scaled by 128), with packed two-wide fused multiply-adds.  The codebook is
+// symmetric with t_{L/2-1} = 0, so idx = #{i : t_i < u} = L/2 + m for u > 0
+// and L/2 - 1 - m otherwise, where m = #{boundaries above 0 that are below
+// |u|}.  Each indicator [|u| > T] is sat(2^100 |u| - 2^100 T): exactly 0 or 1,
+// because the difference of two floats of this range is either 0 or far
+// above 2^-100 (an exact tie at a boundary resolves within rounding of the
+// boundary).  Returns the float bit patterns of 2^23 + idx.
 template <int BMSE>
-__device__ __forceinline__ uint32_t cell_bits(float u, const HalfBook& hb, float& r) {
-  const float a = fabsf(u);
-  const float sp = __saturatef(u * kBig);            // [u > 0]
-  const float sgn = fmaf(2.f, sp, -1.f);             // +1 for u > 0, else -1
-  float m = 0.f, lv = hb.C0;
+__device__ __forceinline__ uint2 cell2(float2 y, float s128, const HalfBook& hb, float2& r) {
+  const float2 u = __fmul2_rn(y, f2(s128));
+  const float2 sp = make_float2(__saturatef(u.x * kBig), __saturatef(u.y * kBig));   // [u > 0]
+  const float2 sgn = __ffma2_rn(f2(2.f), sp, f2(-1.f));                               // sign(u), 0 -> -1
+  const float2 nsgn = __ffma2_rn(f2(-2.f), sp, f2(1.f));
+  float2 m = make_float2(0.f, 0.f), lv = f2(hb.C0);
 #pragma unroll
   for (int i = 0; i < (1 << (BMSE - 1)) - 1; ++i) {
-    const float step = __saturatef(fmaf(a, kBig, hb.Tneg[i]));
-    m += step;
-    lv = fmaf(step, hb.dC[i], lv);
+    const float2 step = make_float2(__saturatef(fmaf(fabsf(u.x), kBig, hb.Tneg[i])),
+                                    __saturatef(fmaf(fabsf(u.y), kBig, hb.Tneg[i])));
+    m = i == 0 ? step : __fadd2_rn(m, step);
+    lv = __ffma2_rn(step, f2(hb.dC[i]), lv);
   }
-  r = fmaf(-sgn, lv, u);                              // u - sign(u) level
-  // idx = (L/2 - 1/2 + sgn/2) + sgn m, an exact small integer; adding 2^23
-  // puts it in the low mantissa bits
+  r = __ffma2_rn(nsgn, lv, u);                                                        // u - sign(u) level
   constexpr float half_l = float(1 << (BMSE - 1)) - 0.5f;
-  const float base = fmaf(sgn, 0.5f, half_l);
-  return __float_as_uint(fmaf(sgn, m, base) + 8388608.f);
+  const float2 base = __ffma2_rn(sgn, f2(0.5f), f2(half_l));                          // L/2 or L/2 - 1
+  const float2 idx = __fadd2_rn(__ffma2_rn(sgn, m, base), f2(8388608.f));
+  return make_uint2(__float_as_uint(idx.x), __float_as_uint(idx.y));
 }
 
 template <int BMSE>
@@ -306,8 +310,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      mbar_expect_tx(bar(kBarConst), 131072u);
-      for (int c = 0; c < 8; ++c) bulk_load(base + 16384u * c, bimg + 16384 * c, 16384u, bar(kBarConst));
+      mbar_expect_tx(bar(kBarConst), kConstBytes);
+      for (int c = 0; c < int(kConstBytes / 16384u); ++c)
+        bulk_load(base + 16384u * c, bimg + 16384 * c, 16384u, bar(kBarConst));
       int64_t i = 0;
       for (; i < my_tiles; ++i) {
         const int kb = int(i & 1);
@@ -357,14 +362,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
         tc_fence_after();
         const uint32_t d1 = tmem + 256u * sl, d2 = d1 + 128u;
         uint32_t acc = 0;
-        for (int pass = 0; pass < 3; ++pass) {
-          const uint32_t a_lo = pass == 2 ? 16u : 0u;
-          const uint32_t b_off = pass == 1 ? kOffPlo : kOffPhi;
+        for (int pass = 0; pass < 2; ++pass) {          // z = r_hi P^T + r_lo P^T
+          const uint32_t a_lo = pass == 1 ? 16u : 0u;
           for (int k = 0; k < 8; ++k) {
             // residual coordinates 16k .. 16k+15: chunk k/2, half k%2 (8 columns of packed pairs)
             const uint32_t a_tmem = d1 + 32u * uint32_t(k >> 1) + 8u * uint32_t(k & 1) + a_lo;
             const uint32_t off = 16384u * uint32_t(k >> 2) + 32u * uint32_t(k & 3);
-            mma_f16_ts(d2, a_tmem, smem_desc(base + b_off + off), kIdescF16, acc);
+            mma_f16_ts(d2, a_tmem, smem_desc(base + kOffP + off), kIdescF16, acc);
             acc = 1;
           }
         }
@@ -409,10 +413,12 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
         tmem_ld32_nowait(d1 + 32u * q0, y0);
         tmem_ld32_nowait(d1 + 32u * (q0 + 1), y1);
         tmem_wait_ld();
+        float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) n2p = fmaf(y0[j], y0[j], n2p);
+        for (int j = 0; j < 32; j += 2) acc = __ffma2_rn(make_float2(y0[j], y0[j + 1]), make_float2(y0[j], y0[j + 1]), acc);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) n2p = fmaf(y1[j], y1[j], n2p);
+        for (int j = 0; j < 32; j += 2) acc = __ffma2_rn(make_float2(y1[j], y1[j + 1]), make_float2(y1[j], y1[j + 1]), acc);
+        n2p = acc.x + acc.y;
       }
       part[half * 128 + row] = n2p;
       named_barrier(1 + slot, 256);
@@ -426,7 +432,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
 #pragma unroll
         for (int c = 0; c < 3; ++c) hb.dC[c] = 0.f;
       }
-      float rr = 0.f;
+      float2 rr2 = make_float2(0.f, 0.f);
 #pragma unroll 1
       for (int qq = 0; qq < 2; ++qq) {
         const int q = q0 + qq;
@@ -441,14 +447,13 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
 #pragma unroll
           for (int jp = 0; jp < 16; jp += 2) {
             const int jj = 16 * hh + jp;
-            float r0, r1;
-            const uint32_t b0 = cell_bits<BMSE>(y[jj] * s128, hb, r0);
-            const uint32_t b1 = cell_bits<BMSE>(y[jj + 1] * s128, hb, r1);
-            rr = fmaf(r0, r0, rr);
-            rr = fmaf(r1, r1, rr);
-            const __half2 hi = __floats2half2_rn(r0, r1);
+            float2 rp;
+            const uint2 bb = cell2<BMSE>(make_float2(y[jj], y[jj + 1]), s128, hb, rp);
+            const uint32_t b0 = bb.x, b1 = bb.y;
+            rr2 = __ffma2_rn(rp, rp, rr2);
+            const __half2 hi = __float22half2_rn(rp);
             const float2 hf = __half22float2(hi);
-            const __half2 lo = __floats2half2_rn(r0 - hf.x, r1 - hf.y);
+            const __half2 lo = __float22half2_rn(__ffma2_rn(hf, f2(-1.f), rp));
             rh[jp >> 1] = *reinterpret_cast<const uint32_t*>(&hi);
             rl[jp >> 1] = *reinterpret_cast<const uint32_t*>(&lo);
 #pragma unroll
@@ -484,7 +489,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       tc_fence_before();
       mbar_arrive(bar(kBarRFull + slot));
-      part[256 + half * 128 + row] = rr;
+      part[256 + half * 128 + row] = rr2.x + rr2.y;
       if (!mbar_wait(bar(kBarD2Full + slot), par, abort_flag, status)) break;
       tc_fence_after();
       float z0[32], z1[32];

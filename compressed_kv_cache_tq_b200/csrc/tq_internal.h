@@ -45,7 +45,7 @@ struct tq_ctx {
   double* dR64 = nullptr;   // fp64 masters on the device (top-k re-scoring)
   double* dP64 = nullptr;
   double* dc64 = nullptr;
-  uint8_t* dBimg = nullptr; // tensor-core B operands (d = m = 128): R_hi, R_lo (bf16), P_hi, P_lo (fp16), smem image
+  uint8_t* dBimg = nullptr; // tensor-core B operands (d = m = 128): R_hi, R_lo (bf16), P (fp16), smem image
   uint32_t* dstatus = nullptr;
   tq::CodebookParams cb;
   tq::CodeLut lut;

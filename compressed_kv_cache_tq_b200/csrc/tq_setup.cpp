@@ -266,6 +266,8 @@ static void build_tables(int d, int bits, int m, uint64_t seed, uint32_t stream_
   R = orthogonal_factor(G, d);
   P.resize(size_t(m) * d);
   fill_gaussian(seed, stream_base + 1, P.size(), P.data());
+  // the JL Gaussian is stored as fp16 samples (nearest value, one rounding)
+  for (double& v : P) v = double(__half2float(__double2half(v)));
   lloyd_max(d, bits - 1, c, t);
 }
 
@@ -336,26 +338,22 @@ tq_status tq_init_ex(int d, int bits, int m, uint64_t seed, uint32_t stream_base
   if (e == cudaSuccess) e = upload(ctx->P, &ctx->dP64);
   if (e == cudaSuccess) e = upload(ctx->c, &ctx->dc64);
   if (e == cudaSuccess && d == 128 && m == 128) {
-    // R split into bf16 hi + lo (keys are bf16, so K R^T needs two MMAs); P
-    // split into fp16 hi + lo (the residual is split the same way in the
-    // kernel).  B operand rows are output coordinates, K the input ones.
+    // R split into bf16 hi + lo (keys are bf16, so K R^T needs two MMAs); the
+    // stored JL samples P are exact in fp16 (the residual is split into fp16
+    // hi + lo in the kernel).  B operand rows are output coordinates, K the
+    // input ones.
     std::vector<__nv_bfloat16> rh(size_t(d) * d), rl(size_t(d) * d);
-    std::vector<__half> ph(size_t(m) * d), pl(size_t(m) * d);
+    std::vector<__half> ph(size_t(m) * d);
     for (size_t i = 0; i < rh.size(); ++i) {
       const double v = ctx->R[i];
       rh[i] = __float2bfloat16_rn(float(v));
       rl[i] = __float2bfloat16_rn(float(v - double(__bfloat162float(rh[i]))));
     }
-    for (size_t i = 0; i < ph.size(); ++i) {
-      const double v = ctx->P[i];
-      ph[i] = __float2half_rn(float(v));
-      pl[i] = __float2half_rn(float(v - double(__half2float(ph[i]))));
-    }
-    std::vector<uint8_t> img(size_t(4) * 128 * 128 * 2);
+    for (size_t i = 0; i < ph.size(); ++i) ph[i] = __double2half(ctx->P[i]);
+    std::vector<uint8_t> img(size_t(3) * 128 * 128 * 2);
     write_swizzled(rh, 128, 128, img.data());
     write_swizzled(rl, 128, 128, img.data() + 32768);
     write_swizzled(ph, 128, 128, img.data() + 65536);
-    write_swizzled(pl, 128, 128, img.data() + 98304);
     e = upload(img, &ctx->dBimg);
   }
   if (e == cudaSuccess) e = cudaMalloc(&ctx->dstatus, sizeof(uint32_t));

@@ -144,17 +144,20 @@ class Tables:
 def make_tables(d: int, bits: int, seed: int, m: int | None = None, stream_base: int = 0) -> Tables:
     """R, S and the codebook from (d, bits, seed), as tq_init builds them.
 
-    Reading (pages silent on layout): G is d x d, row-major, from stream
-    ``stream_base``; P is m x d, row-major, from stream ``stream_base + 1``.
-    The JL matrix applied to the residual is S = P R.  Because R is Haar and
-    independent of P, S has i.i.d. N(0, 1) entries, i.e. it is the pages'
-    "seeded Gaussian" matrix; writing it as P R only fixes which Gaussian.
+    Reading (pages silent on layout and precision): G is d x d, row-major,
+    from stream ``stream_base``; P is m x d, row-major, from stream
+    ``stream_base + 1``, each Gaussian sample stored as the nearest fp16
+    value (the JL matrix as stored).  The JL matrix applied to the residual is
+    S = P R.  Because R is Haar and independent of P, each row of S points in
+    a uniformly random direction; the estimator's constant sqrt(pi/2) is then
+    exact up to E||p_i|| of the stored rows, which differs from the Gaussian
+    value by O(2^-22) relative (pinned by a Monte-Carlo test).
     """
     m = d if m is None else m
     if bits < 2:
         raise ValueError("bits >= 2 (one Lloyd-Max bit plus the QJL bit)")
     G = gaussian_stream(seed, stream_base, d * d).reshape(d, d)
-    P = gaussian_stream(seed, stream_base + 1, m * d).reshape(m, d)
+    P = gaussian_stream(seed, stream_base + 1, m * d).reshape(m, d).astype(np.float16).astype(np.float64)
     R = haar_rotation(G)
     S = P @ R
     c, t = lloyd_max_codebook(d, bits - 1)

@@ -322,7 +322,8 @@ def test_qjl_term_unbiased_over_1e5_seeds_d128():
     qv = rng.standard_normal(d)
     total = 0.0
     for b in range(nseed // per):
-        P = rng.standard_normal((m * per, d))
+        # the JL samples are stored as fp16 values (the method's matrix as stored)
+        P = rng.standard_normal((m * per, d)).astype(np.float16).astype(np.float64)
         tb = O.Tables(d=d, bits=3, m=m * per, R=base.R, P=P, S=P @ base.R, c=base.c, t=base.t)
         qz = O.quantize(k[None], tb)
         # the QJL term of the estimator alone: feed codes whose levels are zero
@@ -335,6 +336,14 @@ def test_qjl_term_unbiased_over_1e5_seeds_d128():
     var = rho ** 2 / m * ((math.pi / 2) * qv @ qv - (r @ qv / rho) ** 2)
     se = math.sqrt(var / nseed)
     assert abs(mean - r @ qv) < 3 * se
+
+
+def test_jl_samples_are_stored_fp16_gaussians():
+    tb = O.make_tables(128, 3, seed=12)
+    raw = O.gaussian_stream(12, 1, 128 * 128).reshape(128, 128)
+    np.testing.assert_array_equal(tb.P, raw.astype(np.float16).astype(np.float64))
+    assert np.max(np.abs(tb.P - raw) / np.maximum(np.abs(raw), 1e-30)) <= 2.0 ** -11
+    np.testing.assert_allclose(tb.S, tb.P @ tb.R, atol=1e-12)
 
 
 def test_full_estimator_unbiased_with_r_and_s_redrawn():
