@@ -33,8 +33,7 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-METRIC = json.load(open(os.path.join(ROOT, "BASELINE.json")))["metric"] if os.path.exists(
-    os.path.join(ROOT, "BASELINE.json")) else "tq_logits keys scored/s"
+METRIC = "tq_logits keys scored/s & HBM GB/s (% of 8 TB/s); tq_quantize vectors/s"
 
 B, HKV, HQ, D, S, BITS = 8, 8, 32, 128, 32768, 4
 SEED_KEYS, SEED_TABLES = 1001, 42
@@ -169,6 +168,64 @@ def run_reference(args, rank):
     return 0
 
 
+def max_over_ranks(x: float, dist, device) -> float:
+    """The largest value of x over all ranks (x itself without a process group)."""
+    if dist is None:
+        return float(x)
+    import torch
+
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def result_line(*, world, n, steps, warmup, ms, q_ms, l_ms, e2e_ms, h2d, d2h, clocks) -> dict:
+    """The JSON result: whole-job rates over all ranks (each rank processes n keys
+    per step; ms and e2e_ms are the slowest rank's), the per-kernel breakdown and
+    the roofline of the dominant kernel."""
+    ms_step = ms / steps
+    hbm, tf, tf_sus, src = peaks()
+    bpk = bytes_per_key()
+    q_bytes = n * (bpk["quantize_in"] + bpk["quantize_out"])
+    l_bytes = n * (bpk["logits_in"] + bpk["logits_out"])
+    kernels = {
+        "tq_quantize": {"ms": q_ms, "bytes": q_bytes, "GB/s": q_bytes / q_ms / 1e6,
+                        "vectors_per_s": n / q_ms * 1e3,
+                        "flops": n * (2 * D * D + 2 * D * D), "TFLOP/s": n * 4 * D * D / q_ms / 1e9},
+        "tq_logits": {"ms": l_ms, "bytes": l_bytes, "GB/s": l_bytes / l_ms / 1e6, "keys_per_s": n / l_ms * 1e3,
+                      "pct_of_8TBs": 100 * l_bytes / l_ms / 1e6 / 8000.0},
+    }
+    dom = "tq_quantize" if q_ms >= l_ms else "tq_logits"
+    ach = kernels[dom]["GB/s"]
+    return {
+        "metric": METRIC,
+        "value": world * n / ms_step * 1e3,
+        "unit": "keys/s",
+        "n_gpus": world,
+        "steps": steps,
+        "warmup": warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "global_batch": B * world, "seq_len": S, "kv_heads": HKV,
+                   "q_heads": HQ, "head_dim": D, "bits": BITS, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2: keys 537 MB, packed cache 143 MB; logits read the cache "
+                         "written one step earlier"},
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": hbm, "unit": "GB/s",
+                     "frac": ach / hbm, "peak_source": src, "traffic": None},
+        "kernels": kernels,
+        "logits_keys_per_s": world * n / l_ms * 1e3,
+        "quantize_vectors_per_s": world * n / q_ms * 1e3,
+        "e2e": {"value": world * n / e2e_ms * 1e3, "unit": "keys/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": 3 * steps,
+        "clocks": clocks,
+    }
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -250,13 +307,8 @@ def main():
             step(i, True)
         t_end.record(stream)
         barrier()
-    ms = t_start.elapsed_time(t_end)
-    if dist is not None:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(t_start.elapsed_time(t_end), dist, dev)
     assert tq.tq_check_device_status(ctx) == 0, "a kernel reported a device-side error"
-    ms_step = ms / args.steps
     q_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / len(ev)
     l_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / len(ev)
 
@@ -286,58 +338,16 @@ def main():
         e2e_step(i)
     b_.record(stream)
     barrier()
-    e2e_ms = a.elapsed_time(b_) / e2e_steps
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(a.elapsed_time(b_) / e2e_steps, dist, dev)
 
     if dist is not None:
         dist.destroy_process_group()
     if rank != 0:
         return 0
 
-    hbm, tf, tf_sus, src = peaks()
-    bpk = bytes_per_key()
-    q_bytes = n * (bpk["quantize_in"] + bpk["quantize_out"])
-    l_bytes = n * (bpk["logits_in"] + bpk["logits_out"])
-    kernels = {
-        "tq_quantize": {"ms": q_ms, "bytes": q_bytes, "GB/s": q_bytes / q_ms / 1e6,
-                        "vectors_per_s": n / q_ms * 1e3,
-                        "flops": n * (2 * D * D + 2 * D * D), "TFLOP/s": n * 4 * D * D / q_ms / 1e9},
-        "tq_logits": {"ms": l_ms, "bytes": l_bytes, "GB/s": l_bytes / l_ms / 1e6, "keys_per_s": n / l_ms * 1e3,
-                      "pct_of_8TBs": 100 * l_bytes / l_ms / 1e6 / 8000.0},
-    }
-    dom = "tq_quantize" if q_ms >= l_ms else "tq_logits"
-    ach = kernels[dom]["GB/s"]
-    line = {
-        "metric": METRIC,
-        "value": world * n / ms_step * 1e3,
-        "unit": "keys/s",
-        "n_gpus": world,
-        "steps": args.steps,
-        "warmup": args.warmup,
-        "ms_per_step": ms_step,
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
-        "dtype": "bf16",
-        "data": "synthetic",
-        "config": {"workload": WORKLOAD, "global_batch": B * world, "seq_len": S, "kv_heads": HKV,
-                   "q_heads": HQ, "head_dim": D, "bits": BITS, "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2: keys 537 MB, packed cache 143 MB; logits read the cache "
-                         "written one step earlier"},
-        "roofline": {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": hbm, "unit": "GB/s",
-                     "frac": ach / hbm, "peak_source": src, "traffic": None},
-        "kernels": kernels,
-        "logits_keys_per_s": world * n / l_ms * 1e3,
-        "quantize_vectors_per_s": world * n / q_ms * 1e3,
-        "e2e": {"value": world * n / e2e_ms * 1e3, "unit": "keys/s",
-                "h2d_bytes_per_step": int(keys.numel() * 2 + q.numel() * 4),
-                "d2h_bytes_per_step": int(out.numel() * 4)},
-        "gpu_launches": 3 * args.steps,
-        "clocks": clocks.summary(),
-    }
+    line = result_line(world=world, n=n, steps=args.steps, warmup=args.warmup, ms=ms, q_ms=q_ms, l_ms=l_ms,
+                       e2e_ms=e2e_ms, h2d=int(keys.numel() * 2 + q.numel() * 4), d2h=int(out.numel() * 4),
+                       clocks=clocks.summary())
     if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline()
     print(json.dumps(line), flush=True)

@@ -14,25 +14,29 @@
 // Precision: R = R_hi + R_lo in bf16 represents R to about 2^-17, so y / n is
 // within about 4e-7 of R k / ||k|| (codes differ from exact arithmetic only
 // for coordinates within that distance of a boundary); n is taken from
-// ||y|| = ||R k|| (relative error about 4e-7); the JL product uses an fp16
-// hi + lo split of r_rot (scaled by 2^7) against P, which is stored exactly in fp16.
+// ||y|| = ||R k|| (relative error about 4e-7); the JL product uses an fp16 hi +
+// lo split of r_rot (scaled by 2^7) against P, which is stored exactly in fp16.
 //
 // Structure (one CTA per SM, persistent over 128-key tiles, two tiles in flight):
-//   warp 0       : TMA producer (the constant B operands once, then key tiles
-//                  into a two-deep ring)
-//   warp 1       : TMEM allocation and the single-thread MMA issue, in the
-//                  order MMA1(0), MMA1(1), MMA2(0), MMA1(2), MMA2(1), ...
-//   warps 2 .. 5 : epilogue of even local tiles (TMEM slot 0)
-//   warps 6 .. 9 : epilogue of odd local tiles (TMEM slot 1)
-//                  one thread per key row (= TMEM lane)
-// Shared memory: B operands R_hi, R_lo, P (96 KB), two key tiles (2 x 32 KB,
-// TMA 128-byte swizzle) and the packed rows of the two slots.
+//   warp 0        : TMA producer (the constant B operands once, then key tiles
+//                   into a three-deep ring)
+//   warp 1        : TMEM allocation and the single-thread MMA issue, in the
+//                   order MMA1(0), MMA1(1), MMA2(0), MMA1(2), MMA2(1), ...
+//   warps 2 .. 17 : epilogue, two teams of eight warps; the team of TMEM slot s
+//                   handles the local tiles of parity s, one thread per key row
+//                   (= TMEM lane) and half of its coordinates (two quarters).
+//                   While one team waits for the tensor cores (the JL product
+//                   of its tile, then the rotation of its next one), the other
+//                   team's cell search keeps the FMA pipes busy.
+// Shared memory: B operands R_hi, R_lo, P (96 KB), three key tiles (3 x 32 KB,
+// TMA 128-byte swizzle) and the two halves' per-row partial sums.
 // TMEM: 512 columns, two slots of 256: y accumulates in columns 0..127 of a
 // slot; the epilogue reads it and writes the residual's fp16 hi / lo pairs
 // back over it (A operand of the JL product, read by the MMA from TMEM); z
 // accumulates in columns 128..255.
 // Every wait on an mbarrier is bounded; a wait that gives up sets the
-// context's status word, and all roles then leave their loops.
+// context's status word, and all roles then leave their loops (there is no
+// unbounded barrier between roles).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -46,28 +50,32 @@ namespace {
 constexpr int kD = 128;
 constexpr int kTile = 128;
 constexpr int kThreadsTc = 576;   // 2 control warps + 16 epilogue warps
+constexpr int kTeamThreads = 256;  // epilogue threads per TMEM slot
 
 constexpr uint32_t kOffRhi = 0, kOffRlo = 32768, kOffP = 65536;
 constexpr uint32_t kConstBytes = 98304;  // R_hi, R_lo (bf16), P (fp16)
-constexpr uint32_t kOffKey = 98304;      // two 32 KB key tiles
-constexpr uint32_t kOffStage = 163840;   // packed rows of the two slots
-constexpr int kStageWords = 20;         // 64-byte row padded to 80 bytes (conflict-free 16-byte accesses)
-constexpr uint32_t kStageBytes = 128u * kStageWords * 4u;
-constexpr uint32_t kOffPart = kOffStage + 2 * kStageBytes;   // row partial sums [slot][n^2 | rr][half][row]
-constexpr uint32_t kOffBar = kOffPart + 2 * 512 * 4;
+constexpr int kKeyStages = 3;            // key-tile ring depth (covers HBM latency under load)
+constexpr uint32_t kOffKey = 98304;      // kKeyStages 32 KB key tiles
+constexpr uint32_t kOffPn2 = kOffKey + 32768u * kKeyStages;   // [slot][parity][half][row] partial ||y||^2
+constexpr uint32_t kOffPrr = kOffPn2 + 2u * 2u * 2u * 128u * 4u;  // [slot][half][row] partial ||r_rot||^2
+constexpr uint32_t kOffBar = kOffPrr + 2u * 2u * 128u * 4u;
 constexpr uint32_t kSmemBytes = kOffBar + 256 + 1024;   // + slack for 1024-byte alignment
+static_assert(kSmemBytes <= 232448, "shared memory per block");
 
 // barriers; the per-slot ones come in pairs (slot 0, slot 1)
 enum Bar {
   kBarConst = 0,
-  kBarKFull = 1,
-  kBarKEmpty = 3,
-  kBarD1Full = 5,
-  kBarRFull = 7,
-  kBarD2Full = 9,
-  kBarD2Free = 11,
-  kNumBars = 13
+  kBarKFull = 1,                        // one per key stage
+  kBarKEmpty = kBarKFull + kKeyStages,
+  kBarD1Full = kBarKEmpty + kKeyStages, // one per TMEM slot from here on
+  kBarN2 = kBarD1Full + 2,              // both halves' partial sums of ||y||^2 written
+  kBarRFull = kBarN2 + 2,               // residual in TMEM
+  kBarRR = kBarRFull + 2,               // both halves' partial sums of ||r_rot||^2 written
+  kBarD2Full = kBarRR + 2,
+  kBarD2Free = kBarD2Full + 2,          // z read
+  kNumBars = kBarD2Free + 2
 };
+static_assert(8 * kNumBars + 8 <= 256, "barrier area");
 
 constexpr long long kWaitCycles = 4000000000LL;   // about 2 s at the boost clock
 
@@ -111,6 +119,25 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     }
   }
   return true;
+}
+// mbar_wait taken by a whole warp: every lane gets the same answer, so that no
+// lane leaves its loop while the others go on into warp-synchronous instructions.
+__device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                               uint32_t* status) {
+  return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, abort_flag, status));
+}
+// Bounded wait that ignores the abort flag: used before the CTA exits, so that
+// no copy or MMA is still in flight when shared and tensor memory are released.
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                           uint32_t* status) {
+  const long long t0 = clock64();
+  while (!mbar_try(bar, parity)) {
+    if (clock64() - t0 > kWaitCycles) {
+      *abort_flag = 1;
+      atomicOr(status, kStatusQuantizeTc);
+      return;
+    }
+  }
 }
 
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
@@ -158,51 +185,39 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
 
-__device__ __forceinline__ void named_barrier(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+// Asynchronous loads of 16 / 32 consecutive TMEM columns of this thread's lane.
+// The registers hold the data only after tmem_wait16 / tmem_wait32 on the same
+// array: the wait takes them as read-write operands, so the compiler cannot
+// move a use above it.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+               : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7]),
+                 "=f"(v[8]), "=f"(v[9]), "=f"(v[10]), "=f"(v[11]), "=f"(v[12]), "=f"(v[13]), "=f"(v[14]), "=f"(v[15])
+               : "r"(taddr));
 }
-
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-
-// 32 consecutive TMEM columns of this thread's lane, without waiting (the
-// registers are valid after tmem_wait_ld()).
-__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-// 32 consecutive TMEM columns of this thread's lane.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+               : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7]),
+                 "=f"(v[8]), "=f"(v[9]), "=f"(v[10]), "=f"(v[11]), "=f"(v[12]), "=f"(v[13]), "=f"(v[14]), "=f"(v[15]),
+                 "=f"(v[16]), "=f"(v[17]), "=f"(v[18]), "=f"(v[19]), "=f"(v[20]), "=f"(v[21]), "=f"(v[22]), "=f"(v[23]),
+                 "=f"(v[24]), "=f"(v[25]), "=f"(v[26]), "=f"(v[27]), "=f"(v[28]), "=f"(v[29]), "=f"(v[30]), "=f"(v[31])
+               : "r"(taddr));
 }
-
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
-      "%14, %15, %16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
-      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-      : "memory");
+__device__ __forceinline__ void tmem_wait16(float (&v)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]), "+f"(v[6]), "+f"(v[7]),
+                 "+f"(v[8]), "+f"(v[9]), "+f"(v[10]), "+f"(v[11]), "+f"(v[12]), "+f"(v[13]), "+f"(v[14]), "+f"(v[15])
+               :
+               : "memory");
+}
+__device__ __forceinline__ void tmem_wait32(float (&v)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+f"(v[0]), "+f"(v[1]), "+f"(v[2]), "+f"(v[3]), "+f"(v[4]), "+f"(v[5]), "+f"(v[6]), "+f"(v[7]),
+                 "+f"(v[8]), "+f"(v[9]), "+f"(v[10]), "+f"(v[11]), "+f"(v[12]), "+f"(v[13]), "+f"(v[14]), "+f"(v[15]),
+                 "+f"(v[16]), "+f"(v[17]), "+f"(v[18]), "+f"(v[19]), "+f"(v[20]), "+f"(v[21]), "+f"(v[22]), "+f"(v[23]),
+                 "+f"(v[24]), "+f"(v[25]), "+f"(v[26]), "+f"(v[27]), "+f"(v[28]), "+f"(v[29]), "+f"(v[30]), "+f"(v[31])
+               :
+               : "memory");
 }
 
 __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
@@ -228,6 +243,12 @@ struct HalfBook {
   float Tneg[3];   // -2^100 x boundaries above 0 (t_{L/2} .. t_{L-2})
   float C0;        // smallest positive level
   float dC[3];     // level steps c_{L/2+i+1} - c_{L/2+i}
+  // two-level search (4 positive levels): first the middle boundary, then the
+  // outer (p2 = 1) or inner (p2 = 0) one; level = B + p_lo A with
+  // A = dC0 + p2 (dC2 - dC0), B = C0 + p2 (C2 - C0)
+  float dT31;      // -2^100 (t_{L-2} - t_{L/2}) : outer minus inner scaled boundary
+  float dA;        // dC2 - dC0
+  float C20;       // C2 - C0
 };
 
 constexpr float kBig = 0x1p100f;
@@ -241,25 +262,38 @@ __device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
 // |u|}.  Each indicator [|u| > T] is sat(2^100 |u| - 2^100 T): exactly 0 or 1,
 // because the difference of two floats of this range is either 0 or far
 // above 2^-100 (an exact tie at a boundary resolves within rounding of the
-// boundary).  Returns the float bit patterns of 2^23 + idx.
+// boundary).  Returns the float bit patterns of 2^23 + (L - 1 - idx): the
+// complemented index costs one operation less (L - 1 - idx = L/2 - [u > 0]
+// - sign(u) m), and complementing every b-bit code of a packed word is
+// complementing the word.
 template <int BMSE>
 __device__ __forceinline__ uint2 cell2(float2 y, float s128, const HalfBook& hb, float2& r) {
   const float2 u = __fmul2_rn(y, f2(s128));
   const float2 sp = make_float2(__saturatef(u.x * kBig), __saturatef(u.y * kBig));   // [u > 0]
-  const float2 sgn = __ffma2_rn(f2(2.f), sp, f2(-1.f));                               // sign(u), 0 -> -1
-  const float2 nsgn = __ffma2_rn(f2(-2.f), sp, f2(1.f));
-  float2 m = make_float2(0.f, 0.f), lv = f2(hb.C0);
-#pragma unroll
-  for (int i = 0; i < (1 << (BMSE - 1)) - 1; ++i) {
-    const float2 step = make_float2(__saturatef(fmaf(fabsf(u.x), kBig, hb.Tneg[i])),
-                                    __saturatef(fmaf(fabsf(u.y), kBig, hb.Tneg[i])));
-    m = i == 0 ? step : __fadd2_rn(m, step);
-    lv = __ffma2_rn(step, f2(hb.dC[i]), lv);
+  const float2 nsgn = __ffma2_rn(f2(-2.f), sp, f2(1.f));                              // -sign(u), 0 -> +1
+  float2 m, lv;
+  if constexpr (BMSE == 3) {
+    const float2 p2 = make_float2(__saturatef(fmaf(fabsf(u.x), kBig, hb.Tneg[1])),
+                                  __saturatef(fmaf(fabsf(u.y), kBig, hb.Tneg[1])));
+    const float2 tsel = __ffma2_rn(p2, f2(hb.dT31), f2(hb.Tneg[0]));   // -2^100 t_outer or t_inner
+    const float2 plo = make_float2(__saturatef(fmaf(fabsf(u.x), kBig, tsel.x)),
+                                   __saturatef(fmaf(fabsf(u.y), kBig, tsel.y)));
+    m = __ffma2_rn(p2, f2(2.f), plo);
+    const float2 A = __ffma2_rn(p2, f2(hb.dA), f2(hb.dC[0]));
+    const float2 B = __ffma2_rn(p2, f2(hb.C20), f2(hb.C0));
+    lv = __ffma2_rn(plo, A, B);
+  } else if constexpr (BMSE == 2) {
+    m = make_float2(__saturatef(fmaf(fabsf(u.x), kBig, hb.Tneg[0])),
+                    __saturatef(fmaf(fabsf(u.y), kBig, hb.Tneg[0])));
+    lv = __ffma2_rn(m, f2(hb.dC[0]), f2(hb.C0));
+  } else {
+    m = make_float2(0.f, 0.f);
+    lv = f2(hb.C0);
   }
   r = __ffma2_rn(nsgn, lv, u);                                                        // u - sign(u) level
-  constexpr float half_l = float(1 << (BMSE - 1)) - 0.5f;
-  const float2 base = __ffma2_rn(sgn, f2(0.5f), f2(half_l));                          // L/2 or L/2 - 1
-  const float2 idx = __fadd2_rn(__ffma2_rn(sgn, m, base), f2(8388608.f));
+  constexpr float kHalfL = float(1 << (BMSE - 1)) + 8388608.f;                        // 2^23 + L/2
+  const float2 t = __ffma2_rn(sp, f2(-1.f), f2(kHalfL));
+  const float2 idx = __ffma2_rn(nsgn, m, t);
   return make_uint2(__float_as_uint(idx.x), __float_as_uint(idx.y));
 }
 
@@ -278,6 +312,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sbase + kOffBar + 8 * kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + kOffBar + 8 * kNumBars + 4);
   auto bar = [&](int i) { return bar0 + 8u * uint32_t(i); };
+  float* pn2 = reinterpret_cast<float*>(sbase + kOffPn2);
+  float* prr = reinterpret_cast<float*>(sbase + kOffPrr);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t num_tiles = (n + kTile - 1) / kTile;
@@ -285,13 +321,17 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
 
   if (threadIdx.x == 0) {
     mbar_init(bar(kBarConst), 1);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kKeyStages; ++s) {
       mbar_init(bar(kBarKFull + s), 1);
       mbar_init(bar(kBarKEmpty + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       mbar_init(bar(kBarD1Full + s), 1);
-      mbar_init(bar(kBarRFull + s), 256);
+      mbar_init(bar(kBarN2 + s), kTeamThreads);
+      mbar_init(bar(kBarRFull + s), kTeamThreads);
+      mbar_init(bar(kBarRR + s), kTeamThreads);
       mbar_init(bar(kBarD2Full + s), 1);
-      mbar_init(bar(kBarD2Free + s), 256);
+      mbar_init(bar(kBarD2Free + s), kTeamThreads);
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -306,123 +346,135 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      mbar_expect_tx(bar(kBarConst), kConstBytes);
-      for (int c = 0; c < int(kConstBytes / 16384u); ++c)
-        bulk_load(base + 16384u * c, bimg + 16384 * c, 16384u, bar(kBarConst));
-      int64_t i = 0;
-      for (; i < my_tiles; ++i) {
-        const int kb = int(i & 1);
-        if (i >= 2 && !mbar_wait(bar(kBarKEmpty + kb), uint32_t(((i >> 1) - 1) & 1), abort_flag, status)) break;
-        const int64_t tile = blockIdx.x + i * gridDim.x;
-        const uint32_t dst = base + kOffKey + 32768u * kb;
-        mbar_expect_tx(bar(kBarKFull + kb), 32768u);
-        tma_load_2d(dst, &key_map, 0, int(tile * kTile), bar(kBarKFull + kb));
-        tma_load_2d(dst + 16384u, &key_map, 64, int(tile * kTile), bar(kBarKFull + kb));
+  if (warp < 2) {
+    if (warp == 0) {
+      // ------------------------------------------------------------ TMA producer
+      if (lane == 0) {
+        mbar_expect_tx(bar(kBarConst), kConstBytes);
+        for (int c = 0; c < int(kConstBytes / 16384u); ++c)
+          bulk_load(base + 16384u * c, bimg + 16384 * c, 16384u, bar(kBarConst));
+        int64_t i = 0;
+        for (; i < my_tiles; ++i) {
+          const int kb = int(i % kKeyStages);
+          if (i >= kKeyStages &&
+              !mbar_wait(bar(kBarKEmpty + kb), uint32_t((i / kKeyStages - 1) & 1), abort_flag, status))
+            break;
+          const int64_t tile = blockIdx.x + i * gridDim.x;
+          const uint32_t dst = base + kOffKey + 32768u * kb;
+          mbar_expect_tx(bar(kBarKFull + kb), 32768u);
+          tma_load_2d(dst, &key_map, 0, int(tile * kTile), bar(kBarKFull + kb));
+          tma_load_2d(dst + 16384u, &key_map, 64, int(tile * kTile), bar(kBarKFull + kb));
+        }
+        // leave no copy in flight: wait for the last loads issued to each buffer
+        for (int64_t j = (i >= kKeyStages ? i - kKeyStages : 0); j < i; ++j)
+          mbar_drain(bar(kBarKFull + int(j % kKeyStages)), uint32_t((j / kKeyStages) & 1), abort_flag, status);
+        mbar_drain(bar(kBarConst), 0u, abort_flag, status);
       }
-      // leave no copy in flight: wait for the last loads issued to each buffer
-      for (int64_t j = (i >= 2 ? i - 2 : 0); j < i; ++j)
-        mbar_wait(bar(kBarKFull + int(j & 1)), uint32_t((j >> 1) & 1), abort_flag, status);
-      mbar_wait(bar(kBarConst), 0u, abort_flag, status);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issue
-    if (lane == 0) {
-      auto issue_mma1 = [&](int64_t i) -> bool {
-        const int sl = int(i & 1);
-        if (!mbar_wait(bar(kBarKFull + sl), uint32_t((i >> 1) & 1), abort_flag, status)) return false;
-        // the slot's y / residual columns are free once the JL MMA of tile i - 2 completed
-        if (i >= 2 && !mbar_wait(bar(kBarD2Full + sl), uint32_t(((i >> 1) - 1) & 1), abort_flag, status))
-          return false;
-        tc_fence_after();
-        const uint32_t d1 = tmem + 256u * sl;
-        const uint32_t kbase = base + kOffKey + 32768u * sl;
-        uint32_t acc = 0;
-        for (int pass = 0; pass < 2; ++pass)
-          for (int kb = 0; kb < 2; ++kb)
-            for (int ks = 0; ks < 4; ++ks) {
-              const uint32_t off = 16384u * kb + 32u * ks;
-              mma_f16(d1, smem_desc(kbase + off), smem_desc(base + (pass ? kOffRlo : kOffRhi) + off), kIdescBf16,
-                      acc);
+    } else if (warp == 1) {
+      // ------------------------------------------------------------ MMA issue
+      if (lane == 0) {
+        auto issue_mma1 = [&](int64_t i) -> bool {
+          const int sl = int(i & 1);
+          const int kb = int(i % kKeyStages);
+          if (!mbar_wait(bar(kBarKFull + kb), uint32_t((i / kKeyStages) & 1), abort_flag, status)) return false;
+          // the slot's y / residual columns are free once the JL MMA of tile i - 2 completed
+          if (i >= 2 && !mbar_wait(bar(kBarD2Full + sl), uint32_t(((i >> 1) - 1) & 1), abort_flag, status))
+            return false;
+          tc_fence_after();
+          const uint32_t d1 = tmem + 256u * sl;
+          const uint32_t kbase = base + kOffKey + 32768u * kb;
+          uint32_t acc = 0;
+          for (int pass = 0; pass < 2; ++pass)
+            for (int kh = 0; kh < 2; ++kh)
+              for (int ks = 0; ks < 4; ++ks) {
+                const uint32_t off = 16384u * kh + 32u * ks;
+                mma_f16(d1, smem_desc(kbase + off), smem_desc(base + (pass ? kOffRlo : kOffRhi) + off), kIdescBf16,
+                        acc);
+                acc = 1;
+              }
+          mma_commit(bar(kBarD1Full + sl));
+          mma_commit(bar(kBarKEmpty + kb));
+          return true;
+        };
+        auto issue_mma2 = [&](int64_t i) -> bool {
+          const int sl = int(i & 1);
+          if (!mbar_wait(bar(kBarRFull + sl), uint32_t((i >> 1) & 1), abort_flag, status)) return false;
+          // the slot's z columns are free once the epilogue of tile i - 2 read them
+          if (i >= 2 && !mbar_wait(bar(kBarD2Free + sl), uint32_t(((i >> 1) - 1) & 1), abort_flag, status))
+            return false;
+          tc_fence_after();
+          const uint32_t d1 = tmem + 256u * sl, d2 = d1 + 128u;
+          uint32_t acc = 0;
+          for (int pass = 0; pass < 2; ++pass) {          // z = r_hi P^T + r_lo P^T
+            const uint32_t a_lo = pass == 1 ? 16u : 0u;
+            for (int k = 0; k < 8; ++k) {
+              // residual coordinates 16k .. 16k+15: chunk k/2, half k%2 (8 columns of packed pairs)
+              const uint32_t a_tmem = d1 + 32u * uint32_t(k >> 1) + 8u * uint32_t(k & 1) + a_lo;
+              const uint32_t off = 16384u * uint32_t(k >> 2) + 32u * uint32_t(k & 3);
+              mma_f16_ts(d2, a_tmem, smem_desc(base + kOffP + off), kIdescF16, acc);
               acc = 1;
             }
-        mma_commit(bar(kBarD1Full + sl));
-        mma_commit(bar(kBarKEmpty + sl));
-        return true;
-      };
-      auto issue_mma2 = [&](int64_t i) -> bool {
-        const int sl = int(i & 1);
-        if (!mbar_wait(bar(kBarRFull + sl), uint32_t((i >> 1) & 1), abort_flag, status)) return false;
-        // the slot's z columns are free once the epilogue of tile i - 2 read them
-        if (i >= 2 && !mbar_wait(bar(kBarD2Free + sl), uint32_t(((i >> 1) - 1) & 1), abort_flag, status))
-          return false;
-        tc_fence_after();
-        const uint32_t d1 = tmem + 256u * sl, d2 = d1 + 128u;
-        uint32_t acc = 0;
-        for (int pass = 0; pass < 2; ++pass) {          // z = r_hi P^T + r_lo P^T
-          const uint32_t a_lo = pass == 1 ? 16u : 0u;
-          for (int k = 0; k < 8; ++k) {
-            // residual coordinates 16k .. 16k+15: chunk k/2, half k%2 (8 columns of packed pairs)
-            const uint32_t a_tmem = d1 + 32u * uint32_t(k >> 1) + 8u * uint32_t(k & 1) + a_lo;
-            const uint32_t off = 16384u * uint32_t(k >> 2) + 32u * uint32_t(k & 3);
-            mma_f16_ts(d2, a_tmem, smem_desc(base + kOffP + off), kIdescF16, acc);
-            acc = 1;
           }
+          mma_commit(bar(kBarD2Full + sl));
+          return true;
+        };
+        int64_t n1 = 0, n2 = 0;   // rotation / JL MMA groups issued
+        bool ok = mbar_wait(bar(kBarConst), 0u, abort_flag, status);
+        if (ok && my_tiles > 0) {
+          ok = issue_mma1(0);
+          n1 += ok;
         }
-        mma_commit(bar(kBarD2Full + sl));
-        return true;
-      };
-      bool ok = mbar_wait(bar(kBarConst), 0u, abort_flag, status);
-      if (ok && my_tiles > 0) ok = issue_mma1(0);
-      int64_t i = 0;
-      for (; ok && i < my_tiles; ++i) {
-        if (i + 1 < my_tiles && !issue_mma1(i + 1)) break;
-        if (!issue_mma2(i)) break;
+        for (int64_t i = 0; ok && i < my_tiles; ++i) {
+          if (i + 1 < my_tiles) {
+            if (!issue_mma1(i + 1)) break;
+            ++n1;
+          }
+          if (!issue_mma2(i)) break;
+          ++n2;
+        }
+        // before TMEM is released: the commit of the last group of each kind
+        // tracks every MMA issued before it
+        if (n1 > 0) mbar_drain(bar(kBarD1Full + int((n1 - 1) & 1)), uint32_t(((n1 - 1) >> 1) & 1), abort_flag, status);
+        if (n2 > 0) mbar_drain(bar(kBarD2Full + int((n2 - 1) & 1)), uint32_t(((n2 - 1) >> 1) & 1), abort_flag, status);
       }
-      // wait for the last MMAs before TMEM is released
-      for (int64_t j = (i >= 2 ? i - 2 : 0); j < i; ++j)
-        mbar_wait(bar(kBarD2Full + int(j & 1)), uint32_t((j >> 1) & 1), abort_flag, status);
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    // 16 warps in 4 groups: group eg serves TMEM slot eg & 1 (local tiles of
-    // that parity) and quarters 2 (eg >> 1), 2 (eg >> 1) + 1 of every row; the
-    // two groups of a slot combine their row partial sums through shared
-    // memory around a named barrier (id 1 + slot, 256 threads).
+    // warp w: team (TMEM slot) ((w - 2) >> 2) & 1, half (w - 2) >> 3 (quarters
+    // 2 half and 2 half + 1 of every row), TMEM lanes 32 (w & 3) .. +31.
     const int eg = (warp - 2) >> 2;
     const int slot = eg & 1, half = eg >> 1;
     const int row = (warp & 3) * 32 + lane;          // TMEM lane = key row within the tile
     const uint32_t lane_addr = uint32_t((warp & 3) * 32) << 16;
     const uint32_t d1 = tmem + 256u * slot + lane_addr, d2 = d1 + 128u;
     constexpr int kRowBytes = kD * BMSE / 8 + kD / 8;  // = 16 (BMSE + 1)
-    float* part = reinterpret_cast<float*>(sbase + kOffPart) + slot * 512;   // [n^2 | rr][half][row]
-    uint32_t* srow = reinterpret_cast<uint32_t*>(sbase + kOffStage + slot * kStageBytes) + row * kStageWords;
     const int q0 = 2 * half;
+    float* rrbuf = prr + slot * 256;
     int64_t k = 0;
     for (int64_t i = slot; i < my_tiles; i += 2, ++k) {
       const uint32_t par = uint32_t(k & 1);
-      if (!mbar_wait(bar(kBarD1Full + slot), par, abort_flag, status)) break;
+      if (!mbar_wait_warp(bar(kBarD1Full + slot), par, abort_flag, status)) break;
       tc_fence_after();
-      // ||k||^2 = ||R k||^2 from the rotated row, half a row per group
-      float n2p = 0.f;
+      // ||k||^2 = ||R k||^2 from the rotated row, half a row per half-team; the
+      // partial sums alternate between two buffers, so that a half that runs
+      // ahead never overwrites sums the other half has not read yet
+      float* n2buf = pn2 + (slot * 2 + int(par)) * 256;
       {
-        float y0[32], y1[32];
-        tmem_ld32_nowait(d1 + 32u * q0, y0);
-        tmem_ld32_nowait(d1 + 32u * (q0 + 1), y1);
-        tmem_wait_ld();
         float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) acc = __ffma2_rn(make_float2(y0[j], y0[j + 1]), make_float2(y0[j], y0[j + 1]), acc);
+        for (int qq = 0; qq < 2; ++qq) {
+          float y[32];
+          tmem_ld32(d1 + 32u * (q0 + qq), y);
+          tmem_wait32(y);
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) acc = __ffma2_rn(make_float2(y1[j], y1[j + 1]), make_float2(y1[j], y1[j + 1]), acc);
-        n2p = acc.x + acc.y;
+          for (int j = 0; j < 32; j += 2)
+            acc = __ffma2_rn(make_float2(y[j], y[j + 1]), make_float2(y[j], y[j + 1]), acc);
+        }
+        n2buf[half * 128 + row] = acc.x + acc.y;
       }
-      part[half * 128 + row] = n2p;
-      named_barrier(1 + slot, 256);
-      const float n2 = part[row] + part[128 + row];
+      mbar_arrive(bar(kBarN2 + slot));
+      if (!mbar_wait_warp(bar(kBarN2 + slot), par, abort_flag, status)) break;
+      const float n2 = n2buf[row] + n2buf[128 + row];
       const float nk = sqrtf(n2);
       const bool zero = !(n2 > 0.f);
       const float s128 = zero ? 0.f : 128.f / nk;
@@ -431,14 +483,18 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
         hb.C0 = 0.f;
 #pragma unroll
         for (int c = 0; c < 3; ++c) hb.dC[c] = 0.f;
+        hb.dA = 0.f;
+        hb.C20 = 0.f;
       }
       float2 rr2 = make_float2(0.f, 0.f);
-#pragma unroll 1
+      uint32_t cw[2][BMSE];
+#pragma unroll
       for (int qq = 0; qq < 2; ++qq) {
         const int q = q0 + qq;
         float y[32];
         tmem_ld32(d1 + 32u * q, y);
-        uint32_t hw[2 * BMSE];
+        tmem_wait32(y);
+        uint32_t hw[2 * BMSE], hw3[2] = {0u, 0u};
 #pragma unroll
         for (int h = 0; h < 2 * BMSE; ++h) hw[h] = 0;
 #pragma unroll
@@ -446,10 +502,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
           uint32_t rh[8], rl[8];
 #pragma unroll
           for (int jp = 0; jp < 16; jp += 2) {
-            const int jj = 16 * hh + jp;
+            const int j0 = 16 * hh + jp;
             float2 rp;
-            const uint2 bb = cell2<BMSE>(make_float2(y[jj], y[jj + 1]), s128, hb, rp);
-            const uint32_t b0 = bb.x, b1 = bb.y;
+            const uint2 bb = cell2<BMSE>(make_float2(y[j0], y[j0 + 1]), s128, hb, rp);
             rr2 = __ffma2_rn(rp, rp, rr2);
             const __half2 hi = __float22half2_rn(rp);
             const float2 hf = __half22float2(hi);
@@ -458,18 +513,16 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
             rl[jp >> 1] = *reinterpret_cast<const uint32_t*>(&lo);
 #pragma unroll
             for (int t2 = 0; t2 < 2; ++t2) {
-              // bits = float pattern of 2^23 + idx: idx in bits 0..2, the constant
-              // part only reaches bits >= 24 of each shifted term
-              const int j = jj + t2;
-              const uint32_t bits = t2 ? b1 : b0;
-              const int rreg = j >> 2, e = j & 3, uu = rreg >> 2, ii = rreg & 3;
+              // bits = float pattern of 2^23 + code: the code in bits 0..2, the
+              // constant part only reaches bits >= 24 of each shifted term
+              const int jc = j0 + t2;
+              const uint32_t bits = t2 ? bb.y : bb.x;
+              const int rreg = jc >> 2, e = jc & 3, uu = rreg >> 2, ii = rreg & 3;
               if constexpr (BMSE == 3) {
-                if (ii < 3) {
+                if (ii < 3)
                   hw[uu * 3 + ii] += bits << (4 * e);
-                } else {
-#pragma unroll
-                  for (int b = 0; b < 3; ++b) hw[uu * 3 + b] |= ((bits >> b) & 1u) << (4 * e + 3);
-                }
+                else
+                  hw3[uu] += bits << (4 * e);     // spread into bit 3 of H0..H2 below
               } else if constexpr (BMSE == 2) {
                 hw[uu * 2 + (ii >> 1)] += bits << (4 * e + 2 * (ii & 1));
               } else {
@@ -482,56 +535,77 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
           tmem_st8(d1 + 32u * q + 8u * hh, rh);
           tmem_st8(d1 + 32u * q + 16u + 8u * hh, rl);
         }
+        if constexpr (BMSE == 3) {
 #pragma unroll
-        for (int w = 0; w < BMSE; ++w)
-          srow[q * (BMSE + 1) + w] = zero ? 0u : __byte_perm(hw[2 * w], hw[2 * w + 1], 0x5410);
+          for (int uu = 0; uu < 2; ++uu)
+#pragma unroll
+            for (int b = 0; b < 3; ++b) hw[uu * 3 + b] |= ((hw3[uu] >> b) & 0x1111u) << 3;
+        }
+#pragma unroll
+        for (int w = 0; w < BMSE; ++w) cw[qq][w] = zero ? 0u : ~__byte_perm(hw[2 * w], hw[2 * w + 1], 0x5410);
       }
       asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       tc_fence_before();
       mbar_arrive(bar(kBarRFull + slot));
-      part[256 + half * 128 + row] = rr2.x + rr2.y;
-      if (!mbar_wait(bar(kBarD2Full + slot), par, abort_flag, status)) break;
+      rrbuf[half * 128 + row] = rr2.x + rr2.y;
+      mbar_arrive(bar(kBarRR + slot));
+      if (!mbar_wait_warp(bar(kBarD2Full + slot), par, abort_flag, status)) break;
       tc_fence_after();
-      float z0[32], z1[32];
-      tmem_ld32_nowait(d2 + 32u * q0, z0);
-      tmem_ld32_nowait(d2 + 32u * (q0 + 1), z1);
-      tmem_wait_ld();
+      // bit = [z >= 0] = not the sign bit (z = -0 cannot arise for a nonzero
+      // residual; zero keys get all ones).  Bit p of quarter q's word holds
+      // coordinate 32q + 16 (p >> 4) + 4 (p & 3) + ((p >> 2) & 3); the bits are
+      // shifted in from the top, p = 31 first.
+      uint32_t sw[2];
 #pragma unroll
       for (int qq = 0; qq < 2; ++qq) {
-        const float* z = qq ? z1 : z0;
-        uint32_t sw = 0;
+        uint32_t neg = 0;
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) {
-          const int rreg = jj >> 2, e = jj & 3, uu = rreg >> 2, ii = rreg & 3;
-          sw |= (z[jj] >= 0.f ? 1u : 0u) << (16 * uu + 4 * e + ii);
+        for (int hz = 1; hz >= 0; --hz) {   // coordinates 32q + 16hz .. +15 fill bits 16hz .. 16hz + 15
+          float z[16];
+          tmem_ld16(d2 + 32u * (q0 + qq) + 16u * hz, z);
+          tmem_wait16(z);
+#pragma unroll
+          for (int p = 15; p >= 0; --p) {
+            const int jj = 4 * (p & 3) + ((p >> 2) & 3);
+            neg = __funnelshift_l(__float_as_uint(z[jj]), neg, 1);
+          }
         }
-        srow[(q0 + qq) * (BMSE + 1) + BMSE] = zero ? 0xFFFFFFFFu : sw;
+        sw[qq] = zero ? 0xFFFFFFFFu : ~neg;
       }
       tc_fence_before();
       mbar_arrive(bar(kBarD2Free + slot));
-      named_barrier(1 + slot, 256);
       const int64_t key = (blockIdx.x + i * gridDim.x) * kTile + row;
       if (key < n) {
-        // each group writes its two quarter chunks; group 0 of the slot writes the norms
+        // this half's two quarter chunks
+        uint32_t wv[2 * (BMSE + 1)];
+#pragma unroll
+        for (int qq = 0; qq < 2; ++qq) {
+#pragma unroll
+          for (int w = 0; w < BMSE; ++w) wv[qq * (BMSE + 1) + w] = cw[qq][w];
+          wv[qq * (BMSE + 1) + BMSE] = sw[qq];
+        }
         uint8_t* dst = payload + key * kRowBytes + q0 * 4 * (BMSE + 1);
-        const uint32_t* src = srow + q0 * (BMSE + 1);
-        if constexpr (BMSE == 3) {
-          reinterpret_cast<uint4*>(dst)[0] = reinterpret_cast<const uint4*>(src)[0];
-          reinterpret_cast<uint4*>(dst)[1] = reinterpret_cast<const uint4*>(src)[1];
-        } else if constexpr (BMSE == 1) {
-          reinterpret_cast<uint4*>(dst)[0] = reinterpret_cast<const uint4*>(src)[0];
+        if constexpr (BMSE == 2) {
+#pragma unroll
+          for (int w = 0; w < 6; ++w) reinterpret_cast<uint32_t*>(dst)[w] = wv[w];
         } else {
 #pragma unroll
-          for (int w = 0; w < 6; ++w) reinterpret_cast<uint32_t*>(dst)[w] = src[w];
-        }
-        if (half == 0) {
-          const float rho = nk * sqrtf(part[256 + row] + part[384 + row]) * (1.0f / 128.f);
-          const uint32_t nn = uint32_t(__half_as_ushort(__float2half_rn(nk))) |
-                              (uint32_t(__half_as_ushort(__float2half_rn(rho))) << 16);
-          reinterpret_cast<uint32_t*>(norms)[key] = nn;
+          for (int v = 0; v < (BMSE + 1) / 2; ++v)
+            reinterpret_cast<uint4*>(dst)[v] = make_uint4(wv[4 * v], wv[4 * v + 1], wv[4 * v + 2], wv[4 * v + 3]);
         }
       }
+      if (half == 0) {
+        // ||r|| = n ||r_rot|| from both halves' sums (r_rot scaled by 128); the
+        // other half writes these sums again only after its next N2 wait, which
+        // needs this thread's next arrival
+        if (!mbar_wait_warp(bar(kBarRR + slot), par, abort_flag, status)) break;
+        const float rho = nk * sqrtf(rrbuf[row] + rrbuf[128 + row]) * (1.0f / 128.f);
+        const uint32_t nn = uint32_t(__half_as_ushort(__float2half_rn(nk))) |
+                            (uint32_t(__half_as_ushort(__float2half_rn(rho))) << 16);
+        if (key < n) reinterpret_cast<uint32_t*>(norms)[key] = nn;
+      }
     }
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");   // none in flight on an early exit
   }
   tc_fence_before();
   __syncthreads();
@@ -560,6 +634,7 @@ bool device_is_sm100() {
   cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
   return major == 10 && minor == 0;
 }
+
 
 }  // namespace
 
@@ -591,6 +666,11 @@ cudaError_t launch_quantize_tc(const tq_ctx* ctx, const void* keys, int dtype, i
   for (int i = 0; i < L / 2 - 1; ++i) hb.Tneg[i] = -float(128.0 * ctx->t[L / 2 + i]) * 0x1p100f;
   hb.C0 = float(128.0 * ctx->c[L / 2]);
   for (int i = 0; i + 1 < L / 2; ++i) hb.dC[i] = float(128.0 * ctx->c[L / 2 + i + 1]) - float(128.0 * ctx->c[L / 2 + i]);
+  if (L == 8) {
+    hb.dT31 = hb.Tneg[2] - hb.Tneg[0];
+    hb.dA = hb.dC[2] - hb.dC[0];
+    hb.C20 = float(128.0 * ctx->c[L / 2 + 2]) - hb.C0;
+  }
   switch (ctx->bmse) {
     case 1: {
       auto k = quantize_tc_kernel<1>;
