@@ -168,6 +168,14 @@ def run_reference(args, rank):
     return 0
 
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per key of the
+# current kernels, from one ncu capture at S = 16384 (1 048 576 keys); per
+# launch it scales with the keys processed.  Summaries: profiles/quantize_tc_decode_s16384.md
+# and profiles/logits_mma_decode_s16384.md.  Set to None when a kernel changes.
+DRAM_BYTES_PER_KEY = {"tq_quantize": (268.648960e6 + 53.591040e6) / 1048576,
+                      "tq_logits": (71.457024e6 + 3.751168e6) / 1048576}
+
+
 def max_over_ranks(x: float, dist, device) -> float:
     """The largest value of x over all ranks (x itself without a process group)."""
     if dist is None:
@@ -215,7 +223,9 @@ def result_line(*, world, n, steps, warmup, ms, q_ms, l_ms, e2e_ms, h2d, d2h, cl
                    "l2": "inputs larger than L2: keys 537 MB, packed cache 143 MB; logits read the cache "
                          "written one step earlier"},
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": hbm, "unit": "GB/s",
-                     "frac": ach / hbm, "peak_source": src, "traffic": None},
+                     "frac": ach / hbm, "peak_source": src,
+                     "traffic": (None if DRAM_BYTES_PER_KEY.get(dom) is None else DRAM_BYTES_PER_KEY[dom] * n),
+                     "traffic_source": "ncu capture at S=16384 scaled by keys (bytes per launch)"},
         "kernels": kernels,
         "logits_keys_per_s": world * n / l_ms * 1e3,
         "quantize_vectors_per_s": world * n / q_ms * 1e3,

@@ -405,13 +405,25 @@ def topk(Q: np.ndarray, codes, bits, n16, rho16, tb: Tables, k: int):
 # ---------------------------------------------------------------------------
 
 
+def layout_dims(d: int, m: int) -> tuple:
+    """Slots of the packed layout: d and m rounded up to multiples of 64.
+
+    Reading (the pages fix no storage format): a dimension that is not a
+    multiple of 64 (d = 200 for the vector-search workload) is stored in the
+    quarter-chunk layout of the next multiple of 64; the slots past d (codes)
+    and past m (sign bits) hold zeros and carry no information.
+    """
+    return -(-d // 64) * 64, -(-m // 64) * 64
+
+
 def row_bytes(d: int, m: int, bmse: int) -> int:
-    return d * bmse // 8 + m // 8
+    dp, mp = layout_dims(d, m)
+    return dp * bmse // 8 + mp // 8
 
 
 def _check_layout_dims(d: int, m: int, bmse: int):
-    if d % 64 or m % 64:
-        raise ValueError("packed layout needs d and m multiples of 64")
+    if d % 8 or m % 8 or d < 8 or m < 8:
+        raise ValueError("packed layout needs d and m multiples of 8")
     if not 1 <= bmse <= 4:
         raise ValueError("1 <= b' <= 4")
 
@@ -471,10 +483,13 @@ def pack_rows(codes: np.ndarray, bits: np.ndarray, bmse: int) -> np.ndarray:
     N, d = codes.shape
     m = bits.shape[1]
     _check_layout_dims(d, m, bmse)
+    dp, mp = layout_dims(d, m)
+    codes = np.concatenate([codes, np.zeros((N, dp - d), dtype=codes.dtype)], axis=1)
+    bits = np.concatenate([bits, np.zeros((N, mp - m), dtype=bits.dtype)], axis=1)
     halves = []
     for q in range(4):
-        halves += _code_halfwords(codes[:, q * d // 4:(q + 1) * d // 4], bmse)
-        halves += _sign_halfwords(bits[:, q * m // 4:(q + 1) * m // 4])
+        halves += _code_halfwords(codes[:, q * dp // 4:(q + 1) * dp // 4], bmse)
+        halves += _sign_halfwords(bits[:, q * mp // 4:(q + 1) * mp // 4])
     hw = np.stack(halves, axis=1).astype(np.uint16)
     out = hw.astype("<u2").view(np.uint8).reshape(N, -1)
     assert out.shape[1] == row_bytes(d, m, bmse)
@@ -482,8 +497,23 @@ def pack_rows(codes: np.ndarray, bits: np.ndarray, bmse: int) -> np.ndarray:
 
 
 def unpack_rows(payload: np.ndarray, d: int, m: int, bmse: int):
-    """Inverse of pack_rows: (N, row_bytes) uint8 -> (codes (N, d), bits (N, m))."""
+    """Inverse of pack_rows: (N, row_bytes) uint8 -> (codes (N, d), bits (N, m)).
+
+    The padding slots (past d and m) are read too and returned separately by
+    ``unpack_padding`` so that tests can check they are zero."""
+    codes, bits = _unpack_slots(payload, d, m, bmse)
+    return codes[:, :d], bits[:, :m]
+
+
+def unpack_padding(payload: np.ndarray, d: int, m: int, bmse: int):
+    """The code and sign slots past d and m (all zero in a valid row)."""
+    codes, bits = _unpack_slots(payload, d, m, bmse)
+    return codes[:, d:], bits[:, m:]
+
+
+def _unpack_slots(payload: np.ndarray, d: int, m: int, bmse: int):
     _check_layout_dims(d, m, bmse)
+    d, m = layout_dims(d, m)
     payload = np.ascontiguousarray(payload, dtype=np.uint8)
     N = payload.shape[0]
     hw = payload.reshape(N, -1).view("<u2").astype(np.uint32)

@@ -70,3 +70,7 @@ def test_argument_validation_without_device(L):
 def test_row_bytes_formula():
     for d, m, b in [(128, 128, 3), (128, 128, 2), (64, 64, 1), (256, 256, 3)]:
         assert O.row_bytes(d, m, b) == d * b // 8 + m // 8
+    # dimensions that are not multiples of 64 are stored in the next multiple of 64
+    for d, m, b in [(200, 200, 1), (200, 200, 3), (72, 136, 2)]:
+        dp, mp = -(-d // 64) * 64, -(-m // 64) * 64
+        assert O.row_bytes(d, m, b) == dp * b // 8 + mp // 8

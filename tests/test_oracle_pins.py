@@ -477,7 +477,7 @@ def test_gqa_logits_head_mapping():
 
 
 @pytest.mark.parametrize("d,m,bmse", [(64, 64, 1), (64, 64, 2), (128, 128, 3), (128, 128, 2),
-                                      (128, 64, 4), (256, 128, 3)])
+                                      (128, 64, 4), (256, 128, 3), (200, 200, 1), (200, 200, 3), (72, 136, 2)])
 def test_pack_unpack_round_trip(d, m, bmse):
     rng = np.random.default_rng(d + m + bmse)
     codes = rng.integers(0, 1 << bmse, (33, d))
@@ -487,6 +487,24 @@ def test_pack_unpack_round_trip(d, m, bmse):
     c2, b2 = O.unpack_rows(p, d, m, bmse)
     np.testing.assert_array_equal(c2, codes)
     np.testing.assert_array_equal(b2, bits)
+    # slots past d and m (layout rounded up to multiples of 64) stay empty
+    pc, pb = O.unpack_padding(p, d, m, bmse)
+    assert pc.shape == (33, -(-d // 64) * 64 - d) and not pc.any()
+    assert pb.shape == (33, -(-m // 64) * 64 - m) and not pb.any()
+
+
+def test_padded_layout_is_the_next_multiple_of_64():
+    # d = 200 codes occupy the first 200 of 256 slots: a row packed at d = 200
+    # equals the d = 256 row of the same codes followed by zero codes.
+    rng = np.random.default_rng(5)
+    codes = rng.integers(0, 8, (7, 200))
+    bits = rng.integers(0, 2, (7, 200)).astype(bool)
+    p200 = O.pack_rows(codes, bits, 3)
+    codes256 = np.concatenate([codes, np.zeros((7, 56), dtype=codes.dtype)], axis=1)
+    bits256 = np.concatenate([bits, np.zeros((7, 56), dtype=bool)], axis=1)
+    np.testing.assert_array_equal(p200, O.pack_rows(codes256, bits256, 3))
+    assert O.row_bytes(200, 200, 3) == 256 * 3 // 8 + 256 // 8 == 128
+    assert O.row_bytes(200, 200, 1) == 64
 
 
 def test_pack_layout_hand_example():
