@@ -1,5 +1,5 @@
 // CUDA-core quantize and dequantize kernels for every supported shape
-// (d, m multiples of 64 up to 256, fp32 or bf16 keys).  The tensor-core
+// (d, m multiples of 8 from 64 to 256, fp32 or bf16 keys).  The tensor-core
 // quantize kernel (k_quantize_tc.cu) covers d = m = 128 with bf16 keys; this
 // file covers the rest and the dequantisation.
 //
@@ -37,10 +37,13 @@ __global__ void __launch_bounds__(kThreads) quantize_simt_kernel(const T* __rest
   float* sk = smem;                          // [kKeys][d] keys, later r_rot
   float* sn = sk + kKeys * d;                // [kKeys] norms
   float* srr = sn + kKeys;                   // [kKeys] ||r_rot||^2
-  uint8_t* scode = reinterpret_cast<uint8_t*>(srr + kKeys);   // [kKeys][d]
-  uint8_t* sbit = scode + kKeys * d;                           // [kKeys][m]
   const RowGeom g = make_geom(d, m, bmse);
+  uint8_t* scode = reinterpret_cast<uint8_t*>(srr + kKeys);   // [kKeys][dp] layout slots
+  uint8_t* sbit = scode + kKeys * g.dp;                        // [kKeys][mp]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // the slots past d and m are never written below: zero them once
+  for (int idx = tid; idx < kKeys * g.dp; idx += kThreads) scode[idx] = 0;
+  for (int idx = tid; idx < kKeys * g.mp; idx += kThreads) sbit[idx] = 0;
 
   for (int64_t base = int64_t(blockIdx.x) * kKeys; base < n; base += int64_t(gridDim.x) * kKeys) {
     const int nk = (n - base) < kKeys ? int(n - base) : kKeys;
@@ -83,7 +86,7 @@ __global__ void __launch_bounds__(kThreads) quantize_simt_kernel(const T* __rest
           for (int i = 0; i < cb.levels - 1; ++i) code += (u > cb.t[i]) ? 1 : 0;
           rr = u - cb.c[code];
         }
-        scode[k * d + j] = uint8_t(code);
+        scode[k * g.dp + j] = uint8_t(code);
         sk[k * d + j] = rr;
       }
     }
@@ -111,13 +114,13 @@ __global__ void __launch_bounds__(kThreads) quantize_simt_kernel(const T* __rest
     for (int ii = 0; ii < 2; ++ii) {
       const int i = tid + ii * kThreads;
       if (i < m)
-        for (int k = 0; k < kKeys; ++k) sbit[k * m + i] = z[ii][k] >= 0.f ? 1 : 0;
+        for (int k = 0; k < kKeys; ++k) sbit[k * g.mp + i] = z[ii][k] >= 0.f ? 1 : 0;
     }
     __syncthreads();
     const int hw_per_row = g.row_bytes / 2;
     for (int idx = tid; idx < nk * hw_per_row; idx += kThreads) {
       const int k = idx / hw_per_row, h = idx - k * hw_per_row;
-      const uint16_t v = pack_halfword(scode + k * d, sbit + k * m, g, h);
+      const uint16_t v = pack_halfword(scode + k * g.dp, sbit + k * g.mp, g, h);
       reinterpret_cast<uint16_t*>(payload + (base + k) * g.row_bytes)[h] = v;
     }
     if (tid < nk) {
@@ -203,7 +206,8 @@ int grid_for(int64_t n) {
 cudaError_t launch_quantize_simt(const tq_ctx* ctx, const void* keys, int dtype, int64_t n, int64_t ld,
                                  uint8_t* payload, uint16_t* norms, cudaStream_t st) {
   const int d = ctx->d, m = ctx->m;
-  const size_t smem = size_t(kKeys) * d * 4 + 2 * kKeys * 4 + size_t(kKeys) * (d + m);
+  const RowGeom g = make_geom(d, m, ctx->bmse);
+  const size_t smem = size_t(kKeys) * d * 4 + 2 * kKeys * 4 + size_t(kKeys) * (g.dp + g.mp);
   const int grid = grid_for(n);
   if (dtype == TQ_F32) {
     auto kern = quantize_simt_kernel<float>;

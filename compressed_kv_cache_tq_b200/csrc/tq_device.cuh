@@ -7,10 +7,13 @@
 
 namespace tq {
 
-// Geometry of the packed row for (d, m, b').
+// Geometry of the packed row for (d, m, b').  The layout has dp and mp slots:
+// d and m rounded up to multiples of 64; the slots past d (codes) and past m
+// (sign bits) are zero.
 struct RowGeom {
   int d, m, bmse;
-  int uq, uqm;         // code units and sign units per quarter (d/64, m/64)
+  int dp, mp;          // layout slots
+  int uq, uqm;         // code units and sign units per quarter (dp/64, mp/64)
   int per_q;           // halfwords per quarter chunk
   int row_bytes;
 };
@@ -20,8 +23,10 @@ __host__ __device__ inline RowGeom make_geom(int d, int m, int bmse) {
   g.d = d;
   g.m = m;
   g.bmse = bmse;
-  g.uq = d / 64;
-  g.uqm = m / 64;
+  g.dp = (d + 63) / 64 * 64;
+  g.mp = (m + 63) / 64 * 64;
+  g.uq = g.dp / 64;
+  g.uqm = g.mp / 64;
   g.per_q = bmse * g.uq + g.uqm;
   g.row_bytes = 8 * g.per_q;   // 4 quarters x 2 bytes x per_q
   return g;
@@ -29,7 +34,7 @@ __host__ __device__ inline RowGeom make_geom(int d, int m, int bmse) {
 
 // Code of rotated coordinate j in a packed row (halfword view).
 __device__ inline int unpack_code(const uint16_t* hw, const RowGeom& g, int j) {
-  const int qd = g.d / 4;
+  const int qd = g.dp / 4;
   const int q = j / qd, rem = j - q * qd;
   const int r = rem >> 2, e = rem & 3, u = r >> 2, i = r & 3;
   const uint16_t* base = hw + q * g.per_q + u * g.bmse;
@@ -47,21 +52,21 @@ __device__ inline int unpack_code(const uint16_t* hw, const RowGeom& g, int j) {
 
 // Sign bit (1 = +1) of JL coordinate i in a packed row.
 __device__ inline int unpack_sign(const uint16_t* hw, const RowGeom& g, int i) {
-  const int qm = g.m / 4;
+  const int qm = g.mp / 4;
   const int q = i / qm, rem = i - q * qm;
   const int r = rem >> 2, e = rem & 3, u = r >> 2, ii = r & 3;
   const uint16_t h = hw[q * g.per_q + g.bmse * g.uq + u];
   return (h >> (4 * e + ii)) & 1;
 }
 
-// Build packed halfword `h` of a row from per-coordinate codes and sign bits
-// held in shared memory (codes[j], bits[i] as bytes).
+// Build packed halfword `h` of a row from per-slot codes and sign bits held in
+// shared memory (codes[0 .. dp), bits[0 .. mp) as bytes, zero past d and m).
 __device__ inline uint16_t pack_halfword(const uint8_t* codes, const uint8_t* bits, const RowGeom& g, int h) {
   const int q = h / g.per_q, loc = h - q * g.per_q;
   uint32_t out = 0;
   if (loc < g.bmse * g.uq) {
     const int u = loc / g.bmse, ih = loc - u * g.bmse;
-    const uint8_t* cq = codes + q * (g.d / 4);
+    const uint8_t* cq = codes + q * (g.dp / 4);
     for (int e = 0; e < 4; ++e) {
       if (g.bmse == 1) {
         for (int i = 0; i < 4; ++i) out |= uint32_t(cq[4 * (4 * u + i) + e] & 1) << (4 * e + i);
@@ -75,7 +80,7 @@ __device__ inline uint16_t pack_halfword(const uint8_t* codes, const uint8_t* bi
     }
   } else {
     const int u = loc - g.bmse * g.uq;
-    const uint8_t* bq = bits + q * (g.m / 4);
+    const uint8_t* bq = bits + q * (g.mp / 4);
     for (int e = 0; e < 4; ++e)
       for (int i = 0; i < 4; ++i) out |= uint32_t(bq[4 * (4 * u + i) + e] & 1) << (4 * e + i);
   }

@@ -256,7 +256,7 @@ void tq_free(tq_ctx* ctx) {
 }
 
 static bool dims_ok(int d, int bits, int m) {
-  return !(d < 64 || d > 256 || d % 64 || m < 64 || m > 256 || m % 64 || bits < 2 || bits > 4);
+  return !(d < 64 || d > 256 || d % 8 || m < 64 || m > 256 || m % 8 || bits < 2 || bits > 4);
 }
 
 static void build_tables(int d, int bits, int m, uint64_t seed, uint32_t stream_base, std::vector<double>& R,
@@ -294,7 +294,8 @@ tq_status tq_init_ex(int d, int bits, int m, uint64_t seed, uint32_t stream_base
   ctx->bits = bits;
   ctx->bmse = bits - 1;
   ctx->levels = 1 << (bits - 1);
-  ctx->row_bytes = d * (bits - 1) / 8 + m / 8;
+  // layout slots: d and m rounded up to multiples of 64 (zero padding slots)
+  ctx->row_bytes = (d + 63) / 64 * 64 * (bits - 1) / 8 + (m + 63) / 64 * 8;
   ctx->seed = seed;
   ctx->stream_base = stream_base;
   cudaGetDevice(&ctx->device);

@@ -33,7 +33,10 @@
  *     message is kept in tq_last_cuda_error()).
  *
  * Packed layout (one row per key; the pages fix no layout, only "no
- * per-block constants"):  d and m are multiples of 64, b' = bits - 1.
+ * per-block constants"):  b' = bits - 1.  The layout has dp and mp slots, d
+ * and m rounded up to multiples of 64 (equal to d and m when they are
+ * multiples of 64); in the formulas below d and m stand for dp and mp, and
+ * the code slots j >= d and sign slots i >= m of the true sizes are zero.
  *   payload row = 4 quarter chunks q = 0..3 of 2 (b' d/64 + m/64) bytes.
  *   Chunk q holds rotated coordinates j = q d/4 + 4r + e (r < d/16, e < 4) as
  *   little-endian 16-bit halfwords: the b' code halfwords of each unit
@@ -44,7 +47,7 @@
  *     b'=3: Hi nibble e bits 0-2 (i<3)     = code(4u+i, e);  bit 3 = bit i of code(4u+3, e)
  *     signs: H nibble e bit i              = [ (S r)_{q m/4 + 4(4u+i) + e} >= 0 ]
  *   norms: two fp16 per key, (||k||, ||r||), round to nearest even.
- *   Rows of a cache are ordered [B][Hkv][S]; row bytes = d b'/8 + m/8.
+ *   Rows of a cache are ordered [B][Hkv][S]; row bytes = dp b'/8 + mp/8.
  */
 #ifndef TQ_H_
 #define TQ_H_
@@ -78,12 +81,12 @@ typedef enum { TQ_F32 = 0, TQ_BF16 = 1 } tq_dtype;
  * P (m x d) is drawn from stream 1 and the JL matrix applied to the residual
  * is S = P R; the codebook has 2^(bits-1) Lloyd-Max levels for the law of one
  * coordinate of a random unit vector in R^d.  m = d.
- * d: multiple of 64, 64 <= d <= 256.  bits: 2..4 (1..3 Lloyd-Max bits + 1 QJL bit).
+ * d: multiple of 8, 64 <= d <= 256.  bits: 2..4 (1..3 Lloyd-Max bits + 1 QJL bit).
  * *out receives a library-owned context; release it with tq_free.
  * Errors: TQ_ERR_ARG (out == NULL), TQ_ERR_UNSUPPORTED (d, bits), TQ_ERR_CUDA. */
 tq_status tq_init(int d, int bits, uint64_t seed, tq_ctx** out);
 
-/* As tq_init with an explicit JL row count m (multiple of 64, <= 256) and the
+/* As tq_init with an explicit JL row count m (multiple of 8, 64 <= m <= 256) and the
  * first Philox stream used (G from stream_base, P from stream_base + 1). */
 tq_status tq_init_ex(int d, int bits, int m, uint64_t seed, uint32_t stream_base, tq_ctx** out);
 

@@ -26,6 +26,8 @@ def check_quantize(payload, norms, K64, tb: O.Tables, report=None):
     norms = np.asarray(norms).view(np.float16).reshape(-1, 2)
     qz = O.quantize(K64, tb)
     codes, bits = O.unpack_rows(payload, tb.d, tb.m, tb.bmse)
+    pad_c, pad_b = O.unpack_padding(payload, tb.d, tb.m, tb.bmse)
+    assert not pad_c.any() and not pad_b.any(), "layout padding slots must be zero"
     code_mis = codes != qz.codes
     code_band = O.code_boundary_distance(qz.u, tb.t) <= O.CODE_BAND
     bad_codes = code_mis & ~code_band

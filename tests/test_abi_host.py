@@ -39,7 +39,8 @@ def test_exports_every_declared_symbol(L):
 
 
 @pytest.mark.parametrize("d,bits,m,seed,base", [(128, 3, 128, 42, 0), (128, 4, 128, 7, 0), (64, 2, 64, 5, 2),
-                                                (256, 3, 128, 9, 0), (64, 4, 192, 1, 4)])
+                                                (256, 3, 128, 9, 0), (64, 4, 192, 1, 4), (200, 2, 200, 42, 0),
+                                                (200, 4, 200, 42, 0)])
 def test_host_tables_match_oracle(L, d, bits, m, seed, base):
     R, P, c, t = L.tq_host_tables(d, bits, seed, m=m, stream_base=base)
     tb = O.make_tables(d, bits, seed, m=m, stream_base=base)
@@ -51,7 +52,9 @@ def test_host_tables_match_oracle(L, d, bits, m, seed, base):
 
 def test_host_tables_reject_unsupported(L):
     lib = L.lib()
-    for d, bits, m in [(100, 3, 100), (128, 5, 128), (128, 1, 128), (512, 3, 512), (128, 3, 96)]:
+    # d, m: multiples of 8 from 64 to 256; bits 2..4
+    for d, bits, m in [(100, 3, 100), (128, 5, 128), (128, 1, 128), (512, 3, 512), (128, 3, 36), (56, 3, 56),
+                       (264, 3, 264)]:
         assert lib.tq_host_tables(d, bits, m, 1, 0, None, None, None, None) == 2
 
 

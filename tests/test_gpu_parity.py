@@ -61,7 +61,8 @@ def test_quantize_toy_fp32(lib):
 
 @pytest.mark.parametrize("d,m,bits,dtype", [(64, 64, 3, torch.bfloat16), (64, 64, 2, torch.float32),
                                             (256, 256, 3, torch.bfloat16), (128, 64, 4, torch.float32),
-                                            (192, 128, 2, torch.bfloat16)])
+                                            (192, 128, 2, torch.bfloat16), (200, 200, 2, torch.float32),
+                                            (200, 200, 4, torch.float32), (72, 136, 3, torch.bfloat16)])
 def test_quantize_other_shapes(lib, d, m, bits, dtype):
     ctx = _ctx(lib, d=d, bits=bits, seed=5, m=m)
     k = W.toy_keys(777, d, seed=d + m)
@@ -141,6 +142,25 @@ def test_logits_against_oracle(lib, bits, B, Hkv, G, S):
             check_close(o[b, hk * G:(hk + 1) * G], scale * s, scale * A)
 
 
+@pytest.mark.parametrize("d,bits", [(200, 2), (200, 4), (72, 3)])
+def test_logits_padded_layout_against_oracle(lib, d, bits):
+    """d not a multiple of 64 (vector-search d = 200): the CUDA-core estimator
+    on the padded layout."""
+    ctx = _ctx(lib, d=d, bits=bits, seed=23)
+    B, Hkv, G, S = 1, 2, 3, 301
+    k = W.search_vectors(B * Hkv * S, d, seed=7, which=0)
+    payload, norms = lib.tq_quantize(ctx, torch.from_numpy(k).to(DEV))
+    q = W.search_vectors(B * Hkv * G, d, seed=7, which=1).reshape(B, Hkv * G, d)
+    out = lib.tq_logits(ctx, torch.from_numpy(q).to(DEV), payload, norms, Hkv)
+    _status_clean(lib, ctx)
+    tb = tables_of(ctx)
+    pl, nr, o = payload.cpu().numpy(), norms.cpu().numpy(), out.cpu().numpy()
+    for hk in range(Hkv):
+        rows = slice(hk * S, (hk + 1) * S)
+        s_, A = oracle_estimates(pl[rows], nr[rows], q[0, hk * G:(hk + 1) * G].astype(np.float64), tb)
+        check_close(o[0, hk * G:(hk + 1) * G], s_, A)
+
+
 def test_toy_logits_all_pairs(lib):
     """toy workload: 64 queries x 4096 keys, all pairs (one GQA group of 64)."""
     ctx = _ctx(lib, bits=3, seed=42)
@@ -154,7 +174,7 @@ def test_toy_logits_all_pairs(lib):
 
 
 @pytest.mark.parametrize("full", [True, False])
-@pytest.mark.parametrize("d,bits", [(128, 4), (64, 2)])
+@pytest.mark.parametrize("d,bits", [(128, 4), (64, 2), (200, 4)])
 def test_dequantize_against_oracle(lib, full, d, bits):
     ctx = _ctx(lib, d=d, bits=bits, seed=13)
     k = W.toy_keys(555, d, seed=8)
@@ -184,11 +204,12 @@ def test_dequantize_full_matches_logits(lib):
     check_close(out[0].cpu().numpy(), ref, A)
 
 
-@pytest.mark.parametrize("bits,n,nq,k", [(3, 5000, 16, 10), (4, 3001, 9, 1), (2, 700, 5, 64), (3, 100, 3, 10)])
-def test_topk_against_oracle(lib, bits, n, nq, k):
-    ctx = _ctx(lib, bits=bits, seed=17)
-    db = W.search_vectors(n, 128, seed=100 + bits, which=0)
-    qs = W.search_vectors(nq, 128, seed=100 + bits, which=1)
+@pytest.mark.parametrize("d,bits,n,nq,k", [(128, 3, 5000, 16, 10), (128, 4, 3001, 9, 1), (128, 2, 700, 5, 64),
+                                           (128, 3, 100, 3, 10), (200, 2, 3000, 7, 10), (200, 4, 2000, 5, 10)])
+def test_topk_against_oracle(lib, d, bits, n, nq, k):
+    ctx = _ctx(lib, d=d, bits=bits, seed=17)
+    db = W.search_vectors(n, d, seed=100 + bits, which=0)
+    qs = W.search_vectors(nq, d, seed=100 + bits, which=1)
     payload, norms = lib.tq_quantize(ctx, torch.from_numpy(db).to(DEV))
     ids, scores = lib.tq_topk(ctx, torch.from_numpy(qs).to(DEV), payload, norms, k)
     _status_clean(lib, ctx)
