@@ -1,0 +1,695 @@
+// Inner-product top-k on the tensor cores (sm_100a): the vector-search use of
+// airosetta.com "Google TurboQuant" (recall@1@k over GloVe-like vectors with
+// near-zero indexing time).  The estimator of one (query, row) pair,
+//   s = n16 sum_j c[idx_j] (Rq)_j + sqrt(pi/2)/m rho16 sum_i sigma_i (Sq)_i,
+// is one inner product s = <Kw, Qw> of a per-row weight vector
+//   Kw = [n16 c[idx_0 .. d-1], sqrt(pi/2)/m rho16 sigma_0 .. m-1, 0 ...]
+// and a per-query vector Qw = [Rq, Sq, 0 ...], both KP = round-up(d + m, 64)
+// long.  Four kernels:
+//   1. decode_rows_kernel: packed rows -> Kw in fp16 (one warp per row), and
+//      the largest code-part norm ||Kw_code|| and sign weight |w| over rows.
+//   2. prep_queries_kernel: Qw in fp16 and the per-query error bound E_q.
+//   3. search_tc_kernel: tcgen05 MMA of 128-query tiles (resident in shared
+//      memory) against 256-row tiles (TMA ring), scores in TMEM; the epilogue
+//      keeps each query's running k best scores and appends every row whose
+//      score is at least (k-th best - 2 E_q) to the query's candidate list.
+//   4. finish_kernel: per query, the candidates sorted by approximate score and
+//      cut at (k-th approximate - 2 E_q), re-scored exactly in fp64 and ordered
+//      by (score descending, id ascending); the first k are the answer.
+// Completeness: every approximate score is within E_q of the exact one.  The
+// k-th largest approximate score A_k is then at most T + E_q (T: the exact
+// k-th largest; otherwise k rows would have exact scores above T), and every
+// row of the exact top k has approximate score >= T - E_q >= A_k - 2 E_q, so
+// it is a candidate.  A CTA that scans only part of the rows uses its own,
+// lower, A_k: its cut keeps a superset.  A query whose candidate list
+// overflows is answered by an exact scan of all rows in the finishing kernel.
+// Error bound: Kw and Qw are rounded to fp16 (relative 2^-11 each) after fp32
+// arithmetic (R q and P R q in fp32: relative error below 2e-4 of ||Kw|| ||q||
+// at d <= 256), and the tensor cores accumulate KP <= 512 exact products in
+// fp32 (below KP 2^-23 of sum |Kw_j Qw_j|).  With
+//   sum_j |Kw_j Qw_j| <= max ||Kw_code|| ||Rq||_2 + max |w| ||Sq||_1
+// (Cauchy-Schwarz on the code part; the sign part has |sigma_i| = 1),
+//   E_q = 1.5e-3 (max ||Kw_code|| ||Rq||_2 + max |w| ||Sq||_1) + an absolute
+// term for fp16 subnormals bounds |s_approx - s| (1.5e-3 > 2^-10 + 512 2^-23
+// + 2e-4).
+#include <cuda_fp16.h>
+
+#include <algorithm>
+
+#include "tc_sm100.cuh"
+#include "tq_device.cuh"
+#include "tq_internal.h"
+
+namespace tq {
+namespace {
+
+using namespace tc;
+
+constexpr int kQT = 128;                 // queries per tile (MMA M)
+constexpr int kRT = 256;                 // database rows per tile (MMA N)
+constexpr int kBStages = 3;              // row-tile K-block ring
+constexpr int kSearchThreads = 192;      // TMA warp, MMA warp, 4 epilogue warps
+constexpr int kMaxK = 32;                // k handled by the epilogue's running top-k
+constexpr int kCap = 2048;               // candidates kept per query
+constexpr float kErrRel = 1.5e-3f;       // relative error bound (see above)
+constexpr float kErrAbs = 0x1p-20f;      // absolute term (fp16 subnormals)
+constexpr uint32_t kIdescSearch = idesc_f16(0, kQT, kRT);   // fp16 x fp16 -> fp32, 128 x 256
+
+template <int KB>
+struct SearchSmem {
+  static constexpr uint32_t kOffA = 0;                           // KB blocks of 128 rows x 128 B
+  static constexpr uint32_t kOffB = KB * 16384u;                 // kBStages blocks of 256 rows x 128 B
+  static constexpr uint32_t kOffBar = kOffB + kBStages * 32768u;
+  static constexpr uint32_t kBytes = kOffBar + 256 + 1024;       // + slack for 1024-byte alignment
+};
+
+enum SBar {
+  kSAFull = 0,
+  kSAFree = 1,
+  kSBFull = 2,
+  kSBEmpty = kSBFull + kBStages,
+  kSDFull = kSBEmpty + kBStages,
+  kSDEmpty = kSDFull + 2,
+  kSDone = kSDEmpty + 2,       // final commit of the MMA thread (tracks every MMA it issued)
+  kSNumBars = kSDone + 1
+};
+
+// Waits test the phase without a suspend-time hint: the pipeline's waits often
+// find the phase incomplete, and a suspended thread resumed far too late.
+__device__ __forceinline__ bool swait(uint32_t bar, uint32_t parity, volatile int* abort_flag, uint32_t* status) {
+  return tc::mbar_wait<false>(bar, parity, abort_flag, status, kStatusSearchTc);
+}
+__device__ __forceinline__ bool swait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                           uint32_t* status) {
+  return tc::mbar_wait_warp<false>(bar, parity, abort_flag, status, kStatusSearchTc);
+}
+__device__ __forceinline__ void sdrain(uint32_t bar, uint32_t parity, volatile int* abort_flag, uint32_t* status) {
+  tc::mbar_drain<false>(bar, parity, abort_flag, status, kStatusSearchTc);
+}
+
+// One warp per row: Kw in fp16, rows n .. n_pad - 1 all zero.  maxk_bits[0]
+// gets the largest ||Kw_code|| and maxk_bits[1] the largest |w| (of the
+// rounded values, as float bits).
+__global__ void __launch_bounds__(256) decode_rows_kernel(const uint8_t* __restrict__ payload,
+                                                          const uint16_t* __restrict__ norms, int64_t n,
+                                                          int64_t n_pad, int d, int m, int bmse, int kp,
+                                                          CodebookParams cb, __half* __restrict__ kw,
+                                                          uint32_t* __restrict__ maxk_bits) {
+  const int lane = threadIdx.x & 31;
+  const int64_t r = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (r >= n_pad) return;
+  const RowGeom g = make_geom(d, m, bmse);
+  const bool real = r < n;
+  const uint16_t* hw = reinterpret_cast<const uint16_t*>(payload + (real ? r : 0) * g.row_bytes);
+  const float n16 = real ? half_bits_to_float(norms[2 * r]) : 0.f;
+  const float w = real ? float(kQjlConst) / float(m) * half_bits_to_float(norms[2 * r + 1]) : 0.f;
+  float ss = 0.f;
+  for (int c = lane; c < kp / 8; c += 32) {
+    __align__(16) __half h[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int j = 8 * c + e;
+      float v = 0.f;
+      if (real) {
+        if (j < d)
+          v = n16 * cb.c[unpack_code(hw, g, j)];
+        else if (j < d + m)
+          v = unpack_sign(hw, g, j - d) ? w : -w;
+      }
+      h[e] = __float2half_rn(v);
+      const float hv = __half2float(h[e]);
+      if (j < d) ss = fmaf(hv, hv, ss);
+    }
+    *reinterpret_cast<uint4*>(kw + r * kp + 8 * c) = *reinterpret_cast<const uint4*>(h);
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+  if (lane == 0 && real) {
+    atomicMax(maxk_bits, __float_as_uint(sqrtf(ss)));
+    atomicMax(maxk_bits + 1, __float_as_uint(fabsf(__half2float(__float2half_rn(w)))));
+  }
+}
+
+// One block per query: Qw = [R q, P R q] in fp16 (the rest of the row was
+// zeroed by the caller) and the error bound E_q (see the top of this file).
+__global__ void __launch_bounds__(256) prep_queries_kernel(const float* __restrict__ q, const float* __restrict__ Rt,
+                                                           const float* __restrict__ Pt, int d, int m, int kp,
+                                                           const uint32_t* __restrict__ maxk_bits,
+                                                           __half* __restrict__ qw, float* __restrict__ qerr) {
+  __shared__ float sq[256], sx[256];
+  __shared__ float red[8], red1[8];
+  const int qi = blockIdx.x, tid = threadIdx.x;
+  for (int i = tid; i < d; i += blockDim.x) sq[i] = q[size_t(qi) * d + i];
+  __syncthreads();
+  float ss = 0.f, s1 = 0.f;   // ||Rq||_2^2 and ||Sq||_1 of the rounded values
+  for (int j = tid; j < d; j += blockDim.x) {
+    float x = 0.f;
+    for (int i = 0; i < d; ++i) x = fmaf(Rt[i * d + j], sq[i], x);
+    sx[j] = x;
+    const __half h = __float2half_rn(x);
+    qw[size_t(qi) * kp + j] = h;
+    ss = fmaf(__half2float(h), __half2float(h), ss);
+  }
+  __syncthreads();
+  for (int i = tid; i < m; i += blockDim.x) {
+    float y = 0.f;
+    for (int j = 0; j < d; ++j) y = fmaf(Pt[j * m + i], sx[j], y);
+    const __half h = __float2half_rn(y);
+    qw[size_t(qi) * kp + d + i] = h;
+    s1 += fabsf(__half2float(h));
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+    s1 += __shfl_xor_sync(0xFFFFFFFFu, s1, o);
+  }
+  if ((tid & 31) == 0) {
+    red[tid >> 5] = ss;
+    red1[tid >> 5] = s1;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    float t = 0.f, t1 = 0.f;
+    for (int w = 0; w < int(blockDim.x / 32); ++w) {
+      t += red[w];
+      t1 += red1[w];
+    }
+    const float rq = sqrtf(t), kc = __uint_as_float(maxk_bits[0]), kw1 = __uint_as_float(maxk_bits[1]);
+    qerr[qi] = kErrRel * (kc * rq + kw1 * t1) + kErrAbs * (kc + float(m) * kw1 + rq + t1);
+  }
+}
+
+// Work unit u = (query tile u / row_tiles, row tile u % row_tiles); CTA b takes
+// units [units b / G, units (b + 1) / G).
+template <int KB>
+__global__ void __launch_bounds__(kSearchThreads, 1) search_tc_kernel(
+    const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap, int64_t nq, int64_t n,
+    int64_t row_tiles, int64_t units, int k, const float* __restrict__ qerr, uint32_t* __restrict__ cnt,
+    uint2* __restrict__ cand, uint32_t* __restrict__ status) {
+  using L = SearchSmem<KB>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* sbase = smem_raw + (base - raw);
+  const uint32_t bar0 = base + L::kOffBar;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sbase + L::kOffBar + 8 * kSNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + L::kOffBar + 8 * kSNumBars + 4);
+  auto bar = [&](int i) { return bar0 + 8u * uint32_t(i); };
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t u0 = units * blockIdx.x / gridDim.x, u1 = units * (blockIdx.x + 1) / gridDim.x;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(kSAFull), 1);
+    mbar_init(bar(kSAFree), 1);
+    for (int s = 0; s < kBStages; ++s) {
+      mbar_init(bar(kSBFull + s), 1);
+      mbar_init(bar(kSBEmpty + s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(kSDFull + s), 1);
+      mbar_init(bar(kSDEmpty + s), 128);
+    }
+    mbar_init(bar(kSDone), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(512));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int64_t qt_prev = -1, it = 0;
+      int na = 0;
+      bool ok = true;
+      for (int64_t u = u0; ok && u < u1; ++u) {
+        const int64_t qt = u / row_tiles, t = u - qt * row_tiles;
+        if (qt != qt_prev) {
+          // the MMAs that read the previous query tile have completed
+          if (na > 0 && !swait(bar(kSAFree), uint32_t((na - 1) & 1), abort_flag, status)) break;
+          mbar_expect_tx(bar(kSAFull), KB * 16384u);
+          for (int kb = 0; kb < KB; ++kb)
+            tma_load_2d(base + L::kOffA + 16384u * kb, &qmap, 64 * kb, int(qt * kQT), bar(kSAFull));
+          ++na;
+          qt_prev = qt;
+        }
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = int(it % kBStages);
+          if (it >= kBStages && !swait(bar(kSBEmpty + s), uint32_t((it / kBStages - 1) & 1), abort_flag, status)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(bar(kSBFull + s), 32768u);
+          tma_load_2d(base + L::kOffB + 32768u * s, &kmap, 64 * kb, int(t * kRT), bar(kSBFull + s));
+        }
+      }
+      // leave no copy in flight
+      for (int64_t j = (it >= kBStages ? it - kBStages : 0); j < it; ++j)
+        sdrain(bar(kSBFull + int(j % kBStages)), uint32_t((j / kBStages) & 1), abort_flag, status);
+      if (na > 0) sdrain(bar(kSAFull), uint32_t((na - 1) & 1), abort_flag, status);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      int64_t qt_prev = -1, it = 0, j = 0;
+      int na = 0;
+      bool ok = true;
+      for (int64_t u = u0; ok && u < u1; ++u, ++j) {
+        const int64_t qt = u / row_tiles;
+        if (qt != qt_prev) {
+          if (na > 0) mma_commit(bar(kSAFree));   // tracks every MMA on the previous query tile
+          if (!swait(bar(kSAFull), uint32_t(na & 1), abort_flag, status)) break;
+          ++na;
+          qt_prev = qt;
+        }
+        const int slot = int(j & 1);
+        if (j >= 2 && !swait(bar(kSDEmpty + slot), uint32_t(((j >> 1) - 1) & 1), abort_flag, status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + 256u * slot;
+        uint32_t acc = 0;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const int s = int(it % kBStages);
+          if (!swait(bar(kSBFull + s), uint32_t((it / kBStages) & 1), abort_flag, status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          for (int ks = 0; ks < 4; ++ks) {
+            mma_f16(d_tmem, smem_desc(base + L::kOffA + 16384u * kb + 32u * ks),
+                    smem_desc(base + L::kOffB + 32768u * s + 32u * ks), kIdescSearch, acc);
+            acc = 1;
+          }
+          mma_commit(bar(kSBEmpty + s));
+        }
+        if (!ok) break;
+        mma_commit(bar(kSDFull + slot));
+      }
+      // one more commit tracks every MMA issued, on every exit path
+      mma_commit(bar(kSDone));
+      sdrain(bar(kSDone), 0u, abort_flag, status);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    // thread = query row of the tile (TMEM lane (warp & 3) * 32 + lane).  The
+    // hot path is one compare per score into a 32-bit mask; the rare hits go
+    // through a short loop (code kept small: the MMA issuer shares the
+    // instruction cache).
+    const int row = (warp & 3) * 32 + lane;
+    const uint32_t lane_base = uint32_t((warp & 3) * 32) << 16;
+    int64_t qt_prev = -1, q = -1;
+    float E2 = 0.f, kth = -INFINITY;
+    float topv[kMaxK];     // the k best scores so far (unordered; dynamic index, local memory)
+    float vl[32];          // a chunk with hits
+    // candidates of the current tile, staged per thread (at most one per
+    // score) and appended with one atomic per tile
+    uint2 stage[kRT];
+    int64_t j = 0;
+    for (int64_t u = u0; u < u1; ++u, ++j) {
+      const int64_t qt = u / row_tiles, t = u - qt * row_tiles;
+      if (qt != qt_prev) {
+        qt_prev = qt;
+        q = qt * kQT + row;
+        E2 = q < nq ? 2.f * qerr[q] : 0.f;
+#pragma unroll 1
+        for (int i = 0; i < k; ++i) topv[i] = -INFINITY;
+        kth = -INFINITY;
+      }
+      const int slot = int(j & 1);
+      if (!swait_warp(bar(kSDFull + slot), uint32_t((j >> 1) & 1), abort_flag, status)) break;
+      tc_fence_after();
+      const int64_t r0 = t * kRT;
+      int ns = 0;
+#pragma unroll 1
+      for (int c = 0; c < kRT / 32; ++c) {
+        float v[32];
+        tmem_ld32(tmem + lane_base + 256u * slot + 32u * c, v);
+        tmem_wait32(v);
+        if (q >= nq) continue;
+        const float thr = kth - E2;
+        uint32_t mask = 0;
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) mask |= (v[jj] >= thr ? 1u : 0u) << jj;
+        const int64_t valid = n - (r0 + 32 * c);   // rows past n are padding
+        if (valid < 32) mask &= valid > 0 ? (1u << valid) - 1u : 0u;
+        if (mask == 0) continue;
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) vl[jj] = v[jj];
+#pragma unroll 1
+        while (mask) {
+          const int jj = __ffs(mask) - 1;
+          mask &= mask - 1;
+          const float a = vl[jj];
+          if (!(a >= kth - E2)) continue;   // kth may have risen within the chunk
+          stage[ns++] = make_uint2(__float_as_uint(a), uint32_t(r0 + 32 * c + jj));
+          if (a > kth) {
+            // replace one of the k kept scores equal to kth, then find the new smallest
+            int im = 0;
+#pragma unroll 1
+            for (int i = 0; i < k; ++i)
+              if (topv[i] == kth) {
+                im = i;
+                break;
+              }
+            topv[im] = a;
+            float mn = INFINITY;
+#pragma unroll 1
+            for (int i = 0; i < k; ++i) mn = fminf(mn, topv[i]);
+            kth = mn;
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(kSDEmpty + slot));
+      if (ns > 0) {
+        const uint32_t pos = atomicAdd(&cnt[q], uint32_t(ns));
+#pragma unroll 1
+        for (int i = 0; i < ns; ++i)
+          if (pos + uint32_t(i) < uint32_t(kCap)) cand[size_t(q) * kCap + pos + i] = stage[i];
+      }
+    }
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");   // none in flight on an early exit
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+  }
+}
+
+// Exact (fp64) estimate of one packed row against x = R q, y = P R q.
+__device__ double exact_score(const uint8_t* __restrict__ payload, const uint16_t* __restrict__ norms, int64_t row,
+                              const RowGeom& g, const double* __restrict__ c, const double* x, const double* y,
+                              double qc) {
+  const uint16_t* hw = reinterpret_cast<const uint16_t*>(payload + row * g.row_bytes);
+  double a = 0.0, b = 0.0;
+  for (int j = 0; j < g.d; ++j) a += c[unpack_code(hw, g, j)] * x[j];
+  for (int i = 0; i < g.m; ++i) b += unpack_sign(hw, g, i) ? y[i] : -y[i];
+  const double n16 = double(half_bits_to_float(norms[2 * row]));
+  const double r16 = double(half_bits_to_float(norms[2 * row + 1]));
+  return n16 * a + qc * r16 * b;
+}
+
+// (score descending, id ascending): true when (sa, ia) comes first
+__device__ __forceinline__ bool first(double sa, int64_t ia, double sb, int64_t ib) {
+  return sa > sb || (sa == sb && ia < ib);
+}
+
+constexpr int kFinishThreads = 512;
+
+// One block per query.  Shared memory: x (d) and y (m) in fp64, then kCap
+// (score, id) pairs for the sorts.
+__global__ void __launch_bounds__(kFinishThreads) finish_kernel(
+    const float* __restrict__ q, int d, int m, int bmse, int k, int64_t n, const uint8_t* __restrict__ payload,
+    const uint16_t* __restrict__ norms, const double* __restrict__ R, const double* __restrict__ P,
+    const double* __restrict__ c, const float* __restrict__ qerr, const uint32_t* __restrict__ cnt,
+    const uint2* __restrict__ cand, int64_t* __restrict__ ids, float* __restrict__ out_scores) {
+  extern __shared__ double smd[];
+  double* sx = smd;                 // d
+  double* sy = sx + 256;            // m
+  double* ssc = sy + 256;           // kCap scores
+  int64_t* sid = reinterpret_cast<int64_t*>(ssc + kCap);   // kCap ids
+  __shared__ double sq[256];
+  __shared__ int s_cut;
+  __shared__ double rs[kFinishThreads / 32];
+  __shared__ int64_t ri[kFinishThreads / 32];
+  __shared__ int rw[kFinishThreads / 32];
+  const int tid = threadIdx.x, nth = blockDim.x;
+  const int qi = blockIdx.x;
+  const RowGeom g = make_geom(d, m, bmse);
+  const double qc = kQjlConst / double(m);
+  for (int i = tid; i < d; i += nth) sq[i] = double(q[size_t(qi) * d + i]);
+  __syncthreads();
+  for (int j = tid; j < d; j += nth) {
+    double s = 0.0;
+    for (int i = 0; i < d; ++i) s += R[size_t(j) * d + i] * sq[i];
+    sx[j] = s;
+  }
+  __syncthreads();
+  for (int i = tid; i < m; i += nth) {
+    double s = 0.0;
+    for (int j = 0; j < d; ++j) s += P[size_t(i) * d + j] * sx[j];
+    sy[i] = s;
+  }
+  __syncthreads();
+  const uint32_t total = cnt[qi];
+  if (total > uint32_t(kCap)) {
+    // the candidate list overflowed: exact scan of every row.  Each thread
+    // keeps its best k in local memory; k rounds of a block-wide argmax.
+    double best_s[kMaxK];
+    int64_t best_i[kMaxK];
+    for (int i = 0; i < k; ++i) {
+      best_s[i] = -INFINITY;
+      best_i[i] = INT64_MAX;
+    }
+    for (int64_t r = tid; r < n; r += nth) {
+      const double s = exact_score(payload, norms, r, g, c, sx, sy, qc);
+      if (first(s, r, best_s[k - 1], best_i[k - 1])) {
+        int p = k - 1;
+        while (p > 0 && first(s, r, best_s[p - 1], best_i[p - 1])) {
+          best_s[p] = best_s[p - 1];
+          best_i[p] = best_i[p - 1];
+          --p;
+        }
+        best_s[p] = s;
+        best_i[p] = r;
+      }
+    }
+    int head = 0;
+    for (int out = 0; out < k; ++out) {
+      double s = head < k ? best_s[head] : -INFINITY;
+      int64_t id = head < k ? best_i[head] : INT64_MAX;
+      int who = tid;
+      for (int o = 16; o; o >>= 1) {
+        const double s2 = __shfl_xor_sync(0xFFFFFFFFu, s, o);
+        const int64_t i2 = __shfl_xor_sync(0xFFFFFFFFu, id, o);
+        const int w2 = __shfl_xor_sync(0xFFFFFFFFu, who, o);
+        if (first(s2, i2, s, id)) {
+          s = s2;
+          id = i2;
+          who = w2;
+        }
+      }
+      if ((tid & 31) == 0) {
+        rs[tid >> 5] = s;
+        ri[tid >> 5] = id;
+        rw[tid >> 5] = who;
+      }
+      __syncthreads();
+      if (tid == 0) {
+        for (int w = 1; w < nth / 32; ++w)
+          if (first(rs[w], ri[w], rs[0], ri[0])) {
+            rs[0] = rs[w];
+            ri[0] = ri[w];
+            rw[0] = rw[w];
+          }
+        ids[size_t(qi) * k + out] = ri[0];
+        out_scores[size_t(qi) * k + out] = float(rs[0]);
+      }
+      __syncthreads();
+      if (tid == rw[0]) ++head;
+      __syncthreads();
+    }
+    return;
+  }
+  // 1. candidates by approximate score, descending
+  const int cn = int(total);
+  int sp = 1;
+  while (sp < cn) sp <<= 1;
+  for (int i = tid; i < sp; i += nth) {
+    if (i < cn) {
+      const uint2 e = cand[size_t(qi) * kCap + i];
+      ssc[i] = double(__uint_as_float(e.x));
+      sid[i] = int64_t(e.y);
+    } else {
+      ssc[i] = -INFINITY;
+      sid[i] = INT64_MAX;
+    }
+  }
+  __syncthreads();
+  for (int size = 2; size <= sp; size <<= 1)
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = tid; i < sp; i += nth) {
+        const int jx = i ^ stride;
+        if (jx > i) {
+          const bool up = (i & size) == 0;
+          const bool i_first = first(ssc[i], sid[i], ssc[jx], sid[jx]);
+          if (up ? !i_first : i_first) {
+            const double ts = ssc[i];
+            ssc[i] = ssc[jx];
+            ssc[jx] = ts;
+            const int64_t ti = sid[i];
+            sid[i] = sid[jx];
+            sid[jx] = ti;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  // 2. keep the prefix within 2 E_q of the k-th approximate score
+  if (tid == 0) {
+    const int kk = cn < k ? cn : k;
+    const double cut = kk > 0 ? ssc[kk - 1] - 2.0 * double(qerr[qi]) : -INFINITY;
+    int mcut = kk;
+    while (mcut < cn && ssc[mcut] >= cut) ++mcut;
+    s_cut = mcut;
+  }
+  __syncthreads();
+  const int mc = s_cut;
+  // 3. exact scores of the kept candidates
+  for (int i = tid; i < mc; i += nth) ssc[i] = exact_score(payload, norms, sid[i], g, c, sx, sy, qc);
+  int sp2 = 1;
+  while (sp2 < mc) sp2 <<= 1;
+  for (int i = mc + tid; i < sp2; i += nth) {
+    ssc[i] = -INFINITY;
+    sid[i] = INT64_MAX;
+  }
+  __syncthreads();
+  for (int size = 2; size <= sp2; size <<= 1)
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = tid; i < sp2; i += nth) {
+        const int jx = i ^ stride;
+        if (jx > i) {
+          const bool up = (i & size) == 0;
+          const bool i_first = first(ssc[i], sid[i], ssc[jx], sid[jx]);
+          if (up ? !i_first : i_first) {
+            const double ts = ssc[i];
+            ssc[i] = ssc[jx];
+            ssc[jx] = ts;
+            const int64_t ti = sid[i];
+            sid[i] = sid[jx];
+            sid[jx] = ti;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  for (int i = tid; i < k; i += nth) {
+    ids[size_t(qi) * k + i] = i < mc ? sid[i] : INT64_MAX;
+    out_scores[size_t(qi) * k + i] = i < mc ? float(ssc[i]) : -INFINITY;
+  }
+}
+
+int key_blocks(const tq_ctx* ctx) { return (ctx->d + ctx->m + 63) / 64; }
+
+size_t align256(size_t b) { return (b + 255) / 256 * 256; }
+
+struct SearchWs {
+  __half* kw;
+  __half* qw;
+  float* qerr;
+  uint32_t* maxk;
+  uint32_t* cnt;
+  uint2* cand;
+  size_t kw_bytes, qw_bytes, total;
+};
+
+SearchWs search_ws(const tq_ctx* ctx, int64_t nq, int64_t n, void* base) {
+  const int kp = 64 * key_blocks(ctx);
+  const int64_t n_pad = (n + kRT - 1) / kRT * kRT, nq_pad = (nq + kQT - 1) / kQT * kQT;
+  SearchWs w{};
+  size_t off = 0;
+  uint8_t* b = static_cast<uint8_t*>(base);
+  auto take = [&](size_t bytes) {
+    uint8_t* p = b ? b + off : nullptr;
+    off += align256(bytes);
+    return p;
+  };
+  w.kw_bytes = size_t(n_pad) * kp * 2;
+  w.qw_bytes = size_t(nq_pad) * kp * 2;
+  w.kw = reinterpret_cast<__half*>(take(w.kw_bytes));
+  w.qw = reinterpret_cast<__half*>(take(w.qw_bytes));
+  w.qerr = reinterpret_cast<float*>(take(size_t(nq_pad) * 4));
+  w.maxk = reinterpret_cast<uint32_t*>(take(8));
+  w.cnt = reinterpret_cast<uint32_t*>(take(size_t(nq_pad) * 4));
+  w.cand = reinterpret_cast<uint2*>(take(size_t(nq) * kCap * 8));
+  w.total = off;
+  return w;
+}
+
+template <int KB>
+cudaError_t launch_search_kernel(const CUtensorMap& qmap, const CUtensorMap& kmap, int64_t nq, int64_t n,
+                                 int64_t row_tiles, int64_t units, int k, const SearchWs& w, uint32_t* status,
+                                 cudaStream_t st) {
+  using L = SearchSmem<KB>;
+  static_assert(L::kBytes <= 232448, "shared memory per block");
+  auto kern = search_tc_kernel<KB>;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(L::kBytes));
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = int(units < sms ? units : sms);
+  kern<<<grid, kSearchThreads, L::kBytes, st>>>(qmap, kmap, nq, n, row_tiles, units, k, w.qerr, w.cnt, w.cand,
+                                                status);
+  return cudaGetLastError();
+}
+
+bool encode_fp16_map(CUtensorMap* map, const void* ptr, int kp, int64_t rows, uint32_t box_rows) {
+  const cuuint64_t dims[2] = {cuuint64_t(kp), cuuint64_t(rows)};
+  const cuuint64_t strides[1] = {cuuint64_t(kp) * 2};
+  const cuuint32_t box[2] = {64u, box_rows};
+  const cuuint32_t estr[2] = {1u, 1u};
+  return get_encode()(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool search_tc_supported(const tq_ctx* ctx, int64_t nq, int64_t n, int k) {
+  const int kb = key_blocks(ctx);
+  return k >= 1 && k <= kMaxK && kb >= 1 && kb <= 8 && n >= 1 && n < (int64_t(1) << 31) && nq >= 1 &&
+         device_is_sm100() && get_encode() != nullptr;
+}
+
+size_t search_ws_bytes(const tq_ctx* ctx, int64_t nq, int64_t n) { return search_ws(ctx, nq, n, nullptr).total; }
+
+cudaError_t launch_search_tc(const tq_ctx* ctx, const float* q, int64_t nq, const uint8_t* payload,
+                             const uint16_t* norms, int64_t n, int k, int64_t* ids, float* scores, void* ws,
+                             cudaStream_t st) {
+  const int kb = key_blocks(ctx), kp = 64 * kb;
+  const int64_t n_pad = (n + kRT - 1) / kRT * kRT, nq_pad = (nq + kQT - 1) / kQT * kQT;
+  const SearchWs w = search_ws(ctx, nq, n, ws);
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(w.qw, 0, w.qw_bytes, st)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(w.maxk, 0, 8, st)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(w.cnt, 0, size_t(nq_pad) * 4, st)) != cudaSuccess) return e;
+  const int64_t warps = n_pad;
+  decode_rows_kernel<<<unsigned((warps * 32 + 255) / 256), 256, 0, st>>>(
+      payload, norms, n, n_pad, ctx->d, ctx->m, ctx->bmse, kp, ctx->cb, w.kw, w.maxk);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  prep_queries_kernel<<<unsigned(nq), 256, 0, st>>>(q, ctx->dRt, ctx->dPt, ctx->d, ctx->m, kp, w.maxk, w.qw,
+                                                     w.qerr);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  CUtensorMap qmap, kmap;
+  if (!encode_fp16_map(&qmap, w.qw, kp, nq_pad, kQT) || !encode_fp16_map(&kmap, w.kw, kp, n_pad, kRT))
+    return cudaErrorInvalidValue;
+  const int64_t row_tiles = n_pad / kRT, units = (nq_pad / kQT) * row_tiles;
+  switch (kb) {
+    case 1: e = launch_search_kernel<1>(qmap, kmap, nq, n, row_tiles, units, k, w, ctx->dstatus, st); break;
+    case 2: e = launch_search_kernel<2>(qmap, kmap, nq, n, row_tiles, units, k, w, ctx->dstatus, st); break;
+    case 3: e = launch_search_kernel<3>(qmap, kmap, nq, n, row_tiles, units, k, w, ctx->dstatus, st); break;
+    case 4: e = launch_search_kernel<4>(qmap, kmap, nq, n, row_tiles, units, k, w, ctx->dstatus, st); break;
+    case 5: e = launch_search_kernel<5>(qmap, kmap, nq, n, row_tiles, units, k, w, ctx->dstatus, st); break;
+    case 6: e = launch_search_kernel<6>(qmap, kmap, nq, n, row_tiles, units, k, w, ctx->dstatus, st); break;
+    case 7: e = launch_search_kernel<7>(qmap, kmap, nq, n, row_tiles, units, k, w, ctx->dstatus, st); break;
+    default: e = launch_search_kernel<8>(qmap, kmap, nq, n, row_tiles, units, k, w, ctx->dstatus, st); break;
+  }
+  if (e != cudaSuccess) return e;
+  const size_t fsmem = size_t(2 * 256 + kCap) * 8 + size_t(kCap) * 8;
+  cudaFuncSetAttribute(finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(fsmem));
+  finish_kernel<<<unsigned(nq), kFinishThreads, fsmem, st>>>(q, ctx->d, ctx->m, ctx->bmse, k, n, payload, norms,
+                                                             ctx->dR64, ctx->dP64, ctx->dc64, w.qerr, w.cnt, w.cand,
+                                                             ids, scores);
+  return cudaGetLastError();
+}
+
+}  // namespace tq

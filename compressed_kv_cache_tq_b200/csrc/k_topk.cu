@@ -1,7 +1,8 @@
 // Inner-product top-k over a packed database (vector search; airosetta.com
 // "Google TurboQuant" names GloVe recall@1@k with near-zero indexing time).
 //
-// Three kernels per block of queries:
+// The tensor-core path (k_search_tc.cu) serves sm_100a and k <= 32; this file
+// is the general path.  Three kernels per block of queries:
 //   1. estimator scores for all (query, row) pairs (the logits kernels with
 //      scale 1, one "KV head" holding the whole database);
 //   2. per query, an exact radix select of the KC-th largest fp32 score and a
@@ -175,7 +176,7 @@ int64_t query_block(int64_t nq, int64_t n) {
 }  // namespace
 
 size_t topk_ws_bytes(const tq_ctx* ctx, int64_t nq, int64_t n, int k) {
-  (void)ctx;
+  if (search_tc_supported(ctx, nq, n, k)) return search_ws_bytes(ctx, nq, n);
   const int64_t qb = query_block(nq, n);
   const int kc = candidates(n, k);
   const size_t scores = ((size_t(qb) * n * 4 + 255) / 256) * 256;
@@ -187,6 +188,9 @@ size_t topk_ws_bytes(const tq_ctx* ctx, int64_t nq, int64_t n, int k) {
 cudaError_t launch_topk(const tq_ctx* ctx, const float* q, int64_t nq, const uint8_t* payload,
                         const uint16_t* norms, int64_t n, int k, int64_t* ids, float* scores, void* ws,
                         cudaStream_t st) {
+  // tensor-core scoring with exact re-scoring of the candidates (sm_100a, k <= 32)
+  if (search_tc_supported(ctx, nq, n, k))
+    return launch_search_tc(ctx, q, nq, payload, norms, n, k, ids, scores, ws, st);
   const int64_t qb = query_block(nq, n);
   const int kc = candidates(n, k);
   const int sp = pow2_at_least(kc);

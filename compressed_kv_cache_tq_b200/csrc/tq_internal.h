@@ -55,6 +55,7 @@ namespace tq {
 
 // Device status bits (set by bounded waits that gave up).
 constexpr uint32_t kStatusQuantizeTc = 1u << 0;
+constexpr uint32_t kStatusSearchTc = 1u << 1;
 
 void set_cuda_error(cudaError_t e);
 
@@ -72,6 +73,11 @@ cudaError_t launch_logits(const tq_ctx* ctx, const float* q, int B, int Hq, int 
                           const uint8_t* payload, const uint16_t* norms, float scale, float* out,
                           void* ws, cudaStream_t st);
 size_t topk_ws_bytes(const tq_ctx* ctx, int64_t nq, int64_t n, int k);
+bool search_tc_supported(const tq_ctx* ctx, int64_t nq, int64_t n, int k);
+size_t search_ws_bytes(const tq_ctx* ctx, int64_t nq, int64_t n);
+cudaError_t launch_search_tc(const tq_ctx* ctx, const float* q, int64_t nq, const uint8_t* payload,
+                             const uint16_t* norms, int64_t n, int k, int64_t* ids, float* scores, void* ws,
+                             cudaStream_t st);
 cudaError_t launch_topk(const tq_ctx* ctx, const float* q, int64_t nq, const uint8_t* payload,
                         const uint16_t* norms, int64_t n, int k, int64_t* ids, float* scores, void* ws,
                         cudaStream_t st);

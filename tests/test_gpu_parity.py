@@ -229,6 +229,46 @@ def test_topk_against_oracle(lib, d, bits, n, nq, k):
                                atol=1e-6 * A.max())
 
 
+@pytest.mark.parametrize("d,bits", [(200, 2), (128, 4)])
+def test_topk_many_query_tiles(lib, d, bits):
+    """More (query tile, row tile) units than SMs: CTAs switch query tiles
+    inside their range of the tensor-core search."""
+    ctx = _ctx(lib, d=d, bits=bits, seed=19)
+    n, nq, k = 20000, 500, 10
+    db = W.search_vectors(n, d, seed=300 + bits, which=0)
+    qs = W.search_vectors(nq, d, seed=300 + bits, which=1)
+    payload, norms = lib.tq_quantize(ctx, torch.from_numpy(db).to(DEV))
+    ids, scores = lib.tq_topk(ctx, torch.from_numpy(qs).to(DEV), payload, norms, k)
+    _status_clean(lib, ctx)
+    s, A = oracle_estimates(payload.cpu().numpy(), norms.cpu().numpy(), qs.astype(np.float64), tables_of(ctx))
+    ids = ids.cpu().numpy()
+    near_tie = 0
+    for i in range(nq):
+        order = np.lexsort((np.arange(n), -s[i]))[:k + 1]
+        if s[i, order[k - 1]] - s[i, order[k]] < 1e-6 * A[i].max():
+            near_tie += 1
+            assert set(ids[i][:k - 1]) <= set(order)
+            continue
+        np.testing.assert_array_equal(ids[i], order[:k])
+    assert near_tie <= nq // 20
+    np.testing.assert_allclose(scores.cpu().numpy(), np.take_along_axis(s, ids, 1), rtol=1e-6, atol=1e-6 * A.max())
+
+
+def test_topk_identical_rows_take_lowest_ids(lib):
+    """3000 copies of one vector: every row ties, the candidate list overflows
+    and the exact scan returns ids 0 .. k-1 (ties go to the lower id)."""
+    ctx = _ctx(lib, d=200, bits=4, seed=3)
+    v = W.search_vectors(1, 200, seed=9, which=0)
+    db = np.repeat(v, 3000, axis=0)
+    qs = W.search_vectors(4, 200, seed=9, which=1)
+    payload, norms = lib.tq_quantize(ctx, torch.from_numpy(db).to(DEV))
+    ids, scores = lib.tq_topk(ctx, torch.from_numpy(qs).to(DEV), payload, norms, 10)
+    _status_clean(lib, ctx)
+    np.testing.assert_array_equal(ids.cpu().numpy(), np.tile(np.arange(10), (4, 1)))
+    s, A = oracle_estimates(payload.cpu().numpy()[:1], norms.cpu().numpy()[:1], qs.astype(np.float64), tables_of(ctx))
+    np.testing.assert_allclose(scores.cpu().numpy(), np.repeat(s, 10, axis=1), rtol=1e-6, atol=1e-6 * A.max())
+
+
 def test_logits_rejects_bad_workspace(lib):
     ctx = _ctx(lib, bits=3, seed=1)
     payload, norms = _cache(lib, ctx, 1, 1, 64, seed=1)
