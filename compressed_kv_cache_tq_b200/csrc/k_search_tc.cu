@@ -13,15 +13,19 @@
 //      memory) against 256-row tiles (TMA ring), scores in TMEM; the epilogue
 //      keeps each query's running k best scores and appends every row whose
 //      score is at least (k-th best - 2 E_q) to the query's candidate list.
-//   4. finish_kernel: per query, the candidates sorted by approximate score and
-//      cut at (k-th approximate - 2 E_q), re-scored exactly in fp64 and ordered
-//      by (score descending, id ascending); the first k are the answer.
+//   4. query_tables_kernel (x = Rq, y = Sq in fp64) and finish_kernel: per
+//      query, the k-th largest approximate score among the candidates (by
+//      bisection), the candidates within 2 E_q of it re-scored exactly in fp64
+//      and ordered by (score descending, id ascending); the first k are the
+//      answer.
 // Completeness: every approximate score is within E_q of the exact one.  The
 // k-th largest approximate score A_k is then at most T + E_q (T: the exact
 // k-th largest; otherwise k rows would have exact scores above T), and every
 // row of the exact top k has approximate score >= T - E_q >= A_k - 2 E_q, so
 // it is a candidate.  A CTA that scans only part of the rows uses its own,
-// lower, A_k: its cut keeps a superset.  A query whose candidate list
+// lower, A_k: its cut keeps a superset.  Segments of the same query share the
+// largest local A_k published so far (each is at most the global one, so the
+// argument holds for their maximum).  A query whose candidate list
 // overflows is answered by an exact scan of all rows in the finishing kernel.
 // Error bound: Kw and Qw are rounded to fp16 (relative 2^-11 each) after fp32
 // arithmetic (R q and P R q in fp32: relative error below 2e-4 of ||Kw|| ||q||
@@ -179,12 +183,43 @@ __global__ void __launch_bounds__(256) prep_queries_kernel(const float* __restri
   }
 }
 
-// Work unit u = (query tile u / row_tiles, row tile u % row_tiles); CTA b takes
-// units [units b / G, units (b + 1) / G).
+// float -> uint32 with the same order
+__device__ __forceinline__ uint32_t order_key(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_float(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+// Work: unit u = (query tile u / row_tiles, row tile u % row_tiles); CTA b
+// takes the contiguous units [U b / G, U (b + 1) / G) of the U = qtiles x
+// row_tiles, so it keeps one query tile (or two) for long stretches.  (A
+// part-major round-robin order that makes all CTAs stream the same rows at
+// the same time measured slower: 17.0 against 13.7 ms at 10^6 x 10^4.)
+struct Units {
+  int64_t row_tiles, u, u1;
+  int64_t qt, t;
+  __device__ Units(int64_t qtiles, int64_t row_tiles_, int64_t cta, int64_t ctas) : row_tiles(row_tiles_) {
+    const int64_t total = qtiles * row_tiles_;
+    u = total * cta / ctas - 1;
+    u1 = total * (cta + 1) / ctas;
+    qt = t = 0;
+  }
+  // advance to the next (query tile, row tile); false when done
+  __device__ bool next() {
+    if (++u >= u1) return false;
+    qt = u / row_tiles;
+    t = u - qt * row_tiles;
+    return true;
+  }
+};
+
 template <int KB>
 __global__ void __launch_bounds__(kSearchThreads, 1) search_tc_kernel(
     const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap, int64_t nq, int64_t n,
-    int64_t row_tiles, int64_t units, int k, const float* __restrict__ qerr, uint32_t* __restrict__ cnt,
+    int64_t qtiles, int64_t row_tiles, int k, const float* __restrict__ qerr,
+    uint32_t* __restrict__ gkth, uint32_t* __restrict__ cnt,
     uint2* __restrict__ cand, uint32_t* __restrict__ status) {
   using L = SearchSmem<KB>;
   extern __shared__ uint8_t smem_raw[];
@@ -196,7 +231,6 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_tc_kernel(
   volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + L::kOffBar + 8 * kSNumBars + 4);
   auto bar = [&](int i) { return bar0 + 8u * uint32_t(i); };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t u0 = units * blockIdx.x / gridDim.x, u1 = units * (blockIdx.x + 1) / gridDim.x;
 
   if (threadIdx.x == 0) {
     mbar_init(bar(kSAFull), 1);
@@ -230,8 +264,9 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_tc_kernel(
       int64_t qt_prev = -1, it = 0;
       int na = 0;
       bool ok = true;
-      for (int64_t u = u0; ok && u < u1; ++u) {
-        const int64_t qt = u / row_tiles, t = u - qt * row_tiles;
+      Units w(qtiles, row_tiles, blockIdx.x, gridDim.x);
+      while (ok && w.next()) {
+        const int64_t qt = w.qt, t = w.t;
         if (qt != qt_prev) {
           // the MMAs that read the previous query tile have completed
           if (na > 0 && !swait(bar(kSAFree), uint32_t((na - 1) & 1), abort_flag, status)) break;
@@ -262,8 +297,9 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_tc_kernel(
       int64_t qt_prev = -1, it = 0, j = 0;
       int na = 0;
       bool ok = true;
-      for (int64_t u = u0; ok && u < u1; ++u, ++j) {
-        const int64_t qt = u / row_tiles;
+      Units w(qtiles, row_tiles, blockIdx.x, gridDim.x);
+      for (; ok && w.next(); ++j) {
+        const int64_t qt = w.qt;
         if (qt != qt_prev) {
           if (na > 0) mma_commit(bar(kSAFree));   // tracks every MMA on the previous query tile
           if (!swait(bar(kSAFull), uint32_t(na & 1), abort_flag, status)) break;
@@ -312,8 +348,9 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_tc_kernel(
     // score) and appended with one atomic per tile
     uint2 stage[kRT];
     int64_t j = 0;
-    for (int64_t u = u0; u < u1; ++u, ++j) {
-      const int64_t qt = u / row_tiles, t = u - qt * row_tiles;
+    Units w(qtiles, row_tiles, blockIdx.x, gridDim.x);
+    for (; w.next(); ++j) {
+      const int64_t qt = w.qt, t = w.t;
       if (qt != qt_prev) {
         qt_prev = qt;
         q = qt * kQT + row;
@@ -327,13 +364,19 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_tc_kernel(
       tc_fence_after();
       const int64_t r0 = t * kRT;
       int ns = 0;
+      // the best k-th score any segment of this query has published (0: none)
+      float gk = -INFINITY;
+      if (q < nq) {
+        const uint32_t gkey = *reinterpret_cast<volatile uint32_t*>(gkth + q);
+        if (gkey) gk = key_float(gkey);
+      }
 #pragma unroll 1
       for (int c = 0; c < kRT / 32; ++c) {
         float v[32];
         tmem_ld32(tmem + lane_base + 256u * slot + 32u * c, v);
         tmem_wait32(v);
         if (q >= nq) continue;
-        const float thr = kth - E2;
+        const float thr = fmaxf(kth, gk) - E2;
         uint32_t mask = 0;
 #pragma unroll
         for (int jj = 0; jj < 32; ++jj) mask |= (v[jj] >= thr ? 1u : 0u) << jj;
@@ -347,7 +390,7 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_tc_kernel(
           const int jj = __ffs(mask) - 1;
           mask &= mask - 1;
           const float a = vl[jj];
-          if (!(a >= kth - E2)) continue;   // kth may have risen within the chunk
+          if (!(a >= fmaxf(kth, gk) - E2)) continue;   // kth may have risen within the chunk
           stage[ns++] = make_uint2(__float_as_uint(a), uint32_t(r0 + 32 * c + jj));
           if (a > kth) {
             // replace one of the k kept scores equal to kth, then find the new smallest
@@ -368,6 +411,7 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_tc_kernel(
       }
       tc_fence_before();
       mbar_arrive(bar(kSDEmpty + slot));
+      if (q < nq && kth > gk) atomicMax(gkth + q, order_key(kth));   // publish this segment's k-th best
       if (ns > 0) {
         const uint32_t pos = atomicAdd(&cnt[q], uint32_t(ns));
 #pragma unroll 1
@@ -403,42 +447,91 @@ __device__ __forceinline__ bool first(double sa, int64_t ia, double sb, int64_t 
   return sa > sb || (sa == sb && ia < ib);
 }
 
-constexpr int kFinishThreads = 512;
+constexpr int kFinishThreads = 256;
+constexpr int kTabQueries = 8;      // queries per block of query_tables_kernel
+
+// x = R q and y = P x in fp64 for kTabQueries queries per block (the tables
+// are read once per block): xy[q] = [x (d), y (m)].
+__global__ void __launch_bounds__(256) query_tables_kernel(const float* __restrict__ q, int64_t nq, int d, int m,
+                                                           const double* __restrict__ R,
+                                                           const double* __restrict__ P,
+                                                           double* __restrict__ xy) {
+  __shared__ double sq[kTabQueries][256];
+  __shared__ double sx[kTabQueries][256];
+  const int64_t q0 = int64_t(blockIdx.x) * kTabQueries;
+  const int nb = int(nq - q0 < kTabQueries ? nq - q0 : kTabQueries);
+  const int tid = threadIdx.x;
+  for (int idx = tid; idx < kTabQueries * d; idx += blockDim.x) {
+    const int qq = idx / d, i = idx - qq * d;
+    sq[qq][i] = qq < nb ? double(q[(q0 + qq) * d + i]) : 0.0;
+  }
+  __syncthreads();
+  for (int j = tid; j < d; j += blockDim.x) {
+    double acc[kTabQueries];
+#pragma unroll
+    for (int qq = 0; qq < kTabQueries; ++qq) acc[qq] = 0.0;
+    for (int i = 0; i < d; ++i) {
+      const double r = R[size_t(j) * d + i];
+#pragma unroll
+      for (int qq = 0; qq < kTabQueries; ++qq) acc[qq] += r * sq[qq][i];
+    }
+#pragma unroll
+    for (int qq = 0; qq < kTabQueries; ++qq) {
+      sx[qq][j] = acc[qq];
+      if (qq < nb) xy[(q0 + qq) * (d + m) + j] = acc[qq];
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < m; i += blockDim.x) {
+    double acc[kTabQueries];
+#pragma unroll
+    for (int qq = 0; qq < kTabQueries; ++qq) acc[qq] = 0.0;
+    for (int j = 0; j < d; ++j) {
+      const double pv = P[size_t(i) * d + j];
+#pragma unroll
+      for (int qq = 0; qq < kTabQueries; ++qq) acc[qq] += pv * sx[qq][j];
+    }
+#pragma unroll
+    for (int qq = 0; qq < kTabQueries; ++qq)
+      if (qq < nb) xy[(q0 + qq) * (d + m) + d + i] = acc[qq];
+  }
+}
+
+// Block-wide sum of one int per thread.
+__device__ __forceinline__ int block_sum(int v, int* red) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  const int w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red[w] = v;
+  __syncthreads();
+  int t = 0;
+  for (int i = 0; i < nw; ++i) t += red[i];
+  return t;
+}
 
 // One block per query.  Shared memory: x (d) and y (m) in fp64, then kCap
-// (score, id) pairs for the sorts.
+// (score, id) pairs for the final sort.
 __global__ void __launch_bounds__(kFinishThreads) finish_kernel(
-    const float* __restrict__ q, int d, int m, int bmse, int k, int64_t n, const uint8_t* __restrict__ payload,
-    const uint16_t* __restrict__ norms, const double* __restrict__ R, const double* __restrict__ P,
-    const double* __restrict__ c, const float* __restrict__ qerr, const uint32_t* __restrict__ cnt,
-    const uint2* __restrict__ cand, int64_t* __restrict__ ids, float* __restrict__ out_scores) {
+    int d, int m, int bmse, int k, int64_t n, const uint8_t* __restrict__ payload,
+    const uint16_t* __restrict__ norms, const double* __restrict__ xy, const double* __restrict__ c,
+    const float* __restrict__ qerr, const uint32_t* __restrict__ cnt, const uint2* __restrict__ cand,
+    int64_t* __restrict__ ids, float* __restrict__ out_scores) {
   extern __shared__ double smd[];
   double* sx = smd;                 // d
   double* sy = sx + 256;            // m
   double* ssc = sy + 256;           // kCap scores
   int64_t* sid = reinterpret_cast<int64_t*>(ssc + kCap);   // kCap ids
-  __shared__ double sq[256];
-  __shared__ int s_cut;
+  __shared__ int red[kFinishThreads / 32];
   __shared__ double rs[kFinishThreads / 32];
   __shared__ int64_t ri[kFinishThreads / 32];
   __shared__ int rw[kFinishThreads / 32];
+  __shared__ int s_mc;
   const int tid = threadIdx.x, nth = blockDim.x;
   const int qi = blockIdx.x;
   const RowGeom g = make_geom(d, m, bmse);
   const double qc = kQjlConst / double(m);
-  for (int i = tid; i < d; i += nth) sq[i] = double(q[size_t(qi) * d + i]);
-  __syncthreads();
-  for (int j = tid; j < d; j += nth) {
-    double s = 0.0;
-    for (int i = 0; i < d; ++i) s += R[size_t(j) * d + i] * sq[i];
-    sx[j] = s;
-  }
-  __syncthreads();
-  for (int i = tid; i < m; i += nth) {
-    double s = 0.0;
-    for (int j = 0; j < d; ++j) s += P[size_t(i) * d + j] * sx[j];
-    sy[i] = s;
-  }
+  for (int i = tid; i < d + m; i += nth) (i < d ? sx[i] : sy[i - d]) = xy[size_t(qi) * (d + m) + i];
   __syncthreads();
   const uint32_t total = cnt[qi];
   if (total > uint32_t(kCap)) {
@@ -451,35 +544,35 @@ __global__ void __launch_bounds__(kFinishThreads) finish_kernel(
       best_i[i] = INT64_MAX;
     }
     for (int64_t r = tid; r < n; r += nth) {
-      const double s = exact_score(payload, norms, r, g, c, sx, sy, qc);
-      if (first(s, r, best_s[k - 1], best_i[k - 1])) {
+      const double sc = exact_score(payload, norms, r, g, c, sx, sy, qc);
+      if (first(sc, r, best_s[k - 1], best_i[k - 1])) {
         int p = k - 1;
-        while (p > 0 && first(s, r, best_s[p - 1], best_i[p - 1])) {
+        while (p > 0 && first(sc, r, best_s[p - 1], best_i[p - 1])) {
           best_s[p] = best_s[p - 1];
           best_i[p] = best_i[p - 1];
           --p;
         }
-        best_s[p] = s;
+        best_s[p] = sc;
         best_i[p] = r;
       }
     }
     int head = 0;
     for (int out = 0; out < k; ++out) {
-      double s = head < k ? best_s[head] : -INFINITY;
+      double sc = head < k ? best_s[head] : -INFINITY;
       int64_t id = head < k ? best_i[head] : INT64_MAX;
       int who = tid;
       for (int o = 16; o; o >>= 1) {
-        const double s2 = __shfl_xor_sync(0xFFFFFFFFu, s, o);
+        const double s2 = __shfl_xor_sync(0xFFFFFFFFu, sc, o);
         const int64_t i2 = __shfl_xor_sync(0xFFFFFFFFu, id, o);
         const int w2 = __shfl_xor_sync(0xFFFFFFFFu, who, o);
-        if (first(s2, i2, s, id)) {
-          s = s2;
+        if (first(s2, i2, sc, id)) {
+          sc = s2;
           id = i2;
           who = w2;
         }
       }
       if ((tid & 31) == 0) {
-        rs[tid >> 5] = s;
+        rs[tid >> 5] = sc;
         ri[tid >> 5] = id;
         rw[tid >> 5] = who;
       }
@@ -500,51 +593,39 @@ __global__ void __launch_bounds__(kFinishThreads) finish_kernel(
     }
     return;
   }
-  // 1. candidates by approximate score, descending
+  // 1. the k-th largest approximate score, by bisection over the order keys
+  constexpr int kPer = kCap / kFinishThreads;
   const int cn = int(total);
-  int sp = 1;
-  while (sp < cn) sp <<= 1;
-  for (int i = tid; i < sp; i += nth) {
-    if (i < cn) {
-      const uint2 e = cand[size_t(qi) * kCap + i];
-      ssc[i] = double(__uint_as_float(e.x));
-      sid[i] = int64_t(e.y);
-    } else {
-      ssc[i] = -INFINITY;
-      sid[i] = INT64_MAX;
+  uint32_t key[kPer];
+#pragma unroll
+  for (int t = 0; t < kPer; ++t) {
+    const int i = tid + t * nth;
+    key[t] = i < cn ? order_key(__uint_as_float(cand[size_t(qi) * kCap + i].x)) : 0u;
+  }
+  const int kk = cn < k ? cn : k;
+  uint32_t T = 0;
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t trial = T | (1u << bit);
+    int ge = 0;
+#pragma unroll
+    for (int t = 0; t < kPer; ++t) ge += (key[t] >= trial) ? 1 : 0;
+    if (block_sum(ge, red) >= kk) T = trial;
+  }
+  // 2. keep the candidates within 2 E_q of it
+  const float cutf = kk > 0 ? key_float(T) - 2.f * qerr[qi] : -INFINITY;
+  if (tid == 0) s_mc = 0;
+  __syncthreads();
+#pragma unroll
+  for (int t = 0; t < kPer; ++t) {
+    const int i = tid + t * nth;
+    if (i < cn && key_float(key[t]) >= cutf) {
+      const int slot = atomicAdd(&s_mc, 1);
+      sid[slot] = int64_t(cand[size_t(qi) * kCap + i].y);
     }
   }
   __syncthreads();
-  for (int size = 2; size <= sp; size <<= 1)
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = tid; i < sp; i += nth) {
-        const int jx = i ^ stride;
-        if (jx > i) {
-          const bool up = (i & size) == 0;
-          const bool i_first = first(ssc[i], sid[i], ssc[jx], sid[jx]);
-          if (up ? !i_first : i_first) {
-            const double ts = ssc[i];
-            ssc[i] = ssc[jx];
-            ssc[jx] = ts;
-            const int64_t ti = sid[i];
-            sid[i] = sid[jx];
-            sid[jx] = ti;
-          }
-        }
-      }
-      __syncthreads();
-    }
-  // 2. keep the prefix within 2 E_q of the k-th approximate score
-  if (tid == 0) {
-    const int kk = cn < k ? cn : k;
-    const double cut = kk > 0 ? ssc[kk - 1] - 2.0 * double(qerr[qi]) : -INFINITY;
-    int mcut = kk;
-    while (mcut < cn && ssc[mcut] >= cut) ++mcut;
-    s_cut = mcut;
-  }
-  __syncthreads();
-  const int mc = s_cut;
-  // 3. exact scores of the kept candidates
+  const int mc = s_mc;
+  // 3. exact scores, then (score descending, id ascending)
   for (int i = tid; i < mc; i += nth) ssc[i] = exact_score(payload, norms, sid[i], g, c, sx, sy, qc);
   int sp2 = 1;
   while (sp2 < mc) sp2 <<= 1;
@@ -588,7 +669,9 @@ struct SearchWs {
   float* qerr;
   uint32_t* maxk;
   uint32_t* cnt;
+  uint32_t* gkth;
   uint2* cand;
+  double* xy;
   size_t kw_bytes, qw_bytes, total;
 };
 
@@ -610,14 +693,16 @@ SearchWs search_ws(const tq_ctx* ctx, int64_t nq, int64_t n, void* base) {
   w.qerr = reinterpret_cast<float*>(take(size_t(nq_pad) * 4));
   w.maxk = reinterpret_cast<uint32_t*>(take(8));
   w.cnt = reinterpret_cast<uint32_t*>(take(size_t(nq_pad) * 4));
+  w.gkth = reinterpret_cast<uint32_t*>(take(size_t(nq_pad) * 4));
   w.cand = reinterpret_cast<uint2*>(take(size_t(nq) * kCap * 8));
+  w.xy = reinterpret_cast<double*>(take(size_t(nq) * (ctx->d + ctx->m) * 8));
   w.total = off;
   return w;
 }
 
 template <int KB>
 cudaError_t launch_search_kernel(const CUtensorMap& qmap, const CUtensorMap& kmap, int64_t nq, int64_t n,
-                                 int64_t row_tiles, int64_t units, int k, const SearchWs& w, uint32_t* status,
+                                 int64_t qtiles, int64_t row_tiles, int k, const SearchWs& w, uint32_t* status,
                                  cudaStream_t st) {
   using L = SearchSmem<KB>;
   static_assert(L::kBytes <= 232448, "shared memory per block");
@@ -626,9 +711,10 @@ cudaError_t launch_search_kernel(const CUtensorMap& qmap, const CUtensorMap& kma
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t units = qtiles * row_tiles;
   const int grid = int(units < sms ? units : sms);
-  kern<<<grid, kSearchThreads, L::kBytes, st>>>(qmap, kmap, nq, n, row_tiles, units, k, w.qerr, w.cnt, w.cand,
-                                                status);
+  kern<<<grid, kSearchThreads, L::kBytes, st>>>(qmap, kmap, nq, n, qtiles, row_tiles, k, w.qerr, w.gkth, w.cnt,
+                                                w.cand, status);
   return cudaGetLastError();
 }
 
@@ -662,6 +748,7 @@ cudaError_t launch_search_tc(const tq_ctx* ctx, const float* q, int64_t nq, cons
   if ((e = cudaMemsetAsync(w.qw, 0, w.qw_bytes, st)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(w.maxk, 0, 8, st)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(w.cnt, 0, size_t(nq_pad) * 4, st)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(w.gkth, 0, size_t(nq_pad) * 4, st)) != cudaSuccess) return e;
   const int64_t warps = n_pad;
   decode_rows_kernel<<<unsigned((warps * 32 + 255) / 256), 256, 0, st>>>(
       payload, norms, n, n_pad, ctx->d, ctx->m, ctx->bmse, kp, ctx->cb, w.kw, w.maxk);
@@ -672,23 +759,25 @@ cudaError_t launch_search_tc(const tq_ctx* ctx, const float* q, int64_t nq, cons
   CUtensorMap qmap, kmap;
   if (!encode_fp16_map(&qmap, w.qw, kp, nq_pad, kQT) || !encode_fp16_map(&kmap, w.kw, kp, n_pad, kRT))
     return cudaErrorInvalidValue;
-  const int64_t row_tiles = n_pad / kRT, units = (nq_pad / kQT) * row_tiles;
+  const int64_t row_tiles = n_pad / kRT, qtiles = nq_pad / kQT;
   switch (kb) {
-    case 1: e = launch_search_kernel<1>(qmap, kmap, nq, n, row_tiles, units, k, w, ctx->dstatus, st); break;
-    case 2: e = launch_search_kernel<2>(qmap, kmap, nq, n, row_tiles, units, k, w, ctx->dstatus, st); break;
-    case 3: e = launch_search_kernel<3>(qmap, kmap, nq, n, row_tiles, units, k, w, ctx->dstatus, st); break;
-    case 4: e = launch_search_kernel<4>(qmap, kmap, nq, n, row_tiles, units, k, w, ctx->dstatus, st); break;
-    case 5: e = launch_search_kernel<5>(qmap, kmap, nq, n, row_tiles, units, k, w, ctx->dstatus, st); break;
-    case 6: e = launch_search_kernel<6>(qmap, kmap, nq, n, row_tiles, units, k, w, ctx->dstatus, st); break;
-    case 7: e = launch_search_kernel<7>(qmap, kmap, nq, n, row_tiles, units, k, w, ctx->dstatus, st); break;
-    default: e = launch_search_kernel<8>(qmap, kmap, nq, n, row_tiles, units, k, w, ctx->dstatus, st); break;
+    case 1: e = launch_search_kernel<1>(qmap, kmap, nq, n, qtiles, row_tiles, k, w, ctx->dstatus, st); break;
+    case 2: e = launch_search_kernel<2>(qmap, kmap, nq, n, qtiles, row_tiles, k, w, ctx->dstatus, st); break;
+    case 3: e = launch_search_kernel<3>(qmap, kmap, nq, n, qtiles, row_tiles, k, w, ctx->dstatus, st); break;
+    case 4: e = launch_search_kernel<4>(qmap, kmap, nq, n, qtiles, row_tiles, k, w, ctx->dstatus, st); break;
+    case 5: e = launch_search_kernel<5>(qmap, kmap, nq, n, qtiles, row_tiles, k, w, ctx->dstatus, st); break;
+    case 6: e = launch_search_kernel<6>(qmap, kmap, nq, n, qtiles, row_tiles, k, w, ctx->dstatus, st); break;
+    case 7: e = launch_search_kernel<7>(qmap, kmap, nq, n, qtiles, row_tiles, k, w, ctx->dstatus, st); break;
+    default: e = launch_search_kernel<8>(qmap, kmap, nq, n, qtiles, row_tiles, k, w, ctx->dstatus, st); break;
   }
   if (e != cudaSuccess) return e;
+  query_tables_kernel<<<unsigned((nq + kTabQueries - 1) / kTabQueries), 256, 0, st>>>(q, nq, ctx->d, ctx->m,
+                                                                                       ctx->dR64, ctx->dP64, w.xy);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   const size_t fsmem = size_t(2 * 256 + kCap) * 8 + size_t(kCap) * 8;
   cudaFuncSetAttribute(finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(fsmem));
-  finish_kernel<<<unsigned(nq), kFinishThreads, fsmem, st>>>(q, ctx->d, ctx->m, ctx->bmse, k, n, payload, norms,
-                                                             ctx->dR64, ctx->dP64, ctx->dc64, w.qerr, w.cnt, w.cand,
-                                                             ids, scores);
+  finish_kernel<<<unsigned(nq), kFinishThreads, fsmem, st>>>(ctx->d, ctx->m, ctx->bmse, k, n, payload, norms, w.xy,
+                                                             ctx->dc64, w.qerr, w.cnt, w.cand, ids, scores);
   return cudaGetLastError();
 }
 
