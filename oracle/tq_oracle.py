@@ -24,6 +24,9 @@ What it computes, step by step, and where the pages say so:
   The pages' formula was lost in extraction (the sentence ending in
   "保證 / 。"); the estimator used is the standard QJL one the surrounding
   text describes (unbiased, one sign bit per projected residual row).
+* m = 0 selects stage 1 alone (the MSE variant, TurboQuant_mse): no sign
+  sketch, and the estimator is its first term, which the same page notes is
+  biased for inner products (factor 2/pi at one bit).
 * Dequantisation "look up the table and rotate back" (same page, stage 1).
 
 Every function below is fp64 and follows the definitions literally: no
@@ -315,14 +318,17 @@ def estimate(Q: np.ndarray, codes, bits, n16, rho16, tb: Tables):
     """
     Q = np.atleast_2d(np.asarray(Q, dtype=np.float64))
     x = Q @ tb.R.T                       # rows: R q
-    y = Q @ tb.S.T                       # rows: S q
     cv = tb.c[np.asarray(codes)]         # (N, d)
-    sig = 2.0 * np.asarray(bits, dtype=np.float64) - 1.0
     n16 = np.asarray(n16, dtype=np.float64)
-    rho16 = np.asarray(rho16, dtype=np.float64)
     k1 = n16[None, :] * (x @ cv.T)
-    k2 = (QJL_CONST / tb.m) * rho16[None, :] * (y @ sig.T)
     a1 = n16[None, :] * (np.abs(x) @ np.abs(cv).T)
+    if tb.m == 0:
+        # m = 0: stage 1 alone (TurboQuant_mse), the first term
+        return k1, a1
+    y = Q @ tb.S.T                       # rows: S q
+    sig = 2.0 * np.asarray(bits, dtype=np.float64) - 1.0
+    rho16 = np.asarray(rho16, dtype=np.float64)
+    k2 = (QJL_CONST / tb.m) * rho16[None, :] * (y @ sig.T)
     a2 = (QJL_CONST / tb.m) * rho16[None, :] * np.sum(np.abs(y), axis=1)[:, None]
     return k1 + k2, a1 + a2
 
@@ -337,7 +343,7 @@ def dequantize(codes, bits, n16, rho16, tb: Tables, full: bool = True):
     n16 = np.asarray(n16, dtype=np.float64)
     rho16 = np.asarray(rho16, dtype=np.float64)
     xh = n16[:, None] * (tb.c[np.asarray(codes)] @ tb.R)
-    if full:
+    if full and tb.m > 0:
         sig = 2.0 * np.asarray(bits, dtype=np.float64) - 1.0
         xh = xh + (QJL_CONST / tb.m) * rho16[:, None] * (sig @ tb.S)
     return xh
@@ -422,8 +428,8 @@ def row_bytes(d: int, m: int, bmse: int) -> int:
 
 
 def _check_layout_dims(d: int, m: int, bmse: int):
-    if d % 8 or m % 8 or d < 8 or m < 8:
-        raise ValueError("packed layout needs d and m multiples of 8")
+    if d % 8 or m % 8 or d < 8 or m < 0:
+        raise ValueError("packed layout needs d and m multiples of 8 (m = 0: no sign bits)")
     if not 1 <= bmse <= 4:
         raise ValueError("1 <= b' <= 4")
 

@@ -522,3 +522,34 @@ def test_pack_layout_hand_example():
     want[0 + 2] |= 1 << 7
     want[12 + 3] = 1 << 14
     np.testing.assert_array_equal(p, want)
+
+
+# --------------------------------------------------------------------------
+# MSE-only variant (m = 0: stage 1 alone)
+# --------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("d,bits", [(64, 2), (128, 4), (200, 3)])
+def test_mse_only_estimator_is_the_first_term(d, bits):
+    """m = 0 uses the same rotation and codebook (stream 0) as m = d, stores no
+    sign bits, and estimates <q, k> by n16 sum_j c[idx_j] (Rq)_j, which is also
+    <q, x_hat> of the stage-1 reconstruction."""
+    rng = np.random.default_rng(d + bits)
+    K = rng.standard_normal((40, d))
+    Q = rng.standard_normal((3, d))
+    t0, t1 = O.make_tables(d, bits, 11, m=0), O.make_tables(d, bits, 11, m=d)
+    np.testing.assert_array_equal(t0.R, t1.R)
+    np.testing.assert_array_equal(t0.c, t1.c)
+    q0, q1 = O.quantize(K, t0), O.quantize(K, t1)
+    np.testing.assert_array_equal(q0.codes, q1.codes)
+    assert q0.bits.shape == (40, 0)
+    s0, A0 = O.estimate(Q, q0.codes, q0.bits, q0.n16, q0.rho16, t0)
+    first = q1.n16.astype(np.float64)[None, :] * ((Q @ t1.R.T) @ t1.c[q1.codes].T)
+    np.testing.assert_allclose(s0, first, rtol=1e-12, atol=1e-12)
+    xh = O.dequantize(q0.codes, q0.bits, q0.n16, q0.rho16, t0, full=True)
+    np.testing.assert_allclose(s0, Q @ xh.T, rtol=1e-10, atol=1e-10)
+    p = O.pack_rows(q0.codes, q0.bits, t0.bmse)
+    assert p.shape == (40, O.row_bytes(d, 0, t0.bmse)) and O.row_bytes(d, 0, t0.bmse) == -(-d // 64) * 64 * t0.bmse // 8
+    c2, b2 = O.unpack_rows(p, d, 0, t0.bmse)
+    np.testing.assert_array_equal(c2, q0.codes)
+    assert b2.shape == (40, 0)
