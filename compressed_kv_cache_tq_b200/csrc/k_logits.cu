@@ -449,7 +449,7 @@ __global__ void __launch_bounds__(256) logits_simt_kernel(const float* __restric
   }
   __syncthreads();
   const RowGeom gm = make_geom(d, m, bmse);
-  const float qc = float(kQjlConst) / float(m);
+  const float qc = m > 0 ? float(kQjlConst) / float(m) : 0.f;   // m = 0: no sign term
   const int64_t base_row = (int64_t(b) * Hkv + hkv) * S;
   for (int64_t s = blockIdx.y * blockDim.x + threadIdx.x; s < S; s += int64_t(gridDim.y) * blockDim.x) {
     const uint16_t* hw = reinterpret_cast<const uint16_t*>(payload + (base_row + s) * gm.row_bytes);
@@ -524,7 +524,7 @@ cudaError_t launch_logits(const tq_ctx* ctx, const float* q, int B, int Hq, int 
   const size_t qp_smem = size_t(2 * D * D + 2 * kMaxSlots * D) * 4;
   cudaFuncSetAttribute(qprep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(qp_smem));
   qprep_kernel<<<unsigned(groups), 128, qp_smem, st>>>(q, Hq, Hkv, nt, ctx->dRt, ctx->dPt, ctx->lut.inv_scale,
-                                                        scale, float(kQjlConst / ctx->m), frags, hs);
+                                                        scale, float(ctx->m > 0 ? kQjlConst / ctx->m : 0.0), frags, hs);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (S == 0) return cudaSuccess;

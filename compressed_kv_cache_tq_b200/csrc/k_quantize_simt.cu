@@ -146,7 +146,7 @@ __global__ void __launch_bounds__(kThreads) dequantize_kernel(const uint8_t* __r
   float* ssig = sv + kKeys * d;     // [kKeys][m] sigma
   const RowGeom g = make_geom(d, m, bmse);
   const int tid = threadIdx.x;
-  const float qc = float(kQjlConst) / float(m);
+  const float qc = m > 0 ? float(kQjlConst) / float(m) : 0.f;   // m = 0: no sign term
   for (int64_t base = int64_t(blockIdx.x) * kKeys; base < n; base += int64_t(gridDim.x) * kKeys) {
     const int nk = (n - base) < kKeys ? int(n - base) : kKeys;
     for (int idx = tid; idx < kKeys * m; idx += kThreads) {

@@ -106,7 +106,7 @@ __global__ void __launch_bounds__(256) decode_rows_kernel(const uint8_t* __restr
   const bool real = r < n;
   const uint16_t* hw = reinterpret_cast<const uint16_t*>(payload + (real ? r : 0) * g.row_bytes);
   const float n16 = real ? half_bits_to_float(norms[2 * r]) : 0.f;
-  const float w = real ? float(kQjlConst) / float(m) * half_bits_to_float(norms[2 * r + 1]) : 0.f;
+  const float w = real && m > 0 ? float(kQjlConst) / float(m) * half_bits_to_float(norms[2 * r + 1]) : 0.f;
   float ss = 0.f;
   for (int c = lane; c < kp / 8; c += 32) {
     __align__(16) __half h[8];
@@ -530,7 +530,7 @@ __global__ void __launch_bounds__(kFinishThreads) finish_kernel(
   const int tid = threadIdx.x, nth = blockDim.x;
   const int qi = blockIdx.x;
   const RowGeom g = make_geom(d, m, bmse);
-  const double qc = kQjlConst / double(m);
+  const double qc = m > 0 ? kQjlConst / double(m) : 0.0;   // m = 0: no sign term
   for (int i = tid; i < d + m; i += nth) (i < d ? sx[i] : sy[i - d]) = xy[size_t(qi) * (d + m) + i];
   __syncthreads();
   const uint32_t total = cnt[qi];

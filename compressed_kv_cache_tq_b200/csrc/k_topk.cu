@@ -110,7 +110,7 @@ __global__ void __launch_bounds__(512) rescore_kernel(const float* __restrict__ 
   }
   __syncthreads();
   const RowGeom g = make_geom(d, m, bmse);
-  const double qc = kQjlConst / double(m);
+  const double qc = m > 0 ? kQjlConst / double(m) : 0.0;   // m = 0: no sign term
   for (int ci = tid; ci < KC; ci += nth) {
     const int64_t row = cand[size_t(qi) * KC + ci];
     const uint16_t* hw = reinterpret_cast<const uint16_t*>(payload + row * g.row_bytes);

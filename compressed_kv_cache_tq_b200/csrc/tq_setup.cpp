@@ -210,6 +210,8 @@ void write_swizzled(const std::vector<T>& src, int rows, int K, uint8_t* dst) {
 
 template <typename T>
 cudaError_t upload(const std::vector<T>& h, T** d) {
+  *d = nullptr;
+  if (h.empty()) return cudaSuccess;   // the JL tables of the MSE-only variant
   cudaError_t e = cudaMalloc(reinterpret_cast<void**>(d), h.size() * sizeof(T));
   if (e != cudaSuccess) return e;
   return cudaMemcpy(*d, h.data(), h.size() * sizeof(T), cudaMemcpyHostToDevice);
@@ -255,8 +257,9 @@ void tq_free(tq_ctx* ctx) {
   delete ctx;
 }
 
+// m = 0: the MSE-only variant (no sign sketch)
 static bool dims_ok(int d, int bits, int m) {
-  return !(d < 64 || d > 256 || d % 8 || m < 64 || m > 256 || m % 8 || bits < 2 || bits > 4);
+  return !(d < 64 || d > 256 || d % 8 || (m != 0 && (m < 64 || m > 256 || m % 8)) || bits < 2 || bits > 4);
 }
 
 static void build_tables(int d, int bits, int m, uint64_t seed, uint32_t stream_base, std::vector<double>& R,

@@ -87,7 +87,10 @@ typedef enum { TQ_F32 = 0, TQ_BF16 = 1 } tq_dtype;
 tq_status tq_init(int d, int bits, uint64_t seed, tq_ctx** out);
 
 /* As tq_init with an explicit JL row count m (multiple of 8, 64 <= m <= 256) and the
- * first Philox stream used (G from stream_base, P from stream_base + 1). */
+ * first Philox stream used (G from stream_base, P from stream_base + 1).
+ * m = 0 selects the MSE-only variant ([p2] stage 1 alone): the same rotation
+ * and codebook, no sign sketch (rows hold only the b' = bits - 1 code bits),
+ * and the estimator is its first term n16 sum_j c[idx_j] (Rq)_j. */
 tq_status tq_init_ex(int d, int bits, int m, uint64_t seed, uint32_t stream_base, tq_ctx** out);
 
 /* Host only, no GPU needed: the fp64 tables tq_init_ex builds for these

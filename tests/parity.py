@@ -39,7 +39,7 @@ def check_quantize(payload, norms, K64, tb: O.Tables, report=None):
     sign_band = O.sign_boundary_distance(qz.z, qz.n, tb.m) <= O.SIGN_BAND
     bad_signs = sign_mis & ~sign_band & ~key_exc[:, None]
     assert not bad_signs.any(), f"{bad_signs.sum()} sign bits differ outside the band, e.g. {np.argwhere(bad_signs)[:5]}"
-    frac_sign = (sign_mis & ~key_exc[:, None]).mean()
+    frac_sign = float((sign_mis & ~key_exc[:, None]).mean()) if sign_mis.size else 0.0   # m = 0: no sign bits
     assert frac_sign < 1e-4, frac_sign
 
     def norm_ok(gpu16, exact, excused):

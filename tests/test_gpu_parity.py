@@ -308,3 +308,66 @@ def test_full_size_sampled(lib, name, B, Hkv, G, S, bits):
                                   q[b, h * G:(h + 1) * G].astype(np.float64), tb)
         got = out[b, h * G:(h + 1) * G][:, torch.from_numpy(s_idx).to(DEV)].cpu().numpy()
         check_close(got, est / math.sqrt(128), A / math.sqrt(128))
+
+
+# --------------------------------------------------------------------------
+# MSE-only variant (m = 0) and decode-time append
+# --------------------------------------------------------------------------
+
+
+@pytest.mark.parametrize("d,bits,dtype", [(128, 4, torch.bfloat16), (64, 2, torch.float32), (200, 3, torch.float32)])
+def test_mse_only_quantize_logits_dequantize(lib, d, bits, dtype):
+    ctx = _ctx(lib, d=d, bits=bits, seed=27, m=0)
+    assert ctx.m == 0 and ctx.row_bytes == -(-d // 64) * 64 * (bits - 1) // 8
+    k = W.toy_keys(900, d, seed=4)
+    kt = torch.from_numpy(k).to(dtype)
+    payload, norms = lib.tq_quantize(ctx, kt.to(DEV))
+    _status_clean(lib, ctx)
+    tb = tables_of(ctx)
+    check_quantize(payload.cpu().numpy(), norms.cpu().numpy(), kt.to(torch.float64).numpy(), tb)
+    q = W.queries((1, 3, d), seed=5)
+    out = lib.tq_logits(ctx, torch.from_numpy(q).to(DEV), payload, norms, 1)
+    _status_clean(lib, ctx)
+    s, A = oracle_estimates(payload.cpu().numpy(), norms.cpu().numpy(), q[0].astype(np.float64), tb)
+    check_close(out.cpu().numpy()[0], s, A)
+    xh = lib.tq_dequantize(ctx, payload, norms, full=True).cpu().numpy()
+    codes, bits_ = O.unpack_rows(payload.cpu().numpy(), d, 0, tb.bmse)
+    nr = norms.cpu().numpy().astype(np.float64)
+    ref = O.dequantize(codes, bits_, nr[:, 0], nr[:, 1], tb, full=True)
+    v = nr[:, :1] * np.abs(tb.c[codes]).sum(1, keepdims=True)
+    assert np.all(np.abs(xh - ref) <= 2e-5 * v)
+
+
+def test_mse_only_topk(lib):
+    ctx = _ctx(lib, d=200, bits=4, seed=31, m=0)
+    n, nq, k = 4000, 20, 10
+    db = W.search_vectors(n, 200, seed=77, which=0)
+    qs = W.search_vectors(nq, 200, seed=77, which=1)
+    payload, norms = lib.tq_quantize(ctx, torch.from_numpy(db).to(DEV))
+    ids, scores = lib.tq_topk(ctx, torch.from_numpy(qs).to(DEV), payload, norms, k)
+    _status_clean(lib, ctx)
+    s, A = oracle_estimates(payload.cpu().numpy(), norms.cpu().numpy(), qs.astype(np.float64), tables_of(ctx))
+    ids = ids.cpu().numpy()
+    for i in range(nq):
+        order = np.lexsort((np.arange(n), -s[i]))[:k + 1]
+        if s[i, order[k - 1]] - s[i, order[k]] < 1e-6 * A[i].max():
+            assert set(ids[i][:k - 1]) <= set(order)
+            continue
+        np.testing.assert_array_equal(ids[i], order[:k])
+
+
+@pytest.mark.parametrize("m", [128, 0])
+def test_decode_time_append_matches_batch(lib, m):
+    """A decode loop quantizes one new key per step into the next cache row;
+    the rows equal those of one batched call (tensor-core path for m = 128 at
+    n = 1, CUDA-core path for m = 0)."""
+    ctx = _ctx(lib, d=128, bits=4, seed=8, m=m)
+    keys = torch.from_numpy(W.toy_keys(40, 128, seed=12)).to(torch.bfloat16).to(DEV)
+    batch_p, batch_n = lib.tq_quantize(ctx, keys)
+    cache_p = torch.zeros_like(batch_p)
+    cache_n = torch.zeros_like(batch_n)
+    for s in range(keys.shape[0]):
+        lib.tq_quantize(ctx, keys[s:s + 1], cache_p[s:s + 1], cache_n[s:s + 1])
+    _status_clean(lib, ctx)
+    assert torch.equal(cache_p, batch_p)
+    assert torch.equal(cache_n, batch_n)
