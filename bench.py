@@ -18,6 +18,10 @@ rank runs the full workload; there is no data-path collective.
 --impl reference runs the CPU oracle (test infrastructure) on a bounded sample
 of the same workload on the host cores, on rank 0 only.
 
+--workload longctx runs the same step on the long-context configuration: one
+sequence of 131072 keys for each of 8 KV heads (keys drawn as above), b = 3
+(2 Lloyd-Max bits + 1 QJL bit), 32 query heads.
+
 --workload search times the vector-search configuration instead (one JSON
 line): 1 000 000 unit vectors of a 100-cluster Gaussian mixture, d = 200 fp32,
 10 000 queries drawn the same way, b = 2 and b = 4, top-10 by the estimator
@@ -44,6 +48,24 @@ METRIC = "tq_logits keys scored/s & HBM GB/s (% of 8 TB/s); tq_quantize vectors/
 B, HKV, HQ, D, S, BITS = 8, 8, 32, 128, 32768, 4
 SEED_KEYS, SEED_TABLES = 1001, 42
 WORKLOAD = "decode_llama31_8b_layer_b8_hkv8_hq32_d128_s32768_b4"
+
+# The key-cache workloads a step can run: (B, Hkv, Hq, d, S, bits, key seed, name).
+# decode: the Llama-3.1-8B-shaped decode layer above.  longctx: one sequence of
+# 131072 keys per KV head, keys drawn as in decode, b = 3 (2 Lloyd-Max bits +
+# 1 QJL bit): quantize every key on append, then the 32 query heads' logits.
+KV_WORKLOADS = {
+    "decode": (8, 8, 32, 128, 32768, 4, 1001, "decode_llama31_8b_layer_b8_hkv8_hq32_d128_s32768_b4"),
+    "longctx": (1, 8, 32, 128, 131072, 3, 1002, "longctx_prefill_decode_b1_hkv8_hq32_d128_s131072_b3"),
+}
+
+
+def set_workload(name: str, seq: int | None = None):
+    """Point the module's shape globals at one of KV_WORKLOADS (seq overrides S)."""
+    global B, HKV, HQ, D, S, BITS, SEED_KEYS, WORKLOAD
+    B, HKV, HQ, D, S, BITS, SEED_KEYS, WORKLOAD = KV_WORKLOADS[name]
+    if seq is not None and seq != S:
+        WORKLOAD = WORKLOAD.replace(f"_s{S}_", f"_s{seq}_")
+        S = seq
 
 
 def peaks():
@@ -148,7 +170,7 @@ def cpu_baseline(budget_s: float = 12.0, max_keys: int = 1 << 19):
     dt = time.perf_counter() - t0
     threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     return {"value": done / dt, "unit": "keys/s", "cores": threads, "kind": "oracle",
-            "sample": f"{done} of {B * HKV * S} keys (quantize + 4-head estimates), {dt:.1f} s, fp64 numpy"}
+            "sample": f"{done} of {B * HKV * S} keys (quantize + {HQ // HKV}-head estimates), {dt:.1f} s, fp64 numpy"}
 
 
 def run_search(args):
@@ -158,15 +180,15 @@ def run_search(args):
 
     from compressed_kv_cache_tq_b200 import tq, workloads as W
 
-    n, nq, d, k = 1_000_000, 10_000, 200, 10
+    n, nq, d, k = args.rows, args.queries, 200, 10
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     db = torch.from_numpy(W.search_vectors(n, d, seed=1004, which=0)).to(dev)
     qs = torch.from_numpy(W.search_vectors(nq, d, seed=1004, which=1)).to(dev)
     # exact top-1 of every query by the plain inner product (fp32, on the device)
     top1 = torch.empty(nq, dtype=torch.int64, device=dev)
-    for q0 in range(0, nq, 1000):
-        top1[q0:q0 + 1000] = (qs[q0:q0 + 1000] @ db.T).argmax(1)
+    for q0 in range(0, nq, 500):
+        top1[q0:q0 + 500] = (qs[q0:q0 + 500] @ db.T).argmax(1)
     stream = torch.cuda.current_stream()
     per_bits = {}
     hbm, tf, tf_sus, src = peaks()
@@ -214,16 +236,22 @@ def run_search(args):
                 "queries_per_s": nq / ms_s * 1e3, "recall_at_1_at_10": recall,
                 "search_TFLOP_s": flops / ms_s / 1e9, "e2e_ms": a.elapsed_time(b_)}
             del ws
-    # the oracle on a bounded sample: 200 000 rows indexed, 128 queries scored against them
-    from oracle import tq_oracle as O
-    tb = O.make_tables(d, 2, SEED_TABLES, m=d)
-    dbh, qh = db[:200_000].double().cpu().numpy(), qs[:128].double().cpu().numpy()
-    t0 = time.perf_counter()
-    qz = O.quantize(dbh, tb)
-    t1 = time.perf_counter()
-    O.topk(qh, qz.codes, qz.bits, qz.n16, qz.rho16, tb, k)
-    t2 = time.perf_counter()
-    cpu_qps = 128 / ((t2 - t1) * n / 200_000)
+    # the oracle on a bounded sample: up to 200 000 rows indexed, 128 queries scored against them
+    cpu = None
+    if not args.no_cpu_baseline:
+        from oracle import tq_oracle as O
+        tb = O.make_tables(d, 2, SEED_TABLES, m=d)
+        n_cpu = min(n, 200_000)
+        dbh, qh = db[:n_cpu].double().cpu().numpy(), qs[:128].double().cpu().numpy()
+        t0 = time.perf_counter()
+        qz = O.quantize(dbh, tb)
+        t1 = time.perf_counter()
+        O.topk(qh, qz.codes, qz.bits, qz.n16, qz.rho16, tb, k)
+        t2 = time.perf_counter()
+        cpu = {"value": qh.shape[0] / ((t2 - t1) * n / n_cpu), "unit": "queries/s", "cores": os.cpu_count(),
+               "kind": "oracle",
+               "sample": f"b=2: {n_cpu} rows indexed in {t1 - t0:.1f} s, {qh.shape[0]} queries scored "
+                         f"against them in {t2 - t1:.1f} s, scaled to {n} rows; fp64 numpy"}
     b4 = per_bits["b4"]
     line = {
         "metric": "tq_topk queries/s (10^6 rows, d=200, top-10) and recall@1@10; index build ms",
@@ -231,8 +259,10 @@ def run_search(args):
         "warmup": args.warmup, "ms_per_step": b4["index_build_ms"] + b4["search_ms"],
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
         "data": "synthetic",
-        "config": {"workload": "vector_search_1m_d200_nq10k_top10", "rows": n, "queries": nq, "d": d, "m": d,
-                   "k": k, "bits": [2, 4], "l2": "the fp16 row matrix (896 MB) exceeds L2"},
+        "config": {"workload": f"vector_search_{n}_d200_nq{nq}_top10", "rows": n, "queries": nq, "d": d, "m": d,
+                   "k": k, "bits": [2, 4],
+                   "l2": f"the fp16 row matrix ({n * 896 / 1e6:.0f} MB) "
+                         + ("exceeds L2" if n * 896 > 126e6 else "fits in L2 (profiling size)")},
         "per_bits": per_bits,
         "roofline": {"bound": "tensor", "kernel": "tq_topk (decode + scoring + re-scoring)",
                      "achieved": b4["search_TFLOP_s"], "peak": tf, "unit": "TFLOP/s",
@@ -242,10 +272,9 @@ def run_search(args):
                 "d2h_bytes_per_step": nq * k * 12},
         "gpu_launches": 4,
         "clocks": clocks.summary(),
-        "cpu_baseline": {"value": cpu_qps, "unit": "queries/s", "cores": os.cpu_count(), "kind": "oracle",
-                         "sample": f"b=2: 200000 rows indexed in {t1 - t0:.1f} s, 128 queries scored against "
-                                   f"them in {t2 - t1:.1f} s, scaled to 10^6 rows; fp64 numpy"},
     }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
     print(json.dumps(line), flush=True)
     return 0
 
@@ -277,8 +306,8 @@ def run_reference(args, rank):
 # current kernels, from one ncu capture at S = 16384 (1 048 576 keys); per
 # launch it scales with the keys processed.  Summaries: profiles/quantize_tc_decode_s16384.md
 # and profiles/logits_mma_decode_s16384.md.  Set to None when a kernel changes.
-DRAM_BYTES_PER_KEY = {"tq_quantize": (268.648960e6 + 53.591040e6) / 1048576,
-                      "tq_logits": (71.457024e6 + 3.751168e6) / 1048576}
+DRAM_BYTES_PER_KEY = {"decode": {"tq_quantize": (268.648960e6 + 53.591040e6) / 1048576,
+                                  "tq_logits": (71.457024e6 + 3.751168e6) / 1048576}}
 
 
 def max_over_ranks(x: float, dist, device) -> float:
@@ -310,6 +339,7 @@ def result_line(*, world, n, steps, warmup, ms, q_ms, l_ms, e2e_ms, h2d, d2h, cl
     }
     dom = "tq_quantize" if q_ms >= l_ms else "tq_logits"
     ach = kernels[dom]["GB/s"]
+    dram = DRAM_BYTES_PER_KEY.get(WORKLOAD.split("_")[0], {}).get(dom)
     return {
         "metric": METRIC,
         "value": world * n / ms_step * 1e3,
@@ -325,11 +355,12 @@ def result_line(*, world, n, steps, warmup, ms, q_ms, l_ms, e2e_ms, h2d, d2h, cl
         "data": "synthetic",
         "config": {"workload": WORKLOAD, "global_batch": B * world, "seq_len": S, "kv_heads": HKV,
                    "q_heads": HQ, "head_dim": D, "bits": BITS, "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2: keys 537 MB, packed cache 143 MB; logits read the cache "
-                         "written one step earlier"},
+                   "l2": f"inputs larger than L2: keys {n * D * 2 / 1e6:.0f} MB, packed caches "
+                         f"{n * (bpk['quantize_out']) / 1e6:.0f} MB each; logits read the cache written one step "
+                         "earlier, with the keys' traffic in between"},
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": hbm, "unit": "GB/s",
                      "frac": ach / hbm, "peak_source": src,
-                     "traffic": (None if DRAM_BYTES_PER_KEY.get(dom) is None else DRAM_BYTES_PER_KEY[dom] * n),
+                     "traffic": None if dram is None else dram * n,
                      "traffic_source": "ncu capture at S=16384 scaled by keys (bytes per launch)"},
         "kernels": kernels,
         "logits_keys_per_s": world * n / l_ms * 1e3,
@@ -348,17 +379,17 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="decode", choices=["decode", "search"])
-    ap.add_argument("--seq", type=int, default=32768,
-                    help="sequence length (default: the decode workload's 32768; smaller values for profiling)")
+    ap.add_argument("--workload", default="decode", choices=["decode", "longctx", "search"])
+    ap.add_argument("--rows", type=int, default=1_000_000, help="search: database rows")
+    ap.add_argument("--queries", type=int, default=10_000, help="search: queries")
+    ap.add_argument("--seq", type=int, default=None,
+                    help="sequence length (default: the workload's own; smaller values for profiling)")
     args = ap.parse_args()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    global S, WORKLOAD
-    if args.seq != S:
-        S = args.seq
-        WORKLOAD = WORKLOAD.replace("s32768", f"s{S}")
+    if args.workload in KV_WORKLOADS:
+        set_workload(args.workload, args.seq)
     if args.impl == "reference":
         return run_reference(args, rank)
     if args.warmup < 3:

@@ -28,6 +28,9 @@ What it computes, step by step, and where the pages say so:
   sketch, and the estimator is its first term, which the same page notes is
   biased for inner products (factor 2/pi at one bit).
 * Dequantisation "look up the table and rotate back" (same page, stage 1).
+* Fractional rates (2.5 bits per channel): a per-KV-head channel split
+  into a high-variance group and a low-variance group, each quantised on
+  its own (readings in the section "Channel split" below).
 
 Every function below is fp64 and follows the definitions literally: no
 blocking, fusion or reordering beyond vectorising over keys.
@@ -387,6 +390,105 @@ def topk(Q: np.ndarray, codes, bits, n16, rho16, tb: Tables, k: int):
         ids[i] = order
         sc[i] = s[i, order]
     return ids, sc, s, A
+
+
+# ---------------------------------------------------------------------------
+# Channel split: fractional bit rates such as 2.5 bits per channel
+#
+# The pages quote 3.5- and 2.5-bit configurations (arXiv summary page:
+# "3.5 bits per channel"; mooersco.com section 2.1: "2.5bit >= 7x";
+# zhengruan.com: 2.5 bits costs a slight quality drop) without saying how a
+# fractional rate is reached, and mooersco.com's FAQ notes that the
+# unrotated channels' variances differ by two orders of magnitude.  Reading:
+# per KV head, the d_hi channels of largest variance form a high group and
+# the rest a low group; each group is quantised as its own vector with its
+# own tables (rotation, JL matrix, codebook) and bit width, and the inner
+# product estimate is the sum of the two groups' estimates, since
+# <q, k> = <q_hi, k_hi> + <q_lo, k_lo> for the same channel split of q and k.
+# ---------------------------------------------------------------------------
+
+
+def split_plan(K: np.ndarray, d_hi: int) -> np.ndarray:
+    """Channel order per KV head for keys K (B, Hkv, S, d).
+
+    For head h, the variance of channel c over all B x S keys of that head
+    is sum_rows (x - mean)^2 / (B S) (the 1 / (B S - 1) of the sample
+    variance would not change the order).  The d_hi channels of largest
+    variance, ties to the lower channel index, come first in ascending
+    channel order, then the other channels in ascending order (reading).
+    Returns perm (Hkv, d) int64: group coordinate p of head h is channel
+    perm[h, p]; coordinates p < d_hi form the high group.
+    """
+    K = np.asarray(K, dtype=np.float64)
+    B, Hkv, S, d = K.shape
+    perm = np.empty((Hkv, d), dtype=np.int64)
+    for h in range(Hkv):
+        X = K[:, h].reshape(B * S, d)
+        if X.shape[0] > 0:
+            mean = X.mean(axis=0)
+            var = np.sum((X - mean) ** 2, axis=0) / X.shape[0]
+        else:
+            var = np.zeros(d)
+        order = sorted(range(d), key=lambda c: (-var[c], c))
+        hi = sorted(order[:d_hi])
+        lo = sorted(order[d_hi:])
+        perm[h] = hi + lo
+    return perm
+
+
+def split_groups(X: np.ndarray, perm: np.ndarray, d_hi: int):
+    """Gather the two channel groups of X (B, H, S, d) or (B, H, d) by perm (H, d):
+    returns (X_hi, X_lo) with the channel axis last."""
+    X = np.asarray(X, dtype=np.float64)
+    H = perm.shape[0]
+    hi = np.stack([X[:, h][..., perm[h, :d_hi]] for h in range(H)], axis=1)
+    lo = np.stack([X[:, h][..., perm[h, d_hi:]] for h in range(H)], axis=1)
+    return hi, lo
+
+
+def split_quantize(K: np.ndarray, perm: np.ndarray, tb_hi: Tables, tb_lo: Tables):
+    """Quantise keys K (B, Hkv, S, d) group by group: the high group (the
+    first tb_hi.d coordinates of perm) with tb_hi, the rest with tb_lo.
+    Returns (Quantized hi, Quantized lo), rows in [B][Hkv][S] order."""
+    B, Hkv, S, d = K.shape
+    assert tb_hi.d + tb_lo.d == d
+    Khi, Klo = split_groups(K, perm, tb_hi.d)
+    return quantize(Khi.reshape(-1, tb_hi.d), tb_hi), quantize(Klo.reshape(-1, tb_lo.d), tb_lo)
+
+
+def split_gqa_logits(q: np.ndarray, perm: np.ndarray, qz_hi: Quantized, qz_lo: Quantized, tb_hi: Tables,
+                     tb_lo: Tables, B: int, Hkv: int, S: int, scale: float = 1.0):
+    """Split-cache attention logits: for query head h (KV head hk = h // G)
+    the estimate of <q_hi, k_hi> with tb_hi plus that of <q_lo, k_lo> with
+    tb_lo, both groups gathered by perm[hk].  Returns (logits, A), each
+    (B, Hq, S), A the sum of both groups' absolute-term sums."""
+    Bq, Hq, d = q.shape
+    G = Hq // Hkv
+    # each query head takes the channel split of the KV head it reads
+    qperm = np.repeat(perm, G, axis=0)
+    q_hi, q_lo = split_groups(q[:, :, None, :], qperm, tb_hi.d)
+    q_hi, q_lo = q_hi[:, :, 0], q_lo[:, :, 0]
+
+    def view(qz, tb):
+        return (qz.codes.reshape(B, Hkv, S, tb.d), qz.bits.reshape(B, Hkv, S, tb.m),
+                qz.n16.reshape(B, Hkv, S), qz.rho16.reshape(B, Hkv, S))
+
+    s_hi, a_hi = gqa_logits(q_hi, *view(qz_hi, tb_hi), tb_hi, scale)
+    s_lo, a_lo = gqa_logits(q_lo, *view(qz_lo, tb_lo), tb_lo, scale)
+    return s_hi + s_lo, a_hi + a_lo
+
+
+def split_dequantize(perm: np.ndarray, qz_hi: Quantized, qz_lo: Quantized, tb_hi: Tables, tb_lo: Tables,
+                     B: int, Hkv: int, S: int, full: bool = True) -> np.ndarray:
+    """Reconstruct keys (B, Hkv, S, d) in the original channel order: each
+    group's reconstruction scattered back to the channels perm names."""
+    xh = dequantize(qz_hi.codes, qz_hi.bits, qz_hi.n16, qz_hi.rho16, tb_hi, full).reshape(B, Hkv, S, tb_hi.d)
+    xl = dequantize(qz_lo.codes, qz_lo.bits, qz_lo.n16, qz_lo.rho16, tb_lo, full).reshape(B, Hkv, S, tb_lo.d)
+    out = np.empty((B, Hkv, S, tb_hi.d + tb_lo.d))
+    for h in range(Hkv):
+        out[:, h][..., perm[h, :tb_hi.d]] = xh[:, h]
+        out[:, h][..., perm[h, tb_hi.d:]] = xl[:, h]
+    return out
 
 
 # ---------------------------------------------------------------------------

@@ -553,3 +553,90 @@ def test_mse_only_estimator_is_the_first_term(d, bits):
     c2, b2 = O.unpack_rows(p, d, 0, t0.bmse)
     np.testing.assert_array_equal(c2, q0.codes)
     assert b2.shape == (40, 0)
+
+
+# --------------------------------------------------------------------------
+# Channel split (fractional bit rates)
+# --------------------------------------------------------------------------
+
+
+def test_split_plan_orders_by_variance_with_ties_to_lower_channel():
+    # channel c of head h alternates +a, -a around an offset mu over the B*S
+    # rows, so its variance is exactly a^2 whatever mu is; the expected order
+    # is written out by hand from the amplitudes
+    B, S, d = 2, 3, 8
+    amp = np.array([[1, 5, 2, 5, 0.5, 3, 4, 0.25],      # head 0: 1 and 3 tie at 5
+                    [7, 1, 1, 1, 6, 2, 9, 8]], float)   # head 1: 1, 2, 3 tie at 1
+    mu = np.array([100.0, -3.0, 0.0, 7.0, -50.0, 2.0, 1.0, 9.0])
+    signs = np.array([1, -1, 1, -1, 1, -1], float).reshape(B, S)
+    K = np.empty((B, 2, S, d))
+    for h in range(2):
+        K[:, h] = mu + signs[:, :, None] * amp[h]
+    perm = O.split_plan(K, 4)
+    # head 0 by amplitude: 5 (ch 1), 5 (ch 3), 4 (ch 6), 3 (ch 5) | the rest
+    assert perm[0].tolist() == [1, 3, 5, 6, 0, 2, 4, 7]
+    # head 1: 9 (ch 6), 8 (ch 7), 7 (ch 0), 6 (ch 4) | 2 (ch 5) and the three 1s
+    assert perm[1].tolist() == [0, 4, 6, 7, 1, 2, 3, 5]
+    # three-way tie at the cut: head 1 with 6 high channels takes the lowest tied one
+    perm6 = O.split_plan(K, 6)
+    assert perm6[1].tolist() == [0, 1, 4, 5, 6, 7, 2, 3]
+
+
+def test_split_plan_of_no_keys_keeps_channel_order():
+    perm = O.split_plan(np.zeros((1, 2, 0, 8)), 3)
+    assert perm.tolist() == [[0, 1, 2, 3, 4, 5, 6, 7]] * 2
+
+
+def test_split_estimator_unbiased_with_both_groups_redrawn():
+    # each group's estimate is unbiased for its part of <q, k>, and the parts
+    # add up to <q, k> under any split of the channels
+    d, nseed = 16, 2000
+    rng = np.random.default_rng(11)
+    k = rng.standard_normal((1, 1, 1, d)) * np.linspace(0.5, 4.0, d)
+    qv = rng.standard_normal((1, 1, d))
+    perm = O.split_plan(np.concatenate([k, -k], axis=2), 8)
+    est = []
+    for s in range(nseed):
+        thi = O.make_tables(8, 3, seed=5000 + 2 * s)
+        tlo = O.make_tables(8, 2, seed=5001 + 2 * s)
+        a, b = O.split_quantize(k, perm, thi, tlo)
+        v, _ = O.split_gqa_logits(qv, perm, a, b, thi, tlo, 1, 1, 1)
+        est.append(v[0, 0, 0])
+    est = np.array(est)
+    se = est.std(ddof=1) / math.sqrt(nseed)
+    assert abs(est.mean() - float(k[0, 0, 0] @ qv[0, 0])) < 3 * se
+
+
+def test_split_dequantize_reproduces_the_split_estimator():
+    rng = np.random.default_rng(12)
+    B, Hkv, S, d, G = 2, 3, 5, 16, 2
+    K = rng.standard_normal((B, Hkv, S, d)) * rng.uniform(0.2, 5.0, (1, Hkv, 1, d))
+    q = rng.standard_normal((B, Hkv * G, d))
+    perm = O.split_plan(K, 8)
+    thi, tlo = O.make_tables(8, 3, 42), O.make_tables(8, 2, 43)
+    a, b = O.split_quantize(K, perm, thi, tlo)
+    s, _ = O.split_gqa_logits(q, perm, a, b, thi, tlo, B, Hkv, S)
+    xh = O.split_dequantize(perm, a, b, thi, tlo, B, Hkv, S, full=True)
+    for h in range(Hkv * G):
+        np.testing.assert_allclose(s[:, h], np.einsum("bd,bsd->bs", q[:, h], xh[:, h // G]), atol=1e-11)
+
+
+def test_split_gives_the_high_variance_channels_the_finer_code():
+    # with strongly unequal channel scales (different per head), the planned
+    # split reconstructs the keys better than the same split with the two
+    # groups' bit widths exchanged
+    rng = np.random.default_rng(13)
+    B, Hkv, S, d = 1, 3, 400, 16
+    scales = np.exp(2.0 * rng.standard_normal((Hkv, d)))
+    K = rng.standard_normal((B, Hkv, S, d)) * scales[None, :, None, :]
+    perm = O.split_plan(K, 8)
+    swapped = np.concatenate([perm[:, 8:], perm[:, :8]], axis=1)
+    thi, tlo = O.make_tables(8, 4, 42), O.make_tables(8, 2, 43)
+    for p, worse in ((perm, False), (swapped, True)):
+        a, b = O.split_quantize(K, p, thi, tlo)
+        x = O.split_dequantize(p, a, b, thi, tlo, B, Hkv, S, full=False)
+        err = np.sum((x - K) ** 2, axis=(0, 2, 3))
+        if not worse:
+            planned = err
+        else:
+            assert np.all(planned < err)
