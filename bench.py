@@ -95,8 +95,14 @@ class ClockSampler:
                                          stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
+            # nvidia-smi takes a moment to start: wait for its first sample, so
+            # that the samples from here on fall inside the timed region
+            t0 = time.time()
+            while not self.lines and time.time() - t0 < 5.0 and self.proc.poll() is None:
+                time.sleep(0.01)
         except Exception:
             self.proc = None
+        self.first = len(self.lines)
         return self
 
     def _read(self):
@@ -104,6 +110,10 @@ class ClockSampler:
             self.lines.append(line.strip())
 
     def __exit__(self, *a):
+        # a short timed region may end before the next sample: wait for one
+        t0 = time.time()
+        while self.proc and len(self.lines) <= self.first and time.time() - t0 < 0.5:
+            time.sleep(0.005)
         if self.proc:
             self.proc.terminate()
             try:
@@ -114,7 +124,7 @@ class ClockSampler:
     def summary(self):
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ln in (self.lines[self.first:] or self.lines):
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 9:
                 continue

@@ -427,14 +427,17 @@ __global__ void __launch_bounds__(256) logits_simt_kernel(const float* __restric
                                                           const float* __restrict__ Pt, int d, int m, int bmse,
                                                           CodebookParams cb, const uint8_t* __restrict__ payload,
                                                           const uint16_t* __restrict__ norms, float scale,
-                                                          float* __restrict__ out) {
+                                                          float* __restrict__ out, ChannelGather gth,
+                                                          int accumulate) {
   extern __shared__ float sm[];
   float* sq = sm;
   float* sx = sq + d;
   float* sy = sx + d;
   const int bh = blockIdx.x;
   const int b = bh / Hq, h = bh % Hq, G = Hq / Hkv, hkv = h / G;
-  for (int i = threadIdx.x; i < d; i += blockDim.x) sq[i] = q[size_t(bh) * d + i];
+  // split: the query's channels in the group order of its KV head
+  for (int i = threadIdx.x; i < d; i += blockDim.x)
+    sq[i] = gth.perm ? q[size_t(bh) * gth.dtot + gth.perm[hkv * gth.dtot + gth.off + i]] : q[size_t(bh) * d + i];
   __syncthreads();
   for (int j = threadIdx.x; j < d; j += blockDim.x) {
     float x = 0.f;
@@ -458,7 +461,8 @@ __global__ void __launch_bounds__(256) logits_simt_kernel(const float* __restric
     for (int i = 0; i < m; ++i) c += unpack_sign(hw, gm, i) ? sy[i] : -sy[i];
     const float n16 = half_bits_to_float(norms[2 * (base_row + s)]);
     const float r16 = half_bits_to_float(norms[2 * (base_row + s) + 1]);
-    out[size_t(bh) * S + s] = scale * (n16 * a + qc * r16 * c);
+    const float v = scale * (n16 * a + qc * r16 * c);
+    out[size_t(bh) * S + s] = accumulate ? out[size_t(bh) * S + s] + v : v;
   }
 }
 
@@ -497,6 +501,17 @@ cudaError_t launch_mma(const tq_ctx* ctx, int B, int Hq, int Hkv, int64_t S, con
 
 }  // namespace
 
+cudaError_t launch_logits_simt(const tq_ctx* ctx, const float* q, int B, int Hq, int Hkv, int64_t S,
+                               const uint8_t* payload, const uint16_t* norms, float scale, float* out,
+                               ChannelGather gather, int accumulate, cudaStream_t st) {
+  if (S == 0 || B == 0 || Hq == 0) return cudaSuccess;
+  const size_t smem = size_t(2 * ctx->d + ctx->m) * 4;
+  dim3 grid(unsigned(B * Hq), unsigned(std::min<int64_t>((S + 255) / 256, 64)));
+  logits_simt_kernel<<<grid, 256, smem, st>>>(q, Hq, Hkv, S, ctx->dRt, ctx->dPt, ctx->d, ctx->m, ctx->bmse,
+                                              ctx->cb, payload, norms, scale, out, gather, accumulate);
+  return cudaGetLastError();
+}
+
 size_t qprep_bytes(const tq_ctx* ctx, int64_t groups, int heads_per_group) {
   if (!fast_path(ctx)) return 256;
   const int nt = (heads_per_group + HPT - 1) / HPT;
@@ -509,13 +524,9 @@ cudaError_t launch_logits(const tq_ctx* ctx, const float* q, int B, int Hq, int 
                           const uint8_t* payload, const uint16_t* norms, float scale, float* out, void* ws,
                           cudaStream_t st) {
   const int G = Hq / Hkv;
-  if (!fast_path(ctx) || G > 8) {
-    const size_t smem = size_t(2 * ctx->d + ctx->m) * 4;
-    dim3 grid(unsigned(B * Hq), unsigned(std::min<int64_t>((S + 255) / 256, 64)));
-    logits_simt_kernel<<<grid, 256, smem, st>>>(q, Hq, Hkv, S, ctx->dRt, ctx->dPt, ctx->d, ctx->m, ctx->bmse,
-                                                ctx->cb, payload, norms, scale, out);
-    return cudaGetLastError();
-  }
+  if (!fast_path(ctx) || G > 8)
+    return launch_logits_simt(ctx, q, B, Hq, Hkv, S, payload, norms, scale, out,
+                              ChannelGather{nullptr, 1, 1, 0, 0}, 0, st);
   const int nt = (G + HPT - 1) / HPT;
   const int64_t groups = int64_t(B) * Hkv;
   uint32_t* frags = static_cast<uint32_t*>(ws);

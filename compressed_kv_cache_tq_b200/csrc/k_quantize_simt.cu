@@ -32,7 +32,8 @@ __global__ void __launch_bounds__(kThreads) quantize_simt_kernel(const T* __rest
                                                                  const float* __restrict__ Pt, int d, int m,
                                                                  int bmse, CodebookParams cb,
                                                                  uint8_t* __restrict__ payload,
-                                                                 uint16_t* __restrict__ norms) {
+                                                                 uint16_t* __restrict__ norms,
+                                                                 ChannelGather gth) {
   extern __shared__ float smem[];
   float* sk = smem;                          // [kKeys][d] keys, later r_rot
   float* sn = sk + kKeys * d;                // [kKeys] norms
@@ -49,7 +50,14 @@ __global__ void __launch_bounds__(kThreads) quantize_simt_kernel(const T* __rest
     const int nk = (n - base) < kKeys ? int(n - base) : kKeys;
     for (int idx = tid; idx < kKeys * d; idx += kThreads) {
       const int k = idx / d, j = idx - k * d;
-      sk[idx] = k < nk ? load_key(keys + (base + k) * ld + j) : 0.f;
+      float v = 0.f;
+      if (k < nk) {
+        const int64_t row = base + k;
+        // split: coordinate j of the group is a channel of the row's KV head
+        const int col = gth.perm ? gth.perm[int((row / gth.S) % gth.Hkv) * gth.dtot + gth.off + j] : j;
+        v = load_key(keys + row * ld + col);
+      }
+      sk[idx] = v;
     }
     if (tid < kKeys) srr[tid] = 0.f;
     __syncthreads();
@@ -204,7 +212,7 @@ int grid_for(int64_t n) {
 }  // namespace
 
 cudaError_t launch_quantize_simt(const tq_ctx* ctx, const void* keys, int dtype, int64_t n, int64_t ld,
-                                 uint8_t* payload, uint16_t* norms, cudaStream_t st) {
+                                 uint8_t* payload, uint16_t* norms, cudaStream_t st, ChannelGather gather) {
   const int d = ctx->d, m = ctx->m;
   const RowGeom g = make_geom(d, m, ctx->bmse);
   const size_t smem = size_t(kKeys) * d * 4 + 2 * kKeys * 4 + size_t(kKeys) * (g.dp + g.mp);
@@ -213,12 +221,12 @@ cudaError_t launch_quantize_simt(const tq_ctx* ctx, const void* keys, int dtype,
     auto kern = quantize_simt_kernel<float>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     kern<<<grid, kThreads, smem, st>>>(static_cast<const float*>(keys), n, ld, ctx->dRt, ctx->dPt, d, m,
-                                        ctx->bmse, ctx->cb, payload, norms);
+                                        ctx->bmse, ctx->cb, payload, norms, gather);
   } else {
     auto kern = quantize_simt_kernel<__nv_bfloat16>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     kern<<<grid, kThreads, smem, st>>>(static_cast<const __nv_bfloat16*>(keys), n, ld, ctx->dRt, ctx->dPt, d,
-                                        m, ctx->bmse, ctx->cb, payload, norms);
+                                        m, ctx->bmse, ctx->cb, payload, norms, gather);
   }
   return cudaGetLastError();
 }

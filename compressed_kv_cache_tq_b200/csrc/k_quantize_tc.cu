@@ -470,6 +470,353 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
   }
 }
 
+// ---------------------------------------------------------------------------
+// Split quantize: keys of d = 128 channels split per KV head into a high and a
+// low group of 64 channels, each group a d = m = 64 quantizer of its own.  The
+// pipeline is the one above with two operands changed: the rotation operand
+// is the head's M_h (M_h k = (R_hi k_hi, R_lo k_lo): both groups' rotations
+// of the gathered key in one product, the gather folded into the columns of
+// M_h), and the JL operand is diag(P_hi, P_lo).  Rotated coordinates 0..63
+// belong to the high group and 64..127 to the low group, which are exactly
+// the TMEM columns of epilogue halves 0 and 1: each half finishes its own
+// group (norm, cells, residual norm, packing) with no exchange between the
+// halves.  Each CTA serves one KV head, so it loads the head's operand once.
+// ---------------------------------------------------------------------------
+
+struct SplitGeom {
+  int64_t S;     // keys per (batch, KV head) pair
+  int64_t tps;   // 128-key tiles per pair
+  int Hkv, head, cph, sub;   // KV heads, this CTA's head, CTAs per head, index among them
+};
+
+template <int BM>
+__device__ __forceinline__ void split_epilogue(uint32_t bar0, uint32_t d1, uint32_t d2, int slot, int q0, int row,
+                                               int64_t my_tiles, const SplitGeom& sg, const HalfBook& book,
+                                               uint8_t* __restrict__ payload, uint16_t* __restrict__ norms,
+                                               volatile int* abort_flag, uint32_t* status) {
+  auto bar = [&](int i) { return bar0 + 8u * uint32_t(i); };
+  int64_t k = 0;
+  for (int64_t i = slot; i < my_tiles; i += 2, ++k) {
+    const uint32_t par = uint32_t(k & 1);
+    if (!mbar_wait_warp(bar(kBarD1Full + slot), par, abort_flag, status)) break;
+    tc_fence_after();
+    // ||k_group||^2 = ||R_group k_group||^2 from this half's 64 rotated coordinates
+    float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int qq = 0; qq < 2; ++qq) {
+      float y[32];
+      tmem_ld32(d1 + 32u * (q0 + qq), y);
+      tmem_wait32(y);
+#pragma unroll
+      for (int j = 0; j < 32; j += 2)
+        acc = __ffma2_rn(make_float2(y[j], y[j + 1]), make_float2(y[j], y[j + 1]), acc);
+    }
+    const float n2 = acc.x + acc.y;
+    const float nk = sqrtf(n2);
+    const bool zero = !(n2 > 0.f);
+    const float s128 = zero ? 0.f : 128.f / nk;
+    HalfBook hb = book;
+    if (zero) {
+      hb.C0 = 0.f;
+#pragma unroll
+      for (int c = 0; c < 3; ++c) hb.dC[c] = 0.f;
+      hb.dA = 0.f;
+      hb.C20 = 0.f;
+    }
+    float2 rr2 = make_float2(0.f, 0.f);
+    uint32_t chw[4][BM];   // code halfwords of the group's four chunks
+#pragma unroll
+    for (int qq = 0; qq < 2; ++qq) {
+      const int q = q0 + qq;
+      float y[32];
+      tmem_ld32(d1 + 32u * q, y);
+      tmem_wait32(y);
+      uint32_t hw[2 * BM], hw3[2] = {0u, 0u};
+#pragma unroll
+      for (int h = 0; h < 2 * BM; ++h) hw[h] = 0;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t rh[8], rl[8];
+#pragma unroll
+        for (int jp = 0; jp < 16; jp += 2) {
+          const int j0 = 16 * hh + jp;
+          float2 rp;
+          const uint2 bb = cell2<BM>(make_float2(y[j0], y[j0 + 1]), s128, hb, rp);
+          rr2 = __ffma2_rn(rp, rp, rr2);
+          const __half2 hi = __float22half2_rn(rp);
+          const float2 hf = __half22float2(hi);
+          const __half2 lo = __float22half2_rn(__ffma2_rn(hf, f2(-1.f), rp));
+          rh[jp >> 1] = *reinterpret_cast<const uint32_t*>(&hi);
+          rl[jp >> 1] = *reinterpret_cast<const uint32_t*>(&lo);
+#pragma unroll
+          for (int t2 = 0; t2 < 2; ++t2) {
+            // coordinate 32 qq + jc of the group: chunk 2 qq + uu, register ii, nibble e
+            const int jc = j0 + t2;
+            const uint32_t bits = t2 ? bb.y : bb.x;
+            const int rreg = jc >> 2, e = jc & 3, uu = rreg >> 2, ii = rreg & 3;
+            if constexpr (BM == 3) {
+              if (ii < 3)
+                hw[uu * 3 + ii] += bits << (4 * e);
+              else
+                hw3[uu] += bits << (4 * e);
+            } else if constexpr (BM == 2) {
+              hw[uu * 2 + (ii >> 1)] += bits << (4 * e + 2 * (ii & 1));
+            } else {
+              hw[uu] += bits << (4 * e + ii);
+            }
+          }
+        }
+        tmem_st8(d1 + 32u * q + 8u * hh, rh);
+        tmem_st8(d1 + 32u * q + 16u + 8u * hh, rl);
+      }
+      if constexpr (BM == 3) {
+#pragma unroll
+        for (int uu = 0; uu < 2; ++uu)
+#pragma unroll
+          for (int b = 0; b < 3; ++b) hw[uu * 3 + b] |= ((hw3[uu] >> b) & 0x1111u) << 3;
+      }
+      // the low halfword of each sum holds the complemented codes
+#pragma unroll
+      for (int uu = 0; uu < 2; ++uu)
+#pragma unroll
+        for (int w = 0; w < BM; ++w) chw[2 * qq + uu][w] = zero ? 0u : (~hw[uu * BM + w]) & 0xFFFFu;
+    }
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+    tc_fence_before();
+    mbar_arrive(bar(kBarRFull + slot));
+    if (!mbar_wait_warp(bar(kBarD2Full + slot), par, abort_flag, status)) break;
+    tc_fence_after();
+    // sign words: bit p of quarter word qq holds group sign coordinate
+    // 32 qq + 16 (p >> 4) + 4 (p & 3) + ((p >> 2) & 3), i.e. the sign
+    // halfwords of chunks 2 qq (low half) and 2 qq + 1 (high half)
+    uint32_t sw[2];
+#pragma unroll
+    for (int qq = 0; qq < 2; ++qq) {
+      uint32_t neg = 0;
+#pragma unroll
+      for (int hz = 1; hz >= 0; --hz) {
+        float z[16];
+        tmem_ld16(d2 + 32u * (q0 + qq) + 16u * hz, z);
+        tmem_wait16(z);
+#pragma unroll
+        for (int p = 15; p >= 0; --p) {
+          const int jj = 4 * (p & 3) + ((p >> 2) & 3);
+          neg = __funnelshift_l(__float_as_uint(z[jj]), neg, 1);
+        }
+      }
+      sw[qq] = zero ? 0xFFFFFFFFu : ~neg;
+    }
+    tc_fence_before();
+    mbar_arrive(bar(kBarD2Free + slot));
+    const int64_t t = sg.sub + i * sg.cph;
+    const int64_t b = t / sg.tps, st = t - b * sg.tps;
+    const int64_t s = st * kTile + row;
+    if (s < sg.S) {
+      const int64_t key = (b * sg.Hkv + sg.head) * sg.S + s;
+      // group row: chunks c = 0..3 of BM code halfwords and one sign halfword
+      uint32_t hv[4 * (BM + 1)];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+#pragma unroll
+        for (int w = 0; w < BM; ++w) hv[c * (BM + 1) + w] = chw[c][w];
+        hv[c * (BM + 1) + BM] = (sw[c >> 1] >> (16 * (c & 1))) & 0xFFFFu;
+      }
+      uint32_t wv[2 * (BM + 1)];
+#pragma unroll
+      for (int x = 0; x < 2 * (BM + 1); ++x) wv[x] = hv[2 * x] | (hv[2 * x + 1] << 16);
+      uint8_t* dst = payload + key * (8 * (BM + 1));
+      if constexpr (BM == 2) {
+#pragma unroll
+        for (int v = 0; v < 3; ++v) reinterpret_cast<uint2*>(dst)[v] = make_uint2(wv[2 * v], wv[2 * v + 1]);
+      } else {
+#pragma unroll
+        for (int v = 0; v < (BM + 1) / 2; ++v)
+          reinterpret_cast<uint4*>(dst)[v] = make_uint4(wv[4 * v], wv[4 * v + 1], wv[4 * v + 2], wv[4 * v + 3]);
+      }
+      const float rho = nk * sqrtf(rr2.x + rr2.y) * (1.0f / 128.f);
+      reinterpret_cast<uint32_t*>(norms)[key] = uint32_t(__half_as_ushort(__float2half_rn(nk))) |
+                                                (uint32_t(__half_as_ushort(__float2half_rn(rho))) << 16);
+    }
+  }
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");   // none in flight on an early exit
+}
+
+template <int BHI, int BLO>
+__global__ void __launch_bounds__(kThreadsTc, 1) quantize_split_tc_kernel(
+    const __grid_constant__ CUtensorMap key_map, int B, int Hkv, int64_t S, int cph,
+    const uint8_t* __restrict__ dimg, HalfBook book_hi, HalfBook book_lo, uint8_t* __restrict__ payload_hi,
+    uint16_t* __restrict__ norms_hi, uint8_t* __restrict__ payload_lo, uint16_t* __restrict__ norms_lo,
+    uint32_t* __restrict__ status) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* sbase = smem_raw + (base - raw);
+  const uint32_t bar0 = base + kOffBar;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sbase + kOffBar + 8 * kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + kOffBar + 8 * kNumBars + 4);
+  auto bar = [&](int i) { return bar0 + 8u * uint32_t(i); };
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  SplitGeom sg;
+  sg.S = S;
+  sg.tps = (S + kTile - 1) / kTile;
+  sg.Hkv = Hkv;
+  sg.head = int(blockIdx.x) / cph;
+  sg.cph = cph;
+  sg.sub = int(blockIdx.x) - sg.head * cph;
+  const int64_t head_tiles = int64_t(B) * sg.tps;
+  const int64_t my_tiles = head_tiles > sg.sub ? (head_tiles - sg.sub + cph - 1) / cph : 0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(kBarConst), 1);
+    for (int st = 0; st < kKeyStages; ++st) {
+      mbar_init(bar(kBarKFull + st), 1);
+      mbar_init(bar(kBarKEmpty + st), 1);
+    }
+    for (int sl = 0; sl < 2; ++sl) {
+      mbar_init(bar(kBarD1Full + sl), 1);
+      mbar_init(bar(kBarRFull + sl), kTeamThreads);
+      mbar_init(bar(kBarD2Full + sl), 1);
+      mbar_init(bar(kBarD2Free + sl), kTeamThreads);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(512));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      mbar_expect_tx(bar(kBarConst), kConstBytes);
+      const uint8_t* himg = dimg + size_t(sg.head) * 65536;   // M_h hi, lo
+      const uint8_t* pimg = dimg + size_t(Hkv) * 65536;       // diag(P_hi, P_lo)
+      for (int c = 0; c < 4; ++c) bulk_load(base + kOffRhi + 16384u * c, himg + 16384 * c, 16384u, bar(kBarConst));
+      for (int c = 0; c < 2; ++c) bulk_load(base + kOffP + 16384u * c, pimg + 16384 * c, 16384u, bar(kBarConst));
+      int64_t i = 0;
+      for (; i < my_tiles; ++i) {
+        const int kb = int(i % kKeyStages);
+        if (i >= kKeyStages &&
+            !mbar_wait(bar(kBarKEmpty + kb), uint32_t((i / kKeyStages - 1) & 1), abort_flag, status))
+          break;
+        const int64_t t = sg.sub + i * cph;
+        const int64_t b = t / sg.tps, st = t - b * sg.tps;
+        const int pair = int(b * Hkv + sg.head);
+        const uint32_t dst = base + kOffKey + 32768u * kb;
+        mbar_expect_tx(bar(kBarKFull + kb), 32768u);
+        tma_load_3d(dst, &key_map, 0, int(st * kTile), pair, bar(kBarKFull + kb));
+        tma_load_3d(dst + 16384u, &key_map, 64, int(st * kTile), pair, bar(kBarKFull + kb));
+      }
+      for (int64_t j = (i >= kKeyStages ? i - kKeyStages : 0); j < i; ++j)
+        mbar_drain(bar(kBarKFull + int(j % kKeyStages)), uint32_t((j / kKeyStages) & 1), abort_flag, status);
+      mbar_drain(bar(kBarConst), 0u, abort_flag, status);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      auto issue_mma1 = [&](int64_t i) -> bool {
+        const int sl = int(i & 1);
+        const int kb = int(i % kKeyStages);
+        if (!mbar_wait(bar(kBarKFull + kb), uint32_t((i / kKeyStages) & 1), abort_flag, status)) return false;
+        if (i >= 2 && !mbar_wait(bar(kBarD2Full + sl), uint32_t(((i >> 1) - 1) & 1), abort_flag, status))
+          return false;
+        tc_fence_after();
+        const uint32_t d1 = tmem + 256u * sl;
+        const uint32_t kbase = base + kOffKey + 32768u * kb;
+        uint32_t acc = 0;
+        for (int pass = 0; pass < 2; ++pass)
+          for (int kh = 0; kh < 2; ++kh)
+            for (int ks = 0; ks < 4; ++ks) {
+              const uint32_t off = 16384u * kh + 32u * ks;
+              mma_f16(d1, smem_desc(kbase + off), smem_desc(base + (pass ? kOffRlo : kOffRhi) + off), kIdescBf16,
+                      acc);
+              acc = 1;
+            }
+        mma_commit(bar(kBarD1Full + sl));
+        mma_commit(bar(kBarKEmpty + kb));
+        return true;
+      };
+      auto issue_mma2 = [&](int64_t i) -> bool {
+        const int sl = int(i & 1);
+        if (!mbar_wait(bar(kBarRFull + sl), uint32_t((i >> 1) & 1), abort_flag, status)) return false;
+        if (i >= 2 && !mbar_wait(bar(kBarD2Free + sl), uint32_t(((i >> 1) - 1) & 1), abort_flag, status))
+          return false;
+        tc_fence_after();
+        const uint32_t d1 = tmem + 256u * sl, d2 = d1 + 128u;
+        uint32_t acc = 0;
+        for (int pass = 0; pass < 2; ++pass) {
+          const uint32_t a_lo = pass == 1 ? 16u : 0u;
+          for (int k = 0; k < 8; ++k) {
+            const uint32_t a_tmem = d1 + 32u * uint32_t(k >> 1) + 8u * uint32_t(k & 1) + a_lo;
+            const uint32_t off = 16384u * uint32_t(k >> 2) + 32u * uint32_t(k & 3);
+            mma_f16_ts(d2, a_tmem, smem_desc(base + kOffP + off), kIdescF16, acc);
+            acc = 1;
+          }
+        }
+        mma_commit(bar(kBarD2Full + sl));
+        return true;
+      };
+      int64_t n1 = 0, n2 = 0;
+      bool ok = mbar_wait(bar(kBarConst), 0u, abort_flag, status);
+      if (ok && my_tiles > 0) {
+        ok = issue_mma1(0);
+        n1 += ok;
+      }
+      for (int64_t i = 0; ok && i < my_tiles; ++i) {
+        if (i + 1 < my_tiles) {
+          if (!issue_mma1(i + 1)) break;
+          ++n1;
+        }
+        if (!issue_mma2(i)) break;
+        ++n2;
+      }
+      if (n1 > 0) mbar_drain(bar(kBarD1Full + int((n1 - 1) & 1)), uint32_t(((n1 - 1) >> 1) & 1), abort_flag, status);
+      if (n2 > 0) mbar_drain(bar(kBarD2Full + int((n2 - 1) & 1)), uint32_t(((n2 - 1) >> 1) & 1), abort_flag, status);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    // warp w: TMEM slot ((w - 2) >> 2) & 1, half (w - 2) >> 3 = group (0 high, 1 low)
+    const int eg = (warp - 2) >> 2;
+    const int slot = eg & 1, half = eg >> 1;
+    const int row = (warp & 3) * 32 + lane;
+    const uint32_t lane_addr = uint32_t((warp & 3) * 32) << 16;
+    const uint32_t d1 = tmem + 256u * slot + lane_addr, d2 = d1 + 128u;
+    if (half == 0)
+      split_epilogue<BHI>(bar0, d1, d2, slot, 0, row, my_tiles, sg, book_hi, payload_hi, norms_hi, abort_flag,
+                          status);
+    else
+      split_epilogue<BLO>(bar0, d1, d2, slot, 2, row, my_tiles, sg, book_lo, payload_lo, norms_lo, abort_flag,
+                          status);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+  }
+}
+
+HalfBook make_halfbook(const tq_ctx* ctx) {
+  HalfBook hb{};
+  const int L = ctx->levels;
+  for (int i = 0; i < L / 2 - 1; ++i) hb.Tneg[i] = -float(128.0 * ctx->t[L / 2 + i]) * 0x1p100f;
+  hb.C0 = float(128.0 * ctx->c[L / 2]);
+  for (int i = 0; i + 1 < L / 2; ++i) hb.dC[i] = float(128.0 * ctx->c[L / 2 + i + 1]) - float(128.0 * ctx->c[L / 2 + i]);
+  if (L == 8) {
+    hb.dT31 = hb.Tneg[2] - hb.Tneg[0];
+    hb.dA = hb.dC[2] - hb.dC[0];
+    hb.C20 = float(128.0 * ctx->c[L / 2 + 2]) - hb.C0;
+  }
+  return hb;
+}
+
 }  // namespace
 
 bool quantize_tc_supported(const tq_ctx* ctx, int dtype, int64_t ld, const void* keys) {
@@ -495,16 +842,7 @@ cudaError_t launch_quantize_tc(const tq_ctx* ctx, const void* keys, int dtype, i
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t tiles = (n + kTile - 1) / kTile;
   const int grid = int(tiles < sms ? tiles : sms);
-  HalfBook hb{};
-  const int L = ctx->levels;
-  for (int i = 0; i < L / 2 - 1; ++i) hb.Tneg[i] = -float(128.0 * ctx->t[L / 2 + i]) * 0x1p100f;
-  hb.C0 = float(128.0 * ctx->c[L / 2]);
-  for (int i = 0; i + 1 < L / 2; ++i) hb.dC[i] = float(128.0 * ctx->c[L / 2 + i + 1]) - float(128.0 * ctx->c[L / 2 + i]);
-  if (L == 8) {
-    hb.dT31 = hb.Tneg[2] - hb.Tneg[0];
-    hb.dA = hb.dC[2] - hb.dC[0];
-    hb.C20 = float(128.0 * ctx->c[L / 2 + 2]) - hb.C0;
-  }
+  const HalfBook hb = make_halfbook(ctx);
   switch (ctx->bmse) {
     case 1: {
       auto k = quantize_tc_kernel<1>;
@@ -526,6 +864,61 @@ cudaError_t launch_quantize_tc(const tq_ctx* ctx, const void* keys, int dtype, i
     }
   }
   return cudaGetLastError();
+}
+
+bool split_tc_supported(const tq_split* sp, int dtype, const void* keys) {
+  return sp->dimg != nullptr && dtype == TQ_BF16 && (reinterpret_cast<uintptr_t>(keys) & 15) == 0 &&
+         device_is_sm100() && get_encode() != nullptr;
+}
+
+namespace {
+
+template <int BHI, int BLO>
+cudaError_t launch_split_kernel(dim3 grid, cudaStream_t st, const CUtensorMap& map, int B, int Hkv, int64_t S,
+                                int cph, const uint8_t* dimg, const HalfBook& bh, const HalfBook& bl,
+                                uint8_t* ph, uint16_t* nh, uint8_t* pl, uint16_t* nl, uint32_t* status) {
+  auto k = quantize_split_tc_kernel<BHI, BLO>;
+  cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
+  k<<<grid, kThreadsTc, kSmemBytes, st>>>(map, B, Hkv, S, cph, dimg, bh, bl, ph, nh, pl, nl, status);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_split_quantize_tc(const tq_split* sp, const void* keys, int B, int64_t S, uint8_t* payload_hi,
+                                     uint16_t* norms_hi, uint8_t* payload_lo, uint16_t* norms_lo, cudaStream_t st) {
+  CUtensorMap map;
+  const int Hkv = sp->Hkv;
+  const cuuint64_t dims[3] = {cuuint64_t(kD), cuuint64_t(S), cuuint64_t(int64_t(B) * Hkv)};
+  const cuuint64_t strides[2] = {cuuint64_t(kD) * 2, cuuint64_t(S) * kD * 2};
+  const cuuint32_t box[3] = {64u, 128u, 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUresult r = get_encode()(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(keys), dims, strides,
+                                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t head_tiles = int64_t(B) * ((S + kTile - 1) / kTile);
+  int64_t cph = sms / Hkv > 1 ? sms / Hkv : 1;
+  if (cph > head_tiles) cph = head_tiles;
+  const dim3 grid(unsigned(Hkv * cph));
+  const HalfBook bh = make_halfbook(sp->hi), bl = make_halfbook(sp->lo);
+  uint32_t* status = sp->hi->dstatus;
+  const uint8_t* img = sp->dimg;
+  const int c = int(cph);
+  switch (sp->hi->bmse * 4 + sp->lo->bmse) {
+    case 5: return launch_split_kernel<1, 1>(grid, st, map, B, Hkv, S, c, img, bh, bl, payload_hi, norms_hi, payload_lo, norms_lo, status);
+    case 6: return launch_split_kernel<1, 2>(grid, st, map, B, Hkv, S, c, img, bh, bl, payload_hi, norms_hi, payload_lo, norms_lo, status);
+    case 7: return launch_split_kernel<1, 3>(grid, st, map, B, Hkv, S, c, img, bh, bl, payload_hi, norms_hi, payload_lo, norms_lo, status);
+    case 9: return launch_split_kernel<2, 1>(grid, st, map, B, Hkv, S, c, img, bh, bl, payload_hi, norms_hi, payload_lo, norms_lo, status);
+    case 10: return launch_split_kernel<2, 2>(grid, st, map, B, Hkv, S, c, img, bh, bl, payload_hi, norms_hi, payload_lo, norms_lo, status);
+    case 11: return launch_split_kernel<2, 3>(grid, st, map, B, Hkv, S, c, img, bh, bl, payload_hi, norms_hi, payload_lo, norms_lo, status);
+    case 13: return launch_split_kernel<3, 1>(grid, st, map, B, Hkv, S, c, img, bh, bl, payload_hi, norms_hi, payload_lo, norms_lo, status);
+    case 14: return launch_split_kernel<3, 2>(grid, st, map, B, Hkv, S, c, img, bh, bl, payload_hi, norms_hi, payload_lo, norms_lo, status);
+    default: return launch_split_kernel<3, 3>(grid, st, map, B, Hkv, S, c, img, bh, bl, payload_hi, norms_hi, payload_lo, norms_lo, status);
+  }
 }
 
 }  // namespace tq

@@ -28,6 +28,15 @@ struct CodeLut {
   float inv_scale;
 };
 
+// Channel gather of the split (per KV head channel order): group coordinate
+// j of key row `row` is channel perm[((row / S) % Hkv) * dtot + off + j] of a
+// row of dtot channels.  perm == nullptr: no gather (coordinate j = column j).
+struct ChannelGather {
+  const int32_t* perm;
+  int64_t S;
+  int Hkv, dtot, off;
+};
+
 }  // namespace tq
 
 struct tq_ctx {
@@ -51,6 +60,17 @@ struct tq_ctx {
   tq::CodeLut lut;
 };
 
+// A per-KV-head channel split of d = hi->d + lo->d channels into two groups,
+// each quantised with its own context (see tq.h, "Channel split").
+struct tq_split {
+  const tq_ctx* hi = nullptr;
+  const tq_ctx* lo = nullptr;
+  int d = 0, Hkv = 0, device = 0;
+  int32_t* dperm = nullptr;   // [Hkv][d] channel of group coordinate p (p < hi->d: high group)
+  uint8_t* dimg = nullptr;    // tensor-core operands of the fast path: per head M_h hi / lo (64 KB), then
+                              // the block-diagonal JL samples (32 KB); nullptr without a fast path
+};
+
 namespace tq {
 
 // Device status bits (set by bounded waits that gave up).
@@ -61,7 +81,8 @@ void set_cuda_error(cudaError_t e);
 
 // Kernel launchers (defined in the .cu files).  All return cudaGetLastError().
 cudaError_t launch_quantize_simt(const tq_ctx* ctx, const void* keys, int dtype, int64_t n, int64_t ld,
-                                 uint8_t* payload, uint16_t* norms, cudaStream_t st);
+                                 uint8_t* payload, uint16_t* norms, cudaStream_t st,
+                                 ChannelGather gather = ChannelGather{nullptr, 1, 1, 0, 0});
 bool quantize_tc_supported(const tq_ctx* ctx, int dtype, int64_t ld, const void* keys);
 cudaError_t launch_quantize_tc(const tq_ctx* ctx, const void* keys, int dtype, int64_t n, int64_t ld,
                                uint8_t* payload, uint16_t* norms, cudaStream_t st);
@@ -72,6 +93,20 @@ size_t qprep_bytes(const tq_ctx* ctx, int64_t groups, int heads_per_group);
 cudaError_t launch_logits(const tq_ctx* ctx, const float* q, int B, int Hq, int Hkv, int64_t S,
                           const uint8_t* payload, const uint16_t* norms, float scale, float* out,
                           void* ws, cudaStream_t st);
+// CUDA-core logits of one group of a split: q rows of gather.dtot channels,
+// gathered per KV head; accumulate != 0 adds to out instead of overwriting.
+cudaError_t launch_logits_simt(const tq_ctx* ctx, const float* q, int B, int Hq, int Hkv, int64_t S,
+                               const uint8_t* payload, const uint16_t* norms, float scale, float* out,
+                               ChannelGather gather, int accumulate, cudaStream_t st);
+
+// Channel split (k_split.cu, k_quantize_tc.cu, k_logits.cu)
+size_t split_plan_ws_bytes(const tq_split* sp);
+cudaError_t launch_split_plan(tq_split* sp, const void* keys, int dtype, int B, int64_t S, void* ws,
+                              cudaStream_t st);
+cudaError_t launch_split_images(tq_split* sp, cudaStream_t st);
+bool split_tc_supported(const tq_split* sp, int dtype, const void* keys);
+cudaError_t launch_split_quantize_tc(const tq_split* sp, const void* keys, int B, int64_t S, uint8_t* payload_hi,
+                                     uint16_t* norms_hi, uint8_t* payload_lo, uint16_t* norms_lo, cudaStream_t st);
 size_t topk_ws_bytes(const tq_ctx* ctx, int64_t nq, int64_t n, int k);
 bool search_tc_supported(const tq_ctx* ctx, int64_t nq, int64_t n, int k);
 size_t search_ws_bytes(const tq_ctx* ctx, int64_t nq, int64_t n);

@@ -55,6 +55,15 @@ def lib() -> ctypes.CDLL:
             "tq_topk_workspace_bytes": (sz, [vp, i64, i64, i32]),
             "tq_topk": (i32, [vp, vp, i64, vp, vp, i64, i32, vp, vp, vp, sz, vp]),
             "tq_check_device_status": (i32, [vp, vp, ctypes.POINTER(u32)]),
+            "tq_split_create": (i32, [vp, vp, i32, ctypes.POINTER(vp)]),
+            "tq_split_free": (None, [vp]),
+            "tq_split_plan_workspace_bytes": (sz, [vp]),
+            "tq_split_plan": (i32, [vp, vp, i32, i32, i64, vp, sz, vp]),
+            "tq_split_set_plan": (i32, [vp, vp]),
+            "tq_split_get_plan": (i32, [vp, vp]),
+            "tq_split_quantize": (i32, [vp, vp, i32, i32, i64, vp, vp, vp, vp, vp]),
+            "tq_split_logits_workspace_bytes": (sz, [vp, i32, i32]),
+            "tq_split_logits": (i32, [vp, vp, i32, i32, i64, vp, vp, vp, vp, f32, vp, vp, sz, vp]),
             "tq_strerror": (ctypes.c_char_p, [i32]),
             "tq_last_cuda_error": (ctypes.c_char_p, []),
         }
@@ -68,7 +77,9 @@ def lib() -> ctypes.CDLL:
 
 EXPORTED = ["tq_init", "tq_init_ex", "tq_host_tables", "tq_free", "tq_info", "tq_export_tables", "tq_quantize", "tq_dequantize",
             "tq_logits_workspace_bytes", "tq_logits", "tq_logits_noalloc", "tq_topk_workspace_bytes", "tq_topk",
-            "tq_check_device_status", "tq_strerror", "tq_last_cuda_error"]
+            "tq_check_device_status", "tq_strerror", "tq_last_cuda_error", "tq_split_create", "tq_split_free",
+            "tq_split_plan_workspace_bytes", "tq_split_plan", "tq_split_set_plan", "tq_split_get_plan",
+            "tq_split_quantize", "tq_split_logits_workspace_bytes", "tq_split_logits"]
 
 
 def _check(status: int, what: str):
@@ -260,3 +271,111 @@ def tq_check_device_status(ctx: Context, stream=None) -> int:
     if st not in (0, 6):
         _check(st, "tq_check_device_status")
     return w.value
+
+
+class Split:
+    """A per-KV-head channel split between two contexts (high group: hi, low group: lo)."""
+
+    def __init__(self, hi: Context, lo: Context, Hkv: int):
+        h = ctypes.c_void_p()
+        _check(lib().tq_split_create(hi.handle, lo.handle, Hkv, ctypes.byref(h)), "tq_split_create")
+        self._h = h
+        self.hi, self.lo, self.Hkv, self.d = hi, lo, Hkv, hi.d + lo.d
+
+    @property
+    def handle(self):
+        return self._h
+
+    def plan(self, keys: torch.Tensor, workspace: torch.Tensor | None = None, stream=None):
+        """Choose the channel order from keys (B, Hkv, S, d) on the device."""
+        _need_cuda(keys, "keys")
+        if keys.dim() != 4 or keys.shape[1] != self.Hkv or keys.shape[3] != self.d:
+            raise ValueError("keys must be (B, Hkv, S, d)")
+        dtype = {torch.float32: TQ_F32, torch.bfloat16: TQ_BF16}.get(keys.dtype)
+        if dtype is None:
+            raise ValueError("keys must be float32 or bfloat16")
+        ws_bytes = int(lib().tq_split_plan_workspace_bytes(self._h))
+        if workspace is None:
+            workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=keys.device)
+        _check(lib().tq_split_plan(self._h, _ptr(keys), dtype, keys.shape[0], keys.shape[2], _ptr(workspace),
+                                   workspace.numel(), ctypes.c_void_p(_stream(stream))), "tq_split_plan")
+
+    def set_plan(self, perm):
+        import numpy as np
+
+        p = np.ascontiguousarray(perm, dtype=np.int32)
+        if p.shape != (self.Hkv, self.d):
+            raise ValueError("perm must be (Hkv, d)")
+        _check(lib().tq_split_set_plan(self._h, p.ctypes.data), "tq_split_set_plan")
+
+    def get_plan(self):
+        import numpy as np
+
+        p = np.empty((self.Hkv, self.d), dtype=np.int32)
+        _check(lib().tq_split_get_plan(self._h, p.ctypes.data), "tq_split_get_plan")
+        return p
+
+    def close(self):
+        if getattr(self, "_h", None):
+            lib().tq_split_free(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def tq_split_create(hi: Context, lo: Context, Hkv: int) -> Split:
+    return Split(hi, lo, Hkv)
+
+
+def tq_split_quantize(sp: Split, keys: torch.Tensor, payload_hi=None, norms_hi=None, payload_lo=None, norms_lo=None,
+                      stream=None):
+    """keys (B, Hkv, S, d) -> (payload_hi, norms_hi, payload_lo, norms_lo), rows (B, Hkv, S)."""
+    _need_cuda(keys, "keys")
+    if keys.dim() != 4 or keys.shape[1] != sp.Hkv or keys.shape[3] != sp.d:
+        raise ValueError("keys must be (B, Hkv, S, d)")
+    dtype = {torch.float32: TQ_F32, torch.bfloat16: TQ_BF16}.get(keys.dtype)
+    if dtype is None:
+        raise ValueError("keys must be float32 or bfloat16")
+    B, _, S, _ = keys.shape
+    n = B * sp.Hkv * S
+    dev = keys.device
+    if payload_hi is None:
+        payload_hi = torch.empty((n, sp.hi.row_bytes), dtype=torch.uint8, device=dev)
+    if norms_hi is None:
+        norms_hi = torch.empty((n, 2), dtype=torch.float16, device=dev)
+    if payload_lo is None:
+        payload_lo = torch.empty((n, sp.lo.row_bytes), dtype=torch.uint8, device=dev)
+    if norms_lo is None:
+        norms_lo = torch.empty((n, 2), dtype=torch.float16, device=dev)
+    _check(lib().tq_split_quantize(sp.handle, _ptr(keys), dtype, B, S, _ptr(payload_hi), _ptr(norms_hi),
+                                   _ptr(payload_lo), _ptr(norms_lo), ctypes.c_void_p(_stream(stream))),
+           "tq_split_quantize")
+    return payload_hi, norms_hi, payload_lo, norms_lo
+
+
+def tq_split_logits(sp: Split, q: torch.Tensor, payload_hi, norms_hi, payload_lo, norms_lo, scale: float = 1.0,
+                    out: torch.Tensor | None = None, workspace: torch.Tensor | None = None, stream=None):
+    """q (B, Hq, d) fp32 against a split cache -> logits (B, Hq, S) fp32."""
+    _need_cuda(q, "q")
+    for t, nm in ((payload_hi, "payload_hi"), (norms_hi, "norms_hi"), (payload_lo, "payload_lo"),
+                  (norms_lo, "norms_lo")):
+        _need_cuda(t, nm)
+    if q.dtype != torch.float32 or q.dim() != 3 or q.shape[2] != sp.d:
+        raise ValueError("q must be float32 (B, Hq, d)")
+    B, Hq, _ = q.shape
+    if payload_hi.shape[0] % (B * sp.Hkv) or payload_lo.shape[0] != payload_hi.shape[0]:
+        raise ValueError("payload rows must be B * Hkv * S")
+    S = payload_hi.shape[0] // (B * sp.Hkv)
+    if out is None:
+        out = torch.empty((B, Hq, S), dtype=torch.float32, device=q.device)
+    ws_bytes = int(lib().tq_split_logits_workspace_bytes(sp.handle, B, Hq))
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=q.device)
+    _check(lib().tq_split_logits(sp.handle, _ptr(q), B, Hq, S, _ptr(payload_hi), _ptr(norms_hi), _ptr(payload_lo),
+                                 _ptr(norms_lo), float(scale), _ptr(out), _ptr(workspace), workspace.numel(),
+                                 ctypes.c_void_p(_stream(stream))), "tq_split_logits")
+    return out

@@ -185,6 +185,75 @@ tq_status tq_topk(const tq_ctx* ctx, const float* q, int64_t nq, const uint8_t* 
                   const uint16_t* norms, int64_t n, int k, int64_t* ids, float* scores,
                   void* workspace, size_t workspace_bytes, void* stream);
 
+/* ------------------------------------------------------------------------
+ * Channel split: fractional bit rates such as 2.5 bits per channel
+ * (arXiv summary page: "3.5 bits per channel"; mooersco.com section 2.1:
+ * "TurboQuant 2.5bit >= 7x"; zhengruan.com: 2.5 bits costs a slight drop).
+ * The pages do not say how a fractional rate is reached; this library's
+ * reading: per KV head, the channels are split into a high-variance group and
+ * a low-variance group (mooersco.com FAQ: unrotated channel variances differ
+ * by orders of magnitude), each group is quantised as its own vector with its
+ * own context (rotation, JL matrix, codebook, bit width), and the estimate of
+ * <q, k> is the sum of the two groups' estimates, since
+ * <q, k> = <q_hi, k_hi> + <q_lo, k_lo> for the same split of q and k.
+ * 2.5 bits per channel at d = 128: 64 channels at bits = 3 plus 64 at 2.
+ *
+ * A split holds, per KV head h, a channel order perm[h][0 .. d-1] (d =
+ * hi.d + lo.d): group coordinate p < hi.d of head h is key channel
+ * perm[h][p] of the high group, coordinate hi.d + p is channel
+ * perm[h][hi.d + p] of the low group.  It starts as the identity order.
+ * Keys are [B][Hkv][S][d] rows (row-major, contiguous); each group is stored
+ * in its own context's packed layout, rows in the same [B][Hkv][S] order.
+ * ------------------------------------------------------------------------ */
+typedef struct tq_split tq_split;
+
+/* A split for Hkv KV heads between the contexts hi and lo (same device, the
+ * current one; hi.d + lo.d <= 512).  The contexts must outlive the split.
+ * Library-owned; release with tq_split_free.  The tensor-core quantizer
+ * covers hi.d = lo.d = hi.m = lo.m = 64 with bf16 keys; other shapes run on
+ * CUDA cores. */
+tq_status tq_split_create(const tq_ctx* hi, const tq_ctx* lo, int Hkv, tq_split** out);
+void tq_split_free(tq_split* sp);
+
+/* Workspace bytes of tq_split_plan (fp64 partial sums). */
+size_t tq_split_plan_workspace_bytes(const tq_split* sp);
+
+/* Choose the channel order from keys [B][Hkv][S][d] (fp32 or bf16, device):
+ * per KV head, the hi.d channels of largest variance over the head's B S
+ * keys, ties to the lower channel index, in ascending channel order, then
+ * the other channels in ascending order.  With no keys (B S = 0) every
+ * variance is 0 and the order is the identity.  Asynchronous on `stream`;
+ * workspace: device, 8-byte aligned, >= tq_split_plan_workspace_bytes. */
+tq_status tq_split_plan(tq_split* sp, const void* keys, tq_dtype dtype, int B, int64_t S, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
+/* Set (host perm, [Hkv][d], each row a permutation of 0..d-1, else
+ * TQ_ERR_ARG) or read (host out-param) the channel order.  Both synchronise
+ * the device. */
+tq_status tq_split_set_plan(tq_split* sp, const int32_t* perm);
+tq_status tq_split_get_plan(const tq_split* sp, int32_t* perm);
+
+/* Quantise keys [B][Hkv][S][d] (device, fp32 or bf16, 16-byte aligned): the
+ * high group of every row with hi into payload_hi / norms_hi (B Hkv S rows of
+ * hi's layout), the low group with lo into payload_lo / norms_lo.  Each group
+ * is quantised exactly as tq_quantize quantises a key of that group's
+ * channels. */
+tq_status tq_split_quantize(const tq_split* sp, const void* keys, tq_dtype dtype, int B, int64_t S,
+                            uint8_t* payload_hi, uint16_t* norms_hi, uint8_t* payload_lo, uint16_t* norms_lo,
+                            void* stream);
+
+/* Workspace bytes of tq_split_logits. */
+size_t tq_split_logits_workspace_bytes(const tq_split* sp, int B, int Hq);
+
+/* Decode logits against a split cache: out[b, h, s] = scale (estimate of the
+ * high group + estimate of the low group), each group's estimate as in
+ * tq_logits with the query's channels gathered by the split of its KV head
+ * h / (Hq / Hkv).  q: device fp32 [B, Hq, d]; out: device fp32 [B, Hq, S];
+ * workspace: device, 256-byte aligned. */
+tq_status tq_split_logits(const tq_split* sp, const float* q, int B, int Hq, int64_t S, const uint8_t* payload_hi,
+                          const uint16_t* norms_hi, const uint8_t* payload_lo, const uint16_t* norms_lo,
+                          float scale, float* out, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Read (and clear) the context's device status word after synchronising the
  * stream: 0 when every kernel finished its bounded waits, otherwise a bit set
  * per kernel that gave up.  Returns TQ_ERR_DEVICE when nonzero. */

@@ -68,6 +68,19 @@ def test_argument_validation_without_device(L):
     assert lib.tq_info(None, None, None, None, None) == 1
     assert lib.tq_strerror(5) == b"workspace too small"
     lib.tq_free(None)
+    # channel split
+    import ctypes
+    h = ctypes.c_void_p()
+    assert lib.tq_split_create(None, None, 8, ctypes.byref(h)) == 1 and not h.value
+    assert lib.tq_split_create(None, None, 8, None) == 1
+    assert lib.tq_split_plan_workspace_bytes(None) == 0
+    assert lib.tq_split_logits_workspace_bytes(None, 1, 4) == 0
+    assert lib.tq_split_plan(None, None, 1, 1, 1, None, 0, None) == 1
+    assert lib.tq_split_set_plan(None, None) == 1
+    assert lib.tq_split_get_plan(None, None) == 1
+    assert lib.tq_split_quantize(None, None, 1, 1, 1, None, None, None, None, None) == 1
+    assert lib.tq_split_logits(None, None, 1, 4, 1, None, None, None, None, 1.0, None, None, 0, None) == 1
+    lib.tq_split_free(None)
 
 
 def test_row_bytes_formula():
