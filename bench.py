@@ -56,6 +56,9 @@ WORKLOAD = "decode_llama31_8b_layer_b8_hkv8_hq32_d128_s32768_b4"
 KV_WORKLOADS = {
     "decode": (8, 8, 32, 128, 32768, 4, 1001, "decode_llama31_8b_layer_b8_hkv8_hq32_d128_s32768_b4"),
     "longctx": (1, 8, 32, 128, 131072, 3, 1002, "longctx_prefill_decode_b1_hkv8_hq32_d128_s131072_b3"),
+    # 2.5 bits per channel: per KV head the 64 channels of largest variance at
+    # b = 3, the other 64 at b = 2, each group its own d = m = 64 quantizer
+    "split": (32, 8, 32, 128, 16384, (3, 2), 1003, "split25_b32_hkv8_hq32_d128_s16384_b3x64_b2x64"),
 }
 
 
@@ -143,44 +146,76 @@ class ClockSampler:
 
 
 def bytes_per_key():
-    row = D * (BITS - 1) // 8 + D // 8
-    return {"quantize_in": 2 * D, "quantize_out": row + 4, "logits_in": row + 4, "logits_out": 4 * (HQ // HKV)}
+    """Algorithmic bytes per key: bf16 key in; packed row(s) and fp16 norm pairs out;
+    the logits read those and write one fp32 logit per query head of the group."""
+    if isinstance(BITS, tuple):   # split: two groups of D / 2 channels
+        g = D // 2
+        row = sum(g * (b - 1) // 8 + g // 8 + 4 for b in BITS)
+    else:
+        row = D * (BITS - 1) // 8 + D // 8 + 4
+    return {"quantize_in": 2 * D, "quantize_out": row, "logits_in": row, "logits_out": 4 * (HQ // HKV)}
+
+
+def quantize_flops_per_key():
+    """Rotation and JL products: 2 d^2 + 2 m d per quantizer (per group for the split)."""
+    if isinstance(BITS, tuple):
+        g = D // 2
+        return 2 * (2 * g * g + 2 * g * g)
+    return 2 * D * D + 2 * D * D
 
 
 def cpu_baseline(budget_s: float = 12.0, max_keys: int = 1 << 19):
-    """The oracle, as it stands, on a bounded sample of the workload (host cores)."""
+    """The oracle, as it stands, on a bounded sample of the workload (host cores).
+
+    Timed: quantisation of the sampled keys and the estimates of their group's
+    query heads.  For the split, the channel plan of each sampled pair is
+    taken from the sample itself, outside the timed part (it is a one-time
+    calibration, not part of a step)."""
     import numpy as np
+    import torch
     from threadpoolctl import threadpool_info
 
     from compressed_kv_cache_tq_b200 import workloads as W
     from oracle import tq_oracle as O
 
-    tb = O.make_tables(D, BITS, SEED_TABLES)
+    split = isinstance(BITS, tuple)
+    if split:
+        tb_hi = O.make_tables(D // 2, BITS[0], SEED_TABLES)
+        tb_lo = O.make_tables(D // 2, BITS[1], SEED_TABLES + 1)
+    else:
+        tb = O.make_tables(D, BITS, SEED_TABLES)
     scales = W.head_channel_scales(HKV, D, SEED_KEYS)
     q = W.queries((B, HQ, D), seed=SEED_KEYS + 7)
     G = HQ // HKV
     chunk = 8192
-    done, t0 = 0, time.perf_counter()
+    done, busy = 0, 0.0
     for b in range(B):
         for h in range(HKV):
             keys = W.decode_keys_pair(b, h, S, D, scales, SEED_KEYS)
-            import torch
-
             kb = torch.from_numpy(keys).to(torch.bfloat16).to(torch.float64).numpy()
+            qh = q[b, h * G:(h + 1) * G].astype(np.float64)
             for s0 in range(0, S, chunk):
-                qz = O.quantize(kb[s0:s0 + chunk], tb)
-                O.estimate(q[b, h * G:(h + 1) * G].astype(np.float64), qz.codes, qz.bits, qz.n16, qz.rho16, tb)
-                done += min(chunk, S - s0)
-                if time.perf_counter() - t0 > budget_s or done >= max_keys:
+                kc = kb[s0:s0 + chunk]
+                if split:
+                    perm = O.split_plan(kc[None, None], D // 2)
+                    t0 = time.perf_counter()
+                    a, c = O.split_quantize(kc[None, None], perm, tb_hi, tb_lo)
+                    O.split_gqa_logits(qh[None], perm, a, c, tb_hi, tb_lo, 1, 1, len(kc))
+                else:
+                    t0 = time.perf_counter()
+                    qz = O.quantize(kc, tb)
+                    O.estimate(qh, qz.codes, qz.bits, qz.n16, qz.rho16, tb)
+                busy += time.perf_counter() - t0
+                done += len(kc)
+                if busy > budget_s or done >= max_keys:
                     break
-            if time.perf_counter() - t0 > budget_s or done >= max_keys:
+            if busy > budget_s or done >= max_keys:
                 break
-        if time.perf_counter() - t0 > budget_s or done >= max_keys:
+        if busy > budget_s or done >= max_keys:
             break
-    dt = time.perf_counter() - t0
     threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
-    return {"value": done / dt, "unit": "keys/s", "cores": threads, "kind": "oracle",
-            "sample": f"{done} of {B * HKV * S} keys (quantize + {HQ // HKV}-head estimates), {dt:.1f} s, fp64 numpy"}
+    return {"value": done / busy, "unit": "keys/s", "cores": threads, "kind": "oracle",
+            "sample": f"{done} of {B * HKV * S} keys (quantize + {G}-head estimates), {busy:.1f} s, fp64 numpy"}
 
 
 def run_search(args):
@@ -340,14 +375,15 @@ def result_line(*, world, n, steps, warmup, ms, q_ms, l_ms, e2e_ms, h2d, d2h, cl
     bpk = bytes_per_key()
     q_bytes = n * (bpk["quantize_in"] + bpk["quantize_out"])
     l_bytes = n * (bpk["logits_in"] + bpk["logits_out"])
+    kq, kl = ("tq_split_quantize", "tq_split_logits") if isinstance(BITS, tuple) else ("tq_quantize", "tq_logits")
+    fl = n * quantize_flops_per_key()
     kernels = {
-        "tq_quantize": {"ms": q_ms, "bytes": q_bytes, "GB/s": q_bytes / q_ms / 1e6,
-                        "vectors_per_s": n / q_ms * 1e3,
-                        "flops": n * (2 * D * D + 2 * D * D), "TFLOP/s": n * 4 * D * D / q_ms / 1e9},
-        "tq_logits": {"ms": l_ms, "bytes": l_bytes, "GB/s": l_bytes / l_ms / 1e6, "keys_per_s": n / l_ms * 1e3,
-                      "pct_of_8TBs": 100 * l_bytes / l_ms / 1e6 / 8000.0},
+        kq: {"ms": q_ms, "bytes": q_bytes, "GB/s": q_bytes / q_ms / 1e6, "vectors_per_s": n / q_ms * 1e3,
+             "flops": fl, "TFLOP/s": fl / q_ms / 1e9},
+        kl: {"ms": l_ms, "bytes": l_bytes, "GB/s": l_bytes / l_ms / 1e6, "keys_per_s": n / l_ms * 1e3,
+             "pct_of_8TBs": 100 * l_bytes / l_ms / 1e6 / 8000.0},
     }
-    dom = "tq_quantize" if q_ms >= l_ms else "tq_logits"
+    dom = kq if q_ms >= l_ms else kl
     ach = kernels[dom]["GB/s"]
     dram = DRAM_BYTES_PER_KEY.get(WORKLOAD.split("_")[0], {}).get(dom)
     return {
@@ -364,7 +400,10 @@ def result_line(*, world, n, steps, warmup, ms, q_ms, l_ms, e2e_ms, h2d, d2h, cl
         "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": WORKLOAD, "global_batch": B * world, "seq_len": S, "kv_heads": HKV,
-                   "q_heads": HQ, "head_dim": D, "bits": BITS, "parallelism": f"replicas x{world}",
+                   "q_heads": HQ, "head_dim": D,
+                   "bits": ({"high_64_channels": BITS[0], "low_64_channels": BITS[1]} if isinstance(BITS, tuple)
+                            else BITS),
+                   "parallelism": f"replicas x{world}",
                    "l2": f"inputs larger than L2: keys {n * D * 2 / 1e6:.0f} MB, packed caches "
                          f"{n * (bpk['quantize_out']) / 1e6:.0f} MB each; logits read the cache written one step "
                          "earlier, with the keys' traffic in between"},
@@ -389,7 +428,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="decode", choices=["decode", "longctx", "search"])
+    ap.add_argument("--workload", default="decode", choices=["decode", "longctx", "split", "search"])
     ap.add_argument("--rows", type=int, default=1_000_000, help="search: database rows")
     ap.add_argument("--queries", type=int, default=10_000, help="search: queries")
     ap.add_argument("--seq", type=int, default=None,
@@ -423,20 +462,55 @@ def main():
     from compressed_kv_cache_tq_b200 import tq, workloads as W
 
     dev = torch.device("cuda", local)
-    ctx = tq.tq_init(D, BITS, SEED_TABLES)
-    keys = W.decode_keys(B, HKV, S, D, SEED_KEYS, device=dev).reshape(-1, D)
+    keys4 = W.decode_keys(B, HKV, S, D, SEED_KEYS, device=dev)
+    keys = keys4.reshape(-1, D)
     n = keys.shape[0]
     q = torch.from_numpy(W.queries((B, HQ, D), seed=SEED_KEYS + 7)).to(dev)
-    caches = [(torch.empty((n, ctx.row_bytes), dtype=torch.uint8, device=dev),
-               torch.empty((n, 2), dtype=torch.float16, device=dev)) for _ in range(2)]
     out = torch.empty((B, HQ, S), dtype=torch.float32, device=dev)
-    ws = torch.empty(tq.tq_logits_workspace_bytes(ctx, B, HQ, HKV), dtype=torch.uint8, device=dev)
     scale = 1.0 / math.sqrt(D)
     stream = torch.cuda.current_stream()
+    extra = {}
+    if isinstance(BITS, tuple):
+        # split: plan the channel groups once from the keys (calibration, timed on its own)
+        hi, lo = tq.tq_init(D // 2, BITS[0], SEED_TABLES), tq.tq_init(D // 2, BITS[1], SEED_TABLES + 1)
+        ctx = hi
+        sp = tq.tq_split_create(hi, lo, HKV)
+        pws = torch.empty(max(1, int(tq.lib().tq_split_plan_workspace_bytes(sp.handle))), dtype=torch.uint8,
+                          device=dev)
+        sp.plan(keys4, workspace=pws)
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        sp.plan(keys4, workspace=pws)
+        b_.record(stream)
+        torch.cuda.synchronize()
+        extra["split_plan_ms"] = a.elapsed_time(b_)
+        caches = [(torch.empty((n, hi.row_bytes), dtype=torch.uint8, device=dev),
+                   torch.empty((n, 2), dtype=torch.float16, device=dev),
+                   torch.empty((n, lo.row_bytes), dtype=torch.uint8, device=dev),
+                   torch.empty((n, 2), dtype=torch.float16, device=dev)) for _ in range(2)]
+        ws = torch.empty(max(256, int(tq.lib().tq_split_logits_workspace_bytes(sp.handle, B, HQ))),
+                         dtype=torch.uint8, device=dev)
+
+        def quantize(k4, c):
+            tq.tq_split_quantize(sp, k4, *c)
+
+        def logits(qq, c):
+            tq.tq_split_logits(sp, qq, *c, scale=scale, out=out, workspace=ws)
+    else:
+        ctx = tq.tq_init(D, BITS, SEED_TABLES)
+        caches = [(torch.empty((n, ctx.row_bytes), dtype=torch.uint8, device=dev),
+                   torch.empty((n, 2), dtype=torch.float16, device=dev)) for _ in range(2)]
+        ws = torch.empty(tq.tq_logits_workspace_bytes(ctx, B, HQ, HKV), dtype=torch.uint8, device=dev)
+
+        def quantize(k4, c):
+            tq.tq_quantize(ctx, k4.reshape(-1, D), c[0], c[1])
+
+        def logits(qq, c):
+            tq.tq_logits(ctx, qq, c[0], c[1], HKV, scale=scale, out=out, workspace=ws)
 
     # fill both caches once so the first logits read valid data
     for c in caches:
-        tq.tq_quantize(ctx, keys, c[0], c[1])
+        quantize(keys4, c)
 
     ev = []
 
@@ -445,10 +519,10 @@ def main():
         if record:
             e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
             e[0].record(stream)
-        tq.tq_quantize(ctx, keys, cw[0], cw[1])
+        quantize(keys4, cw)
         if record:
             e[1].record(stream)
-        tq.tq_logits(ctx, q, cr[0], cr[1], HKV, scale=scale, out=out, workspace=ws)
+        logits(q, cr)
         if record:
             e[2].record(stream)
             ev.append(e)
@@ -474,19 +548,19 @@ def main():
     l_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / len(ev)
 
     # end to end through the public API: pinned host keys in, logits out
-    host_keys = torch.empty(keys.shape, dtype=keys.dtype, pin_memory=True)
-    host_keys.copy_(keys)
+    host_keys = torch.empty(keys4.shape, dtype=keys4.dtype, pin_memory=True)
+    host_keys.copy_(keys4)
     host_q = q.cpu().pin_memory()
     host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-    dkeys = torch.empty_like(keys)
+    dkeys = torch.empty_like(keys4)
     dq = torch.empty_like(q)
 
     def e2e_step(i):
         cw, cr = caches[i % 2], caches[(i + 1) % 2]
         dkeys.copy_(host_keys, non_blocking=True)
         dq.copy_(host_q, non_blocking=True)
-        tq.tq_quantize(ctx, dkeys, cw[0], cw[1])
-        tq.tq_logits(ctx, dq, cr[0], cr[1], HKV, scale=scale, out=out, workspace=ws)
+        quantize(dkeys, cw)
+        logits(dq, cr)
         host_out.copy_(out, non_blocking=True)
 
     e2e_steps = max(3, min(args.steps, 10))
@@ -509,6 +583,7 @@ def main():
     line = result_line(world=world, n=n, steps=args.steps, warmup=args.warmup, ms=ms, q_ms=q_ms, l_ms=l_ms,
                        e2e_ms=e2e_ms, h2d=int(keys.numel() * 2 + q.numel() * 4), d2h=int(out.numel() * 4),
                        clocks=clocks.summary())
+    line.update(extra)
     if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline()
     print(json.dumps(line), flush=True)

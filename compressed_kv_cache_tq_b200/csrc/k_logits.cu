@@ -499,6 +499,355 @@ cudaError_t launch_mma(const tq_ctx* ctx, int B, int Hq, int Hkv, int64_t S, con
   return cudaLaunchKernelEx(&cfg, kern, payload, norms, S, Hq, Hkv, total, frags, hs, ctx->lut, out);
 }
 
+// ---------------------------------------------------------------------------
+// Split cache (two groups of d = m = 64 channels per key, each with its own
+// context; see k_split.cu): the same int8 MMA scheme, group by group.  A
+// thread's quarter of a key is chunk tig of each group row (16 coordinates:
+// two k-steps per group).  The codes and signs of the two groups accumulate
+// separately because each group has its own norms and query scales; the
+// epilogue adds the four terms.
+// ---------------------------------------------------------------------------
+constexpr int GD = 64;          // group dimension of the split fast path
+constexpr int GKS = GD / 32;    // k-steps per group
+
+struct SplitScale {
+  float code[2];   // per group (0 high, 1 low): multiplies the int32 code dot product
+  float sign[2];
+};
+
+// Query preparation of the split: per (batch, KV head) group, the query's
+// channels gathered in the head's split order, x_g = R_g q_g and
+// y_g = P_g x_g (= S_g q_g) per group g, int16 fixed point per (head, group),
+// two int8 limbs, MMA B-fragment order: word
+// ((((nt 2 + g) 2 + xy) 2 + s) 2 + reg) 32 + lane holds K positions
+// k = 4 tig + e (reg 0) or 16 + 4 tig + e (reg 1) of step s, i.e. group
+// coordinates 16 tig + 4 (2 s + reg) + e, for column n = lane / 4 = (head
+// slot 4 nt + n / 2, limb n % 2).
+__global__ void __launch_bounds__(128) qprep_split_kernel(const float* __restrict__ q, int Hq, int Hkv,
+                                                          int nt_per_group, const int32_t* __restrict__ perm,
+                                                          const float* __restrict__ Rt_hi,
+                                                          const float* __restrict__ Pt_hi,
+                                                          const float* __restrict__ Rt_lo,
+                                                          const float* __restrict__ Pt_lo, float inv_hi, float inv_lo,
+                                                          float scale, float qjl_hi, float qjl_lo,
+                                                          uint32_t* __restrict__ frags,
+                                                          SplitScale* __restrict__ hscale) {
+  __shared__ float sq[kMaxSlots][2 * GD];   // gathered queries [high | low]
+  __shared__ float sx[kMaxSlots][2 * GD];
+  __shared__ float red[2][kMaxSlots][4];
+  __shared__ int8_t limbs[kMaxSlots][2][2][2 * GD];   // [slot][x/y][hi/lo limb][coordinate of high | low]
+  const int G = Hq / Hkv;
+  const int slots = nt_per_group * HPT;
+  const int grp = blockIdx.x, b = grp / Hkv, hkv = grp % Hkv;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gi = tid >> 6, j = tid & 63;   // group and group coordinate of this thread
+  asm volatile("griddepcontrol.launch_dependents;");
+  const int ch = perm[hkv * 2 * GD + tid];
+  for (int h = 0; h < slots; ++h) sq[h][tid] = h < G ? q[(size_t(b) * Hq + hkv * G + h) * (2 * GD) + ch] : 0.f;
+  __syncthreads();
+  const float* Rt = gi ? Rt_lo : Rt_hi;
+  const float* Pt = gi ? Pt_lo : Pt_hi;
+  float acc[kMaxSlots];
+#pragma unroll
+  for (int h = 0; h < kMaxSlots; ++h) acc[h] = 0.f;
+  for (int p = 0; p < GD; ++p) {
+    const float r = __ldg(Rt + p * GD + j);   // R_g[j][p]
+#pragma unroll
+    for (int h = 0; h < kMaxSlots; ++h)
+      if (h < slots) acc[h] = fmaf(r, sq[h][gi * GD + p], acc[h]);
+  }
+#pragma unroll
+  for (int h = 0; h < kMaxSlots; ++h)
+    if (h < slots) sx[h][tid] = acc[h];
+  __syncthreads();
+  float accy[kMaxSlots];
+#pragma unroll
+  for (int h = 0; h < kMaxSlots; ++h) accy[h] = 0.f;
+  for (int p = 0; p < GD; ++p) {
+    const float pv = __ldg(Pt + p * GD + j);  // P_g[j][p]
+#pragma unroll
+    for (int h = 0; h < kMaxSlots; ++h)
+      if (h < slots) accy[h] = fmaf(pv, sx[h][gi * GD + p], accy[h]);
+  }
+#pragma unroll
+  for (int h = 0; h < kMaxSlots; ++h) {
+    if (h >= slots) break;
+    float ax = fabsf(acc[h]), ay = fabsf(accy[h]);
+    for (int o = 16; o; o >>= 1) {
+      ax = fmaxf(ax, __shfl_xor_sync(0xffffffffu, ax, o));
+      ay = fmaxf(ay, __shfl_xor_sync(0xffffffffu, ay, o));
+    }
+    if (lane == 0) {
+      red[0][h][warp] = ax;
+      red[1][h][warp] = ay;
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int h = 0; h < kMaxSlots; ++h) {
+    if (h >= slots) break;
+    const float mx = fmaxf(red[0][h][2 * gi], red[0][h][2 * gi + 1]);
+    const float my = fmaxf(red[1][h][2 * gi], red[1][h][2 * gi + 1]);
+    const float kx = mx > 0.f ? 32000.f / mx : 0.f;
+    const float ky = my > 0.f ? 32000.f / my : 0.f;
+    const int xi = __float2int_rn(acc[h] * kx);
+    const int yi = __float2int_rn(accy[h] * ky);
+    const int xh = (xi + 128) >> 8, yh = (yi + 128) >> 8;
+    limbs[h][0][0][tid] = int8_t(xh);
+    limbs[h][0][1][tid] = int8_t(xi - 256 * xh);
+    limbs[h][1][0][tid] = int8_t(yh);
+    limbs[h][1][1][tid] = int8_t(yi - 256 * yh);
+    if (j == 0 && h < G) {
+      SplitScale* hs = hscale + size_t(b) * Hq + hkv * G + h;
+      hs->code[gi] = mx > 0.f ? scale * (gi ? inv_lo : inv_hi) / kx : 0.f;
+      hs->sign[gi] = my > 0.f ? scale * (gi ? qjl_lo : qjl_hi) / ky : 0.f;
+    }
+  }
+  __syncthreads();
+  for (int w = tid; w < nt_per_group * kFragWords; w += 128) {
+    const int ln = w & 31, reg = (w >> 5) & 1, st = (w >> 6) & 1, xy = (w >> 7) & 1, g2 = (w >> 8) & 1;
+    const int nt = w >> 9;
+    const int n = ln >> 2, tig = ln & 3;
+    const int slot = nt * HPT + (n >> 1), limb = n & 1;
+    uint32_t word = 0;
+    for (int e = 0; e < 4; ++e) {
+      const int jj = g2 * GD + tig * (GD / 4) + 4 * (2 * st + reg) + e;
+      word |= uint32_t(uint8_t(limbs[slot][xy][limb][jj])) << (8 * e);
+    }
+    frags[size_t(grp) * nt_per_group * kFragWords + w] = word;
+  }
+}
+
+// One group's chunk tig of a key (d = m = 64): BM code halfwords, then the
+// sign halfword, packed two per word (halfword i in word i / 2).
+template <int BM>
+struct GChunk {
+  uint32_t w[(BM + 2) / 2];
+  __device__ __forceinline__ uint32_t h(int i) const { return (i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xFFFFu); }
+};
+
+template <int BM>
+__device__ __forceinline__ void load_gchunk(GChunk<BM>& c, const uint8_t* row, int tig, bool ok) {
+  const uint8_t* p = row + tig * 2 * (BM + 1);
+  if constexpr (BM == 1) {
+    c.w[0] = ok ? __ldg(reinterpret_cast<const uint32_t*>(p)) : 0u;
+  } else if constexpr (BM == 3) {
+    const uint2 v = ok ? __ldg(reinterpret_cast<const uint2*>(p)) : make_uint2(0u, 0u);
+    c.w[0] = v.x;
+    c.w[1] = v.y;
+  } else {
+    // 6 bytes at a 2-byte boundary
+    const unsigned short* p16 = reinterpret_cast<const unsigned short*>(p);
+    c.w[0] = ok ? uint32_t(__ldg(p16)) | (uint32_t(__ldg(p16 + 1)) << 16) : 0u;
+    c.w[1] = ok ? uint32_t(__ldg(p16 + 2)) : 0u;
+  }
+}
+
+// Byte-permute selectors of the 4 registers of one unit (as code_selectors).
+template <int BM>
+__device__ __forceinline__ void gcode_selectors(const GChunk<BM>& c, uint32_t (&sel)[4]) {
+  if constexpr (BM == 3) {
+    const uint32_t h0 = c.h(0), h1 = c.h(1), h2 = c.h(2);
+    sel[0] = h0 & 0x7777u;
+    sel[1] = h1 & 0x7777u;
+    sel[2] = h2 & 0x7777u;
+    sel[3] = ((h0 >> 3) & 0x1111u) | ((h1 >> 2) & 0x2222u) | ((h2 >> 1) & 0x4444u);
+  } else if constexpr (BM == 2) {
+    sel[0] = c.h(0) & 0x3333u;
+    sel[1] = (c.h(0) >> 2) & 0x3333u;
+    sel[2] = c.h(1) & 0x3333u;
+    sel[3] = (c.h(1) >> 2) & 0x3333u;
+  } else {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) sel[i] = (c.h(0) >> i) & 0x1111u;
+  }
+}
+
+template <int BM>
+__device__ __forceinline__ void gsign_operands(const GChunk<BM>& c, uint32_t (&a)[4]) {
+  const uint32_t h = c.h(BM);
+  a[0] = prmt(0x000001FFu, 0u, h & 0x1111u);
+  a[1] = prmt(0x000100FFu, 0u, h & 0x2222u);
+  a[2] = prmt(0x000000FFu, 0x00000001u, h & 0x4444u);
+  a[3] = prmt(0x000000FFu, 0x00000001u, (h >> 1) & 0x4444u);
+}
+
+// Products of one group for a 16-key row tile: code planes (hi, lo) and signs.
+template <int BM, int NT>
+__device__ __forceinline__ void group_mma(const GChunk<BM>& ca, const GChunk<BM>& cb, const CodeLut& lut,
+                                          const uint32_t (&bx)[NT][GKS][2], const uint32_t (&by)[NT][GKS][2],
+                                          int (&ah)[NT][4], int (&al)[NT][4], int (&sg)[NT][4]) {
+  uint32_t sa[4], sb[4];
+  gcode_selectors<BM>(ca, sa);
+  gcode_selectors<BM>(cb, sb);
+#pragma unroll
+  for (int s = 0; s < GKS; ++s) {
+    const uint32_t h0 = prmt(lut.hi[0], lut.hi[1], sa[2 * s]), h1 = prmt(lut.hi[0], lut.hi[1], sb[2 * s]);
+    const uint32_t h2 = prmt(lut.hi[0], lut.hi[1], sa[2 * s + 1]), h3 = prmt(lut.hi[0], lut.hi[1], sb[2 * s + 1]);
+    const uint32_t l0 = prmt(lut.lo[0], lut.lo[1], sa[2 * s]), l1 = prmt(lut.lo[0], lut.lo[1], sb[2 * s]);
+    const uint32_t l2 = prmt(lut.lo[0], lut.lo[1], sa[2 * s + 1]), l3 = prmt(lut.lo[0], lut.lo[1], sb[2 * s + 1]);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      if (s == 0) {
+        mma_s8_first(ah[nt], h0, h1, h2, h3, bx[nt][s][0], bx[nt][s][1]);
+        mma_s8_first(al[nt], l0, l1, l2, l3, bx[nt][s][0], bx[nt][s][1]);
+      } else {
+        mma_s8(ah[nt], h0, h1, h2, h3, bx[nt][s][0], bx[nt][s][1]);
+        mma_s8(al[nt], l0, l1, l2, l3, bx[nt][s][0], bx[nt][s][1]);
+      }
+    }
+  }
+  uint32_t ga[4], gb[4];
+  gsign_operands<BM>(ca, ga);
+  gsign_operands<BM>(cb, gb);
+#pragma unroll
+  for (int s = 0; s < GKS; ++s)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      if (s == 0)
+        mma_s8_first(sg[nt], ga[0], gb[0], ga[1], gb[1], by[nt][0][0], by[nt][0][1]);
+      else
+        mma_s8(sg[nt], ga[2 * s], gb[2 * s], ga[2 * s + 1], gb[2 * s + 1], by[nt][s][0], by[nt][s][1]);
+    }
+}
+
+__device__ __forceinline__ float limb_sum(const int (&a)[4], const int (&b)[4], int r) {
+  // |cross terms| <= 2 * 64 * 128 * 128 and |low terms| < 2^20: the integer sums fit in 32 bits
+  return fmaf(float(a[r]), 65536.f, float((a[r + 1] + b[r]) * 256 + b[r + 1]));
+}
+
+template <int BHI, int BLO, int NT>
+__device__ __forceinline__ void split_row_tile(const GChunk<BHI>& ha, const GChunk<BHI>& hb, const GChunk<BLO>& la,
+                                               const GChunk<BLO>& lb, uint32_t nha, uint32_t nhb, uint32_t nla,
+                                               uint32_t nlb, bool okA, bool okB, const uint32_t (&bx)[2][NT][GKS][2],
+                                               const uint32_t (&by)[2][NT][GKS][2], const float (&sc)[NT][4],
+                                               float* const (&orow)[NT], int g, const CodeLut& lut_hi,
+                                               const CodeLut& lut_lo) {
+  int hh[NT][4], hl[NT][4], hs[NT][4], lh[NT][4], ll[NT][4], ls[NT][4];
+  group_mma<BHI, NT>(ha, hb, lut_hi, bx[0], by[0], hh, hl, hs);
+  group_mma<BLO, NT>(la, lb, lut_lo, bx[1], by[1], lh, ll, ls);
+  const float2 fha = __half22float2(*reinterpret_cast<const __half2*>(&nha));   // (||k_hi||, ||r_hi||) of key g
+  const float2 fhb = __half22float2(*reinterpret_cast<const __half2*>(&nhb));   // of key g + 8
+  const float2 fla = __half22float2(*reinterpret_cast<const __half2*>(&nla));
+  const float2 flb = __half22float2(*reinterpret_cast<const __half2*>(&nlb));
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    if (!orow[nt]) continue;
+    const float vA = fmaf(fha.x * sc[nt][0], limb_sum(hh[nt], hl[nt], 0),
+                          fmaf(fha.y * sc[nt][1], float(hs[nt][0] * 256 + hs[nt][1]),
+                               fmaf(fla.x * sc[nt][2], limb_sum(lh[nt], ll[nt], 0),
+                                    fla.y * sc[nt][3] * float(ls[nt][0] * 256 + ls[nt][1]))));
+    const float vB = fmaf(fhb.x * sc[nt][0], limb_sum(hh[nt], hl[nt], 2),
+                          fmaf(fhb.y * sc[nt][1], float(hs[nt][2] * 256 + hs[nt][3]),
+                               fmaf(flb.x * sc[nt][2], limb_sum(lh[nt], ll[nt], 2),
+                                    flb.y * sc[nt][3] * float(ls[nt][2] * 256 + ls[nt][3]))));
+    if (okA) orow[nt][g] = vA;
+    if (okB) orow[nt][g + 8] = vB;
+  }
+}
+
+template <int BHI, int BLO, int NT>
+__global__ void __launch_bounds__(kLogitThreads, NT == 1 ? 2 : 1) logits_split_kernel(
+    const uint8_t* __restrict__ payload_hi, const uint16_t* __restrict__ norms_hi,
+    const uint8_t* __restrict__ payload_lo, const uint16_t* __restrict__ norms_lo, int64_t S, int Hq, int Hkv,
+    int64_t total_tiles, const uint32_t* __restrict__ frags, const SplitScale* __restrict__ hscale, CodeLut lut_hi,
+    CodeLut lut_lo, float* __restrict__ out) {
+  constexpr int kRowHi = 8 * (BHI + 1), kRowLo = 8 * (BLO + 1);
+  const int lane = threadIdx.x & 31;
+  const int g = lane >> 2, tig = lane & 3;
+  const int64_t nwarps = int64_t(gridDim.x) * (kLogitThreads / 32);
+  const int64_t gw = int64_t(blockIdx.x) * (kLogitThreads / 32) + (threadIdx.x >> 5);
+  const int64_t t_begin = gw * total_tiles / nwarps, t_end = (gw + 1) * total_tiles / nwarps;
+  const int G = Hq / Hkv;
+  const int64_t tpp = (S + 31) / 32;
+  int64_t grp = t_begin / tpp;
+  int64_t s0 = (t_begin - grp * tpp) * 32;
+
+  auto load_tile = [&](int64_t gi, int64_t so, GChunk<BHI> (&ch)[4], GChunk<BLO> (&cl)[4], uint32_t (&nh)[4],
+                       uint32_t (&nl)[4]) {
+    const int64_t row0 = gi * S + so + g;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const bool ok = so + g + 8 * k < S;
+      load_gchunk<BHI>(ch[k], payload_hi + (row0 + 8 * k) * kRowHi, tig, ok);
+      load_gchunk<BLO>(cl[k], payload_lo + (row0 + 8 * k) * kRowLo, tig, ok);
+      nh[k] = ok ? __ldg(reinterpret_cast<const uint32_t*>(norms_hi) + row0 + 8 * k) : 0u;
+      nl[k] = ok ? __ldg(reinterpret_cast<const uint32_t*>(norms_lo) + row0 + 8 * k) : 0u;
+    }
+  };
+  GChunk<BHI> ch[4];
+  GChunk<BLO> cl[4];
+  uint32_t nh[4], nl[4];
+  if (t_begin < t_end) load_tile(grp, s0, ch, cl, nh, nl);
+
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (t_begin >= t_end) return;
+
+  uint32_t bx[2][NT][GKS][2], by[2][NT][GKS][2];
+  float sc[NT][4];
+  float* orow[NT];
+  auto load_group = [&](int64_t gi) {
+    const int b = int(gi / Hkv), hkv = int(gi - int64_t(b) * Hkv);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const uint32_t* fr = frags + (size_t(gi) * NT + nt) * kFragWords;
+#pragma unroll
+      for (int g2 = 0; g2 < 2; ++g2)
+#pragma unroll
+        for (int s = 0; s < GKS; ++s)
+#pragma unroll
+          for (int r = 0; r < 2; ++r) {
+            bx[g2][nt][s][r] = __ldg(fr + ((((g2 * 2 + 0) * 2 + s) * 2 + r) * 32) + lane);
+            by[g2][nt][s][r] = __ldg(fr + ((((g2 * 2 + 1) * 2 + s) * 2 + r) * 32) + lane);
+          }
+      const int hg = nt * HPT + tig;
+      const int hh = hg < G ? hg : 0;
+      const SplitScale hs = hscale[size_t(b) * Hq + hkv * G + hh];
+      sc[nt][0] = hs.code[0];
+      sc[nt][1] = hs.sign[0];
+      sc[nt][2] = hs.code[1];
+      sc[nt][3] = hs.sign[1];
+      orow[nt] = hg < G ? out + (size_t(b) * Hq + hkv * G + hh) * S : nullptr;
+    }
+  };
+  load_group(grp);
+
+  for (int64_t t = t_begin; t < t_end; ++t) {
+    int64_t ngrp = grp, ns0 = s0 + 32;
+    if (ns0 >= S) {
+      ns0 = 0;
+      ++ngrp;
+    }
+    GChunk<BHI> nch[4];
+    GChunk<BLO> ncl[4];
+    uint32_t nnh[4] = {0u, 0u, 0u, 0u}, nnl[4] = {0u, 0u, 0u, 0u};
+    if (t + 1 < t_end) load_tile(ngrp, ns0, nch, ncl, nnh, nnl);
+
+    float* orow_t[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) orow_t[nt] = orow[nt] ? orow[nt] + s0 : nullptr;
+    split_row_tile<BHI, BLO, NT>(ch[0], ch[1], cl[0], cl[1], nh[0], nh[1], nl[0], nl[1], s0 + g < S,
+                                 s0 + g + 8 < S, bx, by, sc, orow_t, g, lut_hi, lut_lo);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) orow_t[nt] = orow[nt] ? orow[nt] + s0 + 16 : nullptr;
+    split_row_tile<BHI, BLO, NT>(ch[2], ch[3], cl[2], cl[3], nh[2], nh[3], nl[2], nl[3], s0 + g + 16 < S,
+                                 s0 + g + 24 < S, bx, by, sc, orow_t, g, lut_hi, lut_lo);
+
+    if (t + 1 < t_end) {
+      if (ngrp != grp) load_group(ngrp);
+      grp = ngrp;
+      s0 = ns0;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        ch[k] = nch[k];
+        cl[k] = ncl[k];
+        nh[k] = nnh[k];
+        nl[k] = nnl[k];
+      }
+    }
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_logits_simt(const tq_ctx* ctx, const float* q, int B, int Hq, int Hkv, int64_t S,
@@ -547,6 +896,93 @@ cudaError_t launch_logits(const tq_ctx* ctx, const float* q, int B, int Hq, int 
     case 31: return launch_mma<3, 1>(ctx, B, Hq, Hkv, S, payload, norms, out, frags, hs, st);
     default: return launch_mma<3, 2>(ctx, B, Hq, Hkv, S, payload, norms, out, frags, hs, st);
   }
+}
+
+namespace {
+
+bool split_fast_path(const tq_split* sp, int G) {
+  return sp->d == 2 * GD && sp->hi->d == GD && sp->lo->d == GD && sp->hi->m == GD && sp->lo->m == GD &&
+         sp->hi->bmse >= 1 && sp->hi->bmse <= 3 && sp->lo->bmse >= 1 && sp->lo->bmse <= 3 && G <= 8;
+}
+
+template <int BHI, int BLO, int NT>
+cudaError_t launch_split_mma(const tq_split* sp, int B, int Hq, int64_t S, const uint8_t* ph, const uint16_t* nh,
+                             const uint8_t* pl, const uint16_t* nl, float* out, const uint32_t* frags,
+                             const SplitScale* hs, cudaStream_t st) {
+  const int Hkv = sp->Hkv;
+  const int64_t total = int64_t(B) * Hkv * ((S + 31) / 32);
+  auto kern = logits_split_kernel<BHI, BLO, NT>;
+  int per_sm = 1;
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kLogitThreads, 0);
+  int64_t grid = int64_t(sm_count()) * (per_sm > 0 ? per_sm : 1);
+  const int64_t needed = (total + kLogitThreads / 32 - 1) / (kLogitThreads / 32);
+  if (grid > needed) grid = needed;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(grid));
+  cfg.blockDim = dim3(kLogitThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, ph, nh, pl, nl, S, Hq, Hkv, total, frags, hs, sp->hi->lut, sp->lo->lut, out);
+}
+
+template <int NT>
+cudaError_t dispatch_split(const tq_split* sp, int B, int Hq, int64_t S, const uint8_t* ph, const uint16_t* nh,
+                           const uint8_t* pl, const uint16_t* nl, float* out, const uint32_t* frags,
+                           const SplitScale* hs, cudaStream_t st) {
+  switch (sp->hi->bmse * 4 + sp->lo->bmse) {
+    case 5: return launch_split_mma<1, 1, NT>(sp, B, Hq, S, ph, nh, pl, nl, out, frags, hs, st);
+    case 6: return launch_split_mma<1, 2, NT>(sp, B, Hq, S, ph, nh, pl, nl, out, frags, hs, st);
+    case 7: return launch_split_mma<1, 3, NT>(sp, B, Hq, S, ph, nh, pl, nl, out, frags, hs, st);
+    case 9: return launch_split_mma<2, 1, NT>(sp, B, Hq, S, ph, nh, pl, nl, out, frags, hs, st);
+    case 10: return launch_split_mma<2, 2, NT>(sp, B, Hq, S, ph, nh, pl, nl, out, frags, hs, st);
+    case 11: return launch_split_mma<2, 3, NT>(sp, B, Hq, S, ph, nh, pl, nl, out, frags, hs, st);
+    case 13: return launch_split_mma<3, 1, NT>(sp, B, Hq, S, ph, nh, pl, nl, out, frags, hs, st);
+    case 14: return launch_split_mma<3, 2, NT>(sp, B, Hq, S, ph, nh, pl, nl, out, frags, hs, st);
+    default: return launch_split_mma<3, 3, NT>(sp, B, Hq, S, ph, nh, pl, nl, out, frags, hs, st);
+  }
+}
+
+}  // namespace
+
+size_t split_logits_ws_bytes(const tq_split* sp, int B, int Hq) {
+  const int G = Hq / sp->Hkv;
+  if (!split_fast_path(sp, G)) return 256;
+  const int64_t groups = int64_t(B) * sp->Hkv;
+  const int nt = (G + HPT - 1) / HPT;
+  const size_t frag = size_t(groups) * nt * kFragWords * 4;
+  const size_t scales = size_t(groups) * G * sizeof(SplitScale);
+  return ((frag + 255) / 256) * 256 + ((scales + 255) / 256) * 256;
+}
+
+cudaError_t launch_split_logits(const tq_split* sp, const float* q, int B, int Hq, int64_t S, const uint8_t* ph,
+                                const uint16_t* nh, const uint8_t* pl, const uint16_t* nl, float scale, float* out,
+                                void* ws, cudaStream_t st) {
+  const int Hkv = sp->Hkv, G = Hq / Hkv;
+  if (!split_fast_path(sp, G)) {
+    const ChannelGather ghi{sp->dperm, S > 0 ? S : 1, Hkv, sp->d, 0};
+    const ChannelGather glo{sp->dperm, S > 0 ? S : 1, Hkv, sp->d, sp->hi->d};
+    cudaError_t e = launch_logits_simt(sp->hi, q, B, Hq, Hkv, S, ph, nh, scale, out, ghi, 0, st);
+    if (e != cudaSuccess) return e;
+    return launch_logits_simt(sp->lo, q, B, Hq, Hkv, S, pl, nl, scale, out, glo, 1, st);
+  }
+  const int nt = (G + HPT - 1) / HPT;
+  const int64_t groups = int64_t(B) * Hkv;
+  uint32_t* frags = static_cast<uint32_t*>(ws);
+  const size_t frag_bytes = ((size_t(groups) * nt * kFragWords * 4 + 255) / 256) * 256;
+  SplitScale* hs = reinterpret_cast<SplitScale*>(static_cast<uint8_t*>(ws) + frag_bytes);
+  qprep_split_kernel<<<unsigned(groups), 128, 0, st>>>(
+      q, Hq, Hkv, nt, sp->dperm, sp->hi->dRt, sp->hi->dPt, sp->lo->dRt, sp->lo->dPt, sp->hi->lut.inv_scale,
+      sp->lo->lut.inv_scale, scale, float(kQjlConst / sp->hi->m), float(kQjlConst / sp->lo->m), frags, hs);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (S == 0) return cudaSuccess;
+  return nt == 1 ? dispatch_split<1>(sp, B, Hq, S, ph, nh, pl, nl, out, frags, hs, st)
+                 : dispatch_split<2>(sp, B, Hq, S, ph, nh, pl, nl, out, frags, hs, st);
 }
 
 }  // namespace tq

@@ -107,6 +107,10 @@ cudaError_t launch_split_images(tq_split* sp, cudaStream_t st);
 bool split_tc_supported(const tq_split* sp, int dtype, const void* keys);
 cudaError_t launch_split_quantize_tc(const tq_split* sp, const void* keys, int B, int64_t S, uint8_t* payload_hi,
                                      uint16_t* norms_hi, uint8_t* payload_lo, uint16_t* norms_lo, cudaStream_t st);
+size_t split_logits_ws_bytes(const tq_split* sp, int B, int Hq);
+cudaError_t launch_split_logits(const tq_split* sp, const float* q, int B, int Hq, int64_t S, const uint8_t* ph,
+                                const uint16_t* nh, const uint8_t* pl, const uint16_t* nl, float scale, float* out,
+                                void* ws, cudaStream_t st);
 size_t topk_ws_bytes(const tq_ctx* ctx, int64_t nq, int64_t n, int k);
 bool search_tc_supported(const tq_ctx* ctx, int64_t nq, int64_t n, int k);
 size_t search_ws_bytes(const tq_ctx* ctx, int64_t nq, int64_t n);

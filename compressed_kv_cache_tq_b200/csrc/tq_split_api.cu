@@ -127,7 +127,7 @@ tq_status tq_split_quantize(const tq_split* sp, const void* keys, tq_dtype dtype
 
 size_t tq_split_logits_workspace_bytes(const tq_split* sp, int B, int Hq) {
   if (!sp || B <= 0 || Hq <= 0 || Hq % sp->Hkv) return 0;
-  return 256;
+  return tq::split_logits_ws_bytes(sp, B, Hq);
 }
 
 tq_status tq_split_logits(const tq_split* sp, const float* q, int B, int Hq, int64_t S, const uint8_t* payload_hi,
@@ -142,13 +142,8 @@ tq_status tq_split_logits(const tq_split* sp, const float* q, int B, int Hq, int
     return TQ_ERR_ARG;
   if (!workspace || !aligned(workspace, 256)) return TQ_ERR_ARG;
   if (workspace_bytes < tq_split_logits_workspace_bytes(sp, B, Hq)) return TQ_ERR_WORKSPACE;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = tq::launch_logits_simt(sp->hi, q, B, Hq, sp->Hkv, S, payload_hi, norms_hi, scale, out,
-                                         gather_of(sp, S, true), 0, st);
-  if (e == cudaSuccess)
-    e = tq::launch_logits_simt(sp->lo, q, B, Hq, sp->Hkv, S, payload_lo, norms_lo, scale, out,
-                               gather_of(sp, S, false), 1, st);
-  return cuda_status(e);
+  return cuda_status(tq::launch_split_logits(sp, q, B, Hq, S, payload_hi, norms_hi, payload_lo, norms_lo, scale, out,
+                                             workspace, static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

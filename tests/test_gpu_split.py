@@ -198,3 +198,22 @@ def test_split_full_size_sampled(lib):
                                       sel(ph), sel(nh), sel(pl), sel(nl), tb_hi, tb_lo, 1, 1, len(s_idx), scale)
         got = out[b, h * G:(h + 1) * G][:, torch.from_numpy(s_idx).to(DEV)].cpu().numpy()
         check_close(got, ref[0], A[0])
+
+
+@pytest.mark.parametrize("d_hi,d_lo,bits_hi,bits_lo,G", [(72, 64, 3, 2, 4), (64, 64, 3, 2, 16), (64, 128, 2, 4, 2)])
+def test_split_logits_cuda_core_path(lib, d_hi, d_lo, bits_hi, bits_lo, G):
+    """Shapes outside the int8-MMA split kernel (groups other than 64 + 64, more
+    than 8 query heads per KV head) run on CUDA cores."""
+    B, Hkv, S = 2, 2, 150
+    hi, lo = lib.tq_init(d_hi, bits_hi, 42), lib.tq_init(d_lo, bits_lo, 43)
+    sp = lib.tq_split_create(hi, lo, Hkv)
+    keys, K64 = _keys(B, Hkv, S, d_hi + d_lo, seed=321, dtype=torch.float32)
+    perm = O.split_plan(K64, d_hi)
+    sp.set_plan(perm)
+    ph, nh, pl, nl = lib.tq_split_quantize(sp, keys)
+    q = W.queries((B, Hkv * G, d_hi + d_lo), seed=10)
+    out = lib.tq_split_logits(sp, torch.from_numpy(q).to(DEV), ph, nh, pl, nl, scale=0.5)
+    _status_clean(lib, hi, lo)
+    ref, A = _oracle_split_logits(q.astype(np.float64), perm, ph.cpu().numpy(), nh.cpu().numpy(), pl.cpu().numpy(),
+                                  nl.cpu().numpy(), tables_of(hi), tables_of(lo), B, Hkv, S, 0.5)
+    check_close(out.cpu().numpy(), ref, A)
