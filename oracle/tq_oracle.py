@@ -28,6 +28,8 @@ What it computes, step by step, and where the pages say so:
   sketch, and the estimator is its first term, which the same page notes is
   biased for inner products (factor 2/pi at one bit).
 * Dequantisation "look up the table and rotate back" (same page, stage 1).
+* Value path: the decode attention output, softmax of the logits times the
+  values' unbiased reconstructions (reading in the section "Value path").
 * Fractional rates (2.5 bits per channel): a per-KV-head channel split
   into a high-variance group and a low-variance group, each quantised on
   its own (readings in the section "Channel split" below).
@@ -390,6 +392,59 @@ def topk(Q: np.ndarray, codes, bits, n16, rho16, tb: Tables, k: int):
         ids[i] = order
         sc[i] = s[i, order]
     return ids, sc, s, A
+
+
+# ---------------------------------------------------------------------------
+# Value path: decode attention output over a quantised value cache
+#
+# mooersco.com sections 1.2 and 1.3: the keys set the attention weights
+# (softmax of the logits), the values are summed with those weights, and the
+# values are compressed with a JL projection kept as sign bits, the output
+# being recovered by an estimator.  The other pages describe one two-stage
+# quantizer for the whole KV cache.  Reading: values are quantised with the
+# same quantizer as keys (tables of their own), and each value enters the
+# output through its unbiased reconstruction
+#   v_hat = n16 R^T c[idx] + sqrt(pi/2)/m rho16 S^T sigma
+# (stage 1 alone when m = 0), so that
+#   o = sum_s softmax(l)_s v_hat_s,
+# with l the (already scaled) logits of the query head against the keys.
+# ---------------------------------------------------------------------------
+
+
+def softmax(logits: np.ndarray) -> np.ndarray:
+    """Softmax over the last axis in fp64 (shifted by the maximum)."""
+    x = np.asarray(logits, dtype=np.float64)
+    e = np.exp(x - np.max(x, axis=-1, keepdims=True))
+    return e / np.sum(e, axis=-1, keepdims=True)
+
+
+def attention_output(logits: np.ndarray, codes, bits, n16, rho16, tb: Tables, Hkv: int):
+    """Attention output of every query head over a quantised value cache.
+
+    logits: (B, Hq, S), already scaled; value rows ordered (B, Hkv, S), query
+    head h reads KV head h // (Hq / Hkv).  Returns (o, A), each (B, Hq, d):
+    o[b, h] = sum_s softmax(logits[b, h])_s v_hat[b, h // G, s], and A the
+    same weighted sum of the absolute values of every term of v_hat (the
+    scale the tolerance is measured against).
+    """
+    B, Hq, S = logits.shape
+    G = Hq // Hkv
+    p = softmax(logits) if S > 0 else np.zeros((B, Hq, 0))
+    vh = dequantize(codes, bits, n16, rho16, tb, full=True).reshape(B, Hkv, S, tb.d)
+    n16 = np.asarray(n16, dtype=np.float64).reshape(B, Hkv, S)
+    cv = np.abs(tb.c[np.asarray(codes)]).reshape(B, Hkv, S, tb.d)
+    # |terms| of coordinate i: n16 sum_j |R_ji| |c_j| (+ the QJL term's)
+    absv = n16[..., None] * (cv @ np.abs(tb.R))
+    if tb.m > 0:
+        rho16 = np.asarray(rho16, dtype=np.float64).reshape(B, Hkv, S)
+        absv = absv + (QJL_CONST / tb.m) * rho16[..., None] * np.sum(np.abs(tb.S), axis=0)[None, None, None, :]
+    o = np.zeros((B, Hq, tb.d))
+    A = np.zeros((B, Hq, tb.d))
+    for b in range(B):
+        for h in range(Hq):
+            o[b, h] = p[b, h] @ vh[b, h // G]
+            A[b, h] = p[b, h] @ absv[b, h // G]
+    return o, A
 
 
 # ---------------------------------------------------------------------------

@@ -640,3 +640,83 @@ def test_split_gives_the_high_variance_channels_the_finer_code():
             planned = err
         else:
             assert np.all(planned < err)
+
+
+# --------------------------------------------------------------------------
+# Value path: attention output over a quantised value cache
+# --------------------------------------------------------------------------
+
+
+def _value_cache(B, Hkv, S, d, bits, seed, m=None):
+    rng = np.random.default_rng(seed)
+    V = rng.standard_normal((B * Hkv * S, d)) * rng.uniform(0.5, 3.0, d)
+    tb = O.make_tables(d, bits, 40 + seed, m=m)
+    return V, tb, O.quantize(V, tb)
+
+
+def test_softmax_closed_form():
+    p = O.softmax(np.array([[0.0, math.log(3.0)], [5.0, 5.0]]))
+    np.testing.assert_allclose(p, [[0.25, 0.75], [0.5, 0.5]], rtol=0, atol=1e-15)
+    # large logits do not overflow
+    np.testing.assert_allclose(O.softmax(np.array([1000.0, 1000.0 + math.log(3.0)])), [0.25, 0.75], atol=1e-15)
+
+
+def test_attention_of_two_keys_is_the_weighted_reconstruction():
+    V, tb, qz = _value_cache(1, 1, 2, 16, 3, 1)
+    o, _ = O.attention_output(np.array([[[0.0, math.log(3.0)]]]), qz.codes, qz.bits, qz.n16, qz.rho16, tb, 1)
+    xh = O.dequantize(qz.codes, qz.bits, qz.n16, qz.rho16, tb, full=True)
+    np.testing.assert_allclose(o[0, 0], 0.25 * xh[0] + 0.75 * xh[1], atol=1e-12)
+
+
+def test_attention_with_equal_logits_is_the_mean_and_shift_invariant():
+    B, Hkv, S, d = 1, 1, 7, 16
+    V, tb, qz = _value_cache(B, Hkv, S, d, 4, 2)
+    xh = O.dequantize(qz.codes, qz.bits, qz.n16, qz.rho16, tb, full=True)
+    o, _ = O.attention_output(np.full((1, 1, S), 2.5), qz.codes, qz.bits, qz.n16, qz.rho16, tb, Hkv)
+    np.testing.assert_allclose(o[0, 0], xh.mean(axis=0), atol=1e-12)
+    rng = np.random.default_rng(3)
+    lg = rng.standard_normal((1, 1, S)) * 3
+    o1, _ = O.attention_output(lg, qz.codes, qz.bits, qz.n16, qz.rho16, tb, Hkv)
+    o2, _ = O.attention_output(lg + 40.0, qz.codes, qz.bits, qz.n16, qz.rho16, tb, Hkv)
+    np.testing.assert_allclose(o1, o2, atol=1e-12)
+
+
+def test_attention_head_mapping_and_single_key():
+    # S = 1: every head of KV head k returns that key's reconstruction
+    B, Hkv, G, d = 2, 3, 2, 16
+    V, tb, qz = _value_cache(B, Hkv, 1, d, 3, 4)
+    xh = O.dequantize(qz.codes, qz.bits, qz.n16, qz.rho16, tb, full=True).reshape(B, Hkv, d)
+    lg = np.random.default_rng(5).standard_normal((B, Hkv * G, 1))
+    o, A = O.attention_output(lg, qz.codes, qz.bits, qz.n16, qz.rho16, tb, Hkv)
+    for b in range(B):
+        for h in range(Hkv * G):
+            np.testing.assert_allclose(o[b, h], xh[b, h // G], atol=1e-12)
+            assert np.all(A[b, h] >= np.abs(o[b, h]) - 1e-12)
+
+
+def test_attention_output_unbiased_over_value_tables():
+    # given the weights, E over the value quantizer's R and S of the output is
+    # the exact weighted sum of the values (each reconstruction is unbiased)
+    d, S, nseed = 16, 3, 3000
+    rng = np.random.default_rng(6)
+    V = rng.standard_normal((S, d)) * 2
+    lg = np.array([[[0.3, -1.0, 1.2]]])
+    u = rng.standard_normal(d)
+    want = float(O.softmax(lg)[0, 0] @ V @ u)
+    got = []
+    for s in range(nseed):
+        tb = O.make_tables(d, 3, seed=9000 + s)
+        qz = O.quantize(V, tb)
+        o, _ = O.attention_output(lg, qz.codes, qz.bits, qz.n, qz.rho, tb, 1)
+        got.append(o[0, 0] @ u)
+    got = np.array(got)
+    se = got.std(ddof=1) / math.sqrt(nseed)
+    assert abs(got.mean() - want) < 3 * se
+
+
+def test_attention_mse_only_uses_stage_one():
+    V, tb, qz = _value_cache(1, 1, 4, 16, 3, 7, m=0)
+    lg = np.array([[[0.1, 0.2, -0.3, 0.0]]])
+    o, _ = O.attention_output(lg, qz.codes, qz.bits, qz.n16, qz.rho16, tb, 1)
+    xh = qz.n16.astype(np.float64)[:, None] * (tb.c[qz.codes] @ tb.R)
+    np.testing.assert_allclose(o[0, 0], O.softmax(lg)[0, 0] @ xh, atol=1e-12)
