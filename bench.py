@@ -59,13 +59,19 @@ KV_WORKLOADS = {
     # 2.5 bits per channel: per KV head the 64 channels of largest variance at
     # b = 3, the other 64 at b = 2, each group its own d = m = 64 quantizer
     "split": (32, 8, 32, 128, 16384, (3, 2), 1003, "split25_b32_hkv8_hq32_d128_s16384_b3x64_b2x64"),
+    # the decode layer with a quantised value cache as well (values b = 4,
+    # tables of their own): quantize keys and values, logits, attention output
+    "attend": (8, 8, 32, 128, 32768, 4, 1001, "decode_attention_llama31_8b_layer_b8_hkv8_hq32_d128_s32768_b4"),
 }
+SEED_VALUES = 2002
+ATTEND = False
 
 
 def set_workload(name: str, seq: int | None = None):
     """Point the module's shape globals at one of KV_WORKLOADS (seq overrides S)."""
-    global B, HKV, HQ, D, S, BITS, SEED_KEYS, WORKLOAD
+    global B, HKV, HQ, D, S, BITS, SEED_KEYS, WORKLOAD, ATTEND
     B, HKV, HQ, D, S, BITS, SEED_KEYS, WORKLOAD = KV_WORKLOADS[name]
+    ATTEND = name == "attend"
     if seq is not None and seq != S:
         WORKLOAD = WORKLOAD.replace(f"_s{S}_", f"_s{seq}_")
         S = seq
@@ -153,7 +159,12 @@ def bytes_per_key():
         row = sum(g * (b - 1) // 8 + g // 8 + 4 for b in BITS)
     else:
         row = D * (BITS - 1) // 8 + D // 8 + 4
-    return {"quantize_in": 2 * D, "quantize_out": row, "logits_in": row, "logits_out": 4 * (HQ // HKV)}
+    bpk = {"quantize_in": 2 * D, "quantize_out": row, "logits_in": row, "logits_out": 4 * (HQ // HKV)}
+    if ATTEND:
+        # keys and values are both quantised; the attention reads the value
+        # rows and the logits of the group's query heads
+        bpk.update(quantize_in=4 * D, quantize_out=2 * row, attend_in=row + 4 * (HQ // HKV))
+    return bpk
 
 
 def quantize_flops_per_key():
@@ -185,6 +196,9 @@ def cpu_baseline(budget_s: float = 12.0, max_keys: int = 1 << 19):
     else:
         tb = O.make_tables(D, BITS, SEED_TABLES)
     scales = W.head_channel_scales(HKV, D, SEED_KEYS)
+    if ATTEND:
+        tbv = O.make_tables(D, BITS, SEED_TABLES + 100)
+        vscales = W.head_channel_scales(HKV, D, SEED_VALUES)
     q = W.queries((B, HQ, D), seed=SEED_KEYS + 7)
     G = HQ // HKV
     chunk = 8192
@@ -193,10 +207,20 @@ def cpu_baseline(budget_s: float = 12.0, max_keys: int = 1 << 19):
         for h in range(HKV):
             keys = W.decode_keys_pair(b, h, S, D, scales, SEED_KEYS)
             kb = torch.from_numpy(keys).to(torch.bfloat16).to(torch.float64).numpy()
+            if ATTEND:
+                vb = torch.from_numpy(W.decode_keys_pair(b, h, S, D, vscales, SEED_VALUES)).to(
+                    torch.bfloat16).to(torch.float64).numpy()
             qh = q[b, h * G:(h + 1) * G].astype(np.float64)
             for s0 in range(0, S, chunk):
                 kc = kb[s0:s0 + chunk]
-                if split:
+                if ATTEND:
+                    # keys and values of the chunk, logits, attention over the chunk
+                    t0 = time.perf_counter()
+                    qz = O.quantize(kc, tb)
+                    lg, _ = O.estimate(qh, qz.codes, qz.bits, qz.n16, qz.rho16, tb)
+                    vz = O.quantize(vb[s0:s0 + chunk], tbv)
+                    O.attention_output(lg[None] / math.sqrt(D), vz.codes, vz.bits, vz.n16, vz.rho16, tbv, 1)
+                elif split:
                     perm = O.split_plan(kc[None, None], D // 2)
                     t0 = time.perf_counter()
                     a, c = O.split_quantize(kc[None, None], perm, tb_hi, tb_lo)
@@ -215,7 +239,9 @@ def cpu_baseline(budget_s: float = 12.0, max_keys: int = 1 << 19):
             break
     threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
     return {"value": done / busy, "unit": "keys/s", "cores": threads, "kind": "oracle",
-            "sample": f"{done} of {B * HKV * S} keys (quantize + {G}-head estimates), {busy:.1f} s, fp64 numpy"}
+            "sample": f"{done} of {B * HKV * S} keys (quantize + {G}-head estimates"
+                      f"{'; values quantised and attended over each 8192-key chunk' if ATTEND else ''}), "
+                      f"{busy:.1f} s, fp64 numpy"}
 
 
 def run_search(args):
@@ -366,7 +392,7 @@ def max_over_ranks(x: float, dist, device) -> float:
     return float(t.item())
 
 
-def result_line(*, world, n, steps, warmup, ms, q_ms, l_ms, e2e_ms, h2d, d2h, clocks) -> dict:
+def result_line(*, world, n, steps, warmup, ms, q_ms, l_ms, e2e_ms, h2d, d2h, clocks, a_ms=None) -> dict:
     """The JSON result: whole-job rates over all ranks (each rank processes n keys
     per step; ms and e2e_ms are the slowest rank's), the per-kernel breakdown and
     the roofline of the dominant kernel."""
@@ -376,14 +402,18 @@ def result_line(*, world, n, steps, warmup, ms, q_ms, l_ms, e2e_ms, h2d, d2h, cl
     q_bytes = n * (bpk["quantize_in"] + bpk["quantize_out"])
     l_bytes = n * (bpk["logits_in"] + bpk["logits_out"])
     kq, kl = ("tq_split_quantize", "tq_split_logits") if isinstance(BITS, tuple) else ("tq_quantize", "tq_logits")
-    fl = n * quantize_flops_per_key()
+    fl = n * quantize_flops_per_key() * (2 if ATTEND else 1)
     kernels = {
         kq: {"ms": q_ms, "bytes": q_bytes, "GB/s": q_bytes / q_ms / 1e6, "vectors_per_s": n / q_ms * 1e3,
              "flops": fl, "TFLOP/s": fl / q_ms / 1e9},
         kl: {"ms": l_ms, "bytes": l_bytes, "GB/s": l_bytes / l_ms / 1e6, "keys_per_s": n / l_ms * 1e3,
              "pct_of_8TBs": 100 * l_bytes / l_ms / 1e6 / 8000.0},
     }
-    dom = kq if q_ms >= l_ms else kl
+    if a_ms is not None:
+        a_bytes = n * bpk["attend_in"]
+        kernels["tq_attend"] = {"ms": a_ms, "bytes": a_bytes, "GB/s": a_bytes / a_ms / 1e6,
+                                "keys_per_s": n / a_ms * 1e3}
+    dom = max(kernels, key=lambda k: kernels[k]["ms"])
     ach = kernels[dom]["GB/s"]
     dram = DRAM_BYTES_PER_KEY.get(WORKLOAD.split("_")[0], {}).get(dom)
     return {
@@ -416,7 +446,7 @@ def result_line(*, world, n, steps, warmup, ms, q_ms, l_ms, e2e_ms, h2d, d2h, cl
         "quantize_vectors_per_s": world * n / q_ms * 1e3,
         "e2e": {"value": world * n / e2e_ms * 1e3, "unit": "keys/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": 3 * steps,
+        "gpu_launches": (6 if a_ms is not None else 3) * steps,
         "clocks": clocks,
     }
 
@@ -428,7 +458,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="decode", choices=["decode", "longctx", "split", "search"])
+    ap.add_argument("--workload", default="decode", choices=["decode", "longctx", "split", "attend", "search"])
     ap.add_argument("--rows", type=int, default=1_000_000, help="search: database rows")
     ap.add_argument("--queries", type=int, default=10_000, help="search: queries")
     ap.add_argument("--seq", type=int, default=None,
@@ -511,13 +541,34 @@ def main():
     # fill both caches once so the first logits read valid data
     for c in caches:
         quantize(keys4, c)
+    attend = None
+    if ATTEND:
+        vctx = tq.tq_init(D, BITS, SEED_TABLES + 100)
+        vals4 = W.decode_keys(B, HKV, S, D, SEED_VALUES, device=dev)
+        vcaches = [(torch.empty((n, vctx.row_bytes), dtype=torch.uint8, device=dev),
+                    torch.empty((n, 2), dtype=torch.float16, device=dev)) for _ in range(2)]
+        o_att = torch.empty((B, HQ, D), dtype=torch.float32, device=dev)
+        aws = torch.empty(max(256, tq.tq_attend_workspace_bytes(vctx, B, HQ, HKV, S)), dtype=torch.uint8,
+                          device=dev)
+        for c in vcaches:
+            tq.tq_quantize(vctx, vals4.reshape(-1, D), c[0], c[1])
+        kq_only = quantize
+
+        def quantize(k4, c, i=None):
+            kq_only(k4, c)
+            vc = vcaches[0 if c is caches[0] else 1]
+            tq.tq_quantize(vctx, (vals4 if k4 is keys4 else dvals).reshape(-1, D), vc[0], vc[1])
+
+        def attend(c):
+            vc = vcaches[0 if c is caches[0] else 1]
+            tq.tq_attend(vctx, out, vc[0], vc[1], HKV, out=o_att, workspace=aws)
 
     ev = []
 
     def step(i, record):
         cw, cr = caches[i % 2], caches[(i + 1) % 2]
         if record:
-            e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(4 if attend else 3)]
             e[0].record(stream)
         quantize(keys4, cw)
         if record:
@@ -525,6 +576,11 @@ def main():
         logits(q, cr)
         if record:
             e[2].record(stream)
+        if attend:
+            attend(cr)
+            if record:
+                e[3].record(stream)
+        if record:
             ev.append(e)
 
     def barrier():
@@ -546,22 +602,35 @@ def main():
     assert tq.tq_check_device_status(ctx) == 0, "a kernel reported a device-side error"
     q_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / len(ev)
     l_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / len(ev)
+    a_ms = sum(e[2].elapsed_time(e[3]) for e in ev) / len(ev) if attend else None
 
     # end to end through the public API: pinned host keys in, logits out
     host_keys = torch.empty(keys4.shape, dtype=keys4.dtype, pin_memory=True)
     host_keys.copy_(keys4)
+    if ATTEND:
+        host_vals = torch.empty(vals4.shape, dtype=vals4.dtype, pin_memory=True)
+        host_vals.copy_(vals4)
+        dvals = torch.empty_like(vals4)
     host_q = q.cpu().pin_memory()
     host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    if ATTEND:
+        host_att = torch.empty(o_att.shape, dtype=o_att.dtype, pin_memory=True)
     dkeys = torch.empty_like(keys4)
     dq = torch.empty_like(q)
 
     def e2e_step(i):
         cw, cr = caches[i % 2], caches[(i + 1) % 2]
         dkeys.copy_(host_keys, non_blocking=True)
+        if ATTEND:
+            dvals.copy_(host_vals, non_blocking=True)
         dq.copy_(host_q, non_blocking=True)
         quantize(dkeys, cw)
         logits(dq, cr)
-        host_out.copy_(out, non_blocking=True)
+        if attend:
+            attend(cr)
+            host_att.copy_(o_att, non_blocking=True)
+        else:
+            host_out.copy_(out, non_blocking=True)
 
     e2e_steps = max(3, min(args.steps, 10))
     for i in range(3):
@@ -581,7 +650,9 @@ def main():
         return 0
 
     line = result_line(world=world, n=n, steps=args.steps, warmup=args.warmup, ms=ms, q_ms=q_ms, l_ms=l_ms,
-                       e2e_ms=e2e_ms, h2d=int(keys.numel() * 2 + q.numel() * 4), d2h=int(out.numel() * 4),
+                       e2e_ms=e2e_ms, a_ms=a_ms,
+                       h2d=int(keys.numel() * 2 * (2 if ATTEND else 1) + q.numel() * 4),
+                       d2h=int((o_att if ATTEND else out).numel() * 4),
                        clocks=clocks.summary())
     line.update(extra)
     if not args.no_cpu_baseline and world == 1:

@@ -1,0 +1,407 @@
+// Decode attention output over a quantised value cache (the value path).
+//
+// mooersco.com sections 1.2-1.3: the keys set the attention weights through
+// the softmax of the logits, the values are summed with those weights, and
+// the output is recovered from the compressed values by an estimator.  Values
+// are quantised here with the same quantizer as keys (their own context), and
+// each value enters through its unbiased reconstruction
+//   v_hat = n16 R^T c[idx] + sqrt(pi/2)/m rho16 S^T sigma      (S = P R)
+// so for one query head with weights w_s = exp(l_s - max l):
+//   o = R^T (a + sqrt(pi/2)/m P^T b) / sum_s w_s,
+//   a = sum_s w_s n16_s c[idx_s]   (rotated domain, d),
+//   b = sum_s w_s rho16_s sigma_s  (sign domain, m).
+// The rotations are applied once per head, after the sums, not once per key.
+//
+// Kernel 1 (attend_partial_kernel): one block per (batch, KV head, key chunk)
+// computes, for every query head of the group, the chunk's maximum logit, the
+// sum of its weights and its a, b (flash-decoding style partials).  Key tiles
+// of 64 rows are staged in shared memory (prefetched into registers one tile
+// ahead); warp w takes keys w, w + 8, ...; lane L decodes one "slot" of the
+// packed layout per key (4 coordinates: register r = 4u + i of quarter q,
+// nibbles e = 0..3) and accumulates G heads with packed two-wide FMAs.
+// Kernel 2 (attend_combine_kernel): one block per query head merges the
+// partials and applies P^T and R^T.
+#include <math.h>
+
+#include "tq_device.cuh"
+#include "tq_internal.h"
+
+namespace tq {
+namespace {
+
+constexpr int kAttThreads = 256;
+constexpr int kAttWarps = kAttThreads / 32;
+constexpr int kAttTile = 64;          // keys per staged tile
+constexpr int kAttMaxLd = 4;          // 8-byte words per thread per tile (rows of up to 128 bytes)
+constexpr int kAttMaxHeads = 8;
+
+__device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
+
+// Codes of the 4 coordinates (r = 4u + i, e = 0..3) of one slot from the
+// unit's code halfwords h[0 .. BM-1] (layout in include/tq.h).
+template <int BM>
+__device__ __forceinline__ void slot_codes(const uint32_t (&h)[BM], int i, int (&code)[4]) {
+  if constexpr (BM == 1) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) code[e] = (h[0] >> (4 * e + i)) & 1;
+  } else if constexpr (BM == 2) {
+    const uint32_t hs = (i >> 1) ? h[1] : h[0];
+    const int sh = 2 * (i & 1);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) code[e] = (hs >> (4 * e + sh)) & 3;
+  } else {
+    const uint32_t hs = i == 0 ? h[0] : (i == 1 ? h[1] : h[2]);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int lo = (hs >> (4 * e)) & 7;
+      const int hi = ((h[0] >> (4 * e + 3)) & 1) | (((h[1] >> (4 * e + 3)) & 1) << 1) |
+                     (((h[2] >> (4 * e + 3)) & 1) << 2);
+      code[e] = i < 3 ? lo : hi;
+    }
+  }
+}
+
+// Partials: part[((grp * nsplit + split) * G + h) * (2 + dp + mp)] = {max, sum, a[dp], b[mp]}.
+template <int BM, int GP, int NS>
+__global__ void __launch_bounds__(kAttThreads) attend_partial_kernel(
+    const float* __restrict__ logits, int Hq, int Hkv, int64_t S, int64_t chunk, int nsplit,
+    const uint8_t* __restrict__ payload, const uint16_t* __restrict__ norms, RowGeom g, CodebookParams cb,
+    float* __restrict__ part) {
+  extern __shared__ __align__(16) uint8_t sm[];
+  const int rb = g.row_bytes;
+  uint8_t* srows = sm;                                                        // [kAttTile][rb]
+  float* swn = reinterpret_cast<float*>(sm + kAttTile * rb);                  // [kAttTile][GP]  w n16
+  float* swr = swn + kAttTile * GP;                                           // [kAttTile][GP]  w rho16
+  float* sacc = swr + kAttTile * GP;                                          // [GP][dp + mp]
+  float* sred = sacc + GP * (g.dp + g.mp);                                    // [GP][kAttWarps] maxima
+  float* smx = sred + GP * kAttWarps;                                         // [GP] chunk maximum
+  float* sl = smx + GP;                                                       // [GP] sum of weights
+  float* sc = sl + GP;                                                        // [8] codebook
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int G = Hq / Hkv;
+  const int grp = blockIdx.x / nsplit, split = blockIdx.x - grp * nsplit;
+  const int b = grp / Hkv, hkv = grp - b * Hkv;
+  const int64_t s_begin = int64_t(split) * chunk;
+  const int64_t s_end = s_begin + chunk < S ? s_begin + chunk : S;
+  const float* lg = logits + (size_t(b) * Hq + size_t(hkv) * G) * S;   // head h at lg + h S
+  const uint8_t* rows = payload + (size_t(grp) * S) * rb;
+  const uint32_t* nrm = reinterpret_cast<const uint32_t*>(norms) + size_t(grp) * S;
+
+  for (int i = tid; i < GP * (g.dp + g.mp); i += kAttThreads) sacc[i] = 0.f;
+  if (tid < 8) sc[tid] = cb.c[tid];
+  if (tid < GP) sl[tid] = 0.f;
+
+  // pass 1: the chunk's maximum logit per head
+  float mx[GP];
+#pragma unroll
+  for (int h = 0; h < GP; ++h) mx[h] = -INFINITY;
+  for (int64_t s = s_begin + tid; s < s_end; s += kAttThreads)
+#pragma unroll
+    for (int h = 0; h < GP; ++h)
+      if (h < G) mx[h] = fmaxf(mx[h], lg[size_t(h) * S + s]);
+#pragma unroll
+  for (int h = 0; h < GP; ++h) {
+    float v = mx[h];
+    for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if (lane == 0) sred[h * kAttWarps + warp] = v;
+  }
+  __syncthreads();
+  if (tid < GP) {
+    float v = sred[tid * kAttWarps];
+    for (int w = 1; w < kAttWarps; ++w) v = fmaxf(v, sred[tid * kAttWarps + w]);
+    smx[tid] = v;
+  }
+  __syncthreads();
+
+  // this lane's slots: code slot t -> quarter, unit, register i; sign slot likewise
+  const int nslot_c = g.dp / 4, nslot_s = g.mp / 4;
+  int c_off[NS], c_i[NS], c_j[NS], s_off[NS], s_i[NS], s_k[NS];
+#pragma unroll
+  for (int ns = 0; ns < NS; ++ns) {
+    const int t = lane + 32 * ns;
+    const int q = t / (4 * g.uq), rem = t - q * 4 * g.uq, u = rem >> 2;
+    c_i[ns] = rem & 3;
+    c_off[ns] = q * g.per_q + u * BM;                       // halfword index of the unit's codes
+    c_j[ns] = q * (g.dp / 4) + 4 * (4 * u + c_i[ns]);       // first coordinate (e = 0)
+    const int qs = g.uqm > 0 ? t / (4 * g.uqm) : 0, rs = t - qs * 4 * (g.uqm > 0 ? g.uqm : 1), us = rs >> 2;
+    s_i[ns] = rs & 3;
+    s_off[ns] = qs * g.per_q + BM * g.uq + us;
+    s_k[ns] = qs * (g.mp / 4) + 4 * (4 * us + s_i[ns]);
+  }
+  float2 accC[NS][GP / 2][4], accS[NS][GP / 2][4];
+#pragma unroll
+  for (int ns = 0; ns < NS; ++ns)
+#pragma unroll
+    for (int hp = 0; hp < GP / 2; ++hp)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        accC[ns][hp][e] = make_float2(0.f, 0.f);
+        accS[ns][hp][e] = make_float2(0.f, 0.f);
+      }
+  // weights: thread (key k = tid % 64, head tid / 64 + 4 it) of each tile
+  constexpr int kWIt = (kAttTile * GP + kAttThreads - 1) / kAttThreads;
+  float lsum[kWIt];
+#pragma unroll
+  for (int it = 0; it < kWIt; ++it) lsum[it] = 0.f;
+
+  // pass 2: tiles of keys, staged one ahead in registers
+  const int words = kAttTile * rb / 8;
+  uint2 ld[kAttMaxLd];
+  auto fetch = [&](int64_t s0) {
+    const int nk = int(s_end - s0 < kAttTile ? s_end - s0 : kAttTile);
+    const int nw = nk * rb / 8;
+    const uint2* src = reinterpret_cast<const uint2*>(rows + size_t(s0) * rb);
+#pragma unroll
+    for (int k = 0; k < kAttMaxLd; ++k) {
+      const int w = tid + k * kAttThreads;
+      ld[k] = (w < nw) ? __ldg(src + w) : make_uint2(0u, 0u);
+    }
+  };
+  const bool have = s_begin < s_end;
+  if (have) fetch(s_begin);
+  for (int64_t s0 = s_begin; s0 < s_end; s0 += kAttTile) {
+    const int nk = int(s_end - s0 < kAttTile ? s_end - s0 : kAttTile);
+    // stage this tile: rows, then the weights w n16 and w rho16 of every (key, head)
+#pragma unroll
+    for (int k = 0; k < kAttMaxLd; ++k) {
+      const int w = tid + k * kAttThreads;
+      if (w < words) reinterpret_cast<uint2*>(srows)[w] = ld[k];
+    }
+#pragma unroll
+    for (int it = 0; it < kWIt; ++it) {
+      const int idx = tid + it * kAttThreads;
+      if (idx < kAttTile * GP) {
+        const int k = idx % kAttTile, h = idx / kAttTile;
+        float wn = 0.f, wr = 0.f;
+        if (k < nk && h < G) {
+          const float w = expf(lg[size_t(h) * S + s0 + k] - smx[h]);
+          const uint32_t nn = __ldg(nrm + s0 + k);
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&nn));
+          wn = w * f.x;
+          wr = w * f.y;
+          lsum[it] += w;
+        }
+        swn[k * GP + h] = wn;
+        swr[k * GP + h] = wr;
+      }
+    }
+    __syncthreads();
+    if (s0 + kAttTile < s_end) fetch(s0 + kAttTile);   // next tile in flight during the math
+    for (int k = warp; k < nk; k += kAttWarps) {
+      const uint16_t* hw = reinterpret_cast<const uint16_t*>(srows + k * rb);
+      float2 wn2[GP / 2], wr2[GP / 2];
+#pragma unroll
+      for (int hp = 0; hp < GP / 2; ++hp) {
+        wn2[hp] = *reinterpret_cast<const float2*>(swn + k * GP + 2 * hp);
+        wr2[hp] = *reinterpret_cast<const float2*>(swr + k * GP + 2 * hp);
+      }
+#pragma unroll
+      for (int ns = 0; ns < NS; ++ns) {
+        const int t = lane + 32 * ns;
+        if (t < nslot_c) {
+          uint32_t h[BM];
+#pragma unroll
+          for (int x = 0; x < BM; ++x) h[x] = hw[c_off[ns] + x];
+          int code[4];
+          slot_codes<BM>(h, c_i[ns], code);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 cv = f2(sc[code[e]]);
+#pragma unroll
+            for (int hp = 0; hp < GP / 2; ++hp) accC[ns][hp][e] = __ffma2_rn(cv, wn2[hp], accC[ns][hp][e]);
+          }
+        }
+        if (t < nslot_s) {
+          const uint32_t hs = hw[s_off[ns]];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 sg = f2(((hs >> (4 * e + s_i[ns])) & 1u) ? 1.f : -1.f);
+#pragma unroll
+            for (int hp = 0; hp < GP / 2; ++hp) accS[ns][hp][e] = __ffma2_rn(sg, wr2[hp], accS[ns][hp][e]);
+          }
+        }
+      }
+    }
+    __syncthreads();
+  }
+
+  // merge the warps' sums into shared memory, then write the block's partial
+#pragma unroll
+  for (int ns = 0; ns < NS; ++ns) {
+    const int t = lane + 32 * ns;
+#pragma unroll
+    for (int hp = 0; hp < GP / 2; ++hp)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (t < nslot_c) {
+          atomicAdd(sacc + (2 * hp) * (g.dp + g.mp) + c_j[ns] + e, accC[ns][hp][e].x);
+          atomicAdd(sacc + (2 * hp + 1) * (g.dp + g.mp) + c_j[ns] + e, accC[ns][hp][e].y);
+        }
+        if (t < nslot_s) {
+          atomicAdd(sacc + (2 * hp) * (g.dp + g.mp) + g.dp + s_k[ns] + e, accS[ns][hp][e].x);
+          atomicAdd(sacc + (2 * hp + 1) * (g.dp + g.mp) + g.dp + s_k[ns] + e, accS[ns][hp][e].y);
+        }
+      }
+  }
+  // every lane of a warp holds the same head in lsum[it] (32 consecutive keys)
+#pragma unroll
+  for (int it = 0; it < kWIt; ++it) {
+    float v = lsum[it];
+    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    const int h = (tid + it * kAttThreads) / kAttTile;
+    if (lane == 0 && h < GP) atomicAdd(sl + h, v);
+  }
+  __syncthreads();
+  const int rec = 2 + g.dp + g.mp;
+  for (int h = 0; h < G; ++h) {
+    float* out = part + (size_t(blockIdx.x) * G + h) * rec;
+    for (int i = tid; i < g.dp + g.mp; i += kAttThreads) out[2 + i] = sacc[h * (g.dp + g.mp) + i];
+    if (tid == 0) {
+      out[0] = smx[h];
+      out[1] = sl[h];
+    }
+  }
+}
+
+// One block per query head: merge the chunk partials, then
+// o = R^T (a + sqrt(pi/2)/m P^T b) / L.
+__global__ void __launch_bounds__(256) attend_combine_kernel(const float* __restrict__ part, int Hq, int Hkv,
+                                                             int nsplit, const float* __restrict__ R,
+                                                             const float* __restrict__ P, int d, int m, RowGeom g,
+                                                             float* __restrict__ out) {
+  extern __shared__ float sv[];
+  float* sa = sv;          // [dp] merged a, then u
+  float* sb = sa + g.dp;   // [mp] merged b
+  __shared__ float sf[1024];   // per-split factors exp(m_i - M)
+  __shared__ float sL;
+  const int bh = blockIdx.x, b = bh / Hq, h = bh - b * Hq;
+  const int G = Hq / Hkv, hkv = h / G, hl = h - hkv * G;
+  const int grp = b * Hkv + hkv;
+  const int rec = 2 + g.dp + g.mp;
+  const float* p0 = part + (size_t(grp) * nsplit * G + hl) * rec;   // split i at p0 + i G rec
+  if (threadIdx.x == 0) {
+    float M = -INFINITY;
+    for (int i = 0; i < nsplit; ++i) M = fmaxf(M, p0[size_t(i) * G * rec]);
+    float L = 0.f;
+    for (int i = 0; i < nsplit; ++i) {
+      const float mi = p0[size_t(i) * G * rec];
+      const float f = (M == -INFINITY || mi == -INFINITY) ? 0.f : expf(mi - M);
+      if (i < 1024) sf[i] = f;
+      L += f * p0[size_t(i) * G * rec + 1];
+    }
+    sL = L;
+  }
+  __syncthreads();
+  const float L = sL;
+  for (int j = threadIdx.x; j < g.dp + g.mp; j += blockDim.x) {
+    float acc = 0.f;
+    for (int i = 0; i < nsplit; ++i) acc = fmaf(sf[i], p0[size_t(i) * G * rec + 2 + j], acc);
+    sv[j] = acc;
+  }
+  __syncthreads();
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  const float qc = m > 0 ? float(kQjlConst) / float(m) : 0.f;
+  float u_own = 0.f;
+  if (threadIdx.x < d) {
+    const int j = threadIdx.x;
+    float t = 0.f;
+    for (int k = 0; k < m; ++k) t = fmaf(P[size_t(k) * d + j], sb[k], t);
+    u_own = (sa[j] + qc * t) * inv;
+  }
+  __syncthreads();
+  if (threadIdx.x < d) sa[threadIdx.x] = u_own;
+  __syncthreads();
+  if (threadIdx.x < d) {
+    const int i = threadIdx.x;
+    float o = 0.f;
+    for (int j = 0; j < d; ++j) o = fmaf(R[size_t(j) * d + i], sa[j], o);
+    out[size_t(bh) * d + i] = o;
+  }
+}
+
+struct AttPlan {
+  int nsplit;
+  int64_t chunk;
+};
+
+AttPlan att_plan(int B, int Hkv, int64_t S) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t groups = int64_t(B) * Hkv;
+  int64_t ns = (int64_t(sms) * 4 + groups - 1) / groups;
+  const int64_t max_ns = (S + kAttTile - 1) / kAttTile;
+  if (ns > max_ns) ns = max_ns;
+  if (ns > 1024) ns = 1024;
+  if (ns < 1) ns = 1;
+  int64_t chunk = (S + ns - 1) / ns;
+  chunk = (chunk + kAttTile - 1) / kAttTile * kAttTile;
+  if (chunk < kAttTile) chunk = kAttTile;
+  ns = (S + chunk - 1) / chunk;
+  if (ns < 1) ns = 1;
+  return AttPlan{int(ns), chunk};
+}
+
+template <int BM, int GP, int NS>
+cudaError_t launch_partial(const tq_ctx* ctx, const float* logits, int B, int Hq, int Hkv, int64_t S, AttPlan ap,
+                           const uint8_t* payload, const uint16_t* norms, float* part, cudaStream_t st) {
+  const RowGeom g = make_geom(ctx->d, ctx->m, ctx->bmse);
+  const size_t smem = size_t(kAttTile) * g.row_bytes + size_t(2 * kAttTile * GP) * 4 +
+                      size_t(GP) * (g.dp + g.mp) * 4 + size_t(GP * kAttWarps + 2 * GP + 8) * 4;
+  auto kern = attend_partial_kernel<BM, GP, NS>;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  kern<<<unsigned(int64_t(B) * Hkv * ap.nsplit), kAttThreads, smem, st>>>(logits, Hq, Hkv, S, ap.chunk, ap.nsplit,
+                                                                          payload, norms, g, ctx->cb, part);
+  return cudaGetLastError();
+}
+
+template <int BM, int NS>
+cudaError_t dispatch_heads(const tq_ctx* ctx, const float* logits, int B, int Hq, int Hkv, int64_t S, AttPlan ap,
+                           const uint8_t* payload, const uint16_t* norms, float* part, cudaStream_t st) {
+  const int G = Hq / Hkv;
+  if (G <= 2) return launch_partial<BM, 2, NS>(ctx, logits, B, Hq, Hkv, S, ap, payload, norms, part, st);
+  if (G <= 4) return launch_partial<BM, 4, NS>(ctx, logits, B, Hq, Hkv, S, ap, payload, norms, part, st);
+  return launch_partial<BM, 8, NS>(ctx, logits, B, Hq, Hkv, S, ap, payload, norms, part, st);
+}
+
+template <int NS>
+cudaError_t dispatch_bits(const tq_ctx* ctx, const float* logits, int B, int Hq, int Hkv, int64_t S, AttPlan ap,
+                          const uint8_t* payload, const uint16_t* norms, float* part, cudaStream_t st) {
+  switch (ctx->bmse) {
+    case 1: return dispatch_heads<1, NS>(ctx, logits, B, Hq, Hkv, S, ap, payload, norms, part, st);
+    case 2: return dispatch_heads<2, NS>(ctx, logits, B, Hq, Hkv, S, ap, payload, norms, part, st);
+    default: return dispatch_heads<3, NS>(ctx, logits, B, Hq, Hkv, S, ap, payload, norms, part, st);
+  }
+}
+
+}  // namespace
+
+bool attend_supported(const tq_ctx* ctx, int Hq, int Hkv) {
+  return Hq / Hkv <= kAttMaxHeads && ctx->bmse >= 1 && ctx->bmse <= 3 && ctx->d <= 256 && ctx->m <= 256;
+}
+
+size_t attend_ws_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int64_t S) {
+  const AttPlan ap = att_plan(B, Hkv, S);
+  const RowGeom g = make_geom(ctx->d, ctx->m, ctx->bmse);
+  const size_t rec = size_t(2 + g.dp + g.mp);
+  const size_t bytes = size_t(B) * Hkv * ap.nsplit * size_t(Hq / Hkv) * rec * 4;
+  return (bytes + 255) / 256 * 256;
+}
+
+cudaError_t launch_attend(const tq_ctx* ctx, const float* logits, int B, int Hq, int Hkv, int64_t S,
+                          const uint8_t* payload, const uint16_t* norms, float* out, void* ws, cudaStream_t st) {
+  const AttPlan ap = att_plan(B, Hkv, S);
+  const RowGeom g = make_geom(ctx->d, ctx->m, ctx->bmse);
+  float* part = static_cast<float*>(ws);
+  const bool two = g.dp > 128 || g.mp > 128;
+  cudaError_t e = two ? dispatch_bits<2>(ctx, logits, B, Hq, Hkv, S, ap, payload, norms, part, st)
+                      : dispatch_bits<1>(ctx, logits, B, Hq, Hkv, S, ap, payload, norms, part, st);
+  if (e != cudaSuccess) return e;
+  const size_t smem = size_t(g.dp + g.mp) * 4;
+  attend_combine_kernel<<<unsigned(B * Hq), 256, smem, st>>>(part, Hq, Hkv, ap.nsplit, ctx->dR, ctx->dP, ctx->d,
+                                                             ctx->m, g, out);
+  return cudaGetLastError();
+}
+
+}  // namespace tq

@@ -64,6 +64,26 @@ tq_status tq_logits(const tq_ctx* ctx, const float* q, int B, int Hq, int Hkv, i
                                        static_cast<cudaStream_t>(stream)));
 }
 
+size_t tq_attend_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int64_t S) {
+  if (!ctx || B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || S < 0) return 0;
+  return tq::attend_ws_bytes(ctx, B, Hq, Hkv, S);
+}
+
+tq_status tq_attend(const tq_ctx* ctx, const float* logits, int B, int Hq, int Hkv, int64_t S,
+                    const uint8_t* payload, const uint16_t* norms, float* out, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  if (!ctx || B < 0 || Hq < 0 || Hkv < 0 || S < 0) return TQ_ERR_ARG;
+  if (B == 0 || Hq == 0) return TQ_OK;
+  if (Hkv == 0 || Hq % Hkv) return TQ_ERR_ARG;
+  if (!out || (S > 0 && (!logits || !payload || !norms))) return TQ_ERR_ARG;
+  if (!aligned(payload, 16) || !aligned(norms, 4) || !aligned(logits, 4) || !aligned(out, 4)) return TQ_ERR_ARG;
+  if (!tq::attend_supported(ctx, Hq, Hkv)) return TQ_ERR_UNSUPPORTED;
+  if (!workspace || !aligned(workspace, 256)) return TQ_ERR_ARG;
+  if (workspace_bytes < tq_attend_workspace_bytes(ctx, B, Hq, Hkv, S)) return TQ_ERR_WORKSPACE;
+  return cuda_status(tq::launch_attend(ctx, logits, B, Hq, Hkv, S, payload, norms, out, workspace,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
 size_t tq_topk_workspace_bytes(const tq_ctx* ctx, int64_t nq, int64_t n, int k) {
   if (!ctx || nq <= 0 || n <= 0 || k <= 0) return 0;
   return tq::topk_ws_bytes(ctx, nq, n, k);

@@ -99,6 +99,12 @@ cudaError_t launch_logits_simt(const tq_ctx* ctx, const float* q, int B, int Hq,
                                const uint8_t* payload, const uint16_t* norms, float scale, float* out,
                                ChannelGather gather, int accumulate, cudaStream_t st);
 
+// Value path (k_attend.cu)
+bool attend_supported(const tq_ctx* ctx, int Hq, int Hkv);
+size_t attend_ws_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int64_t S);
+cudaError_t launch_attend(const tq_ctx* ctx, const float* logits, int B, int Hq, int Hkv, int64_t S,
+                          const uint8_t* payload, const uint16_t* norms, float* out, void* ws, cudaStream_t st);
+
 // Channel split (k_split.cu, k_quantize_tc.cu, k_logits.cu)
 size_t split_plan_ws_bytes(const tq_split* sp);
 cudaError_t launch_split_plan(tq_split* sp, const void* keys, int dtype, int B, int64_t S, void* ws,

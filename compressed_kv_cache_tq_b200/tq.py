@@ -55,6 +55,8 @@ def lib() -> ctypes.CDLL:
             "tq_topk_workspace_bytes": (sz, [vp, i64, i64, i32]),
             "tq_topk": (i32, [vp, vp, i64, vp, vp, i64, i32, vp, vp, vp, sz, vp]),
             "tq_check_device_status": (i32, [vp, vp, ctypes.POINTER(u32)]),
+            "tq_attend_workspace_bytes": (sz, [vp, i32, i32, i32, i64]),
+            "tq_attend": (i32, [vp, vp, i32, i32, i32, i64, vp, vp, vp, vp, sz, vp]),
             "tq_split_create": (i32, [vp, vp, i32, ctypes.POINTER(vp)]),
             "tq_split_free": (None, [vp]),
             "tq_split_plan_workspace_bytes": (sz, [vp]),
@@ -77,7 +79,8 @@ def lib() -> ctypes.CDLL:
 
 EXPORTED = ["tq_init", "tq_init_ex", "tq_host_tables", "tq_free", "tq_info", "tq_export_tables", "tq_quantize", "tq_dequantize",
             "tq_logits_workspace_bytes", "tq_logits", "tq_logits_noalloc", "tq_topk_workspace_bytes", "tq_topk",
-            "tq_check_device_status", "tq_strerror", "tq_last_cuda_error", "tq_split_create", "tq_split_free",
+            "tq_check_device_status", "tq_strerror", "tq_last_cuda_error", "tq_attend_workspace_bytes", "tq_attend",
+            "tq_split_create", "tq_split_free",
             "tq_split_plan_workspace_bytes", "tq_split_plan", "tq_split_set_plan", "tq_split_get_plan",
             "tq_split_quantize", "tq_split_logits_workspace_bytes", "tq_split_logits"]
 
@@ -241,6 +244,31 @@ def tq_logits_noalloc(ctx: Context, q: torch.Tensor, payload: torch.Tensor, norm
         out = torch.empty((B, Hq, S), dtype=torch.float32, device=q.device)
     _check(lib().tq_logits_noalloc(ctx.handle, _ptr(q), B, Hq, Hkv, S, _ptr(payload), _ptr(norms), float(scale),
                                    _ptr(out), ctypes.c_void_p(_stream(stream))), "tq_logits_noalloc")
+    return out
+
+
+def tq_attend_workspace_bytes(ctx: Context, B: int, Hq: int, Hkv: int, S: int) -> int:
+    return int(lib().tq_attend_workspace_bytes(ctx.handle, B, Hq, Hkv, S))
+
+
+def tq_attend(ctx: Context, logits: torch.Tensor, payload: torch.Tensor, norms: torch.Tensor, Hkv: int,
+              out: torch.Tensor | None = None, workspace: torch.Tensor | None = None, stream=None):
+    """logits (B, Hq, S) fp32 against a value cache (rows (B, Hkv, S)) -> out (B, Hq, d) fp32."""
+    _need_cuda(logits, "logits")
+    _need_cuda(payload, "payload")
+    _need_cuda(norms, "norms")
+    if logits.dtype != torch.float32 or logits.dim() != 3:
+        raise ValueError("logits must be float32 (B, Hq, S)")
+    B, Hq, S = logits.shape
+    if payload.shape[0] != B * Hkv * S:
+        raise ValueError("payload rows must be B * Hkv * S")
+    if out is None:
+        out = torch.empty((B, Hq, ctx.d), dtype=torch.float32, device=logits.device)
+    ws_bytes = tq_attend_workspace_bytes(ctx, B, Hq, Hkv, S)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=logits.device)
+    _check(lib().tq_attend(ctx.handle, _ptr(logits), B, Hq, Hkv, S, _ptr(payload), _ptr(norms), _ptr(out),
+                           _ptr(workspace), workspace.numel(), ctypes.c_void_p(_stream(stream))), "tq_attend")
     return out
 
 

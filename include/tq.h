@@ -171,6 +171,25 @@ tq_status tq_logits_noalloc(const tq_ctx* ctx, const float* q, int B, int Hq, in
                             const uint8_t* payload, const uint16_t* norms, float scale, float* out,
                             void* stream);
 
+/* Workspace bytes of tq_attend (per-chunk partial sums). */
+size_t tq_attend_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int64_t S);
+
+/* Decode attention output over a quantised value cache (the value path;
+ * mooersco.com sections 1.2-1.3: the softmax of the logits weights the
+ * values, and the output is recovered from the compressed values).  The
+ * values are rows of ctx's packed layout ([B][Hkv][S], quantised with
+ * tq_quantize under their own context); each enters through its unbiased
+ * reconstruction v_hat = n16 R^T c[idx] + sqrt(pi/2)/m rho16 S^T sigma (the
+ * first term only when ctx->m = 0):
+ *   out[b, h] = sum_s softmax(logits[b, h, :])_s v_hat[b, h / (Hq/Hkv), s].
+ * logits: device fp32 [B, Hq, S], already scaled (for instance tq_logits'
+ * output).  out: device fp32 [B, Hq, d].  S = 0 gives zeros.
+ * Hq / Hkv <= 8 (TQ_ERR_UNSUPPORTED otherwise).
+ * workspace: device, 256-byte aligned, >= tq_attend_workspace_bytes. */
+tq_status tq_attend(const tq_ctx* ctx, const float* logits, int B, int Hq, int Hkv, int64_t S,
+                    const uint8_t* payload, const uint16_t* norms, float* out, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
 /* Workspace bytes tq_topk needs for nq queries against n database rows. */
 size_t tq_topk_workspace_bytes(const tq_ctx* ctx, int64_t nq, int64_t n, int k);
 
