@@ -62,16 +62,21 @@ KV_WORKLOADS = {
     # the decode layer with a quantised value cache as well (values b = 4,
     # tables of their own): quantize keys and values, logits, attention output
     "attend": (8, 8, 32, 128, 32768, 4, 1001, "decode_attention_llama31_8b_layer_b8_hkv8_hq32_d128_s32768_b4"),
+    # the MSE-only variant (stage 1 alone, no sign sketch) on the decode layer:
+    # b = 4 gives 3 Lloyd-Max bits per coordinate, 48-byte rows
+    "mse": (8, 8, 32, 128, 32768, 4, 1001, "decode_mse_only_llama31_8b_layer_b8_hkv8_hq32_d128_s32768_b4_m0"),
 }
 SEED_VALUES = 2002
 ATTEND = False
+JL_ROWS = None   # m of the key quantizer (None: m = d; 0: the MSE-only variant)
 
 
 def set_workload(name: str, seq: int | None = None):
     """Point the module's shape globals at one of KV_WORKLOADS (seq overrides S)."""
-    global B, HKV, HQ, D, S, BITS, SEED_KEYS, WORKLOAD, ATTEND
+    global B, HKV, HQ, D, S, BITS, SEED_KEYS, WORKLOAD, ATTEND, JL_ROWS
     B, HKV, HQ, D, S, BITS, SEED_KEYS, WORKLOAD = KV_WORKLOADS[name]
     ATTEND = name == "attend"
+    JL_ROWS = 0 if name == "mse" else None
     if seq is not None and seq != S:
         WORKLOAD = WORKLOAD.replace(f"_s{S}_", f"_s{seq}_")
         S = seq
@@ -158,7 +163,8 @@ def bytes_per_key():
         g = D // 2
         row = sum(g * (b - 1) // 8 + g // 8 + 4 for b in BITS)
     else:
-        row = D * (BITS - 1) // 8 + D // 8 + 4
+        m = D if JL_ROWS is None else JL_ROWS
+        row = D * (BITS - 1) // 8 + m // 8 + 4
     bpk = {"quantize_in": 2 * D, "quantize_out": row, "logits_in": row, "logits_out": 4 * (HQ // HKV)}
     if ATTEND:
         # keys and values are both quantised; the attention reads the value
@@ -172,7 +178,8 @@ def quantize_flops_per_key():
     if isinstance(BITS, tuple):
         g = D // 2
         return 2 * (2 * g * g + 2 * g * g)
-    return 2 * D * D + 2 * D * D
+    m = D if JL_ROWS is None else JL_ROWS
+    return 2 * D * D + 2 * m * D
 
 
 def cpu_baseline(budget_s: float = 12.0, max_keys: int = 1 << 19):
@@ -194,7 +201,7 @@ def cpu_baseline(budget_s: float = 12.0, max_keys: int = 1 << 19):
         tb_hi = O.make_tables(D // 2, BITS[0], SEED_TABLES)
         tb_lo = O.make_tables(D // 2, BITS[1], SEED_TABLES + 1)
     else:
-        tb = O.make_tables(D, BITS, SEED_TABLES)
+        tb = O.make_tables(D, BITS, SEED_TABLES, m=JL_ROWS)
     scales = W.head_channel_scales(HKV, D, SEED_KEYS)
     if ATTEND:
         tbv = O.make_tables(D, BITS, SEED_TABLES + 100)
@@ -433,6 +440,7 @@ def result_line(*, world, n, steps, warmup, ms, q_ms, l_ms, e2e_ms, h2d, d2h, cl
                    "q_heads": HQ, "head_dim": D,
                    "bits": ({"high_64_channels": BITS[0], "low_64_channels": BITS[1]} if isinstance(BITS, tuple)
                             else BITS),
+                   "jl_rows": D if JL_ROWS is None else JL_ROWS,
                    "parallelism": f"replicas x{world}",
                    "l2": f"inputs larger than L2: keys {n * D * 2 / 1e6:.0f} MB, packed caches "
                          f"{n * (bpk['quantize_out']) / 1e6:.0f} MB each; logits read the cache written one step "
@@ -458,7 +466,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="decode", choices=["decode", "longctx", "split", "attend", "search"])
+    ap.add_argument("--workload", default="decode", choices=["decode", "longctx", "split", "attend", "mse", "search"])
     ap.add_argument("--rows", type=int, default=1_000_000, help="search: database rows")
     ap.add_argument("--queries", type=int, default=10_000, help="search: queries")
     ap.add_argument("--seq", type=int, default=None,
@@ -527,7 +535,7 @@ def main():
         def logits(qq, c):
             tq.tq_split_logits(sp, qq, *c, scale=scale, out=out, workspace=ws)
     else:
-        ctx = tq.tq_init(D, BITS, SEED_TABLES)
+        ctx = tq.tq_init(D, BITS, SEED_TABLES, m=JL_ROWS)
         caches = [(torch.empty((n, ctx.row_bytes), dtype=torch.uint8, device=dev),
                    torch.empty((n, 2), dtype=torch.float16, device=dev)) for _ in range(2)]
         ws = torch.empty(tq.tq_logits_workspace_bytes(ctx, B, HQ, HKV), dtype=torch.uint8, device=dev)

@@ -31,39 +31,31 @@ namespace {
 
 constexpr int kAttThreads = 256;
 constexpr int kAttWarps = kAttThreads / 32;
-constexpr int kAttTile = 64;          // keys per staged tile
-constexpr int kAttMaxLd = 4;          // 8-byte words per thread per tile (rows of up to 128 bytes)
+constexpr int kAttTile = 128;         // keys per staged tile
+constexpr int kAttMaxLd = 8;          // 8-byte words per thread per tile (rows of up to 128 bytes)
 constexpr int kAttMaxHeads = 8;
 
 __device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
 
-// Codes of the 4 coordinates (r = 4u + i, e = 0..3) of one slot from the
-// unit's code halfwords h[0 .. BM-1] (layout in include/tq.h).
+// The slot's 4 codes (r = 4u + i, e = 0..3) as nibbles e of one word, from the
+// unit's code halfwords h[0 .. BM-1] (layout in include/tq.h): code e is
+// (v >> 4e) & (2^BM - 1).  For b' = 3, register 3's code bits sit in bit 3 of
+// the nibbles of h0, h1, h2 and are gathered first.
 template <int BM>
-__device__ __forceinline__ void slot_codes(const uint32_t (&h)[BM], int i, int (&code)[4]) {
+__device__ __forceinline__ uint32_t slot_word(const uint32_t (&h)[BM], int i) {
   if constexpr (BM == 1) {
-#pragma unroll
-    for (int e = 0; e < 4; ++e) code[e] = (h[0] >> (4 * e + i)) & 1;
+    return (h[0] >> i) & 0x1111u;
   } else if constexpr (BM == 2) {
-    const uint32_t hs = (i >> 1) ? h[1] : h[0];
-    const int sh = 2 * (i & 1);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) code[e] = (hs >> (4 * e + sh)) & 3;
+    return (((i >> 1) ? h[1] : h[0]) >> (2 * (i & 1))) & 0x3333u;
   } else {
-    const uint32_t hs = i == 0 ? h[0] : (i == 1 ? h[1] : h[2]);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int lo = (hs >> (4 * e)) & 7;
-      const int hi = ((h[0] >> (4 * e + 3)) & 1) | (((h[1] >> (4 * e + 3)) & 1) << 1) |
-                     (((h[2] >> (4 * e + 3)) & 1) << 2);
-      code[e] = i < 3 ? lo : hi;
-    }
+    const uint32_t r3 = ((h[0] >> 3) & 0x1111u) | ((h[1] >> 2) & 0x2222u) | ((h[2] >> 1) & 0x4444u);
+    return i == 3 ? r3 : ((i == 0 ? h[0] : (i == 1 ? h[1] : h[2])) & 0x7777u);
   }
 }
 
 // Partials: part[((grp * nsplit + split) * G + h) * (2 + dp + mp)] = {max, sum, a[dp], b[mp]}.
 template <int BM, int GP, int NS>
-__global__ void __launch_bounds__(kAttThreads) attend_partial_kernel(
+__global__ void __launch_bounds__(kAttThreads, GP * NS <= 4 ? 3 : 1) attend_partial_kernel(
     const float* __restrict__ logits, int Hq, int Hkv, int64_t S, int64_t chunk, int nsplit,
     const uint8_t* __restrict__ payload, const uint16_t* __restrict__ norms, RowGeom g, CodebookParams cb,
     float* __restrict__ part) {
@@ -96,10 +88,22 @@ __global__ void __launch_bounds__(kAttThreads) attend_partial_kernel(
   float mx[GP];
 #pragma unroll
   for (int h = 0; h < GP; ++h) mx[h] = -INFINITY;
-  for (int64_t s = s_begin + tid; s < s_end; s += kAttThreads)
+  // eight independent loads in flight per thread and head
+  for (int64_t s = s_begin + tid; s < s_end; s += 8 * kAttThreads) {
 #pragma unroll
-    for (int h = 0; h < GP; ++h)
-      if (h < G) mx[h] = fmaxf(mx[h], lg[size_t(h) * S + s]);
+    for (int h = 0; h < GP; ++h) {
+      if (h < G) {
+        float v[8];
+#pragma unroll
+        for (int x = 0; x < 8; ++x) {
+          const int64_t sx = s + int64_t(x) * kAttThreads;
+          v[x] = sx < s_end ? __ldg(lg + size_t(h) * S + sx) : -INFINITY;
+        }
+#pragma unroll
+        for (int x = 0; x < 8; ++x) mx[h] = fmaxf(mx[h], v[x]);
+      }
+    }
+  }
 #pragma unroll
   for (int h = 0; h < GP; ++h) {
     float v = mx[h];
@@ -139,7 +143,7 @@ __global__ void __launch_bounds__(kAttThreads) attend_partial_kernel(
         accC[ns][hp][e] = make_float2(0.f, 0.f);
         accS[ns][hp][e] = make_float2(0.f, 0.f);
       }
-  // weights: thread (key k = tid % 64, head tid / 64 + 4 it) of each tile
+  // weights: thread (key k = tid % kAttTile, head tid / kAttTile + 2 it) of each tile
   constexpr int kWIt = (kAttTile * GP + kAttThreads - 1) / kAttThreads;
   float lsum[kWIt];
 #pragma unroll
@@ -148,6 +152,8 @@ __global__ void __launch_bounds__(kAttThreads) attend_partial_kernel(
   // pass 2: tiles of keys, staged one ahead in registers
   const int words = kAttTile * rb / 8;
   uint2 ld[kAttMaxLd];
+  float lgv[kWIt];      // logit of this thread's (key, head) pairs in the next tile
+  uint32_t nnv[kWIt];   // and the key's norms
   auto fetch = [&](int64_t s0) {
     const int nk = int(s_end - s0 < kAttTile ? s_end - s0 : kAttTile);
     const int nw = nk * rb / 8;
@@ -156,6 +162,14 @@ __global__ void __launch_bounds__(kAttThreads) attend_partial_kernel(
     for (int k = 0; k < kAttMaxLd; ++k) {
       const int w = tid + k * kAttThreads;
       ld[k] = (w < nw) ? __ldg(src + w) : make_uint2(0u, 0u);
+    }
+#pragma unroll
+    for (int it = 0; it < kWIt; ++it) {
+      const int idx = tid + it * kAttThreads;
+      const int k = idx % kAttTile, h = idx / kAttTile;
+      const bool ok = k < nk && h < G;
+      lgv[it] = ok ? __ldg(lg + size_t(h) * S + s0 + k) : 0.f;
+      nnv[it] = ok ? __ldg(nrm + s0 + k) : 0u;
     }
   };
   const bool have = s_begin < s_end;
@@ -175,8 +189,8 @@ __global__ void __launch_bounds__(kAttThreads) attend_partial_kernel(
         const int k = idx % kAttTile, h = idx / kAttTile;
         float wn = 0.f, wr = 0.f;
         if (k < nk && h < G) {
-          const float w = expf(lg[size_t(h) * S + s0 + k] - smx[h]);
-          const uint32_t nn = __ldg(nrm + s0 + k);
+          const float w = expf(lgv[it] - smx[h]);
+          const uint32_t nn = nnv[it];
           const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&nn));
           wn = w * f.x;
           wr = w * f.y;
@@ -203,20 +217,22 @@ __global__ void __launch_bounds__(kAttThreads) attend_partial_kernel(
           uint32_t h[BM];
 #pragma unroll
           for (int x = 0; x < BM; ++x) h[x] = hw[c_off[ns] + x];
-          int code[4];
-          slot_codes<BM>(h, c_i[ns], code);
+          const uint32_t v = slot_word<BM>(h, c_i[ns]);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float2 cv = f2(sc[code[e]]);
+            const float2 cv = f2(sc[(v >> (4 * e)) & 7u]);
 #pragma unroll
             for (int hp = 0; hp < GP / 2; ++hp) accC[ns][hp][e] = __ffma2_rn(cv, wn2[hp], accC[ns][hp][e]);
           }
         }
         if (t < nslot_s) {
+          // sign bit 4e + i of the halfword moved to bit 31 and inverted: +1.0f for a set bit, -1.0f otherwise
           const uint32_t hs = hw[s_off[ns]];
+          const int sh0 = 31 - s_i[ns];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float2 sg = f2(((hs >> (4 * e + s_i[ns])) & 1u) ? 1.f : -1.f);
+            const uint32_t x = hs << (sh0 - 4 * e);
+            const float2 sg = f2(__uint_as_float((~x & 0x80000000u) | 0x3f800000u));
 #pragma unroll
             for (int hp = 0; hp < GP / 2; ++hp) accS[ns][hp][e] = __ffma2_rn(sg, wr2[hp], accS[ns][hp][e]);
           }
@@ -244,7 +260,7 @@ __global__ void __launch_bounds__(kAttThreads) attend_partial_kernel(
         }
       }
   }
-  // every lane of a warp holds the same head in lsum[it] (32 consecutive keys)
+  // every lane of a warp holds the same head in lsum[it] (32 consecutive keys of one head)
 #pragma unroll
   for (int it = 0; it < kWIt; ++it) {
     float v = lsum[it];
@@ -329,16 +345,28 @@ AttPlan att_plan(int B, int Hkv, int64_t S) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  // key chunks per (batch, KV head): the number of waves of resident blocks
+  // (three per SM) times the chunk length is the time; take the split count
+  // that minimises it, with a small cost per split for the merge
   const int64_t groups = int64_t(B) * Hkv;
-  int64_t ns = (int64_t(sms) * 4 + groups - 1) / groups;
-  const int64_t max_ns = (S + kAttTile - 1) / kAttTile;
-  if (ns > max_ns) ns = max_ns;
-  if (ns > 1024) ns = 1024;
-  if (ns < 1) ns = 1;
-  int64_t chunk = (S + ns - 1) / ns;
+  const int64_t cap = int64_t(sms) * 3;
+  int64_t max_ns = (S + kAttTile - 1) / kAttTile;
+  if (max_ns > 1024) max_ns = 1024;
+  if (max_ns < 1) max_ns = 1;
+  int64_t best = 1;
+  double best_cost = 1e300;
+  for (int64_t ns = 1; ns <= max_ns; ++ns) {
+    const double waves = double((groups * ns + cap - 1) / cap);
+    const double cost = waves / double(ns) + 0.0002 * double(ns);
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = ns;
+    }
+  }
+  int64_t chunk = (S + best - 1) / best;
   chunk = (chunk + kAttTile - 1) / kAttTile * kAttTile;
   if (chunk < kAttTile) chunk = kAttTile;
-  ns = (S + chunk - 1) / chunk;
+  int64_t ns = (S + chunk - 1) / chunk;
   if (ns < 1) ns = 1;
   return AttPlan{int(ns), chunk};
 }

@@ -22,6 +22,7 @@
 #include <cuda_fp16.h>
 
 #include <algorithm>
+#include <type_traits>
 
 #include "tq_device.cuh"
 #include "tq_internal.h"
@@ -73,9 +74,10 @@ __global__ void __launch_bounds__(128) qprep_kernel(const float* __restrict__ q,
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(uint32_t(__cvta_generic_to_shared(matR + 4 * i))),
                  "l"(Rt + 4 * i)
                  : "memory");
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(uint32_t(__cvta_generic_to_shared(matP + 4 * i))),
-                 "l"(Pt + 4 * i)
-                 : "memory");
+    if (Pt)   // no JL matrix in the MSE-only variant
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(uint32_t(__cvta_generic_to_shared(matP + 4 * i))),
+                   "l"(Pt + 4 * i)
+                   : "memory");
   }
   for (int h = 0; h < slots; ++h) sq[h * D + tid] = h < G ? q[(size_t(b) * Hq + hkv * G + h) * D + tid] : 0.f;
   asm volatile("cp.async.wait_all;" ::: "memory");
@@ -97,12 +99,14 @@ __global__ void __launch_bounds__(128) qprep_kernel(const float* __restrict__ q,
   float accy[kMaxSlots];
 #pragma unroll
   for (int h = 0; h < kMaxSlots; ++h) accy[h] = 0.f;
+  if (Pt) {
 #pragma unroll 4
-  for (int j = 0; j < D; ++j) {
-    const float p = matP[j * D + tid];
+    for (int j = 0; j < D; ++j) {
+      const float p = matP[j * D + tid];
 #pragma unroll
-    for (int h = 0; h < kMaxSlots; ++h)
-      if (h < slots) accy[h] = fmaf(p, sx[h * D + j], accy[h]);
+      for (int h = 0; h < kMaxSlots; ++h)
+        if (h < slots) accy[h] = fmaf(p, sx[h * D + j], accy[h]);
+    }
   }
   // per-slot max |x|, max |y|
 #pragma unroll
@@ -184,16 +188,27 @@ __device__ __forceinline__ void mma_s8_first(int (&c)[4], uint32_t a0, uint32_t 
 
 // Chunk of one key for one quarter: BMSE * 2 halfwords of codes (two units)
 // and 2 halfwords of signs, as 32-bit words.
-template <int BMSE>
+template <int BMSE, bool JL = true>
 struct Chunk {
-  static constexpr int kWords = BMSE + 1;
+  static constexpr int kWords = BMSE + (JL ? 1 : 0);
   uint32_t w[kWords];
 };
 
-template <int BMSE>
-__device__ __forceinline__ void load_chunk(Chunk<BMSE>& c, const uint8_t* row, int tig, bool ok) {
-  const uint32_t* p = reinterpret_cast<const uint32_t*>(row + tig * 4 * (BMSE + 1));
-  if constexpr (BMSE == 3) {
+template <int BMSE, bool JL>
+__device__ __forceinline__ void load_chunk(Chunk<BMSE, JL>& c, const uint8_t* row, int tig, bool ok) {
+  constexpr int kW = Chunk<BMSE, JL>::kWords;
+  const uint32_t* p = reinterpret_cast<const uint32_t*>(row + tig * 4 * kW);
+  if constexpr (!JL) {
+    // MSE-only rows: the quarter's code words only (4 BMSE bytes)
+    if constexpr (kW == 2) {
+      const uint2 v = ok ? __ldg(reinterpret_cast<const uint2*>(p)) : make_uint2(0, 0);
+      c.w[0] = v.x;
+      c.w[1] = v.y;
+    } else {
+#pragma unroll
+      for (int i = 0; i < kW; ++i) c.w[i] = ok ? __ldg(p + i) : 0u;
+    }
+  } else if constexpr (BMSE == 3) {
     uint4 v = ok ? __ldg(reinterpret_cast<const uint4*>(p)) : make_uint4(0, 0, 0, 0);
     c.w[0] = v.x;
     c.w[1] = v.y;
@@ -210,15 +225,15 @@ __device__ __forceinline__ void load_chunk(Chunk<BMSE>& c, const uint8_t* row, i
 }
 
 // Halfword h of the chunk (h = 0 .. 2 BMSE + 1) in the low 16 bits.
-template <int BMSE>
-__device__ __forceinline__ uint32_t chunk_half(const Chunk<BMSE>& c, int h) {
+template <int BMSE, bool JL>
+__device__ __forceinline__ uint32_t chunk_half(const Chunk<BMSE, JL>& c, int h) {
   return (h & 1) ? (c.w[h >> 1] >> 16) : c.w[h >> 1];
 }
 
 // Byte-permute selectors (4 nibbles, mode bit clear) for the 8 registers of a
 // quarter: codes of register r, nibble e = coordinate (r, e).
-template <int BMSE>
-__device__ __forceinline__ void code_selectors(const Chunk<BMSE>& c, uint32_t (&sel)[8]) {
+template <int BMSE, bool JL>
+__device__ __forceinline__ void code_selectors(const Chunk<BMSE, JL>& c, uint32_t (&sel)[8]) {
 #pragma unroll
   for (int u = 0; u < 2; ++u) {
     if constexpr (BMSE == 3) {
@@ -248,8 +263,8 @@ __device__ __forceinline__ void code_selectors(const Chunk<BMSE>& c, uint32_t (&
 // Masking that bit in place gives selector nibbles 0 or 2^i; the two byte
 // tables put -1 at byte 0 and +1 at byte 2^i (bit 3 is the byte-permute mode
 // bit, so register 4u + 3 shifts it down to bit 2 first).
-template <int BMSE>
-__device__ __forceinline__ void sign_operands(const Chunk<BMSE>& c, uint32_t (&a)[8]) {
+template <int BMSE, bool JL>
+__device__ __forceinline__ void sign_operands(const Chunk<BMSE, JL>& c, uint32_t (&a)[8]) {
 #pragma unroll
   for (int u = 0; u < 2; ++u) {
     const uint32_t h = chunk_half(c, 2 * BMSE + u);
@@ -261,16 +276,16 @@ __device__ __forceinline__ void sign_operands(const Chunk<BMSE>& c, uint32_t (&a
 }
 
 // One 16-key MMA row tile of a 32-key tile: decode, multiply, combine, store.
-template <int BMSE, int NT>
-__device__ __forceinline__ void row_tile(const Chunk<BMSE>& ca, const Chunk<BMSE>& cb, uint32_t na, uint32_t nb,
+template <int BMSE, int NT, bool JL>
+__device__ __forceinline__ void row_tile(const Chunk<BMSE, JL>& ca, const Chunk<BMSE, JL>& cb, uint32_t na, uint32_t nb,
                                          bool okA, bool okB, const uint32_t (&bx)[NT][KS][2],
                                          const uint32_t (&by)[NT][KS][2], const float (&sc_code)[NT],
                                          const float (&sc_sign)[NT], float* const (&orow)[NT], int g, const CodeLut& lut) {
   int acc_hi[NT][4], acc_lo[NT][4], acc_sg[NT][4];
   {
     uint32_t sa[8], sb[8];
-    code_selectors<BMSE>(ca, sa);
-    code_selectors<BMSE>(cb, sb);
+    code_selectors<BMSE, JL>(ca, sa);
+    code_selectors<BMSE, JL>(cb, sb);
 #pragma unroll
     for (int s = 0; s < KS; ++s) {
       const uint32_t ah0 = prmt(lut.hi[0], lut.hi[1], sa[2 * s]), ah1 = prmt(lut.hi[0], lut.hi[1], sb[2 * s]);
@@ -291,12 +306,12 @@ __device__ __forceinline__ void row_tile(const Chunk<BMSE>& ca, const Chunk<BMSE
       }
     }
   }
-  {
+  if constexpr (JL) {
     // sign registers: selectors keep one bit per nibble; the byte table maps
     // that bit's two possible selector values to -1 and +1
     uint32_t ga[8], gb[8];
-    sign_operands<BMSE>(ca, ga);
-    sign_operands<BMSE>(cb, gb);
+    sign_operands<BMSE, JL>(ca, ga);
+    sign_operands<BMSE, JL>(cb, gb);
 #pragma unroll
     for (int s = 0; s < KS; ++s)
 #pragma unroll
@@ -315,8 +330,8 @@ __device__ __forceinline__ void row_tile(const Chunk<BMSE>& ca, const Chunk<BMSE
     // |cross terms| <= 2 * 128 * 128 * 128 and |low terms| < 2^21: the integer sums fit in 32 bits
     const float codeA = fmaf(float(acc_hi[nt][0]), 65536.f, float((acc_hi[nt][1] + acc_lo[nt][0]) * 256 + acc_lo[nt][1]));
     const float codeB = fmaf(float(acc_hi[nt][2]), 65536.f, float((acc_hi[nt][3] + acc_lo[nt][2]) * 256 + acc_lo[nt][3]));
-    const float signA = float(acc_sg[nt][0] * 256 + acc_sg[nt][1]);
-    const float signB = float(acc_sg[nt][2] * 256 + acc_sg[nt][3]);
+    const float signA = JL ? float(acc_sg[nt][0] * 256 + acc_sg[nt][1]) : 0.f;
+    const float signB = JL ? float(acc_sg[nt][2] * 256 + acc_sg[nt][3]) : 0.f;
     if (orow[nt]) {
       if (okA) orow[nt][g] = fmaf(fa.x * sc_code[nt], codeA, fa.y * sc_sign[nt] * signA);
       if (okB) orow[nt][g + 8] = fmaf(fb.x * sc_code[nt], codeB, fb.y * sc_sign[nt] * signB);
@@ -326,12 +341,12 @@ __device__ __forceinline__ void row_tile(const Chunk<BMSE>& ca, const Chunk<BMSE
 
 // Each warp streams a contiguous range of 32-key tiles (two MMA row tiles
 // sharing the query fragments of their (batch, KV head) group).
-template <int BMSE, int NT>
+template <int BMSE, int NT, bool JL>
 __global__ void __launch_bounds__(kLogitThreads) logits_mma_kernel(
     const uint8_t* __restrict__ payload, const uint16_t* __restrict__ norms, int64_t S, int Hq, int Hkv,
     int64_t total_tiles, const uint32_t* __restrict__ frags, const HeadScale* __restrict__ hscale, CodeLut lut,
     float* __restrict__ out) {
-  constexpr int kRowBytes = D * BMSE / 8 + D / 8;
+  constexpr int kRowBytes = D * BMSE / 8 + (JL ? D / 8 : 0);
   const int lane = threadIdx.x & 31;
   const int g = lane >> 2, tig = lane & 3;
   const int64_t nwarps = int64_t(gridDim.x) * (kLogitThreads / 32);
@@ -344,16 +359,16 @@ __global__ void __launch_bounds__(kLogitThreads) logits_mma_kernel(
   int64_t grp = t_begin / tpp;
   int64_t s0 = (t_begin - grp * tpp) * 32;
 
-  auto load_tile = [&](int64_t gi, int64_t so, Chunk<BMSE> (&c)[4], uint32_t (&nn)[4]) {
+  auto load_tile = [&](int64_t gi, int64_t so, Chunk<BMSE, JL> (&c)[4], uint32_t (&nn)[4]) {
     const int64_t row0 = gi * S + so + g;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const bool ok = so + g + 8 * k < S;
-      load_chunk<BMSE>(c[k], payload + (row0 + 8 * k) * kRowBytes, tig, ok);
+      load_chunk<BMSE, JL>(c[k], payload + (row0 + 8 * k) * kRowBytes, tig, ok);
       nn[k] = ok ? __ldg(reinterpret_cast<const uint32_t*>(norms) + row0 + 8 * k) : 0u;
     }
   };
-  Chunk<BMSE> cur[4];
+  Chunk<BMSE, JL> cur[4];
   uint32_t curn[4];
   if (t_begin < t_end) load_tile(grp, s0, cur, curn);
 
@@ -393,19 +408,19 @@ __global__ void __launch_bounds__(kLogitThreads) logits_mma_kernel(
       ns0 = 0;
       ++ngrp;
     }
-    Chunk<BMSE> nxt[4];
+    Chunk<BMSE, JL> nxt[4];
     uint32_t nxtn[4] = {0u, 0u, 0u, 0u};
     if (t + 1 < t_end) load_tile(ngrp, ns0, nxt, nxtn);
 
     float* orow_t[NT];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) orow_t[nt] = orow[nt] ? orow[nt] + s0 : nullptr;
-    row_tile<BMSE, NT>(cur[0], cur[1], curn[0], curn[1], s0 + g < S, s0 + g + 8 < S, bx, by, sc_code, sc_sign,
-                       orow_t, g, lut);
+    row_tile<BMSE, NT, JL>(cur[0], cur[1], curn[0], curn[1], s0 + g < S, s0 + g + 8 < S, bx, by, sc_code, sc_sign,
+                           orow_t, g, lut);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) orow_t[nt] = orow[nt] ? orow[nt] + s0 + 16 : nullptr;
-    row_tile<BMSE, NT>(cur[2], cur[3], curn[2], curn[3], s0 + g + 16 < S, s0 + g + 24 < S, bx, by, sc_code,
-                       sc_sign, orow_t, g, lut);
+    row_tile<BMSE, NT, JL>(cur[2], cur[3], curn[2], curn[3], s0 + g + 16 < S, s0 + g + 24 < S, bx, by, sc_code,
+                           sc_sign, orow_t, g, lut);
 
     if (t + 1 < t_end) {
       if (ngrp != grp) load_group(ngrp);
@@ -473,14 +488,16 @@ int sm_count() {
   return sms;
 }
 
-bool fast_path(const tq_ctx* ctx) { return ctx->d == D && ctx->m == D && ctx->bmse >= 1 && ctx->bmse <= 3; }
+bool fast_path(const tq_ctx* ctx) {
+  return ctx->d == D && (ctx->m == D || ctx->m == 0) && ctx->bmse >= 1 && ctx->bmse <= 3;
+}
 
-template <int BMSE, int NT>
+template <int BMSE, int NT, bool JL>
 cudaError_t launch_mma(const tq_ctx* ctx, int B, int Hq, int Hkv, int64_t S, const uint8_t* payload,
                        const uint16_t* norms, float* out, const uint32_t* frags, const HeadScale* hs,
                        cudaStream_t st) {
   const int64_t total = int64_t(B) * Hkv * ((S + 31) / 32);
-  auto kern = logits_mma_kernel<BMSE, NT>;
+  auto kern = logits_mma_kernel<BMSE, NT, JL>;
   int per_sm = 1;
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kLogitThreads, 0);
   int64_t grid = int64_t(sm_count()) * (per_sm > 0 ? per_sm : 1);
@@ -888,14 +905,18 @@ cudaError_t launch_logits(const tq_ctx* ctx, const float* q, int B, int Hq, int 
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (S == 0) return cudaSuccess;
-  switch (ctx->bmse * 10 + nt) {
-    case 11: return launch_mma<1, 1>(ctx, B, Hq, Hkv, S, payload, norms, out, frags, hs, st);
-    case 12: return launch_mma<1, 2>(ctx, B, Hq, Hkv, S, payload, norms, out, frags, hs, st);
-    case 21: return launch_mma<2, 1>(ctx, B, Hq, Hkv, S, payload, norms, out, frags, hs, st);
-    case 22: return launch_mma<2, 2>(ctx, B, Hq, Hkv, S, payload, norms, out, frags, hs, st);
-    case 31: return launch_mma<3, 1>(ctx, B, Hq, Hkv, S, payload, norms, out, frags, hs, st);
-    default: return launch_mma<3, 2>(ctx, B, Hq, Hkv, S, payload, norms, out, frags, hs, st);
-  }
+  auto go = [&](auto jl) -> cudaError_t {
+    constexpr bool J = decltype(jl)::value;
+    switch (ctx->bmse * 10 + nt) {
+      case 11: return launch_mma<1, 1, J>(ctx, B, Hq, Hkv, S, payload, norms, out, frags, hs, st);
+      case 12: return launch_mma<1, 2, J>(ctx, B, Hq, Hkv, S, payload, norms, out, frags, hs, st);
+      case 21: return launch_mma<2, 1, J>(ctx, B, Hq, Hkv, S, payload, norms, out, frags, hs, st);
+      case 22: return launch_mma<2, 2, J>(ctx, B, Hq, Hkv, S, payload, norms, out, frags, hs, st);
+      case 31: return launch_mma<3, 1, J>(ctx, B, Hq, Hkv, S, payload, norms, out, frags, hs, st);
+      default: return launch_mma<3, 2, J>(ctx, B, Hq, Hkv, S, payload, norms, out, frags, hs, st);
+    }
+  };
+  return ctx->m > 0 ? go(std::true_type{}) : go(std::false_type{});
 }
 
 namespace {

@@ -152,7 +152,7 @@ __device__ __forceinline__ uint2 cell2(float2 y, float s128, const HalfBook& hb,
   return make_uint2(__float_as_uint(idx.x), __float_as_uint(idx.y));
 }
 
-template <int BMSE>
+template <int BMSE, bool JL>
 __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid_constant__ CUtensorMap key_map,
                                                                    int64_t n, const uint8_t* __restrict__ bimg,
                                                                    HalfBook book,
@@ -205,8 +205,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
     if (warp == 0) {
       // ------------------------------------------------------------ TMA producer
       if (lane == 0) {
-        mbar_expect_tx(bar(kBarConst), kConstBytes);
-        for (int c = 0; c < int(kConstBytes / 16384u); ++c)
+        // R_hi, R_lo and (with the sign sketch) P
+        constexpr uint32_t kConst = JL ? kConstBytes : kOffP;
+        mbar_expect_tx(bar(kBarConst), kConst);
+        for (int c = 0; c < int(kConst / 16384u); ++c)
           bulk_load(base + 16384u * c, bimg + 16384 * c, 16384u, bar(kBarConst));
         int64_t i = 0;
         for (; i < my_tiles; ++i) {
@@ -233,7 +235,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
           const int kb = int(i % kKeyStages);
           if (!mbar_wait(bar(kBarKFull + kb), uint32_t((i / kKeyStages) & 1), abort_flag, status)) return false;
           // the slot's y / residual columns are free once the JL MMA of tile i - 2 completed
-          if (i >= 2 && !mbar_wait(bar(kBarD2Full + sl), uint32_t(((i >> 1) - 1) & 1), abort_flag, status))
+          // (without the sign sketch: once the epilogue of tile i - 2 has read y)
+          if (i >= 2 &&
+              !mbar_wait(bar((JL ? kBarD2Full : kBarRFull) + sl), uint32_t(((i >> 1) - 1) & 1), abort_flag, status))
             return false;
           tc_fence_after();
           const uint32_t d1 = tmem + 256u * sl;
@@ -284,8 +288,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
             if (!issue_mma1(i + 1)) break;
             ++n1;
           }
-          if (!issue_mma2(i)) break;
-          ++n2;
+          if constexpr (JL) {
+            if (!issue_mma2(i)) break;
+            ++n2;
+          }
         }
         // before TMEM is released: the commit of the last group of each kind
         // tracks every MMA issued before it
@@ -302,7 +308,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
     const int row = (warp & 3) * 32 + lane;          // TMEM lane = key row within the tile
     const uint32_t lane_addr = uint32_t((warp & 3) * 32) << 16;
     const uint32_t d1 = tmem + 256u * slot + lane_addr, d2 = d1 + 128u;
-    constexpr int kRowBytes = kD * BMSE / 8 + kD / 8;  // = 16 (BMSE + 1)
+    constexpr int kW = BMSE + (JL ? 1 : 0);          // words per quarter chunk
+    constexpr int kRowBytes = 16 * kW;               // kD BMSE / 8 (+ kD / 8 sign bytes)
     const int q0 = 2 * half;
     float* rrbuf = prr + slot * 256;
     int64_t k = 0;
@@ -387,8 +394,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
           }
           // the residual overwrites the columns of y just read (A operand of the JL product):
           // coordinates 32q + 16hh .. +15 -> hi pairs at column 32q + 8hh, lo pairs 16 further
-          tmem_st8(d1 + 32u * q + 8u * hh, rh);
-          tmem_st8(d1 + 32u * q + 16u + 8u * hh, rl);
+          if constexpr (JL) {
+            tmem_st8(d1 + 32u * q + 8u * hh, rh);
+            tmem_st8(d1 + 32u * q + 16u + 8u * hh, rl);
+          }
         }
         if constexpr (BMSE == 3) {
 #pragma unroll
@@ -399,18 +408,19 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
 #pragma unroll
         for (int w = 0; w < BMSE; ++w) cw[qq][w] = zero ? 0u : ~__byte_perm(hw[2 * w], hw[2 * w + 1], 0x5410);
       }
-      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      if constexpr (JL) asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       tc_fence_before();
-      mbar_arrive(bar(kBarRFull + slot));
+      mbar_arrive(bar(kBarRFull + slot));   // residual in TMEM (without the sketch: y read)
       rrbuf[half * 128 + row] = rr2.x + rr2.y;
       mbar_arrive(bar(kBarRR + slot));
+      uint32_t sw[2] = {0u, 0u};
+      if constexpr (JL) {
       if (!mbar_wait_warp(bar(kBarD2Full + slot), par, abort_flag, status)) break;
       tc_fence_after();
       // bit = [z >= 0] = not the sign bit (z = -0 cannot arise for a nonzero
       // residual; zero keys get all ones).  Bit p of quarter q's word holds
       // coordinate 32q + 16 (p >> 4) + 4 (p & 3) + ((p >> 2) & 3); the bits are
       // shifted in from the top, p = 31 first.
-      uint32_t sw[2];
 #pragma unroll
       for (int qq = 0; qq < 2; ++qq) {
         uint32_t neg = 0;
@@ -429,24 +439,25 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
       }
       tc_fence_before();
       mbar_arrive(bar(kBarD2Free + slot));
+      }
       const int64_t key = (blockIdx.x + i * gridDim.x) * kTile + row;
       if (key < n) {
         // this half's two quarter chunks
-        uint32_t wv[2 * (BMSE + 1)];
+        uint32_t wv[2 * kW];
 #pragma unroll
         for (int qq = 0; qq < 2; ++qq) {
 #pragma unroll
-          for (int w = 0; w < BMSE; ++w) wv[qq * (BMSE + 1) + w] = cw[qq][w];
-          wv[qq * (BMSE + 1) + BMSE] = sw[qq];
+          for (int w = 0; w < BMSE; ++w) wv[qq * kW + w] = cw[qq][w];
+          if constexpr (JL) wv[qq * kW + BMSE] = sw[qq];
         }
-        uint8_t* dst = payload + key * kRowBytes + q0 * 4 * (BMSE + 1);
-        if constexpr (BMSE == 2) {
+        uint8_t* dst = payload + key * kRowBytes + q0 * 4 * kW;
+        if constexpr (kW % 2 == 0) {   // 16-byte aligned half rows
 #pragma unroll
-          for (int w = 0; w < 6; ++w) reinterpret_cast<uint32_t*>(dst)[w] = wv[w];
-        } else {
-#pragma unroll
-          for (int v = 0; v < (BMSE + 1) / 2; ++v)
+          for (int v = 0; v < kW / 2; ++v)
             reinterpret_cast<uint4*>(dst)[v] = make_uint4(wv[4 * v], wv[4 * v + 1], wv[4 * v + 2], wv[4 * v + 3]);
+        } else {                       // 8-byte aligned
+#pragma unroll
+          for (int v = 0; v < kW; ++v) reinterpret_cast<uint2*>(dst)[v] = make_uint2(wv[2 * v], wv[2 * v + 1]);
         }
       }
       if (half == 0) {
@@ -820,7 +831,7 @@ HalfBook make_halfbook(const tq_ctx* ctx) {
 }  // namespace
 
 bool quantize_tc_supported(const tq_ctx* ctx, int dtype, int64_t ld, const void* keys) {
-  return ctx->d == kD && ctx->m == kD && dtype == TQ_BF16 && ctx->bmse >= 1 && ctx->bmse <= 3 &&
+  return ctx->d == kD && (ctx->m == kD || ctx->m == 0) && dtype == TQ_BF16 && ctx->bmse >= 1 && ctx->bmse <= 3 &&
          ctx->dBimg != nullptr && ld % 8 == 0 && (reinterpret_cast<uintptr_t>(keys) & 15) == 0 &&
          device_is_sm100() && get_encode() != nullptr;
 }
@@ -843,25 +854,18 @@ cudaError_t launch_quantize_tc(const tq_ctx* ctx, const void* keys, int dtype, i
   const int64_t tiles = (n + kTile - 1) / kTile;
   const int grid = int(tiles < sms ? tiles : sms);
   const HalfBook hb = make_halfbook(ctx);
-  switch (ctx->bmse) {
-    case 1: {
-      auto k = quantize_tc_kernel<1>;
-      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
-      k<<<grid, kThreadsTc, kSmemBytes, st>>>(map, n, ctx->dBimg, hb, payload, norms, ctx->dstatus);
-      break;
-    }
-    case 2: {
-      auto k = quantize_tc_kernel<2>;
-      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
-      k<<<grid, kThreadsTc, kSmemBytes, st>>>(map, n, ctx->dBimg, hb, payload, norms, ctx->dstatus);
-      break;
-    }
-    default: {
-      auto k = quantize_tc_kernel<3>;
-      cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
-      k<<<grid, kThreadsTc, kSmemBytes, st>>>(map, n, ctx->dBimg, hb, payload, norms, ctx->dstatus);
-      break;
-    }
+  auto run = [&](auto kern) {
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
+    kern<<<grid, kThreadsTc, kSmemBytes, st>>>(map, n, ctx->dBimg, hb, payload, norms, ctx->dstatus);
+  };
+  const bool jl = ctx->m > 0;
+  switch (ctx->bmse * 2 + (jl ? 1 : 0)) {
+    case 2: run(quantize_tc_kernel<1, false>); break;
+    case 3: run(quantize_tc_kernel<1, true>); break;
+    case 4: run(quantize_tc_kernel<2, false>); break;
+    case 5: run(quantize_tc_kernel<2, true>); break;
+    case 6: run(quantize_tc_kernel<3, false>); break;
+    default: run(quantize_tc_kernel<3, true>); break;
   }
   return cudaGetLastError();
 }

@@ -341,7 +341,7 @@ tq_status tq_init_ex(int d, int bits, int m, uint64_t seed, uint32_t stream_base
   if (e == cudaSuccess) e = upload(ctx->R, &ctx->dR64);
   if (e == cudaSuccess) e = upload(ctx->P, &ctx->dP64);
   if (e == cudaSuccess) e = upload(ctx->c, &ctx->dc64);
-  if (e == cudaSuccess && d == 128 && m == 128) {
+  if (e == cudaSuccess && d == 128 && (m == 128 || m == 0)) {
     // R split into bf16 hi + lo (keys are bf16, so K R^T needs two MMAs); the
     // stored JL samples P are exact in fp16 (the residual is split into fp16
     // hi + lo in the kernel).  B operand rows are output coordinates, K the
@@ -357,7 +357,7 @@ tq_status tq_init_ex(int d, int bits, int m, uint64_t seed, uint32_t stream_base
     std::vector<uint8_t> img(size_t(3) * 128 * 128 * 2);
     write_swizzled(rh, 128, 128, img.data());
     write_swizzled(rl, 128, 128, img.data() + 32768);
-    write_swizzled(ph, 128, 128, img.data() + 65536);
+    if (m == 128) write_swizzled(ph, 128, 128, img.data() + 65536);   // m = 0: no JL operand
     e = upload(img, &ctx->dBimg);
   }
   if (e == cudaSuccess) e = cudaMalloc(&ctx->dstatus, sizeof(uint32_t));

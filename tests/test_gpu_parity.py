@@ -37,10 +37,13 @@ def test_device_tables_match_oracle(lib):
     assert np.max(np.abs(c - tb.c)) < 1e-12 and np.max(np.abs(t - tb.t)) < 1e-12
 
 
+@pytest.mark.parametrize("m", [128, 0])
 @pytest.mark.parametrize("bits", [2, 3, 4])
 @pytest.mark.parametrize("n", [1, 127, 441, 4133])
-def test_quantize_bf16_tensor_core_path(lib, bits, n):
-    ctx = _ctx(lib, bits=bits, seed=7 + bits)
+def test_quantize_bf16_tensor_core_path(lib, bits, n, m):
+    """d = 128 bf16 keys on the tensor-core quantizer, with the sign sketch
+    (m = 128) and without it (m = 0, the MSE-only variant)."""
+    ctx = _ctx(lib, bits=bits, seed=7 + bits, m=m)
     scales = W.head_channel_scales(1, 128, seed=3)
     k32 = W.decode_keys_pair(0, 0, n, 128, scales, seed=3 + n)
     kb = torch.from_numpy(k32).to(torch.bfloat16)
@@ -122,11 +125,14 @@ def _cache(lib, ctx, B, Hkv, S, seed):
     return lib.tq_quantize(ctx, kb)
 
 
+@pytest.mark.parametrize("m", [128, 0])
 @pytest.mark.parametrize("bits,B,Hkv,G,S", [(3, 2, 2, 4, 1037), (4, 1, 3, 4, 515), (4, 2, 2, 1, 200),
                                             (3, 1, 2, 2, 333), (2, 2, 1, 8, 129), (4, 1, 1, 12, 100),
                                             (4, 1, 2, 3, 16)])
-def test_logits_against_oracle(lib, bits, B, Hkv, G, S):
-    ctx = _ctx(lib, bits=bits, seed=21)
+def test_logits_against_oracle(lib, bits, B, Hkv, G, S, m):
+    """With the sign term (m = 128) and without it (m = 0, MSE-only); G <= 8
+    runs on the int8 MMA kernel, G = 12 on CUDA cores."""
+    ctx = _ctx(lib, bits=bits, seed=21, m=m)
     payload, norms = _cache(lib, ctx, B, Hkv, S, seed=31)
     Hq = Hkv * G
     q = W.queries((B, Hq, 128), seed=41)
