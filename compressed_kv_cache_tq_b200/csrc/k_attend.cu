@@ -16,9 +16,10 @@
 // computes, for every query head of the group, the chunk's maximum logit, the
 // sum of its weights and its a, b (flash-decoding style partials).  Key tiles
 // of 64 rows are staged in shared memory (prefetched into registers one tile
-// ahead); warp w takes keys w, w + 8, ...; lane L decodes one "slot" of the
-// packed layout per key (4 coordinates: register r = 4u + i of quarter q,
-// nibbles e = 0..3) and accumulates G heads with packed two-wide FMAs.
+// ahead); warp w takes the key pairs (k, k + 64) for k = w, w + 8, ...; lane
+// L decodes one "slot" of the packed layout of both keys (4 coordinates:
+// register r = 4u + i of quarter q, nibbles e = 0..3) and accumulates each
+// head with packed two-wide FMAs over the key pair.
 // Kernel 2 (attend_combine_kernel): one block per query head merges the
 // partials and applies P^T and R^T.
 #include <math.h>
@@ -55,7 +56,7 @@ __device__ __forceinline__ uint32_t slot_word(const uint32_t (&h)[BM], int i) {
 
 // Partials: part[((grp * nsplit + split) * G + h) * (2 + dp + mp)] = {max, sum, a[dp], b[mp]}.
 template <int BM, int GP, int NS>
-__global__ void __launch_bounds__(kAttThreads, GP * NS <= 4 ? 3 : 1) attend_partial_kernel(
+__global__ void __launch_bounds__(kAttThreads, GP * NS <= 2 ? 3 : (GP * NS <= 4 ? 2 : 1)) attend_partial_kernel(
     const float* __restrict__ logits, int Hq, int Hkv, int64_t S, int64_t chunk, int nsplit,
     const uint8_t* __restrict__ payload, const uint16_t* __restrict__ norms, RowGeom g, CodebookParams cb,
     float* __restrict__ part) {
@@ -133,15 +134,16 @@ __global__ void __launch_bounds__(kAttThreads, GP * NS <= 4 ? 3 : 1) attend_part
     s_off[ns] = qs * g.per_q + BM * g.uq + us;
     s_k[ns] = qs * (g.mp / 4) + 4 * (4 * us + s_i[ns]);
   }
-  float2 accC[NS][GP / 2][4], accS[NS][GP / 2][4];
+  // per head and coordinate, two partial sums: keys k (x) and k + kAttTile / 2 (y) of each tile
+  float2 accC[NS][GP][4], accS[NS][GP][4];
 #pragma unroll
   for (int ns = 0; ns < NS; ++ns)
 #pragma unroll
-    for (int hp = 0; hp < GP / 2; ++hp)
+    for (int h = 0; h < GP; ++h)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        accC[ns][hp][e] = make_float2(0.f, 0.f);
-        accS[ns][hp][e] = make_float2(0.f, 0.f);
+        accC[ns][h][e] = make_float2(0.f, 0.f);
+        accS[ns][h][e] = make_float2(0.f, 0.f);
       }
   // weights: thread (key k = tid % kAttTile, head tid / kAttTile + 2 it) of each tile
   constexpr int kWIt = (kAttTile * GP + kAttThreads - 1) / kAttThreads;
@@ -196,45 +198,53 @@ __global__ void __launch_bounds__(kAttThreads, GP * NS <= 4 ? 3 : 1) attend_part
           wr = w * f.y;
           lsum[it] += w;
         }
-        swn[k * GP + h] = wn;
-        swr[k * GP + h] = wr;
+        // key pairs (kp, kp + kAttTile / 2) side by side: [kp][h][2]
+        const int kp = k % (kAttTile / 2), half = k / (kAttTile / 2);
+        swn[(kp * GP + h) * 2 + half] = wn;
+        swr[(kp * GP + h) * 2 + half] = wr;
       }
     }
     __syncthreads();
     if (s0 + kAttTile < s_end) fetch(s0 + kAttTile);   // next tile in flight during the math
-    for (int k = warp; k < nk; k += kAttWarps) {
-      const uint16_t* hw = reinterpret_cast<const uint16_t*>(srows + k * rb);
-      float2 wn2[GP / 2], wr2[GP / 2];
+    const int npair = nk < kAttTile / 2 ? nk : kAttTile / 2;   // rows past nk are zero with zero weight
+    for (int kp = warp; kp < npair; kp += kAttWarps) {
+      const uint16_t* hwA = reinterpret_cast<const uint16_t*>(srows + kp * rb);
+      const uint16_t* hwB = reinterpret_cast<const uint16_t*>(srows + (kp + kAttTile / 2) * rb);
+      float2 wn2[GP], wr2[GP];
 #pragma unroll
-      for (int hp = 0; hp < GP / 2; ++hp) {
-        wn2[hp] = *reinterpret_cast<const float2*>(swn + k * GP + 2 * hp);
-        wr2[hp] = *reinterpret_cast<const float2*>(swr + k * GP + 2 * hp);
+      for (int h = 0; h < GP; ++h) {
+        wn2[h] = *reinterpret_cast<const float2*>(swn + (kp * GP + h) * 2);
+        wr2[h] = *reinterpret_cast<const float2*>(swr + (kp * GP + h) * 2);
       }
 #pragma unroll
       for (int ns = 0; ns < NS; ++ns) {
         const int t = lane + 32 * ns;
         if (t < nslot_c) {
-          uint32_t h[BM];
+          uint32_t ha[BM], hb[BM];
 #pragma unroll
-          for (int x = 0; x < BM; ++x) h[x] = hw[c_off[ns] + x];
-          const uint32_t v = slot_word<BM>(h, c_i[ns]);
+          for (int x = 0; x < BM; ++x) {
+            ha[x] = hwA[c_off[ns] + x];
+            hb[x] = hwB[c_off[ns] + x];
+          }
+          const uint32_t va = slot_word<BM>(ha, c_i[ns]), vb = slot_word<BM>(hb, c_i[ns]);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float2 cv = f2(sc[(v >> (4 * e)) & 7u]);
+            const float2 cv = make_float2(sc[(va >> (4 * e)) & 7u], sc[(vb >> (4 * e)) & 7u]);
 #pragma unroll
-            for (int hp = 0; hp < GP / 2; ++hp) accC[ns][hp][e] = __ffma2_rn(cv, wn2[hp], accC[ns][hp][e]);
+            for (int h = 0; h < GP; ++h) accC[ns][h][e] = __ffma2_rn(cv, wn2[h], accC[ns][h][e]);
           }
         }
         if (t < nslot_s) {
           // sign bit 4e + i of the halfword moved to bit 31 and inverted: +1.0f for a set bit, -1.0f otherwise
-          const uint32_t hs = hw[s_off[ns]];
+          const uint32_t sa = hwA[s_off[ns]], sb = hwB[s_off[ns]];
           const int sh0 = 31 - s_i[ns];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const uint32_t x = hs << (sh0 - 4 * e);
-            const float2 sg = f2(__uint_as_float((~x & 0x80000000u) | 0x3f800000u));
+            const uint32_t xa = sa << (sh0 - 4 * e), xb = sb << (sh0 - 4 * e);
+            const float2 sg = make_float2(__uint_as_float((~xa & 0x80000000u) | 0x3f800000u),
+                                          __uint_as_float((~xb & 0x80000000u) | 0x3f800000u));
 #pragma unroll
-            for (int hp = 0; hp < GP / 2; ++hp) accS[ns][hp][e] = __ffma2_rn(sg, wr2[hp], accS[ns][hp][e]);
+            for (int h = 0; h < GP; ++h) accS[ns][h][e] = __ffma2_rn(sg, wr2[h], accS[ns][h][e]);
           }
         }
       }
@@ -247,17 +257,12 @@ __global__ void __launch_bounds__(kAttThreads, GP * NS <= 4 ? 3 : 1) attend_part
   for (int ns = 0; ns < NS; ++ns) {
     const int t = lane + 32 * ns;
 #pragma unroll
-    for (int hp = 0; hp < GP / 2; ++hp)
+    for (int h = 0; h < GP; ++h)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        if (t < nslot_c) {
-          atomicAdd(sacc + (2 * hp) * (g.dp + g.mp) + c_j[ns] + e, accC[ns][hp][e].x);
-          atomicAdd(sacc + (2 * hp + 1) * (g.dp + g.mp) + c_j[ns] + e, accC[ns][hp][e].y);
-        }
-        if (t < nslot_s) {
-          atomicAdd(sacc + (2 * hp) * (g.dp + g.mp) + g.dp + s_k[ns] + e, accS[ns][hp][e].x);
-          atomicAdd(sacc + (2 * hp + 1) * (g.dp + g.mp) + g.dp + s_k[ns] + e, accS[ns][hp][e].y);
-        }
+        if (t < nslot_c) atomicAdd(sacc + h * (g.dp + g.mp) + c_j[ns] + e, accC[ns][h][e].x + accC[ns][h][e].y);
+        if (t < nslot_s)
+          atomicAdd(sacc + h * (g.dp + g.mp) + g.dp + s_k[ns] + e, accS[ns][h][e].x + accS[ns][h][e].y);
       }
   }
   // every lane of a warp holds the same head in lsum[it] (32 consecutive keys of one head)
@@ -296,16 +301,29 @@ __global__ void __launch_bounds__(256) attend_combine_kernel(const float* __rest
   const int grp = b * Hkv + hkv;
   const int rec = 2 + g.dp + g.mp;
   const float* p0 = part + (size_t(grp) * nsplit * G + hl) * rec;   // split i at p0 + i G rec
+  // M = max_i m_i and L = sum_i exp(m_i - M) l_i over the splits, in parallel
+  __shared__ float sr[8];
+  float mloc = -INFINITY;
+  for (int i = threadIdx.x; i < nsplit; i += blockDim.x) mloc = fmaxf(mloc, p0[size_t(i) * G * rec]);
+  for (int o = 16; o; o >>= 1) mloc = fmaxf(mloc, __shfl_xor_sync(0xffffffffu, mloc, o));
+  if ((threadIdx.x & 31) == 0) sr[threadIdx.x >> 5] = mloc;
+  __syncthreads();
+  float M = sr[0];
+  for (int w = 1; w < int(blockDim.x >> 5); ++w) M = fmaxf(M, sr[w]);
+  __syncthreads();
+  float lloc = 0.f;
+  for (int i = threadIdx.x; i < nsplit; i += blockDim.x) {
+    const float mi = p0[size_t(i) * G * rec];
+    const float f = (M == -INFINITY || mi == -INFINITY) ? 0.f : expf(mi - M);
+    sf[i] = f;
+    lloc = fmaf(f, p0[size_t(i) * G * rec + 1], lloc);
+  }
+  for (int o = 16; o; o >>= 1) lloc += __shfl_xor_sync(0xffffffffu, lloc, o);
+  if ((threadIdx.x & 31) == 0) sr[threadIdx.x >> 5] = lloc;
+  __syncthreads();
   if (threadIdx.x == 0) {
-    float M = -INFINITY;
-    for (int i = 0; i < nsplit; ++i) M = fmaxf(M, p0[size_t(i) * G * rec]);
     float L = 0.f;
-    for (int i = 0; i < nsplit; ++i) {
-      const float mi = p0[size_t(i) * G * rec];
-      const float f = (M == -INFINITY || mi == -INFINITY) ? 0.f : expf(mi - M);
-      if (i < 1024) sf[i] = f;
-      L += f * p0[size_t(i) * G * rec + 1];
-    }
+    for (int w = 0; w < int(blockDim.x >> 5); ++w) L += sr[w];
     sL = L;
   }
   __syncthreads();
@@ -346,10 +364,10 @@ AttPlan att_plan(int B, int Hkv, int64_t S) {
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   // key chunks per (batch, KV head): the number of waves of resident blocks
-  // (three per SM) times the chunk length is the time; take the split count
+  // (two per SM) times the chunk length is the time; take the split count
   // that minimises it, with a small cost per split for the merge
   const int64_t groups = int64_t(B) * Hkv;
-  const int64_t cap = int64_t(sms) * 3;
+  const int64_t cap = int64_t(sms) * 2;
   int64_t max_ns = (S + kAttTile - 1) / kAttTile;
   if (max_ns > 1024) max_ns = 1024;
   if (max_ns < 1) max_ns = 1;
