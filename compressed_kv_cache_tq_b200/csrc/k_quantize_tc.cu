@@ -488,10 +488,12 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
 // is the head's M_h (M_h k = (R_hi k_hi, R_lo k_lo): both groups' rotations
 // of the gathered key in one product, the gather folded into the columns of
 // M_h), and the JL operand is diag(P_hi, P_lo).  Rotated coordinates 0..63
-// belong to the high group and 64..127 to the low group, which are exactly
-// the TMEM columns of epilogue halves 0 and 1: each half finishes its own
-// group (norm, cells, residual norm, packing) with no exchange between the
-// halves.  Each CTA serves one KV head, so it loads the head's operand once.
+// belong to the high group and 64..127 to the low group.  Each epilogue
+// thread takes one quarter of each group (so both halves run the same code,
+// which keeps the instruction footprint of one epilogue), and the halves
+// combine their partial group norms and residual norms through shared memory
+// as the single-context kernel does.  Each CTA serves one KV head, so it loads
+// the head's operand once.
 // ---------------------------------------------------------------------------
 
 struct SplitGeom {
@@ -500,153 +502,208 @@ struct SplitGeom {
   int Hkv, head, cph, sub;   // KV heads, this CTA's head, CTAs per head, index among them
 };
 
+// Shared memory of the split kernel: the single-context layout up to the key
+// ring, then per-group partial sums exchanged between the epilogue halves.
+constexpr uint32_t kOffSPn2 = kOffPn2;                                    // [slot][parity][half][group][row] ||y_g||^2
+constexpr uint32_t kOffSPrr = kOffSPn2 + 2u * 2u * 2u * 2u * 128u * 4u;   // [slot][half][group][row] ||r_g||^2
+constexpr uint32_t kOffSBar = kOffSPrr + 2u * 2u * 2u * 128u * 4u;
+constexpr uint32_t kSmemSplit = kOffSBar + 256 + 1024;
+static_assert(kSmemSplit <= 232448, "shared memory per block");
+
+// One 32-coordinate quarter q of a group (b' = BM): cells, residual to TMEM
+// (fp16 hi / lo pairs over the columns of y), and the code halfwords of the
+// group's chunks 2 (q & 1) and 2 (q & 1) + 1.  Returns the quarter's part of
+// ||r_rot||^2 (scaled by 128^2).
 template <int BM>
-__device__ __forceinline__ void split_epilogue(uint32_t bar0, uint32_t d1, uint32_t d2, int slot, int q0, int row,
-                                               int64_t my_tiles, const SplitGeom& sg, const HalfBook& book,
-                                               uint8_t* __restrict__ payload, uint16_t* __restrict__ norms,
+__device__ __forceinline__ float split_quarter(uint32_t d1, int q, float s128, bool zero, const HalfBook& hb,
+                                               uint32_t (&chw)[2][BM]) {
+  float y[32];
+  tmem_ld32(d1 + 32u * q, y);
+  tmem_wait32(y);
+  float2 rr2 = make_float2(0.f, 0.f);
+  uint32_t hw[2 * BM], hw3[2] = {0u, 0u};
+#pragma unroll
+  for (int h = 0; h < 2 * BM; ++h) hw[h] = 0;
+#pragma unroll
+  for (int hh = 0; hh < 2; ++hh) {
+    uint32_t rh[8], rl[8];
+#pragma unroll
+    for (int jp = 0; jp < 16; jp += 2) {
+      const int j0 = 16 * hh + jp;
+      float2 rp;
+      const uint2 bb = cell2<BM>(make_float2(y[j0], y[j0 + 1]), s128, hb, rp);
+      rr2 = __ffma2_rn(rp, rp, rr2);
+      const __half2 hi = __float22half2_rn(rp);
+      const float2 hf = __half22float2(hi);
+      const __half2 lo = __float22half2_rn(__ffma2_rn(hf, f2(-1.f), rp));
+      rh[jp >> 1] = *reinterpret_cast<const uint32_t*>(&hi);
+      rl[jp >> 1] = *reinterpret_cast<const uint32_t*>(&lo);
+#pragma unroll
+      for (int t2 = 0; t2 < 2; ++t2) {
+        // quarter coordinate jc: chunk unit uu, register ii, nibble e
+        const int jc = j0 + t2;
+        const uint32_t bits = t2 ? bb.y : bb.x;
+        const int rreg = jc >> 2, e = jc & 3, uu = rreg >> 2, ii = rreg & 3;
+        if constexpr (BM == 3) {
+          if (ii < 3)
+            hw[uu * 3 + ii] += bits << (4 * e);
+          else
+            hw3[uu] += bits << (4 * e);
+        } else if constexpr (BM == 2) {
+          hw[uu * 2 + (ii >> 1)] += bits << (4 * e + 2 * (ii & 1));
+        } else {
+          hw[uu] += bits << (4 * e + ii);
+        }
+      }
+    }
+    tmem_st8(d1 + 32u * q + 8u * hh, rh);
+    tmem_st8(d1 + 32u * q + 16u + 8u * hh, rl);
+  }
+  if constexpr (BM == 3) {
+#pragma unroll
+    for (int uu = 0; uu < 2; ++uu)
+#pragma unroll
+      for (int b = 0; b < 3; ++b) hw[uu * 3 + b] |= ((hw3[uu] >> b) & 0x1111u) << 3;
+  }
+  // the low halfword of each sum holds the complemented codes
+#pragma unroll
+  for (int uu = 0; uu < 2; ++uu)
+#pragma unroll
+    for (int w = 0; w < BM; ++w) chw[uu][w] = zero ? 0u : (~hw[uu * BM + w]) & 0xFFFFu;
+  return rr2.x + rr2.y;
+}
+
+// Sign word of z quarter q: bit p = sign coordinate 32 (q & 1) + 16 (p >> 4)
+// + 4 (p & 3) + ((p >> 2) & 3) of the group, i.e. the sign halfwords of the
+// group's chunks 2 (q & 1) (low half) and 2 (q & 1) + 1 (high half).
+__device__ __forceinline__ uint32_t split_signs(uint32_t d2, int q, bool zero) {
+  uint32_t neg = 0;
+#pragma unroll
+  for (int hz = 1; hz >= 0; --hz) {
+    float z[16];
+    tmem_ld16(d2 + 32u * q + 16u * hz, z);
+    tmem_wait16(z);
+#pragma unroll
+    for (int p = 15; p >= 0; --p) {
+      const int jj = 4 * (p & 3) + ((p >> 2) & 3);
+      neg = __funnelshift_l(__float_as_uint(z[jj]), neg, 1);
+    }
+  }
+  return zero ? 0xFFFFFFFFu : ~neg;
+}
+
+// This half's part of a group row: chunks 2 half and 2 half + 1, each BM code
+// halfwords then the sign halfword; BM + 1 words at byte 4 half (BM + 1).
+template <int BM>
+__device__ __forceinline__ void split_store(uint8_t* row, int half, const uint32_t (&chw)[2][BM], uint32_t sw) {
+  uint32_t hv[2 * (BM + 1)];
+#pragma unroll
+  for (int uu = 0; uu < 2; ++uu) {
+#pragma unroll
+    for (int w = 0; w < BM; ++w) hv[uu * (BM + 1) + w] = chw[uu][w];
+    hv[uu * (BM + 1) + BM] = (sw >> (16 * uu)) & 0xFFFFu;
+  }
+  uint32_t wv[BM + 1];
+#pragma unroll
+  for (int x = 0; x < BM + 1; ++x) wv[x] = hv[2 * x] | (hv[2 * x + 1] << 16);
+  uint8_t* dst = row + 4 * half * (BM + 1);
+  if constexpr (BM == 3) {
+    *reinterpret_cast<uint4*>(dst) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+  } else if constexpr (BM == 1) {
+    *reinterpret_cast<uint2*>(dst) = make_uint2(wv[0], wv[1]);
+  } else {
+#pragma unroll
+    for (int x = 0; x < BM + 1; ++x) reinterpret_cast<uint32_t*>(dst)[x] = wv[x];
+  }
+}
+
+// Epilogue of the split kernel: every thread takes quarter `half` of the high
+// group (TMEM columns 32 half ..) and quarter `half` of the low group (64 +
+// 32 half ..), so both halves run the same code; the group norms and residual
+// norms combine the two halves' partial sums through shared memory, as in the
+// single-context kernel.
+template <int BHI, int BLO>
+__device__ __forceinline__ void split_epilogue(uint32_t bar0, uint32_t d1, uint32_t d2, int slot, int half, int row,
+                                               int64_t my_tiles, const SplitGeom& sg, const HalfBook& book_hi,
+                                               const HalfBook& book_lo, uint8_t* __restrict__ payload_hi,
+                                               uint16_t* __restrict__ norms_hi, uint8_t* __restrict__ payload_lo,
+                                               uint16_t* __restrict__ norms_lo, float* pn2, float* prr,
                                                volatile int* abort_flag, uint32_t* status) {
   auto bar = [&](int i) { return bar0 + 8u * uint32_t(i); };
+  float* rrbuf = prr + slot * 512;
+  const int qh = half, ql = 2 + half;   // this thread's quarter of each group
   int64_t k = 0;
   for (int64_t i = slot; i < my_tiles; i += 2, ++k) {
     const uint32_t par = uint32_t(k & 1);
     if (!mbar_wait_warp(bar(kBarD1Full + slot), par, abort_flag, status)) break;
     tc_fence_after();
-    // ||k_group||^2 = ||R_group k_group||^2 from this half's 64 rotated coordinates
-    float2 acc = make_float2(0.f, 0.f);
+    // partial ||y_g||^2 of both groups; double-buffered by tile parity, so a
+    // half that runs ahead never overwrites sums the other half still reads
+    float* n2buf = pn2 + (slot * 2 + int(par)) * 512;
 #pragma unroll
-    for (int qq = 0; qq < 2; ++qq) {
+    for (int g = 0; g < 2; ++g) {
       float y[32];
-      tmem_ld32(d1 + 32u * (q0 + qq), y);
+      tmem_ld32(d1 + 32u * (g ? ql : qh), y);
       tmem_wait32(y);
+      float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
       for (int j = 0; j < 32; j += 2)
         acc = __ffma2_rn(make_float2(y[j], y[j + 1]), make_float2(y[j], y[j + 1]), acc);
+      n2buf[(half * 2 + g) * 128 + row] = acc.x + acc.y;
     }
-    const float n2 = acc.x + acc.y;
-    const float nk = sqrtf(n2);
-    const bool zero = !(n2 > 0.f);
-    const float s128 = zero ? 0.f : 128.f / nk;
-    HalfBook hb = book;
-    if (zero) {
-      hb.C0 = 0.f;
+    mbar_arrive(bar(kBarN2 + slot));
+    if (!mbar_wait_warp(bar(kBarN2 + slot), par, abort_flag, status)) break;
+    float nk[2], s128[2];
+    bool zero[2];
+    HalfBook hb[2] = {book_hi, book_lo};
 #pragma unroll
-      for (int c = 0; c < 3; ++c) hb.dC[c] = 0.f;
-      hb.dA = 0.f;
-      hb.C20 = 0.f;
-    }
-    float2 rr2 = make_float2(0.f, 0.f);
-    uint32_t chw[4][BM];   // code halfwords of the group's four chunks
+    for (int g = 0; g < 2; ++g) {
+      const float n2 = n2buf[g * 128 + row] + n2buf[(2 + g) * 128 + row];
+      nk[g] = sqrtf(n2);
+      zero[g] = !(n2 > 0.f);
+      s128[g] = zero[g] ? 0.f : 128.f / nk[g];
+      if (zero[g]) {
+        hb[g].C0 = 0.f;
 #pragma unroll
-    for (int qq = 0; qq < 2; ++qq) {
-      const int q = q0 + qq;
-      float y[32];
-      tmem_ld32(d1 + 32u * q, y);
-      tmem_wait32(y);
-      uint32_t hw[2 * BM], hw3[2] = {0u, 0u};
-#pragma unroll
-      for (int h = 0; h < 2 * BM; ++h) hw[h] = 0;
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t rh[8], rl[8];
-#pragma unroll
-        for (int jp = 0; jp < 16; jp += 2) {
-          const int j0 = 16 * hh + jp;
-          float2 rp;
-          const uint2 bb = cell2<BM>(make_float2(y[j0], y[j0 + 1]), s128, hb, rp);
-          rr2 = __ffma2_rn(rp, rp, rr2);
-          const __half2 hi = __float22half2_rn(rp);
-          const float2 hf = __half22float2(hi);
-          const __half2 lo = __float22half2_rn(__ffma2_rn(hf, f2(-1.f), rp));
-          rh[jp >> 1] = *reinterpret_cast<const uint32_t*>(&hi);
-          rl[jp >> 1] = *reinterpret_cast<const uint32_t*>(&lo);
-#pragma unroll
-          for (int t2 = 0; t2 < 2; ++t2) {
-            // coordinate 32 qq + jc of the group: chunk 2 qq + uu, register ii, nibble e
-            const int jc = j0 + t2;
-            const uint32_t bits = t2 ? bb.y : bb.x;
-            const int rreg = jc >> 2, e = jc & 3, uu = rreg >> 2, ii = rreg & 3;
-            if constexpr (BM == 3) {
-              if (ii < 3)
-                hw[uu * 3 + ii] += bits << (4 * e);
-              else
-                hw3[uu] += bits << (4 * e);
-            } else if constexpr (BM == 2) {
-              hw[uu * 2 + (ii >> 1)] += bits << (4 * e + 2 * (ii & 1));
-            } else {
-              hw[uu] += bits << (4 * e + ii);
-            }
-          }
-        }
-        tmem_st8(d1 + 32u * q + 8u * hh, rh);
-        tmem_st8(d1 + 32u * q + 16u + 8u * hh, rl);
+        for (int c = 0; c < 3; ++c) hb[g].dC[c] = 0.f;
+        hb[g].dA = 0.f;
+        hb[g].C20 = 0.f;
       }
-      if constexpr (BM == 3) {
-#pragma unroll
-        for (int uu = 0; uu < 2; ++uu)
-#pragma unroll
-          for (int b = 0; b < 3; ++b) hw[uu * 3 + b] |= ((hw3[uu] >> b) & 0x1111u) << 3;
-      }
-      // the low halfword of each sum holds the complemented codes
-#pragma unroll
-      for (int uu = 0; uu < 2; ++uu)
-#pragma unroll
-        for (int w = 0; w < BM; ++w) chw[2 * qq + uu][w] = zero ? 0u : (~hw[uu * BM + w]) & 0xFFFFu;
     }
+    uint32_t chi[2][BHI], clo[2][BLO];
+    const float rr_hi = split_quarter<BHI>(d1, qh, s128[0], zero[0], hb[0], chi);
+    const float rr_lo = split_quarter<BLO>(d1, ql, s128[1], zero[1], hb[1], clo);
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
     tc_fence_before();
     mbar_arrive(bar(kBarRFull + slot));
+    rrbuf[(half * 2 + 0) * 128 + row] = rr_hi;
+    rrbuf[(half * 2 + 1) * 128 + row] = rr_lo;
+    mbar_arrive(bar(kBarRR + slot));
     if (!mbar_wait_warp(bar(kBarD2Full + slot), par, abort_flag, status)) break;
     tc_fence_after();
-    // sign words: bit p of quarter word qq holds group sign coordinate
-    // 32 qq + 16 (p >> 4) + 4 (p & 3) + ((p >> 2) & 3), i.e. the sign
-    // halfwords of chunks 2 qq (low half) and 2 qq + 1 (high half)
-    uint32_t sw[2];
-#pragma unroll
-    for (int qq = 0; qq < 2; ++qq) {
-      uint32_t neg = 0;
-#pragma unroll
-      for (int hz = 1; hz >= 0; --hz) {
-        float z[16];
-        tmem_ld16(d2 + 32u * (q0 + qq) + 16u * hz, z);
-        tmem_wait16(z);
-#pragma unroll
-        for (int p = 15; p >= 0; --p) {
-          const int jj = 4 * (p & 3) + ((p >> 2) & 3);
-          neg = __funnelshift_l(__float_as_uint(z[jj]), neg, 1);
-        }
-      }
-      sw[qq] = zero ? 0xFFFFFFFFu : ~neg;
-    }
+    const uint32_t sw_hi = split_signs(d2, qh, zero[0]);
+    const uint32_t sw_lo = split_signs(d2, ql, zero[1]);
     tc_fence_before();
     mbar_arrive(bar(kBarD2Free + slot));
     const int64_t t = sg.sub + i * sg.cph;
     const int64_t b = t / sg.tps, st = t - b * sg.tps;
     const int64_t s = st * kTile + row;
-    if (s < sg.S) {
-      const int64_t key = (b * sg.Hkv + sg.head) * sg.S + s;
-      // group row: chunks c = 0..3 of BM code halfwords and one sign halfword
-      uint32_t hv[4 * (BM + 1)];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-#pragma unroll
-        for (int w = 0; w < BM; ++w) hv[c * (BM + 1) + w] = chw[c][w];
-        hv[c * (BM + 1) + BM] = (sw[c >> 1] >> (16 * (c & 1))) & 0xFFFFu;
-      }
-      uint32_t wv[2 * (BM + 1)];
-#pragma unroll
-      for (int x = 0; x < 2 * (BM + 1); ++x) wv[x] = hv[2 * x] | (hv[2 * x + 1] << 16);
-      uint8_t* dst = payload + key * (8 * (BM + 1));
-      if constexpr (BM == 2) {
-#pragma unroll
-        for (int v = 0; v < 3; ++v) reinterpret_cast<uint2*>(dst)[v] = make_uint2(wv[2 * v], wv[2 * v + 1]);
-      } else {
-#pragma unroll
-        for (int v = 0; v < (BM + 1) / 2; ++v)
-          reinterpret_cast<uint4*>(dst)[v] = make_uint4(wv[4 * v], wv[4 * v + 1], wv[4 * v + 2], wv[4 * v + 3]);
-      }
-      const float rho = nk * sqrtf(rr2.x + rr2.y) * (1.0f / 128.f);
-      reinterpret_cast<uint32_t*>(norms)[key] = uint32_t(__half_as_ushort(__float2half_rn(nk))) |
-                                                (uint32_t(__half_as_ushort(__float2half_rn(rho))) << 16);
+    const bool valid = s < sg.S;
+    const int64_t key = (b * sg.Hkv + sg.head) * sg.S + s;
+    if (valid) {
+      split_store<BHI>(payload_hi + key * (8 * (BHI + 1)), half, chi, sw_hi);
+      split_store<BLO>(payload_lo + key * (8 * (BLO + 1)), half, clo, sw_lo);
+    }
+    // both halves' residual sums of this tile: half 0 writes the high group's
+    // norms, half 1 the low group's.  A half rewrites these sums only after its
+    // next N2 wait, which needs the other half's next arrival.
+    if (!mbar_wait_warp(bar(kBarRR + slot), par, abort_flag, status)) break;
+    const int g = half;
+    const float rho = nk[g] * sqrtf(rrbuf[g * 128 + row] + rrbuf[(2 + g) * 128 + row]) * (1.0f / 128.f);
+    if (valid) {
+      uint16_t* nr = g ? norms_lo : norms_hi;
+      reinterpret_cast<uint32_t*>(nr)[key] = uint32_t(__half_as_ushort(__float2half_rn(nk[g]))) |
+                                             (uint32_t(__half_as_ushort(__float2half_rn(rho))) << 16);
     }
   }
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");   // none in flight on an early exit
@@ -662,9 +719,11 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_split_tc_kernel(
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
   uint8_t* sbase = smem_raw + (base - raw);
-  const uint32_t bar0 = base + kOffBar;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sbase + kOffBar + 8 * kNumBars);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + kOffBar + 8 * kNumBars + 4);
+  const uint32_t bar0 = base + kOffSBar;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sbase + kOffSBar + 8 * kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + kOffSBar + 8 * kNumBars + 4);
+  float* pn2 = reinterpret_cast<float*>(sbase + kOffSPn2);
+  float* prr = reinterpret_cast<float*>(sbase + kOffSPrr);
   auto bar = [&](int i) { return bar0 + 8u * uint32_t(i); };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -686,7 +745,9 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_split_tc_kernel(
     }
     for (int sl = 0; sl < 2; ++sl) {
       mbar_init(bar(kBarD1Full + sl), 1);
+      mbar_init(bar(kBarN2 + sl), kTeamThreads);
       mbar_init(bar(kBarRFull + sl), kTeamThreads);
+      mbar_init(bar(kBarRR + sl), kTeamThreads);
       mbar_init(bar(kBarD2Full + sl), 1);
       mbar_init(bar(kBarD2Free + sl), kTeamThreads);
     }
@@ -793,18 +854,14 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_split_tc_kernel(
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    // warp w: TMEM slot ((w - 2) >> 2) & 1, half (w - 2) >> 3 = group (0 high, 1 low)
+    // warp w: TMEM slot ((w - 2) >> 2) & 1, half (w - 2) >> 3
     const int eg = (warp - 2) >> 2;
     const int slot = eg & 1, half = eg >> 1;
     const int row = (warp & 3) * 32 + lane;
     const uint32_t lane_addr = uint32_t((warp & 3) * 32) << 16;
     const uint32_t d1 = tmem + 256u * slot + lane_addr, d2 = d1 + 128u;
-    if (half == 0)
-      split_epilogue<BHI>(bar0, d1, d2, slot, 0, row, my_tiles, sg, book_hi, payload_hi, norms_hi, abort_flag,
-                          status);
-    else
-      split_epilogue<BLO>(bar0, d1, d2, slot, 2, row, my_tiles, sg, book_lo, payload_lo, norms_lo, abort_flag,
-                          status);
+    split_epilogue<BHI, BLO>(bar0, d1, d2, slot, half, row, my_tiles, sg, book_hi, book_lo, payload_hi, norms_hi,
+                             payload_lo, norms_lo, pn2, prr, abort_flag, status);
   }
   tc_fence_before();
   __syncthreads();
@@ -882,8 +939,8 @@ cudaError_t launch_split_kernel(dim3 grid, cudaStream_t st, const CUtensorMap& m
                                 int cph, const uint8_t* dimg, const HalfBook& bh, const HalfBook& bl,
                                 uint8_t* ph, uint16_t* nh, uint8_t* pl, uint16_t* nl, uint32_t* status) {
   auto k = quantize_split_tc_kernel<BHI, BLO>;
-  cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
-  k<<<grid, kThreadsTc, kSmemBytes, st>>>(map, B, Hkv, S, cph, dimg, bh, bl, ph, nh, pl, nl, status);
+  cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemSplit));
+  k<<<grid, kThreadsTc, kSmemSplit, st>>>(map, B, Hkv, S, cph, dimg, bh, bl, ph, nh, pl, nl, status);
   return cudaGetLastError();
 }
 
