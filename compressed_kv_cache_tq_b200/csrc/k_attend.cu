@@ -22,6 +22,7 @@
 // head with packed two-wide FMAs over the key pair.
 // Kernel 2 (attend_combine_kernel): one block per query head merges the
 // partials and applies P^T and R^T.
+#include <cuda_fp16.h>
 #include <math.h>
 
 #include "tq_device.cuh"
@@ -35,6 +36,7 @@ constexpr int kAttWarps = kAttThreads / 32;
 constexpr int kAttTile = 128;         // keys per staged tile
 constexpr int kAttMaxLd = 8;          // 8-byte words per thread per tile (rows of up to 128 bytes)
 constexpr int kAttMaxHeads = 8;
+constexpr int kAttMmaTile = 256;      // keys per staged tile of the tensor-core kernel
 
 __device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
 
@@ -285,6 +287,306 @@ __global__ void __launch_bounds__(kAttThreads, GP * NS <= 2 ? 3 : (GP * NS <= 4 
   }
 }
 
+// ---------------------------------------------------------------------------
+// Tensor-core partial sums (d = m = 128, up to 4 query heads per KV head).
+// The sums contract over keys: for a 16-key step, D[coordinate][column] +=
+// A[coordinate][key] B[key][column] with the fp16 m16n8k16 MMA, columns =
+// (head, hi / lo limb of the weight).  Thread (g, tig) of a warp builds the A
+// operand of unit g of the packed rows (16 coordinates: register i, nibble e)
+// for its four keys 2 tig, 2 tig + 1, 2 tig + 8, 2 tig + 9 of the step:
+// codes -> fp16 codebook values by byte permutes over the two byte planes of
+// the fp16 levels, then a byte transpose from (key, 4 coordinates) to
+// (coordinate, 2 keys); sign bits -> fp16 +-1 by one shift and one
+// logic op per register.  Row mapping: m-tile 2 i + (e >> 1), row g + 8 (e & 1).
+// B holds the weights w n16 (codes) and w rho16 (signs) of the same keys as
+// fp16 hi + lo limbs.  Precision: each product carries the fp16 rounding of
+// its codebook level (<= 2^-11 relative) and of the weight's hi + lo split
+// (<= 2^-22); sums are fp32.
+// ---------------------------------------------------------------------------
+
+// fp16 bits of the codebook levels as two byte planes (level v: lo byte v, hi byte v).
+struct HalfLut {
+  uint32_t lo[2], hi[2];
+};
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Byte-permute selector of register i (coordinates (i, e = 0..3) in its nibbles)
+// from the unit's code halfwords.
+template <int BM>
+__device__ __forceinline__ uint32_t reg_selector(const uint32_t (&h)[BM], int i) {
+  if constexpr (BM == 3) {
+    if (i < 3) return h[i] & 0x7777u;
+    return ((h[0] >> 3) & 0x1111u) | ((h[1] >> 2) & 0x2222u) | ((h[2] >> 1) & 0x4444u);
+  } else if constexpr (BM == 2) {
+    return (h[i >> 1] >> (2 * (i & 1))) & 0x3333u;
+  } else {
+    return (h[0] >> i) & 0x1111u;
+  }
+}
+
+// Two weights (keys a, b) of one column as an fp16 pair: the hi limb, or the
+// lo limb w - hi.
+// Branch-free (the lanes of a warp take different limbs, and the MMA that
+// consumes the pair needs the whole warp converged).
+__device__ __forceinline__ uint32_t weight_pair(float wa, float wb, bool lo_limb) {
+  const __half ha = __float2half_rn(wa), hb = __float2half_rn(wb);
+  const __half la = __float2half_rn(wa - __half2float(ha)), lb = __float2half_rn(wb - __half2float(hb));
+  const uint32_t hi2 = uint32_t(__half_as_ushort(ha)) | (uint32_t(__half_as_ushort(hb)) << 16);
+  const uint32_t lo2 = uint32_t(__half_as_ushort(la)) | (uint32_t(__half_as_ushort(lb)) << 16);
+  return lo_limb ? lo2 : hi2;
+}
+
+template <int BM, bool JL>
+__global__ void __launch_bounds__(kAttThreads, 2) attend_mma_kernel(
+    const float* __restrict__ logits, int Hq, int Hkv, int64_t S, int64_t chunk, int nsplit,
+    const uint8_t* __restrict__ payload, const uint16_t* __restrict__ norms, HalfLut lut,
+    float* __restrict__ part) {
+  constexpr int GP = 4;
+  constexpr int kPerQ = 2 * BM + (JL ? 2 : 0);   // halfwords per quarter chunk (d = m = 128)
+  constexpr int rb = 8 * kPerQ;                   // row bytes
+  constexpr int kAcc = 256;                       // a (128 coordinates) then b (128 sign coordinates)
+  constexpr int T = kAttMmaTile;
+  extern __shared__ __align__(16) uint8_t sm[];
+  uint8_t* srows0 = sm;                                                       // [2][T][rb] rows, double-buffered
+  float* swn = reinterpret_cast<float*>(sm + 2 * T * rb);                     // [T][GP]  w n16
+  float* swr = swn + T * GP;                                                  // [T][GP]  w rho16
+  float* sacc = swr + T * GP;                                                 // [GP][kAcc]
+  float* sred = sacc + GP * kAcc;                                             // [GP][kAttWarps] maxima
+  float* smx = sred + GP * kAttWarps;                                         // [GP] chunk maximum
+  float* sl = smx + GP;                                                       // [GP] sum of weights
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, tig = lane & 3;
+  const int G = Hq / Hkv;
+  const int grp = blockIdx.x / nsplit, split = blockIdx.x - grp * nsplit;
+  const int b = grp / Hkv, hkv = grp - b * Hkv;
+  const int64_t s_begin = int64_t(split) * chunk;
+  const int64_t s_end = s_begin + chunk < S ? s_begin + chunk : S;
+  const float* lg = logits + (size_t(b) * Hq + size_t(hkv) * G) * S;   // head h at lg + h S
+  const uint8_t* rows = payload + (size_t(grp) * S) * rb;
+  const uint32_t* nrm = reinterpret_cast<const uint32_t*>(norms) + size_t(grp) * S;
+
+  for (int i = tid; i < GP * kAcc; i += kAttThreads) sacc[i] = 0.f;
+  if (tid < GP) sl[tid] = 0.f;
+
+  // pass 1: the chunk's maximum logit per head
+  float mx[GP];
+#pragma unroll
+  for (int h = 0; h < GP; ++h) mx[h] = -INFINITY;
+  for (int64_t s = s_begin + tid; s < s_end; s += 8 * kAttThreads) {
+#pragma unroll
+    for (int h = 0; h < GP; ++h) {
+      if (h < G) {
+        float v[8];
+#pragma unroll
+        for (int x = 0; x < 8; ++x) {
+          const int64_t sx = s + int64_t(x) * kAttThreads;
+          v[x] = sx < s_end ? __ldg(lg + size_t(h) * S + sx) : -INFINITY;
+        }
+#pragma unroll
+        for (int x = 0; x < 8; ++x) mx[h] = fmaxf(mx[h], v[x]);
+      }
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < GP; ++h) {
+    float v = mx[h];
+    for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if (lane == 0) sred[h * kAttWarps + warp] = v;
+  }
+  __syncthreads();
+  if (tid < GP) {
+    float v = sred[tid * kAttWarps];
+    for (int w = 1; w < kAttWarps; ++w) v = fmaxf(v, sred[tid * kAttWarps + w]);
+    smx[tid] = v;
+  }
+  __syncthreads();
+
+  // unit g of every row (quarter g >> 1, unit g & 1): code and sign halfwords
+  const int code_off = (g >> 1) * kPerQ + (g & 1) * BM;
+  const int sign_off = (g >> 1) * kPerQ + 2 * BM + (g & 1);
+  const int wcol_head = g >> 1;          // B column g: head g / 2, limb g % 2
+  const bool wcol_lo = (g & 1) != 0;
+  float accC[8][4], accS[8][4];
+#pragma unroll
+  for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      accC[mt][c] = 0.f;
+      accS[mt][c] = 0.f;
+    }
+  constexpr int kWIt = T * GP / kAttThreads;
+  float lsum[kWIt];
+#pragma unroll
+  for (int it = 0; it < kWIt; ++it) lsum[it] = 0.f;
+
+  // rows: asynchronous 16-byte copies into the tile's buffer (rows past the
+  // chunk keep stale bytes; their weights are zero); logits and norms of the
+  // next tile prefetched into registers
+  auto copy_rows = [&](int64_t s0, uint8_t* dst) {
+    const int nk = int(s_end - s0 < T ? s_end - s0 : T);
+    const int nc = nk * rb / 16;
+    const uint8_t* src = rows + size_t(s0) * rb;
+    for (int c = tid; c < nc; c += kAttThreads)
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(uint32_t(__cvta_generic_to_shared(dst + 16 * c))),
+                   "l"(src + 16 * c)
+                   : "memory");
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  float lgv[kWIt];
+  uint32_t nnv[kWIt];
+  auto fetch_w = [&](int64_t s0) {
+    const int nk = int(s_end - s0 < T ? s_end - s0 : T);
+#pragma unroll
+    for (int it = 0; it < kWIt; ++it) {
+      const int idx = tid + it * kAttThreads;
+      const int k = idx % T, h = idx / T;
+      const bool ok = k < nk && h < G;
+      lgv[it] = ok ? __ldg(lg + size_t(h) * S + s0 + k) : 0.f;
+      nnv[it] = ok ? __ldg(nrm + s0 + k) : 0u;
+    }
+  };
+  if (s_begin < s_end) {
+    copy_rows(s_begin, srows0);
+    fetch_w(s_begin);
+  }
+  int buf = 0;
+  for (int64_t s0 = s_begin; s0 < s_end; s0 += T, buf ^= 1) {
+    const int nk = int(s_end - s0 < T ? s_end - s0 : T);
+    uint8_t* srows = srows0 + buf * T * rb;
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    __syncthreads();   // this tile's rows visible; every warp is done with the previous tile
+    if (s0 + T < s_end) copy_rows(s0 + T, srows0 + (buf ^ 1) * T * rb);
+#pragma unroll
+    for (int it = 0; it < kWIt; ++it) {
+      const int idx = tid + it * kAttThreads;
+      const int k = idx % T, h = idx / T;
+      float wn = 0.f, wr = 0.f;
+      if (k < nk && h < G) {
+        // exp(l - max) as 2^((l - max) log2 e)
+        const float w = exp2f((lgv[it] - smx[h]) * 1.4426950408889634f);
+        const uint32_t nn = nnv[it];
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&nn));
+        wn = w * f.x;
+        wr = w * f.y;
+        lsum[it] += w;
+      }
+      swn[k * GP + h] = wn;
+      swr[k * GP + h] = wr;
+    }
+    if (s0 + T < s_end) fetch_w(s0 + T);   // next tile's logits and norms in flight during the math
+    __syncthreads();
+#pragma unroll 1
+    for (int kb = warp * 16; kb < nk; kb += kAttWarps * 16) {   // 16-key steps; keys past nk have zero weight
+      __syncwarp();
+      const int kk[4] = {kb + 2 * tig, kb + 2 * tig + 1, kb + 2 * tig + 8, kb + 2 * tig + 9};
+      const uint32_t bC0 = weight_pair(swn[kk[0] * GP + wcol_head], swn[kk[1] * GP + wcol_head], wcol_lo);
+      const uint32_t bC1 = weight_pair(swn[kk[2] * GP + wcol_head], swn[kk[3] * GP + wcol_head], wcol_lo);
+      uint32_t hc[4][BM];
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        const uint16_t* hw = reinterpret_cast<const uint16_t*>(srows + kk[x] * rb);
+#pragma unroll
+        for (int y = 0; y < BM; ++y) hc[x][y] = hw[code_off + y];
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint32_t lo[4], hi[4];
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          const uint32_t sel = reg_selector<BM>(hc[x], i);
+          lo[x] = prmt(lut.lo[0], lut.lo[1], sel);
+          hi[x] = prmt(lut.hi[0], lut.hi[1], sel);
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          // bytes (key a, e = 2h), (key b, 2h), (a, 2h + 1), (b, 2h + 1) of each plane
+          const uint32_t ps = h ? 0x7362u : 0x5140u;
+          const uint32_t p01 = prmt(lo[0], lo[1], ps), q01 = prmt(hi[0], hi[1], ps);
+          const uint32_t p23 = prmt(lo[2], lo[3], ps), q23 = prmt(hi[2], hi[3], ps);
+          // fp16 pairs: row g (e = 2h) and row g + 8 (e = 2h + 1), keys (2 tig, 2 tig + 1) / (+8, +9)
+          const uint32_t a0 = prmt(p01, q01, 0x5140u), a1 = prmt(p01, q01, 0x7362u);
+          const uint32_t a2 = prmt(p23, q23, 0x5140u), a3 = prmt(p23, q23, 0x7362u);
+          mma_16816(accC[2 * i + h], a0, a1, a2, a3, bC0, bC1);
+        }
+      }
+      if constexpr (JL) {
+        const uint32_t bS0 = weight_pair(swr[kk[0] * GP + wcol_head], swr[kk[1] * GP + wcol_head], wcol_lo);
+        const uint32_t bS1 = weight_pair(swr[kk[2] * GP + wcol_head], swr[kk[3] * GP + wcol_head], wcol_lo);
+        uint32_t hs[4];
+#pragma unroll
+        for (int x = 0; x < 4; ++x) hs[x] = reinterpret_cast<const uint16_t*>(srows + kk[x] * rb)[sign_off];
+        // inverted sign bits of a key pair in the two halves: bit 4e + i of the
+        // halfword goes to bit 15 (key a) and bit 31 (key b) after a left shift
+        // by 15 - 4e - i; set means -1 (fp16 sign bit) over 1.0 (0x3C00)
+        const uint32_t w01 = ~(hs[0] | (hs[1] << 16)), w23 = ~(hs[2] | (hs[3] << 16));
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int e0 = 2 * h, e1 = 2 * h + 1;
+            const uint32_t a0 = ((w01 << (15 - 4 * e0 - i)) & 0x80008000u) | 0x3C003C00u;
+            const uint32_t a1 = ((w01 << (15 - 4 * e1 - i)) & 0x80008000u) | 0x3C003C00u;
+            const uint32_t a2 = ((w23 << (15 - 4 * e0 - i)) & 0x80008000u) | 0x3C003C00u;
+            const uint32_t a3 = ((w23 << (15 - 4 * e1 - i)) & 0x80008000u) | 0x3C003C00u;
+            mma_16816(accS[2 * i + h], a0, a1, a2, a3, bS0, bS1);
+          }
+      }
+    }
+  }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  __syncthreads();
+
+  // the rows of this thread's accumulators: unit g, register i, nibble e; head tig
+  if (tig < G) {
+    const int q = g >> 1, u = g & 1;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int j0 = q * 32 + 4 * (4 * u + i) + 2 * h;   // e = 2h (row g) and 2h + 1 (row g + 8)
+        atomicAdd(sacc + tig * kAcc + j0, accC[2 * i + h][0] + accC[2 * i + h][1]);
+        atomicAdd(sacc + tig * kAcc + j0 + 1, accC[2 * i + h][2] + accC[2 * i + h][3]);
+        if constexpr (JL) {
+          atomicAdd(sacc + tig * kAcc + 128 + j0, accS[2 * i + h][0] + accS[2 * i + h][1]);
+          atomicAdd(sacc + tig * kAcc + 128 + j0 + 1, accS[2 * i + h][2] + accS[2 * i + h][3]);
+        }
+      }
+  }
+#pragma unroll
+  for (int it = 0; it < kWIt; ++it) {
+    float v = lsum[it];
+    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    const int h = (tid + it * kAttThreads) / T;
+    if (lane == 0 && h < GP) atomicAdd(sl + h, v);
+  }
+  __syncthreads();
+  // partial record {max, sum, a[128], b[128 or 0]} in the generic layout (dp + mp slots)
+  constexpr int rec = 2 + 128 + (JL ? 128 : 0);
+  for (int h = 0; h < G; ++h) {
+    float* out = part + (size_t(blockIdx.x) * G + h) * rec;
+    for (int i = tid; i < rec - 2; i += kAttThreads) out[2 + i] = sacc[h * kAcc + i];
+    if (tid == 0) {
+      out[0] = smx[h];
+      out[1] = sl[h];
+    }
+  }
+}
+
 // One block per query head: merge the chunk partials, then
 // o = R^T (a + sqrt(pi/2)/m P^T b) / L.
 __global__ void __launch_bounds__(256) attend_combine_kernel(const float* __restrict__ part, int Hq, int Hkv,
@@ -411,6 +713,26 @@ cudaError_t dispatch_heads(const tq_ctx* ctx, const float* logits, int B, int Hq
   return launch_partial<BM, 8, NS>(ctx, logits, B, Hq, Hkv, S, ap, payload, norms, part, st);
 }
 
+template <int BM, bool JL>
+cudaError_t launch_mma_partial(const tq_ctx* ctx, const float* logits, int B, int Hq, int Hkv, int64_t S,
+                               AttPlan ap, const uint8_t* payload, const uint16_t* norms, float* part,
+                               cudaStream_t st) {
+  HalfLut lut{};
+  for (int v = 0; v < ctx->levels; ++v) {
+    const uint16_t bits = __half_as_ushort(__double2half(ctx->c[v]));
+    lut.lo[v / 4] |= uint32_t(bits & 0xFF) << (8 * (v % 4));
+    lut.hi[v / 4] |= uint32_t(bits >> 8) << (8 * (v % 4));
+  }
+  constexpr int rb = 8 * (2 * BM + (JL ? 2 : 0));
+  const size_t smem = size_t(2 * kAttMmaTile) * rb + size_t(2 * kAttMmaTile * 4) * 4 + size_t(4 * 256) * 4 +
+                      size_t(4 * kAttWarps + 8) * 4;
+  auto kern = attend_mma_kernel<BM, JL>;
+  cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  kern<<<unsigned(int64_t(B) * Hkv * ap.nsplit), kAttThreads, smem, st>>>(logits, Hq, Hkv, S, ap.chunk, ap.nsplit,
+                                                                          payload, norms, lut, part);
+  return cudaGetLastError();
+}
+
 template <int NS>
 cudaError_t dispatch_bits(const tq_ctx* ctx, const float* logits, int B, int Hq, int Hkv, int64_t S, AttPlan ap,
                           const uint8_t* payload, const uint16_t* norms, float* part, cudaStream_t st) {
@@ -441,8 +763,21 @@ cudaError_t launch_attend(const tq_ctx* ctx, const float* logits, int B, int Hq,
   const RowGeom g = make_geom(ctx->d, ctx->m, ctx->bmse);
   float* part = static_cast<float*>(ws);
   const bool two = g.dp > 128 || g.mp > 128;
-  cudaError_t e = two ? dispatch_bits<2>(ctx, logits, B, Hq, Hkv, S, ap, payload, norms, part, st)
-                      : dispatch_bits<1>(ctx, logits, B, Hq, Hkv, S, ap, payload, norms, part, st);
+  cudaError_t e;
+  if (ctx->d == 128 && (ctx->m == 128 || ctx->m == 0) && Hq / Hkv <= 4) {
+    // tensor-core partial sums
+    switch (ctx->bmse * 2 + (ctx->m > 0 ? 1 : 0)) {
+      case 2: e = launch_mma_partial<1, false>(ctx, logits, B, Hq, Hkv, S, ap, payload, norms, part, st); break;
+      case 3: e = launch_mma_partial<1, true>(ctx, logits, B, Hq, Hkv, S, ap, payload, norms, part, st); break;
+      case 4: e = launch_mma_partial<2, false>(ctx, logits, B, Hq, Hkv, S, ap, payload, norms, part, st); break;
+      case 5: e = launch_mma_partial<2, true>(ctx, logits, B, Hq, Hkv, S, ap, payload, norms, part, st); break;
+      case 6: e = launch_mma_partial<3, false>(ctx, logits, B, Hq, Hkv, S, ap, payload, norms, part, st); break;
+      default: e = launch_mma_partial<3, true>(ctx, logits, B, Hq, Hkv, S, ap, payload, norms, part, st); break;
+    }
+  } else {
+    e = two ? dispatch_bits<2>(ctx, logits, B, Hq, Hkv, S, ap, payload, norms, part, st)
+            : dispatch_bits<1>(ctx, logits, B, Hq, Hkv, S, ap, payload, norms, part, st);
+  }
   if (e != cudaSuccess) return e;
   const size_t smem = size_t(g.dp + g.mp) * 4;
   attend_combine_kernel<<<unsigned(B * Hq), 256, smem, st>>>(part, Hq, Hkv, ap.nsplit, ctx->dR, ctx->dP, ctx->d,
