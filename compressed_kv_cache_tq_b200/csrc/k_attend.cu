@@ -358,11 +358,14 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_mma_kernel(
   constexpr int GP = 4;
   constexpr int kPerQ = 2 * BM + (JL ? 2 : 0);   // halfwords per quarter chunk (d = m = 128)
   constexpr int rb = 8 * kPerQ;                   // row bytes
+  // row stride in shared memory: an odd number of 16-byte chunks, so that the
+  // rows two apart read by the four lanes of a quad fall in different banks
+  constexpr int rs = (rb / 16) % 2 ? rb : rb + 16;
   constexpr int kAcc = 256;                       // a (128 coordinates) then b (128 sign coordinates)
   constexpr int T = kAttMmaTile;
   extern __shared__ __align__(16) uint8_t sm[];
-  uint8_t* srows0 = sm;                                                       // [2][T][rb] rows, double-buffered
-  float* swn = reinterpret_cast<float*>(sm + 2 * T * rb);                     // [T][GP]  w n16
+  uint8_t* srows0 = sm;                                                       // [2][T][rs] rows, double-buffered
+  float* swn = reinterpret_cast<float*>(sm + 2 * T * rs);                     // [T][GP]  w n16
   float* swr = swn + T * GP;                                                  // [T][GP]  w rho16
   float* sacc = swr + T * GP;                                                 // [GP][kAcc]
   float* sred = sacc + GP * kAcc;                                             // [GP][kAttWarps] maxima
@@ -439,12 +442,16 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_mma_kernel(
   // next tile prefetched into registers
   auto copy_rows = [&](int64_t s0, uint8_t* dst) {
     const int nk = int(s_end - s0 < T ? s_end - s0 : T);
-    const int nc = nk * rb / 16;
+    constexpr int kc = rb / 16;   // 16-byte chunks per row
+    const int nc = nk * kc;
     const uint8_t* src = rows + size_t(s0) * rb;
-    for (int c = tid; c < nc; c += kAttThreads)
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(uint32_t(__cvta_generic_to_shared(dst + 16 * c))),
+    for (int c = tid; c < nc; c += kAttThreads) {
+      const int r = c / kc, cc = c - r * kc;
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                       uint32_t(__cvta_generic_to_shared(dst + r * rs + 16 * cc))),
                    "l"(src + 16 * c)
                    : "memory");
+    }
     asm volatile("cp.async.commit_group;" ::: "memory");
   };
   float lgv[kWIt];
@@ -467,10 +474,10 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_mma_kernel(
   int buf = 0;
   for (int64_t s0 = s_begin; s0 < s_end; s0 += T, buf ^= 1) {
     const int nk = int(s_end - s0 < T ? s_end - s0 : T);
-    uint8_t* srows = srows0 + buf * T * rb;
+    uint8_t* srows = srows0 + buf * T * rs;
     asm volatile("cp.async.wait_group 0;" ::: "memory");
     __syncthreads();   // this tile's rows visible; every warp is done with the previous tile
-    if (s0 + T < s_end) copy_rows(s0 + T, srows0 + (buf ^ 1) * T * rb);
+    if (s0 + T < s_end) copy_rows(s0 + T, srows0 + (buf ^ 1) * T * rs);
 #pragma unroll
     for (int it = 0; it < kWIt; ++it) {
       const int idx = tid + it * kAttThreads;
@@ -499,7 +506,7 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_mma_kernel(
       uint32_t hc[4][BM];
 #pragma unroll
       for (int x = 0; x < 4; ++x) {
-        const uint16_t* hw = reinterpret_cast<const uint16_t*>(srows + kk[x] * rb);
+        const uint16_t* hw = reinterpret_cast<const uint16_t*>(srows + kk[x] * rs);
 #pragma unroll
         for (int y = 0; y < BM; ++y) hc[x][y] = hw[code_off + y];
       }
@@ -529,7 +536,7 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_mma_kernel(
         const uint32_t bS1 = weight_pair(swr[kk[2] * GP + wcol_head], swr[kk[3] * GP + wcol_head], wcol_lo);
         uint32_t hs[4];
 #pragma unroll
-        for (int x = 0; x < 4; ++x) hs[x] = reinterpret_cast<const uint16_t*>(srows + kk[x] * rb)[sign_off];
+        for (int x = 0; x < 4; ++x) hs[x] = reinterpret_cast<const uint16_t*>(srows + kk[x] * rs)[sign_off];
         // inverted sign bits of a key pair in the two halves: bit 4e + i of the
         // halfword goes to bit 15 (key a) and bit 31 (key b) after a left shift
         // by 15 - 4e - i; set means -1 (fp16 sign bit) over 1.0 (0x3C00)
@@ -632,6 +639,7 @@ __global__ void __launch_bounds__(256) attend_combine_kernel(const float* __rest
   const float L = sL;
   for (int j = threadIdx.x; j < g.dp + g.mp; j += blockDim.x) {
     float acc = 0.f;
+#pragma unroll 4
     for (int i = 0; i < nsplit; ++i) acc = fmaf(sf[i], p0[size_t(i) * G * rec + 2 + j], acc);
     sv[j] = acc;
   }
@@ -642,6 +650,7 @@ __global__ void __launch_bounds__(256) attend_combine_kernel(const float* __rest
   if (threadIdx.x < d) {
     const int j = threadIdx.x;
     float t = 0.f;
+#pragma unroll 8
     for (int k = 0; k < m; ++k) t = fmaf(P[size_t(k) * d + j], sb[k], t);
     u_own = (sa[j] + qc * t) * inv;
   }
@@ -651,6 +660,7 @@ __global__ void __launch_bounds__(256) attend_combine_kernel(const float* __rest
   if (threadIdx.x < d) {
     const int i = threadIdx.x;
     float o = 0.f;
+#pragma unroll 8
     for (int j = 0; j < d; ++j) o = fmaf(R[size_t(j) * d + i], sa[j], o);
     out[size_t(bh) * d + i] = o;
   }
@@ -724,7 +734,8 @@ cudaError_t launch_mma_partial(const tq_ctx* ctx, const float* logits, int B, in
     lut.hi[v / 4] |= uint32_t(bits >> 8) << (8 * (v % 4));
   }
   constexpr int rb = 8 * (2 * BM + (JL ? 2 : 0));
-  const size_t smem = size_t(2 * kAttMmaTile) * rb + size_t(2 * kAttMmaTile * 4) * 4 + size_t(4 * 256) * 4 +
+  constexpr int rs = (rb / 16) % 2 ? rb : rb + 16;   // padded row stride (as in the kernel)
+  const size_t smem = size_t(2 * kAttMmaTile) * rs + size_t(2 * kAttMmaTile * 4) * 4 + size_t(4 * 256) * 4 +
                       size_t(4 * kAttWarps + 8) * 4;
   auto kern = attend_mma_kernel<BM, JL>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
