@@ -39,8 +39,13 @@ def _oracle_attention(logits, payload, norms, tb, Hkv):
 @pytest.mark.parametrize("B,Hkv,G,S,d,bits,m", [(2, 2, 4, 517, 128, 4, 128), (1, 3, 2, 64, 128, 3, 128),
                                                 (2, 1, 8, 1000, 128, 2, 128), (1, 2, 1, 33, 64, 3, 64),
                                                 (1, 1, 4, 300, 200, 3, 200), (1, 2, 4, 257, 128, 4, 0),
-                                                (2, 2, 4, 1, 128, 4, 128), (1, 2, 3, 190, 128, 3, 128)])
+                                                (2, 2, 4, 1, 128, 4, 128), (1, 2, 3, 190, 128, 3, 128),
+                                                (1, 2, 1, 300, 128, 4, 128), (2, 1, 2, 700, 128, 2, 128),
+                                                (1, 1, 4, 600, 128, 2, 0), (1, 1, 4, 3000, 128, 3, 0)])
 def test_attend_against_oracle(lib, B, Hkv, G, S, d, bits, m):
+    """d = m = 128 (or m = 0) with up to 4 query heads per KV head runs on the
+    tensor-core kernel, the other shapes on CUDA cores; S up to 3000 gives
+    several key tiles per chunk."""
     ctx = lib.tq_init(d, bits, 77, m=m)
     v, V64 = _values(B, Hkv, S, d, seed=2001 + S)
     payload, norms = lib.tq_quantize(ctx, v)
@@ -102,7 +107,8 @@ def test_decode_attention_end_to_end(lib):
 
 def test_attend_full_size_sampled(lib):
     """The decode workload's shape (batch 8, 8 KV heads, 32 query heads, seq
-    32768, b = 4): every output of three (batch, KV head) groups."""
+    32768, b = 4, several key tiles per chunk and several chunks per group):
+    every output of six (batch, KV head) groups."""
     B, Hkv, G, S, d = 8, 8, 4, 32768, 128
     ctx = lib.tq_init(d, 4, 142)
     v = W.decode_keys(B, Hkv, S, d, 2002, device=DEV).reshape(-1, d)
@@ -113,7 +119,7 @@ def test_attend_full_size_sampled(lib):
     assert lib.tq_check_device_status(ctx) == 0
     tb = tables_of(ctx)
     lg = logits.cpu().numpy().astype(np.float64)
-    for b, h in [(0, 0), (B - 1, Hkv - 1), (3, 5)]:
+    for b, h in [(0, 0), (B - 1, Hkv - 1), (3, 5), (4, 6), (2, 0), (5, 1)]:
         rows = slice((b * Hkv + h) * S, (b * Hkv + h + 1) * S)
         ref, A = _oracle_attention(lg[b:b + 1, h * G:(h + 1) * G], payload[rows].cpu().numpy(),
                                    norms[rows].cpu().numpy(), tb, 1)
