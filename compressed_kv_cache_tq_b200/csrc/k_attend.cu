@@ -37,6 +37,7 @@ constexpr int kAttTile = 128;         // keys per staged tile
 constexpr int kAttMaxLd = 8;          // 8-byte words per thread per tile (rows of up to 128 bytes)
 constexpr int kAttMaxHeads = 8;
 constexpr int kAttMmaTile = 256;      // keys per staged tile of the tensor-core kernel
+constexpr int kAttStages = 2;         // row tiles in flight per block (cp.async ring)
 
 __device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
 
@@ -338,16 +339,11 @@ __device__ __forceinline__ uint32_t reg_selector(const uint32_t (&h)[BM], int i)
   }
 }
 
-// Two weights (keys a, b) of one column as an fp16 pair: the hi limb, or the
-// lo limb w - hi.
-// Branch-free (the lanes of a warp take different limbs, and the MMA that
-// consumes the pair needs the whole warp converged).
-__device__ __forceinline__ uint32_t weight_pair(float wa, float wb, bool lo_limb) {
-  const __half ha = __float2half_rn(wa), hb = __float2half_rn(wb);
-  const __half la = __float2half_rn(wa - __half2float(ha)), lb = __float2half_rn(wb - __half2float(hb));
-  const uint32_t hi2 = uint32_t(__half_as_ushort(ha)) | (uint32_t(__half_as_ushort(hb)) << 16);
-  const uint32_t lo2 = uint32_t(__half_as_ushort(la)) | (uint32_t(__half_as_ushort(lb)) << 16);
-  return lo_limb ? lo2 : hi2;
+// A weight as its fp16 hi limb (low half) and lo limb w - hi (high half).
+__device__ __forceinline__ uint32_t limb_pair(float w) {
+  const __half hi = __float2half_rn(w);
+  const __half lo = __float2half_rn(w - __half2float(hi));
+  return uint32_t(__half_as_ushort(hi)) | (uint32_t(__half_as_ushort(lo)) << 16);
 }
 
 template <int BM, bool JL>
@@ -364,10 +360,11 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_mma_kernel(
   constexpr int kAcc = 256;                       // a (128 coordinates) then b (128 sign coordinates)
   constexpr int T = kAttMmaTile;
   extern __shared__ __align__(16) uint8_t sm[];
-  uint8_t* srows0 = sm;                                                       // [2][T][rs] rows, double-buffered
-  float* swn = reinterpret_cast<float*>(sm + 2 * T * rs);                     // [T][GP]  w n16
-  float* swr = swn + T * GP;                                                  // [T][GP]  w rho16
-  float* sacc = swr + T * GP;                                                 // [GP][kAcc]
+  uint8_t* srows0 = sm;                                                       // [kAttStages][T][rs] row ring
+  // weights as fp16 (hi, lo) limb pairs: w n16 for the codes, w rho16 for the signs
+  uint32_t* swn = reinterpret_cast<uint32_t*>(sm + kAttStages * T * rs);      // [T][GP]
+  uint32_t* swr = swn + T * GP;                                               // [T][GP]
+  float* sacc = reinterpret_cast<float*>(swr + T * GP);                       // [GP][kAcc]
   float* sred = sacc + GP * kAcc;                                             // [GP][kAttWarps] maxima
   float* smx = sred + GP * kAttWarps;                                         // [GP] chunk maximum
   float* sl = smx + GP;                                                       // [GP] sum of weights
@@ -423,7 +420,7 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_mma_kernel(
   const int code_off = (g >> 1) * kPerQ + (g & 1) * BM;
   const int sign_off = (g >> 1) * kPerQ + 2 * BM + (g & 1);
   const int wcol_head = g >> 1;          // B column g: head g / 2, limb g % 2
-  const bool wcol_lo = (g & 1) != 0;
+  const uint32_t wsel = (g & 1) ? 0x7632u : 0x5410u;   // picks that limb of two keys' limb pairs
   float accC[8][4], accS[8][4];
 #pragma unroll
   for (int mt = 0; mt < 8; ++mt)
@@ -441,7 +438,7 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_mma_kernel(
   // chunk keep stale bytes; their weights are zero); logits and norms of the
   // next tile prefetched into registers
   auto copy_rows = [&](int64_t s0, uint8_t* dst) {
-    const int nk = int(s_end - s0 < T ? s_end - s0 : T);
+    const int nk = int(s_end - s0 < T ? s_end - s0 : T);   // <= 0 past the chunk: an empty group
     constexpr int kc = rb / 16;   // 16-byte chunks per row
     const int nc = nk * kc;
     const uint8_t* src = rows + size_t(s0) * rb;
@@ -467,17 +464,19 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_mma_kernel(
       nnv[it] = ok ? __ldg(nrm + s0 + k) : 0u;
     }
   };
+  // one commit group per tile, kAttStages - 1 tiles ahead of the one in use
   if (s_begin < s_end) {
-    copy_rows(s_begin, srows0);
+#pragma unroll
+    for (int st = 0; st < kAttStages - 1; ++st) copy_rows(s_begin + int64_t(st) * T, srows0 + st * T * rs);
     fetch_w(s_begin);
   }
-  int buf = 0;
-  for (int64_t s0 = s_begin; s0 < s_end; s0 += T, buf ^= 1) {
+  int ti = 0;
+  for (int64_t s0 = s_begin; s0 < s_end; s0 += T, ++ti) {
     const int nk = int(s_end - s0 < T ? s_end - s0 : T);
-    uint8_t* srows = srows0 + buf * T * rs;
-    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    uint8_t* srows = srows0 + (ti % kAttStages) * T * rs;
+    asm volatile("cp.async.wait_group %0;" ::"n"(kAttStages - 2) : "memory");
     __syncthreads();   // this tile's rows visible; every warp is done with the previous tile
-    if (s0 + T < s_end) copy_rows(s0 + T, srows0 + (buf ^ 1) * T * rs);
+    copy_rows(s0 + int64_t(kAttStages - 1) * T, srows0 + ((ti + kAttStages - 1) % kAttStages) * T * rs);
 #pragma unroll
     for (int it = 0; it < kWIt; ++it) {
       const int idx = tid + it * kAttThreads;
@@ -492,17 +491,17 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_mma_kernel(
         wr = w * f.y;
         lsum[it] += w;
       }
-      swn[k * GP + h] = wn;
-      swr[k * GP + h] = wr;
+      swn[k * GP + h] = limb_pair(wn);
+      swr[k * GP + h] = limb_pair(wr);
     }
     if (s0 + T < s_end) fetch_w(s0 + T);   // next tile's logits and norms in flight during the math
     __syncthreads();
-#pragma unroll 1
+#pragma unroll 2
     for (int kb = warp * 16; kb < nk; kb += kAttWarps * 16) {   // 16-key steps; keys past nk have zero weight
       __syncwarp();
       const int kk[4] = {kb + 2 * tig, kb + 2 * tig + 1, kb + 2 * tig + 8, kb + 2 * tig + 9};
-      const uint32_t bC0 = weight_pair(swn[kk[0] * GP + wcol_head], swn[kk[1] * GP + wcol_head], wcol_lo);
-      const uint32_t bC1 = weight_pair(swn[kk[2] * GP + wcol_head], swn[kk[3] * GP + wcol_head], wcol_lo);
+      const uint32_t bC0 = prmt(swn[kk[0] * GP + wcol_head], swn[kk[1] * GP + wcol_head], wsel);
+      const uint32_t bC1 = prmt(swn[kk[2] * GP + wcol_head], swn[kk[3] * GP + wcol_head], wsel);
       uint32_t hc[4][BM];
 #pragma unroll
       for (int x = 0; x < 4; ++x) {
@@ -532,8 +531,8 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_mma_kernel(
         }
       }
       if constexpr (JL) {
-        const uint32_t bS0 = weight_pair(swr[kk[0] * GP + wcol_head], swr[kk[1] * GP + wcol_head], wcol_lo);
-        const uint32_t bS1 = weight_pair(swr[kk[2] * GP + wcol_head], swr[kk[3] * GP + wcol_head], wcol_lo);
+        const uint32_t bS0 = prmt(swr[kk[0] * GP + wcol_head], swr[kk[1] * GP + wcol_head], wsel);
+        const uint32_t bS1 = prmt(swr[kk[2] * GP + wcol_head], swr[kk[3] * GP + wcol_head], wsel);
         uint32_t hs[4];
 #pragma unroll
         for (int x = 0; x < 4; ++x) hs[x] = reinterpret_cast<const uint16_t*>(srows + kk[x] * rs)[sign_off];
@@ -735,7 +734,7 @@ cudaError_t launch_mma_partial(const tq_ctx* ctx, const float* logits, int B, in
   }
   constexpr int rb = 8 * (2 * BM + (JL ? 2 : 0));
   constexpr int rs = (rb / 16) % 2 ? rb : rb + 16;   // padded row stride (as in the kernel)
-  const size_t smem = size_t(2 * kAttMmaTile) * rs + size_t(2 * kAttMmaTile * 4) * 4 + size_t(4 * 256) * 4 +
+  const size_t smem = size_t(kAttStages * kAttMmaTile) * rs + size_t(2 * kAttMmaTile * 4) * 4 + size_t(4 * 256) * 4 +
                       size_t(4 * kAttWarps + 8) * 4;
   auto kern = attend_mma_kernel<BM, JL>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
