@@ -1,8 +1,10 @@
 // Channel split of a key cache into a high-variance and a low-variance group
-// (fractional bit rates such as 2.5 bits per channel: arXiv summary page
-// "3.5 bits per channel", mooersco.com section 2.1 "TurboQuant 2.5bit",
-// zhengruan.com on the 2.5-bit quality; mooersco.com's FAQ on channel
-// variances that differ by orders of magnitude before rotation).
+// (fractional bit rates such as 2.5 bits per channel: the rom4ai.github.io
+// note "TurboQuant: Online Vector Quantization with Near-Optimal Distortion
+// Rate" states the cache size as 3.5 bits per channel; mooersco.com section
+// 2.1 lists a 2.5-bit setting; zhengruan.com reports its small quality loss;
+// mooersco.com's FAQ says channel variances differ by orders of magnitude
+// before rotation).
 //
 // Plan: per KV head, the variance of every channel over all B x S keys of the
 // head; the hi->d channels of largest variance (ties to the lower channel)

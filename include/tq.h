@@ -206,8 +206,10 @@ tq_status tq_topk(const tq_ctx* ctx, const float* q, int64_t nq, const uint8_t* 
 
 /* ------------------------------------------------------------------------
  * Channel split: fractional bit rates such as 2.5 bits per channel
- * (arXiv summary page: "3.5 bits per channel"; mooersco.com section 2.1:
- * "TurboQuant 2.5bit >= 7x"; zhengruan.com: 2.5 bits costs a slight drop).
+ * (the rom4ai.github.io note "TurboQuant: Online Vector Quantization with
+ * Near-Optimal Distortion Rate" sizes the cache at 3.5 bits per channel;
+ * mooersco.com section 2.1 lists a 2.5-bit setting; zhengruan.com reports a
+ * small quality loss at 2.5 bits).
  * The pages do not say how a fractional rate is reached; this library's
  * reading: per KV head, the channels are split into a high-variance group and
  * a low-variance group (mooersco.com FAQ: unrotated channel variances differ

@@ -450,11 +450,13 @@ def attention_output(logits: np.ndarray, codes, bits, n16, rho16, tb: Tables, Hk
 # ---------------------------------------------------------------------------
 # Channel split: fractional bit rates such as 2.5 bits per channel
 #
-# The pages quote 3.5- and 2.5-bit configurations (arXiv summary page:
-# "3.5 bits per channel"; mooersco.com section 2.1: "2.5bit >= 7x";
-# zhengruan.com: 2.5 bits costs a slight quality drop) without saying how a
-# fractional rate is reached, and mooersco.com's FAQ notes that the
-# unrotated channels' variances differ by two orders of magnitude.  Reading:
+# The pages give 3.5- and 2.5-bit settings (the rom4ai.github.io note
+# "TurboQuant: Online Vector Quantization with Near-Optimal Distortion Rate"
+# sizes the cache at 3.5 bits per channel; mooersco.com section 2.1 lists a
+# 2.5-bit setting with at least 7x less memory; zhengruan.com reports a small
+# quality loss at 2.5 bits) without saying how a fractional rate is reached,
+# and mooersco.com's FAQ notes that the unrotated channels' variances differ
+# by two orders of magnitude.  Reading:
 # per KV head, the d_hi channels of largest variance form a high group and
 # the rest a low group; each group is quantised as its own vector with its
 # own tables (rotation, JL matrix, codebook) and bit width, and the inner
