@@ -22,6 +22,18 @@ of the same workload on the host cores, on rank 0 only.
 sequence of 131072 keys for each of 8 KV heads (keys drawn as above), b = 3
 (2 Lloyd-Max bits + 1 QJL bit), 32 query heads.
 
+--workload split runs the 2.5-bit channel split: 32 x 8 x 16384 keys, per KV
+head the 64 channels of largest variance at b = 3 and the other 64 at b = 2
+(each group its own d = 64 quantizer); a step is tq_split_quantize plus
+tq_split_logits (the channel plan is computed once, before the steps).
+
+--workload attend adds a quantised value cache to the decode layer: a step
+quantizes keys and values, computes the logits and the attention output
+(tq_attend).
+
+--workload mse runs the decode layer with the MSE-only variant (m = 0: no
+sign sketch).
+
 --workload search times the vector-search configuration instead (one JSON
 line): 1 000 000 unit vectors of a 100-cluster Gaussian mixture, d = 200 fp32,
 10 000 queries drawn the same way, b = 2 and b = 4, top-10 by the estimator

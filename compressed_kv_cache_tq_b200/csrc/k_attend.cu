@@ -39,8 +39,6 @@ constexpr int kAttMaxHeads = 8;
 constexpr int kAttMmaTile = 256;      // keys per staged tile of the tensor-core kernel
 constexpr int kAttStages = 2;         // row tiles in flight per block (cp.async ring)
 
-__device__ __forceinline__ float2 f2(float a) { return make_float2(a, a); }
-
 // The slot's 4 codes (r = 4u + i, e = 0..3) as nibbles e of one word, from the
 // unit's code halfwords h[0 .. BM-1] (layout in include/tq.h): code e is
 // (v >> 4e) & (2^BM - 1).  For b' = 3, register 3's code bits sit in bit 3 of
