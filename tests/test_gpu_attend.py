@@ -124,3 +124,24 @@ def test_attend_full_size_sampled(lib):
         ref, A = _oracle_attention(lg[b:b + 1, h * G:(h + 1) * G], payload[rows].cpu().numpy(),
                                    norms[rows].cpu().numpy(), tb, 1)
         check_close(out[b, h * G:(h + 1) * G].cpu().numpy(), ref[0], A[0])
+
+
+def test_attend_argument_errors(lib):
+    """A short workspace and misaligned rows are refused before any launch."""
+    import ctypes
+
+    ctx = lib.tq_init(128, 4, 77)
+    v, _ = _values(1, 2, 64, 128, seed=6)
+    payload, norms = lib.tq_quantize(ctx, v)
+    logits = torch.zeros((1, 8, 64), device=DEV)
+    out = torch.empty((1, 8, 128), device=DEV)
+    L = lib.lib()
+    need = lib.tq_attend_workspace_bytes(ctx, 1, 8, 2, 64)
+    ws = torch.empty(need, dtype=torch.uint8, device=DEV)
+    vp = ctypes.c_void_p
+    assert L.tq_attend(ctx.handle, vp(logits.data_ptr()), 1, 8, 2, 64, vp(payload.data_ptr()), vp(norms.data_ptr()),
+                       vp(out.data_ptr()), vp(ws.data_ptr()), need - 1, None) == 5
+    assert L.tq_attend(ctx.handle, vp(logits.data_ptr()), 1, 8, 2, 64, vp(payload.data_ptr() + 8),
+                       vp(norms.data_ptr()), vp(out.data_ptr()), vp(ws.data_ptr()), need, None) == 1
+    assert L.tq_attend(ctx.handle, vp(logits.data_ptr()), 1, 8, 3, 64, vp(payload.data_ptr()), vp(norms.data_ptr()),
+                       vp(out.data_ptr()), vp(ws.data_ptr()), need, None) == 1

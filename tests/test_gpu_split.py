@@ -217,3 +217,36 @@ def test_split_logits_cuda_core_path(lib, d_hi, d_lo, bits_hi, bits_lo, G):
     ref, A = _oracle_split_logits(q.astype(np.float64), perm, ph.cpu().numpy(), nh.cpu().numpy(), pl.cpu().numpy(),
                                   nl.cpu().numpy(), tables_of(hi), tables_of(lo), B, Hkv, S, 0.5)
     check_close(out.cpu().numpy(), ref, A)
+
+
+def test_split_argument_errors(lib):
+    """Misaligned buffers, a short workspace and mismatched shapes are refused
+    with an error status before any launch."""
+    import ctypes
+
+    hi, lo = lib.tq_init(64, 3, 42), lib.tq_init(64, 2, 43)
+    sp = lib.tq_split_create(hi, lo, 2)
+    keys = torch.zeros((1, 2, 16, 128), dtype=torch.bfloat16, device=DEV)
+    L = lib.lib()
+    ph = torch.empty((32, hi.row_bytes + 16), dtype=torch.uint8, device=DEV)
+    nh = torch.empty((32, 2), dtype=torch.float16, device=DEV)
+    pl = torch.empty((32, lo.row_bytes), dtype=torch.uint8, device=DEV)
+    nl = torch.empty((32, 2), dtype=torch.float16, device=DEV)
+    vp = ctypes.c_void_p
+    # keys pointer off 16-byte alignment
+    st = L.tq_split_quantize(sp.handle, vp(keys.data_ptr() + 2), 1, 1, 16, vp(ph.data_ptr()), vp(nh.data_ptr()),
+                             vp(pl.data_ptr()), vp(nl.data_ptr()), None)
+    assert st == 1
+    # plan workspace too small
+    ws = torch.empty(64, dtype=torch.uint8, device=DEV)
+    assert L.tq_split_plan(sp.handle, vp(keys.data_ptr()), 1, 1, 16, vp(ws.data_ptr()), 64, None) == 5
+    # query heads not a multiple of the KV heads
+    q = torch.zeros((1, 3, 128), device=DEV)
+    out = torch.empty((1, 3, 16), device=DEV)
+    ws2 = torch.empty(1 << 16, dtype=torch.uint8, device=DEV)
+    assert L.tq_split_logits(sp.handle, vp(q.data_ptr()), 1, 3, 16, vp(ph.data_ptr()), vp(nh.data_ptr()),
+                             vp(pl.data_ptr()), vp(nl.data_ptr()), 1.0, vp(out.data_ptr()), vp(ws2.data_ptr()),
+                             ws2.numel(), None) == 1
+    # a split of 512 channels (the largest: two 256-channel contexts) is accepted
+    sp2 = lib.tq_split_create(lib.tq_init(256, 3, 3), lib.tq_init(256, 2, 4), 1)
+    sp2.close()
