@@ -264,16 +264,34 @@ def cpu_baseline(budget_s: float = 12.0, max_keys: int = 1 << 19):
 
 
 def run_search(args):
-    """Vector-search workload: index build + top-10 of 10 000 queries over 10^6 rows."""
+    """Vector-search workload: index build + top-10 of 10 000 queries over 10^6 rows.
+
+    With --gpus N (torchrun, NCCL) the database is split by rows over the
+    ranks (strong scaling: the total stays 10^6 rows): each rank indexes and
+    searches its block, and the per-rank top-10 lists are all-gathered and
+    merged on the device (compressed_kv_cache_tq_b200.sharded)."""
     import numpy as np
     import torch
 
-    from compressed_kv_cache_tq_b200 import tq, workloads as W
+    from compressed_kv_cache_tq_b200 import sharded, tq, workloads as W
 
     n, nq, d, k = args.rows, args.queries, 200, 10
-    dev = torch.device("cuda", 0)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    first, count = sharded.shard_rows(n, world, rank)
+    firsts = [sharded.shard_rows(n, world, r)[0] for r in range(world)]
     db = torch.from_numpy(W.search_vectors(n, d, seed=1004, which=0)).to(dev)
+    shard = db[first:first + count]
     qs = torch.from_numpy(W.search_vectors(nq, d, seed=1004, which=1)).to(dev)
     # exact top-1 of every query by the plain inner product (fp32, on the device)
     top1 = torch.empty(nq, dtype=torch.int64, device=dev)
@@ -282,24 +300,33 @@ def run_search(args):
     stream = torch.cuda.current_stream()
     per_bits = {}
     hbm, tf, tf_sus, src = peaks()
-    with ClockSampler(0) as clocks:
+
+    def search(ctx, qv, payload, norms, ws):
+        ids, scores = tq.tq_topk(ctx, qv, payload, norms, k, workspace=ws)
+        if world > 1:
+            ids, scores = sharded.gather_topk(ids, scores, firsts, k)
+        return ids, scores
+
+    with ClockSampler(local) as clocks:
         for bits in (2, 4):
             ctx = tq.tq_init(d, bits, SEED_TABLES)
-            payload = torch.empty((n, ctx.row_bytes), dtype=torch.uint8, device=dev)
-            norms = torch.empty((n, 2), dtype=torch.float16, device=dev)
-            ws = torch.empty(tq.tq_topk_workspace_bytes(ctx, nq, n, k), dtype=torch.uint8, device=dev)
+            payload = torch.empty((count, ctx.row_bytes), dtype=torch.uint8, device=dev)
+            norms = torch.empty((count, 2), dtype=torch.float16, device=dev)
+            ws = torch.empty(tq.tq_topk_workspace_bytes(ctx, nq, count, k), dtype=torch.uint8, device=dev)
             ids = scores = None
             for _ in range(args.warmup):
-                tq.tq_quantize(ctx, db, payload, norms)
-                ids, scores = tq.tq_topk(ctx, qs, payload, norms, k, workspace=ws)
+                tq.tq_quantize(ctx, shard, payload, norms)
+                ids, scores = search(ctx, qs, payload, norms, ws)
             torch.cuda.synchronize()
             ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
             t_build, t_search = [], []
             for _ in range(args.steps):
+                if dist is not None:
+                    dist.barrier()
                 ev[0].record(stream)
-                tq.tq_quantize(ctx, db, payload, norms)
+                tq.tq_quantize(ctx, shard, payload, norms)
                 ev[1].record(stream)
-                ids, scores = tq.tq_topk(ctx, qs, payload, norms, k, workspace=ws)
+                ids, scores = search(ctx, qs, payload, norms, ws)
                 ev[2].record(stream)
                 torch.cuda.synchronize()
                 t_build.append(ev[0].elapsed_time(ev[1]))
@@ -311,24 +338,32 @@ def run_search(args):
             hid = torch.empty((nq, k), dtype=torch.int64, pin_memory=True)
             hsc = torch.empty((nq, k), dtype=torch.float32, pin_memory=True)
             dq = torch.empty_like(qs)
+            if dist is not None:
+                dist.barrier()
             a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
             dq.copy_(hq, non_blocking=True)
-            i2, s2 = tq.tq_topk(ctx, dq, payload, norms, k, workspace=ws)
+            i2, s2 = search(ctx, dq, payload, norms, ws)
             hid.copy_(i2, non_blocking=True)
             hsc.copy_(s2, non_blocking=True)
             b_.record(stream)
             torch.cuda.synchronize()
-            ms_s = sorted(t_search)[len(t_search) // 2]
-            flops = 2.0 * (d + d) * n * nq
+            ms_b = max_over_ranks(sorted(t_build)[len(t_build) // 2], dist, dev)
+            ms_s = max_over_ranks(sorted(t_search)[len(t_search) // 2], dist, dev)
+            e2e = max_over_ranks(a.elapsed_time(b_), dist, dev)
+            flops = 2.0 * (d + d) * count * nq   # this rank's share of the contraction
             per_bits[f"b{bits}"] = {
-                "index_build_ms": sorted(t_build)[len(t_build) // 2], "search_ms": ms_s,
+                "index_build_ms": ms_b, "search_ms": ms_s,
                 "queries_per_s": nq / ms_s * 1e3, "recall_at_1_at_10": recall,
-                "search_TFLOP_s": flops / ms_s / 1e9, "e2e_ms": a.elapsed_time(b_)}
+                "search_TFLOP_s_per_gpu": flops / ms_s / 1e9, "e2e_ms": e2e}
             del ws
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
     # the oracle on a bounded sample: up to 200 000 rows indexed, 128 queries scored against them
     cpu = None
-    if not args.no_cpu_baseline:
+    if not args.no_cpu_baseline and world == 1:
         from oracle import tq_oracle as O
         tb = O.make_tables(d, 2, SEED_TABLES, m=d)
         n_cpu = min(n, 200_000)
@@ -345,22 +380,22 @@ def run_search(args):
     b4 = per_bits["b4"]
     line = {
         "metric": "tq_topk queries/s (10^6 rows, d=200, top-10) and recall@1@10; index build ms",
-        "value": b4["queries_per_s"], "unit": "queries/s", "n_gpus": 1, "steps": args.steps,
+        "value": b4["queries_per_s"], "unit": "queries/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": b4["index_build_ms"] + b4["search_ms"],
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+        "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f16",
         "data": "synthetic",
         "config": {"workload": f"vector_search_{n}_d200_nq{nq}_top10", "rows": n, "queries": nq, "d": d, "m": d,
-                   "k": k, "bits": [2, 4],
+                   "k": k, "bits": [2, 4], "parallelism": f"rows sharded x{world}",
                    "l2": f"the fp16 row matrix ({n * 896 / 1e6:.0f} MB) "
                          + ("exceeds L2" if n * 896 > 126e6 else "fits in L2 (profiling size)")},
         "per_bits": per_bits,
-        "roofline": {"bound": "tensor", "kernel": "tq_topk (decode + scoring + re-scoring)",
-                     "achieved": b4["search_TFLOP_s"], "peak": tf, "unit": "TFLOP/s",
-                     "frac": b4["search_TFLOP_s"] / tf, "peak_source": src + " (bf16 GEMM; fp16 has the same rate)",
-                     "traffic": None},
+        "roofline": {"bound": "tensor", "kernel": "tq_topk (decode + scoring + re-scoring), per GPU",
+                     "achieved": b4["search_TFLOP_s_per_gpu"], "peak": tf, "unit": "TFLOP/s",
+                     "frac": b4["search_TFLOP_s_per_gpu"] / tf,
+                     "peak_source": src + " (bf16 GEMM; fp16 has the same rate)", "traffic": None},
         "e2e": {"value": nq / b4["e2e_ms"] * 1e3, "unit": "queries/s", "h2d_bytes_per_step": nq * d * 4,
                 "d2h_bytes_per_step": nq * k * 12},
-        "gpu_launches": 4,
+        "gpu_launches": 4 + (1 if world > 1 else 0),
         "clocks": clocks.summary(),
     }
     if cpu is not None:

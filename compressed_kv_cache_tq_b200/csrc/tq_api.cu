@@ -102,4 +102,20 @@ tq_status tq_topk(const tq_ctx* ctx, const float* q, int64_t nq, const uint8_t* 
                                      static_cast<cudaStream_t>(stream)));
 }
 
+tq_status tq_topk_merge(const float* scores, const int64_t* ids, const int64_t* first_rows, int parts, int64_t nq,
+                        int k, int64_t* out_ids, float* out_scores, void* stream) {
+  if (parts < 1 || parts > tq::kMaxMergeParts || nq < 0 || k < 1) return TQ_ERR_ARG;
+  if (int64_t(parts) * k > tq::kMaxMergeCandidates) return TQ_ERR_UNSUPPORTED;
+  if (nq == 0) return TQ_OK;
+  if (!scores || !ids || !first_rows || !out_ids || !out_scores) return TQ_ERR_ARG;
+  if (!aligned(scores, 4) || !aligned(ids, 8) || !aligned(out_ids, 8) || !aligned(out_scores, 4)) return TQ_ERR_ARG;
+  tq::MergeOffsets off{};
+  for (int p = 0; p < parts; ++p) {
+    if (first_rows[p] < 0) return TQ_ERR_ARG;
+    off.first_row[p] = first_rows[p];
+  }
+  return cuda_status(tq::launch_topk_merge(scores, ids, off, nq, parts, k, out_ids, out_scores,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -99,6 +99,15 @@ cudaError_t launch_logits_simt(const tq_ctx* ctx, const float* q, int B, int Hq,
                                const uint8_t* payload, const uint16_t* norms, float scale, float* out,
                                ChannelGather gather, int accumulate, cudaStream_t st);
 
+// Merge of per-shard top-k lists (k_topk_merge.cu)
+constexpr int kMaxMergeParts = 64;
+constexpr int kMaxMergeCandidates = 4096;   // parts * k
+struct MergeOffsets {
+  int64_t first_row[kMaxMergeParts];
+};
+cudaError_t launch_topk_merge(const float* scores, const int64_t* ids, const MergeOffsets& off, int64_t nq, int parts,
+                              int k, int64_t* out_ids, float* out_scores, cudaStream_t st);
+
 // Value path (k_attend.cu)
 bool attend_supported(const tq_ctx* ctx, int Hq, int Hkv);
 size_t attend_ws_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int64_t S);

@@ -55,6 +55,7 @@ def lib() -> ctypes.CDLL:
             "tq_topk_workspace_bytes": (sz, [vp, i64, i64, i32]),
             "tq_topk": (i32, [vp, vp, i64, vp, vp, i64, i32, vp, vp, vp, sz, vp]),
             "tq_check_device_status": (i32, [vp, vp, ctypes.POINTER(u32)]),
+            "tq_topk_merge": (i32, [vp, vp, vp, i32, i64, i32, vp, vp, vp]),
             "tq_attend_workspace_bytes": (sz, [vp, i32, i32, i32, i64]),
             "tq_attend": (i32, [vp, vp, i32, i32, i32, i64, vp, vp, vp, vp, sz, vp]),
             "tq_split_create": (i32, [vp, vp, i32, ctypes.POINTER(vp)]),
@@ -79,7 +80,8 @@ def lib() -> ctypes.CDLL:
 
 EXPORTED = ["tq_init", "tq_init_ex", "tq_host_tables", "tq_free", "tq_info", "tq_export_tables", "tq_quantize", "tq_dequantize",
             "tq_logits_workspace_bytes", "tq_logits", "tq_logits_noalloc", "tq_topk_workspace_bytes", "tq_topk",
-            "tq_check_device_status", "tq_strerror", "tq_last_cuda_error", "tq_attend_workspace_bytes", "tq_attend",
+            "tq_check_device_status", "tq_strerror", "tq_last_cuda_error", "tq_topk_merge",
+            "tq_attend_workspace_bytes", "tq_attend",
             "tq_split_create", "tq_split_free",
             "tq_split_plan_workspace_bytes", "tq_split_plan", "tq_split_set_plan", "tq_split_get_plan",
             "tq_split_quantize", "tq_split_logits_workspace_bytes", "tq_split_logits"]
@@ -291,6 +293,28 @@ def tq_topk(ctx: Context, q: torch.Tensor, payload: torch.Tensor, norms: torch.T
     _check(lib().tq_topk(ctx.handle, _ptr(q), nq, _ptr(payload), _ptr(norms), n, k, _ptr(ids), _ptr(scores),
                          _ptr(workspace), workspace.numel(), ctypes.c_void_p(_stream(stream))), "tq_topk")
     return ids, scores
+
+
+def tq_topk_merge(scores: torch.Tensor, ids: torch.Tensor, first_rows, k: int, stream=None):
+    """scores fp32 / ids int64 [parts, nq, k] (shard-local ids), first_rows: one int per shard
+    -> (ids int64 (nq, k) global, scores fp32 (nq, k))."""
+    import numpy as np
+
+    _need_cuda(scores, "scores")
+    _need_cuda(ids, "ids")
+    if scores.dim() != 3 or scores.shape != ids.shape or scores.dtype != torch.float32 or ids.dtype != torch.int64:
+        raise ValueError("scores (fp32) and ids (int64) must both be (parts, nq, k)")
+    parts, nq, kk = scores.shape
+    fr = np.ascontiguousarray(np.asarray(first_rows, dtype=np.int64))
+    if fr.shape != (parts,):
+        raise ValueError("first_rows must hold one row offset per part")
+    out_ids = torch.empty((nq, k), dtype=torch.int64, device=scores.device)
+    out_sc = torch.empty((nq, k), dtype=torch.float32, device=scores.device)
+    if kk != k:
+        raise ValueError("each part must hold k candidates per query")
+    _check(lib().tq_topk_merge(_ptr(scores), _ptr(ids), fr.ctypes.data, parts, nq, k, _ptr(out_ids), _ptr(out_sc),
+                               ctypes.c_void_p(_stream(stream))), "tq_topk_merge")
+    return out_ids, out_sc
 
 
 def tq_check_device_status(ctx: Context, stream=None) -> int:

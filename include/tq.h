@@ -275,6 +275,21 @@ tq_status tq_split_logits(const tq_split* sp, const float* q, int B, int Hq, int
                           const uint16_t* norms_hi, const uint8_t* payload_lo, const uint16_t* norms_lo,
                           float scale, float* out, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Merge of per-shard top-k lists (a database split by rows over several
+ * devices or calls, each shard searched with tq_topk; airosetta.com "Google
+ * TurboQuant" on vector search): scores and ids are device arrays
+ * [parts][nq][k] as tq_topk returns them (ids local to their shard);
+ * first_rows (host, parts entries) gives each shard's first global row.  Per
+ * query, out_ids / out_scores (device [nq][k]) receive the k best candidates
+ * by score descending and global id ascending, ids made global.  Each shard
+ * must hold at least k rows.  1 <= parts <= 64, parts * k <= 4096
+ * (TQ_ERR_UNSUPPORTED above).  Candidates are ordered by their fp32 scores:
+ * two rows whose exact scores round to one fp32 value are ordered by id, which
+ * can differ from a single tq_topk call over the whole database only at such
+ * near-ties.  Needs no context. */
+tq_status tq_topk_merge(const float* scores, const int64_t* ids, const int64_t* first_rows, int parts, int64_t nq,
+                        int k, int64_t* out_ids, float* out_scores, void* stream);
+
 /* Read (and clear) the context's device status word after synchronising the
  * stream: 0 when every kernel finished its bounded waits, otherwise a bit set
  * per kernel that gave up.  Returns TQ_ERR_DEVICE when nonzero. */
