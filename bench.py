@@ -429,10 +429,10 @@ def run_reference(args, rank):
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per key of the
 # current kernels, from one ncu capture at S = 16384 (1 048 576 keys); per
-# launch it scales with the keys processed.  Summaries: profiles/quantize_tc_decode_s16384.md
-# and profiles/logits_mma_decode_s16384.md.  Set to None when a kernel changes.
-DRAM_BYTES_PER_KEY = {"decode": {"tq_quantize": (268.648960e6 + 53.591040e6) / 1048576,
-                                  "tq_logits": (71.457024e6 + 3.751168e6) / 1048576}}
+# launch it scales with the keys processed.  Summary with the command:
+# profiles/traffic_decode_s16384.md.  Set to None when a kernel changes.
+DRAM_BYTES_PER_KEY = {"decode": {"tq_quantize": (268.711424e6 + 50.201600e6) / 1048576,
+                                  "tq_logits": (71.455744e6 + 0.465664e6) / 1048576}}
 
 
 def max_over_ranks(x: float, dist, device) -> float:
