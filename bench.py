@@ -435,6 +435,37 @@ DRAM_BYTES_PER_KEY = {"decode": {"tq_quantize": (268.711424e6 + 50.201600e6) / 1
                                   "tq_logits": (71.455744e6 + 0.465664e6) / 1048576}}
 
 
+def dense_logits_context(keys4, q, reps: int = 20) -> dict:
+    """Context for the pages' comparison of 4-bit logits with 32-bit ones: the
+    same logits as a dense torch matmul (cuBLAS) of the queries with the
+    unquantised keys, in fp32 and bf16, timed with CUDA events like the
+    kernels.  Not part of the path; any failure only drops the field."""
+    import torch
+
+    res = {"what": "torch.matmul(q, K^T) over unquantised keys [B, Hkv, S, d] per GQA group (cuBLAS), "
+                   "keys larger than L2"}
+    try:
+        Bk, Hk, Sk, Dk = keys4.shape
+        G = q.shape[1] // Hk
+        for name, dt in (("fp32", torch.float32), ("bf16", torch.bfloat16)):
+            K = keys4.to(dt)
+            qq = q.to(dt).reshape(Bk, Hk, G, Dk)
+            for _ in range(3):
+                torch.matmul(qq, K.transpose(-1, -2))
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for _ in range(reps):
+                torch.matmul(qq, K.transpose(-1, -2))
+            b.record()
+            torch.cuda.synchronize()
+            res[f"{name}_ms"] = a.elapsed_time(b) / reps
+            del K, qq
+    except Exception as e:   # context only
+        res["error"] = type(e).__name__
+    return res
+
+
 def max_over_ranks(x: float, dist, device) -> float:
     """The largest value of x over all ranks (x itself without a process group)."""
     if dist is None:
@@ -710,6 +741,12 @@ def main():
                        d2h=int((o_att if ATTEND else out).numel() * 4),
                        clocks=clocks.summary())
     line.update(extra)
+    if world == 1:
+        ctx_d = dense_logits_context(keys4, q)
+        for name in ("fp32", "bf16"):
+            if f"{name}_ms" in ctx_d:
+                ctx_d[f"logits_speedup_vs_{name}"] = ctx_d[f"{name}_ms"] / l_ms
+        line["context_dense_logits"] = ctx_d
     if not args.no_cpu_baseline and world == 1:
         line["cpu_baseline"] = cpu_baseline()
     print(json.dumps(line), flush=True)
