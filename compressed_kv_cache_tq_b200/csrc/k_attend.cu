@@ -12,16 +12,20 @@
 //   b = sum_s w_s rho16_s sigma_s  (sign domain, m).
 // The rotations are applied once per head, after the sums, not once per key.
 //
-// Kernel 1 (attend_partial_kernel): one block per (batch, KV head, key chunk)
-// computes, for every query head of the group, the chunk's maximum logit, the
-// sum of its weights and its a, b (flash-decoding style partials).  Key tiles
-// of 64 rows are staged in shared memory (prefetched into registers one tile
-// ahead); warp w takes the key pairs (k, k + 64) for k = w, w + 8, ...; lane
-// L decodes one "slot" of the packed layout of both keys (4 coordinates:
-// register r = 4u + i of quarter q, nibbles e = 0..3) and accumulates each
-// head with packed two-wide FMAs over the key pair.
-// Kernel 2 (attend_combine_kernel): one block per query head merges the
-// partials and applies P^T and R^T.
+// Partial sums: one block per (batch, KV head, key chunk) computes, for every
+// query head of the group, the chunk's maximum logit, the sum of its weights
+// and its a, b (flash-decoding style partials), by one of two kernels:
+//   attend_mma_kernel (d = m = 128 or m = 0, up to 4 query heads per KV
+//     head): fp16 tensor-core MMAs over 16-key steps, described above the
+//     kernel;
+//   attend_partial_kernel (every other shape): key tiles of 128 rows staged
+//     in shared memory (prefetched into registers one tile ahead); warp w
+//     takes the key pairs (k, k + 64) for k = w, w + 8, ...; lane L decodes
+//     one "slot" of the packed layout of both keys (4 coordinates: register
+//     r = 4u + i of quarter q, nibbles e = 0..3) and accumulates each head
+//     with packed two-wide FMAs over the key pair.
+// attend_combine_kernel: one block per query head merges the partials and
+// applies P^T and R^T.
 #include <cuda_fp16.h>
 #include <math.h>
 
