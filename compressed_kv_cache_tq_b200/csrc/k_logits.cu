@@ -4,7 +4,10 @@
 // for every (query head, key) of a GQA decode step.  The work is HBM bound
 // (mooersco.com section 2.2): 4 query heads share each key of a KV head.
 //
-// Fast path (d = m = 128, b' = 1..3, this file's logits_mma_kernel):
+// Fast path (d = 128, m = 128 or 0, b' = 1..3, this file's logits_mma_kernel;
+// with m = 0, the MSE-only variant, the sign term and its MMAs are dropped;
+// logits_split_kernel applies the same scheme to the two 64-channel groups of
+// a channel split):
 //   * one warp streams 16-key tiles; thread (g, tig) loads chunk tig of keys
 //     g and g + 8 with coalesced 32/128-bit loads (the packed layout puts a
 //     quarter of every key's codes and signs in one contiguous chunk);

@@ -1,4 +1,8 @@
-// Tensor-core quantize kernel for d = m = 128 and bf16 keys (sm_100a).
+// Tensor-core quantize kernels for bf16 keys of d = 128 (sm_100a):
+//   quantize_tc_kernel<b', JL>   one context, m = 128 (JL) or m = 0 (the
+//                                MSE-only variant: no JL product, no signs);
+//   quantize_split_tc_kernel     the per-KV-head channel split into two
+//                                64-channel groups (described further down).
 //
 // What it computes per key k (airosetta.com "Google TurboQuant", stage 1 and
 // stage 2; mooersco.com section 1.1 "rotated = key @ rotation"):
@@ -34,6 +38,9 @@
 // slot; the epilogue reads it and writes the residual's fp16 hi / lo pairs
 // back over it (A operand of the JL product, read by the MMA from TMEM); z
 // accumulates in columns 128..255.
+// Without the sketch (m = 0) P is not loaded, there is no JL product, and a
+// TMEM slot's y columns are released to the next rotation as soon as the
+// epilogue has read them.
 // Every wait on an mbarrier is bounded; a wait that gives up sets the
 // context's status word, and all roles then leave their loops (there is no
 // unbounded barrier between roles).
