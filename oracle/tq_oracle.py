@@ -11,7 +11,7 @@ What it computes, step by step, and where the pages say so:
 * Random rotation R: QR factorisation of a seeded Gaussian matrix
   (airosetta.com "Google TurboQuant", section "第一階段：PolarQuant").
   The pages give no generator, no sign rule and no Q-vs-Q^T choice; the
-  readings used here are listed on each function and in the design doc.
+  readings used here are listed on each function.
 * Coordinate law of a rotated unit vector: a Beta-type law on [-1, 1]
   with density proportional to (1 - x^2)^((d-3)/2) (same section: the
   coordinates "follow a known, concentrated Beta distribution").
@@ -723,7 +723,7 @@ def pack_norms(n16: np.ndarray, rho16: np.ndarray) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
-# Parity bands (readings of the benchmark spec's tolerance)
+# Parity bands (the readings of the stated tolerances that the parity tests apply)
 # ---------------------------------------------------------------------------
 
 CODE_BAND = 1e-5     # |u_j - t_i| on the unit-sphere scale

@@ -1,5 +1,5 @@
 """Comparison helpers: GPU outputs against the oracle, with the bands the
-spec tolerance allows (readings listed in the design doc)."""
+stated tolerances allow (each band's reading is on its constant in oracle/tq_oracle.py)."""
 
 from __future__ import annotations
 
