@@ -56,7 +56,8 @@ def check_quantize(payload, norms, K64, tb: O.Tables, report=None):
     nr_ok = norm_ok(norms[:, 1], qz.rho, key_exc)
     assert nr_ok.all(), f"||r|| differs: {np.argwhere(~nr_ok)[:5].ravel()}"
     stats = dict(code_mismatch=float(frac_code), sign_mismatch=float(frac_sign),
-                 code_near_boundary=float(code_band.mean()), sign_near_boundary=float(sign_band.mean()),
+                 code_near_boundary=float(code_band.mean()) if code_band.size else 0.0,
+                 sign_near_boundary=float(sign_band.mean()) if sign_band.size else 0.0,   # m = 0: no sign bits
                  keys=int(len(qz.n)))
     if report is not None:
         report.update(stats)
