@@ -81,6 +81,33 @@ def test_argument_validation_without_device(L):
     assert lib.tq_split_quantize(None, None, 1, 1, 1, None, None, None, None, None) == 1
     assert lib.tq_split_logits(None, None, 1, 4, 1, None, None, None, None, 1.0, None, None, 0, None) == 1
     lib.tq_split_free(None)
+    # value path
+    assert lib.tq_attend_workspace_bytes(None, 1, 8, 2, 64) == 0
+    assert lib.tq_attend(None, None, 1, 8, 2, 64, None, None, None, None, 0, None) == 1
+
+
+def test_topk_merge_validation_without_device(L):
+    """tq_topk_merge refuses bad counts, pointers and shard offsets on the
+    host; nothing is dereferenced on the device before these checks pass
+    (the fake device addresses below are never touched)."""
+    lib = L.lib()
+    dev = ctypes.c_void_p(1 << 20)           # aligned, never dereferenced
+    odd = ctypes.c_void_p((1 << 20) + 2)     # misaligned for 4- and 8-byte elements
+    first = (ctypes.c_int64 * 64)(*range(0, 6400, 100))
+    fp = ctypes.cast(first, ctypes.c_void_p)
+    assert lib.tq_topk_merge(dev, dev, fp, 0, 4, 10, dev, dev, None) == 1          # no parts
+    assert lib.tq_topk_merge(dev, dev, fp, 65, 4, 10, dev, dev, None) == 1         # more than 64 parts
+    assert lib.tq_topk_merge(dev, dev, fp, 2, -1, 10, dev, dev, None) == 1         # negative query count
+    assert lib.tq_topk_merge(dev, dev, fp, 2, 4, 0, dev, dev, None) == 1           # k = 0
+    assert lib.tq_topk_merge(dev, dev, fp, 64, 4, 65, dev, dev, None) == 2         # 4160 candidates > 4096
+    assert lib.tq_topk_merge(None, None, None, 2, 0, 10, None, None, None) == 0    # no queries: nothing to do
+    assert lib.tq_topk_merge(None, dev, fp, 2, 4, 10, dev, dev, None) == 1         # null scores
+    assert lib.tq_topk_merge(dev, dev, None, 2, 4, 10, dev, dev, None) == 1        # null offsets
+    assert lib.tq_topk_merge(odd, dev, fp, 2, 4, 10, dev, dev, None) == 1          # scores misaligned
+    assert lib.tq_topk_merge(dev, odd, fp, 2, 4, 10, dev, dev, None) == 1          # ids misaligned
+    assert lib.tq_topk_merge(dev, dev, fp, 2, 4, 10, odd, dev, None) == 1          # out ids misaligned
+    first[1] = -5
+    assert lib.tq_topk_merge(dev, dev, fp, 2, 4, 10, dev, dev, None) == 1          # negative first row
 
 
 def test_row_bytes_formula():
