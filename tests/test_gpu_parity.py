@@ -260,6 +260,67 @@ def test_topk_many_query_tiles(lib, d, bits):
     np.testing.assert_allclose(scores.cpu().numpy(), np.take_along_axis(s, ids, 1), rtol=1e-6, atol=1e-6 * A.max())
 
 
+def _oracle_scores_chunked(payload, norms, Q64, tb: O.Tables, chunk: int = 131072):
+    """Oracle estimates (and abs-term sums) of every (query, row) pair, taken
+    over row chunks so that host memory stays bounded at 10^6 rows."""
+    n = payload.shape[0]
+    s = np.empty((Q64.shape[0], n))
+    A = np.empty_like(s)
+    for r0 in range(0, n, chunk):
+        r1 = min(n, r0 + chunk)
+        s[:, r0:r1], A[:, r0:r1] = oracle_estimates(payload[r0:r1], norms[r0:r1], Q64, tb)
+    return s, A
+
+
+def _oracle_topk_order(si: np.ndarray, k: int) -> np.ndarray:
+    """The oracle's first k + 1 rows of one query: score descending, ties to the lower id."""
+    n = si.shape[0]
+    if n <= k + 1:
+        cand = np.arange(n)
+    else:
+        thr = np.partition(si, n - (k + 1))[n - (k + 1)]
+        cand = np.nonzero(si >= thr)[0]
+    return cand[np.lexsort((cand, -si[cand]))][:k + 1]
+
+
+def _search_sampled(lib, n, nq, bits, k=10, d=200, n_sample=8, chunk=131072, max_near_tie=2):
+    ctx = _ctx(lib, d=d, bits=bits, seed=42)
+    db = W.search_vectors(n, d, seed=1004, which=0)
+    qs = W.search_vectors(nq, d, seed=1004, which=1)
+    payload, norms = lib.tq_quantize(ctx, torch.from_numpy(db).to(DEV))
+    ids, scores = lib.tq_topk(ctx, torch.from_numpy(qs).to(DEV), payload, norms, k)
+    _status_clean(lib, ctx)
+    tb = tables_of(ctx)
+    pay, nrm = payload.cpu().numpy(), norms.cpu().numpy()
+    rng = np.random.default_rng(100 + bits)
+    rows = np.sort(rng.choice(n, min(n, 2000), replace=False))
+    rows[-1] = n - 1
+    check_quantize(pay[rows], nrm[rows], db[rows].astype(np.float64), tb)
+    sample = np.concatenate([[0, nq - 1], rng.choice(np.arange(1, nq - 1), n_sample - 2, replace=False)])
+    s, A = _oracle_scores_chunked(pay, nrm, qs[sample].astype(np.float64), tb, chunk)
+    got_ids, got_scores = ids.cpu().numpy()[sample], scores.cpu().numpy()[sample]
+    near_tie = 0
+    for i in range(len(sample)):
+        order = _oracle_topk_order(s[i], k)
+        if k < n and s[i, order[k - 1]] - s[i, order[k]] < 1e-6 * A[i].max():
+            near_tie += 1
+            assert set(got_ids[i][:k - 1]) <= set(order)
+            continue
+        np.testing.assert_array_equal(got_ids[i], order[:k])
+    assert near_tie <= max_near_tie
+    np.testing.assert_allclose(got_scores, np.take_along_axis(s, got_ids, 1), rtol=1e-6, atol=1e-6 * A.max())
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_search_full_size_sampled(lib, bits):
+    """The search workload in the launch configuration bench.py times: 10^6
+    unit vectors in d = 200 indexed, 10^4 queries, k = 10, tables seed 42.
+    2000 sampled rows of the index against the oracle's quantisation, and the
+    answers of eight queries (the first, the last, six seeded) against the
+    oracle's top-k over all 10^6 rows."""
+    _search_sampled(lib, 1_000_000, 10_000, bits)
+
+
 def test_topk_identical_rows_take_lowest_ids(lib):
     """3000 copies of one vector: every row ties, the candidate list overflows
     and the exact scan returns ids 0 .. k-1 (ties go to the lower id)."""
@@ -290,10 +351,12 @@ def test_logits_rejects_bad_workspace(lib):
 # --------------------------------------------------------------------------
 
 
-@pytest.mark.parametrize("name,B,Hkv,G,S,bits", [("decode", 8, 8, 4, 32768, 4), ("longctx", 1, 8, 4, 131072, 3)])
-def test_full_size_sampled(lib, name, B, Hkv, G, S, bits):
-    seed = 1001 if name == "decode" else 1002
-    ctx = _ctx(lib, bits=bits, seed=42)
+@pytest.mark.parametrize("name,B,Hkv,G,S,bits,m", [("decode", 8, 8, 4, 32768, 4, 128),
+                                                   ("longctx", 1, 8, 4, 131072, 3, 128),
+                                                   ("decode_mse_only", 8, 8, 4, 32768, 4, 0)])
+def test_full_size_sampled(lib, name, B, Hkv, G, S, bits, m):
+    seed = 1002 if name == "longctx" else 1001
+    ctx = _ctx(lib, bits=bits, seed=42, m=m)
     keys = W.decode_keys(B, Hkv, S, 128, seed, device=DEV).reshape(-1, 128)
     payload, norms = lib.tq_quantize(ctx, keys)
     Hq = Hkv * G
