@@ -97,6 +97,7 @@ tq_status tq_topk(const tq_ctx* ctx, const float* q, int64_t nq, const uint8_t* 
   if (k < 1 || k > 256 || k > n) return TQ_ERR_ARG;
   if (!q || !payload || !norms || !ids || !scores || !workspace) return TQ_ERR_ARG;
   if (!aligned(payload, 16) || !aligned(norms, 4) || !aligned(workspace, 256)) return TQ_ERR_ARG;
+  if (!aligned(q, 4) || !aligned(ids, 8) || !aligned(scores, 4)) return TQ_ERR_ARG;
   if (workspace_bytes < tq_topk_workspace_bytes(ctx, nq, n, k)) return TQ_ERR_WORKSPACE;
   return cuda_status(tq::launch_topk(ctx, q, nq, payload, norms, n, k, ids, scores, workspace,
                                      static_cast<cudaStream_t>(stream)));

@@ -111,6 +111,35 @@ def _need_cuda(t: torch.Tensor, name: str):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _need_tensor(t, name: str, dtype: torch.dtype, shape: tuple, device=None):
+    """t must be a contiguous tensor of `dtype` with `shape` (a None entry
+    matches any size), on `device` when one is given.  The C ABI receives bare
+    pointers and derives every extent from the sizes passed beside them, so a
+    buffer that disagrees with them would be read or written out of bounds:
+    it is refused here, before any launch."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != len(shape) or any(w is not None and g != w for g, w in zip(t.shape, shape)):
+        want = "(" + ", ".join("*" if w is None else str(w) for w in shape) + ")"
+        raise ValueError(f"{name} must have shape {want}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+
+
+def _need_rows(ctx, payload, norms, rows, device, suffix=""):
+    """Packed rows of ctx's layout: payload uint8 (rows, row_bytes), norms fp16 (rows, 2)."""
+    _need_tensor(payload, "payload" + suffix, torch.uint8, (rows, ctx.row_bytes), device)
+    _need_tensor(norms, "norms" + suffix, torch.float16, (payload.shape[0], 2), device)
+
+
+def _need_workspace(ws, device):
+    _need_tensor(ws, "workspace", torch.uint8, (None,), device)
+
+
 class Context:
     """A quantizer: R, S, codebook for (d, bits, m, seed) on the current device."""
 
@@ -188,6 +217,7 @@ def tq_quantize(ctx: Context, keys: torch.Tensor, payload: torch.Tensor | None =
         payload = torch.empty((n, ctx.row_bytes), dtype=torch.uint8, device=keys.device)
     if norms is None:
         norms = torch.empty((n, 2), dtype=torch.float16, device=keys.device)
+    _need_rows(ctx, payload, norms, n, keys.device)
     _check(lib().tq_quantize(ctx.handle, _ptr(keys), dtype, n, keys.stride(0), _ptr(payload), _ptr(norms),
                              ctypes.c_void_p(_stream(stream))), "tq_quantize")
     return payload, norms
@@ -196,10 +226,11 @@ def tq_quantize(ctx: Context, keys: torch.Tensor, payload: torch.Tensor | None =
 def tq_dequantize(ctx: Context, payload: torch.Tensor, norms: torch.Tensor, full: bool = True,
                   out: torch.Tensor | None = None, stream=None):
     _need_cuda(payload, "payload")
-    _need_cuda(norms, "norms")
+    _need_rows(ctx, payload, norms, None, payload.device)
     n = payload.shape[0]
     if out is None:
         out = torch.empty((n, ctx.d), dtype=torch.float32, device=payload.device)
+    _need_tensor(out, "out", torch.float32, (n, ctx.d), payload.device)
     _check(lib().tq_dequantize(ctx.handle, _ptr(payload), _ptr(norms), n, int(full), _ptr(out),
                                ctypes.c_void_p(_stream(stream))), "tq_dequantize")
     return out
@@ -222,11 +253,14 @@ def tq_logits(ctx: Context, q: torch.Tensor, payload: torch.Tensor, norms: torch
     if payload.shape[0] % (B * Hkv):
         raise ValueError("payload rows must be B * Hkv * S")
     S = payload.shape[0] // (B * Hkv)
+    _need_rows(ctx, payload, norms, None, q.device)
     if out is None:
         out = torch.empty((B, Hq, S), dtype=torch.float32, device=q.device)
+    _need_tensor(out, "out", torch.float32, (B, Hq, S), q.device)
     ws_bytes = tq_logits_workspace_bytes(ctx, B, Hq, Hkv)
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=q.device)
+    _need_workspace(workspace, q.device)
     _check(lib().tq_logits(ctx.handle, _ptr(q), B, Hq, Hkv, S, _ptr(payload), _ptr(norms), float(scale), _ptr(out),
                            _ptr(workspace), workspace.numel(), ctypes.c_void_p(_stream(stream))), "tq_logits")
     return out
@@ -241,9 +275,13 @@ def tq_logits_noalloc(ctx: Context, q: torch.Tensor, payload: torch.Tensor, norm
     if q.dtype != torch.float32 or q.dim() != 3 or q.shape[2] != ctx.d:
         raise ValueError("q must be float32 (B, Hq, d)")
     B, Hq, _ = q.shape
+    if Hkv < 1 or B * Hkv == 0 or payload.shape[0] % (B * Hkv):
+        raise ValueError("payload rows must be B * Hkv * S")
     S = payload.shape[0] // (B * Hkv)
+    _need_rows(ctx, payload, norms, None, q.device)
     if out is None:
         out = torch.empty((B, Hq, S), dtype=torch.float32, device=q.device)
+    _need_tensor(out, "out", torch.float32, (B, Hq, S), q.device)
     _check(lib().tq_logits_noalloc(ctx.handle, _ptr(q), B, Hq, Hkv, S, _ptr(payload), _ptr(norms), float(scale),
                                    _ptr(out), ctypes.c_void_p(_stream(stream))), "tq_logits_noalloc")
     return out
@@ -264,11 +302,14 @@ def tq_attend(ctx: Context, logits: torch.Tensor, payload: torch.Tensor, norms: 
     B, Hq, S = logits.shape
     if payload.shape[0] != B * Hkv * S:
         raise ValueError("payload rows must be B * Hkv * S")
+    _need_rows(ctx, payload, norms, B * Hkv * S, logits.device)
     if out is None:
         out = torch.empty((B, Hq, ctx.d), dtype=torch.float32, device=logits.device)
+    _need_tensor(out, "out", torch.float32, (B, Hq, ctx.d), logits.device)
     ws_bytes = tq_attend_workspace_bytes(ctx, B, Hq, Hkv, S)
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=logits.device)
+    _need_workspace(workspace, logits.device)
     _check(lib().tq_attend(ctx.handle, _ptr(logits), B, Hq, Hkv, S, _ptr(payload), _ptr(norms), _ptr(out),
                            _ptr(workspace), workspace.numel(), ctypes.c_void_p(_stream(stream))), "tq_attend")
     return out
@@ -284,12 +325,15 @@ def tq_topk(ctx: Context, q: torch.Tensor, payload: torch.Tensor, norms: torch.T
     _need_cuda(q, "q")
     _need_cuda(payload, "payload")
     _need_cuda(norms, "norms")
+    _need_tensor(q, "q", torch.float32, (None, ctx.d), q.device)
+    _need_rows(ctx, payload, norms, None, q.device)
     nq, n = q.shape[0], payload.shape[0]
     ids = torch.empty((nq, k), dtype=torch.int64, device=q.device)
     scores = torch.empty((nq, k), dtype=torch.float32, device=q.device)
     ws_bytes = tq_topk_workspace_bytes(ctx, nq, n, k)
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=q.device)
+    _need_workspace(workspace, q.device)
     _check(lib().tq_topk(ctx.handle, _ptr(q), nq, _ptr(payload), _ptr(norms), n, k, _ptr(ids), _ptr(scores),
                          _ptr(workspace), workspace.numel(), ctypes.c_void_p(_stream(stream))), "tq_topk")
     return ids, scores
@@ -304,6 +348,8 @@ def tq_topk_merge(scores: torch.Tensor, ids: torch.Tensor, first_rows, k: int, s
     _need_cuda(ids, "ids")
     if scores.dim() != 3 or scores.shape != ids.shape or scores.dtype != torch.float32 or ids.dtype != torch.int64:
         raise ValueError("scores (fp32) and ids (int64) must both be (parts, nq, k)")
+    if ids.device != scores.device:
+        raise ValueError("scores and ids must be on the same device")
     parts, nq, kk = scores.shape
     fr = np.ascontiguousarray(np.asarray(first_rows, dtype=np.int64))
     if fr.shape != (parts,):
@@ -349,6 +395,7 @@ class Split:
         ws_bytes = int(lib().tq_split_plan_workspace_bytes(self._h))
         if workspace is None:
             workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=keys.device)
+        _need_workspace(workspace, keys.device)
         _check(lib().tq_split_plan(self._h, _ptr(keys), dtype, keys.shape[0], keys.shape[2], _ptr(workspace),
                                    workspace.numel(), ctypes.c_void_p(_stream(stream))), "tq_split_plan")
 
@@ -403,6 +450,8 @@ def tq_split_quantize(sp: Split, keys: torch.Tensor, payload_hi=None, norms_hi=N
         payload_lo = torch.empty((n, sp.lo.row_bytes), dtype=torch.uint8, device=dev)
     if norms_lo is None:
         norms_lo = torch.empty((n, 2), dtype=torch.float16, device=dev)
+    _need_rows(sp.hi, payload_hi, norms_hi, n, dev, "_hi")
+    _need_rows(sp.lo, payload_lo, norms_lo, n, dev, "_lo")
     _check(lib().tq_split_quantize(sp.handle, _ptr(keys), dtype, B, S, _ptr(payload_hi), _ptr(norms_hi),
                                    _ptr(payload_lo), _ptr(norms_lo), ctypes.c_void_p(_stream(stream))),
            "tq_split_quantize")
@@ -422,11 +471,15 @@ def tq_split_logits(sp: Split, q: torch.Tensor, payload_hi, norms_hi, payload_lo
     if payload_hi.shape[0] % (B * sp.Hkv) or payload_lo.shape[0] != payload_hi.shape[0]:
         raise ValueError("payload rows must be B * Hkv * S")
     S = payload_hi.shape[0] // (B * sp.Hkv)
+    _need_rows(sp.hi, payload_hi, norms_hi, None, q.device, "_hi")
+    _need_rows(sp.lo, payload_lo, norms_lo, payload_hi.shape[0], q.device, "_lo")
     if out is None:
         out = torch.empty((B, Hq, S), dtype=torch.float32, device=q.device)
+    _need_tensor(out, "out", torch.float32, (B, Hq, S), q.device)
     ws_bytes = int(lib().tq_split_logits_workspace_bytes(sp.handle, B, Hq))
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=q.device)
+    _need_workspace(workspace, q.device)
     _check(lib().tq_split_logits(sp.handle, _ptr(q), B, Hq, S, _ptr(payload_hi), _ptr(norms_hi), _ptr(payload_lo),
                                  _ptr(norms_lo), float(scale), _ptr(out), _ptr(workspace), workspace.numel(),
                                  ctypes.c_void_p(_stream(stream))), "tq_split_logits")

@@ -199,7 +199,10 @@ size_t tq_topk_workspace_bytes(const tq_ctx* ctx, int64_t nq, int64_t n, int k);
  * score descending and id ascending on ties.  Candidates are selected with
  * the fast estimator and re-scored in fp64 before the final order.
  * q: device fp32 [nq, d]; ids: device int64 [nq, k]; scores: device fp32
- * [nq, k].  1 <= k <= 256, k <= n. */
+ * [nq, k].  1 <= k <= 256, k <= n.
+ * Errors: TQ_ERR_ARG (a null or misaligned pointer: payload 16 bytes, norms,
+ * q and scores 4, ids 8, workspace 256; k out of range); TQ_ERR_WORKSPACE
+ * when workspace_bytes < tq_topk_workspace_bytes; TQ_ERR_CUDA. */
 tq_status tq_topk(const tq_ctx* ctx, const float* q, int64_t nq, const uint8_t* payload,
                   const uint16_t* norms, int64_t n, int k, int64_t* ids, float* scores,
                   void* workspace, size_t workspace_bytes, void* stream);

@@ -117,3 +117,41 @@ def test_row_bytes_formula():
     for d, m, b in [(200, 200, 1), (200, 200, 3), (72, 136, 2)]:
         dp, mp = -(-d // 64) * 64, -(-m // 64) * 64
         assert O.row_bytes(d, m, b) == dp * b // 8 + mp // 8
+
+
+def test_binding_refuses_buffers_that_disagree_with_the_sizes(L):
+    """The binding checks dtype, shape, contiguity and device of every buffer
+    before it hands bare pointers to the C ABI (CPU tensors stand in here)."""
+    import types
+
+    import torch
+
+    ctx = types.SimpleNamespace(row_bytes=64, d=128)
+    pay = torch.zeros((10, 64), dtype=torch.uint8)
+    nrm = torch.zeros((10, 2), dtype=torch.float16)
+    L._need_rows(ctx, pay, nrm, 10, pay.device)
+    L._need_rows(ctx, pay, nrm, None, None)
+    bad = [
+        (torch.zeros((9, 64), dtype=torch.uint8), nrm, 10),           # fewer rows than keys
+        (torch.zeros((10, 48), dtype=torch.uint8), nrm, 10),          # another layout's row size
+        (torch.zeros((10, 64), dtype=torch.int8), nrm, 10),           # wrong dtype
+        (torch.zeros((640,), dtype=torch.uint8), nrm, 10),            # flat
+        (torch.zeros((64, 10), dtype=torch.uint8).t(), nrm, 10),      # not contiguous
+        (pay, torch.zeros((10, 2), dtype=torch.float32), 10),         # norms not fp16
+        (pay, torch.zeros((9, 2), dtype=torch.float16), None),        # norms for fewer rows
+        (pay, torch.zeros((20,), dtype=torch.float16), None),         # norms flat
+    ]
+    for p, n_, rows in bad:
+        with pytest.raises(ValueError):
+            L._need_rows(ctx, p, n_, rows, None)
+    with pytest.raises(ValueError):
+        L._need_rows(ctx, pay, nrm, 10, torch.device("meta"))         # another device
+    with pytest.raises(TypeError):
+        L._need_tensor(None, "out", torch.float32, (1,))
+    L._need_tensor(torch.zeros((2, 8, 5)), "out", torch.float32, (2, 8, 5))
+    with pytest.raises(ValueError):
+        L._need_tensor(torch.zeros((2, 8, 4)), "out", torch.float32, (2, 8, 5))
+    L._need_workspace(torch.zeros(300, dtype=torch.uint8), None)
+    for ws in (torch.zeros(300, dtype=torch.float32), torch.zeros((2, 150), dtype=torch.uint8)):
+        with pytest.raises(ValueError):
+            L._need_workspace(ws, None)
