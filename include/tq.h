@@ -90,12 +90,15 @@ tq_status tq_init(int d, int bits, uint64_t seed, tq_ctx** out);
  * first Philox stream used (G from stream_base, P from stream_base + 1).
  * m = 0 selects the MSE-only variant ([p2] stage 1 alone): the same rotation
  * and codebook, no sign sketch (rows hold only the b' = bits - 1 code bits),
- * and the estimator is its first term n16 sum_j c[idx_j] (Rq)_j. */
+ * and the estimator is its first term n16 sum_j c[idx_j] (Rq)_j.
+ * Errors: as tq_init; TQ_ERR_UNSUPPORTED also for m outside {0} u [64, 256]
+ * or not a multiple of 8. */
 tq_status tq_init_ex(int d, int bits, int m, uint64_t seed, uint32_t stream_base, tq_ctx** out);
 
 /* Host only, no GPU needed: the fp64 tables tq_init_ex builds for these
  * arguments (R d*d, P m*d, c 2^(bits-1), t 2^(bits-1)-1; host pointers, any
- * may be NULL).  Same validation as tq_init_ex. */
+ * may be NULL).  Errors: TQ_ERR_UNSUPPORTED for the shapes tq_init_ex
+ * refuses. */
 tq_status tq_host_tables(int d, int bits, int m, uint64_t seed, uint32_t stream_base, double* R, double* P,
                          double* c, double* t);
 
@@ -103,13 +106,13 @@ tq_status tq_host_tables(int d, int bits, int m, uint64_t seed, uint32_t stream_
 void tq_free(tq_ctx* ctx);
 
 /* Sizes: d, bits, m and the packed payload bytes per key (host out-params,
- * any may be NULL). */
+ * any may be NULL).  Errors: TQ_ERR_ARG (ctx == NULL). */
 tq_status tq_info(const tq_ctx* ctx, int* d, int* bits, int* m, int* row_bytes);
 
 /* Copy the fp64 master tables to host memory for inspection: R (d*d,
  * row-major), P (m*d), codebook levels c (2^(bits-1)) and boundaries t
  * (2^(bits-1) - 1), ascending, on the unit-sphere scale.  Host pointers;
- * any may be NULL. */
+ * any may be NULL.  Errors: TQ_ERR_ARG (ctx == NULL). */
 tq_status tq_export_tables(const tq_ctx* ctx, double* R, double* P, double* c, double* t);
 
 /* Quantise n keys ([p2] stages 1 and 2): per key k (row i of `keys`, leading
@@ -119,18 +122,24 @@ tq_status tq_export_tables(const tq_ctx* ctx, double* R, double* P, double* c, d
  * layout.  keys: device, dtype TQ_F32 or TQ_BF16, 16-byte aligned, ld >= d and
  * ld a multiple of 8.  payload: device, n * row_bytes bytes.  norms: device,
  * n * 2 fp16 values.  A zero key gets codes 0, all sign bits 1, norms 0.
- * n == 0 is a no-op. */
+ * n == 0 is a no-op.
+ * Errors: TQ_ERR_ARG (ctx NULL; n < 0; a NULL buffer; dtype; ld < d or not a
+ * multiple of 8; keys or payload not 16-byte aligned, norms not 4-byte
+ * aligned); TQ_ERR_CUDA. */
 tq_status tq_quantize(const tq_ctx* ctx, const void* keys, tq_dtype dtype, int64_t n, int64_t ld,
                       uint8_t* payload, uint16_t* norms, void* stream);
 
 /* Reconstruct n keys from the packed layout ([p2] stage 1: look up the
  * codebook and rotate back): out[i] = n16 R^T c[idx] when full == 0, plus the
  * QJL term sqrt(pi/2)/m rho16 S^T sigma when full != 0 (then <q, out[i]>
- * equals the inner-product estimate).  out: device fp32, n * d. */
+ * equals the inner-product estimate).  out: device fp32, n * d.
+ * Errors: TQ_ERR_ARG (ctx NULL; n < 0; a NULL buffer; payload or norms not
+ * 2-byte aligned, out not 4-byte aligned); TQ_ERR_CUDA. */
 tq_status tq_dequantize(const tq_ctx* ctx, const uint8_t* payload, const uint16_t* norms, int64_t n,
                         int full, float* out, void* stream);
 
-/* Workspace bytes tq_logits needs for B*Hq query heads (prepared queries). */
+/* Workspace bytes tq_logits needs for B*Hq query heads (prepared queries);
+ * 0 for invalid arguments (ctx NULL, a size <= 0, Hq not a multiple of Hkv). */
 size_t tq_logits_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv);
 
 /* Decode attention logits against a packed KV cache ([p2] stage 2
@@ -140,7 +149,12 @@ size_t tq_logits_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv);
  * for q = q[b, h], key row (b, h / (Hq/Hkv), s).
  * q: device fp32 [B, Hq, d].  payload/norms: device, rows [B, Hkv, S].
  * out: device fp32 [B, Hq, S].  Hq must be a multiple of Hkv.
- * workspace: device, >= tq_logits_workspace_bytes, 256-byte aligned. */
+ * workspace: device, >= tq_logits_workspace_bytes, 256-byte aligned.
+ * B = 0 or Hq = 0 is a no-op.
+ * Errors: TQ_ERR_ARG (ctx NULL; a negative size; Hkv = 0 or Hq not a
+ * multiple of Hkv; a NULL buffer; payload not 16-byte aligned, norms, q or
+ * out not 4-byte aligned; workspace NULL or misaligned); TQ_ERR_WORKSPACE
+ * (workspace_bytes too small); TQ_ERR_CUDA. */
 tq_status tq_logits(const tq_ctx* ctx, const float* q, int B, int Hq, int Hkv, int64_t S,
                     const uint8_t* payload, const uint16_t* norms, float scale, float* out,
                     void* workspace, size_t workspace_bytes, void* stream);
@@ -171,7 +185,8 @@ tq_status tq_logits_noalloc(const tq_ctx* ctx, const float* q, int B, int Hq, in
                             const uint8_t* payload, const uint16_t* norms, float scale, float* out,
                             void* stream);
 
-/* Workspace bytes of tq_attend (per-chunk partial sums). */
+/* Workspace bytes of tq_attend (per-chunk partial sums); 0 for invalid
+ * arguments. */
 size_t tq_attend_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int64_t S);
 
 /* Decode attention output over a quantised value cache (the value path;
@@ -185,12 +200,18 @@ size_t tq_attend_workspace_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int6
  * logits: device fp32 [B, Hq, S], already scaled (for instance tq_logits'
  * output).  out: device fp32 [B, Hq, d].  S = 0 gives zeros.
  * Hq / Hkv <= 8 (TQ_ERR_UNSUPPORTED otherwise).
- * workspace: device, 256-byte aligned, >= tq_attend_workspace_bytes. */
+ * workspace: device, 256-byte aligned, >= tq_attend_workspace_bytes.
+ * B = 0 or Hq = 0 is a no-op.
+ * Errors: TQ_ERR_ARG (ctx NULL; a negative size; Hkv = 0 or Hq not a
+ * multiple of Hkv; a NULL buffer; payload not 16-byte aligned, norms, logits
+ * or out not 4-byte aligned; workspace NULL or misaligned);
+ * TQ_ERR_UNSUPPORTED; TQ_ERR_WORKSPACE; TQ_ERR_CUDA. */
 tq_status tq_attend(const tq_ctx* ctx, const float* logits, int B, int Hq, int Hkv, int64_t S,
                     const uint8_t* payload, const uint16_t* norms, float* out, void* workspace,
                     size_t workspace_bytes, void* stream);
 
-/* Workspace bytes tq_topk needs for nq queries against n database rows. */
+/* Workspace bytes tq_topk needs for nq queries against n database rows; 0
+ * for invalid arguments. */
 size_t tq_topk_workspace_bytes(const tq_ctx* ctx, int64_t nq, int64_t n, int k);
 
 /* Inner-product top-k over a packed database (vector search, [p2] "GloVe
@@ -235,11 +256,14 @@ typedef struct tq_split tq_split;
  * current one; hi.d + lo.d <= 512).  The contexts must outlive the split.
  * Library-owned; release with tq_split_free.  The tensor-core quantizer
  * covers hi.d = lo.d = hi.m = lo.m = 64 with bf16 keys; other shapes run on
- * CUDA cores. */
+ * CUDA cores.  Synchronises the device (uploads the identity order).
+ * Errors: TQ_ERR_ARG (out NULL; hi or lo NULL; Hkv < 1; contexts of
+ * different devices or not of the current one); TQ_ERR_UNSUPPORTED
+ * (hi.d + lo.d > 512); TQ_ERR_NOMEM, TQ_ERR_CUDA. */
 tq_status tq_split_create(const tq_ctx* hi, const tq_ctx* lo, int Hkv, tq_split** out);
 void tq_split_free(tq_split* sp);
 
-/* Workspace bytes of tq_split_plan (fp64 partial sums). */
+/* Workspace bytes of tq_split_plan (fp64 partial sums); 0 when sp is NULL. */
 size_t tq_split_plan_workspace_bytes(const tq_split* sp);
 
 /* Choose the channel order from keys [B][Hkv][S][d] (fp32 or bf16, device):
@@ -247,7 +271,10 @@ size_t tq_split_plan_workspace_bytes(const tq_split* sp);
  * keys, ties to the lower channel index, in ascending channel order, then
  * the other channels in ascending order.  With no keys (B S = 0) every
  * variance is 0 and the order is the identity.  Asynchronous on `stream`;
- * workspace: device, 8-byte aligned, >= tq_split_plan_workspace_bytes. */
+ * workspace: device, 8-byte aligned, >= tq_split_plan_workspace_bytes.
+ * Errors: TQ_ERR_ARG (sp NULL; B or S negative; dtype; keys NULL with
+ * B S > 0 or not aligned to its element; workspace NULL or misaligned);
+ * TQ_ERR_WORKSPACE; TQ_ERR_CUDA. */
 tq_status tq_split_plan(tq_split* sp, const void* keys, tq_dtype dtype, int B, int64_t S, void* workspace,
                         size_t workspace_bytes, void* stream);
 
@@ -261,19 +288,22 @@ tq_status tq_split_get_plan(const tq_split* sp, int32_t* perm);
  * high group of every row with hi into payload_hi / norms_hi (B Hkv S rows of
  * hi's layout), the low group with lo into payload_lo / norms_lo.  Each group
  * is quantised exactly as tq_quantize quantises a key of that group's
- * channels. */
+ * channels.  B S = 0 is a no-op.
+ * Errors: TQ_ERR_ARG (sp NULL; B or S negative; dtype; a NULL buffer; keys
+ * or payloads not 16-byte aligned, norms not 4-byte aligned); TQ_ERR_CUDA. */
 tq_status tq_split_quantize(const tq_split* sp, const void* keys, tq_dtype dtype, int B, int64_t S,
                             uint8_t* payload_hi, uint16_t* norms_hi, uint8_t* payload_lo, uint16_t* norms_lo,
                             void* stream);
 
-/* Workspace bytes of tq_split_logits. */
+/* Workspace bytes of tq_split_logits; 0 for invalid arguments. */
 size_t tq_split_logits_workspace_bytes(const tq_split* sp, int B, int Hq);
 
 /* Decode logits against a split cache: out[b, h, s] = scale (estimate of the
  * high group + estimate of the low group), each group's estimate as in
  * tq_logits with the query's channels gathered by the split of its KV head
  * h / (Hq / Hkv).  q: device fp32 [B, Hq, d]; out: device fp32 [B, Hq, S];
- * workspace: device, 256-byte aligned. */
+ * workspace: device, 256-byte aligned.  B = 0 or Hq = 0 is a no-op.
+ * Errors: as tq_logits (the split's Hkv in place of the argument). */
 tq_status tq_split_logits(const tq_split* sp, const float* q, int B, int Hq, int64_t S, const uint8_t* payload_hi,
                           const uint16_t* norms_hi, const uint8_t* payload_lo, const uint16_t* norms_lo,
                           float scale, float* out, void* workspace, size_t workspace_bytes, void* stream);
