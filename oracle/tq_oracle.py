@@ -724,10 +724,19 @@ def pack_norms(n16: np.ndarray, rho16: np.ndarray) -> np.ndarray:
 
 # ---------------------------------------------------------------------------
 # Parity bands (the readings of the stated tolerances that the parity tests apply)
+#
+# The stated tolerance: codes and sign bits bit-exact except where the rotated
+# value lies within 1e-5 of a decision boundary.  The code decision variable
+# u_j = (R k)_j / ||k|| is one coordinate of the unit vector k / ||k|| in an
+# orthonormal basis, so its band is |u_j - t_i| <= 1e-5 as it stands.  The
+# sign decision variable is (S r)_i = <s_i, r>; read on the same unit-sphere
+# scale it is the coordinate of the unit residual r / ||r|| along the unit JL
+# direction s_i / ||s_i||, i.e. the cosine of the angle between them, and the
+# band is |(S r)_i| <= 1e-5 ||s_i|| ||r||.
 # ---------------------------------------------------------------------------
 
 CODE_BAND = 1e-5     # |u_j - t_i| on the unit-sphere scale
-SIGN_BAND = 1e-5     # |(S r)_i| / (sqrt(m) ||k||): JL row scaled to unit norm, key to unit norm
+SIGN_BAND = 1e-5     # |(S r)_i| / (||s_i|| ||r||): cosine between the JL row and the residual
 NORM_BAND = 1e-5     # relative distance of the exact norm to an fp16 rounding midpoint
 
 
@@ -736,20 +745,44 @@ def code_boundary_distance(u: np.ndarray, t: np.ndarray) -> np.ndarray:
     return np.min(np.abs(u[..., None] - t), axis=-1)
 
 
-def sign_boundary_distance(z: np.ndarray, n: np.ndarray, m: int) -> np.ndarray:
-    """|z_i| / (sqrt(m) ||k||): the sign decision variable on the unit scale."""
-    nn = np.where(n == 0, 1.0, n)
-    return np.abs(z) / (math.sqrt(m) * nn[:, None])
+def sign_boundary_distance(z: np.ndarray, rho: np.ndarray, S: np.ndarray) -> np.ndarray:
+    """|z_i| / (||s_i|| ||r||) for z = S r (rows of z: keys, columns: JL rows).
+
+    A key with a zero residual (rho = 0, e.g. the zero key) has z = 0 and sign
+    bits fixed by the reading [0 >= 0]; it gets distance inf (never excused)."""
+    rho = np.asarray(rho, dtype=np.float64)
+    rn = np.sqrt(np.sum(np.asarray(S, dtype=np.float64) ** 2, axis=1))
+    den = rho[:, None] * rn[None, :]
+    with np.errstate(divide="ignore", invalid="ignore"):
+        out = np.abs(z) / np.where(den > 0, den, 1.0)
+    out[np.broadcast_to(den <= 0, out.shape)] = np.inf
+    return out
+
+
+FP16_MAX = 65504.0
+FP16_OVERFLOW = 65520.0   # the rounding midpoint above the largest fp16: values >= it round to inf
 
 
 def fp16_midpoint_distance(v: np.ndarray) -> np.ndarray:
-    """Relative distance of v to the nearest fp16 rounding midpoint."""
+    """Relative distance of |v| to the nearest fp16 rounding midpoint.
+
+    The rounding midpoints of round-to-nearest fp16 are the means of two
+    adjacent representable values: (h + next_up(h)) / 2 and
+    (h + next_down(h)) / 2 around h = fp16(|v|); h = 0 has only the one
+    above it (0 is a value, not a midpoint).  Above the largest finite value
+    65504 the midpoint is the overflow threshold 65520 (values from there on
+    round to inf).  v = 0 gets inf."""
     v = np.abs(np.asarray(v, dtype=np.float64))
-    h = v.astype(np.float16).astype(np.float64)
-    up = np.nextafter(h.astype(np.float16), np.float16(np.inf)).astype(np.float64)
-    dn = np.nextafter(h.astype(np.float16), np.float16(0)).astype(np.float64)
-    mids = np.stack([(h + up) / 2, (h + dn) / 2], axis=-1)
+    with np.errstate(over="ignore"):
+        h16 = v.astype(np.float16)
+        h = h16.astype(np.float64)
+        up = np.nextafter(h16, np.float16(np.inf)).astype(np.float64)
+        dn = np.nextafter(h16, np.float16(0)).astype(np.float64)
+    with np.errstate(invalid="ignore"):
+        mid_up = np.where(h >= FP16_MAX, FP16_OVERFLOW, (h + up) / 2)
+        mid_dn = np.where(np.isinf(h), FP16_OVERFLOW, np.where(h == 0, np.inf, (h + dn) / 2))
+        dist = np.minimum(np.abs(mid_up - v), np.abs(mid_dn - v))
     with np.errstate(divide="ignore", invalid="ignore"):
-        rel = np.min(np.abs(mids - v[..., None]), axis=-1) / np.where(v == 0, 1.0, v)
-    rel[v == 0] = np.inf
+        rel = dist / np.where(v == 0, 1.0, v)
+    rel = np.where(v == 0, np.inf, rel)
     return rel

@@ -524,6 +524,101 @@ def test_pack_layout_hand_example():
     np.testing.assert_array_equal(p, want)
 
 
+def test_pack_layout_hand_example_one_bit_codes_more_sign_rows():
+    # d = 64, m = 128, b' = 1: chunk q = 1 code halfword (unit 0) + 2 sign
+    # halfwords (units 0, 1) = 3 halfwords; the row is 12 halfwords.
+    d, m = 64, 128
+    codes = np.zeros((1, d), dtype=np.int64)
+    bits = np.zeros((1, m), dtype=bool)
+    codes[0, 16 * 2 + 4 * 3 + 1] = 1   # quarter 2, register 3, nibble 1 -> chunk 2's H0, bit 4*1+3 = 7
+    codes[0, 0] = 1                    # quarter 0, register 0, nibble 0 -> bit 0 of halfword 0
+    bits[0, 32 * 1 + 4 * 6 + 0] = True  # quarter 1, sign register 6 = unit 1, i = 2, nibble 0 -> bit 2
+    bits[0, 127] = True                # quarter 3, register 7 = unit 1, i = 3, nibble 3 -> bit 15
+    p = O.pack_rows(codes, bits, 1)[0].view("<u2")
+    assert p.shape == (12,) and O.row_bytes(d, m, 1) == 24
+    want = np.zeros(12, dtype=np.uint16)
+    want[0] = 0x0001
+    want[2 * 3 + 0] = 0x0080
+    want[1 * 3 + 1 + 1] = 0x0004
+    want[3 * 3 + 1 + 1] = 0x8000
+    np.testing.assert_array_equal(p, want)
+    c2, b2 = O.unpack_rows(O.pack_rows(codes, bits, 1), d, m, 1)
+    np.testing.assert_array_equal(c2, codes)
+    np.testing.assert_array_equal(b2, bits)
+
+
+def test_pack_layout_hand_example_two_bit_codes_fewer_sign_rows():
+    # d = 128, m = 64, b' = 2: chunk q = 2 units x 2 code halfwords + 1 sign
+    # halfword = 5 halfwords; the row is 20 halfwords.
+    d, m = 128, 64
+    codes = np.zeros((1, d), dtype=np.int64)
+    bits = np.zeros((1, m), dtype=bool)
+    codes[0, 32 * 1 + 4 * 5 + 2] = 3   # quarter 1, register 5 = unit 1, pair i = 0, second code,
+    #                                    nibble 2 -> bits 10-11 of chunk 1's halfword 2 * 1 + 0
+    codes[0, 4 * 2 + 3] = 2            # quarter 0, register 2 = unit 0, pair 1, first code, nibble 3
+    #                                    -> bits 12-13 of halfword 1
+    codes[0, 127] = 1                  # quarter 3, register 7 = unit 1, pair 1, second code, nibble 3
+    #                                    -> bits 14-15 of chunk 3's halfword 2 + 1
+    bits[0, 16 * 2 + 4 * 1 + 3] = True  # quarter 2, sign register 1, nibble 3 -> bit 13 of chunk 2's sign halfword
+    p = O.pack_rows(codes, bits, 2)[0].view("<u2")
+    assert p.shape == (20,) and O.row_bytes(d, m, 2) == 40
+    want = np.zeros(20, dtype=np.uint16)
+    want[5 * 1 + 2] = 3 << 10
+    want[0 + 1] = 2 << 12
+    want[5 * 3 + 2 + 1] = 1 << 14
+    want[5 * 2 + 4] = 1 << 13
+    np.testing.assert_array_equal(p, want)
+    c2, b2 = O.unpack_rows(O.pack_rows(codes, bits, 2), d, m, 2)
+    np.testing.assert_array_equal(c2, codes)
+    np.testing.assert_array_equal(b2, bits)
+
+
+def test_sign_boundary_distance_is_the_cosine():
+    # rows s_0 = (3, 4) (norm 5) and s_1 = (0, 2); r = (1, 0): z = (3, 0)
+    S = np.array([[3.0, 4.0], [0.0, 2.0]])
+    r = np.array([[1.0, 0.0], [0.0, -0.5], [0.0, 0.0]])
+    z = r @ S.T
+    rho = np.linalg.norm(r, axis=1)
+    dist = O.sign_boundary_distance(z, rho, S)
+    np.testing.assert_allclose(dist[0], [3 / 5, 0.0], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(dist[1], [4 / 5, 1.0], rtol=0, atol=1e-15)
+    assert np.all(np.isinf(dist[2]))   # zero residual: never excused
+
+
+def test_fp16_midpoint_distance_hand_values():
+    f = O.fp16_midpoint_distance
+    # exact midpoints: 1 + 2^-11 (between 1 and 1 + 2^-10), 2049 (between 2048
+    # and 2050), 2^-25 (between 0 and the smallest subnormal 2^-24), 1.5 2^-24
+    # (between the first two subnormals), 65520 (the overflow threshold)
+    for v in [1 + 2.0**-11, 2049.0, 2.0**-25, 1.5 * 2.0**-24, 65520.0, -(1 + 2.0**-11)]:
+        assert f(np.array([v]))[0] == 0.0, v
+    # 1.0: spacing 2^-11 below 1, so the nearest midpoint is 1 - 2^-12
+    assert f(np.array([1.0]))[0] == 2.0**-12
+    # 65504 (largest finite): midpoints 65488 below and 65520 above, both 16 away
+    assert f(np.array([65504.0]))[0] == 16.0 / 65504.0
+    # 1e5 rounds to inf: the nearest midpoint is the overflow threshold
+    assert f(np.array([1e5]))[0] == (1e5 - 65520.0) / 1e5
+    # 3.0 is representable with spacing 2^-9 on both sides
+    assert f(np.array([3.0]))[0] == 2.0**-10 / 3.0
+    assert np.isinf(f(np.array([0.0]))[0])
+
+
+def test_fp16_midpoint_distance_against_all_midpoints():
+    # every rounding midpoint of fp16, from the list of all finite non-negative
+    # fp16 values; the helper's distance equals the brute-force nearest one
+    allh = np.arange(0, 0x7C00, dtype=np.uint16).view(np.float16).astype(np.float64)
+    mids = np.concatenate([(allh[:-1] + allh[1:]) / 2, [65520.0]])
+    rng = np.random.default_rng(3)
+    v = np.concatenate([np.exp(rng.uniform(np.log(1e-8), np.log(2e5), 20000)),
+                        mids[rng.integers(0, len(mids), 200)],
+                        allh[rng.integers(1, len(allh), 200)]])
+    pos = np.searchsorted(mids, v)
+    lo = mids[np.clip(pos - 1, 0, len(mids) - 1)]
+    hi = mids[np.clip(pos, 0, len(mids) - 1)]
+    want = np.minimum(np.abs(v - lo), np.abs(v - hi)) / v
+    np.testing.assert_array_equal(O.fp16_midpoint_distance(v), want)
+
+
 # --------------------------------------------------------------------------
 # MSE-only variant (m = 0: stage 1 alone)
 # --------------------------------------------------------------------------
