@@ -33,7 +33,7 @@ __global__ void __launch_bounds__(kThreads) quantize_simt_kernel(const T* __rest
                                                                  int bmse, CodebookParams cb,
                                                                  uint8_t* __restrict__ payload,
                                                                  uint16_t* __restrict__ norms,
-                                                                 ChannelGather gth) {
+                                                                 ChannelGather gth, uint32_t* __restrict__ status) {
   extern __shared__ float smem[];
   float* sk = smem;                          // [kKeys][d] keys, later r_rot
   float* sn = sk + kKeys * d;                // [kKeys] norms
@@ -134,8 +134,11 @@ __global__ void __launch_bounds__(kThreads) quantize_simt_kernel(const T* __rest
     if (tid < nk) {
       const float nk_ = sn[tid];
       const float rho = nk_ * sqrtf(srr[tid]);
-      norms[2 * (base + tid)] = __half_as_ushort(__float2half_rn(nk_));
-      norms[2 * (base + tid) + 1] = __half_as_ushort(__float2half_rn(rho));
+      const uint32_t nn = uint32_t(__half_as_ushort(__float2half_rn(nk_))) |
+                          (uint32_t(__half_as_ushort(__float2half_rn(rho))) << 16);
+      norms[2 * (base + tid)] = uint16_t(nn);
+      norms[2 * (base + tid) + 1] = uint16_t(nn >> 16);
+      flag_norm_range(nn, status);
     }
     __syncthreads();
   }
@@ -212,8 +215,10 @@ int grid_for(int64_t n) {
 }  // namespace
 
 cudaError_t launch_quantize_simt(const tq_ctx* ctx, const void* keys, int dtype, int64_t n, int64_t ld,
-                                 uint8_t* payload, uint16_t* norms, cudaStream_t st, ChannelGather gather) {
+                                 uint8_t* payload, uint16_t* norms, cudaStream_t st, ChannelGather gather,
+                                 uint32_t* status) {
   const int d = ctx->d, m = ctx->m;
+  if (!status) status = ctx->dstatus;
   const RowGeom g = make_geom(d, m, ctx->bmse);
   const size_t smem = size_t(kKeys) * d * 4 + 2 * kKeys * 4 + size_t(kKeys) * (g.dp + g.mp);
   const int grid = grid_for(n);
@@ -221,12 +226,12 @@ cudaError_t launch_quantize_simt(const tq_ctx* ctx, const void* keys, int dtype,
     auto kern = quantize_simt_kernel<float>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     kern<<<grid, kThreads, smem, st>>>(static_cast<const float*>(keys), n, ld, ctx->dRt, ctx->dPt, d, m,
-                                        ctx->bmse, ctx->cb, payload, norms, gather);
+                                        ctx->bmse, ctx->cb, payload, norms, gather, status);
   } else {
     auto kern = quantize_simt_kernel<__nv_bfloat16>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
     kern<<<grid, kThreads, smem, st>>>(static_cast<const __nv_bfloat16*>(keys), n, ld, ctx->dRt, ctx->dPt, d,
-                                        m, ctx->bmse, ctx->cb, payload, norms, gather);
+                                        m, ctx->bmse, ctx->cb, payload, norms, gather, status);
   }
   return cudaGetLastError();
 }

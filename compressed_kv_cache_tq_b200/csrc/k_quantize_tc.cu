@@ -475,7 +475,10 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
         const float rho = nk * sqrtf(rrbuf[row] + rrbuf[128 + row]) * (1.0f / 128.f);
         const uint32_t nn = uint32_t(__half_as_ushort(__float2half_rn(nk))) |
                             (uint32_t(__half_as_ushort(__float2half_rn(rho))) << 16);
-        if (key < n) reinterpret_cast<uint32_t*>(norms)[key] = nn;
+        if (key < n) {
+          reinterpret_cast<uint32_t*>(norms)[key] = nn;
+          flag_norm_range(nn, status);
+        }
       }
     }
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");   // none in flight on an early exit
@@ -709,8 +712,10 @@ __device__ __forceinline__ void split_epilogue(uint32_t bar0, uint32_t d1, uint3
     const float rho = nk[g] * sqrtf(rrbuf[g * 128 + row] + rrbuf[(2 + g) * 128 + row]) * (1.0f / 128.f);
     if (valid) {
       uint16_t* nr = g ? norms_lo : norms_hi;
-      reinterpret_cast<uint32_t*>(nr)[key] = uint32_t(__half_as_ushort(__float2half_rn(nk[g]))) |
-                                             (uint32_t(__half_as_ushort(__float2half_rn(rho))) << 16);
+      const uint32_t nn = uint32_t(__half_as_ushort(__float2half_rn(nk[g]))) |
+                          (uint32_t(__half_as_ushort(__float2half_rn(rho))) << 16);
+      reinterpret_cast<uint32_t*>(nr)[key] = nn;
+      flag_norm_range(nn, status);
     }
   }
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");   // none in flight on an early exit

@@ -18,8 +18,10 @@ namespace {
 
 constexpr int kMergeThreads = 256;
 
+// Monotone unsigned key of a float score; -0 and +0 map to the same key, so
+// that they tie (and fall back to the id order) as equal scores do in tq_topk.
 __device__ __forceinline__ uint32_t order_key(float f) {
-  const uint32_t u = __float_as_uint(f);
+  const uint32_t u = f == 0.f ? 0u : __float_as_uint(f);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 

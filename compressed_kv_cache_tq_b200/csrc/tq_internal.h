@@ -74,15 +74,25 @@ struct tq_split {
 namespace tq {
 
 // Device status bits (set by bounded waits that gave up).
-constexpr uint32_t kStatusQuantizeTc = 1u << 0;
-constexpr uint32_t kStatusSearchTc = 1u << 1;
+constexpr uint32_t kStatusQuantizeTc = TQ_STATUS_QUANTIZE_WAIT;
+constexpr uint32_t kStatusSearchTc = TQ_STATUS_SEARCH_WAIT;
+constexpr uint32_t kStatusRange = TQ_STATUS_RANGE;   // a stored norm is not finite in fp16
+
+#ifdef __CUDACC__
+// Set the range bit when either fp16 norm of a packed pair (||k|| low,
+// ||r|| high) is inf or NaN.
+__device__ __forceinline__ void flag_norm_range(uint32_t pair, uint32_t* status) {
+  if (((pair & 0x7C00u) == 0x7C00u) || ((pair & 0x7C000000u) == 0x7C000000u)) atomicOr(status, kStatusRange);
+}
+#endif
 
 void set_cuda_error(cudaError_t e);
 
 // Kernel launchers (defined in the .cu files).  All return cudaGetLastError().
 cudaError_t launch_quantize_simt(const tq_ctx* ctx, const void* keys, int dtype, int64_t n, int64_t ld,
                                  uint8_t* payload, uint16_t* norms, cudaStream_t st,
-                                 ChannelGather gather = ChannelGather{nullptr, 1, 1, 0, 0});
+                                 ChannelGather gather = ChannelGather{nullptr, 1, 1, 0, 0},
+                                 uint32_t* status = nullptr);   // range bit target (nullptr: ctx's)
 bool quantize_tc_supported(const tq_ctx* ctx, int dtype, int64_t ld, const void* keys);
 cudaError_t launch_quantize_tc(const tq_ctx* ctx, const void* keys, int dtype, int64_t n, int64_t ld,
                                uint8_t* payload, uint16_t* norms, cudaStream_t st);

@@ -239,6 +239,7 @@ const char* tq_strerror(tq_status s) {
     case TQ_ERR_NOMEM: return "out of memory";
     case TQ_ERR_WORKSPACE: return "workspace too small";
     case TQ_ERR_DEVICE: return "a kernel reported a device-side error";
+    case TQ_ERR_RANGE: return "a norm exceeded the fp16 range";
   }
   return "unknown status";
 }
@@ -405,7 +406,8 @@ tq_status tq_check_device_status(const tq_ctx* ctx, void* stream, uint32_t* word
     return TQ_ERR_CUDA;
   }
   if (word) *word = h;
-  return h ? TQ_ERR_DEVICE : TQ_OK;
+  if (h & (tq::kStatusQuantizeTc | tq::kStatusSearchTc)) return TQ_ERR_DEVICE;
+  return h ? TQ_ERR_RANGE : TQ_OK;
 }
 
 }  // extern "C"

@@ -121,7 +121,8 @@ tq_status tq_split_quantize(const tq_split* sp, const void* keys, tq_dtype dtype
   cudaError_t e = tq::launch_quantize_simt(sp->hi, keys, dtype, n, sp->d, payload_hi, norms_hi, st,
                                            gather_of(sp, S, true));
   if (e == cudaSuccess)
-    e = tq::launch_quantize_simt(sp->lo, keys, dtype, n, sp->d, payload_lo, norms_lo, st, gather_of(sp, S, false));
+    e = tq::launch_quantize_simt(sp->lo, keys, dtype, n, sp->d, payload_lo, norms_lo, st, gather_of(sp, S, false),
+                                 sp->hi->dstatus);
   return cuda_status(e);
 }
 

@@ -18,7 +18,11 @@ LIB_PATH = os.path.join(_HERE, "libtq.so")
 TQ_F32, TQ_BF16 = 0, 1
 
 _STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape or type", 3: "CUDA error",
-           4: "out of memory", 5: "workspace too small", 6: "device-side error"}
+           4: "out of memory", 5: "workspace too small", 6: "device-side error",
+           7: "a norm exceeded the fp16 range"}
+
+# Bits of the context status word (tq_check_device_status).
+STATUS_QUANTIZE_WAIT, STATUS_SEARCH_WAIT, STATUS_RANGE = 0x1, 0x2, 0x4
 
 
 class TQError(RuntimeError):
@@ -364,9 +368,10 @@ def tq_topk_merge(scores: torch.Tensor, ids: torch.Tensor, first_rows, k: int, s
 
 
 def tq_check_device_status(ctx: Context, stream=None) -> int:
+    """The context's status word (0: clean; STATUS_* bits otherwise), cleared by the read."""
     w = ctypes.c_uint32()
     st = lib().tq_check_device_status(ctx.handle, ctypes.c_void_p(_stream(stream)), ctypes.byref(w))
-    if st not in (0, 6):
+    if st not in (0, 6, 7):
         _check(st, "tq_check_device_status")
     return w.value
 

@@ -30,7 +30,9 @@
  *   - Errors never abort the process.  TQ_ERR_ARG: a null pointer, a negative
  *     or inconsistent size, a misaligned pointer.  TQ_ERR_UNSUPPORTED: a shape
  *     the kernels do not cover.  TQ_ERR_CUDA: a CUDA runtime error (the
- *     message is kept in tq_last_cuda_error()).
+ *     message is kept in tq_last_cuda_error()).  TQ_ERR_RANGE: a quantised
+ *     key's norm did not fit in fp16 (reported through the context's status
+ *     word, see tq_check_device_status, since the kernels run asynchronously).
  *
  * Packed layout (one row per key; the pages fix no layout, only "no
  * per-block constants"):  b' = bits - 1.  The layout has dp and mp slots, d
@@ -68,7 +70,8 @@ typedef enum {
   TQ_ERR_CUDA = 3,
   TQ_ERR_NOMEM = 4,
   TQ_ERR_WORKSPACE = 5,
-  TQ_ERR_DEVICE = 6
+  TQ_ERR_DEVICE = 6,
+  TQ_ERR_RANGE = 7
 } tq_status;
 
 typedef enum { TQ_F32 = 0, TQ_BF16 = 1 } tq_dtype;
@@ -122,6 +125,11 @@ tq_status tq_export_tables(const tq_ctx* ctx, double* R, double* P, double* c, d
  * layout.  keys: device, dtype TQ_F32 or TQ_BF16, 16-byte aligned, ld >= d and
  * ld a multiple of 8.  payload: device, n * row_bytes bytes.  norms: device,
  * n * 2 fp16 values.  A zero key gets codes 0, all sign bits 1, norms 0.
+ * A key whose norm rounds past the fp16 range (||k|| >= 65520, or a key with
+ * non-finite entries) is stored with an infinite (or NaN) norm, and the
+ * kernel sets the range bit of the context's status word:
+ * tq_check_device_status then returns TQ_ERR_RANGE.  Such a row must not be
+ * scored (its logits are inf or NaN).
  * n == 0 is a no-op.
  * Errors: TQ_ERR_ARG (ctx NULL; n < 0; a NULL buffer; dtype; ld < d or not a
  * multiple of 8; keys or payload not 16-byte aligned, norms not 4-byte
@@ -178,9 +186,12 @@ tq_status tq_logits(const tq_ctx* ctx, const float* q, int B, int Hq, int Hkv, i
  * in it has to start at zero (each call rewrites all it reads).  Calls whose
  * kernels overlap on the GPU (for example on two streams) race on the array:
  * order them.
- * Errors: as tq_logits; TQ_ERR_WORKSPACE when tq_logits_workspace_bytes for
- * (B, Hq, Hkv) exceeds TQ_NOALLOC_SCRATCH_BYTES (about 500 (batch, KV head)
- * groups of up to 4 query heads each). */
+ * The looked-up address belongs to the device's context at that time: after
+ * a cudaDeviceReset of the device, do not call this entry point on it again.
+ * Errors: as tq_logits; TQ_ERR_ARG also when the current device is not ctx's
+ * device; TQ_ERR_WORKSPACE when tq_logits_workspace_bytes for (B, Hq, Hkv)
+ * exceeds TQ_NOALLOC_SCRATCH_BYTES (about 500 (batch, KV head) groups of up
+ * to 4 query heads each). */
 tq_status tq_logits_noalloc(const tq_ctx* ctx, const float* q, int B, int Hq, int Hkv, int64_t S,
                             const uint8_t* payload, const uint16_t* norms, float scale, float* out,
                             void* stream);
@@ -288,7 +299,8 @@ tq_status tq_split_get_plan(const tq_split* sp, int32_t* perm);
  * high group of every row with hi into payload_hi / norms_hi (B Hkv S rows of
  * hi's layout), the low group with lo into payload_lo / norms_lo.  Each group
  * is quantised exactly as tq_quantize quantises a key of that group's
- * channels.  B S = 0 is a no-op.
+ * channels.  A group norm outside the fp16 range sets the range bit of hi's
+ * status word (tq_check_device_status on hi).  B S = 0 is a no-op.
  * Errors: TQ_ERR_ARG (sp NULL; B or S negative; dtype; a NULL buffer; keys
  * or payloads not 16-byte aligned, norms not 4-byte aligned); TQ_ERR_CUDA. */
 tq_status tq_split_quantize(const tq_split* sp, const void* keys, tq_dtype dtype, int B, int64_t S,
@@ -323,9 +335,17 @@ tq_status tq_split_logits(const tq_split* sp, const float* q, int B, int Hq, int
 tq_status tq_topk_merge(const float* scores, const int64_t* ids, const int64_t* first_rows, int parts, int64_t nq,
                         int k, int64_t* out_ids, float* out_scores, void* stream);
 
+/* Status word bits (tq_check_device_status). */
+#define TQ_STATUS_QUANTIZE_WAIT 0x1u   /* the tensor-core quantizer gave up a bounded wait */
+#define TQ_STATUS_SEARCH_WAIT 0x2u     /* the tensor-core search gave up a bounded wait */
+#define TQ_STATUS_RANGE 0x4u           /* a quantised key's norm was not finite in fp16 */
+
 /* Read (and clear) the context's device status word after synchronising the
- * stream: 0 when every kernel finished its bounded waits, otherwise a bit set
- * per kernel that gave up.  Returns TQ_ERR_DEVICE when nonzero. */
+ * stream: 0 when every kernel finished its bounded waits and every stored
+ * norm was finite; otherwise the TQ_STATUS_* bits of what happened since the
+ * last check.  Returns TQ_ERR_DEVICE when a wait bit is set, else
+ * TQ_ERR_RANGE when the range bit is set, else TQ_OK (word: host, may be
+ * NULL).  Errors: TQ_ERR_ARG (ctx NULL), TQ_ERR_CUDA. */
 tq_status tq_check_device_status(const tq_ctx* ctx, void* stream, uint32_t* word);
 
 const char* tq_strerror(tq_status s);
