@@ -77,21 +77,37 @@ KV_WORKLOADS = {
     # the MSE-only variant (stage 1 alone, no sign sketch) on the decode layer:
     # b = 4 gives 3 Lloyd-Max bits per coordinate, 48-byte rows
     "mse": (8, 8, 32, 128, 32768, 4, 1001, "decode_mse_only_llama31_8b_layer_b8_hkv8_hq32_d128_s32768_b4_m0"),
+    # the toy configuration: 4096 fp32 keys (N(0,1), 4 seeded channels x10),
+    # 64 fp32 queries scoring all 64 x 4096 pairs (one GQA group of 64), b = 3;
+    # one batch is launch-latency bound (about 2 MB), so the batch of the step
+    # replicates it 256 times (B = 256 copies of the same keys and queries)
+    "toy": (256, 1, 64, 128, 4096, 3, 1000, "toy_n4096_d128_fp32_b3_q64_all_pairs_x256_replicas"),
 }
 SEED_VALUES = 2002
 ATTEND = False
 JL_ROWS = None   # m of the key quantizer (None: m = d; 0: the MSE-only variant)
+KEY_DTYPE = "bf16"   # storage type of the keys fed to the quantizer
+TOY = False
+KV_NAME = "decode"
 
 
-def set_workload(name: str, seq: int | None = None):
-    """Point the module's shape globals at one of KV_WORKLOADS (seq overrides S)."""
-    global B, HKV, HQ, D, S, BITS, SEED_KEYS, WORKLOAD, ATTEND, JL_ROWS
+def set_workload(name: str, seq: int | None = None, batch: int | None = None):
+    """Point the module's shape globals at one of KV_WORKLOADS (seq overrides S,
+    batch overrides B)."""
+    global B, HKV, HQ, D, S, BITS, SEED_KEYS, WORKLOAD, ATTEND, JL_ROWS, KEY_DTYPE, TOY, KV_NAME
     B, HKV, HQ, D, S, BITS, SEED_KEYS, WORKLOAD = KV_WORKLOADS[name]
+    KV_NAME = name
     ATTEND = name == "attend"
     JL_ROWS = 0 if name == "mse" else None
+    TOY = name == "toy"
+    KEY_DTYPE = "fp32" if TOY else "bf16"
     if seq is not None and seq != S:
         WORKLOAD = WORKLOAD.replace(f"_s{S}_", f"_s{seq}_")
         S = seq
+    if batch is not None and batch != B:
+        WORKLOAD = (WORKLOAD.replace(f"_x{B}_replicas", f"_x{batch}_replicas") if TOY
+                    else WORKLOAD.replace(f"_b{B}_", f"_b{batch}_"))
+        B = batch
 
 
 def peaks():
@@ -103,18 +119,64 @@ def peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
+    """SM clocks and throttle reasons sampled while the timed region runs.
+
+    NVML is polled every 2 ms from a thread (so that even a timed region of a
+    few milliseconds gets samples); without NVML, nvidia-smi is sampled every
+    20 ms instead."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
         self.lines = []
+        self.samples = []        # (sm_mhz, max_mhz, reasons) from NVML
+        self.stop = False
+        self.nvml = None
+
+    def _nvml_open(self):
+        import pynvml
+        import torch
+
+        pynvml.nvmlInit()
+        uuid = str(torch.cuda.get_device_properties(self.gpu).uuid)
+        h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        bits = {"hw_slowdown": pynvml.nvmlClocksEventReasonHwSlowdown,
+                "hw_thermal_slowdown": pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                "sw_thermal_slowdown": pynvml.nvmlClocksEventReasonSwThermalSlowdown,
+                "sw_power_cap": pynvml.nvmlClocksEventReasonSwPowerCap}
+        return pynvml, h, bits
+
+    def _poll(self):
+        pynvml, h, bits = self.nvml
+        mx = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        while not self.stop:
+            try:
+                sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((float(sm), float(mx), [n for n, b in bits.items() if r & b]))
+            except Exception:
+                break
+            time.sleep(0.002)
 
     def __enter__(self):
+        try:
+            self.nvml = self._nvml_open()
+            self.t = threading.Thread(target=self._poll, daemon=True)
+            self.t.start()
+            t0 = time.time()
+            while not self.samples and time.time() - t0 < 2.0 and self.t.is_alive():
+                time.sleep(0.001)
+            if self.samples:
+                self.first = len(self.samples)
+                return self
+        except Exception:
+            self.nvml = None
+        self.stop = True
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
                                           "--format=csv,noheader,nounits", "-lms", "20"],
@@ -136,6 +198,13 @@ class ClockSampler:
             self.lines.append(line.strip())
 
     def __exit__(self, *a):
+        if self.nvml is not None and not self.stop:
+            t0 = time.time()
+            while len(self.samples) <= self.first and time.time() - t0 < 0.1:
+                time.sleep(0.001)
+            self.stop = True
+            self.t.join(timeout=1.0)
+            return
         # a short timed region may end before the next sample: wait for one
         t0 = time.time()
         while self.proc and len(self.lines) <= self.first and time.time() - t0 < 0.5:
@@ -149,23 +218,31 @@ class ClockSampler:
 
     def summary(self):
         sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in (self.lines[self.first:] or self.lines):
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
-            except ValueError:
-                continue
-            for nm, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(nm)
+        if self.nvml is not None:
+            for v, m, r in (self.samples[self.first:] or self.samples):
+                sm.append(v)
+                mx = m
+                reasons.update(r)
+            src = "nvml, 2 ms"
+        else:
+            for ln in (self.lines[self.first:] or self.lines):
+                f = [x.strip() for x in ln.split(",")]
+                if len(f) < 9:
+                    continue
+                try:
+                    sm.append(float(f[1]))
+                    mx = float(f[2])
+                except ValueError:
+                    continue
+                for nm, v in zip(self.NAMES, f[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(nm)
+            src = "nvidia-smi, 20 ms"
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
         sm.sort()
-        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm),
+                "source": src}
 
 
 def bytes_per_key():
@@ -177,7 +254,8 @@ def bytes_per_key():
     else:
         m = D if JL_ROWS is None else JL_ROWS
         row = D * (BITS - 1) // 8 + m // 8 + 4
-    bpk = {"quantize_in": 2 * D, "quantize_out": row, "logits_in": row, "logits_out": 4 * (HQ // HKV)}
+    kin = (4 if KEY_DTYPE == "fp32" else 2) * D
+    bpk = {"quantize_in": kin, "quantize_out": row, "logits_in": row, "logits_out": 4 * (HQ // HKV)}
     if ATTEND:
         # keys and values are both quantised; the attention reads the value
         # rows and the logits of the group's query heads
@@ -202,9 +280,9 @@ def kv_config(world: int) -> dict:
             "q_heads": HQ, "head_dim": D,
             "bits": ({"high_64_channels": BITS[0], "low_64_channels": BITS[1]} if isinstance(BITS, tuple)
                      else BITS),
-            "jl_rows": D if JL_ROWS is None else JL_ROWS,
+            "jl_rows": D if JL_ROWS is None else JL_ROWS, "key_dtype": KEY_DTYPE,
             "parallelism": f"replicas x{world}",
-            "l2": f"inputs larger than L2: keys {n * D * 2 / 1e6:.0f} MB, packed caches "
+            "l2": f"inputs larger than L2: keys {n * bpk['quantize_in'] / 1e6:.0f} MB, packed caches "
                   f"{n * (bpk['quantize_out']) / 1e6:.0f} MB each; logits read the cache written one step "
                   "earlier, with the keys' traffic in between"}
 
@@ -258,7 +336,31 @@ def search_cpu_baseline(db, qs, n: int, k: int, bits: int = 4) -> dict:
                       f"against them in {t_score:.1f} s, scaled to {n} rows; fp64 numpy"}
 
 
-def cpu_baseline(budget_s: float = 12.0, max_keys: int = 1 << 19):
+def host_queries():
+    """The step's queries [B, Hq, d] (fp32 numpy): N(0, 1); the toy batch
+    repeats its 64 queries in every replica."""
+    from compressed_kv_cache_tq_b200 import workloads as W
+
+    if TOY:
+        import numpy as np
+
+        return np.repeat(W.queries((1, HQ, D), seed=SEED_KEYS + 1), B, axis=0)
+    return W.queries((B, HQ, D), seed=SEED_KEYS + 7)
+
+
+def device_keys(dev):
+    """The step's keys [B, Hkv, S, d] on the device (bf16, or fp32 for the toy batch)."""
+    import torch
+
+    from compressed_kv_cache_tq_b200 import workloads as W
+
+    if TOY:
+        k = torch.from_numpy(W.toy_keys(S, D, SEED_KEYS)).to(dev)
+        return k.expand(B, HKV, S, D).contiguous()
+    return W.decode_keys(B, HKV, S, D, SEED_KEYS, device=dev)
+
+
+def cpu_baseline(budget_s: float = 12.0, max_keys: int = 1 << 19, chunk: int = 8192):
     """The oracle, as it stands, on a bounded sample of the workload (host cores).
 
     Timed: quantisation of the sampled keys and the estimates of their group's
@@ -278,18 +380,21 @@ def cpu_baseline(budget_s: float = 12.0, max_keys: int = 1 << 19):
         tb_lo = O.make_tables(D // 2, BITS[1], SEED_TABLES + 1)
     else:
         tb = O.make_tables(D, BITS, SEED_TABLES, m=JL_ROWS)
-    scales = W.head_channel_scales(HKV, D, SEED_KEYS)
+    scales = None if TOY else W.head_channel_scales(HKV, D, SEED_KEYS)
     if ATTEND:
         tbv = O.make_tables(D, BITS, SEED_TABLES + 100)
         vscales = W.head_channel_scales(HKV, D, SEED_VALUES)
-    q = W.queries((B, HQ, D), seed=SEED_KEYS + 7)
+    q = host_queries()
     G = HQ // HKV
-    chunk = 8192
+    chunk = min(chunk, S)
     done, busy = 0, 0.0
     for b in range(B):
         for h in range(HKV):
-            keys = W.decode_keys_pair(b, h, S, D, scales, SEED_KEYS)
-            kb = torch.from_numpy(keys).to(torch.bfloat16).to(torch.float64).numpy()
+            if TOY:   # every replica holds the same fp32 keys
+                kb = W.toy_keys(S, D, SEED_KEYS).astype(np.float64)
+            else:
+                keys = W.decode_keys_pair(b, h, S, D, scales, SEED_KEYS)
+                kb = torch.from_numpy(keys).to(torch.bfloat16).to(torch.float64).numpy()
             if ATTEND:
                 vb = torch.from_numpy(W.decode_keys_pair(b, h, S, D, vscales, SEED_VALUES)).to(
                     torch.bfloat16).to(torch.float64).numpy()
@@ -327,31 +432,19 @@ def cpu_baseline(budget_s: float = 12.0, max_keys: int = 1 << 19):
                       f"{busy:.1f} s, fp64 numpy"}
 
 
-def run_search(args):
-    """Vector-search workload: index build + top-10 of 10 000 queries over 10^6 rows.
-
-    With --gpus N (torchrun, NCCL) the database is split by rows over the
-    ranks (strong scaling: the total stays 10^6 rows): each rank indexes and
-    searches its block, and the per-rank top-10 lists are all-gathered and
-    merged on the device (compressed_kv_cache_tq_b200.sharded)."""
-    import numpy as np
+def measure_search(n: int, nq: int, steps: int, warmup: int, local: int = 0, dist=None, rank: int = 0,
+                   world: int = 1, bits_list=(2, 4)) -> dict:
+    """Vector-search workload: index build + top-10 of nq queries over n rows
+    (d = 200), per bit rate.  With a process group the database is split by
+    rows over the ranks: each rank indexes and searches its block, and the
+    per-rank top-10 lists are all-gathered and merged on the device
+    (compressed_kv_cache_tq_b200.sharded).  Times are the slowest rank's."""
     import torch
 
     from compressed_kv_cache_tq_b200 import sharded, tq, workloads as W
 
-    n, nq, d, k = args.rows, args.queries, 200, 10
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    d, k = 200, 10
     dev = torch.device("cuda", local)
-    torch.cuda.set_device(dev)
-    dist = None
-    if world > 1:
-        import datetime
-
-        import torch.distributed as dist
-
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     first, count = sharded.shard_rows(n, world, rank)
     firsts = [sharded.shard_rows(n, world, r)[0] for r in range(world)]
     db = torch.from_numpy(W.search_vectors(n, d, seed=1004, which=0)).to(dev)
@@ -372,19 +465,19 @@ def run_search(args):
         return ids, scores
 
     with ClockSampler(local) as clocks:
-        for bits in (2, 4):
+        for bits in bits_list:
             ctx = tq.tq_init(d, bits, SEED_TABLES)
             payload = torch.empty((count, ctx.row_bytes), dtype=torch.uint8, device=dev)
             norms = torch.empty((count, 2), dtype=torch.float16, device=dev)
             ws = torch.empty(tq.tq_topk_workspace_bytes(ctx, nq, count, k), dtype=torch.uint8, device=dev)
             ids = scores = None
-            for _ in range(args.warmup):
+            for _ in range(warmup):
                 tq.tq_quantize(ctx, shard, payload, norms)
                 ids, scores = search(ctx, qs, payload, norms, ws)
             torch.cuda.synchronize()
             ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
             t_build, t_search = [], []
-            for _ in range(args.steps):
+            for _ in range(steps):
                 if dist is not None:
                     dist.barrier()
                 ev[0].record(stream)
@@ -416,21 +509,48 @@ def run_search(args):
             ms_s = max_over_ranks(sorted(t_search)[len(t_search) // 2], dist, dev)
             e2e = max_over_ranks(a.elapsed_time(b_), dist, dev)
             flops = 2.0 * (d + d) * count * nq   # this rank's share of the contraction
+            # index build: fp32 rows in, packed rows + norms out
+            b_bytes = count * (4 * d + ctx.row_bytes + 4)
             per_bits[f"b{bits}"] = {
                 "index_build_ms": ms_b, "search_ms": ms_s,
                 "queries_per_s": nq / ms_s * 1e3, "recall_at_1_at_10": recall,
-                "search_TFLOP_s_per_gpu": flops / ms_s / 1e9, "e2e_ms": e2e}
+                "search_TFLOP_s_per_gpu": flops / ms_s / 1e9, "search_frac_of_measured_tensor": flops / ms_s / 1e9 / tf,
+                "index_build_GB_s": b_bytes / ms_b / 1e6, "index_build_frac_of_measured_hbm": b_bytes / ms_b / 1e6 / hbm,
+                "e2e_ms": e2e}
             del ws
+    return {"per_bits": per_bits, "clocks": clocks.summary(), "db": db, "qs": qs, "n": n, "nq": nq, "d": d, "k": k}
+
+
+def run_search(args):
+    """The vector-search JSON line (--workload search)."""
+    import torch
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    res = measure_search(args.rows, args.queries, args.steps, args.warmup, local, dist, rank, world)
     if dist is not None:
         dist.destroy_process_group()
     if rank != 0:
         return 0
+    n, nq, d, k = res["n"], res["nq"], res["d"], res["k"]
+    hbm, tf, tf_sus, src = peaks()
     # the oracle on a bounded sample: up to 200 000 rows indexed, 128 queries scored against them
     cpu = None
     if not args.no_cpu_baseline and world == 1:
         n_cpu = min(n, 200_000)
-        cpu = search_cpu_baseline(db[:n_cpu].double().cpu().numpy(), qs[:128].double().cpu().numpy(), n, k)
-    b4 = per_bits["b4"]
+        cpu = search_cpu_baseline(res["db"][:n_cpu].double().cpu().numpy(), res["qs"][:128].double().cpu().numpy(),
+                                  n, k)
+    b4 = res["per_bits"]["b4"]
     line = {
         "metric": SEARCH_METRIC,
         "value": b4["queries_per_s"], "unit": "queries/s", "n_gpus": world, "steps": args.steps,
@@ -438,7 +558,7 @@ def run_search(args):
         "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "f16",
         "data": "synthetic",
         "config": search_config(n, nq, d, k, world),
-        "per_bits": per_bits,
+        "per_bits": res["per_bits"],
         "roofline": {"bound": "tensor", "kernel": "tq_topk (decode + scoring + re-scoring), per GPU",
                      "achieved": b4["search_TFLOP_s_per_gpu"], "peak": tf, "unit": "TFLOP/s",
                      "frac": b4["search_TFLOP_s_per_gpu"] / tf,
@@ -446,7 +566,7 @@ def run_search(args):
         "e2e": {"value": nq / b4["e2e_ms"] * 1e3, "unit": "queries/s", "h2d_bytes_per_step": nq * d * 4,
                 "d2h_bytes_per_step": nq * k * 12},
         "gpu_launches": 4 + (1 if world > 1 else 0),
-        "clocks": clocks.summary(),
+        "clocks": res["clocks"],
     }
     if cpu is not None:
         line["cpu_baseline"] = cpu
@@ -502,13 +622,16 @@ def run_reference(args, rank):
         return 0
     if args.workload == "search":
         return run_reference_search(args)
-    budget = min(2.0, max(0.1, 60.0 / max(1, args.steps + args.warmup)))
+    # each step a bounded sample, sized so that all steps take about a minute
+    budget = min(2.0, max(0.005, 60.0 / max(1, args.steps + args.warmup)))
+    chunk = 8192 if budget >= 0.5 else (2048 if budget >= 0.05 else 256)
     for _ in range(args.warmup):
-        cpu_baseline(budget_s=min(budget, 3.0), max_keys=8192)
+        cpu_baseline(budget_s=min(budget, 3.0), max_keys=chunk, chunk=chunk)
     vals = []
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        vals.append(cpu_baseline(budget_s=budget, max_keys=1 << 16))
+        vals.append(cpu_baseline(budget_s=budget, max_keys=max(chunk, 1 << 16 if budget >= 0.5 else chunk),
+                                 chunk=chunk))
     dt = time.perf_counter() - t0
     v = sum(x["value"] for x in vals) / len(vals)
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "keys/s", "n_gpus": args.gpus,
@@ -526,8 +649,7 @@ def run_reference(args, rank):
 # current kernels, from one ncu capture at S = 16384 (1 048 576 keys); per
 # launch it scales with the keys processed.  Summary with the command:
 # profiles/traffic_decode_s16384.md.  Set to None when a kernel changes.
-DRAM_BYTES_PER_KEY = {"decode": {"tq_quantize": (268.711424e6 + 50.201600e6) / 1048576,
-                                  "tq_logits": (71.455744e6 + 0.465664e6) / 1048576}}
+DRAM_BYTES_PER_KEY = {}
 
 
 def dense_logits_context(keys4, q, reps: int = 20) -> dict:
@@ -607,7 +729,7 @@ def result_line(*, world, n, steps, warmup, ms, q_ms, l_ms, e2e_ms, h2d, d2h, cl
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "bf16",
+        "dtype": "bf16" if KEY_DTYPE == "bf16" else "f32",
         "data": "synthetic",
         "config": kv_config(world),
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": hbm, "unit": "GB/s",
@@ -624,51 +746,25 @@ def result_line(*, world, n, steps, warmup, ms, q_ms, l_ms, e2e_ms, h2d, d2h, cl
     }
 
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=500)
-    ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="decode", choices=["decode", "longctx", "split", "attend", "mse", "search"])
-    ap.add_argument("--rows", type=int, default=1_000_000, help="search: database rows")
-    ap.add_argument("--queries", type=int, default=10_000, help="search: queries")
-    ap.add_argument("--seq", type=int, default=None,
-                    help="sequence length (default: the workload's own; smaller values for profiling)")
-    args = ap.parse_args()
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if args.workload in KV_WORKLOADS:
-        set_workload(args.workload, args.seq)
-    if args.impl == "reference":
-        return run_reference(args, rank)
-    if args.warmup < 3:
-        args.warmup = 3
-    if args.workload == "search":
-        if args.steps == 500:
-            args.steps = 5
-        return run_search(args)
+def measure_kv(steps: int, warmup: int, local: int, dist=None, target_s: float | None = None,
+               e2e: bool = True, keep: bool = False) -> dict:
+    """One key-cache workload (the module's current shape globals) on this rank's GPU.
 
+    A step quantizes the step's keys into one of two packed caches and scores
+    the queries against the other (written one step earlier); with ATTEND it
+    also quantizes values and computes the attention output.  Times: CUDA
+    events on the launching stream, max over ranks.  With target_s, the step
+    count is chosen from the warm-up time so that the timed loop lasts about
+    target_s seconds.  keep: return the device tensors too (parity checks)."""
     import torch
-
-    torch.cuda.set_device(local)
-    dist = None
-    if world > 1:
-        import datetime
-
-        import torch.distributed as dist
-
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
 
     from compressed_kv_cache_tq_b200 import tq, workloads as W
 
     dev = torch.device("cuda", local)
-    keys4 = W.decode_keys(B, HKV, S, D, SEED_KEYS, device=dev)
+    keys4 = device_keys(dev)
     keys = keys4.reshape(-1, D)
     n = keys.shape[0]
-    q = torch.from_numpy(W.queries((B, HQ, D), seed=SEED_KEYS + 7)).to(dev)
+    q = torch.from_numpy(host_queries()).to(dev)
     out = torch.empty((B, HQ, S), dtype=torch.float32, device=dev)
     scale = 1.0 / math.sqrt(D)
     stream = torch.cuda.current_stream()
@@ -715,6 +811,7 @@ def main():
     for c in caches:
         quantize(keys4, c)
     attend = None
+    vals4 = dvals = None
     if ATTEND:
         vctx = tq.tq_init(D, BITS, SEED_TABLES + 100)
         vals4 = W.decode_keys(B, HKV, S, D, SEED_VALUES, device=dev)
@@ -727,7 +824,7 @@ def main():
             tq.tq_quantize(vctx, vals4.reshape(-1, D), c[0], c[1])
         kq_only = quantize
 
-        def quantize(k4, c, i=None):
+        def quantize(k4, c):
             kq_only(k4, c)
             vc = vcaches[0 if c is caches[0] else 1]
             tq.tq_quantize(vctx, (vals4 if k4 is keys4 else dvals).reshape(-1, D), vc[0], vc[1])
@@ -761,13 +858,22 @@ def main():
             dist.barrier()
         torch.cuda.synchronize()
 
-    for i in range(args.warmup):
+    for i in range(warmup):
         step(i, False)
     barrier()
+    if target_s is not None:
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(3):
+            step(i, False)
+        b_.record(stream)
+        torch.cuda.synchronize()
+        per = a.elapsed_time(b_) / 3
+        steps = int(max(10, min(20000, target_s * 1e3 / max(per, 1e-3))))
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clocks:
         t_start.record(stream)
-        for i in range(args.steps):
+        for i in range(steps):
             step(i, True)
         t_end.record(stream)
         barrier()
@@ -776,66 +882,220 @@ def main():
     q_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / len(ev)
     l_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / len(ev)
     a_ms = sum(e[2].elapsed_time(e[3]) for e in ev) / len(ev) if attend else None
+    res = {"steps": steps, "ms": ms, "q_ms": q_ms, "l_ms": l_ms, "a_ms": a_ms, "n": n, "clocks": clocks.summary(),
+           "extra": extra, "h2d": int(keys.numel() * keys.element_size() * (2 if ATTEND else 1) + q.numel() * 4),
+           "d2h": int((B * HQ * D if ATTEND else out.numel()) * 4)}
 
-    # end to end through the public API: pinned host keys in, logits out
-    host_keys = torch.empty(keys4.shape, dtype=keys4.dtype, pin_memory=True)
-    host_keys.copy_(keys4)
-    if ATTEND:
-        host_vals = torch.empty(vals4.shape, dtype=vals4.dtype, pin_memory=True)
-        host_vals.copy_(vals4)
-        dvals = torch.empty_like(vals4)
-    host_q = q.cpu().pin_memory()
-    host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-    if ATTEND:
-        host_att = torch.empty(o_att.shape, dtype=o_att.dtype, pin_memory=True)
-    dkeys = torch.empty_like(keys4)
-    dq = torch.empty_like(q)
-
-    def e2e_step(i):
-        cw, cr = caches[i % 2], caches[(i + 1) % 2]
-        dkeys.copy_(host_keys, non_blocking=True)
+    if e2e:
+        # end to end through the public API: pinned host keys in, logits (or attention output) out
+        host_keys = torch.empty(keys4.shape, dtype=keys4.dtype, pin_memory=True)
+        host_keys.copy_(keys4)
         if ATTEND:
-            dvals.copy_(host_vals, non_blocking=True)
-        dq.copy_(host_q, non_blocking=True)
-        quantize(dkeys, cw)
-        logits(dq, cr)
-        if attend:
-            attend(cr)
-            host_att.copy_(o_att, non_blocking=True)
-        else:
-            host_out.copy_(out, non_blocking=True)
+            host_vals = torch.empty(vals4.shape, dtype=vals4.dtype, pin_memory=True)
+            host_vals.copy_(vals4)
+            dvals = torch.empty_like(vals4)
+            host_att = torch.empty(o_att.shape, dtype=o_att.dtype, pin_memory=True)
+        host_q = q.cpu().pin_memory()
+        host_out = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+        dkeys = torch.empty_like(keys4)
+        dq = torch.empty_like(q)
 
-    e2e_steps = max(3, min(args.steps, 10))
-    for i in range(3):
-        e2e_step(i)
-    barrier()
-    a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for i in range(e2e_steps):
-        e2e_step(i)
-    b_.record(stream)
-    barrier()
-    e2e_ms = max_over_ranks(a.elapsed_time(b_) / e2e_steps, dist, dev)
+        def e2e_step(i):
+            cw, cr = caches[i % 2], caches[(i + 1) % 2]
+            dkeys.copy_(host_keys, non_blocking=True)
+            if ATTEND:
+                dvals.copy_(host_vals, non_blocking=True)
+            dq.copy_(host_q, non_blocking=True)
+            quantize(dkeys, cw)
+            logits(dq, cr)
+            if attend:
+                attend(cr)
+                host_att.copy_(o_att, non_blocking=True)
+            else:
+                host_out.copy_(out, non_blocking=True)
 
+        e2e_steps = max(3, min(steps, 10))
+        for i in range(3):
+            e2e_step(i)
+        barrier()
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(e2e_steps):
+            e2e_step(i)
+        b_.record(stream)
+        barrier()
+        res["e2e_ms"] = max_over_ranks(a.elapsed_time(b_) / e2e_steps, dist, dev)
+    if keep:
+        res.update(keys4=keys4, q=q, out=out, cache=caches[0], ctx=ctx, scale=scale)
+    return res
+
+
+def kv_entry(res: dict, cpu: dict | None) -> dict:
+    """A `configs` entry: the workload's step and kernels, each kernel's
+    algorithmic bytes per second against the measured HBM bandwidth."""
+    line = result_line(world=1, n=res["n"], steps=res["steps"], warmup=3, ms=res["ms"], q_ms=res["q_ms"],
+                       l_ms=res["l_ms"], e2e_ms=res.get("e2e_ms", res["ms"] / res["steps"]), a_ms=res["a_ms"],
+                       h2d=res["h2d"], d2h=res["d2h"], clocks=res["clocks"])
+    hbm = peaks()[0]
+    for kern in line["kernels"].values():
+        kern["frac_of_measured_hbm"] = kern["GB/s"] / hbm
+    ent = {"workload": WORKLOAD, "steps": res["steps"], "ms_per_step": line["ms_per_step"],
+           "keys_per_s": line["value"], "kernels": line["kernels"], "roofline": line["roofline"],
+           "clocks": res["clocks"], **res["extra"]}
+    if cpu is not None:
+        ent["cpu_baseline"] = cpu
+    return ent
+
+
+def oracle_parity(res: dict, n_keys: int = 102400) -> dict:
+    """The oracle check of the run's own outputs (test infrastructure, CPU):
+    about n_keys sampled rows of the packed cache the timed steps wrote, from
+    every (batch, KV head) pair, against the oracle's quantisation of the same
+    keys, and the logits of those rows against the oracle's estimates from the
+    packed rows.  Reports the fractions of mismatching codes and sign bits and
+    of coordinates near a decision boundary."""
+    import numpy as np
+    import torch
+
+    from tests.parity import REL_FLOOR, check_close, check_quantize, merge_stats, oracle_estimates, tables_of
+
+    rep, lrep = {}, {}
+    t0 = time.perf_counter()
+    try:
+        tb = tables_of(res["ctx"])
+        G = HQ // HKV
+        per = max(1, n_keys // (B * HKV))
+        rng = np.random.default_rng(7)
+        payload, norms = res["cache"][0], res["cache"][1]
+        for b in range(B):
+            for h in range(HKV):
+                s_idx = np.sort(rng.choice(S, min(S, per), replace=False))
+                rows = torch.from_numpy((b * HKV + h) * S + s_idx).to(payload.device)
+                k64 = res["keys4"][b, h][rows - (b * HKV + h) * S].to(torch.float64).cpu().numpy()
+                pl, nr = payload[rows].cpu().numpy(), norms[rows].cpu().numpy()
+                st, _ = check_quantize(pl, nr, k64, tb)
+                merge_stats(rep, st)
+                est, A = oracle_estimates(pl, nr, res["q"][b, h * G:(h + 1) * G].cpu().double().numpy(), tb)
+                got = res["out"][b, h * G:(h + 1) * G][:, rows - (b * HKV + h) * S].cpu().numpy()
+                check_close(got, res["scale"] * est, res["scale"] * A, rel_floor=REL_FLOOR, report=lrep)
+        ok, err = True, None
+    except AssertionError as e:
+        ok, err = False, str(e)[:300]
+    out = {"ok": ok, "checked_against": "oracle (fp64 numpy)", **rep,
+           "logits_worst_err_of_term_scale": lrep.get("logits_worst_of_A"),
+           "logits_worst_rel_err": lrep.get("logits_worst_rel"), "logits_rel_floor": REL_FLOOR,
+           "seconds": time.perf_counter() - t0}
+    if err:
+        out["error"] = err
+    return out
+
+
+def configs_block(local: int, no_cpu: bool, search_rows: int, search_queries: int) -> dict:
+    """Every other configuration of the workload table, measured in this
+    process after the headline workload (about a second of timed steps each),
+    with its own oracle baseline on a bounded sample of the same workload."""
+    import torch
+
+    block = {}
+    hbm, tf, _, src = peaks()
+    for name, batch in (("toy", 1), ("toy", None), ("longctx", None), ("split", None), ("mse", None),
+                        ("attend", None)):
+        set_workload(name, batch=batch)
+        key = name if batch is None else f"{name}_single_batch"
+        try:
+            res = measure_kv(10, 3, local, target_s=0.5 if batch == 1 else 1.0, e2e=False)
+            cpu = None if no_cpu else cpu_baseline(budget_s=6.0, max_keys=1 << 17)
+            block[key] = kv_entry(res, cpu)
+        except Exception as e:   # one config failing must not hide the others
+            block[key] = {"workload": WORKLOAD, "error": f"{type(e).__name__}: {str(e)[:200]}"}
+        torch.cuda.empty_cache()
+    set_workload("decode")
+    try:
+        res = measure_search(search_rows, search_queries, 3, 3, local)
+        ent = {"workload": search_config(search_rows, search_queries, 200, 10, 1)["workload"],
+               "per_bits": res["per_bits"], "clocks": res["clocks"],
+               "peaks": {"hbm_GB_s": hbm, "tensor_TFLOP_s": tf, "source": src}}
+        if not no_cpu:
+            n_cpu = min(search_rows, 50_000)
+            ent["cpu_baseline"] = search_cpu_baseline(res["db"][:n_cpu].double().cpu().numpy(),
+                                                      res["qs"][:32].double().cpu().numpy(), search_rows, 10)
+        block["search"] = ent
+        del res
+    except Exception as e:
+        block["search"] = {"error": f"{type(e).__name__}: {str(e)[:200]}"}
+    torch.cuda.empty_cache()
+    return block
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other configurations measured after the headline workload")
+    ap.add_argument("--workload", default="decode",
+                    choices=["decode", "longctx", "split", "attend", "mse", "toy", "search"])
+    ap.add_argument("--rows", type=int, default=1_000_000, help="search: database rows")
+    ap.add_argument("--queries", type=int, default=10_000, help="search: queries")
+    ap.add_argument("--seq", type=int, default=None,
+                    help="sequence length (default: the workload's own; smaller values for profiling)")
+    args = ap.parse_args()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.workload in KV_WORKLOADS:
+        set_workload(args.workload, args.seq)
+    if args.impl == "reference":
+        return run_reference(args, rank)
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.workload == "search":
+        if args.steps == 3000:
+            args.steps = 5
+        return run_search(args)
+
+    import torch
+
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    solo = world == 1 and rank == 0
+    res = measure_kv(args.steps, args.warmup, local, dist, keep=solo and not args.no_cpu_baseline)
     if dist is not None:
         dist.destroy_process_group()
     if rank != 0:
         return 0
 
-    line = result_line(world=world, n=n, steps=args.steps, warmup=args.warmup, ms=ms, q_ms=q_ms, l_ms=l_ms,
-                       e2e_ms=e2e_ms, a_ms=a_ms,
-                       h2d=int(keys.numel() * 2 * (2 if ATTEND else 1) + q.numel() * 4),
-                       d2h=int((o_att if ATTEND else out).numel() * 4),
-                       clocks=clocks.summary())
-    line.update(extra)
-    if world == 1:
-        ctx_d = dense_logits_context(keys4, q)
+    line = result_line(world=world, n=res["n"], steps=args.steps, warmup=args.warmup, ms=res["ms"], q_ms=res["q_ms"],
+                       l_ms=res["l_ms"], e2e_ms=res["e2e_ms"], a_ms=res["a_ms"], h2d=res["h2d"], d2h=res["d2h"],
+                       clocks=res["clocks"])
+    line.update(res["extra"])
+    if solo:
+        ctx_d = dense_logits_context(device_keys(torch.device("cuda", local)), res.get("q", torch.from_numpy(
+            host_queries()).cuda(local)))
         for name in ("fp32", "bf16"):
             if f"{name}_ms" in ctx_d:
-                ctx_d[f"logits_speedup_vs_{name}"] = ctx_d[f"{name}_ms"] / l_ms
+                ctx_d[f"logits_speedup_vs_{name}"] = ctx_d[f"{name}_ms"] / res["l_ms"]
         line["context_dense_logits"] = ctx_d
-    if not args.no_cpu_baseline and world == 1:
+    if solo and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
+        if not isinstance(BITS, tuple):
+            # the oracle check of what the timed steps wrote (test infrastructure, host cores)
+            line["parity"] = oracle_parity(res)
+    for kk in ("keys4", "q", "out", "cache", "ctx"):
+        res.pop(kk, None)
+    torch.cuda.empty_cache()
+    if solo and not args.no_configs and args.workload == "decode" and args.seq is None:
+        line["configs"] = configs_block(local, args.no_cpu_baseline, args.rows, args.queries)
     print(json.dumps(line), flush=True)
     return 0
 

@@ -72,3 +72,17 @@ def test_result_line_names_the_dominant_kernel():
     assert line["roofline"]["kernel"] == "tq_attend"
     assert line["gpu_launches"] == 60
     assert set(line["kernels"]) == {"tq_quantize", "tq_logits", "tq_attend"}
+
+
+def test_toy_workload_fp32_keys_and_replicas():
+    bench.set_workload("toy")
+    assert (bench.B, bench.HKV, bench.HQ, bench.S, bench.BITS, bench.KEY_DTYPE) == (256, 1, 64, 4096, 3, "fp32")
+    bpk = bench.bytes_per_key()
+    # fp32 keys in; 64 fp32 logits out per key (all 64 x 4096 pairs)
+    assert bpk == {"quantize_in": 512, "quantize_out": O.row_bytes(128, 128, 2) + 4,
+                   "logits_in": O.row_bytes(128, 128, 2) + 4, "logits_out": 256}
+    assert bench.kv_config(1)["key_dtype"] == "fp32"
+    bench.set_workload("toy", batch=1)
+    assert bench.B == 1 and bench.WORKLOAD.endswith("_x1_replicas")
+    q = bench.host_queries()
+    assert q.shape == (1, 64, 128) and q.dtype.name == "float32"
