@@ -28,7 +28,7 @@ cudaError_t scratch_address(int dev, void** out) {
   std::lock_guard<std::mutex> lock(g_mutex);
   if (!g_scratch_addr[dev]) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_logits_scratch);
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_logits_scratch);
     if (e != cudaSuccess) return e;
     g_scratch_addr[dev] = p;
   }
