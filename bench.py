@@ -1030,7 +1030,7 @@ def configs_block(local: int, no_cpu: bool, search_rows: int, search_queries: in
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -1053,7 +1053,7 @@ def main():
     if args.warmup < 3:
         args.warmup = 3
     if args.workload == "search":
-        if args.steps == 3000:
+        if args.steps == 1000:
             args.steps = 5
         return run_search(args)
 

@@ -423,6 +423,14 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_mma_kernel(
   const int sign_off = (g >> 1) * kPerQ + 2 * BM + (g & 1);
   const int wcol_head = g >> 1;          // B column g: head g / 2, limb g % 2
   const uint32_t wsel = (g & 1) ? 0x7632u : 0x5410u;   // picks that limb of two keys' limb pairs
+  // b' = 3 with signs: a quarter chunk is 16 bytes (halfwords 0-2 unit 0
+  // codes, 3-5 unit 1 codes, 6 / 7 the units' signs); unit g & 1's halfwords
+  // come out of one 16-byte load
+  constexpr bool kQuad16 = (BM == 3 && JL && rb == 64);
+  // byte-permute selector of the unit's halfwords: (x, y) -> hw 0 or hw 3,
+  // (y, z) -> hw 2 or hw 5, (w, w) -> hw 6 or hw 7; with ^ 0x2222,
+  // (x, z) -> hw 1 or hw 4 (the upper halves of the results are don't-cares)
+  const uint32_t sel_u = (g & 1) ? 0x7676u : 0x1010u;
   float accC[8][4], accS[8][4];
 #pragma unroll
   for (int mt = 0; mt < 8; ++mt)
@@ -493,8 +501,8 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_mma_kernel(
         wr = w * f.y;
         lsum[it] += w;
       }
-      swn[k * GP + h] = limb_pair(wn);
-      swr[k * GP + h] = limb_pair(wr);
+      swn[((k >> 1) * GP + h) * 2 + (k & 1)] = limb_pair(wn);
+      swr[((k >> 1) * GP + h) * 2 + (k & 1)] = limb_pair(wr);
     }
     if (s0 + T < s_end) fetch_w(s0 + T);   // next tile's logits and norms in flight during the math
     __syncthreads();
@@ -502,14 +510,34 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_mma_kernel(
     for (int kb = warp * 16; kb < nk; kb += kAttWarps * 16) {   // 16-key steps; keys past nk have zero weight
       __syncwarp();
       const int kk[4] = {kb + 2 * tig, kb + 2 * tig + 1, kb + 2 * tig + 8, kb + 2 * tig + 9};
-      const uint32_t bC0 = prmt(swn[kk[0] * GP + wcol_head], swn[kk[1] * GP + wcol_head], wsel);
-      const uint32_t bC1 = prmt(swn[kk[2] * GP + wcol_head], swn[kk[3] * GP + wcol_head], wsel);
+      // the limb pairs of keys (2 tig, 2 tig + 1) and (+8, +9) for head wcol_head
+      const int p0 = (kb >> 1) + tig;
+      const uint2 wn0 = *reinterpret_cast<const uint2*>(swn + (p0 * GP + wcol_head) * 2);
+      const uint2 wn1 = *reinterpret_cast<const uint2*>(swn + ((p0 + 4) * GP + wcol_head) * 2);
+      const uint32_t bC0 = prmt(wn0.x, wn0.y, wsel);
+      const uint32_t bC1 = prmt(wn1.x, wn1.y, wsel);
       uint32_t hc[4][BM];
+      uint32_t hsg[4];
+      if constexpr (kQuad16) {
+        // one 16-byte load of the key's quarter chunk; this thread's unit's
+        // halfwords picked by byte permutes (upper halves are don't-cares for
+        // the code selectors, zero for the sign halfword)
 #pragma unroll
-      for (int x = 0; x < 4; ++x) {
-        const uint16_t* hw = reinterpret_cast<const uint16_t*>(srows + kk[x] * rs);
+        for (int x = 0; x < 4; ++x) {
+          const uint4 rw = *reinterpret_cast<const uint4*>(srows + kk[x] * rs + (g >> 1) * 16);
+          hc[x][0] = prmt(rw.x, rw.y, sel_u);
+          hc[x][1] = prmt(rw.x, rw.z, sel_u ^ 0x2222u);
+          hc[x][2] = prmt(rw.y, rw.z, sel_u);
+          hsg[x] = prmt(rw.w, rw.w, sel_u);
+        }
+      } else {
 #pragma unroll
-        for (int y = 0; y < BM; ++y) hc[x][y] = hw[code_off + y];
+        for (int x = 0; x < 4; ++x) {
+          const uint16_t* hw = reinterpret_cast<const uint16_t*>(srows + kk[x] * rs);
+#pragma unroll
+          for (int y = 0; y < BM; ++y) hc[x][y] = hw[code_off + y];
+          if constexpr (JL) hsg[x] = hw[sign_off];
+        }
       }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -533,15 +561,15 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_mma_kernel(
         }
       }
       if constexpr (JL) {
-        const uint32_t bS0 = prmt(swr[kk[0] * GP + wcol_head], swr[kk[1] * GP + wcol_head], wsel);
-        const uint32_t bS1 = prmt(swr[kk[2] * GP + wcol_head], swr[kk[3] * GP + wcol_head], wsel);
-        uint32_t hs[4];
-#pragma unroll
-        for (int x = 0; x < 4; ++x) hs[x] = reinterpret_cast<const uint16_t*>(srows + kk[x] * rs)[sign_off];
+        const uint2 wr0 = *reinterpret_cast<const uint2*>(swr + (p0 * GP + wcol_head) * 2);
+        const uint2 wr1 = *reinterpret_cast<const uint2*>(swr + ((p0 + 4) * GP + wcol_head) * 2);
+        const uint32_t bS0 = prmt(wr0.x, wr0.y, wsel);
+        const uint32_t bS1 = prmt(wr1.x, wr1.y, wsel);
+        const uint32_t(&hs)[4] = hsg;
         // inverted sign bits of a key pair in the two halves: bit 4e + i of the
         // halfword goes to bit 15 (key a) and bit 31 (key b) after a left shift
         // by 15 - 4e - i; set means -1 (fp16 sign bit) over 1.0 (0x3C00)
-        const uint32_t w01 = ~(hs[0] | (hs[1] << 16)), w23 = ~(hs[2] | (hs[3] << 16));
+        const uint32_t w01 = ~prmt(hs[0], hs[1], 0x5410u), w23 = ~prmt(hs[2], hs[3], 0x5410u);
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll

@@ -43,32 +43,51 @@ constexpr int kLogitThreads = 256;
 constexpr int kFragWords = 2 * KS * 2 * 32;
 
 struct HeadScale {
-  float code;   // multiplies the int32 code dot product
-  float sign;   // multiplies the int32 sign dot product
+  float code;      // multiplies the code dot product (int32, after the correction below)
+  float sign;      // multiplies the sign dot product
+  int32_t ccode;   // one-bit codes: integer correction of the code dot product (see qprep_kernel)
+  int32_t csign;   // integer correction of the sign dot product
 };
+
+// Coordinate j (of d = 128) is "register 3" of its unit when ((j % 32) / 4) % 4 == 3
+// (the register whose operand bytes come from the mode bit of a byte permute).
+__device__ __forceinline__ bool reg3_coordinate(int j) { return ((j >> 2) & 3) == 3; }
 
 // ---------------------------------------------------------------------------
 // Query preparation: x = R q, y = P x (= S q), int16 fixed point per head,
 // split into two signed int8 limbs, written in MMA B-fragment order.
-// One block per (batch, kv head) group computes all 4 NT head slots; slots
-// >= G are zero.  R^T and P^T are copied to shared memory (128 KB) at once.
+// One block per (batch, KV head group, chunk of up to 8 query heads): it
+// computes the NT head slots of the chunk (slots past the group's heads are
+// zero).  R^T and P^T are copied to shared memory (128 KB) at once.
+//
+// The logits kernel turns a one-bit field (sign bit, or a one-bit code) into
+// operand bytes a = -bit (registers 0..2 of a unit) or a = 1 - bit (register
+// 3), so the B operand holds -y (and -x for one-bit codes); then
+//   sum_i sigma_i y_i = 2 sum_i bit_i y_i - Y = 2 acc + (2 Y3 - Y),
+// acc = sum_i a_i (-y_i) = sum_i bit_i y_i - Y3, with Y = sum_i y_i and Y3 the
+// sum over register-3 coordinates; csign = 2 Y3 - Y (exact integers).
+// One-bit codes (levels -c1, +c1) use the same form with x.
 // ---------------------------------------------------------------------------
 constexpr int kMaxSlots = 8;
 
-__global__ void __launch_bounds__(128) qprep_kernel(const float* __restrict__ q, int Hq, int Hkv, int nt_per_group,
+__global__ void __launch_bounds__(128) qprep_kernel(const float* __restrict__ q, int Hq, int Hkv, int nchunk, int nt,
                                                     const float* __restrict__ Rt, const float* __restrict__ Pt,
                                                     float code_inv_scale, float scale, float qjl_over_m,
-                                                    uint32_t* __restrict__ frags, HeadScale* __restrict__ hscale) {
+                                                    int one_bit_codes, uint32_t* __restrict__ frags,
+                                                    HeadScale* __restrict__ hscale) {
   extern __shared__ float smq[];
   float* matR = smq;                                 // [D][D] R^T
   float* matP = matR + D * D;                        // [D][D] P^T
   float* sq = matP + D * D;                          // [slots][D] queries
   float* sx = sq + kMaxSlots * D;                    // [slots][D] x
   __shared__ float red[2][kMaxSlots][4];
+  __shared__ int ired[4][kMaxSlots][4];              // [Y, Y3, X, X3][slot][warp]
   __shared__ int8_t limbs[kMaxSlots][2][2][D];       // [slot][x/y][hi/lo][coordinate]
   const int G = Hq / Hkv;
-  const int slots = nt_per_group * HPT;
-  const int grp = blockIdx.x, b = grp / Hkv, hkv = grp % Hkv;
+  const int slots = nt * HPT;
+  const int vg = blockIdx.x, grp = vg / nchunk, chunk = vg - grp * nchunk;
+  const int b = grp / Hkv, hkv = grp % Hkv;
+  const int h0 = chunk * 2 * HPT;                    // first head of the chunk within the group
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   // the logits grid may start streaming the cache now; it waits for this grid before reading fragments
   asm volatile("griddepcontrol.launch_dependents;");
@@ -82,7 +101,8 @@ __global__ void __launch_bounds__(128) qprep_kernel(const float* __restrict__ q,
                    "l"(Pt + 4 * i)
                    : "memory");
   }
-  for (int h = 0; h < slots; ++h) sq[h * D + tid] = h < G ? q[(size_t(b) * Hq + hkv * G + h) * D + tid] : 0.f;
+  for (int h = 0; h < slots; ++h)
+    sq[h * D + tid] = h0 + h < G ? q[(size_t(b) * Hq + hkv * G + h0 + h) * D + tid] : 0.f;
   asm volatile("cp.async.wait_all;" ::: "memory");
   __syncthreads();
   float acc[kMaxSlots];
@@ -126,6 +146,7 @@ __global__ void __launch_bounds__(128) qprep_kernel(const float* __restrict__ q,
     }
   }
   __syncthreads();
+  float kxs[kMaxSlots], kys[kMaxSlots];
 #pragma unroll
   for (int h = 0; h < kMaxSlots; ++h) {
     if (h >= slots) break;
@@ -133,33 +154,63 @@ __global__ void __launch_bounds__(128) qprep_kernel(const float* __restrict__ q,
     const float my = fmaxf(fmaxf(red[1][h][0], red[1][h][1]), fmaxf(red[1][h][2], red[1][h][3]));
     const float kx = mx > 0.f ? 32000.f / mx : 0.f;
     const float ky = my > 0.f ? 32000.f / my : 0.f;
+    kxs[h] = kx;
+    kys[h] = ky;
     const int xi = __float2int_rn(acc[h] * kx);
     const int yi = __float2int_rn(accy[h] * ky);
-    const int xh = (xi + 128) >> 8, yh = (yi + 128) >> 8;
+    // the B operand holds -y (and -x for one-bit codes): see the comment above
+    const int xb = one_bit_codes ? -xi : xi, yb = -yi;
+    const int xh = (xb + 128) >> 8, yh = (yb + 128) >> 8;
     limbs[h][0][0][tid] = int8_t(xh);
-    limbs[h][0][1][tid] = int8_t(xi - 256 * xh);
+    limbs[h][0][1][tid] = int8_t(xb - 256 * xh);
     limbs[h][1][0][tid] = int8_t(yh);
-    limbs[h][1][1][tid] = int8_t(yi - 256 * yh);
-    if (tid == 0 && h < G) {
-      hscale[size_t(b) * Hq + hkv * G + h].code = mx > 0.f ? scale * code_inv_scale / kx : 0.f;
-      hscale[size_t(b) * Hq + hkv * G + h].sign = my > 0.f ? scale * qjl_over_m / ky : 0.f;
+    limbs[h][1][1][tid] = int8_t(yb - 256 * yh);
+    int ty = yi, ty3 = reg3_coordinate(tid) ? yi : 0, tx = xi, tx3 = reg3_coordinate(tid) ? xi : 0;
+    for (int o = 16; o; o >>= 1) {
+      ty += __shfl_xor_sync(0xffffffffu, ty, o);
+      ty3 += __shfl_xor_sync(0xffffffffu, ty3, o);
+      tx += __shfl_xor_sync(0xffffffffu, tx, o);
+      tx3 += __shfl_xor_sync(0xffffffffu, tx3, o);
+    }
+    if (lane == 0) {
+      ired[0][h][warp] = ty;
+      ired[1][h][warp] = ty3;
+      ired[2][h][warp] = tx;
+      ired[3][h][warp] = tx3;
     }
   }
   __syncthreads();
-  // Fragment word (xy, s, reg, lane) of N-tile nt holds B[k = 16 reg + 4 tig + e][n = lane / 4],
-  // e = 0..3; column n is (head slot 4 nt + n / 2, limb n % 2); K position k of step s is
+#pragma unroll
+  for (int h = 0; h < kMaxSlots; ++h) {
+    if (h >= slots) break;
+    if (tid == 0 && h0 + h < G) {
+      const int Y = ired[0][h][0] + ired[0][h][1] + ired[0][h][2] + ired[0][h][3];
+      const int Y3 = ired[1][h][0] + ired[1][h][1] + ired[1][h][2] + ired[1][h][3];
+      const int X = ired[2][h][0] + ired[2][h][1] + ired[2][h][2] + ired[2][h][3];
+      const int X3 = ired[3][h][0] + ired[3][h][1] + ired[3][h][2] + ired[3][h][3];
+      HeadScale hs;
+      hs.code = kxs[h] > 0.f ? scale * code_inv_scale / kxs[h] : 0.f;
+      hs.sign = kys[h] > 0.f ? scale * qjl_over_m / kys[h] : 0.f;
+      hs.ccode = 2 * X3 - X;
+      hs.csign = 2 * Y3 - Y;
+      hscale[size_t(b) * Hq + hkv * G + h0 + h] = hs;
+    }
+  }
+  __syncthreads();
+  // Fragment word (xy, s, reg, lane) of N-tile t holds B[k = 16 reg + 4 tig + e][n = lane / 4],
+  // e = 0..3; column n is (head slot 4 t + n / 2, limb n % 2); K position k of step s is
   // coordinate tig * D/4 + 4 (2s + reg) + e.
-  for (int w = tid; w < nt_per_group * kFragWords; w += 128) {
-    const int nt = w / kFragWords, rem = w - nt * kFragWords;
+  for (int w = tid; w < nt * kFragWords; w += 128) {
+    const int t = w / kFragWords, rem = w - t * kFragWords;
     const int ln = rem & 31, reg = (rem >> 5) & 1, s = (rem >> 6) % KS, xy = (rem >> 6) / KS;
     const int n = ln >> 2, tig = ln & 3;
-    const int slot = nt * HPT + (n >> 1), limb = n & 1;
+    const int slot = t * HPT + (n >> 1), limb = n & 1;
     uint32_t word = 0;
     for (int e = 0; e < 4; ++e) {
       const int j = tig * (D / 4) + 4 * (2 * s + reg) + e;
       word |= uint32_t(uint8_t(limbs[slot][xy][limb][j])) << (8 * e);
     }
-    frags[size_t(grp) * nt_per_group * kFragWords + w] = word;
+    frags[size_t(vg) * nt * kFragWords + w] = word;
   }
 }
 
@@ -227,54 +278,81 @@ __device__ __forceinline__ void load_chunk(Chunk<BMSE, JL>& c, const uint8_t* ro
   }
 }
 
-// Halfword h of the chunk (h = 0 .. 2 BMSE + 1) in the low 16 bits.
-template <int BMSE, bool JL>
-__device__ __forceinline__ uint32_t chunk_half(const Chunk<BMSE, JL>& c, int h) {
-  return (h & 1) ? (c.w[h >> 1] >> 16) : c.w[h >> 1];
+__device__ __forceinline__ uint32_t mad_hi(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("mad.hi.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ uint32_t mad_lo(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
 }
 
-// Byte-permute selectors (4 nibbles, mode bit clear) for the 8 registers of a
-// quarter: codes of register r, nibble e = coordinate (r, e).
+// Shifts and subtractions of the operand expansion done as integer
+// multiply-adds (x >> k = hi(x * 2^(32 - k)); x - y = x + y * (2^32 - 1)):
+// they run on the FMA pipe, which this kernel leaves mostly idle, instead of
+// the integer ALU pipe that the byte permutes and masks fill.  The
+// multipliers are derived from a kernel argument equal to 1, so that the
+// compiler cannot fold the products back into shifts.
+struct FmaShifts {
+  uint32_t s1, s2, s3, s13, s14, s15, s16, s17, s18, s19, neg1;
+  __device__ __forceinline__ explicit FmaShifts(uint32_t one)
+      : s1(one << 31), s2(one << 30), s3(one << 29), s13(one << 19), s14(one << 18), s15(one << 17),
+        s16(one << 16), s17(one << 15), s18(one << 14), s19(one << 13), neg1(0u - one) {}
+};
+
+// Byte-permute selectors (4 nibbles, mode bit clear) of the 8 code registers
+// of a quarter: nibble e of selector r is the code of coordinate (r, e).
+// Only the low 16 bits of a selector are read by the permute, so the upper
+// halfword of a word needs no mask.
 template <int BMSE, bool JL>
-__device__ __forceinline__ void code_selectors(const Chunk<BMSE, JL>& c, uint32_t (&sel)[8]) {
+__device__ __forceinline__ void code_selectors(const Chunk<BMSE, JL>& c, const FmaShifts& f, uint32_t (&sel)[8]) {
+  if constexpr (BMSE == 3) {
+    // words: w0 = H0(u0) | H1(u0), w1 = H2(u0) | H0(u1), w2 = H1(u1) | H2(u1) (low | high halfword)
+    const uint32_t m0 = c.w[0] & 0x77777777u, m1 = c.w[1] & 0x77777777u, m2 = c.w[2] & 0x77777777u;
+    const uint32_t b0 = mad_lo(m0, f.neg1, c.w[0]), b1 = mad_lo(m1, f.neg1, c.w[1]);
+    const uint32_t b2 = mad_lo(m2, f.neg1, c.w[2]);   // bit 3 of every nibble
+    sel[0] = m0;
+    sel[1] = mad_hi(m0, f.s16, 0u);
+    sel[2] = m1;
+    sel[4] = mad_hi(m1, f.s16, 0u);
+    sel[5] = m2;
+    sel[6] = mad_hi(m2, f.s16, 0u);
+    // register 3 of a unit: bit i of its code is bit 3 of the nibble of H_i (disjoint bits: sums are ORs)
+    sel[3] = mad_hi(b0, f.s3, mad_hi(b0, f.s18, mad_hi(b1, f.s1, 0u)));     // H0 >> 3, H1 >> 2, H2 >> 1
+    sel[7] = mad_hi(b1, f.s19, mad_hi(b2, f.s2, mad_hi(b2, f.s17, 0u)));    // H0 >> 3, H1 >> 2, H2 >> 1
+  } else if constexpr (BMSE == 2) {
 #pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    if constexpr (BMSE == 3) {
-      const uint32_t h0 = chunk_half(c, 3 * u), h1 = chunk_half(c, 3 * u + 1), h2 = chunk_half(c, 3 * u + 2);
-      sel[4 * u + 0] = h0 & 0x7777u;
-      sel[4 * u + 1] = h1 & 0x7777u;
-      sel[4 * u + 2] = h2 & 0x7777u;
-      sel[4 * u + 3] = ((h0 >> 3) & 0x1111u) | ((h1 >> 2) & 0x2222u) | ((h2 >> 1) & 0x4444u);
-    } else if constexpr (BMSE == 2) {
-      const uint32_t h0 = chunk_half(c, 2 * u), h1 = chunk_half(c, 2 * u + 1);
-      sel[4 * u + 0] = h0 & 0x3333u;
-      sel[4 * u + 1] = (h0 >> 2) & 0x3333u;
-      sel[4 * u + 2] = h1 & 0x3333u;
-      sel[4 * u + 3] = (h1 >> 2) & 0x3333u;
-    } else {
-      const uint32_t h0 = chunk_half(c, u);
-      sel[4 * u + 0] = h0 & 0x1111u;
-      sel[4 * u + 1] = (h0 >> 1) & 0x1111u;
-      sel[4 * u + 2] = (h0 >> 2) & 0x1111u;
-      sel[4 * u + 3] = (h0 >> 3) & 0x1111u;
+    for (int u = 0; u < 2; ++u) {
+      // word u = H0(u) | H1(u): H0 holds registers 4u (bits 0-1 of a nibble) and 4u + 1 (bits 2-3),
+      // H1 registers 4u + 2 and 4u + 3
+      const uint32_t a = c.w[u] & 0x33333333u;
+      const uint32_t b = mad_hi(c.w[u], f.s2, 0u) & 0x33333333u;
+      sel[4 * u + 0] = a;
+      sel[4 * u + 1] = b;
+      sel[4 * u + 2] = mad_hi(a, f.s16, 0u);
+      sel[4 * u + 3] = mad_hi(b, f.s16, 0u);
     }
   }
 }
 
-// int8 {-1, +1} operands for the 8 sign registers of a quarter.  Register
-// 4u + i of unit u takes bit i of every nibble of the unit's sign halfword.
-// Masking that bit in place gives selector nibbles 0 or 2^i; the two byte
-// tables put -1 at byte 0 and +1 at byte 2^i (bit 3 is the byte-permute mode
-// bit, so register 4u + 3 shifts it down to bit 2 first).
-template <int BMSE, bool JL>
-__device__ __forceinline__ void sign_operands(const Chunk<BMSE, JL>& c, uint32_t (&a)[8]) {
+// Operand bytes of a one-bit field (a sign bit, or a one-bit code) for the 8
+// registers of a quarter: unit u's halfword has bit i of nibble e for
+// register 4u + i, coordinate e.  The raw halfword is the permute selector:
+// the byte tables of registers 0..2 hold -bit(j, i) in {0x00, 0xFF}, which
+// the selector's mode bit (nibble bit 3) leaves unchanged, and the table of
+// register 3 is all 0x01, which the mode bit turns into 0x00; so the bytes are
+// -bit (registers 0..2) and 1 - bit (register 3), without any mask.
+__device__ __forceinline__ void bit_operands(uint32_t w, const FmaShifts& f, uint32_t (&a)[8]) {
+  const uint32_t h1 = mad_hi(w, f.s16, 0u);
 #pragma unroll
   for (int u = 0; u < 2; ++u) {
-    const uint32_t h = chunk_half(c, 2 * BMSE + u);
-    a[4 * u + 0] = prmt(0x000001FFu, 0u, h & 0x1111u);
-    a[4 * u + 1] = prmt(0x000100FFu, 0u, h & 0x2222u);
-    a[4 * u + 2] = prmt(0x000000FFu, 0x00000001u, h & 0x4444u);
-    a[4 * u + 3] = prmt(0x000000FFu, 0x00000001u, (h >> 1) & 0x4444u);
+    const uint32_t h = u ? h1 : w;
+    a[4 * u + 0] = prmt(0xFF00FF00u, 0xFF00FF00u, h);
+    a[4 * u + 1] = prmt(0xFFFF0000u, 0xFFFF0000u, h);
+    a[4 * u + 2] = prmt(0x00000000u, 0xFFFFFFFFu, h);
+    a[4 * u + 3] = prmt(0x01010101u, 0x01010101u, h);
   }
 }
 
@@ -282,13 +360,13 @@ __device__ __forceinline__ void sign_operands(const Chunk<BMSE, JL>& c, uint32_t
 template <int BMSE, int NT, bool JL>
 __device__ __forceinline__ void row_tile(const Chunk<BMSE, JL>& ca, const Chunk<BMSE, JL>& cb, uint32_t na, uint32_t nb,
                                          bool okA, bool okB, const uint32_t (&bx)[NT][KS][2],
-                                         const uint32_t (&by)[NT][KS][2], const float (&sc_code)[NT],
-                                         const float (&sc_sign)[NT], float* const (&orow)[NT], int g, const CodeLut& lut) {
+                                         const uint32_t (&by)[NT][KS][2], const HeadScale (&hs)[NT],
+                                         float* const (&orow)[NT], int g, const CodeLut& lut, const FmaShifts& f) {
   int acc_hi[NT][4], acc_lo[NT][4], acc_sg[NT][4];
-  {
+  if constexpr (BMSE >= 2) {
     uint32_t sa[8], sb[8];
-    code_selectors<BMSE, JL>(ca, sa);
-    code_selectors<BMSE, JL>(cb, sb);
+    code_selectors<BMSE, JL>(ca, f, sa);
+    code_selectors<BMSE, JL>(cb, f, sb);
 #pragma unroll
     for (int s = 0; s < KS; ++s) {
       const uint32_t ah0 = prmt(lut.hi[0], lut.hi[1], sa[2 * s]), ah1 = prmt(lut.hi[0], lut.hi[1], sb[2 * s]);
@@ -308,13 +386,25 @@ __device__ __forceinline__ void row_tile(const Chunk<BMSE, JL>& ca, const Chunk<
         }
       }
     }
+  } else {
+    // one-bit codes (levels -c1, +c1): the one-bit operand form, one MMA per k-step
+    uint32_t ga[8], gb[8];
+    bit_operands(ca.w[0], f, ga);
+    bit_operands(cb.w[0], f, gb);
+#pragma unroll
+    for (int s = 0; s < KS; ++s)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        if (s == 0)
+          mma_s8_first(acc_hi[nt], ga[0], gb[0], ga[1], gb[1], bx[nt][0][0], bx[nt][0][1]);
+        else
+          mma_s8(acc_hi[nt], ga[2 * s], gb[2 * s], ga[2 * s + 1], gb[2 * s + 1], bx[nt][s][0], bx[nt][s][1]);
+      }
   }
   if constexpr (JL) {
-    // sign registers: selectors keep one bit per nibble; the byte table maps
-    // that bit's two possible selector values to -1 and +1
     uint32_t ga[8], gb[8];
-    sign_operands<BMSE, JL>(ca, ga);
-    sign_operands<BMSE, JL>(cb, gb);
+    bit_operands(ca.w[BMSE], f, ga);
+    bit_operands(cb.w[BMSE], f, gb);
 #pragma unroll
     for (int s = 0; s < KS; ++s)
 #pragma unroll
@@ -330,26 +420,36 @@ __device__ __forceinline__ void row_tile(const Chunk<BMSE, JL>& ca, const Chunk<
   const float2 fb = __half22float2(*reinterpret_cast<const __half2*>(&nb));   // of key g + 8
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
-    // |cross terms| <= 2 * 128 * 128 * 128 and |low terms| < 2^21: the integer sums fit in 32 bits
-    const float codeA = fmaf(float(acc_hi[nt][0]), 65536.f, float((acc_hi[nt][1] + acc_lo[nt][0]) * 256 + acc_lo[nt][1]));
-    const float codeB = fmaf(float(acc_hi[nt][2]), 65536.f, float((acc_hi[nt][3] + acc_lo[nt][2]) * 256 + acc_lo[nt][3]));
-    const float signA = JL ? float(acc_sg[nt][0] * 256 + acc_sg[nt][1]) : 0.f;
-    const float signB = JL ? float(acc_sg[nt][2] * 256 + acc_sg[nt][3]) : 0.f;
+    float codeA, codeB;
+    if constexpr (BMSE >= 2) {
+      // |cross terms| <= 2 * 128 * 128 * 128 and |low terms| < 2^21: the integer sums fit in 32 bits
+      codeA = fmaf(float(acc_hi[nt][0]), 65536.f, float((acc_hi[nt][1] + acc_lo[nt][0]) * 256 + acc_lo[nt][1]));
+      codeB = fmaf(float(acc_hi[nt][2]), 65536.f, float((acc_hi[nt][3] + acc_lo[nt][2]) * 256 + acc_lo[nt][3]));
+    } else {
+      codeA = float(2 * (acc_hi[nt][0] * 256 + acc_hi[nt][1]) + hs[nt].ccode);
+      codeB = float(2 * (acc_hi[nt][2] * 256 + acc_hi[nt][3]) + hs[nt].ccode);
+    }
+    const float signA = JL ? float(2 * (acc_sg[nt][0] * 256 + acc_sg[nt][1]) + hs[nt].csign) : 0.f;
+    const float signB = JL ? float(2 * (acc_sg[nt][2] * 256 + acc_sg[nt][3]) + hs[nt].csign) : 0.f;
     if (orow[nt]) {
-      if (okA) orow[nt][g] = fmaf(fa.x * sc_code[nt], codeA, fa.y * sc_sign[nt] * signA);
-      if (okB) orow[nt][g + 8] = fmaf(fb.x * sc_code[nt], codeB, fb.y * sc_sign[nt] * signB);
+      if (okA) orow[nt][g] = fmaf(fa.x * hs[nt].code, codeA, fa.y * hs[nt].sign * signA);
+      if (okB) orow[nt][g + 8] = fmaf(fb.x * hs[nt].code, codeB, fb.y * hs[nt].sign * signB);
     }
   }
 }
 
 // Each warp streams a contiguous range of 32-key tiles (two MMA row tiles
-// sharing the query fragments of their (batch, KV head) group).
+// sharing the query fragments of their group).  A tile's group is a
+// (batch, KV head, chunk of up to 8 query heads) triple: with more than 8
+// query heads per KV head, every chunk reads the rows again (from L2, as the
+// chunks of one KV head are adjacent in the tile order).
 template <int BMSE, int NT, bool JL>
 __global__ void __launch_bounds__(kLogitThreads) logits_mma_kernel(
-    const uint8_t* __restrict__ payload, const uint16_t* __restrict__ norms, int64_t S, int Hq, int Hkv,
+    const uint8_t* __restrict__ payload, const uint16_t* __restrict__ norms, int64_t S, int Hq, int Hkv, int nchunk,
     int64_t total_tiles, const uint32_t* __restrict__ frags, const HeadScale* __restrict__ hscale, CodeLut lut,
-    float* __restrict__ out) {
+    uint32_t one, float* __restrict__ out) {
   constexpr int kRowBytes = D * BMSE / 8 + (JL ? D / 8 : 0);
+  const FmaShifts fsh(one);
   const int lane = threadIdx.x & 31;
   const int g = lane >> 2, tig = lane & 3;
   const int64_t nwarps = int64_t(gridDim.x) * (kLogitThreads / 32);
@@ -363,7 +463,7 @@ __global__ void __launch_bounds__(kLogitThreads) logits_mma_kernel(
   int64_t s0 = (t_begin - grp * tpp) * 32;
 
   auto load_tile = [&](int64_t gi, int64_t so, Chunk<BMSE, JL> (&c)[4], uint32_t (&nn)[4]) {
-    const int64_t row0 = gi * S + so + g;
+    const int64_t row0 = (gi / nchunk) * S + so + g;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const bool ok = so + g + 8 * k < S;
@@ -380,10 +480,12 @@ __global__ void __launch_bounds__(kLogitThreads) logits_mma_kernel(
   if (t_begin >= t_end) return;
 
   uint32_t bx[NT][KS][2], by[NT][KS][2];
-  float sc_code[NT], sc_sign[NT];
+  HeadScale hs[NT];
   float* orow[NT];
   auto load_group = [&](int64_t gi) {
-    const int b = int(gi / Hkv), hkv = int(gi - int64_t(b) * Hkv);
+    const int64_t rg = gi / nchunk;
+    const int chunk = int(gi - rg * nchunk);
+    const int b = int(rg / Hkv), hkv = int(rg - int64_t(b) * Hkv);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const uint32_t* fr = frags + (size_t(gi) * NT + nt) * kFragWords;
@@ -394,11 +496,9 @@ __global__ void __launch_bounds__(kLogitThreads) logits_mma_kernel(
           bx[nt][s][r] = __ldg(fr + ((0 * KS + s) * 2 + r) * 32 + lane);
           by[nt][s][r] = __ldg(fr + ((1 * KS + s) * 2 + r) * 32 + lane);
         }
-      const int hg = nt * HPT + tig;
+      const int hg = chunk * 2 * HPT + nt * HPT + tig;
       const int hh = hg < G ? hg : 0;
-      const HeadScale hs = hscale[size_t(b) * Hq + hkv * G + hh];
-      sc_code[nt] = hs.code;
-      sc_sign[nt] = hs.sign;
+      hs[nt] = hscale[size_t(b) * Hq + hkv * G + hh];
       orow[nt] = hg < G ? out + (size_t(b) * Hq + hkv * G + hh) * S : nullptr;
     }
   };
@@ -418,12 +518,12 @@ __global__ void __launch_bounds__(kLogitThreads) logits_mma_kernel(
     float* orow_t[NT];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) orow_t[nt] = orow[nt] ? orow[nt] + s0 : nullptr;
-    row_tile<BMSE, NT, JL>(cur[0], cur[1], curn[0], curn[1], s0 + g < S, s0 + g + 8 < S, bx, by, sc_code, sc_sign,
-                           orow_t, g, lut);
+    row_tile<BMSE, NT, JL>(cur[0], cur[1], curn[0], curn[1], s0 + g < S, s0 + g + 8 < S, bx, by, hs, orow_t, g, lut,
+                           fsh);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) orow_t[nt] = orow[nt] ? orow[nt] + s0 + 16 : nullptr;
-    row_tile<BMSE, NT, JL>(cur[2], cur[3], curn[2], curn[3], s0 + g + 16 < S, s0 + g + 24 < S, bx, by, sc_code,
-                           sc_sign, orow_t, g, lut);
+    row_tile<BMSE, NT, JL>(cur[2], cur[3], curn[2], curn[3], s0 + g + 16 < S, s0 + g + 24 < S, bx, by, hs, orow_t, g,
+                           lut, fsh);
 
     if (t + 1 < t_end) {
       if (ngrp != grp) load_group(ngrp);
@@ -496,10 +596,10 @@ bool fast_path(const tq_ctx* ctx) {
 }
 
 template <int BMSE, int NT, bool JL>
-cudaError_t launch_mma(const tq_ctx* ctx, int B, int Hq, int Hkv, int64_t S, const uint8_t* payload,
+cudaError_t launch_mma(const tq_ctx* ctx, int B, int Hq, int Hkv, int64_t S, int nchunk, const uint8_t* payload,
                        const uint16_t* norms, float* out, const uint32_t* frags, const HeadScale* hs,
                        cudaStream_t st) {
-  const int64_t total = int64_t(B) * Hkv * ((S + 31) / 32);
+  const int64_t total = int64_t(B) * Hkv * nchunk * ((S + 31) / 32);
   auto kern = logits_mma_kernel<BMSE, NT, JL>;
   int per_sm = 1;
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kLogitThreads, 0);
@@ -516,7 +616,7 @@ cudaError_t launch_mma(const tq_ctx* ctx, int B, int Hq, int Hkv, int64_t S, con
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, payload, norms, S, Hq, Hkv, total, frags, hs, ctx->lut, out);
+  return cudaLaunchKernelEx(&cfg, kern, payload, norms, S, Hq, Hkv, nchunk, total, frags, hs, ctx->lut, 1u, out);
 }
 
 // ---------------------------------------------------------------------------
@@ -881,10 +981,13 @@ cudaError_t launch_logits_simt(const tq_ctx* ctx, const float* q, int B, int Hq,
   return cudaGetLastError();
 }
 
+// Query heads per chunk of a (batch, KV head) group and the MMA N-tiles of a chunk.
+int chunks_of(int G) { return (G + 2 * HPT - 1) / (2 * HPT); }
+int tiles_of(int G) { return G >= 2 * HPT ? 2 : (G + HPT - 1) / HPT; }
+
 size_t qprep_bytes(const tq_ctx* ctx, int64_t groups, int heads_per_group) {
   if (!fast_path(ctx)) return 256;
-  const int nt = (heads_per_group + HPT - 1) / HPT;
-  const size_t frag = size_t(groups) * nt * kFragWords * 4;
+  const size_t frag = size_t(groups) * chunks_of(heads_per_group) * tiles_of(heads_per_group) * kFragWords * 4;
   const size_t scales = size_t(groups) * heads_per_group * sizeof(HeadScale);
   return ((frag + 255) / 256) * 256 + ((scales + 255) / 256) * 256;
 }
@@ -893,30 +996,33 @@ cudaError_t launch_logits(const tq_ctx* ctx, const float* q, int B, int Hq, int 
                           const uint8_t* payload, const uint16_t* norms, float scale, float* out, void* ws,
                           cudaStream_t st) {
   const int G = Hq / Hkv;
-  if (!fast_path(ctx) || G > 8)
+  if (!fast_path(ctx))
     return launch_logits_simt(ctx, q, B, Hq, Hkv, S, payload, norms, scale, out,
                               ChannelGather{nullptr, 1, 1, 0, 0}, 0, st);
-  const int nt = (G + HPT - 1) / HPT;
+  const int nchunk = chunks_of(G), nt = tiles_of(G);
   const int64_t groups = int64_t(B) * Hkv;
   uint32_t* frags = static_cast<uint32_t*>(ws);
-  const size_t frag_bytes = ((size_t(groups) * nt * kFragWords * 4 + 255) / 256) * 256;
+  const size_t frag_bytes = ((size_t(groups) * nchunk * nt * kFragWords * 4 + 255) / 256) * 256;
   HeadScale* hs = reinterpret_cast<HeadScale*>(static_cast<uint8_t*>(ws) + frag_bytes);
   const size_t qp_smem = size_t(2 * D * D + 2 * kMaxSlots * D) * 4;
   cudaFuncSetAttribute(qprep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(qp_smem));
-  qprep_kernel<<<unsigned(groups), 128, qp_smem, st>>>(q, Hq, Hkv, nt, ctx->dRt, ctx->dPt, ctx->lut.inv_scale,
-                                                        scale, float(ctx->m > 0 ? kQjlConst / ctx->m : 0.0), frags, hs);
+  // one-bit codes (levels -c1, +c1) use the one-bit operand form: the code scale is c1
+  const float code_scale = ctx->bmse == 1 ? float(ctx->c[1]) : ctx->lut.inv_scale;
+  qprep_kernel<<<unsigned(groups * nchunk), 128, qp_smem, st>>>(
+      q, Hq, Hkv, nchunk, nt, ctx->dRt, ctx->dPt, code_scale, scale,
+      float(ctx->m > 0 ? kQjlConst / ctx->m : 0.0), ctx->bmse == 1 ? 1 : 0, frags, hs);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (S == 0) return cudaSuccess;
   auto go = [&](auto jl) -> cudaError_t {
     constexpr bool J = decltype(jl)::value;
     switch (ctx->bmse * 10 + nt) {
-      case 11: return launch_mma<1, 1, J>(ctx, B, Hq, Hkv, S, payload, norms, out, frags, hs, st);
-      case 12: return launch_mma<1, 2, J>(ctx, B, Hq, Hkv, S, payload, norms, out, frags, hs, st);
-      case 21: return launch_mma<2, 1, J>(ctx, B, Hq, Hkv, S, payload, norms, out, frags, hs, st);
-      case 22: return launch_mma<2, 2, J>(ctx, B, Hq, Hkv, S, payload, norms, out, frags, hs, st);
-      case 31: return launch_mma<3, 1, J>(ctx, B, Hq, Hkv, S, payload, norms, out, frags, hs, st);
-      default: return launch_mma<3, 2, J>(ctx, B, Hq, Hkv, S, payload, norms, out, frags, hs, st);
+      case 11: return launch_mma<1, 1, J>(ctx, B, Hq, Hkv, S, nchunk, payload, norms, out, frags, hs, st);
+      case 12: return launch_mma<1, 2, J>(ctx, B, Hq, Hkv, S, nchunk, payload, norms, out, frags, hs, st);
+      case 21: return launch_mma<2, 1, J>(ctx, B, Hq, Hkv, S, nchunk, payload, norms, out, frags, hs, st);
+      case 22: return launch_mma<2, 2, J>(ctx, B, Hq, Hkv, S, nchunk, payload, norms, out, frags, hs, st);
+      case 31: return launch_mma<3, 1, J>(ctx, B, Hq, Hkv, S, nchunk, payload, norms, out, frags, hs, st);
+      default: return launch_mma<3, 2, J>(ctx, B, Hq, Hkv, S, nchunk, payload, norms, out, frags, hs, st);
     }
   };
   return ctx->m > 0 ? go(std::true_type{}) : go(std::false_type{});
