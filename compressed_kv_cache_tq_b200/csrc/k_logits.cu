@@ -278,61 +278,38 @@ __device__ __forceinline__ void load_chunk(Chunk<BMSE, JL>& c, const uint8_t* ro
   }
 }
 
-__device__ __forceinline__ uint32_t mad_hi(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t d;
-  asm("mad.hi.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
-__device__ __forceinline__ uint32_t mad_lo(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t d;
-  asm("mad.lo.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
-
-// Shifts and subtractions of the operand expansion done as integer
-// multiply-adds (x >> k = hi(x * 2^(32 - k)); x - y = x + y * (2^32 - 1)):
-// they run on the FMA pipe, which this kernel leaves mostly idle, instead of
-// the integer ALU pipe that the byte permutes and masks fill.  The
-// multipliers are derived from a kernel argument equal to 1, so that the
-// compiler cannot fold the products back into shifts.
-struct FmaShifts {
-  uint32_t s1, s2, s3, s13, s14, s15, s16, s17, s18, s19, neg1;
-  __device__ __forceinline__ explicit FmaShifts(uint32_t one)
-      : s1(one << 31), s2(one << 30), s3(one << 29), s13(one << 19), s14(one << 18), s15(one << 17),
-        s16(one << 16), s17(one << 15), s18(one << 14), s19(one << 13), neg1(0u - one) {}
-};
-
 // Byte-permute selectors (4 nibbles, mode bit clear) of the 8 code registers
 // of a quarter: nibble e of selector r is the code of coordinate (r, e).
-// Only the low 16 bits of a selector are read by the permute, so the upper
-// halfword of a word needs no mask.
+// Only the low 16 bits of a selector are read by the permute, so a word can
+// be masked once for both of its halfwords, and the upper halfword of a word
+// needs only a shift.
 template <int BMSE, bool JL>
-__device__ __forceinline__ void code_selectors(const Chunk<BMSE, JL>& c, const FmaShifts& f, uint32_t (&sel)[8]) {
+__device__ __forceinline__ void code_selectors(const Chunk<BMSE, JL>& c, uint32_t (&sel)[8]) {
   if constexpr (BMSE == 3) {
     // words: w0 = H0(u0) | H1(u0), w1 = H2(u0) | H0(u1), w2 = H1(u1) | H2(u1) (low | high halfword)
     const uint32_t m0 = c.w[0] & 0x77777777u, m1 = c.w[1] & 0x77777777u, m2 = c.w[2] & 0x77777777u;
-    const uint32_t b0 = mad_lo(m0, f.neg1, c.w[0]), b1 = mad_lo(m1, f.neg1, c.w[1]);
-    const uint32_t b2 = mad_lo(m2, f.neg1, c.w[2]);   // bit 3 of every nibble
+    const uint32_t b0 = c.w[0] & 0x88888888u, b1 = c.w[1] & 0x88888888u, b2 = c.w[2] & 0x88888888u;
     sel[0] = m0;
-    sel[1] = mad_hi(m0, f.s16, 0u);
+    sel[1] = m0 >> 16;
     sel[2] = m1;
-    sel[4] = mad_hi(m1, f.s16, 0u);
+    sel[4] = m1 >> 16;
     sel[5] = m2;
-    sel[6] = mad_hi(m2, f.s16, 0u);
-    // register 3 of a unit: bit i of its code is bit 3 of the nibble of H_i (disjoint bits: sums are ORs)
-    sel[3] = mad_hi(b0, f.s3, mad_hi(b0, f.s18, mad_hi(b1, f.s1, 0u)));     // H0 >> 3, H1 >> 2, H2 >> 1
-    sel[7] = mad_hi(b1, f.s19, mad_hi(b2, f.s2, mad_hi(b2, f.s17, 0u)));    // H0 >> 3, H1 >> 2, H2 >> 1
+    sel[6] = m2 >> 16;
+    // register 3 of a unit: bit i of its code is bit 3 of the nibble of H_i
+    // (the shifted terms have disjoint bits in the low halfword)
+    sel[3] = (b0 >> 3) | (b0 >> 18) | (b1 >> 1);     // H0(u0) >> 3, H1(u0) >> 2, H2(u0) >> 1
+    sel[7] = (b1 >> 19) | (b2 >> 2) | (b2 >> 17);    // H0(u1) >> 3, H1(u1) >> 2, H2(u1) >> 1
   } else if constexpr (BMSE == 2) {
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       // word u = H0(u) | H1(u): H0 holds registers 4u (bits 0-1 of a nibble) and 4u + 1 (bits 2-3),
       // H1 registers 4u + 2 and 4u + 3
       const uint32_t a = c.w[u] & 0x33333333u;
-      const uint32_t b = mad_hi(c.w[u], f.s2, 0u) & 0x33333333u;
+      const uint32_t b = (c.w[u] >> 2) & 0x33333333u;
       sel[4 * u + 0] = a;
       sel[4 * u + 1] = b;
-      sel[4 * u + 2] = mad_hi(a, f.s16, 0u);
-      sel[4 * u + 3] = mad_hi(b, f.s16, 0u);
+      sel[4 * u + 2] = a >> 16;
+      sel[4 * u + 3] = b >> 16;
     }
   }
 }
@@ -344,8 +321,8 @@ __device__ __forceinline__ void code_selectors(const Chunk<BMSE, JL>& c, const F
 // the selector's mode bit (nibble bit 3) leaves unchanged, and the table of
 // register 3 is all 0x01, which the mode bit turns into 0x00; so the bytes are
 // -bit (registers 0..2) and 1 - bit (register 3), without any mask.
-__device__ __forceinline__ void bit_operands(uint32_t w, const FmaShifts& f, uint32_t (&a)[8]) {
-  const uint32_t h1 = mad_hi(w, f.s16, 0u);
+__device__ __forceinline__ void bit_operands(uint32_t w, uint32_t (&a)[8]) {
+  const uint32_t h1 = w >> 16;
 #pragma unroll
   for (int u = 0; u < 2; ++u) {
     const uint32_t h = u ? h1 : w;
@@ -361,12 +338,12 @@ template <int BMSE, int NT, bool JL>
 __device__ __forceinline__ void row_tile(const Chunk<BMSE, JL>& ca, const Chunk<BMSE, JL>& cb, uint32_t na, uint32_t nb,
                                          bool okA, bool okB, const uint32_t (&bx)[NT][KS][2],
                                          const uint32_t (&by)[NT][KS][2], const HeadScale (&hs)[NT],
-                                         float* const (&orow)[NT], int g, const CodeLut& lut, const FmaShifts& f) {
+                                         float* const (&orow)[NT], int g, const CodeLut& lut) {
   int acc_hi[NT][4], acc_lo[NT][4], acc_sg[NT][4];
   if constexpr (BMSE >= 2) {
     uint32_t sa[8], sb[8];
-    code_selectors<BMSE, JL>(ca, f, sa);
-    code_selectors<BMSE, JL>(cb, f, sb);
+    code_selectors<BMSE, JL>(ca, sa);
+    code_selectors<BMSE, JL>(cb, sb);
 #pragma unroll
     for (int s = 0; s < KS; ++s) {
       const uint32_t ah0 = prmt(lut.hi[0], lut.hi[1], sa[2 * s]), ah1 = prmt(lut.hi[0], lut.hi[1], sb[2 * s]);
@@ -389,8 +366,8 @@ __device__ __forceinline__ void row_tile(const Chunk<BMSE, JL>& ca, const Chunk<
   } else {
     // one-bit codes (levels -c1, +c1): the one-bit operand form, one MMA per k-step
     uint32_t ga[8], gb[8];
-    bit_operands(ca.w[0], f, ga);
-    bit_operands(cb.w[0], f, gb);
+    bit_operands(ca.w[0], ga);
+    bit_operands(cb.w[0], gb);
 #pragma unroll
     for (int s = 0; s < KS; ++s)
 #pragma unroll
@@ -403,8 +380,8 @@ __device__ __forceinline__ void row_tile(const Chunk<BMSE, JL>& ca, const Chunk<
   }
   if constexpr (JL) {
     uint32_t ga[8], gb[8];
-    bit_operands(ca.w[BMSE], f, ga);
-    bit_operands(cb.w[BMSE], f, gb);
+    bit_operands(ca.w[BMSE], ga);
+    bit_operands(cb.w[BMSE], gb);
 #pragma unroll
     for (int s = 0; s < KS; ++s)
 #pragma unroll
@@ -439,17 +416,41 @@ __device__ __forceinline__ void row_tile(const Chunk<BMSE, JL>& ca, const Chunk<
 }
 
 // Each warp streams a contiguous range of 32-key tiles (two MMA row tiles
-// sharing the query fragments of their group).  A tile's group is a
+// sharing the query fragments of their group), the next tile's rows loaded
+// with 128-bit loads before this tile's math.  A tile's group is a
 // (batch, KV head, chunk of up to 8 query heads) triple: with more than 8
 // query heads per KV head, every chunk reads the rows again (from L2, as the
 // chunks of one KV head are adjacent in the tile order).
+
+// Tile cursor: (row group, head chunk, first key) advanced without divisions.
+struct TileCursor {
+  int64_t rg;
+  int chunk;
+  int64_t s0;
+  __device__ __forceinline__ void init(int64_t t, int64_t tpp, int nchunk) {
+    const int64_t vg = t / tpp;
+    s0 = (t - vg * tpp) * 32;
+    rg = vg / nchunk;
+    chunk = int(vg - rg * nchunk);
+  }
+  __device__ __forceinline__ void next(int64_t S, int nchunk) {
+    s0 += 32;
+    if (s0 >= S) {
+      s0 = 0;
+      if (++chunk == nchunk) {
+        chunk = 0;
+        ++rg;
+      }
+    }
+  }
+};
+
 template <int BMSE, int NT, bool JL>
 __global__ void __launch_bounds__(kLogitThreads) logits_mma_kernel(
     const uint8_t* __restrict__ payload, const uint16_t* __restrict__ norms, int64_t S, int Hq, int Hkv, int nchunk,
     int64_t total_tiles, const uint32_t* __restrict__ frags, const HeadScale* __restrict__ hscale, CodeLut lut,
-    uint32_t one, float* __restrict__ out) {
+    float* __restrict__ out) {
   constexpr int kRowBytes = D * BMSE / 8 + (JL ? D / 8 : 0);
-  const FmaShifts fsh(one);
   const int lane = threadIdx.x & 31;
   const int g = lane >> 2, tig = lane & 3;
   const int64_t nwarps = int64_t(gridDim.x) * (kLogitThreads / 32);
@@ -457,23 +458,22 @@ __global__ void __launch_bounds__(kLogitThreads) logits_mma_kernel(
   const int64_t t_begin = gw * total_tiles / nwarps, t_end = (gw + 1) * total_tiles / nwarps;
   const int G = Hq / Hkv;
   const int64_t tpp = (S + 31) / 32;
+  const uint32_t* norms32 = reinterpret_cast<const uint32_t*>(norms);
 
-  // tile t = (group, key offset s0); advanced incrementally, no division per tile
-  int64_t grp = t_begin / tpp;
-  int64_t s0 = (t_begin - grp * tpp) * 32;
-
-  auto load_tile = [&](int64_t gi, int64_t so, Chunk<BMSE, JL> (&c)[4], uint32_t (&nn)[4]) {
-    const int64_t row0 = (gi / nchunk) * S + so + g;
+  auto load_tile = [&](const TileCursor& c, Chunk<BMSE, JL> (&ch)[4], uint32_t (&nn)[4]) {
+    const int64_t row0 = c.rg * S + c.s0 + g;
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-      const bool ok = so + g + 8 * k < S;
-      load_chunk<BMSE, JL>(c[k], payload + (row0 + 8 * k) * kRowBytes, tig, ok);
-      nn[k] = ok ? __ldg(reinterpret_cast<const uint32_t*>(norms) + row0 + 8 * k) : 0u;
+      const bool ok = c.s0 + g + 8 * k < S;
+      load_chunk<BMSE, JL>(ch[k], payload + (row0 + 8 * k) * kRowBytes, tig, ok);
+      nn[k] = ok ? __ldg(norms32 + row0 + 8 * k) : 0u;
     }
   };
+  TileCursor cc;
+  cc.init(t_begin, tpp, nchunk);
   Chunk<BMSE, JL> cur[4];
   uint32_t curn[4];
-  if (t_begin < t_end) load_tile(grp, s0, cur, curn);
+  if (t_begin < t_end) load_tile(cc, cur, curn);
 
   // the query fragments are written by the preceding query-preparation grid
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -482,10 +482,9 @@ __global__ void __launch_bounds__(kLogitThreads) logits_mma_kernel(
   uint32_t bx[NT][KS][2], by[NT][KS][2];
   HeadScale hs[NT];
   float* orow[NT];
-  auto load_group = [&](int64_t gi) {
-    const int64_t rg = gi / nchunk;
-    const int chunk = int(gi - rg * nchunk);
-    const int b = int(rg / Hkv), hkv = int(rg - int64_t(b) * Hkv);
+  auto load_group = [&](const TileCursor& c) {
+    const int b = int(c.rg / Hkv), hkv = int(c.rg - int64_t(b) * Hkv);
+    const int64_t gi = c.rg * nchunk + c.chunk;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
       const uint32_t* fr = frags + (size_t(gi) * NT + nt) * kFragWords;
@@ -496,39 +495,35 @@ __global__ void __launch_bounds__(kLogitThreads) logits_mma_kernel(
           bx[nt][s][r] = __ldg(fr + ((0 * KS + s) * 2 + r) * 32 + lane);
           by[nt][s][r] = __ldg(fr + ((1 * KS + s) * 2 + r) * 32 + lane);
         }
-      const int hg = chunk * 2 * HPT + nt * HPT + tig;
+      const int hg = c.chunk * 2 * HPT + nt * HPT + tig;
       const int hh = hg < G ? hg : 0;
       hs[nt] = hscale[size_t(b) * Hq + hkv * G + hh];
       orow[nt] = hg < G ? out + (size_t(b) * Hq + hkv * G + hh) * S : nullptr;
     }
   };
-  load_group(grp);
+  load_group(cc);
 
   for (int64_t t = t_begin; t < t_end; ++t) {
     // next tile coordinates and its loads, issued before this tile's math
-    int64_t ngrp = grp, ns0 = s0 + 32;
-    if (ns0 >= S) {
-      ns0 = 0;
-      ++ngrp;
-    }
+    TileCursor nc = cc;
+    nc.next(S, nchunk);
     Chunk<BMSE, JL> nxt[4];
     uint32_t nxtn[4] = {0u, 0u, 0u, 0u};
-    if (t + 1 < t_end) load_tile(ngrp, ns0, nxt, nxtn);
+    if (t + 1 < t_end) load_tile(nc, nxt, nxtn);
 
     float* orow_t[NT];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) orow_t[nt] = orow[nt] ? orow[nt] + s0 : nullptr;
-    row_tile<BMSE, NT, JL>(cur[0], cur[1], curn[0], curn[1], s0 + g < S, s0 + g + 8 < S, bx, by, hs, orow_t, g, lut,
-                           fsh);
+    for (int nt = 0; nt < NT; ++nt) orow_t[nt] = orow[nt] ? orow[nt] + cc.s0 : nullptr;
+    row_tile<BMSE, NT, JL>(cur[0], cur[1], curn[0], curn[1], cc.s0 + g < S, cc.s0 + g + 8 < S, bx, by, hs, orow_t, g,
+                           lut);
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) orow_t[nt] = orow[nt] ? orow[nt] + s0 + 16 : nullptr;
-    row_tile<BMSE, NT, JL>(cur[2], cur[3], curn[2], curn[3], s0 + g + 16 < S, s0 + g + 24 < S, bx, by, hs, orow_t, g,
-                           lut, fsh);
+    for (int nt = 0; nt < NT; ++nt) orow_t[nt] = orow[nt] ? orow[nt] + cc.s0 + 16 : nullptr;
+    row_tile<BMSE, NT, JL>(cur[2], cur[3], curn[2], curn[3], cc.s0 + g + 16 < S, cc.s0 + g + 24 < S, bx, by, hs,
+                           orow_t, g, lut);
 
     if (t + 1 < t_end) {
-      if (ngrp != grp) load_group(ngrp);
-      grp = ngrp;
-      s0 = ns0;
+      if (nc.rg != cc.rg || nc.chunk != cc.chunk) load_group(nc);
+      cc = nc;
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         cur[k] = nxt[k];
@@ -616,7 +611,7 @@ cudaError_t launch_mma(const tq_ctx* ctx, int B, int Hq, int Hkv, int64_t S, int
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, payload, norms, S, Hq, Hkv, nchunk, total, frags, hs, ctx->lut, 1u, out);
+  return cudaLaunchKernelEx(&cfg, kern, payload, norms, S, Hq, Hkv, nchunk, total, frags, hs, ctx->lut, out);
 }
 
 // ---------------------------------------------------------------------------

@@ -1,6 +1,8 @@
-// Tensor-core quantize kernels for bf16 keys of d = 128 (sm_100a):
-//   quantize_tc_kernel<b', JL>   one context, m = 128 (JL) or m = 0 (the
+// Tensor-core quantize kernels for keys of d = 128 (sm_100a):
+//   quantize_tc_kernel<b', JL, F32>  one context, m = 128 (JL) or m = 0 (the
 //                                MSE-only variant: no JL product, no signs);
+//                                bf16 keys, or fp32 keys (F32: split into bf16
+//                                hi + lo on the way in, described below);
 //   quantize_split_tc_kernel     the per-KV-head channel split into two
 //                                64-channel groups (described further down).
 //
@@ -49,6 +51,8 @@
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
 
+#include <type_traits>
+
 #include "tc_sm100.cuh"
 #include "tq_internal.h"
 
@@ -85,14 +89,56 @@ enum Bar {
 };
 static_assert(8 * kNumBars + 8 <= 256, "barrier area");
 
+// fp32 keys: TMA brings 128-row x 32-column fp32 quarter tiles (16 KB, 128-byte
+// swizzle) into a staging ring; two converter warps split each key into
+// bf16 hi = RN(k) and lo = RN(k - hi) and write them as the A operand of one
+// K half (hi 16 KB, lo 16 KB, 128-byte swizzle) into a two-entry ring; the
+// rotation is then K_hi R_hi + K_hi R_lo + K_lo R_hi (K_lo R_lo is below
+// 2^-18 of the product).
+constexpr int kThreadsF32 = 640;    // 2 control + 2 converter + 16 epilogue warps
+constexpr int kStageF32 = 3;        // fp32 quarter tiles in flight
+constexpr int kRingF32 = 2;         // bf16 K halves
+constexpr uint32_t kOffStageF = kConstBytes;
+constexpr uint32_t kOffRingF = kOffStageF + 16384u * kStageF32;
+
+template <bool F32>
+struct QLayout {
+  static constexpr int kThreads = F32 ? kThreadsF32 : kThreadsTc;
+  static constexpr int kEpi0 = F32 ? 4 : 2;   // first epilogue warp
+  static constexpr uint32_t kOffPn2 = F32 ? kOffRingF + 32768u * kRingF32 : kOffKey + 32768u * kKeyStages;
+  static constexpr uint32_t kOffPrr = kOffPn2 + 2u * 2u * 2u * 128u * 4u;
+  static constexpr uint32_t kOffBar = kOffPrr + 2u * 2u * 128u * 4u;
+  static constexpr uint32_t kSmem = kOffBar + 256 + 1024;
+  // barriers: constants, key pipeline (bf16: key stages; fp32: staging, then
+  // the bf16 ring), then one pair per TMEM slot
+  static constexpr int kStages = F32 ? kStageF32 : kKeyStages;
+  static constexpr int kKFull = 1, kKEmpty = kKFull + kStages;
+  static constexpr int kRingFull = kKEmpty + kStages, kRingEmpty = kRingFull + (F32 ? kRingF32 : 0);
+  static constexpr int kD1Full = kRingEmpty + (F32 ? kRingF32 : 0);
+  static constexpr int kN2 = kD1Full + 2, kRFull = kN2 + 2, kRR = kRFull + 2, kD2Full = kRR + 2, kD2Free = kD2Full + 2;
+  static constexpr int kNumBars = kD2Free + 2;
+  static_assert(kSmem <= 232448, "shared memory per block");
+  static_assert(8 * kNumBars + 8 <= 256, "barrier area");
+};
+
 using namespace tc;
 
+// Cycles a wait of this file's kernels spins before it gives up: set by
+// thread 0 of each block before the first wait (the context's test budget,
+// or about 2 s).  The drains before a block exits always use the full budget,
+// so that no copy or MMA is in flight when shared and tensor memory are freed.
+__shared__ long long g_wait_budget;
+
+// A budget below the default (the test hook) waits by non-blocking tests, so
+// that a suspended try_wait cannot outlast it.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag, uint32_t* status) {
-  return tc::mbar_wait(bar, parity, abort_flag, status, kStatusQuantizeTc);
+  if (g_wait_budget < tc::kWaitCycles)
+    return tc::mbar_wait_polling(bar, parity, abort_flag, status, kStatusQuantizeTc, g_wait_budget);
+  return tc::mbar_wait(bar, parity, abort_flag, status, kStatusQuantizeTc, g_wait_budget);
 }
 __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                                uint32_t* status) {
-  return tc::mbar_wait_warp(bar, parity, abort_flag, status, kStatusQuantizeTc);
+  return __all_sync(0xFFFFFFFFu, mbar_wait(bar, parity, abort_flag, status));
 }
 __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                            uint32_t* status) {
@@ -159,23 +205,25 @@ __device__ __forceinline__ uint2 cell2(float2 y, float s128, const HalfBook& hb,
   return make_uint2(__float_as_uint(idx.x), __float_as_uint(idx.y));
 }
 
-template <int BMSE, bool JL>
-__global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid_constant__ CUtensorMap key_map,
+template <int BMSE, bool JL, bool F32>
+__global__ void __launch_bounds__(QLayout<F32>::kThreads, 1) quantize_tc_kernel(const __grid_constant__ CUtensorMap key_map,
                                                                    int64_t n, const uint8_t* __restrict__ bimg,
                                                                    HalfBook book,
                                                                    uint8_t* __restrict__ payload,
                                                                    uint16_t* __restrict__ norms,
-                                                                   uint32_t* __restrict__ status) {
+                                                                   uint32_t* __restrict__ status,
+                                                                   long long wait_budget) {
+  using QL = QLayout<F32>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;   // the swizzle pattern is anchored to 1024-byte boundaries
   uint8_t* sbase = smem_raw + (base - raw);
-  const uint32_t bar0 = base + kOffBar;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sbase + kOffBar + 8 * kNumBars);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + kOffBar + 8 * kNumBars + 4);
+  const uint32_t bar0 = base + QL::kOffBar;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sbase + QL::kOffBar + 8 * QL::kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + QL::kOffBar + 8 * QL::kNumBars + 4);
   auto bar = [&](int i) { return bar0 + 8u * uint32_t(i); };
-  float* pn2 = reinterpret_cast<float*>(sbase + kOffPn2);
-  float* prr = reinterpret_cast<float*>(sbase + kOffPrr);
+  float* pn2 = reinterpret_cast<float*>(sbase + QL::kOffPn2);
+  float* prr = reinterpret_cast<float*>(sbase + QL::kOffPrr);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t num_tiles = (n + kTile - 1) / kTile;
@@ -183,19 +231,26 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
 
   if (threadIdx.x == 0) {
     mbar_init(bar(kBarConst), 1);
-    for (int s = 0; s < kKeyStages; ++s) {
-      mbar_init(bar(kBarKFull + s), 1);
-      mbar_init(bar(kBarKEmpty + s), 1);
+    for (int s = 0; s < QL::kStages; ++s) {
+      mbar_init(bar(QL::kKFull + s), 1);
+      mbar_init(bar(QL::kKEmpty + s), F32 ? 64 : 1);   // fp32: released by the two converter warps
+    }
+    if constexpr (F32) {
+      for (int s = 0; s < kRingF32; ++s) {
+        mbar_init(bar(QL::kRingFull + s), 64);         // written by the two converter warps
+        mbar_init(bar(QL::kRingEmpty + s), 1);         // MMA commit
+      }
     }
     for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(kBarD1Full + s), 1);
-      mbar_init(bar(kBarN2 + s), kTeamThreads);
-      mbar_init(bar(kBarRFull + s), kTeamThreads);
-      mbar_init(bar(kBarRR + s), kTeamThreads);
-      mbar_init(bar(kBarD2Full + s), 1);
-      mbar_init(bar(kBarD2Free + s), kTeamThreads);
+      mbar_init(bar(QL::kD1Full + s), 1);
+      mbar_init(bar(QL::kN2 + s), kTeamThreads);
+      mbar_init(bar(QL::kRFull + s), kTeamThreads);
+      mbar_init(bar(QL::kRR + s), kTeamThreads);
+      mbar_init(bar(QL::kD2Full + s), 1);
+      mbar_init(bar(QL::kD2Free + s), kTeamThreads);
     }
     *abort_flag = 0;
+    g_wait_budget = wait_budget > 0 ? wait_budget : tc::kWaitCycles;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
@@ -217,21 +272,30 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
         mbar_expect_tx(bar(kBarConst), kConst);
         for (int c = 0; c < int(kConst / 16384u); ++c)
           bulk_load(base + 16384u * c, bimg + 16384 * c, 16384u, bar(kBarConst));
+        // bf16 keys: one 32 KB tile per stage; fp32 keys: four 16 KB quarter tiles per tile
+        constexpr int kPer = F32 ? 4 : 1;
+        constexpr int kStg = QL::kStages;
+        const int64_t loads = my_tiles * kPer;
         int64_t i = 0;
-        for (; i < my_tiles; ++i) {
-          const int kb = int(i % kKeyStages);
-          if (i >= kKeyStages &&
-              !mbar_wait(bar(kBarKEmpty + kb), uint32_t((i / kKeyStages - 1) & 1), abort_flag, status))
+        for (; i < loads; ++i) {
+          const int kb = int(i % kStg);
+          if (i >= kStg && !mbar_wait(bar(QL::kKEmpty + kb), uint32_t((i / kStg - 1) & 1), abort_flag, status))
             break;
-          const int64_t tile = blockIdx.x + i * gridDim.x;
-          const uint32_t dst = base + kOffKey + 32768u * kb;
-          mbar_expect_tx(bar(kBarKFull + kb), 32768u);
-          tma_load_2d(dst, &key_map, 0, int(tile * kTile), bar(kBarKFull + kb));
-          tma_load_2d(dst + 16384u, &key_map, 64, int(tile * kTile), bar(kBarKFull + kb));
+          const int64_t tile = blockIdx.x + (i / kPer) * gridDim.x;
+          if constexpr (F32) {
+            mbar_expect_tx(bar(QL::kKFull + kb), 16384u);
+            tma_load_2d(base + kOffStageF + 16384u * kb, &key_map, 32 * int(i & 3), int(tile * kTile),
+                        bar(QL::kKFull + kb));
+          } else {
+            const uint32_t dst = base + kOffKey + 32768u * kb;
+            mbar_expect_tx(bar(QL::kKFull + kb), 32768u);
+            tma_load_2d(dst, &key_map, 0, int(tile * kTile), bar(QL::kKFull + kb));
+            tma_load_2d(dst + 16384u, &key_map, 64, int(tile * kTile), bar(QL::kKFull + kb));
+          }
         }
         // leave no copy in flight: wait for the last loads issued to each buffer
-        for (int64_t j = (i >= kKeyStages ? i - kKeyStages : 0); j < i; ++j)
-          mbar_drain(bar(kBarKFull + int(j % kKeyStages)), uint32_t((j / kKeyStages) & 1), abort_flag, status);
+        for (int64_t j = (i >= kStg ? i - kStg : 0); j < i; ++j)
+          mbar_drain(bar(QL::kKFull + int(j % kStg)), uint32_t((j / kStg) & 1), abort_flag, status);
         mbar_drain(bar(kBarConst), 0u, abort_flag, status);
       }
     } else if (warp == 1) {
@@ -239,12 +303,39 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
       if (lane == 0) {
         auto issue_mma1 = [&](int64_t i) -> bool {
           const int sl = int(i & 1);
+          if constexpr (F32) {
+            // the slot's columns are free as in the bf16 case; then per K half
+            // of the bf16 ring: K_hi R_hi + K_hi R_lo + K_lo R_hi
+            if (i >= 2 &&
+                !mbar_wait(bar((JL ? QL::kD2Full : QL::kRFull) + sl), uint32_t(((i >> 1) - 1) & 1), abort_flag,
+                           status))
+              return false;
+            const uint32_t d1 = tmem + 256u * sl;
+            uint32_t acc = 0;
+            for (int kh = 0; kh < 2; ++kh) {
+              const int64_t e = 2 * i + kh;
+              const int rs = int(e & 1);
+              if (!mbar_wait(bar(QL::kRingFull + rs), uint32_t((e >> 1) & 1), abort_flag, status)) return false;
+              tc_fence_after();
+              const uint32_t abase = base + kOffRingF + 32768u * rs;
+              for (int pass = 0; pass < 3; ++pass)
+                for (int ks = 0; ks < 4; ++ks) {
+                  const uint32_t a = abase + (pass == 2 ? 16384u : 0u) + 32u * ks;
+                  const uint32_t b = base + (pass == 1 ? kOffRlo : kOffRhi) + 16384u * kh + 32u * ks;
+                  mma_f16(d1, smem_desc(a), smem_desc(b), kIdescBf16, acc);
+                  acc = 1;
+                }
+              mma_commit(bar(QL::kRingEmpty + rs));
+            }
+            mma_commit(bar(QL::kD1Full + sl));
+            return true;
+          }
           const int kb = int(i % kKeyStages);
-          if (!mbar_wait(bar(kBarKFull + kb), uint32_t((i / kKeyStages) & 1), abort_flag, status)) return false;
+          if (!mbar_wait(bar(QL::kKFull + kb), uint32_t((i / kKeyStages) & 1), abort_flag, status)) return false;
           // the slot's y / residual columns are free once the JL MMA of tile i - 2 completed
           // (without the sign sketch: once the epilogue of tile i - 2 has read y)
           if (i >= 2 &&
-              !mbar_wait(bar((JL ? kBarD2Full : kBarRFull) + sl), uint32_t(((i >> 1) - 1) & 1), abort_flag, status))
+              !mbar_wait(bar((JL ? QL::kD2Full : QL::kRFull) + sl), uint32_t(((i >> 1) - 1) & 1), abort_flag, status))
             return false;
           tc_fence_after();
           const uint32_t d1 = tmem + 256u * sl;
@@ -258,15 +349,15 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
                         acc);
                 acc = 1;
               }
-          mma_commit(bar(kBarD1Full + sl));
-          mma_commit(bar(kBarKEmpty + kb));
+          mma_commit(bar(QL::kD1Full + sl));
+          mma_commit(bar(QL::kKEmpty + kb));
           return true;
         };
         auto issue_mma2 = [&](int64_t i) -> bool {
           const int sl = int(i & 1);
-          if (!mbar_wait(bar(kBarRFull + sl), uint32_t((i >> 1) & 1), abort_flag, status)) return false;
+          if (!mbar_wait(bar(QL::kRFull + sl), uint32_t((i >> 1) & 1), abort_flag, status)) return false;
           // the slot's z columns are free once the epilogue of tile i - 2 read them
-          if (i >= 2 && !mbar_wait(bar(kBarD2Free + sl), uint32_t(((i >> 1) - 1) & 1), abort_flag, status))
+          if (i >= 2 && !mbar_wait(bar(QL::kD2Free + sl), uint32_t(((i >> 1) - 1) & 1), abort_flag, status))
             return false;
           tc_fence_after();
           const uint32_t d1 = tmem + 256u * sl, d2 = d1 + 128u;
@@ -281,7 +372,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
               acc = 1;
             }
           }
-          mma_commit(bar(kBarD2Full + sl));
+          mma_commit(bar(QL::kD2Full + sl));
           return true;
         };
         int64_t n1 = 0, n2 = 0;   // rotation / JL MMA groups issued
@@ -302,15 +393,59 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
         }
         // before TMEM is released: the commit of the last group of each kind
         // tracks every MMA issued before it
-        if (n1 > 0) mbar_drain(bar(kBarD1Full + int((n1 - 1) & 1)), uint32_t(((n1 - 1) >> 1) & 1), abort_flag, status);
-        if (n2 > 0) mbar_drain(bar(kBarD2Full + int((n2 - 1) & 1)), uint32_t(((n2 - 1) >> 1) & 1), abort_flag, status);
+        if (n1 > 0) mbar_drain(bar(QL::kD1Full + int((n1 - 1) & 1)), uint32_t(((n1 - 1) >> 1) & 1), abort_flag, status);
+        if (n2 > 0) mbar_drain(bar(QL::kD2Full + int((n2 - 1) & 1)), uint32_t(((n2 - 1) >> 1) & 1), abort_flag, status);
       }
+    }
+  } else if (F32 && warp < 4) {
+    // ------------------------------------------------------------ fp32 -> bf16 hi / lo converter
+    // quarter tile j (tile j / 4, columns 32 (j % 4) ..): row r, 8-float group
+    // g of the staging tile -> 16-byte chunk 4 (j % 2) + g of row r of K half
+    // (j % 4) / 2 of the ring entry (both 128-byte swizzled)
+    const int c = threadIdx.x - 64;
+    const int64_t loads = 4 * my_tiles;
+    for (int64_t j = 0; j < loads; ++j) {
+      const int sb = int(j % kStageF32);
+      const int q = int(j & 3);
+      const int64_t e = j >> 1;             // ring entry use: (tile, K half)
+      const int rs = int(e & 1);
+      if ((q & 1) == 0 && e >= 2 &&
+          !mbar_wait_warp(bar(QL::kRingEmpty + rs), uint32_t(((e >> 1) - 1) & 1), abort_flag, status))
+        break;
+      if (!mbar_wait_warp(bar(QL::kKFull + sb), uint32_t((j / kStageF32) & 1), abort_flag, status)) break;
+      const uint8_t* src = sbase + kOffStageF + 16384u * sb;
+      uint8_t* dst = sbase + kOffRingF + 32768u * rs;
+#pragma unroll 2
+      for (int gi = c; gi < 512; gi += 64) {
+        const int r = gi >> 2, g = gi & 3;
+        const float4 a = *reinterpret_cast<const float4*>(src + r * 128 + (((2 * g) ^ (r & 7)) << 4));
+        const float4 b = *reinterpret_cast<const float4*>(src + r * 128 + (((2 * g + 1) ^ (r & 7)) << 4));
+        const float2 x[4] = {make_float2(a.x, a.y), make_float2(a.z, a.w), make_float2(b.x, b.y),
+                             make_float2(b.z, b.w)};
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const __nv_bfloat162 h = __float22bfloat162_rn(x[t]);
+          const float2 hf = __bfloat1622float2(h);
+          const __nv_bfloat162 l = __float22bfloat162_rn(__ffma2_rn(hf, f2(-1.f), x[t]));
+          hi[t] = *reinterpret_cast<const uint32_t*>(&h);
+          lo[t] = *reinterpret_cast<const uint32_t*>(&l);
+        }
+        const uint32_t off = uint32_t(r * 128 + (((4 * (q & 1) + g) ^ (r & 7)) << 4));
+        *reinterpret_cast<uint4*>(dst + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4*>(dst + 16384u + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+      }
+      // the tensor core reads the ring through the async proxy
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive(bar(QL::kKEmpty + sb));
+      if (q & 1) mbar_arrive(bar(QL::kRingFull + rs));
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    // warp w: team (TMEM slot) ((w - 2) >> 2) & 1, half (w - 2) >> 3 (quarters
-    // 2 half and 2 half + 1 of every row), TMEM lanes 32 (w & 3) .. +31.
-    const int eg = (warp - 2) >> 2;
+    // warp w (e = w - first epilogue warp): team (TMEM slot) (e >> 2) & 1,
+    // half e >> 3 (quarters 2 half and 2 half + 1 of every row), TMEM lanes
+    // 32 (w & 3) .. +31.
+    const int eg = (warp - QL::kEpi0) >> 2;
     const int slot = eg & 1, half = eg >> 1;
     const int row = (warp & 3) * 32 + lane;          // TMEM lane = key row within the tile
     const uint32_t lane_addr = uint32_t((warp & 3) * 32) << 16;
@@ -322,7 +457,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
     int64_t k = 0;
     for (int64_t i = slot; i < my_tiles; i += 2, ++k) {
       const uint32_t par = uint32_t(k & 1);
-      if (!mbar_wait_warp(bar(kBarD1Full + slot), par, abort_flag, status)) break;
+      if (!mbar_wait_warp(bar(QL::kD1Full + slot), par, abort_flag, status)) break;
       tc_fence_after();
       // ||k||^2 = ||R k||^2 from the rotated row, half a row per half-team; the
       // partial sums alternate between two buffers, so that a half that runs
@@ -341,8 +476,8 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
         }
         n2buf[half * 128 + row] = acc.x + acc.y;
       }
-      mbar_arrive(bar(kBarN2 + slot));
-      if (!mbar_wait_warp(bar(kBarN2 + slot), par, abort_flag, status)) break;
+      mbar_arrive(bar(QL::kN2 + slot));
+      if (!mbar_wait_warp(bar(QL::kN2 + slot), par, abort_flag, status)) break;
       const float n2 = n2buf[row] + n2buf[128 + row];
       const float nk = sqrtf(n2);
       const bool zero = !(n2 > 0.f);
@@ -417,12 +552,12 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
       }
       if constexpr (JL) asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
       tc_fence_before();
-      mbar_arrive(bar(kBarRFull + slot));   // residual in TMEM (without the sketch: y read)
+      mbar_arrive(bar(QL::kRFull + slot));   // residual in TMEM (without the sketch: y read)
       rrbuf[half * 128 + row] = rr2.x + rr2.y;
-      mbar_arrive(bar(kBarRR + slot));
+      mbar_arrive(bar(QL::kRR + slot));
       uint32_t sw[2] = {0u, 0u};
       if constexpr (JL) {
-      if (!mbar_wait_warp(bar(kBarD2Full + slot), par, abort_flag, status)) break;
+      if (!mbar_wait_warp(bar(QL::kD2Full + slot), par, abort_flag, status)) break;
       tc_fence_after();
       // bit = [z >= 0] = not the sign bit (z = -0 cannot arise for a nonzero
       // residual; zero keys get all ones).  Bit p of quarter q's word holds
@@ -445,7 +580,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
         sw[qq] = zero ? 0xFFFFFFFFu : ~neg;
       }
       tc_fence_before();
-      mbar_arrive(bar(kBarD2Free + slot));
+      mbar_arrive(bar(QL::kD2Free + slot));
       }
       const int64_t key = (blockIdx.x + i * gridDim.x) * kTile + row;
       if (key < n) {
@@ -471,7 +606,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_tc_kernel(const __grid
         // ||r|| = n ||r_rot|| from both halves' sums (r_rot scaled by 128); the
         // other half writes these sums again only after its next N2 wait, which
         // needs this thread's next arrival
-        if (!mbar_wait_warp(bar(kBarRR + slot), par, abort_flag, status)) break;
+        if (!mbar_wait_warp(bar(QL::kRR + slot), par, abort_flag, status)) break;
         const float rho = nk * sqrtf(rrbuf[row] + rrbuf[128 + row]) * (1.0f / 128.f);
         const uint32_t nn = uint32_t(__half_as_ushort(__float2half_rn(nk))) |
                             (uint32_t(__half_as_ushort(__float2half_rn(rho))) << 16);
@@ -764,6 +899,7 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_split_tc_kernel(
       mbar_init(bar(kBarD2Free + sl), kTeamThreads);
     }
     *abort_flag = 0;
+    g_wait_budget = tc::kWaitCycles;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
@@ -900,22 +1036,24 @@ HalfBook make_halfbook(const tq_ctx* ctx) {
 }  // namespace
 
 bool quantize_tc_supported(const tq_ctx* ctx, int dtype, int64_t ld, const void* keys) {
-  return ctx->d == kD && (ctx->m == kD || ctx->m == 0) && dtype == TQ_BF16 && ctx->bmse >= 1 && ctx->bmse <= 3 &&
-         ctx->dBimg != nullptr && ld % 8 == 0 && (reinterpret_cast<uintptr_t>(keys) & 15) == 0 &&
-         device_is_sm100() && get_encode() != nullptr;
+  return ctx->d == kD && (ctx->m == kD || ctx->m == 0) && (dtype == TQ_BF16 || dtype == TQ_F32) &&
+         ctx->bmse >= 1 && ctx->bmse <= 3 && ctx->dBimg != nullptr && ld % 8 == 0 &&
+         (reinterpret_cast<uintptr_t>(keys) & 15) == 0 && device_is_sm100() && get_encode() != nullptr;
 }
 
 cudaError_t launch_quantize_tc(const tq_ctx* ctx, const void* keys, int dtype, int64_t n, int64_t ld,
                                uint8_t* payload, uint16_t* norms, cudaStream_t st) {
-  (void)dtype;
+  const bool f32 = dtype == TQ_F32;
   CUtensorMap map;
   const cuuint64_t dims[2] = {cuuint64_t(kD), cuuint64_t(n)};
-  const cuuint64_t strides[1] = {cuuint64_t(ld) * 2};
-  const cuuint32_t box[2] = {64u, 128u};
+  const cuuint64_t strides[1] = {cuuint64_t(ld) * (f32 ? 4 : 2)};
+  // bf16: 64-column halves (128 bytes per row); fp32: 32-column quarters (128 bytes per row)
+  const cuuint32_t box[2] = {f32 ? 32u : 64u, 128u};
   const cuuint32_t estr[2] = {1u, 1u};
-  const CUresult r = get_encode()(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(keys), dims, strides,
-                                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const CUresult r = get_encode()(&map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                                  const_cast<void*>(keys), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
@@ -923,19 +1061,28 @@ cudaError_t launch_quantize_tc(const tq_ctx* ctx, const void* keys, int dtype, i
   const int64_t tiles = (n + kTile - 1) / kTile;
   const int grid = int(tiles < sms ? tiles : sms);
   const HalfBook hb = make_halfbook(ctx);
-  auto run = [&](auto kern) {
-    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmemBytes));
-    kern<<<grid, kThreadsTc, kSmemBytes, st>>>(map, n, ctx->dBimg, hb, payload, norms, ctx->dstatus);
+  auto run = [&](auto kern, auto f) {
+    using QL = QLayout<decltype(f)::value>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(QL::kSmem));
+    kern<<<grid, QL::kThreads, QL::kSmem, st>>>(map, n, ctx->dBimg, hb, payload, norms, ctx->dstatus,
+                                                ctx->wait_budget);
   };
   const bool jl = ctx->m > 0;
-  switch (ctx->bmse * 2 + (jl ? 1 : 0)) {
-    case 2: run(quantize_tc_kernel<1, false>); break;
-    case 3: run(quantize_tc_kernel<1, true>); break;
-    case 4: run(quantize_tc_kernel<2, false>); break;
-    case 5: run(quantize_tc_kernel<2, true>); break;
-    case 6: run(quantize_tc_kernel<3, false>); break;
-    default: run(quantize_tc_kernel<3, true>); break;
-  }
+  auto go = [&](auto f) {
+    constexpr bool F = decltype(f)::value;
+    switch (ctx->bmse * 2 + (jl ? 1 : 0)) {
+      case 2: run(quantize_tc_kernel<1, false, F>, f); break;
+      case 3: run(quantize_tc_kernel<1, true, F>, f); break;
+      case 4: run(quantize_tc_kernel<2, false, F>, f); break;
+      case 5: run(quantize_tc_kernel<2, true, F>, f); break;
+      case 6: run(quantize_tc_kernel<3, false, F>, f); break;
+      default: run(quantize_tc_kernel<3, true, F>, f); break;
+    }
+  };
+  if (f32)
+    go(std::true_type{});
+  else
+    go(std::false_type{});
   return cudaGetLastError();
 }
 

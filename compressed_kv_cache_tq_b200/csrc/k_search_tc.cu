@@ -192,36 +192,25 @@ __device__ __forceinline__ float key_float(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
-// Work: the rows are swept by all CTAs together, block by block, so that the
-// query tiles' reads of one row tile meet in L2: row tiles are cut into
-// blocks of kSweep; within block beta (Wb row tiles) the Q Wb units (query
-// tile, row tile) are ordered query-tile-major and CTA c of C takes the
-// contiguous range [(Q Wb c + r) / C, (Q Wb (c + 1) + r) / C), r = 61 beta
-// mod C (rotating which CTAs round up); odd blocks run the range backwards,
-// so a CTA that spans two query tiles switches once per block.
-constexpr int64_t kSweep = 64;
+// Work: unit u = (query tile u / row_tiles, row tile u % row_tiles); CTA b
+// takes the contiguous units [U b / G, U (b + 1) / G) of the U = qtiles x
+// row_tiles, so it keeps one query tile (or two) for long stretches.  (A
+// part-major round-robin order that makes all CTAs stream the same rows at
+// the same time measured slower: 17.0 against 13.7 ms at 10^6 x 10^4.)
 struct Units {
-  int64_t Q, T, C, c, nb;
-  int64_t beta, i0, n, cur;
+  int64_t row_tiles, u, u1;
   int64_t qt, t;
-  __device__ Units(int64_t qtiles, int64_t row_tiles, int64_t cta, int64_t ctas)
-      : Q(qtiles), T(row_tiles), C(ctas), c(cta), nb((row_tiles + kSweep - 1) / kSweep), beta(-1), i0(0), n(0),
-        cur(0), qt(0), t(0) {}
+  __device__ Units(int64_t qtiles, int64_t row_tiles_, int64_t cta, int64_t ctas) : row_tiles(row_tiles_) {
+    const int64_t total = qtiles * row_tiles_;
+    u = total * cta / ctas - 1;
+    u1 = total * (cta + 1) / ctas;
+    qt = t = 0;
+  }
   // advance to the next (query tile, row tile); false when done
   __device__ bool next() {
-    while (cur >= n) {
-      if (++beta >= nb) return false;
-      const int64_t wb = (beta + 1) * kSweep <= T ? kSweep : T - beta * kSweep;
-      const int64_t u = Q * wb, r = (beta * 61) % C;
-      i0 = (u * c + r) / C;
-      n = (u * (c + 1) + r) / C - i0;
-      cur = 0;
-    }
-    const int64_t wb = (beta + 1) * kSweep <= T ? kSweep : T - beta * kSweep;
-    const int64_t idx = (beta & 1) ? i0 + n - 1 - cur : i0 + cur;
-    ++cur;
-    qt = idx / wb;
-    t = beta * kSweep + (idx - qt * wb);
+    if (++u >= u1) return false;
+    qt = u / row_tiles;
+    t = u - qt * row_tiles;
     return true;
   }
 };

@@ -53,16 +53,45 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
   }
   return ok != 0;
 }
+// Non-blocking test of the phase (never suspends the thread).
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.b32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait by non-blocking tests only, for short budgets (a try_wait may
+// suspend the thread for longer than the budget before it returns).
+__device__ __forceinline__ bool mbar_wait_polling(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                                  uint32_t* status, uint32_t status_bit, long long budget) {
+  const long long t0 = clock64();
+  while (!mbar_test(bar, parity)) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > budget) {
+      *abort_flag = 1;
+      atomicOr(status, status_bit);
+      return false;
+    }
+  }
+  return true;
+}
+
 // Bounded wait: false when the budget ran out or another role gave up (the
 // one that gives up sets `abort_flag` and ORs `status_bit` into `*status`).
+// budget: SM clock cycles to spin before giving up.
 template <bool kSuspend = true>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          uint32_t* status, uint32_t status_bit) {
+                                          uint32_t* status, uint32_t status_bit, long long budget = kWaitCycles) {
   if (mbar_try<kSuspend>(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try<kSuspend>(bar, parity)) {
     if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitCycles) {
+    if (clock64() - t0 > budget) {
       *abort_flag = 1;
       atomicOr(status, status_bit);
       return false;
@@ -74,8 +103,9 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 // lane leaves its loop while the others go on into warp-synchronous instructions.
 template <bool kSuspend = true>
 __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                               uint32_t* status, uint32_t status_bit) {
-  return __all_sync(0xFFFFFFFFu, mbar_wait<kSuspend>(bar, parity, abort_flag, status, status_bit));
+                                               uint32_t* status, uint32_t status_bit,
+                                               long long budget = kWaitCycles) {
+  return __all_sync(0xFFFFFFFFu, mbar_wait<kSuspend>(bar, parity, abort_flag, status, status_bit, budget));
 }
 // Bounded wait that ignores the abort flag: used before the CTA exits, so that
 // no copy or MMA is still in flight when shared and tensor memory are released.

@@ -56,6 +56,7 @@ struct tq_ctx {
   double* dc64 = nullptr;
   uint8_t* dBimg = nullptr; // tensor-core B operands (d = m = 128): R_hi, R_lo (bf16), P (fp16), smem image
   uint32_t* dstatus = nullptr;
+  long long wait_budget = 0;   // tensor-core quantizer: cycles a wait spins before giving up (0: default)
   tq::CodebookParams cb;
   tq::CodeLut lut;
 };

@@ -394,6 +394,12 @@ tq_status tq_export_tables(const tq_ctx* ctx, double* R, double* P, double* c, d
   return TQ_OK;
 }
 
+tq_status tq_set_wait_budget(tq_ctx* ctx, int64_t cycles) {
+  if (!ctx || cycles < 0) return TQ_ERR_ARG;
+  ctx->wait_budget = cycles;
+  return TQ_OK;
+}
+
 tq_status tq_check_device_status(const tq_ctx* ctx, void* stream, uint32_t* word) {
   if (!ctx) return TQ_ERR_ARG;
   uint32_t h = 0;

@@ -59,6 +59,7 @@ def lib() -> ctypes.CDLL:
             "tq_topk_workspace_bytes": (sz, [vp, i64, i64, i32]),
             "tq_topk": (i32, [vp, vp, i64, vp, vp, i64, i32, vp, vp, vp, sz, vp]),
             "tq_check_device_status": (i32, [vp, vp, ctypes.POINTER(u32)]),
+            "tq_set_wait_budget": (i32, [vp, i64]),
             "tq_topk_merge": (i32, [vp, vp, vp, i32, i64, i32, vp, vp, vp]),
             "tq_attend_workspace_bytes": (sz, [vp, i32, i32, i32, i64]),
             "tq_attend": (i32, [vp, vp, i32, i32, i32, i64, vp, vp, vp, vp, sz, vp]),
@@ -84,7 +85,7 @@ def lib() -> ctypes.CDLL:
 
 EXPORTED = ["tq_init", "tq_init_ex", "tq_host_tables", "tq_free", "tq_info", "tq_export_tables", "tq_quantize", "tq_dequantize",
             "tq_logits_workspace_bytes", "tq_logits", "tq_logits_noalloc", "tq_topk_workspace_bytes", "tq_topk",
-            "tq_check_device_status", "tq_strerror", "tq_last_cuda_error", "tq_topk_merge",
+            "tq_check_device_status", "tq_set_wait_budget", "tq_strerror", "tq_last_cuda_error", "tq_topk_merge",
             "tq_attend_workspace_bytes", "tq_attend",
             "tq_split_create", "tq_split_free",
             "tq_split_plan_workspace_bytes", "tq_split_plan", "tq_split_set_plan", "tq_split_get_plan",

@@ -348,6 +348,19 @@ tq_status tq_topk_merge(const float* scores, const int64_t* ids, const int64_t* 
  * NULL).  Errors: TQ_ERR_ARG (ctx NULL), TQ_ERR_CUDA. */
 tq_status tq_check_device_status(const tq_ctx* ctx, void* stream, uint32_t* word);
 
+/* Test hook for the failure path of the bounded waits: the number of SM
+ * clock cycles each bounded wait of the tensor-core quantizer (tq_quantize
+ * on d = 128) spins before it gives up; 0 restores the default (about 2 s).
+ * A wait that gives up makes every role of the kernel leave its loop (the
+ * copies and MMAs already issued are drained with the default budget before
+ * the block exits), the rows of that call are left incomplete, and the
+ * context's status word gets TQ_STATUS_QUANTIZE_WAIT, so that
+ * tq_check_device_status returns TQ_ERR_DEVICE; the context stays usable.
+ * With a budget of a few cycles the first wait that is not satisfied at once
+ * gives up.  Not for production use; must not race with calls on ctx.
+ * Errors: TQ_ERR_ARG (ctx NULL, cycles < 0). */
+tq_status tq_set_wait_budget(tq_ctx* ctx, int64_t cycles);
+
 const char* tq_strerror(tq_status s);
 const char* tq_last_cuda_error(void);
 

@@ -737,7 +737,20 @@ def pack_norms(n16: np.ndarray, rho16: np.ndarray) -> np.ndarray:
 
 CODE_BAND = 1e-5     # |u_j - t_i| on the unit-sphere scale
 SIGN_BAND = 1e-5     # |(S r)_i| / (||s_i|| ||r||): cosine between the JL row and the residual
-NORM_BAND = 1e-5     # relative distance of the exact norm to an fp16 rounding midpoint
+NORM_BAND = 1e-5     # distance of the exact norm to an fp16 rounding midpoint, on the unit-sphere scale
+
+
+def norm_band(n: np.ndarray, rho: np.ndarray):
+    """Relative bands of the two stored norms (reading of the same 1e-5 on
+    the unit-sphere scale as the code band): ||k|| / ||k|| = 1 is the scale of
+    ||k||, so its band is 1e-5 relative; ||r|| / ||k|| is the length of the
+    residual on the unit sphere, so a band of 1e-5 there is 1e-5 ||k|| / ||r||
+    relative to ||r||.  Returns (band_n, band_rho) per key."""
+    n = np.asarray(n, dtype=np.float64)
+    rho = np.asarray(rho, dtype=np.float64)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        band_rho = np.where(rho > 0, NORM_BAND * n / np.where(rho > 0, rho, 1.0), 0.0)
+    return np.full(n.shape, NORM_BAND), band_rho
 
 
 def code_boundary_distance(u: np.ndarray, t: np.ndarray) -> np.ndarray:

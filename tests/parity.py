@@ -22,8 +22,9 @@ def check_quantize(payload, norms, K64, tb: O.Tables, report=None):
 
     Codes must be equal except within CODE_BAND of a boundary; sign bits equal
     except within SIGN_BAND of 0 (cosine of the JL row and the residual) or in
-    a key with an excused code difference; fp16 norms equal except within
-    NORM_BAND of a rounding midpoint (then one ulp either way).  Mismatching
+    a key with an excused code difference; fp16 norms equal except near a
+    rounding midpoint (O.norm_band: 1e-5 on the unit-sphere scale; then one
+    ulp either way).  Mismatching
     coordinates must stay below 1e-4.
 
     Returns (stats, quantized): stats holds the fractions the benchmark spec asks
@@ -55,18 +56,20 @@ def check_quantize(payload, norms, K64, tb: O.Tables, report=None):
     assert frac_sign < MISMATCH_LIMIT, frac_sign
     narrow = np.abs(qz.z) <= 1e-5 * qz.rho[:, None]
 
-    def norm_ok(gpu16, exact, excused):
+    band_n, band_rho = O.norm_band(qz.n, qz.rho)
+
+    def norm_ok(gpu16, exact, excused, band):
         want = exact.astype(np.float16)
         same = gpu16 == want
-        near = O.fp16_midpoint_distance(exact) <= O.NORM_BAND
+        near = O.fp16_midpoint_distance(exact) <= band
         one_ulp = np.abs(gpu16.astype(np.float64) - want.astype(np.float64)) <= \
             np.abs(np.spacing(want).astype(np.float64)) * 1.0001
         ok = same | (near & one_ulp) | excused
         return ok, same
 
-    nk_ok, nk_same = norm_ok(norms[:, 0], qz.n, np.zeros(len(qz.n), bool))
+    nk_ok, nk_same = norm_ok(norms[:, 0], qz.n, np.zeros(len(qz.n), bool), band_n)
     assert nk_ok.all(), f"||k|| differs: {np.argwhere(~nk_ok)[:5].ravel()}"
-    nr_ok, nr_same = norm_ok(norms[:, 1], qz.rho, key_exc)
+    nr_ok, nr_same = norm_ok(norms[:, 1], qz.rho, key_exc, band_rho)
     assert nr_ok.all(), f"||r|| differs: {np.argwhere(~nr_ok)[:5].ravel()}"
     stats = dict(keys=int(len(qz.n)), coords=int(code_mis.size), sign_bits=int(sign_mis.size),
                  code_mismatch=frac_code, sign_mismatch=frac_sign,

@@ -67,6 +67,7 @@ def test_argument_validation_without_device(L):
     assert lib.tq_logits(None, None, 1, 4, 1, 10, None, None, 1.0, None, None, 0, None) == 1
     assert lib.tq_logits_noalloc(None, None, 1, 4, 1, 10, None, None, 1.0, None, None) == 1
     assert lib.tq_check_device_status(None, None, None) == 1
+    assert lib.tq_set_wait_budget(None, 0) == 1
     assert lib.tq_strerror(7) == b"a norm exceeded the fp16 range"
     assert lib.tq_info(None, None, None, None, None) == 1
     assert lib.tq_strerror(5) == b"workspace too small"

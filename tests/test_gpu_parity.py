@@ -37,20 +37,47 @@ def test_device_tables_match_oracle(lib):
     assert np.max(np.abs(c - tb.c)) < 1e-12 and np.max(np.abs(t - tb.t)) < 1e-12
 
 
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
 @pytest.mark.parametrize("m", [128, 0])
 @pytest.mark.parametrize("bits", [2, 3, 4])
 @pytest.mark.parametrize("n", [1, 127, 441, 4133])
-def test_quantize_bf16_tensor_core_path(lib, bits, n, m):
-    """d = 128 bf16 keys on the tensor-core quantizer, with the sign sketch
-    (m = 128) and without it (m = 0, the MSE-only variant)."""
+def test_quantize_tensor_core_path(lib, bits, n, m, dtype):
+    """d = 128 keys on the tensor-core quantizer, bf16 keys and fp32 keys (split
+    into bf16 hi + lo on the way in), with the sign sketch (m = 128) and
+    without it (m = 0, the MSE-only variant)."""
     ctx = _ctx(lib, bits=bits, seed=7 + bits, m=m)
     scales = W.head_channel_scales(1, 128, seed=3)
     k32 = W.decode_keys_pair(0, 0, n, 128, scales, seed=3 + n)
-    kb = torch.from_numpy(k32).to(torch.bfloat16)
+    kb = torch.from_numpy(k32).to(dtype)
     payload, norms = lib.tq_quantize(ctx, kb.to(DEV))
     _status_clean(lib, ctx)
     rep = {}
     check_quantize(payload.cpu().numpy(), norms.cpu().numpy(), kb.to(torch.float64).numpy(), tables_of(ctx), rep)
+
+
+@pytest.mark.parametrize("bits", [3, 4])
+def test_quantize_fp32_strided_and_ragged(lib, bits):
+    """fp32 keys with a leading dimension above d (TMA rows 544 bytes apart)
+    and a ragged last tile, against the oracle; equal to the rows quantised
+    from a contiguous copy."""
+    ctx = _ctx(lib, bits=bits, seed=9)
+    n, ld = 3 * 128 + 77, 136
+    k = W.toy_keys(n, 128, seed=21)
+    wide = torch.zeros((n, ld), dtype=torch.float32)
+    wide[:, :128] = torch.from_numpy(k)
+    dev = wide.to(DEV)
+    payload = torch.empty((n, ctx.row_bytes), dtype=torch.uint8, device=DEV)
+    norms = torch.empty((n, 2), dtype=torch.float16, device=DEV)
+    import ctypes
+
+    st = lib.lib().tq_quantize(ctx.handle, ctypes.c_void_p(dev.data_ptr()), 0, n, ld,
+                               ctypes.c_void_p(payload.data_ptr()), ctypes.c_void_p(norms.data_ptr()),
+                               ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0
+    _status_clean(lib, ctx)
+    check_quantize(payload.cpu().numpy(), norms.cpu().numpy(), k.astype(np.float64), tables_of(ctx))
+    p2, n2 = lib.tq_quantize(ctx, torch.from_numpy(k).to(DEV))
+    assert torch.equal(p2, payload) and torch.equal(n2.view(torch.int16), norms.view(torch.int16))
 
 
 def test_quantize_toy_fp32(lib):
@@ -130,6 +157,32 @@ def test_quantize_flags_norms_out_of_fp16_range(lib, dtype, d, m):
     nr = norms.cpu().numpy().view(np.float16)
     assert np.isinf(nr[333, 0]) and np.all(np.isfinite(np.delete(nr, 333, axis=0)))
     assert lib.tq_check_device_status(ctx) == 0
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_bounded_wait_gives_up_and_context_recovers(lib, dtype):
+    """The failure path of the tensor-core quantizer's bounded waits, forced
+    with the test hook: with a wait budget of a few cycles the first wait that
+    is not satisfied at once gives up, every role leaves its loop, the kernel
+    returns, and the status word reports it (TQ_ERR_DEVICE); with the default
+    budget restored the next call on the same context is complete and equal
+    to the oracle."""
+    import ctypes
+
+    L = lib.lib()
+    ctx = _ctx(lib, bits=4, seed=12)
+    kt = torch.from_numpy(W.toy_keys(4133, 128, seed=31)).to(dtype)
+    assert L.tq_set_wait_budget(ctx.handle, -1) == 1
+    assert L.tq_set_wait_budget(ctx.handle, 4) == 0
+    lib.tq_quantize(ctx, kt.to(DEV))
+    torch.cuda.synchronize()
+    w = ctypes.c_uint32()
+    assert L.tq_check_device_status(ctx.handle, None, ctypes.byref(w)) == 6   # TQ_ERR_DEVICE
+    assert w.value & lib.STATUS_QUANTIZE_WAIT
+    assert L.tq_set_wait_budget(ctx.handle, 0) == 0
+    payload, norms = lib.tq_quantize(ctx, kt.to(DEV))
+    _status_clean(lib, ctx)
+    check_quantize(payload.cpu().numpy(), norms.cpu().numpy(), kt.to(torch.float64).numpy(), tables_of(ctx))
 
 
 def test_quantize_is_deterministic(lib):

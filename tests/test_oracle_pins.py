@@ -585,6 +585,14 @@ def test_sign_boundary_distance_is_the_cosine():
     assert np.all(np.isinf(dist[2]))   # zero residual: never excused
 
 
+def test_norm_band_is_one_unit_sphere_band():
+    # ||k|| = 10, ||r|| = 2: ||r|| / ||k|| = 0.2 on the unit sphere; a 1e-5 band
+    # there is 1e-5 * 10 / 2 = 5e-5 relative to ||r||; a zero residual has none
+    bn, br = O.norm_band(np.array([10.0, 3.0]), np.array([2.0, 0.0]))
+    np.testing.assert_allclose(bn, [1e-5, 1e-5], rtol=0, atol=0)
+    np.testing.assert_allclose(br, [5e-5, 0.0], rtol=1e-15, atol=0)
+
+
 def test_fp16_midpoint_distance_hand_values():
     f = O.fp16_midpoint_distance
     # exact midpoints: 1 + 2^-11 (between 1 and 1 + 2^-10), 2049 (between 2048
