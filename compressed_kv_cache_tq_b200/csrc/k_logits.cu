@@ -283,6 +283,12 @@ __device__ __forceinline__ void load_chunk(Chunk<BMSE, JL>& c, const uint8_t* ro
 // Only the low 16 bits of a selector are read by the permute, so a word can
 // be masked once for both of its halfwords, and the upper halfword of a word
 // needs only a shift.
+// Byte-permute selectors (4 nibbles, mode bit clear) of the 8 code registers
+// of a quarter: nibble e of selector r is the code of coordinate (r, e).
+// Only the low 16 bits of a selector are read by the permute, so a word can
+// be masked once for both of its halfwords, and the upper halfword of a word
+// needs only a shift.  (Shifts as multiply-highs on the FMA pipe measured
+// slower: their latency lengthens the dependency chains.)
 template <int BMSE, bool JL>
 __device__ __forceinline__ void code_selectors(const Chunk<BMSE, JL>& c, uint32_t (&sel)[8]) {
   if constexpr (BMSE == 3) {
@@ -626,8 +632,10 @@ constexpr int GD = 64;          // group dimension of the split fast path
 constexpr int GKS = GD / 32;    // k-steps per group
 
 struct SplitScale {
-  float code[2];   // per group (0 high, 1 low): multiplies the int32 code dot product
-  float sign[2];
+  float code[2];     // per group (0 high, 1 low): multiplies the code dot product
+  float sign[2];     // multiplies the sign dot product
+  int32_t ccode[2];  // one-bit codes: integer correction of the code dot product (as in qprep_kernel)
+  int32_t csign[2];  // integer correction of the sign dot product
 };
 
 // Query preparation of the split: per (batch, KV head) group, the query's
@@ -644,12 +652,13 @@ __global__ void __launch_bounds__(128) qprep_split_kernel(const float* __restric
                                                           const float* __restrict__ Pt_hi,
                                                           const float* __restrict__ Rt_lo,
                                                           const float* __restrict__ Pt_lo, float inv_hi, float inv_lo,
-                                                          float scale, float qjl_hi, float qjl_lo,
-                                                          uint32_t* __restrict__ frags,
+                                                          float scale, float qjl_hi, float qjl_lo, int one_bit_hi,
+                                                          int one_bit_lo, uint32_t* __restrict__ frags,
                                                           SplitScale* __restrict__ hscale) {
   __shared__ float sq[kMaxSlots][2 * GD];   // gathered queries [high | low]
   __shared__ float sx[kMaxSlots][2 * GD];
   __shared__ float red[2][kMaxSlots][4];
+  __shared__ int ired[4][kMaxSlots][4];     // [Y, Y3, X, X3][slot][warp]
   __shared__ int8_t limbs[kMaxSlots][2][2][2 * GD];   // [slot][x/y][hi/lo limb][coordinate of high | low]
   const int G = Hq / Hkv;
   const int slots = nt_per_group * HPT;
@@ -707,11 +716,27 @@ __global__ void __launch_bounds__(128) qprep_split_kernel(const float* __restric
     const float ky = my > 0.f ? 32000.f / my : 0.f;
     const int xi = __float2int_rn(acc[h] * kx);
     const int yi = __float2int_rn(accy[h] * ky);
-    const int xh = (xi + 128) >> 8, yh = (yi + 128) >> 8;
+    // the B operand holds -y (and -x for a group of one-bit codes): the
+    // one-bit operand form of qprep_kernel
+    const int xb = (gi ? one_bit_lo : one_bit_hi) ? -xi : xi, yb = -yi;
+    const int xh = (xb + 128) >> 8, yh = (yb + 128) >> 8;
     limbs[h][0][0][tid] = int8_t(xh);
-    limbs[h][0][1][tid] = int8_t(xi - 256 * xh);
+    limbs[h][0][1][tid] = int8_t(xb - 256 * xh);
     limbs[h][1][0][tid] = int8_t(yh);
-    limbs[h][1][1][tid] = int8_t(yi - 256 * yh);
+    limbs[h][1][1][tid] = int8_t(yb - 256 * yh);
+    int ty = yi, ty3 = reg3_coordinate(j) ? yi : 0, tx = xi, tx3 = reg3_coordinate(j) ? xi : 0;
+    for (int o = 16; o; o >>= 1) {
+      ty += __shfl_xor_sync(0xffffffffu, ty, o);
+      ty3 += __shfl_xor_sync(0xffffffffu, ty3, o);
+      tx += __shfl_xor_sync(0xffffffffu, tx, o);
+      tx3 += __shfl_xor_sync(0xffffffffu, tx3, o);
+    }
+    if (lane == 0) {
+      ired[0][h][warp] = ty;
+      ired[1][h][warp] = ty3;
+      ired[2][h][warp] = tx;
+      ired[3][h][warp] = tx3;
+    }
     if (j == 0 && h < G) {
       SplitScale* hs = hscale + size_t(b) * Hq + hkv * G + h;
       hs->code[gi] = mx > 0.f ? scale * (gi ? inv_lo : inv_hi) / kx : 0.f;
@@ -719,6 +744,18 @@ __global__ void __launch_bounds__(128) qprep_split_kernel(const float* __restric
     }
   }
   __syncthreads();
+  // group gi's integer corrections from its two warps' sums
+  if (j == 0) {
+#pragma unroll
+    for (int h = 0; h < kMaxSlots; ++h) {
+      if (h >= slots || h >= G) break;
+      SplitScale* hs = hscale + size_t(b) * Hq + hkv * G + h;
+      const int Y = ired[0][h][2 * gi] + ired[0][h][2 * gi + 1], Y3 = ired[1][h][2 * gi] + ired[1][h][2 * gi + 1];
+      const int X = ired[2][h][2 * gi] + ired[2][h][2 * gi + 1], X3 = ired[3][h][2 * gi] + ired[3][h][2 * gi + 1];
+      hs->ccode[gi] = 2 * X3 - X;
+      hs->csign[gi] = 2 * Y3 - Y;
+    }
+  }
   for (int w = tid; w < nt_per_group * kFragWords; w += 128) {
     const int ln = w & 31, reg = (w >> 5) & 1, st = (w >> 6) & 1, xy = (w >> 7) & 1, g2 = (w >> 8) & 1;
     const int nt = w >> 9;
@@ -772,49 +809,61 @@ __device__ __forceinline__ void gcode_selectors(const GChunk<BM>& c, uint32_t (&
     sel[1] = (c.h(0) >> 2) & 0x3333u;
     sel[2] = c.h(1) & 0x3333u;
     sel[3] = (c.h(1) >> 2) & 0x3333u;
-  } else {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) sel[i] = (c.h(0) >> i) & 0x1111u;
   }
 }
 
-template <int BM>
-__device__ __forceinline__ void gsign_operands(const GChunk<BM>& c, uint32_t (&a)[4]) {
-  const uint32_t h = c.h(BM);
-  a[0] = prmt(0x000001FFu, 0u, h & 0x1111u);
-  a[1] = prmt(0x000100FFu, 0u, h & 0x2222u);
-  a[2] = prmt(0x000000FFu, 0x00000001u, h & 0x4444u);
-  a[3] = prmt(0x000000FFu, 0x00000001u, (h >> 1) & 0x4444u);
+// The one-bit operand form (see bit_operands) for the 4 registers of one unit.
+__device__ __forceinline__ void bit_operands4(uint32_t h, uint32_t (&a)[4]) {
+  a[0] = prmt(0xFF00FF00u, 0xFF00FF00u, h);
+  a[1] = prmt(0xFFFF0000u, 0xFFFF0000u, h);
+  a[2] = prmt(0x00000000u, 0xFFFFFFFFu, h);
+  a[3] = prmt(0x01010101u, 0x01010101u, h);
 }
 
-// Products of one group for a 16-key row tile: code planes (hi, lo) and signs.
+// Products of one group for a 16-key row tile: code planes (hi, lo; one-bit
+// codes: one plane in the one-bit form, in ah) and signs.
 template <int BM, int NT>
 __device__ __forceinline__ void group_mma(const GChunk<BM>& ca, const GChunk<BM>& cb, const CodeLut& lut,
                                           const uint32_t (&bx)[NT][GKS][2], const uint32_t (&by)[NT][GKS][2],
                                           int (&ah)[NT][4], int (&al)[NT][4], int (&sg)[NT][4]) {
-  uint32_t sa[4], sb[4];
-  gcode_selectors<BM>(ca, sa);
-  gcode_selectors<BM>(cb, sb);
+  if constexpr (BM >= 2) {
+    uint32_t sa[4], sb[4];
+    gcode_selectors<BM>(ca, sa);
+    gcode_selectors<BM>(cb, sb);
 #pragma unroll
-  for (int s = 0; s < GKS; ++s) {
-    const uint32_t h0 = prmt(lut.hi[0], lut.hi[1], sa[2 * s]), h1 = prmt(lut.hi[0], lut.hi[1], sb[2 * s]);
-    const uint32_t h2 = prmt(lut.hi[0], lut.hi[1], sa[2 * s + 1]), h3 = prmt(lut.hi[0], lut.hi[1], sb[2 * s + 1]);
-    const uint32_t l0 = prmt(lut.lo[0], lut.lo[1], sa[2 * s]), l1 = prmt(lut.lo[0], lut.lo[1], sb[2 * s]);
-    const uint32_t l2 = prmt(lut.lo[0], lut.lo[1], sa[2 * s + 1]), l3 = prmt(lut.lo[0], lut.lo[1], sb[2 * s + 1]);
+    for (int s = 0; s < GKS; ++s) {
+      const uint32_t h0 = prmt(lut.hi[0], lut.hi[1], sa[2 * s]), h1 = prmt(lut.hi[0], lut.hi[1], sb[2 * s]);
+      const uint32_t h2 = prmt(lut.hi[0], lut.hi[1], sa[2 * s + 1]), h3 = prmt(lut.hi[0], lut.hi[1], sb[2 * s + 1]);
+      const uint32_t l0 = prmt(lut.lo[0], lut.lo[1], sa[2 * s]), l1 = prmt(lut.lo[0], lut.lo[1], sb[2 * s]);
+      const uint32_t l2 = prmt(lut.lo[0], lut.lo[1], sa[2 * s + 1]), l3 = prmt(lut.lo[0], lut.lo[1], sb[2 * s + 1]);
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      if (s == 0) {
-        mma_s8_first(ah[nt], h0, h1, h2, h3, bx[nt][s][0], bx[nt][s][1]);
-        mma_s8_first(al[nt], l0, l1, l2, l3, bx[nt][s][0], bx[nt][s][1]);
-      } else {
-        mma_s8(ah[nt], h0, h1, h2, h3, bx[nt][s][0], bx[nt][s][1]);
-        mma_s8(al[nt], l0, l1, l2, l3, bx[nt][s][0], bx[nt][s][1]);
+      for (int nt = 0; nt < NT; ++nt) {
+        if (s == 0) {
+          mma_s8_first(ah[nt], h0, h1, h2, h3, bx[nt][s][0], bx[nt][s][1]);
+          mma_s8_first(al[nt], l0, l1, l2, l3, bx[nt][s][0], bx[nt][s][1]);
+        } else {
+          mma_s8(ah[nt], h0, h1, h2, h3, bx[nt][s][0], bx[nt][s][1]);
+          mma_s8(al[nt], l0, l1, l2, l3, bx[nt][s][0], bx[nt][s][1]);
+        }
       }
     }
+  } else {
+    uint32_t ca4[4], cb4[4];
+    bit_operands4(ca.h(0), ca4);
+    bit_operands4(cb.h(0), cb4);
+#pragma unroll
+    for (int s = 0; s < GKS; ++s)
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        if (s == 0)
+          mma_s8_first(ah[nt], ca4[0], cb4[0], ca4[1], cb4[1], bx[nt][0][0], bx[nt][0][1]);
+        else
+          mma_s8(ah[nt], ca4[2 * s], cb4[2 * s], ca4[2 * s + 1], cb4[2 * s + 1], bx[nt][s][0], bx[nt][s][1]);
+      }
   }
   uint32_t ga[4], gb[4];
-  gsign_operands<BM>(ca, ga);
-  gsign_operands<BM>(cb, gb);
+  bit_operands4(ca.h(BM), ga);
+  bit_operands4(cb.h(BM), gb);
 #pragma unroll
   for (int s = 0; s < GKS; ++s)
 #pragma unroll
@@ -826,16 +875,23 @@ __device__ __forceinline__ void group_mma(const GChunk<BM>& ca, const GChunk<BM>
     }
 }
 
-__device__ __forceinline__ float limb_sum(const int (&a)[4], const int (&b)[4], int r) {
-  // |cross terms| <= 2 * 64 * 128 * 128 and |low terms| < 2^20: the integer sums fit in 32 bits
-  return fmaf(float(a[r]), 65536.f, float((a[r + 1] + b[r]) * 256 + b[r + 1]));
+// Code dot product of key row r (0: key g, 2: key g + 8) of a group.
+template <int BM>
+__device__ __forceinline__ float group_code(const int (&a)[4], const int (&b)[4], int r, int ccode) {
+  if constexpr (BM >= 2)   // |cross terms| <= 2 * 64 * 128 * 128 and |low terms| < 2^20: the sums fit in 32 bits
+    return fmaf(float(a[r]), 65536.f, float((a[r + 1] + b[r]) * 256 + b[r + 1]));
+  else
+    return float(2 * (a[r] * 256 + a[r + 1]) + ccode);
+}
+__device__ __forceinline__ float group_sign(const int (&a)[4], int r, int csign) {
+  return float(2 * (a[r] * 256 + a[r + 1]) + csign);
 }
 
 template <int BHI, int BLO, int NT>
 __device__ __forceinline__ void split_row_tile(const GChunk<BHI>& ha, const GChunk<BHI>& hb, const GChunk<BLO>& la,
                                                const GChunk<BLO>& lb, uint32_t nha, uint32_t nhb, uint32_t nla,
                                                uint32_t nlb, bool okA, bool okB, const uint32_t (&bx)[2][NT][GKS][2],
-                                               const uint32_t (&by)[2][NT][GKS][2], const float (&sc)[NT][4],
+                                               const uint32_t (&by)[2][NT][GKS][2], const SplitScale (&sc)[NT],
                                                float* const (&orow)[NT], int g, const CodeLut& lut_hi,
                                                const CodeLut& lut_lo) {
   int hh[NT][4], hl[NT][4], hs[NT][4], lh[NT][4], ll[NT][4], ls[NT][4];
@@ -848,14 +904,15 @@ __device__ __forceinline__ void split_row_tile(const GChunk<BHI>& ha, const GChu
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
     if (!orow[nt]) continue;
-    const float vA = fmaf(fha.x * sc[nt][0], limb_sum(hh[nt], hl[nt], 0),
-                          fmaf(fha.y * sc[nt][1], float(hs[nt][0] * 256 + hs[nt][1]),
-                               fmaf(fla.x * sc[nt][2], limb_sum(lh[nt], ll[nt], 0),
-                                    fla.y * sc[nt][3] * float(ls[nt][0] * 256 + ls[nt][1]))));
-    const float vB = fmaf(fhb.x * sc[nt][0], limb_sum(hh[nt], hl[nt], 2),
-                          fmaf(fhb.y * sc[nt][1], float(hs[nt][2] * 256 + hs[nt][3]),
-                               fmaf(flb.x * sc[nt][2], limb_sum(lh[nt], ll[nt], 2),
-                                    flb.y * sc[nt][3] * float(ls[nt][2] * 256 + ls[nt][3]))));
+    const SplitScale& c = sc[nt];
+    const float vA = fmaf(fha.x * c.code[0], group_code<BHI>(hh[nt], hl[nt], 0, c.ccode[0]),
+                          fmaf(fha.y * c.sign[0], group_sign(hs[nt], 0, c.csign[0]),
+                               fmaf(fla.x * c.code[1], group_code<BLO>(lh[nt], ll[nt], 0, c.ccode[1]),
+                                    fla.y * c.sign[1] * group_sign(ls[nt], 0, c.csign[1]))));
+    const float vB = fmaf(fhb.x * c.code[0], group_code<BHI>(hh[nt], hl[nt], 2, c.ccode[0]),
+                          fmaf(fhb.y * c.sign[0], group_sign(hs[nt], 2, c.csign[0]),
+                               fmaf(flb.x * c.code[1], group_code<BLO>(lh[nt], ll[nt], 2, c.ccode[1]),
+                                    flb.y * c.sign[1] * group_sign(ls[nt], 2, c.csign[1]))));
     if (okA) orow[nt][g] = vA;
     if (okB) orow[nt][g + 8] = vB;
   }
@@ -899,7 +956,7 @@ __global__ void __launch_bounds__(kLogitThreads, NT == 1 ? 2 : 1) logits_split_k
   if (t_begin >= t_end) return;
 
   uint32_t bx[2][NT][GKS][2], by[2][NT][GKS][2];
-  float sc[NT][4];
+  SplitScale sc[NT];
   float* orow[NT];
   auto load_group = [&](int64_t gi) {
     const int b = int(gi / Hkv), hkv = int(gi - int64_t(b) * Hkv);
@@ -917,11 +974,7 @@ __global__ void __launch_bounds__(kLogitThreads, NT == 1 ? 2 : 1) logits_split_k
           }
       const int hg = nt * HPT + tig;
       const int hh = hg < G ? hg : 0;
-      const SplitScale hs = hscale[size_t(b) * Hq + hkv * G + hh];
-      sc[nt][0] = hs.code[0];
-      sc[nt][1] = hs.sign[0];
-      sc[nt][2] = hs.code[1];
-      sc[nt][3] = hs.sign[1];
+      sc[nt] = hscale[size_t(b) * Hq + hkv * G + hh];
       orow[nt] = hg < G ? out + (size_t(b) * Hq + hkv * G + hh) * S : nullptr;
     }
   };
@@ -1101,8 +1154,10 @@ cudaError_t launch_split_logits(const tq_split* sp, const float* q, int B, int H
   const size_t frag_bytes = ((size_t(groups) * nt * kFragWords * 4 + 255) / 256) * 256;
   SplitScale* hs = reinterpret_cast<SplitScale*>(static_cast<uint8_t*>(ws) + frag_bytes);
   qprep_split_kernel<<<unsigned(groups), 128, 0, st>>>(
-      q, Hq, Hkv, nt, sp->dperm, sp->hi->dRt, sp->hi->dPt, sp->lo->dRt, sp->lo->dPt, sp->hi->lut.inv_scale,
-      sp->lo->lut.inv_scale, scale, float(kQjlConst / sp->hi->m), float(kQjlConst / sp->lo->m), frags, hs);
+      q, Hq, Hkv, nt, sp->dperm, sp->hi->dRt, sp->hi->dPt, sp->lo->dRt, sp->lo->dPt,
+      sp->hi->bmse == 1 ? float(sp->hi->c[1]) : sp->hi->lut.inv_scale,
+      sp->lo->bmse == 1 ? float(sp->lo->c[1]) : sp->lo->lut.inv_scale, scale, float(kQjlConst / sp->hi->m),
+      float(kQjlConst / sp->lo->m), sp->hi->bmse == 1 ? 1 : 0, sp->lo->bmse == 1 ? 1 : 0, frags, hs);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (S == 0) return cudaSuccess;
