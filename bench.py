@@ -649,7 +649,8 @@ def run_reference(args, rank):
 # current kernels, from one ncu capture at S = 16384 (1 048 576 keys); per
 # launch it scales with the keys processed.  Summary with the command:
 # profiles/traffic_decode_s16384.md.  Set to None when a kernel changes.
-DRAM_BYTES_PER_KEY = {}
+DRAM_BYTES_PER_KEY = {"decode": {"tq_quantize": (268.719872e6 + 47.794176e6) / 1048576,
+                                  "tq_logits": (71.457536e6 + 0.553472e6) / 1048576}}
 
 
 def dense_logits_context(keys4, q, reps: int = 20) -> dict:
