@@ -464,15 +464,17 @@ __global__ void __launch_bounds__(QLayout<F32>::kThreads, 1) quantize_tc_kernel(
       // ahead never overwrites sums the other half has not read yet
       float* n2buf = pn2 + (slot * 2 + int(par)) * 256;
       {
+        // both quarters loaded before one wait (one TMEM round trip)
+        float y0[32], y1[32];
+        tmem_ld32(d1 + 32u * q0, y0);
+        tmem_ld32(d1 + 32u * (q0 + 1), y1);
+        tmem_wait32(y0);
+        tmem_wait32(y1);
         float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int qq = 0; qq < 2; ++qq) {
-          float y[32];
-          tmem_ld32(d1 + 32u * (q0 + qq), y);
-          tmem_wait32(y);
-#pragma unroll
-          for (int j = 0; j < 32; j += 2)
-            acc = __ffma2_rn(make_float2(y[j], y[j + 1]), make_float2(y[j], y[j + 1]), acc);
+        for (int j = 0; j < 32; j += 2) {
+          acc = __ffma2_rn(make_float2(y0[j], y0[j + 1]), make_float2(y0[j], y0[j + 1]), acc);
+          acc = __ffma2_rn(make_float2(y1[j], y1[j + 1]), make_float2(y1[j], y1[j + 1]), acc);
         }
         n2buf[half * 128 + row] = acc.x + acc.y;
       }
@@ -1019,6 +1021,460 @@ __global__ void __launch_bounds__(kThreadsTc, 1) quantize_split_tc_kernel(
   }
 }
 
+// ---------------------------------------------------------------------------
+// Wide quantizer: 192 < d <= 256 with m = d (the vector-search workload's
+// d = 200), fp32 keys.  The layout has dp = mp = 256 slots (four quarters of
+// 64); the products run over Np = d rounded up to 16 output coordinates and
+// input coordinates (13 k-steps at d = 200).  R_hi, R_lo (bf16) and P (fp16)
+// padded with zeros do not fit in shared memory at this size (3 x 104 KB), so
+// they stream from L2 as 64-column atoms (Np rows of 128 bytes) through a
+// three-entry ring, in the order the MMA issuer uses them: per key tile
+// R_hi / R_lo of atoms 0..3 for the rotation, then P of atoms 0..3 for the
+// JL product.  One tile at a time in tensor memory: y (then the residual's
+// fp16 hi / lo pairs) in columns [0, Np), z in [256, 256 + Np).
+//   warp 0     : TMA producer (fp32 quarter tiles, operand atoms)
+//   warp 1     : TMEM allocation, single-thread MMA issue
+//   warps 2, 3 : fp32 -> bf16 hi / lo converters (as in the fp32 path above)
+//   warps 4..19: epilogue, thread (key row, quarter): 64 layout slots of a row
+// Slots past d get code 0, sign bit 0 and no residual (the layout's padding).
+// ---------------------------------------------------------------------------
+constexpr int kWThreads = 640;
+constexpr int kWStage = 3;                      // fp32 quarter tiles (128 x 32, 16 KB)
+constexpr int kWRing = 2;                       // bf16 key atoms (hi 16 KB + lo 16 KB)
+constexpr int kWBRing = 3;                      // operand atoms (up to 256 rows x 128 B)
+constexpr uint32_t kWOffStage = 0;
+constexpr uint32_t kWOffRing = kWOffStage + 16384u * kWStage;
+constexpr uint32_t kWOffB = kWOffRing + 32768u * kWRing;
+constexpr uint32_t kWBAtomMax = 256u * 128u;
+constexpr uint32_t kWOffN2 = kWOffB + kWBAtomMax * kWBRing;   // [parity][quarter][row] partial ||y||^2
+constexpr uint32_t kWOffRR = kWOffN2 + 2u * 4u * 128u * 4u;   // [parity][quarter][row] partial ||r_rot||^2
+constexpr uint32_t kWOffBar = kWOffRR + 2u * 4u * 128u * 4u;
+constexpr uint32_t kWSmem = kWOffBar + 256 + 1024;
+static_assert(kWSmem <= 232448, "shared memory per block");
+
+enum WBar {
+  kWSFull = 0,                          // staging quarter tiles
+  kWSEmpty = kWSFull + kWStage,
+  kWRFull = kWSEmpty + kWStage,         // bf16 key atoms
+  kWREmpty = kWRFull + kWRing,
+  kWBFull = kWREmpty + kWRing,          // operand atoms
+  kWBEmpty = kWBFull + kWBRing,
+  kWD1Full = kWBEmpty + kWBRing,        // y in TMEM
+  kWN2 = kWD1Full + 1,                  // all quarters' partial ||y||^2 written
+  kWResid = kWN2 + 1,                   // residual in TMEM
+  kWD2Full = kWResid + 1,               // z in TMEM
+  kWD2Free = kWD2Full + 1,              // z read
+  kWRR = kWD2Free + 1,                  // all quarters' partial ||r_rot||^2 written
+  kWNumBars = kWRR + 1
+};
+static_assert(8 * kWNumBars + 8 <= 256, "barrier area");
+
+// Bits of the stored words that belong to slots below d, per quarter: code
+// words (2 b' per quarter) and sign words (2 per quarter).
+struct WideMasks {
+  uint32_t code[4][6];
+  uint32_t sign[4][2];
+};
+
+template <int BMSE>
+__global__ void __launch_bounds__(kWThreads, 1) quantize_wide_kernel(const __grid_constant__ CUtensorMap key_map,
+                                                                     int64_t n, int d, int np,
+                                                                     const uint8_t* __restrict__ bimg,
+                                                                     HalfBook book,
+                                                                     const __grid_constant__ WideMasks masks,
+                                                                     uint8_t* __restrict__ payload,
+                                                                     uint16_t* __restrict__ norms,
+                                                                     uint32_t* __restrict__ status,
+                                                                     long long wait_budget) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* sbase = smem_raw + (base - raw);
+  const uint32_t bar0 = base + kWOffBar;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sbase + kWOffBar + 8 * kWNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(sbase + kWOffBar + 8 * kWNumBars + 4);
+  auto bar = [&](int i) { return bar0 + 8u * uint32_t(i); };
+  float* pn2 = reinterpret_cast<float*>(sbase + kWOffN2);
+  float* prr = reinterpret_cast<float*>(sbase + kWOffRR);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t num_tiles = (n + kTile - 1) / kTile;
+  const int64_t my_tiles = num_tiles > blockIdx.x ? (num_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+  const int ka = (np + 63) / 64;          // operand atoms per matrix
+  const int qt = (np + 31) / 32;          // fp32 quarter tiles per key tile
+  const uint32_t atom_bytes = uint32_t(np) * 128u;
+  const size_t mat_bytes = size_t(np) * 256 * 2;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kWStage; ++s) {
+      mbar_init(bar(kWSFull + s), 1);
+      mbar_init(bar(kWSEmpty + s), 64);
+    }
+    for (int s = 0; s < kWRing; ++s) {
+      mbar_init(bar(kWRFull + s), 64);
+      mbar_init(bar(kWREmpty + s), 1);
+    }
+    for (int s = 0; s < kWBRing; ++s) {
+      mbar_init(bar(kWBFull + s), 1);
+      mbar_init(bar(kWBEmpty + s), 1);
+    }
+    mbar_init(bar(kWD1Full), 1);
+    mbar_init(bar(kWN2), 512);
+    mbar_init(bar(kWResid), 512);
+    mbar_init(bar(kWD2Full), 1);
+    mbar_init(bar(kWD2Free), 512);
+    mbar_init(bar(kWRR), 512);
+    *abort_flag = 0;
+    g_wait_budget = wait_budget > 0 ? wait_budget : tc::kWaitCycles;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(512));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int64_t sq = 0, bq = 0;   // staging loads, operand atom loads issued
+      bool ok = true;
+      auto load_b = [&](int mat, int a) -> bool {
+        const int sb = int(bq % kWBRing);
+        if (bq >= kWBRing &&
+            !mbar_wait(bar(kWBEmpty + sb), uint32_t((bq / kWBRing - 1) & 1), abort_flag, status))
+          return false;
+        mbar_expect_tx(bar(kWBFull + sb), atom_bytes);
+        bulk_load(base + kWOffB + kWBAtomMax * sb, bimg + mat * mat_bytes + size_t(a) * atom_bytes, atom_bytes,
+                  bar(kWBFull + sb));
+        ++bq;
+        return true;
+      };
+      for (int64_t i = 0; ok && i < my_tiles; ++i) {
+        const int64_t tile = blockIdx.x + i * gridDim.x;
+        for (int a = 0; ok && a < ka; ++a) {
+          for (int h = 0; ok && h < 2; ++h) {
+            const int q = 2 * a + h;
+            if (q >= qt) break;
+            const int s = int(sq % kWStage);
+            if (sq >= kWStage &&
+                !mbar_wait(bar(kWSEmpty + s), uint32_t((sq / kWStage - 1) & 1), abort_flag, status)) {
+              ok = false;
+              break;
+            }
+            mbar_expect_tx(bar(kWSFull + s), 16384u);
+            tma_load_2d(base + kWOffStage + 16384u * s, &key_map, 32 * q, int(tile * kTile), bar(kWSFull + s));
+            ++sq;
+          }
+          if (ok) ok = load_b(0, a) && load_b(1, a);   // R_hi, R_lo of atom a
+        }
+        for (int a = 0; ok && a < ka; ++a) ok = load_b(2, a);   // P
+      }
+      // leave no copy in flight: wait for the last loads issued to each buffer
+      for (int64_t j = (sq >= kWStage ? sq - kWStage : 0); j < sq; ++j)
+        mbar_drain(bar(kWSFull + int(j % kWStage)), uint32_t((j / kWStage) & 1), abort_flag, status);
+      for (int64_t j = (bq >= kWBRing ? bq - kWBRing : 0); j < bq; ++j)
+        mbar_drain(bar(kWBFull + int(j % kWBRing)), uint32_t((j / kWBRing) & 1), abort_flag, status);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      const uint32_t idesc1 = idesc_f16(1, 128, uint32_t(np)), idesc2 = idesc_f16(0, 128, uint32_t(np));
+      const uint32_t ty = tmem, tz = tmem + 256u;
+      int64_t bq = 0, n1 = 0, n2 = 0;
+      bool ok = true;
+      auto wait_b = [&]() -> uint32_t {
+        const int sb = int(bq % kWBRing);
+        if (!mbar_wait(bar(kWBFull + sb), uint32_t((bq / kWBRing) & 1), abort_flag, status)) return 0u;
+        return base + kWOffB + kWBAtomMax * sb;
+      };
+      auto free_b = [&]() {
+        mma_commit(bar(kWBEmpty + int(bq % kWBRing)));
+        ++bq;
+      };
+      for (int64_t i = 0; ok && i < my_tiles; ++i) {
+        // y's columns hold the previous tile's residual until its JL product completed
+        if (i >= 1 && !mbar_wait(bar(kWD2Full), uint32_t((i - 1) & 1), abort_flag, status)) break;
+        tc_fence_after();
+        uint32_t acc = 0;
+        for (int a = 0; ok && a < ka; ++a) {
+          const int64_t e = i * ka + a;
+          const int rs = int(e & 1);
+          if (!mbar_wait(bar(kWRFull + rs), uint32_t((e >> 1) & 1), abort_flag, status)) {
+            ok = false;
+            break;
+          }
+          const uint32_t abase = base + kWOffRing + 32768u * rs;
+          for (int mat = 0; mat < 2; ++mat) {
+            const uint32_t bb = wait_b();
+            if (!bb) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            for (int ks = 0; ks < 4 && 64 * a + 16 * ks < np; ++ks) {
+              // R_hi: K_hi R_hi + K_lo R_hi; R_lo: K_hi R_lo
+              mma_f16(ty, smem_desc(abase + 32u * ks), smem_desc(bb + 32u * ks), idesc1, acc);
+              acc = 1;
+              if (mat == 0) mma_f16(ty, smem_desc(abase + 16384u + 32u * ks), smem_desc(bb + 32u * ks), idesc1, 1u);
+            }
+            free_b();
+          }
+          if (!ok) break;
+          mma_commit(bar(kWREmpty + rs));
+        }
+        if (!ok) break;
+        mma_commit(bar(kWD1Full));
+        ++n1;
+        // JL product once the epilogue has written the residual and read the previous z
+        if (!mbar_wait(bar(kWResid), uint32_t(i & 1), abort_flag, status)) break;
+        if (i >= 1 && !mbar_wait(bar(kWD2Free), uint32_t((i - 1) & 1), abort_flag, status)) break;
+        tc_fence_after();
+        acc = 0;
+        for (int a = 0; ok && a < ka; ++a) {
+          const uint32_t bb = wait_b();
+          if (!bb) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          for (int ks = 0; ks < 4 && 64 * a + 16 * ks < np; ++ks) {
+            const uint32_t k16 = uint32_t(4 * a + ks);   // residual coordinates 16 k16 .. +15
+            mma_f16_ts(tz, ty + 16u * k16, smem_desc(bb + 32u * ks), idesc2, acc);
+            acc = 1;
+            mma_f16_ts(tz, ty + 16u * k16 + 8u, smem_desc(bb + 32u * ks), idesc2, 1u);
+          }
+          free_b();
+        }
+        if (!ok) break;
+        mma_commit(bar(kWD2Full));
+        ++n2;
+      }
+      // before TMEM is released: the last commit of each kind tracks every MMA issued before it
+      if (n1 > 0) mbar_drain(bar(kWD1Full), uint32_t((n1 - 1) & 1), abort_flag, status);
+      if (n2 > 0) mbar_drain(bar(kWD2Full), uint32_t((n2 - 1) & 1), abort_flag, status);
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ fp32 -> bf16 hi / lo converter
+    const int c = threadIdx.x - 64;
+    for (int64_t i = 0; i < my_tiles; ++i) {
+      bool ok = true;
+      for (int q = 0; q < qt; ++q) {
+        const int64_t j = i * qt + q;              // staging use
+        const int sb = int(j % kWStage);
+        const int64_t e = i * ka + (q >> 1);       // key atom use
+        const int rs = int(e & 1);
+        if ((q & 1) == 0 && e >= 2 &&
+            !mbar_wait_warp(bar(kWREmpty + rs), uint32_t(((e >> 1) - 1) & 1), abort_flag, status)) {
+          ok = false;
+          break;
+        }
+        if (!mbar_wait_warp(bar(kWSFull + sb), uint32_t((j / kWStage) & 1), abort_flag, status)) {
+          ok = false;
+          break;
+        }
+        const uint8_t* src = sbase + kWOffStage + 16384u * sb;
+        uint8_t* dst = sbase + kWOffRing + 32768u * rs;
+#pragma unroll 2
+        for (int gi = c; gi < 512; gi += 64) {
+          const int r = gi >> 2, g = gi & 3;
+          const float4 a4 = *reinterpret_cast<const float4*>(src + r * 128 + (((2 * g) ^ (r & 7)) << 4));
+          const float4 b4 = *reinterpret_cast<const float4*>(src + r * 128 + (((2 * g + 1) ^ (r & 7)) << 4));
+          const float2 x[4] = {make_float2(a4.x, a4.y), make_float2(a4.z, a4.w), make_float2(b4.x, b4.y),
+                               make_float2(b4.z, b4.w)};
+          uint32_t hi[4], lo[4];
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const __nv_bfloat162 h = __float22bfloat162_rn(x[t]);
+            const float2 hf = __bfloat1622float2(h);
+            const __nv_bfloat162 l = __float22bfloat162_rn(__ffma2_rn(hf, f2(-1.f), x[t]));
+            hi[t] = *reinterpret_cast<const uint32_t*>(&h);
+            lo[t] = *reinterpret_cast<const uint32_t*>(&l);
+          }
+          const uint32_t off = uint32_t(r * 128 + (((4 * (q & 1) + g) ^ (r & 7)) << 4));
+          *reinterpret_cast<uint4*>(dst + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<uint4*>(dst + 16384u + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_arrive(bar(kWSEmpty + sb));
+        if ((q & 1) || q == qt - 1) mbar_arrive(bar(kWRFull + rs));
+      }
+      if (!ok) break;
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int qd = (warp - 4) >> 2;                   // layout quarter: slots 64 qd .. 64 qd + 63
+    const int row = (warp & 3) * 32 + lane;           // TMEM lane = key row within the tile
+    const uint32_t lane_addr = uint32_t((warp & 3) * 32) << 16;
+    const uint32_t ty = tmem + lane_addr + 64u * qd, tz = tmem + lane_addr + 256u + 64u * qd;
+    const int valid = d - 64 * qd < 64 ? (d - 64 * qd > 0 ? d - 64 * qd : 0) : 64;   // slots below d
+    constexpr int kW = BMSE + 1;                      // words per half quarter (32 slots)
+    const int row_bytes = 8 * (4 * BMSE + 4);
+    for (int64_t i = 0; i < my_tiles; ++i) {
+      const uint32_t par = uint32_t(i & 1);
+      if (!mbar_wait_warp(bar(kWD1Full), par, abort_flag, status)) break;
+      tc_fence_after();
+      float y[2][32];
+      tmem_ld32(ty, y[0]);
+      tmem_ld32(ty + 32u, y[1]);
+      tmem_wait32(y[0]);
+      tmem_wait32(y[1]);
+      float* n2buf = pn2 + int(par) * 512;
+      {
+        float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int j = 0; j < 32; j += 2) {
+            const float2 v = make_float2(32 * h + j < valid ? y[h][j] : 0.f, 32 * h + j + 1 < valid ? y[h][j + 1] : 0.f);
+            acc = __ffma2_rn(v, v, acc);
+          }
+        n2buf[qd * 128 + row] = acc.x + acc.y;
+      }
+      mbar_arrive(bar(kWN2));
+      if (!mbar_wait_warp(bar(kWN2), par, abort_flag, status)) break;
+      const float n2 = n2buf[row] + n2buf[128 + row] + n2buf[256 + row] + n2buf[384 + row];
+      const float nk = sqrtf(n2);
+      const bool zero = !(n2 > 0.f);
+      const float s128 = zero ? 0.f : 128.f / nk;
+      HalfBook hb = book;
+      if (zero) {
+        hb.C0 = 0.f;
+#pragma unroll
+        for (int c = 0; c < 3; ++c) hb.dC[c] = 0.f;
+        hb.dA = 0.f;
+        hb.C20 = 0.f;
+      }
+      float2 rr2 = make_float2(0.f, 0.f);
+      uint32_t cw[2][BMSE];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        // slots 32 h .. 32 h + 31 of the quarter: units 2 h and 2 h + 1
+        uint32_t hw[2 * BMSE], hw3[2] = {0u, 0u};
+#pragma unroll
+        for (int t = 0; t < 2 * BMSE; ++t) hw[t] = 0;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t rh[8], rl[8];
+#pragma unroll
+          for (int jp = 0; jp < 16; jp += 2) {
+            const int j0 = 16 * hh + jp;
+            float2 rp;
+            const uint2 bb = cell2<BMSE>(make_float2(y[h][j0], y[h][j0 + 1]), s128, hb, rp);
+            // slots past d: no residual (their code and sign bits are masked below)
+            if (32 * h + j0 >= valid) rp.x = 0.f;
+            if (32 * h + j0 + 1 >= valid) rp.y = 0.f;
+            rr2 = __ffma2_rn(rp, rp, rr2);
+            const __half2 hi = __float22half2_rn(rp);
+            const float2 hf = __half22float2(hi);
+            const __half2 lo = __float22half2_rn(__ffma2_rn(hf, f2(-1.f), rp));
+            rh[jp >> 1] = *reinterpret_cast<const uint32_t*>(&hi);
+            rl[jp >> 1] = *reinterpret_cast<const uint32_t*>(&lo);
+#pragma unroll
+            for (int t2 = 0; t2 < 2; ++t2) {
+              const int jc = j0 + t2;
+              const uint32_t bits = t2 ? bb.y : bb.x;
+              const int rreg = jc >> 2, e = jc & 3, uu = rreg >> 2, ii = rreg & 3;
+              if constexpr (BMSE == 3) {
+                if (ii < 3)
+                  hw[uu * 3 + ii] += bits << (4 * e);
+                else
+                  hw3[uu] += bits << (4 * e);
+              } else if constexpr (BMSE == 2) {
+                hw[uu * 2 + (ii >> 1)] += bits << (4 * e + 2 * (ii & 1));
+              } else {
+                hw[uu] += bits << (4 * e + ii);
+              }
+            }
+          }
+          // residual coordinates 64 qd + 32 h + 16 hh .. +15 (group k16 = 4 qd + 2 h + hh):
+          // hi pairs at column 16 k16, lo pairs at 16 k16 + 8
+          tmem_st8(ty + 32u * h + 16u * hh, rh);
+          tmem_st8(ty + 32u * h + 16u * hh + 8u, rl);
+        }
+        if constexpr (BMSE == 3) {
+#pragma unroll
+          for (int uu = 0; uu < 2; ++uu)
+#pragma unroll
+            for (int b = 0; b < 3; ++b) hw[uu * 3 + b] |= ((hw3[uu] >> b) & 0x1111u) << 3;
+        }
+#pragma unroll
+        for (int w = 0; w < BMSE; ++w) cw[h][w] = zero ? 0u : ~__byte_perm(hw[2 * w], hw[2 * w + 1], 0x5410);
+      }
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      tc_fence_before();
+      mbar_arrive(bar(kWResid));
+      float* rrbuf = prr + int(par) * 512;
+      rrbuf[qd * 128 + row] = rr2.x + rr2.y;
+      mbar_arrive(bar(kWRR));
+      if (!mbar_wait_warp(bar(kWD2Full), par, abort_flag, status)) break;
+      tc_fence_after();
+      // bit = [z >= 0]; bit p of half h's word holds slot 32 h + 16 (p >> 4) + 4 (p & 3) + ((p >> 2) & 3)
+      uint32_t sw[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t neg = 0;
+#pragma unroll
+        for (int hz = 1; hz >= 0; --hz) {
+          float z[16];
+          tmem_ld16(tz + 32u * h + 16u * hz, z);
+          tmem_wait16(z);
+#pragma unroll
+          for (int p = 15; p >= 0; --p) {
+            const int jj = 4 * (p & 3) + ((p >> 2) & 3);
+            neg = __funnelshift_l(__float_as_uint(z[jj]), neg, 1);
+          }
+        }
+        sw[h] = zero ? 0xFFFFFFFFu : ~neg;
+      }
+      tc_fence_before();
+      mbar_arrive(bar(kWD2Free));
+      const int64_t key = (blockIdx.x + i * gridDim.x) * kTile + row;
+      if (key < n) {
+        // quarter chunk: the 4 b' code halfwords of units 0..3, then the 4 sign halfwords
+        uint32_t wv[2 * kW];
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int w = 0; w < BMSE; ++w) wv[h * BMSE + w] = cw[h][w] & masks.code[qd][h * BMSE + w];
+        wv[2 * BMSE] = sw[0] & masks.sign[qd][0];
+        wv[2 * BMSE + 1] = sw[1] & masks.sign[qd][1];
+        uint8_t* dst = payload + key * row_bytes + qd * 8 * kW;
+        if constexpr (kW % 2 == 0) {
+#pragma unroll
+          for (int v = 0; v < kW / 2; ++v)
+            reinterpret_cast<uint4*>(dst)[v] = make_uint4(wv[4 * v], wv[4 * v + 1], wv[4 * v + 2], wv[4 * v + 3]);
+        } else {
+#pragma unroll
+          for (int v = 0; v < kW; ++v) reinterpret_cast<uint2*>(dst)[v] = make_uint2(wv[2 * v], wv[2 * v + 1]);
+        }
+      }
+      if (qd == 0) {
+        if (!mbar_wait_warp(bar(kWRR), par, abort_flag, status)) break;
+        const float rr = rrbuf[row] + rrbuf[128 + row] + rrbuf[256 + row] + rrbuf[384 + row];
+        const float rho = nk * sqrtf(rr) * (1.0f / 128.f);
+        const uint32_t nn = uint32_t(__half_as_ushort(__float2half_rn(nk))) |
+                            (uint32_t(__half_as_ushort(__float2half_rn(rho))) << 16);
+        if (key < n) {
+          reinterpret_cast<uint32_t*>(norms)[key] = nn;
+          flag_norm_range(nn, status);
+        }
+      }
+    }
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
+  }
+}
+
 HalfBook make_halfbook(const tq_ctx* ctx) {
   HalfBook hb{};
   const int L = ctx->levels;
@@ -1083,6 +1539,73 @@ cudaError_t launch_quantize_tc(const tq_ctx* ctx, const void* keys, int dtype, i
     go(std::true_type{});
   else
     go(std::false_type{});
+  return cudaGetLastError();
+}
+
+bool quantize_wide_supported(const tq_ctx* ctx, int dtype, int64_t ld, const void* keys) {
+  return ctx->dBimgWide != nullptr && ctx->d > 192 && ctx->d <= 256 && ctx->m == ctx->d && dtype == TQ_F32 &&
+         ctx->bmse >= 1 && ctx->bmse <= 3 && ld % 4 == 0 && (reinterpret_cast<uintptr_t>(keys) & 15) == 0 &&
+         device_is_sm100() && get_encode() != nullptr;
+}
+
+namespace {
+
+// Bits of the stored code and sign words that belong to slots below d (the
+// packing of quantize_wide_kernel: half h of a quarter holds units 2h, 2h+1).
+WideMasks wide_masks(int d, int bmse) {
+  WideMasks wm{};
+  for (int qd = 0; qd < 4; ++qd)
+    for (int jq = 0; jq < 64; ++jq) {
+      if (64 * qd + jq >= d) continue;
+      const int e = jq & 3, i = (jq >> 2) & 3, u = jq >> 4, h = u >> 1, uu = u & 1;
+      auto set_code = [&](int hw, int bit) { wm.code[qd][h * bmse + (hw >> 1)] |= 1u << (bit + 16 * (hw & 1)); };
+      if (bmse == 3) {
+        if (i < 3) {
+          for (int b = 0; b < 3; ++b) set_code(uu * 3 + i, 4 * e + b);
+        } else {
+          for (int b = 0; b < 3; ++b) set_code(uu * 3 + b, 4 * e + 3);
+        }
+      } else if (bmse == 2) {
+        for (int b = 0; b < 2; ++b) set_code(uu * 2 + (i >> 1), 4 * e + 2 * (i & 1) + b);
+      } else {
+        set_code(uu, 4 * e + i);
+      }
+      wm.sign[qd][h] |= 1u << (16 * uu + 4 * e + i);
+    }
+  return wm;
+}
+
+}  // namespace
+
+cudaError_t launch_quantize_wide(const tq_ctx* ctx, const void* keys, int64_t n, int64_t ld, uint8_t* payload,
+                                 uint16_t* norms, cudaStream_t st) {
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {cuuint64_t(ctx->d), cuuint64_t(n)};
+  const cuuint64_t strides[1] = {cuuint64_t(ld) * 4};
+  const cuuint32_t box[2] = {32u, 128u};
+  const cuuint32_t estr[2] = {1u, 1u};
+  const CUresult r = get_encode()(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(keys), dims, strides,
+                                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t tiles = (n + kTile - 1) / kTile;
+  const int grid = int(tiles < sms ? tiles : sms);
+  const HalfBook hb = make_halfbook(ctx);
+  const WideMasks wm = wide_masks(ctx->d, ctx->bmse);
+  const int np = (ctx->d + 15) / 16 * 16;
+  auto run = [&](auto kern) {
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kWSmem));
+    kern<<<grid, kWThreads, kWSmem, st>>>(map, n, ctx->d, np, ctx->dBimgWide, hb, wm, payload, norms, ctx->dstatus,
+                                         ctx->wait_budget);
+  };
+  switch (ctx->bmse) {
+    case 1: run(quantize_wide_kernel<1>); break;
+    case 2: run(quantize_wide_kernel<2>); break;
+    default: run(quantize_wide_kernel<3>); break;
+  }
   return cudaGetLastError();
 }
 

@@ -30,6 +30,8 @@ tq_status tq_quantize(const tq_ctx* ctx, const void* keys, tq_dtype dtype, int64
   cudaError_t e;
   if (tq::quantize_tc_supported(ctx, dtype, ld, keys))
     e = tq::launch_quantize_tc(ctx, keys, dtype, n, ld, payload, norms, st);
+  else if (tq::quantize_wide_supported(ctx, dtype, ld, keys))
+    e = tq::launch_quantize_wide(ctx, keys, n, ld, payload, norms, st);
   else
     e = tq::launch_quantize_simt(ctx, keys, dtype, n, ld, payload, norms, st);
   return cuda_status(e);

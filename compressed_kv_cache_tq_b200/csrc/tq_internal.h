@@ -55,6 +55,8 @@ struct tq_ctx {
   double* dP64 = nullptr;
   double* dc64 = nullptr;
   uint8_t* dBimg = nullptr; // tensor-core B operands (d = m = 128): R_hi, R_lo (bf16), P (fp16), smem image
+  uint8_t* dBimgWide = nullptr;  // wide tensor-core quantizer (192 < d <= 256, m = d): R_hi, R_lo, P as
+                                 // 4 streamed 64-column atoms each (Np = d rounded up to 16 rows)
   uint32_t* dstatus = nullptr;
   long long wait_budget = 0;   // tensor-core quantizer: cycles a wait spins before giving up (0: default)
   tq::CodebookParams cb;
@@ -97,6 +99,9 @@ cudaError_t launch_quantize_simt(const tq_ctx* ctx, const void* keys, int dtype,
 bool quantize_tc_supported(const tq_ctx* ctx, int dtype, int64_t ld, const void* keys);
 cudaError_t launch_quantize_tc(const tq_ctx* ctx, const void* keys, int dtype, int64_t n, int64_t ld,
                                uint8_t* payload, uint16_t* norms, cudaStream_t st);
+bool quantize_wide_supported(const tq_ctx* ctx, int dtype, int64_t ld, const void* keys);
+cudaError_t launch_quantize_wide(const tq_ctx* ctx, const void* keys, int64_t n, int64_t ld, uint8_t* payload,
+                                 uint16_t* norms, cudaStream_t st);
 cudaError_t launch_dequantize(const tq_ctx* ctx, const uint8_t* payload, const uint16_t* norms, int64_t n,
                               int full, float* out, cudaStream_t st);
 

@@ -254,6 +254,7 @@ void tq_free(tq_ctx* ctx) {
   cudaFree(ctx->dP64);
   cudaFree(ctx->dc64);
   cudaFree(ctx->dBimg);
+  cudaFree(ctx->dBimgWide);
   cudaFree(ctx->dstatus);
   delete ctx;
 }
@@ -360,6 +361,30 @@ tq_status tq_init_ex(int d, int bits, int m, uint64_t seed, uint32_t stream_base
     write_swizzled(rl, 128, 128, img.data() + 32768);
     if (m == 128) write_swizzled(ph, 128, 128, img.data() + 65536);   // m = 0: no JL operand
     e = upload(img, &ctx->dBimg);
+  }
+  if (e == cudaSuccess && d > 192 && d <= 256 && m == d) {
+    // Wide quantizer (192 < d <= 256, m = d: a layout of 256 slots): the same operands padded with
+    // zeros to Np = d rounded up to 16 rows and 256 input columns, stored as
+    // four 64-column atoms per matrix (R_hi, R_lo, P), each atom contiguous
+    // (Np rows of 128 bytes, 128-byte swizzle) so that it streams into shared
+    // memory with one bulk copy.
+    const int np = (d + 15) / 16 * 16, kp = 256;
+    std::vector<__nv_bfloat16> rh(size_t(np) * kp, __float2bfloat16_rn(0.f)), rl(rh);
+    std::vector<__half> ph(size_t(np) * kp, __float2half_rn(0.f));
+    for (int i = 0; i < d; ++i)
+      for (int j = 0; j < d; ++j) {
+        const double v = ctx->R[size_t(i) * d + j];
+        const __nv_bfloat16 hi = __float2bfloat16_rn(float(v));
+        rh[size_t(i) * kp + j] = hi;
+        rl[size_t(i) * kp + j] = __float2bfloat16_rn(float(v - double(__bfloat162float(hi))));
+        ph[size_t(i) * kp + j] = __double2half(ctx->P[size_t(i) * d + j]);
+      }
+    const size_t mat = size_t(np) * kp * 2;
+    std::vector<uint8_t> img(3 * mat);
+    write_swizzled(rh, np, kp, img.data());
+    write_swizzled(rl, np, kp, img.data() + mat);
+    write_swizzled(ph, np, kp, img.data() + 2 * mat);
+    e = upload(img, &ctx->dBimgWide);
   }
   if (e == cudaSuccess) e = cudaMalloc(&ctx->dstatus, sizeof(uint32_t));
   if (e == cudaSuccess) e = cudaMemset(ctx->dstatus, 0, sizeof(uint32_t));

@@ -102,6 +102,36 @@ def test_quantize_other_shapes(lib, d, m, bits, dtype):
     check_quantize(payload.cpu().numpy(), norms.cpu().numpy(), kt.to(torch.float64).numpy(), tables_of(ctx))
 
 
+@pytest.mark.parametrize("d,bits", [(200, 2), (200, 3), (200, 4), (208, 3), (256, 2), (232, 4)])
+def test_quantize_wide_tensor_core_path(lib, d, bits):
+    """fp32 keys with 192 < d <= 256 (a layout of 256 slots) and m = d on the wide tensor-core
+    quantizer (operands streamed from L2, one tile in tensor memory): several
+    tiles with a ragged tail, a leading dimension above d, layout padding
+    slots zero; equal to the rows quantised from a contiguous copy."""
+    import ctypes
+
+    ctx = _ctx(lib, d=d, bits=bits, seed=5)
+    n = 3 * 128 + 45
+    ld = d + 8
+    k = W.search_vectors(n, d, seed=d + bits, which=0) * np.float32(7.0)
+    k[7] = 0.0                                    # zero key
+    wide = torch.zeros((n, ld), dtype=torch.float32)
+    wide[:, :d] = torch.from_numpy(k)
+    dev = wide.to(DEV)
+    payload = torch.empty((n, ctx.row_bytes), dtype=torch.uint8, device=DEV)
+    norms = torch.empty((n, 2), dtype=torch.float16, device=DEV)
+    st = lib.lib().tq_quantize(ctx.handle, ctypes.c_void_p(dev.data_ptr()), 0, n, ld,
+                               ctypes.c_void_p(payload.data_ptr()), ctypes.c_void_p(norms.data_ptr()),
+                               ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0
+    _status_clean(lib, ctx)
+    check_quantize(payload.cpu().numpy(), norms.cpu().numpy(), k.astype(np.float64), tables_of(ctx))
+    p2, n2 = lib.tq_quantize(ctx, torch.from_numpy(k).to(DEV))
+    assert torch.equal(p2, payload) and torch.equal(n2.view(torch.int16), norms.view(torch.int16))
+    codes, bits_ = O.unpack_rows(payload.cpu().numpy()[7:8], d, d, bits - 1)
+    assert not codes.any() and bits_.all()
+
+
 def test_quantize_edge_cases(lib):
     ctx = _ctx(lib, bits=4, seed=3)
     k = W.toy_keys(300, 128, seed=9)
