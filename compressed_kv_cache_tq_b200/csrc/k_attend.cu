@@ -382,9 +382,46 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_mma_kernel(
   const uint8_t* rows = payload + (size_t(grp) * S) * rb;
   const uint32_t* nrm = reinterpret_cast<const uint32_t*>(norms) + size_t(grp) * S;
 
-  for (int i = tid; i < GP * kAcc; i += kAttThreads) sacc[i] = 0.f;
   if (tid < GP) sl[tid] = 0.f;
 
+  constexpr int kWIt = T * GP / kAttThreads;   // (key, head) weights per thread and tile
+  // rows: asynchronous 16-byte copies into the tile's buffer (rows past the
+  // chunk keep stale bytes; their weights are zero); logits and norms of the
+  // next tile prefetched into registers
+  auto copy_rows = [&](int64_t s0, uint8_t* dst) {
+    const int nk = int(s_end - s0 < T ? s_end - s0 : T);   // <= 0 past the chunk: an empty group
+    constexpr int kc = rb / 16;   // 16-byte chunks per row
+    const int nc = nk * kc;
+    const uint8_t* src = rows + size_t(s0) * rb;
+    for (int c = tid; c < nc; c += kAttThreads) {
+      const int r = c / kc, cc = c - r * kc;
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                       uint32_t(__cvta_generic_to_shared(dst + r * rs + 16 * cc))),
+                   "l"(src + 16 * c)
+                   : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  float lgv[kWIt];
+  uint32_t nnv[kWIt];
+  auto fetch_w = [&](int64_t s0) {
+    const int nk = int(s_end - s0 < T ? s_end - s0 : T);
+#pragma unroll
+    for (int it = 0; it < kWIt; ++it) {
+      const int idx = tid + it * kAttThreads;
+      const int k = idx % T, h = idx / T;
+      const bool ok = k < nk && h < G;
+      lgv[it] = ok ? __ldg(lg + size_t(h) * S + s0 + k) : 0.f;
+      nnv[it] = ok ? __ldg(nrm + s0 + k) : 0u;
+    }
+  };
+  // one commit group per tile, kAttStages - 1 tiles ahead of the one in use;
+  // the first tile's rows, logits and norms are in flight during pass 1
+  if (s_begin < s_end) {
+#pragma unroll
+    for (int st = 0; st < kAttStages - 1; ++st) copy_rows(s_begin + int64_t(st) * T, srows0 + st * T * rs);
+    fetch_w(s_begin);
+  }
   // pass 1: the chunk's maximum logit per head
   float mx[GP];
 #pragma unroll
@@ -439,47 +476,10 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_mma_kernel(
       accC[mt][c] = 0.f;
       accS[mt][c] = 0.f;
     }
-  constexpr int kWIt = T * GP / kAttThreads;
   float lsum[kWIt];
 #pragma unroll
   for (int it = 0; it < kWIt; ++it) lsum[it] = 0.f;
 
-  // rows: asynchronous 16-byte copies into the tile's buffer (rows past the
-  // chunk keep stale bytes; their weights are zero); logits and norms of the
-  // next tile prefetched into registers
-  auto copy_rows = [&](int64_t s0, uint8_t* dst) {
-    const int nk = int(s_end - s0 < T ? s_end - s0 : T);   // <= 0 past the chunk: an empty group
-    constexpr int kc = rb / 16;   // 16-byte chunks per row
-    const int nc = nk * kc;
-    const uint8_t* src = rows + size_t(s0) * rb;
-    for (int c = tid; c < nc; c += kAttThreads) {
-      const int r = c / kc, cc = c - r * kc;
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
-                       uint32_t(__cvta_generic_to_shared(dst + r * rs + 16 * cc))),
-                   "l"(src + 16 * c)
-                   : "memory");
-    }
-    asm volatile("cp.async.commit_group;" ::: "memory");
-  };
-  float lgv[kWIt];
-  uint32_t nnv[kWIt];
-  auto fetch_w = [&](int64_t s0) {
-    const int nk = int(s_end - s0 < T ? s_end - s0 : T);
-#pragma unroll
-    for (int it = 0; it < kWIt; ++it) {
-      const int idx = tid + it * kAttThreads;
-      const int k = idx % T, h = idx / T;
-      const bool ok = k < nk && h < G;
-      lgv[it] = ok ? __ldg(lg + size_t(h) * S + s0 + k) : 0.f;
-      nnv[it] = ok ? __ldg(nrm + s0 + k) : 0u;
-    }
-  };
-  // one commit group per tile, kAttStages - 1 tiles ahead of the one in use
-  if (s_begin < s_end) {
-#pragma unroll
-    for (int st = 0; st < kAttStages - 1; ++st) copy_rows(s_begin + int64_t(st) * T, srows0 + st * T * rs);
-    fetch_w(s_begin);
-  }
   int ti = 0;
   for (int64_t s0 = s_begin; s0 < s_end; s0 += T, ++ti) {
     const int nk = int(s_end - s0 < T ? s_end - s0 : T);
@@ -587,20 +587,28 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_mma_kernel(
   asm volatile("cp.async.wait_group 0;" ::: "memory");
   __syncthreads();
 
-  // the rows of this thread's accumulators: unit g, register i, nibble e; head tig
-  if (tig < G) {
+  // the warps' accumulators meet in shared memory (the row ring and the
+  // weight buffers are free now): warp w writes its sums for head tig to
+  // red[w][tig][.], then every thread adds up the eight warps for its outputs
+  // (no atomics: the eight warps' sums for one output all hit one address)
+  constexpr int kRed = (JL ? 256 : 128) + 4;   // a row of red: a (128), b (128 or none), padding
+  static_assert(kAttWarps * GP * kRed * 4 <= kAttStages * T * rs + 2 * T * GP * 4 + GP * kAcc * 4,
+                "reduction buffer");
+  float* red = reinterpret_cast<float*>(sm);
+  {
+    // the rows of this thread's accumulators: unit g, register i, nibble e; head tig
+    float* rw = red + (warp * GP + tig) * kRed;
     const int q = g >> 1, u = g & 1;
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int j0 = q * 32 + 4 * (4 * u + i) + 2 * h;   // e = 2h (row g) and 2h + 1 (row g + 8)
-        atomicAdd(sacc + tig * kAcc + j0, accC[2 * i + h][0] + accC[2 * i + h][1]);
-        atomicAdd(sacc + tig * kAcc + j0 + 1, accC[2 * i + h][2] + accC[2 * i + h][3]);
-        if constexpr (JL) {
-          atomicAdd(sacc + tig * kAcc + 128 + j0, accS[2 * i + h][0] + accS[2 * i + h][1]);
-          atomicAdd(sacc + tig * kAcc + 128 + j0 + 1, accS[2 * i + h][2] + accS[2 * i + h][3]);
-        }
+        *reinterpret_cast<float2*>(rw + j0) =
+            make_float2(accC[2 * i + h][0] + accC[2 * i + h][1], accC[2 * i + h][2] + accC[2 * i + h][3]);
+        if constexpr (JL)
+          *reinterpret_cast<float2*>(rw + 128 + j0) =
+              make_float2(accS[2 * i + h][0] + accS[2 * i + h][1], accS[2 * i + h][2] + accS[2 * i + h][3]);
       }
   }
 #pragma unroll
@@ -613,13 +621,17 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_mma_kernel(
   __syncthreads();
   // partial record {max, sum, a[128], b[128 or 0]} in the generic layout (dp + mp slots)
   constexpr int rec = 2 + 128 + (JL ? 128 : 0);
-  for (int h = 0; h < G; ++h) {
-    float* out = part + (size_t(blockIdx.x) * G + h) * rec;
-    for (int i = tid; i < rec - 2; i += kAttThreads) out[2 + i] = sacc[h * kAcc + i];
-    if (tid == 0) {
-      out[0] = smx[h];
-      out[1] = sl[h];
-    }
+  for (int o = tid; o < G * (rec - 2); o += kAttThreads) {
+    const int h = o / (rec - 2), j = o - h * (rec - 2);
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < kAttWarps; ++w) v += red[(w * GP + h) * kRed + j];
+    part[(size_t(blockIdx.x) * G + h) * rec + 2 + j] = v;
+  }
+  if (tid < G) {
+    float* out = part + (size_t(blockIdx.x) * G + tid) * rec;
+    out[0] = smx[tid];
+    out[1] = sl[tid];
   }
 }
 
