@@ -40,8 +40,8 @@ constexpr int kAttWarps = kAttThreads / 32;
 constexpr int kAttTile = 128;         // keys per staged tile
 constexpr int kAttMaxLd = 8;          // 8-byte words per thread per tile (rows of up to 128 bytes)
 constexpr int kAttMaxHeads = 8;
-constexpr int kAttMmaTile = 256;      // keys per staged tile of the tensor-core kernel
 constexpr int kAttStages = 2;         // row tiles in flight per block (cp.async ring)
+constexpr int kWStages = 4;           // 16-key steps in flight per warp (tensor-core kernel)
 
 // The slot's 4 codes (r = 4u + i, e = 0..3) as nibbles e of one word, from the
 // unit's code halfwords h[0 .. BM-1] (layout in include/tq.h): code e is
@@ -341,35 +341,36 @@ __device__ __forceinline__ uint32_t reg_selector(const uint32_t (&h)[BM], int i)
   }
 }
 
-// A weight as its fp16 hi limb (low half) and lo limb w - hi (high half).
-__device__ __forceinline__ uint32_t limb_pair(float w) {
-  const __half hi = __float2half_rn(w);
-  const __half lo = __float2half_rn(w - __half2float(hi));
-  return uint32_t(__half_as_ushort(hi)) | (uint32_t(__half_as_ushort(lo)) << 16);
-}
+// Per-warp staging ring of the tensor-core kernel: kWStages 16-key steps, each
+// the packed rows (padded stride), the logits of the GP heads and the norms.
+template <int BM, bool JL>
+struct WarpRing {
+  static constexpr int kPerQ = 2 * BM + (JL ? 2 : 0);    // halfwords per quarter chunk (d = m = 128)
+  static constexpr int rb = 8 * kPerQ;                    // row bytes (a multiple of 16)
+  // row stride: an odd number of 16-byte chunks, so that the rows two apart
+  // read by the four lanes of a quad fall in different banks
+  static constexpr int rs = (rb / 16) % 2 ? rb : rb + 16;
+  static constexpr int kRows = 16 * rs;                   // bytes of one step's rows
+  static constexpr int kStep = kRows + 4 * 16 * 4 + 16 * 4;   // + logits [4][16] + norms [16]
+  static constexpr int kWarp = kWStages * kStep;
+};
 
 template <int BM, bool JL>
 __global__ void __launch_bounds__(kAttThreads, 2) attend_mma_kernel(
     const float* __restrict__ logits, int Hq, int Hkv, int64_t S, int64_t chunk, int nsplit,
     const uint8_t* __restrict__ payload, const uint16_t* __restrict__ norms, HalfLut lut,
     float* __restrict__ part) {
+  using WR = WarpRing<BM, JL>;
   constexpr int GP = 4;
-  constexpr int kPerQ = 2 * BM + (JL ? 2 : 0);   // halfwords per quarter chunk (d = m = 128)
-  constexpr int rb = 8 * kPerQ;                   // row bytes
-  // row stride in shared memory: an odd number of 16-byte chunks, so that the
-  // rows two apart read by the four lanes of a quad fall in different banks
-  constexpr int rs = (rb / 16) % 2 ? rb : rb + 16;
-  constexpr int kAcc = 256;                       // a (128 coordinates) then b (128 sign coordinates)
-  constexpr int T = kAttMmaTile;
+  constexpr int kPerQ = WR::kPerQ, rb = WR::rb, rs = WR::rs;
+  constexpr int kRed = (JL ? 256 : 128) + 4;   // a row of the reduction buffer: a (128), b (128 or none), padding
+  constexpr float kL2e = 1.4426950408889634f;
+  // b' = 3 with signs: a quarter chunk is 16 bytes (halfwords 0-2 unit 0
+  // codes, 3-5 unit 1 codes, 6 / 7 the units' signs); unit g & 1's halfwords
+  // come out of one 16-byte load
+  constexpr bool kQuad16 = (BM == 3 && JL && rb == 64);
   extern __shared__ __align__(16) uint8_t sm[];
-  uint8_t* srows0 = sm;                                                       // [kAttStages][T][rs] row ring
-  // weights as fp16 (hi, lo) limb pairs: w n16 for the codes, w rho16 for the signs
-  uint32_t* swn = reinterpret_cast<uint32_t*>(sm + kAttStages * T * rs);      // [T][GP]
-  uint32_t* swr = swn + T * GP;                                               // [T][GP]
-  float* sacc = reinterpret_cast<float*>(swr + T * GP);                       // [GP][kAcc]
-  float* sred = sacc + GP * kAcc;                                             // [GP][kAttWarps] maxima
-  float* smx = sred + GP * kAttWarps;                                         // [GP] chunk maximum
-  float* sl = smx + GP;                                                       // [GP] sum of weights
+  __shared__ float wmax[kAttWarps][GP], wsum[kAttWarps][GP], wfac[kAttWarps][GP];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, tig = lane & 3;
@@ -381,93 +382,62 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_mma_kernel(
   const float* lg = logits + (size_t(b) * Hq + size_t(hkv) * G) * S;   // head h at lg + h S
   const uint8_t* rows = payload + (size_t(grp) * S) * rb;
   const uint32_t* nrm = reinterpret_cast<const uint32_t*>(norms) + size_t(grp) * S;
+  uint8_t* ring = sm + warp * WR::kWarp;
 
-  if (tid < GP) sl[tid] = 0.f;
+  // this warp's 16-key steps: a contiguous share of the block's chunk
+  const int64_t nsteps = s_end > s_begin ? (s_end - s_begin + 15) / 16 : 0;
+  const int64_t st0 = nsteps * warp / kAttWarps, st1 = nsteps * (warp + 1) / kAttWarps;
 
-  constexpr int kWIt = T * GP / kAttThreads;   // (key, head) weights per thread and tile
-  // rows: asynchronous 16-byte copies into the tile's buffer (rows past the
-  // chunk keep stale bytes; their weights are zero); logits and norms of the
-  // next tile prefetched into registers
-  auto copy_rows = [&](int64_t s0, uint8_t* dst) {
-    const int nk = int(s_end - s0 < T ? s_end - s0 : T);   // <= 0 past the chunk: an empty group
-    constexpr int kc = rb / 16;   // 16-byte chunks per row
-    const int nc = nk * kc;
-    const uint8_t* src = rows + size_t(s0) * rb;
-    for (int c = tid; c < nc; c += kAttThreads) {
-      const int r = c / kc, cc = c - r * kc;
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
-                       uint32_t(__cvta_generic_to_shared(dst + r * rs + 16 * cc))),
-                   "l"(src + 16 * c)
-                   : "memory");
-    }
-    asm volatile("cp.async.commit_group;" ::: "memory");
-  };
-  float lgv[kWIt];
-  uint32_t nnv[kWIt];
-  auto fetch_w = [&](int64_t s0) {
-    const int nk = int(s_end - s0 < T ? s_end - s0 : T);
+  // step st into its ring stage: rows by 16-byte copies, logits and norms by
+  // 4-byte copies; entries past the chunk get logit -inf (weight 0) and keep
+  // stale row bytes (finite levels times weight 0)
+  auto stage = [&](int64_t st) {
+    if (st < st1) {
+      uint8_t* dst = ring + int(st % kWStages) * WR::kStep;
+      const int64_t s0 = s_begin + 16 * st;
+      const int nk = int(s_end - s0 < 16 ? s_end - s0 : 16);
+      constexpr int kc = rb / 16;
+      for (int c = lane; c < 16 * kc; c += 32) {
+        const int r = c / kc, cc = c - r * kc;
+        if (r < nk)
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                           uint32_t(__cvta_generic_to_shared(dst + r * rs + 16 * cc))),
+                       "l"(rows + size_t(s0 + r) * rb + 16 * cc)
+                       : "memory");
+      }
+      float* sl = reinterpret_cast<float*>(dst + WR::kRows);   // [GP][16]
 #pragma unroll
-    for (int it = 0; it < kWIt; ++it) {
-      const int idx = tid + it * kAttThreads;
-      const int k = idx % T, h = idx / T;
-      const bool ok = k < nk && h < G;
-      lgv[it] = ok ? __ldg(lg + size_t(h) * S + s0 + k) : 0.f;
-      nnv[it] = ok ? __ldg(nrm + s0 + k) : 0u;
-    }
-  };
-  // one commit group per tile, kAttStages - 1 tiles ahead of the one in use;
-  // the first tile's rows, logits and norms are in flight during pass 1
-  if (s_begin < s_end) {
-#pragma unroll
-    for (int st = 0; st < kAttStages - 1; ++st) copy_rows(s_begin + int64_t(st) * T, srows0 + st * T * rs);
-    fetch_w(s_begin);
-  }
-  // pass 1: the chunk's maximum logit per head
-  float mx[GP];
-#pragma unroll
-  for (int h = 0; h < GP; ++h) mx[h] = -INFINITY;
-  for (int64_t s = s_begin + tid; s < s_end; s += 8 * kAttThreads) {
-#pragma unroll
-    for (int h = 0; h < GP; ++h) {
-      if (h < G) {
-        float v[8];
-#pragma unroll
-        for (int x = 0; x < 8; ++x) {
-          const int64_t sx = s + int64_t(x) * kAttThreads;
-          v[x] = sx < s_end ? __ldg(lg + size_t(h) * S + sx) : -INFINITY;
-        }
-#pragma unroll
-        for (int x = 0; x < 8; ++x) mx[h] = fmaxf(mx[h], v[x]);
+      for (int t = 0; t < 2; ++t) {
+        const int e = lane + 32 * t, h = e >> 4, k = e & 15;
+        if (h < G && k < nk)
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(uint32_t(__cvta_generic_to_shared(sl + e))),
+                       "l"(lg + size_t(h) * S + s0 + k)
+                       : "memory");
+        else
+          sl[e] = -INFINITY;
+      }
+      uint32_t* sn = reinterpret_cast<uint32_t*>(dst + WR::kRows + 4 * 16 * 4);   // [16]
+      if (lane < 16) {
+        if (lane < nk)
+          asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(uint32_t(__cvta_generic_to_shared(sn + lane))),
+                       "l"(nrm + s0 + lane)
+                       : "memory");
+        else
+          sn[lane] = 0u;
       }
     }
-  }
-#pragma unroll
-  for (int h = 0; h < GP; ++h) {
-    float v = mx[h];
-    for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-    if (lane == 0) sred[h * kAttWarps + warp] = v;
-  }
-  __syncthreads();
-  if (tid < GP) {
-    float v = sred[tid * kAttWarps];
-    for (int w = 1; w < kAttWarps; ++w) v = fmaxf(v, sred[tid * kAttWarps + w]);
-    smx[tid] = v;
-  }
-  __syncthreads();
+    asm volatile("cp.async.commit_group;" ::: "memory");   // one group per step, empty past the range
+  };
 
   // unit g of every row (quarter g >> 1, unit g & 1): code and sign halfwords
   const int code_off = (g >> 1) * kPerQ + (g & 1) * BM;
   const int sign_off = (g >> 1) * kPerQ + 2 * BM + (g & 1);
-  const int wcol_head = g >> 1;          // B column g: head g / 2, limb g % 2
-  const uint32_t wsel = (g & 1) ? 0x7632u : 0x5410u;   // picks that limb of two keys' limb pairs
-  // b' = 3 with signs: a quarter chunk is 16 bytes (halfwords 0-2 unit 0
-  // codes, 3-5 unit 1 codes, 6 / 7 the units' signs); unit g & 1's halfwords
-  // come out of one 16-byte load
-  constexpr bool kQuad16 = (BM == 3 && JL && rb == 64);
   // byte-permute selector of the unit's halfwords: (x, y) -> hw 0 or hw 3,
   // (y, z) -> hw 2 or hw 5, (w, w) -> hw 6 or hw 7; with ^ 0x2222,
   // (x, z) -> hw 1 or hw 4 (the upper halves of the results are don't-cares)
   const uint32_t sel_u = (g & 1) ? 0x7676u : 0x1010u;
+  // B column g: head hb = g / 2, limb g % 2 of the weight
+  const int hb = g >> 1;
   float accC[8][4], accS[8][4];
 #pragma unroll
   for (int mt = 0; mt < 8; ++mt)
@@ -476,124 +446,144 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_mma_kernel(
       accC[mt][c] = 0.f;
       accS[mt][c] = 0.f;
     }
-  float lsum[kWIt];
-#pragma unroll
-  for (int it = 0; it < kWIt; ++it) lsum[it] = 0.f;
+  // running maximum of head hb's logits over this warp's keys so far (the
+  // accumulators and the weight sum are kept relative to it) and the weight sum
+  float mrun = -INFINITY, lsum = 0.f;
 
-  int ti = 0;
-  for (int64_t s0 = s_begin; s0 < s_end; s0 += T, ++ti) {
-    const int nk = int(s_end - s0 < T ? s_end - s0 : T);
-    uint8_t* srows = srows0 + (ti % kAttStages) * T * rs;
-    asm volatile("cp.async.wait_group %0;" ::"n"(kAttStages - 2) : "memory");
-    __syncthreads();   // this tile's rows visible; every warp is done with the previous tile
-    copy_rows(s0 + int64_t(kAttStages - 1) * T, srows0 + ((ti + kAttStages - 1) % kAttStages) * T * rs);
 #pragma unroll
-    for (int it = 0; it < kWIt; ++it) {
-      const int idx = tid + it * kAttThreads;
-      const int k = idx % T, h = idx / T;
-      float wn = 0.f, wr = 0.f;
-      if (k < nk && h < G) {
-        // exp(l - max) as 2^((l - max) log2 e)
-        const float w = exp2f((lgv[it] - smx[h]) * 1.4426950408889634f);
-        const uint32_t nn = nnv[it];
-        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&nn));
-        wn = w * f.x;
-        wr = w * f.y;
-        lsum[it] += w;
-      }
-      swn[((k >> 1) * GP + h) * 2 + (k & 1)] = limb_pair(wn);
-      swr[((k >> 1) * GP + h) * 2 + (k & 1)] = limb_pair(wr);
+  for (int j = 0; j < kWStages - 1; ++j) stage(st0 + j);
+  for (int64_t st = st0; st < st1; ++st) {
+    stage(st + kWStages - 1);   // into the stage the previous step used (all lanes are past it)
+    asm volatile("cp.async.wait_group %0;" ::"n"(kWStages - 1) : "memory");
+    __syncwarp();
+    const uint8_t* srows = ring + int(st % kWStages) * WR::kStep;
+    const float* sl = reinterpret_cast<const float*>(srows + WR::kRows) + hb * 16;
+    const uint32_t* sn = reinterpret_cast<const uint32_t*>(srows + WR::kRows + 4 * 16 * 4);
+    // keys 2 tig, 2 tig + 1, 2 tig + 8, 2 tig + 9 of the step
+    const float2 l01 = *reinterpret_cast<const float2*>(sl + 2 * tig);
+    const float2 l89 = *reinterpret_cast<const float2*>(sl + 2 * tig + 8);
+    const uint2 n01 = *reinterpret_cast<const uint2*>(sn + 2 * tig);
+    const uint2 n89 = *reinterpret_cast<const uint2*>(sn + 2 * tig + 8);
+    const float lv[4] = {l01.x, l01.y, l89.x, l89.y};
+    const uint32_t nv[4] = {n01.x, n01.y, n89.x, n89.y};
+    // the step's maximum of head hb (the 8 lanes of the head), then rescale
+    // what was summed against the old maximum if it rose
+    float lm = fmaxf(fmaxf(lv[0], lv[1]), fmaxf(lv[2], lv[3]));
+    lm = fmaxf(lm, __shfl_xor_sync(0xffffffffu, lm, 1));
+    lm = fmaxf(lm, __shfl_xor_sync(0xffffffffu, lm, 2));
+    lm = fmaxf(lm, __shfl_xor_sync(0xffffffffu, lm, 4));
+    const bool rise = lm > mrun;
+    if (__any_sync(0xffffffffu, rise)) {
+      const float f = rise ? exp2f((mrun - lm) * kL2e) : 1.f;   // 0 while nothing was summed (mrun = -inf)
+      const float fa = __shfl_sync(0xffffffffu, f, 8 * tig);      // lane 8 tig has head tig: this lane's accumulators
+      lsum *= f;
+      if (rise) mrun = lm;
+#pragma unroll
+      for (int mt = 0; mt < 8; ++mt)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          accC[mt][c] *= fa;
+          if constexpr (JL) accS[mt][c] *= fa;
+        }
     }
-    if (s0 + T < s_end) fetch_w(s0 + T);   // next tile's logits and norms in flight during the math
-    __syncthreads();
-#pragma unroll 2
-    for (int kb = warp * 16; kb < nk; kb += kAttWarps * 16) {   // 16-key steps; keys past nk have zero weight
-      __syncwarp();
-      const int kk[4] = {kb + 2 * tig, kb + 2 * tig + 1, kb + 2 * tig + 8, kb + 2 * tig + 9};
-      // the limb pairs of keys (2 tig, 2 tig + 1) and (+8, +9) for head wcol_head
-      const int p0 = (kb >> 1) + tig;
-      const uint2 wn0 = *reinterpret_cast<const uint2*>(swn + (p0 * GP + wcol_head) * 2);
-      const uint2 wn1 = *reinterpret_cast<const uint2*>(swn + ((p0 + 4) * GP + wcol_head) * 2);
-      const uint32_t bC0 = prmt(wn0.x, wn0.y, wsel);
-      const uint32_t bC1 = prmt(wn1.x, wn1.y, wsel);
-      uint32_t hc[4][BM];
-      uint32_t hsg[4];
-      if constexpr (kQuad16) {
-        // one 16-byte load of the key's quarter chunk; this thread's unit's
-        // halfwords picked by byte permutes (upper halves are don't-cares for
-        // the code selectors, zero for the sign halfword)
+    // weights exp(l - mrun) times the norms, as this lane's fp16 limb of key pairs
+    float wn[4], wr[4];
 #pragma unroll
-        for (int x = 0; x < 4; ++x) {
-          const uint4 rw = *reinterpret_cast<const uint4*>(srows + kk[x] * rs + (g >> 1) * 16);
-          hc[x][0] = prmt(rw.x, rw.y, sel_u);
-          hc[x][1] = prmt(rw.x, rw.z, sel_u ^ 0x2222u);
-          hc[x][2] = prmt(rw.y, rw.z, sel_u);
-          hsg[x] = prmt(rw.w, rw.w, sel_u);
-        }
-      } else {
+    for (int x = 0; x < 4; ++x) {
+      const float w = lv[x] > -INFINITY ? exp2f((lv[x] - mrun) * kL2e) : 0.f;
+      lsum += w;
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&nv[x]));
+      wn[x] = w * f.x;
+      wr[x] = w * f.y;
+    }
+    auto limb2 = [&](float a, float c) -> uint32_t {
+      const __half2 hi = __floats2half2_rn(a, c);
+      const float2 hf = __half22float2(hi);
+      const __half2 lo = __floats2half2_rn(a - hf.x, c - hf.y);
+      const __half2 r = (g & 1) ? lo : hi;
+      return *reinterpret_cast<const uint32_t*>(&r);
+    };
+    const uint32_t bC0 = limb2(wn[0], wn[1]), bC1 = limb2(wn[2], wn[3]);
+    const int kk[4] = {2 * tig, 2 * tig + 1, 2 * tig + 8, 2 * tig + 9};
+    uint32_t hc[4][BM];
+    uint32_t hsg[4];
+    if constexpr (kQuad16) {
+      // one 16-byte load of the key's quarter chunk; this thread's unit's
+      // halfwords picked by byte permutes (upper halves are don't-cares for
+      // the code selectors, zero for the sign halfword)
 #pragma unroll
-        for (int x = 0; x < 4; ++x) {
-          const uint16_t* hw = reinterpret_cast<const uint16_t*>(srows + kk[x] * rs);
+      for (int x = 0; x < 4; ++x) {
+        const uint4 rw = *reinterpret_cast<const uint4*>(srows + kk[x] * rs + (g >> 1) * 16);
+        hc[x][0] = prmt(rw.x, rw.y, sel_u);
+        hc[x][1] = prmt(rw.x, rw.z, sel_u ^ 0x2222u);
+        hc[x][2] = prmt(rw.y, rw.z, sel_u);
+        hsg[x] = prmt(rw.w, rw.w, sel_u);
+      }
+    } else {
 #pragma unroll
-          for (int y = 0; y < BM; ++y) hc[x][y] = hw[code_off + y];
-          if constexpr (JL) hsg[x] = hw[sign_off];
-        }
+      for (int x = 0; x < 4; ++x) {
+        const uint16_t* hw = reinterpret_cast<const uint16_t*>(srows + kk[x] * rs);
+#pragma unroll
+        for (int y = 0; y < BM; ++y) hc[x][y] = hw[code_off + y];
+        if constexpr (JL) hsg[x] = hw[sign_off];
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t lo[4], hi[4];
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        const uint32_t sel = reg_selector<BM>(hc[x], i);
+        lo[x] = prmt(lut.lo[0], lut.lo[1], sel);
+        hi[x] = prmt(lut.hi[0], lut.hi[1], sel);
       }
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        uint32_t lo[4], hi[4];
+      for (int h = 0; h < 2; ++h) {
+        // bytes (key a, e = 2h), (key b, 2h), (a, 2h + 1), (b, 2h + 1) of each plane
+        const uint32_t ps = h ? 0x7362u : 0x5140u;
+        const uint32_t p01 = prmt(lo[0], lo[1], ps), q01 = prmt(hi[0], hi[1], ps);
+        const uint32_t p23 = prmt(lo[2], lo[3], ps), q23 = prmt(hi[2], hi[3], ps);
+        // fp16 pairs: row g (e = 2h) and row g + 8 (e = 2h + 1), keys (2 tig, 2 tig + 1) / (+8, +9)
+        const uint32_t a0 = prmt(p01, q01, 0x5140u), a1 = prmt(p01, q01, 0x7362u);
+        const uint32_t a2 = prmt(p23, q23, 0x5140u), a3 = prmt(p23, q23, 0x7362u);
+        mma_16816(accC[2 * i + h], a0, a1, a2, a3, bC0, bC1);
+      }
+    }
+    if constexpr (JL) {
+      const uint32_t bS0 = limb2(wr[0], wr[1]), bS1 = limb2(wr[2], wr[3]);
+      // inverted sign bits of a key pair in the two halves: bit 4e + i of the
+      // halfword goes to bit 15 (key a) and bit 31 (key b) after a left shift
+      // by 15 - 4e - i; set means -1 (fp16 sign bit) over 1.0 (0x3C00)
+      const uint32_t w01 = ~prmt(hsg[0], hsg[1], 0x5410u), w23 = ~prmt(hsg[2], hsg[3], 0x5410u);
 #pragma unroll
-        for (int x = 0; x < 4; ++x) {
-          const uint32_t sel = reg_selector<BM>(hc[x], i);
-          lo[x] = prmt(lut.lo[0], lut.lo[1], sel);
-          hi[x] = prmt(lut.hi[0], lut.hi[1], sel);
-        }
+      for (int i = 0; i < 4; ++i)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          // bytes (key a, e = 2h), (key b, 2h), (a, 2h + 1), (b, 2h + 1) of each plane
-          const uint32_t ps = h ? 0x7362u : 0x5140u;
-          const uint32_t p01 = prmt(lo[0], lo[1], ps), q01 = prmt(hi[0], hi[1], ps);
-          const uint32_t p23 = prmt(lo[2], lo[3], ps), q23 = prmt(hi[2], hi[3], ps);
-          // fp16 pairs: row g (e = 2h) and row g + 8 (e = 2h + 1), keys (2 tig, 2 tig + 1) / (+8, +9)
-          const uint32_t a0 = prmt(p01, q01, 0x5140u), a1 = prmt(p01, q01, 0x7362u);
-          const uint32_t a2 = prmt(p23, q23, 0x5140u), a3 = prmt(p23, q23, 0x7362u);
-          mma_16816(accC[2 * i + h], a0, a1, a2, a3, bC0, bC1);
+          const int e0 = 2 * h, e1 = 2 * h + 1;
+          const uint32_t a0 = ((w01 << (15 - 4 * e0 - i)) & 0x80008000u) | 0x3C003C00u;
+          const uint32_t a1 = ((w01 << (15 - 4 * e1 - i)) & 0x80008000u) | 0x3C003C00u;
+          const uint32_t a2 = ((w23 << (15 - 4 * e0 - i)) & 0x80008000u) | 0x3C003C00u;
+          const uint32_t a3 = ((w23 << (15 - 4 * e1 - i)) & 0x80008000u) | 0x3C003C00u;
+          mma_16816(accS[2 * i + h], a0, a1, a2, a3, bS0, bS1);
         }
-      }
-      if constexpr (JL) {
-        const uint2 wr0 = *reinterpret_cast<const uint2*>(swr + (p0 * GP + wcol_head) * 2);
-        const uint2 wr1 = *reinterpret_cast<const uint2*>(swr + ((p0 + 4) * GP + wcol_head) * 2);
-        const uint32_t bS0 = prmt(wr0.x, wr0.y, wsel);
-        const uint32_t bS1 = prmt(wr1.x, wr1.y, wsel);
-        const uint32_t(&hs)[4] = hsg;
-        // inverted sign bits of a key pair in the two halves: bit 4e + i of the
-        // halfword goes to bit 15 (key a) and bit 31 (key b) after a left shift
-        // by 15 - 4e - i; set means -1 (fp16 sign bit) over 1.0 (0x3C00)
-        const uint32_t w01 = ~prmt(hs[0], hs[1], 0x5410u), w23 = ~prmt(hs[2], hs[3], 0x5410u);
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int e0 = 2 * h, e1 = 2 * h + 1;
-            const uint32_t a0 = ((w01 << (15 - 4 * e0 - i)) & 0x80008000u) | 0x3C003C00u;
-            const uint32_t a1 = ((w01 << (15 - 4 * e1 - i)) & 0x80008000u) | 0x3C003C00u;
-            const uint32_t a2 = ((w23 << (15 - 4 * e0 - i)) & 0x80008000u) | 0x3C003C00u;
-            const uint32_t a3 = ((w23 << (15 - 4 * e1 - i)) & 0x80008000u) | 0x3C003C00u;
-            mma_16816(accS[2 * i + h], a0, a1, a2, a3, bS0, bS1);
-          }
-      }
     }
+    __syncwarp();   // every lane is done with this stage before it is refilled
   }
   asm volatile("cp.async.wait_group 0;" ::: "memory");
-  __syncthreads();
+  // head hb's weight sum over this warp's keys: the lanes of one limb cover
+  // the step's keys once (the two limb lanes computed the same weights)
+  lsum += __shfl_xor_sync(0xffffffffu, lsum, 1);
+  lsum += __shfl_xor_sync(0xffffffffu, lsum, 2);
+  if (tig == 0 && (g & 1) == 0) {
+    wmax[warp][hb] = mrun;
+    wsum[warp][hb] = lsum;
+  }
+  __syncthreads();   // every warp is done with its ring: the reduction buffer reuses it
 
-  // the warps' accumulators meet in shared memory (the row ring and the
-  // weight buffers are free now): warp w writes its sums for head tig to
-  // red[w][tig][.], then every thread adds up the eight warps for its outputs
-  // (no atomics: the eight warps' sums for one output all hit one address)
-  constexpr int kRed = (JL ? 256 : 128) + 4;   // a row of red: a (128), b (128 or none), padding
-  static_assert(kAttWarps * GP * kRed * 4 <= kAttStages * T * rs + 2 * T * GP * 4 + GP * kAcc * 4,
-                "reduction buffer");
+  // the warps' accumulators meet in shared memory: warp w writes its sums for
+  // head tig to red[w][tig][.], relative to its own maximum; the block's
+  // record takes them relative to the block's maximum
+  static_assert(kAttWarps * GP * kRed * 4 <= kAttWarps * WR::kWarp, "reduction buffer");
   float* red = reinterpret_cast<float*>(sm);
   {
     // the rows of this thread's accumulators: unit g, register i, nibble e; head tig
@@ -611,12 +601,11 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_mma_kernel(
               make_float2(accS[2 * i + h][0] + accS[2 * i + h][1], accS[2 * i + h][2] + accS[2 * i + h][3]);
       }
   }
-#pragma unroll
-  for (int it = 0; it < kWIt; ++it) {
-    float v = lsum[it];
-    for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    const int h = (tid + it * kAttThreads) / T;
-    if (lane == 0 && h < GP) atomicAdd(sl + h, v);
+  if (tid < kAttWarps * GP) {
+    const int w = tid / GP, h = tid - w * GP;
+    float M = wmax[0][h];
+    for (int v = 1; v < kAttWarps; ++v) M = fmaxf(M, wmax[v][h]);
+    wfac[w][h] = wmax[w][h] == -INFINITY ? 0.f : exp2f((wmax[w][h] - M) * kL2e);
   }
   __syncthreads();
   // partial record {max, sum, a[128], b[128 or 0]} in the generic layout (dp + mp slots)
@@ -625,13 +614,16 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_mma_kernel(
     const int h = o / (rec - 2), j = o - h * (rec - 2);
     float v = 0.f;
 #pragma unroll
-    for (int w = 0; w < kAttWarps; ++w) v += red[(w * GP + h) * kRed + j];
+    for (int w = 0; w < kAttWarps; ++w) v = fmaf(wfac[w][h], red[(w * GP + h) * kRed + j], v);
     part[(size_t(blockIdx.x) * G + h) * rec + 2 + j] = v;
   }
   if (tid < G) {
+    float M = wmax[0][tid], L = 0.f;
+    for (int w = 1; w < kAttWarps; ++w) M = fmaxf(M, wmax[w][tid]);
+    for (int w = 0; w < kAttWarps; ++w) L = fmaf(wfac[w][tid], wsum[w][tid], L);
     float* out = part + (size_t(blockIdx.x) * G + tid) * rec;
-    out[0] = smx[tid];
-    out[1] = sl[tid];
+    out[0] = M;
+    out[1] = L;
   }
 }
 
@@ -712,13 +704,15 @@ struct AttPlan {
   int64_t chunk;
 };
 
-AttPlan att_plan(int B, int Hkv, int64_t S) {
+// Key chunks per (batch, KV head).  The time is the number of waves of
+// resident blocks (two per SM) times a block's time, taken as a fixed part
+// plus the chunk length.  The tensor-core kernel's fixed part (ring fill,
+// the merge of its warps' partial sums) was measured at the cost of about
+// 180 keys; the CUDA-core kernel's is charged as a small cost per split.
+AttPlan att_plan(int B, int Hkv, int64_t S, bool mma) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // key chunks per (batch, KV head): the number of waves of resident blocks
-  // (two per SM) times the chunk length is the time; take the split count
-  // that minimises it, with a small cost per split for the merge
   const int64_t groups = int64_t(B) * Hkv;
   const int64_t cap = int64_t(sms) * 2;
   int64_t max_ns = (S + kAttTile - 1) / kAttTile;
@@ -728,7 +722,8 @@ AttPlan att_plan(int B, int Hkv, int64_t S) {
   double best_cost = 1e300;
   for (int64_t ns = 1; ns <= max_ns; ++ns) {
     const double waves = double((groups * ns + cap - 1) / cap);
-    const double cost = waves / double(ns) + 0.0002 * double(ns);
+    const double cost = mma ? waves * (180.0 + double(S) / double(ns))
+                            : waves / double(ns) + 0.0002 * double(ns);
     if (cost < best_cost) {
       best_cost = cost;
       best = ns;
@@ -740,6 +735,12 @@ AttPlan att_plan(int B, int Hkv, int64_t S) {
   int64_t ns = (S + chunk - 1) / chunk;
   if (ns < 1) ns = 1;
   return AttPlan{int(ns), chunk};
+}
+
+// The tensor-core kernel serves d = m = 128 (or m = 0) with up to 4 query
+// heads per KV head.
+bool attend_uses_mma(const tq_ctx* ctx, int Hq, int Hkv) {
+  return ctx->d == 128 && (ctx->m == 128 || ctx->m == 0) && Hq / Hkv <= 4;
 }
 
 template <int BM, int GP, int NS>
@@ -774,10 +775,7 @@ cudaError_t launch_mma_partial(const tq_ctx* ctx, const float* logits, int B, in
     lut.lo[v / 4] |= uint32_t(bits & 0xFF) << (8 * (v % 4));
     lut.hi[v / 4] |= uint32_t(bits >> 8) << (8 * (v % 4));
   }
-  constexpr int rb = 8 * (2 * BM + (JL ? 2 : 0));
-  constexpr int rs = (rb / 16) % 2 ? rb : rb + 16;   // padded row stride (as in the kernel)
-  const size_t smem = size_t(kAttStages * kAttMmaTile) * rs + size_t(2 * kAttMmaTile * 4) * 4 + size_t(4 * 256) * 4 +
-                      size_t(4 * kAttWarps + 8) * 4;
+  const size_t smem = size_t(kAttWarps) * WarpRing<BM, JL>::kWarp;   // the warps' rings (then the reduction buffer)
   auto kern = attend_mma_kernel<BM, JL>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   kern<<<unsigned(int64_t(B) * Hkv * ap.nsplit), kAttThreads, smem, st>>>(logits, Hq, Hkv, S, ap.chunk, ap.nsplit,
@@ -802,7 +800,7 @@ bool attend_supported(const tq_ctx* ctx, int Hq, int Hkv) {
 }
 
 size_t attend_ws_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int64_t S) {
-  const AttPlan ap = att_plan(B, Hkv, S);
+  const AttPlan ap = att_plan(B, Hkv, S, attend_uses_mma(ctx, Hq, Hkv));
   const RowGeom g = make_geom(ctx->d, ctx->m, ctx->bmse);
   const size_t rec = size_t(2 + g.dp + g.mp);
   const size_t bytes = size_t(B) * Hkv * ap.nsplit * size_t(Hq / Hkv) * rec * 4;
@@ -811,12 +809,12 @@ size_t attend_ws_bytes(const tq_ctx* ctx, int B, int Hq, int Hkv, int64_t S) {
 
 cudaError_t launch_attend(const tq_ctx* ctx, const float* logits, int B, int Hq, int Hkv, int64_t S,
                           const uint8_t* payload, const uint16_t* norms, float* out, void* ws, cudaStream_t st) {
-  const AttPlan ap = att_plan(B, Hkv, S);
+  const AttPlan ap = att_plan(B, Hkv, S, attend_uses_mma(ctx, Hq, Hkv));
   const RowGeom g = make_geom(ctx->d, ctx->m, ctx->bmse);
   float* part = static_cast<float*>(ws);
   const bool two = g.dp > 128 || g.mp > 128;
   cudaError_t e;
-  if (ctx->d == 128 && (ctx->m == 128 || ctx->m == 0) && Hq / Hkv <= 4) {
+  if (attend_uses_mma(ctx, Hq, Hkv)) {
     // tensor-core partial sums
     switch (ctx->bmse * 2 + (ctx->m > 0 ? 1 : 0)) {
       case 2: e = launch_mma_partial<1, false>(ctx, logits, B, Hq, Hkv, S, ap, payload, norms, part, st); break;
