@@ -627,6 +627,23 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_mma_kernel(
   }
 }
 
+// sum over k in [k0, k1) of M[k][j] v[k], M row-major with rows of length d
+// (threads of consecutive j read consecutive addresses): sixteen loads are
+// issued before their products, four accumulators.
+__device__ __forceinline__ float colsum(const float* __restrict__ M, int d, int j, const float* v, int k0, int k1) {
+  float t[4] = {0.f, 0.f, 0.f, 0.f};
+  int k = k0;
+  for (; k + 16 <= k1; k += 16) {
+    float mv[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) mv[u] = __ldg(M + size_t(k + u) * d + j);
+#pragma unroll
+    for (int u = 0; u < 16; ++u) t[u & 3] = fmaf(mv[u], v[k + u], t[u & 3]);
+  }
+  for (; k < k1; ++k) t[0] = fmaf(__ldg(M + size_t(k) * d + j), v[k], t[0]);
+  return (t[0] + t[1]) + (t[2] + t[3]);
+}
+
 // One block per query head: merge the chunk partials, then
 // o = R^T (a + sqrt(pi/2)/m P^T b) / L.
 __global__ void __launch_bounds__(256) attend_combine_kernel(const float* __restrict__ part, int Hq, int Hkv,
@@ -679,24 +696,27 @@ __global__ void __launch_bounds__(256) attend_combine_kernel(const float* __rest
   __syncthreads();
   const float inv = L > 0.f ? 1.f / L : 0.f;
   const float qc = m > 0 ? float(kQjlConst) / float(m) : 0.f;
+  // the two products run two threads per output when d <= 128 (each half of
+  // the sum); each thread loads 16 matrix entries before it multiplies, so
+  // that the L2 latency is paid once per 16 terms
+  __shared__ float sp[2][256];
+  const int nh = 2 * d <= int(blockDim.x) ? 2 : 1;
+  const int jt = int(threadIdx.x) % d, ht = int(threadIdx.x) / d;
+  if (ht < nh) sp[ht][jt] = colsum(P, d, jt, sb, m * ht / nh, m * (ht + 1) / nh);   // (P^T b)_j, part ht
+  __syncthreads();
   float u_own = 0.f;
   if (threadIdx.x < d) {
     const int j = threadIdx.x;
-    float t = 0.f;
-#pragma unroll 8
-    for (int k = 0; k < m; ++k) t = fmaf(P[size_t(k) * d + j], sb[k], t);
+    const float t = nh == 2 ? sp[0][j] + sp[1][j] : sp[0][j];
     u_own = (sa[j] + qc * t) * inv;
   }
   __syncthreads();
   if (threadIdx.x < d) sa[threadIdx.x] = u_own;
   __syncthreads();
-  if (threadIdx.x < d) {
-    const int i = threadIdx.x;
-    float o = 0.f;
-#pragma unroll 8
-    for (int j = 0; j < d; ++j) o = fmaf(R[size_t(j) * d + i], sa[j], o);
-    out[size_t(bh) * d + i] = o;
-  }
+  if (ht < nh) sp[ht][jt] = colsum(R, d, jt, sa, d * ht / nh, d * (ht + 1) / nh);   // (R^T u)_i, part ht
+  __syncthreads();
+  if (threadIdx.x < d) out[size_t(bh) * d + threadIdx.x] = nh == 2 ? sp[0][threadIdx.x] + sp[1][threadIdx.x]
+                                                                 : sp[0][threadIdx.x];
 }
 
 struct AttPlan {
