@@ -16,8 +16,9 @@
 // query head of the group, the chunk's maximum logit, the sum of its weights
 // and its a, b (flash-decoding style partials), by one of two kernels:
 //   attend_mma_kernel (d = m = 128 or m = 0, up to 4 query heads per KV
-//     head): fp16 tensor-core MMAs over 16-key steps, described above the
-//     kernel;
+//     head): fp16 tensor-core MMAs over 16-key steps; each warp takes a
+//     contiguous share of the chunk with its own running maximum, and the
+//     block merges its eight warps' partials (described above the kernel);
 //   attend_partial_kernel (every other shape): key tiles of 128 rows staged
 //     in shared memory (prefetched into registers one tile ahead); warp w
 //     takes the key pairs (k, k + 64) for k = w, w + 8, ...; lane L decodes
@@ -305,6 +306,13 @@ __global__ void __launch_bounds__(kAttThreads, GP * NS <= 2 ? 3 : (GP * NS <= 4 
 // fp16 hi + lo limbs.  Precision: each product carries the fp16 rounding of
 // its codebook level (<= 2^-11 relative) and of the weight's hi + lo split
 // (<= 2^-22); sums are fp32.
+// Schedule: a warp streams its share of the block's chunk in 16-key steps
+// through a private four-stage cp.async ring (rows, logits, norms), with no
+// block-wide barrier until the end.  Weights are exp(l - M) against the
+// warp's running maximum M per head (flash-decoding's online softmax): when a
+// step raises M, the warp's accumulators and weight sum are scaled by
+// exp(M_old - M_new) first.  At the end the eight warps' partial sums meet in
+// shared memory, each scaled to the block's maximum.
 // ---------------------------------------------------------------------------
 
 // fp16 bits of the codebook levels as two byte planes (level v: lo byte v, hi byte v).
