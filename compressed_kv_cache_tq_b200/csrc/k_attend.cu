@@ -633,6 +633,8 @@ __global__ void __launch_bounds__(kAttThreads, 2) attend_mma_kernel(
     out[0] = M;
     out[1] = L;
   }
+  // the merge kernel may be scheduled once every block has written its record
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 // sum over k in [k0, k1) of M[k][j] v[k], M row-major with rows of length d
@@ -658,6 +660,8 @@ __global__ void __launch_bounds__(256) attend_combine_kernel(const float* __rest
                                                              int nsplit, const float* __restrict__ R,
                                                              const float* __restrict__ P, int d, int m, RowGeom g,
                                                              float* __restrict__ out) {
+  // launched as a programmatic dependent of the partial sums: wait for their records
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   extern __shared__ float sv[];
   float* sa = sv;          // [dp] merged a, then u
   float* sb = sa + g.dp;   // [mp] merged b
@@ -857,10 +861,21 @@ cudaError_t launch_attend(const tq_ctx* ctx, const float* logits, int B, int Hq,
             : dispatch_bits<1>(ctx, logits, B, Hq, Hkv, S, ap, payload, norms, part, st);
   }
   if (e != cudaSuccess) return e;
-  const size_t smem = size_t(g.dp + g.mp) * 4;
-  attend_combine_kernel<<<unsigned(B * Hq), 256, smem, st>>>(part, Hq, Hkv, ap.nsplit, ctx->dR, ctx->dP, ctx->d,
-                                                             ctx->m, g, out);
-  return cudaGetLastError();
+  // the merge overlaps its launch with the end of the partial sums
+  // (programmatic dependent launch; it waits for their completion first)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(B * Hq));
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = size_t(g.dp + g.mp) * 4;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, attend_combine_kernel, static_cast<const float*>(part), Hq, Hkv, ap.nsplit,
+                            static_cast<const float*>(ctx->dR), static_cast<const float*>(ctx->dP), ctx->d, ctx->m, g,
+                            out);
 }
 
 }  // namespace tq

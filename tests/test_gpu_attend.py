@@ -58,6 +58,35 @@ def test_attend_against_oracle(lib, B, Hkv, G, S, d, bits, m):
     check_close(out.cpu().numpy(), ref, A)
 
 
+def test_attend_running_maximum_and_masked_keys(lib):
+    """Logits whose maximum keeps rising along the keys (each warp's running
+    maximum, and with it every partial sum, is rescaled many times), falling
+    ones, a wide range (most weights underflow), and masked keys (-inf): a
+    random 30 % of the keys, and the whole first half of one head's keys, so
+    that some chunks of that head have no weight at all."""
+    B, Hkv, G, S, d = 1, 2, 4, 3000, 128
+    ctx = lib.tq_init(d, 4, 91)
+    v, V64 = _values(B, Hkv, S, d, seed=4401)
+    payload, norms = lib.tq_quantize(ctx, v)
+    tb = tables_of(ctx)
+    logits = W.queries((B, Hkv * G, S), seed=4402).astype(np.float64)
+    ramp = np.arange(S) / S
+    logits[0, 0] += 40.0 * ramp            # rising
+    logits[0, 1] -= 40.0 * ramp            # falling
+    logits[0, 2] *= 20.0                   # wide range
+    logits[0, 3] += 8.0 * np.sin(ramp * 37.0)
+    rng = np.random.default_rng(4403)
+    logits[0, 4:8][:, rng.random(S) < 0.3] = -np.inf
+    logits[0, 5, : S // 2] = -np.inf
+    out = lib.tq_attend(ctx, torch.from_numpy(logits.astype(np.float32)).to(DEV), payload, norms, Hkv)
+    torch.cuda.synchronize()
+    ref, A = _oracle_attention(logits.astype(np.float32).astype(np.float64), payload.cpu().numpy(),
+                               norms.cpu().numpy(), tb, Hkv)
+    got = out.cpu().numpy()
+    assert np.isfinite(got).all()
+    check_close(got, ref, A)
+
+
 def test_attend_without_keys_is_zero(lib):
     ctx = lib.tq_init(128, 4, 77)
     payload = torch.empty((0, ctx.row_bytes), dtype=torch.uint8, device=DEV)
