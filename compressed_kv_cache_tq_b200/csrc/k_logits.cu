@@ -56,9 +56,10 @@ __device__ __forceinline__ bool reg3_coordinate(int j) { return ((j >> 2) & 3) =
 // ---------------------------------------------------------------------------
 // Query preparation: x = R q, y = P x (= S q), int16 fixed point per head,
 // split into two signed int8 limbs, written in MMA B-fragment order.
-// One block per (batch, KV head group, chunk of up to 8 query heads): it
-// computes the NT head slots of the chunk (slots past the group's heads are
-// zero).  R^T and P^T are copied to shared memory (128 KB) at once.
+// One block per (batch, KV head group, up to kQChunks chunks of up to 8
+// query heads): R^T and P^T are copied to shared memory (128 KB) once, then
+// the block computes the NT head slots of each of its chunks in turn (slots
+// past the group's heads are zero).
 //
 // The logits kernel turns a one-bit field (sign bit, or a one-bit code) into
 // operand bytes a = -bit (registers 0..2 of a unit) or a = 1 - bit (register
@@ -69,30 +70,33 @@ __device__ __forceinline__ bool reg3_coordinate(int j) { return ((j >> 2) & 3) =
 // One-bit codes (levels -c1, +c1) use the same form with x.
 // ---------------------------------------------------------------------------
 constexpr int kMaxSlots = 8;
+constexpr int kQChunks = 8;   // head chunks per query-preparation block (64 heads)
 
-__global__ void __launch_bounds__(128) qprep_kernel(const float* __restrict__ q, int Hq, int Hkv, int nchunk, int nt,
+__global__ void __launch_bounds__(256) qprep_kernel(const float* __restrict__ q, int Hq, int Hkv, int nchunk, int nt,
                                                     const float* __restrict__ Rt, const float* __restrict__ Pt,
                                                     float code_inv_scale, float scale, float qjl_over_m,
                                                     int one_bit_codes, uint32_t* __restrict__ frags,
                                                     HeadScale* __restrict__ hscale) {
-  extern __shared__ float smq[];
+  extern __shared__ __align__(16) float smq[];
   float* matR = smq;                                 // [D][D] R^T
   float* matP = matR + D * D;                        // [D][D] P^T
   float* sq = matP + D * D;                          // [slots][D] queries
   float* sx = sq + kMaxSlots * D;                    // [slots][D] x
   __shared__ float red[2][kMaxSlots][4];
-  __shared__ int ired[4][kMaxSlots][4];              // [Y, Y3, X, X3][slot][warp]
+  __shared__ int ired[4][kMaxSlots][4];              // [Y, Y3, X, X3][slot][warp of the quad]
   __shared__ int8_t limbs[kMaxSlots][2][2][D];       // [slot][x/y][hi/lo][coordinate]
   const int G = Hq / Hkv;
   const int slots = nt * HPT;
-  const int vg = blockIdx.x, grp = vg / nchunk, chunk = vg - grp * nchunk;
+  const int nblk = (nchunk + kQChunks - 1) / kQChunks;
+  const int grp = blockIdx.x / nblk, cb = blockIdx.x - grp * nblk;
   const int b = grp / Hkv, hkv = grp % Hkv;
-  const int h0 = chunk * 2 * HPT;                    // first head of the chunk within the group
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // thread (quad hq, coordinate j): the slots 4 hq .. 4 hq + 3 at coordinate j
+  const int j = tid & (D - 1), hq = tid >> 7, wq = warp & 3;
   // the logits grid may start streaming the cache now; it waits for this grid before reading fragments
   asm volatile("griddepcontrol.launch_dependents;");
   // both matrices in flight at once (asynchronous 16-byte copies)
-  for (int i = tid; i < D * D / 4; i += 128) {
+  for (int i = tid; i < D * D / 4; i += 256) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(uint32_t(__cvta_generic_to_shared(matR + 4 * i))),
                  "l"(Rt + 4 * i)
                  : "memory");
@@ -101,116 +105,129 @@ __global__ void __launch_bounds__(128) qprep_kernel(const float* __restrict__ q,
                    "l"(Pt + 4 * i)
                    : "memory");
   }
-  for (int h = 0; h < slots; ++h)
-    sq[h * D + tid] = h0 + h < G ? q[(size_t(b) * Hq + hkv * G + h0 + h) * D + tid] : 0.f;
-  asm volatile("cp.async.wait_all;" ::: "memory");
-  __syncthreads();
-  float acc[kMaxSlots];
+  // 128 x 128 matrix (transposed, in shared memory) times the quad's four
+  // vectors v[4 hq + k] (in shared memory, read four coordinates at a time)
+  auto matvec4 = [&](const float* mat, const float* v, float (&acc)[4]) {
 #pragma unroll
-  for (int h = 0; h < kMaxSlots; ++h) acc[h] = 0.f;
-#pragma unroll 4
-  for (int i = 0; i < D; ++i) {
-    const float r = matR[i * D + tid];
+    for (int k = 0; k < 4; ++k) acc[k] = 0.f;
+#pragma unroll 2
+    for (int i = 0; i < D; i += 4) {
+      const float r0 = mat[i * D + j], r1 = mat[(i + 1) * D + j], r2 = mat[(i + 2) * D + j],
+                  r3 = mat[(i + 3) * D + j];
 #pragma unroll
-    for (int h = 0; h < kMaxSlots; ++h)
-      if (h < slots) acc[h] = fmaf(r, sq[h * D + i], acc[h]);
-  }
-#pragma unroll
-  for (int h = 0; h < kMaxSlots; ++h)
-    if (h < slots) sx[h * D + tid] = acc[h];
-  __syncthreads();
-  float accy[kMaxSlots];
-#pragma unroll
-  for (int h = 0; h < kMaxSlots; ++h) accy[h] = 0.f;
-  if (Pt) {
-#pragma unroll 4
-    for (int j = 0; j < D; ++j) {
-      const float p = matP[j * D + tid];
-#pragma unroll
-      for (int h = 0; h < kMaxSlots; ++h)
-        if (h < slots) accy[h] = fmaf(p, sx[h * D + j], accy[h]);
+      for (int k = 0; k < 4; ++k) {
+        const float4 vv = *reinterpret_cast<const float4*>(v + (4 * hq + k) * D + i);
+        acc[k] = fmaf(r3, vv.w, fmaf(r2, vv.z, fmaf(r1, vv.y, fmaf(r0, vv.x, acc[k]))));
+      }
     }
-  }
-  // per-slot max |x|, max |y|
+  };
+  const bool quad_on = 4 * hq < slots;              // nt = 1: only the first quad has slots
+  const int c_end = (cb + 1) * kQChunks < nchunk ? (cb + 1) * kQChunks : nchunk;
+  for (int chunk = cb * kQChunks; chunk < c_end; ++chunk) {
+    const int vg = grp * nchunk + chunk;
+    const int h0 = chunk * 2 * HPT;                  // first head of the chunk within the group
+    if (chunk > cb * kQChunks) __syncthreads();       // the previous chunk's buffers are read
+    for (int idx = tid; idx < slots * D; idx += 256) {
+      const int h = idx / D, c = idx - h * D;
+      sq[idx] = h0 + h < G ? q[(size_t(b) * Hq + hkv * G + h0 + h) * D + c] : 0.f;
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncthreads();
+    float acc[4], accy[4];
+    if (quad_on) {
+      matvec4(matR, sq, acc);
 #pragma unroll
-  for (int h = 0; h < kMaxSlots; ++h) {
-    if (h >= slots) break;
-    float ax = fabsf(acc[h]), ay = fabsf(accy[h]);
-    for (int o = 16; o; o >>= 1) {
-      ax = fmaxf(ax, __shfl_xor_sync(0xffffffffu, ax, o));
-      ay = fmaxf(ay, __shfl_xor_sync(0xffffffffu, ay, o));
+      for (int k = 0; k < 4; ++k) sx[(4 * hq + k) * D + j] = acc[k];
     }
-    if (lane == 0) {
-      red[0][h][warp] = ax;
-      red[1][h][warp] = ay;
-    }
-  }
-  __syncthreads();
-  float kxs[kMaxSlots], kys[kMaxSlots];
+    __syncthreads();
 #pragma unroll
-  for (int h = 0; h < kMaxSlots; ++h) {
-    if (h >= slots) break;
-    const float mx = fmaxf(fmaxf(red[0][h][0], red[0][h][1]), fmaxf(red[0][h][2], red[0][h][3]));
-    const float my = fmaxf(fmaxf(red[1][h][0], red[1][h][1]), fmaxf(red[1][h][2], red[1][h][3]));
-    const float kx = mx > 0.f ? 32000.f / mx : 0.f;
-    const float ky = my > 0.f ? 32000.f / my : 0.f;
-    kxs[h] = kx;
-    kys[h] = ky;
-    const int xi = __float2int_rn(acc[h] * kx);
-    const int yi = __float2int_rn(accy[h] * ky);
-    // the B operand holds -y (and -x for one-bit codes): see the comment above
-    const int xb = one_bit_codes ? -xi : xi, yb = -yi;
-    const int xh = (xb + 128) >> 8, yh = (yb + 128) >> 8;
-    limbs[h][0][0][tid] = int8_t(xh);
-    limbs[h][0][1][tid] = int8_t(xb - 256 * xh);
-    limbs[h][1][0][tid] = int8_t(yh);
-    limbs[h][1][1][tid] = int8_t(yb - 256 * yh);
-    int ty = yi, ty3 = reg3_coordinate(tid) ? yi : 0, tx = xi, tx3 = reg3_coordinate(tid) ? xi : 0;
-    for (int o = 16; o; o >>= 1) {
-      ty += __shfl_xor_sync(0xffffffffu, ty, o);
-      ty3 += __shfl_xor_sync(0xffffffffu, ty3, o);
-      tx += __shfl_xor_sync(0xffffffffu, tx, o);
-      tx3 += __shfl_xor_sync(0xffffffffu, tx3, o);
-    }
-    if (lane == 0) {
-      ired[0][h][warp] = ty;
-      ired[1][h][warp] = ty3;
-      ired[2][h][warp] = tx;
-      ired[3][h][warp] = tx3;
-    }
-  }
-  __syncthreads();
+    for (int k = 0; k < 4; ++k) accy[k] = 0.f;
+    if (quad_on && Pt) matvec4(matP, sx, accy);
+    // per-slot max |x|, max |y| over the quad's four warps
+    if (quad_on) {
 #pragma unroll
-  for (int h = 0; h < kMaxSlots; ++h) {
-    if (h >= slots) break;
-    if (tid == 0 && h0 + h < G) {
-      const int Y = ired[0][h][0] + ired[0][h][1] + ired[0][h][2] + ired[0][h][3];
-      const int Y3 = ired[1][h][0] + ired[1][h][1] + ired[1][h][2] + ired[1][h][3];
-      const int X = ired[2][h][0] + ired[2][h][1] + ired[2][h][2] + ired[2][h][3];
-      const int X3 = ired[3][h][0] + ired[3][h][1] + ired[3][h][2] + ired[3][h][3];
-      HeadScale hs;
-      hs.code = kxs[h] > 0.f ? scale * code_inv_scale / kxs[h] : 0.f;
-      hs.sign = kys[h] > 0.f ? scale * qjl_over_m / kys[h] : 0.f;
-      hs.ccode = 2 * X3 - X;
-      hs.csign = 2 * Y3 - Y;
-      hscale[size_t(b) * Hq + hkv * G + h0 + h] = hs;
+      for (int k = 0; k < 4; ++k) {
+        float ax = fabsf(acc[k]), ay = fabsf(accy[k]);
+        for (int o = 16; o; o >>= 1) {
+          ax = fmaxf(ax, __shfl_xor_sync(0xffffffffu, ax, o));
+          ay = fmaxf(ay, __shfl_xor_sync(0xffffffffu, ay, o));
+        }
+        if (lane == 0) {
+          red[0][4 * hq + k][wq] = ax;
+          red[1][4 * hq + k][wq] = ay;
+        }
+      }
     }
-  }
-  __syncthreads();
-  // Fragment word (xy, s, reg, lane) of N-tile t holds B[k = 16 reg + 4 tig + e][n = lane / 4],
-  // e = 0..3; column n is (head slot 4 t + n / 2, limb n % 2); K position k of step s is
-  // coordinate tig * D/4 + 4 (2s + reg) + e.
-  for (int w = tid; w < nt * kFragWords; w += 128) {
-    const int t = w / kFragWords, rem = w - t * kFragWords;
-    const int ln = rem & 31, reg = (rem >> 5) & 1, s = (rem >> 6) % KS, xy = (rem >> 6) / KS;
-    const int n = ln >> 2, tig = ln & 3;
-    const int slot = t * HPT + (n >> 1), limb = n & 1;
-    uint32_t word = 0;
-    for (int e = 0; e < 4; ++e) {
-      const int j = tig * (D / 4) + 4 * (2 * s + reg) + e;
-      word |= uint32_t(uint8_t(limbs[slot][xy][limb][j])) << (8 * e);
+    __syncthreads();
+    float kxs[4], kys[4];
+    if (quad_on) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int h = 4 * hq + k;
+        const float mx = fmaxf(fmaxf(red[0][h][0], red[0][h][1]), fmaxf(red[0][h][2], red[0][h][3]));
+        const float my = fmaxf(fmaxf(red[1][h][0], red[1][h][1]), fmaxf(red[1][h][2], red[1][h][3]));
+        const float kx = mx > 0.f ? 32000.f / mx : 0.f;
+        const float ky = my > 0.f ? 32000.f / my : 0.f;
+        kxs[k] = kx;
+        kys[k] = ky;
+        const int xi = __float2int_rn(acc[k] * kx);
+        const int yi = __float2int_rn(accy[k] * ky);
+        // the B operand holds -y (and -x for one-bit codes): see the comment above
+        const int xb = one_bit_codes ? -xi : xi, yb = -yi;
+        const int xh = (xb + 128) >> 8, yh = (yb + 128) >> 8;
+        limbs[h][0][0][j] = int8_t(xh);
+        limbs[h][0][1][j] = int8_t(xb - 256 * xh);
+        limbs[h][1][0][j] = int8_t(yh);
+        limbs[h][1][1][j] = int8_t(yb - 256 * yh);
+        int ty = yi, ty3 = reg3_coordinate(j) ? yi : 0, tx = xi, tx3 = reg3_coordinate(j) ? xi : 0;
+        for (int o = 16; o; o >>= 1) {
+          ty += __shfl_xor_sync(0xffffffffu, ty, o);
+          ty3 += __shfl_xor_sync(0xffffffffu, ty3, o);
+          tx += __shfl_xor_sync(0xffffffffu, tx, o);
+          tx3 += __shfl_xor_sync(0xffffffffu, tx3, o);
+        }
+        if (lane == 0) {
+          ired[0][h][wq] = ty;
+          ired[1][h][wq] = ty3;
+          ired[2][h][wq] = tx;
+          ired[3][h][wq] = tx3;
+        }
+      }
     }
-    frags[size_t(vg) * nt * kFragWords + w] = word;
+    __syncthreads();
+    if (quad_on && j == 0) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int h = 4 * hq + k;
+        if (h0 + h < G) {
+          const int Y = ired[0][h][0] + ired[0][h][1] + ired[0][h][2] + ired[0][h][3];
+          const int Y3 = ired[1][h][0] + ired[1][h][1] + ired[1][h][2] + ired[1][h][3];
+          const int X = ired[2][h][0] + ired[2][h][1] + ired[2][h][2] + ired[2][h][3];
+          const int X3 = ired[3][h][0] + ired[3][h][1] + ired[3][h][2] + ired[3][h][3];
+          HeadScale hsc;
+          hsc.code = kxs[k] > 0.f ? scale * code_inv_scale / kxs[k] : 0.f;
+          hsc.sign = kys[k] > 0.f ? scale * qjl_over_m / kys[k] : 0.f;
+          hsc.ccode = 2 * X3 - X;
+          hsc.csign = 2 * Y3 - Y;
+          hscale[size_t(b) * Hq + hkv * G + h0 + h] = hsc;
+        }
+      }
+    }
+    // Fragment word (xy, s, reg, lane) of N-tile t holds B[k = 16 reg + 4 tig + e][n = lane / 4],
+    // e = 0..3; column n is (head slot 4 t + n / 2, limb n % 2); K position k of step s is
+    // coordinate tig * D/4 + 4 (2s + reg) + e.
+    for (int w = tid; w < nt * kFragWords; w += 256) {
+      const int t = w / kFragWords, rem = w - t * kFragWords;
+      const int ln = rem & 31, reg = (rem >> 5) & 1, s = (rem >> 6) % KS, xy = (rem >> 6) / KS;
+      const int n = ln >> 2, tig = ln & 3;
+      const int slot = t * HPT + (n >> 1), limb = n & 1;
+      uint32_t word = 0;
+      for (int e = 0; e < 4; ++e) {
+        const int c = tig * (D / 4) + 4 * (2 * s + reg) + e;
+        word |= uint32_t(uint8_t(limbs[slot][xy][limb][c])) << (8 * e);
+      }
+      frags[size_t(vg) * nt * kFragWords + w] = word;
+    }
   }
 }
 
@@ -1056,7 +1073,7 @@ cudaError_t launch_logits(const tq_ctx* ctx, const float* q, int B, int Hq, int 
   cudaFuncSetAttribute(qprep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(qp_smem));
   // one-bit codes (levels -c1, +c1) use the one-bit operand form: the code scale is c1
   const float code_scale = ctx->bmse == 1 ? float(ctx->c[1]) : ctx->lut.inv_scale;
-  qprep_kernel<<<unsigned(groups * nchunk), 128, qp_smem, st>>>(
+  qprep_kernel<<<unsigned(groups * ((nchunk + kQChunks - 1) / kQChunks)), 256, qp_smem, st>>>(
       q, Hq, Hkv, nchunk, nt, ctx->dRt, ctx->dPt, code_scale, scale,
       float(ctx->m > 0 ? kQjlConst / ctx->m : 0.0), ctx->bmse == 1 ? 1 : 0, frags, hs);
   cudaError_t e = cudaGetLastError();
