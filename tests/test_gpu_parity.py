@@ -234,10 +234,12 @@ def _cache(lib, ctx, B, Hkv, S, seed):
 @pytest.mark.parametrize("m", [128, 0])
 @pytest.mark.parametrize("bits,B,Hkv,G,S", [(3, 2, 2, 4, 1037), (4, 1, 3, 4, 515), (4, 2, 2, 1, 200),
                                             (3, 1, 2, 2, 333), (2, 2, 1, 8, 129), (4, 1, 1, 12, 100),
-                                            (4, 1, 2, 3, 16)])
+                                            (4, 1, 2, 3, 16), (3, 1, 1, 64, 300), (4, 2, 1, 16, 257),
+                                            (2, 1, 2, 12, 100), (4, 1, 1, 9, 77)])
 def test_logits_against_oracle(lib, bits, B, Hkv, G, S, m):
-    """With the sign term (m = 128) and without it (m = 0, MSE-only); G <= 8
-    runs on the int8 MMA kernel, G = 12 on CUDA cores."""
+    """With the sign term (m = 128) and without it (m = 0, MSE-only), on the
+    int8 MMA kernel; G > 8 (9, 12, 16 and the toy batch's 64) runs as chunks
+    of 8 query heads that each stream the rows again."""
     ctx = _ctx(lib, bits=bits, seed=21, m=m)
     payload, norms = _cache(lib, ctx, B, Hkv, S, seed=31)
     Hq = Hkv * G
