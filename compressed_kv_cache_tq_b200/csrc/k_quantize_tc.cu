@@ -415,25 +415,37 @@ __global__ void __launch_bounds__(QLayout<F32>::kThreads, 1) quantize_tc_kernel(
       if (!mbar_wait_warp(bar(QL::kKFull + sb), uint32_t((j / kStageF32) & 1), abort_flag, status)) break;
       const uint8_t* src = sbase + kOffStageF + 16384u * sb;
       uint8_t* dst = sbase + kOffRingF + 32768u * rs;
-#pragma unroll 2
-      for (int gi = c; gi < 512; gi += 64) {
-        const int r = gi >> 2, g = gi & 3;
-        const float4 a = *reinterpret_cast<const float4*>(src + r * 128 + (((2 * g) ^ (r & 7)) << 4));
-        const float4 b = *reinterpret_cast<const float4*>(src + r * 128 + (((2 * g + 1) ^ (r & 7)) << 4));
-        const float2 x[4] = {make_float2(a.x, a.y), make_float2(a.z, a.w), make_float2(b.x, b.y),
-                             make_float2(b.z, b.w)};
-        uint32_t hi[4], lo[4];
+      // thread c converts rows c / 4 + 16 u (u = 0..7) of 8-float group c % 4, four
+      // rows' loads issued before their conversions and stores (the swizzle of
+      // those rows is the same: r % 8 = (c / 4) % 8)
+      const int r0 = c >> 2, g = c & 3, sw = r0 & 7;
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const __nv_bfloat162 h = __float22bfloat162_rn(x[t]);
-          const float2 hf = __bfloat1622float2(h);
-          const __nv_bfloat162 l = __float22bfloat162_rn(__ffma2_rn(hf, f2(-1.f), x[t]));
-          hi[t] = *reinterpret_cast<const uint32_t*>(&h);
-          lo[t] = *reinterpret_cast<const uint32_t*>(&l);
+      for (int b4 = 0; b4 < 2; ++b4) {
+        float4 va[4], vb[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int r = r0 + 16 * (4 * b4 + u);
+          va[u] = *reinterpret_cast<const float4*>(src + r * 128 + (((2 * g) ^ sw) << 4));
+          vb[u] = *reinterpret_cast<const float4*>(src + r * 128 + (((2 * g + 1) ^ sw) << 4));
         }
-        const uint32_t off = uint32_t(r * 128 + (((4 * (q & 1) + g) ^ (r & 7)) << 4));
-        *reinterpret_cast<uint4*>(dst + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-        *reinterpret_cast<uint4*>(dst + 16384u + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int r = r0 + 16 * (4 * b4 + u);
+          const float2 x[4] = {make_float2(va[u].x, va[u].y), make_float2(va[u].z, va[u].w), make_float2(vb[u].x, vb[u].y),
+                               make_float2(vb[u].z, vb[u].w)};
+          uint32_t hi[4], lo[4];
+#pragma unroll
+          for (int t = 0; t < 4; ++t) {
+            const __nv_bfloat162 h = __float22bfloat162_rn(x[t]);
+            const float2 hf = __bfloat1622float2(h);
+            const __nv_bfloat162 l = __float22bfloat162_rn(__ffma2_rn(hf, f2(-1.f), x[t]));
+            hi[t] = *reinterpret_cast<const uint32_t*>(&h);
+            lo[t] = *reinterpret_cast<const uint32_t*>(&l);
+          }
+          const uint32_t off = uint32_t(r * 128 + (((4 * (q & 1) + g) ^ sw) << 4));
+          *reinterpret_cast<uint4*>(dst + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+          *reinterpret_cast<uint4*>(dst + 16384u + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
       }
       // the tensor core reads the ring through the async proxy
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -1279,25 +1291,37 @@ __global__ void __launch_bounds__(kWThreads, 1) quantize_wide_kernel(const __gri
         }
         const uint8_t* src = sbase + kWOffStage + 16384u * sb;
         uint8_t* dst = sbase + kWOffRing + 32768u * rs;
-#pragma unroll 2
-        for (int gi = c; gi < 512; gi += 64) {
-          const int r = gi >> 2, g = gi & 3;
-          const float4 a4 = *reinterpret_cast<const float4*>(src + r * 128 + (((2 * g) ^ (r & 7)) << 4));
-          const float4 b4 = *reinterpret_cast<const float4*>(src + r * 128 + (((2 * g + 1) ^ (r & 7)) << 4));
-          const float2 x[4] = {make_float2(a4.x, a4.y), make_float2(a4.z, a4.w), make_float2(b4.x, b4.y),
-                               make_float2(b4.z, b4.w)};
-          uint32_t hi[4], lo[4];
+        // thread c converts rows c / 4 + 16 u (u = 0..7) of 8-float group c % 4, four
+        // rows' loads issued before their conversions and stores (the swizzle of
+        // those rows is the same: r % 8 = (c / 4) % 8)
+        const int r0 = c >> 2, g = c & 3, sw = r0 & 7;
 #pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            const __nv_bfloat162 h = __float22bfloat162_rn(x[t]);
-            const float2 hf = __bfloat1622float2(h);
-            const __nv_bfloat162 l = __float22bfloat162_rn(__ffma2_rn(hf, f2(-1.f), x[t]));
-            hi[t] = *reinterpret_cast<const uint32_t*>(&h);
-            lo[t] = *reinterpret_cast<const uint32_t*>(&l);
+        for (int b4 = 0; b4 < 2; ++b4) {
+          float4 va[4], vb[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int r = r0 + 16 * (4 * b4 + u);
+            va[u] = *reinterpret_cast<const float4*>(src + r * 128 + (((2 * g) ^ sw) << 4));
+            vb[u] = *reinterpret_cast<const float4*>(src + r * 128 + (((2 * g + 1) ^ sw) << 4));
           }
-          const uint32_t off = uint32_t(r * 128 + (((4 * (q & 1) + g) ^ (r & 7)) << 4));
-          *reinterpret_cast<uint4*>(dst + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-          *reinterpret_cast<uint4*>(dst + 16384u + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int r = r0 + 16 * (4 * b4 + u);
+            const float2 x[4] = {make_float2(va[u].x, va[u].y), make_float2(va[u].z, va[u].w), make_float2(vb[u].x, vb[u].y),
+                                 make_float2(vb[u].z, vb[u].w)};
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+              const __nv_bfloat162 h = __float22bfloat162_rn(x[t]);
+              const float2 hf = __bfloat1622float2(h);
+              const __nv_bfloat162 l = __float22bfloat162_rn(__ffma2_rn(hf, f2(-1.f), x[t]));
+              hi[t] = *reinterpret_cast<const uint32_t*>(&h);
+              lo[t] = *reinterpret_cast<const uint32_t*>(&l);
+            }
+            const uint32_t off = uint32_t(r * 128 + (((4 * (q & 1) + g) ^ sw) << 4));
+            *reinterpret_cast<uint4*>(dst + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<uint4*>(dst + 16384u + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+          }
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         mbar_arrive(bar(kWSEmpty + sb));
