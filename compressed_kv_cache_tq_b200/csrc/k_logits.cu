@@ -56,7 +56,7 @@ __device__ __forceinline__ bool reg3_coordinate(int j) { return ((j >> 2) & 3) =
 // ---------------------------------------------------------------------------
 // Query preparation: x = R q, y = P x (= S q), int16 fixed point per head,
 // split into two signed int8 limbs, written in MMA B-fragment order.
-// One block per (batch, KV head group, up to kQChunks chunks of up to 8
+// One block per (batch, KV head group, up to cpb chunks of up to 8
 // query heads): R^T and P^T are copied to shared memory (128 KB) once, then
 // the block computes the NT head slots of each of its chunks in turn (slots
 // past the group's heads are zero).
@@ -70,9 +70,10 @@ __device__ __forceinline__ bool reg3_coordinate(int j) { return ((j >> 2) & 3) =
 // One-bit codes (levels -c1, +c1) use the same form with x.
 // ---------------------------------------------------------------------------
 constexpr int kMaxSlots = 8;
-constexpr int kQChunks = 8;   // head chunks per query-preparation block (64 heads)
+constexpr int kQChunks = 8;   // at most this many head chunks per query-preparation block
 
-__global__ void __launch_bounds__(256) qprep_kernel(const float* __restrict__ q, int Hq, int Hkv, int nchunk, int nt,
+__global__ void __launch_bounds__(256) qprep_kernel(const float* __restrict__ q, int Hq, int Hkv, int nchunk, int cpb,
+                                                    int nt,
                                                     const float* __restrict__ Rt, const float* __restrict__ Pt,
                                                     float code_inv_scale, float scale, float qjl_over_m,
                                                     int one_bit_codes, uint32_t* __restrict__ frags,
@@ -87,7 +88,7 @@ __global__ void __launch_bounds__(256) qprep_kernel(const float* __restrict__ q,
   __shared__ int8_t limbs[kMaxSlots][2][2][D];       // [slot][x/y][hi/lo][coordinate]
   const int G = Hq / Hkv;
   const int slots = nt * HPT;
-  const int nblk = (nchunk + kQChunks - 1) / kQChunks;
+  const int nblk = (nchunk + cpb - 1) / cpb;
   const int grp = blockIdx.x / nblk, cb = blockIdx.x - grp * nblk;
   const int b = grp / Hkv, hkv = grp % Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -122,11 +123,11 @@ __global__ void __launch_bounds__(256) qprep_kernel(const float* __restrict__ q,
     }
   };
   const bool quad_on = 4 * hq < slots;              // nt = 1: only the first quad has slots
-  const int c_end = (cb + 1) * kQChunks < nchunk ? (cb + 1) * kQChunks : nchunk;
-  for (int chunk = cb * kQChunks; chunk < c_end; ++chunk) {
+  const int c_end = (cb + 1) * cpb < nchunk ? (cb + 1) * cpb : nchunk;
+  for (int chunk = cb * cpb; chunk < c_end; ++chunk) {
     const int vg = grp * nchunk + chunk;
     const int h0 = chunk * 2 * HPT;                  // first head of the chunk within the group
-    if (chunk > cb * kQChunks) __syncthreads();       // the previous chunk's buffers are read
+    if (chunk > cb * cpb) __syncthreads();            // the previous chunk's buffers are read
     for (int idx = tid; idx < slots * D; idx += 256) {
       const int h = idx / D, c = idx - h * D;
       sq[idx] = h0 + h < G ? q[(size_t(b) * Hq + hkv * G + h0 + h) * D + c] : 0.f;
@@ -1073,8 +1074,16 @@ cudaError_t launch_logits(const tq_ctx* ctx, const float* q, int B, int Hq, int 
   cudaFuncSetAttribute(qprep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(qp_smem));
   // one-bit codes (levels -c1, +c1) use the one-bit operand form: the code scale is c1
   const float code_scale = ctx->bmse == 1 ? float(ctx->c[1]) : ctx->lut.inv_scale;
-  qprep_kernel<<<unsigned(groups * ((nchunk + kQChunks - 1) / kQChunks)), 256, qp_smem, st>>>(
-      q, Hq, Hkv, nchunk, nt, ctx->dRt, ctx->dPt, code_scale, scale,
+  // blocks per group: as many as two waves of blocks allow (a small batch is
+  // latency bound: one chunk per block), down to one per group for large
+  // batches (each block then copies R and P once for up to kQChunks chunks);
+  // the chunks are split evenly over a group's blocks
+  int64_t nbg = 2 * int64_t(sm_count()) / groups;
+  if (nbg < (nchunk + kQChunks - 1) / kQChunks) nbg = (nchunk + kQChunks - 1) / kQChunks;
+  if (nbg > nchunk) nbg = nchunk;
+  const int cpb = int((nchunk + nbg - 1) / nbg);
+  qprep_kernel<<<unsigned(groups * ((nchunk + cpb - 1) / cpb)), 256, qp_smem, st>>>(
+      q, Hq, Hkv, nchunk, cpb, nt, ctx->dRt, ctx->dPt, code_scale, scale,
       float(ctx->m > 0 ? kQjlConst / ctx->m : 0.0), ctx->bmse == 1 ? 1 : 0, frags, hs);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
