@@ -7,7 +7,7 @@ import numpy as np
 
 from oracle import tq_oracle as O
 
-# The benchmark spec's bar for the fraction of mismatching coordinates.
+# The limit on the fraction of mismatching coordinates (codes or sign bits).
 MISMATCH_LIMIT = 1e-4
 
 
@@ -24,14 +24,13 @@ def check_quantize(payload, norms, K64, tb: O.Tables, report=None):
     except within SIGN_BAND of 0 (cosine of the JL row and the residual) or in
     a key with an excused code difference; fp16 norms equal except near a
     rounding midpoint (O.norm_band: 1e-5 on the unit-sphere scale; then one
-    ulp either way).  Mismatching
-    coordinates must stay below 1e-4.
+    ulp either way).  Mismatching coordinates must stay below 1e-4.
 
-    Returns (stats, quantized): stats holds the fractions the benchmark spec asks
-    to report (mismatching codes and sign bits, coordinates near a boundary)
-    plus the sign mismatches that the literal narrower band |(S r)_i| <= 1e-5
-    ||r|| would not excuse (diagnostic, not asserted).  With `report` (a
-    dict), the stats are also merged into it.
+    Returns (stats, quantized): stats holds the reported fractions
+    (mismatching codes and sign bits, coordinates near a boundary) plus the
+    sign mismatches that the literal narrower band |(S r)_i| <= 1e-5 ||r||
+    would not excuse (diagnostic, not asserted).  With `report` (a dict),
+    the stats are also merged into it.
     """
     payload = np.asarray(payload)
     norms = np.asarray(norms).view(np.float16).reshape(-1, 2)
@@ -120,7 +119,7 @@ def check_close(gpu, ref, A, tol=1e-3, rel_floor=None, report=None):
     """|gpu - ref| <= tol * A elementwise (the logits tolerance: A is the sum
     of the absolute values of the estimator's terms, since logits cross 0).
     With rel_floor, also |gpu - ref| <= tol * |ref| wherever |ref| >=
-    rel_floor * A (the plain relative error of the benchmark spec, away from 0).
+    rel_floor * A (the plain relative error, away from 0).
     Returns the worst A-relative error; with `report`, records both worsts."""
     gpu = np.asarray(gpu, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
