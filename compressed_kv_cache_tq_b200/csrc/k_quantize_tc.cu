@@ -1215,8 +1215,8 @@ __global__ void __launch_bounds__(kWThreads, 1) quantize_wide_kernel(const __gri
         uint32_t acc = 0;
         for (int a = 0; ok && a < ka; ++a) {
           const int64_t e = i * ka + a;
-          const int rs = int(e & 1);
-          if (!mbar_wait(bar(kWRFull + rs), uint32_t((e >> 1) & 1), abort_flag, status)) {
+          const int rs = int(e % kWRing);
+          if (!mbar_wait(bar(kWRFull + rs), uint32_t((e / kWRing) & 1), abort_flag, status)) {
             ok = false;
             break;
           }
@@ -1279,9 +1279,9 @@ __global__ void __launch_bounds__(kWThreads, 1) quantize_wide_kernel(const __gri
         const int64_t j = i * qt + q;              // staging use
         const int sb = int(j % kWStage);
         const int64_t e = i * ka + (q >> 1);       // key atom use
-        const int rs = int(e & 1);
-        if ((q & 1) == 0 && e >= 2 &&
-            !mbar_wait_warp(bar(kWREmpty + rs), uint32_t(((e >> 1) - 1) & 1), abort_flag, status)) {
+        const int rs = int(e % kWRing);
+        if ((q & 1) == 0 && e >= kWRing &&
+            !mbar_wait_warp(bar(kWREmpty + rs), uint32_t((e / kWRing - 1) & 1), abort_flag, status)) {
           ok = false;
           break;
         }
