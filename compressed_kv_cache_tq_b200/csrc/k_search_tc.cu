@@ -94,43 +94,127 @@ __device__ __forceinline__ void sdrain(uint32_t bar, uint32_t parity, volatile i
 // One warp per row: Kw in fp16, rows n .. n_pad - 1 all zero.  maxk_bits[0]
 // gets the largest ||Kw_code|| and maxk_bits[1] the largest |w| (of the
 // rounded values, as float bits).
+// Kw entries 8 c .. 8 c + 7 of one row (lv: the levels, n16: the row's norm,
+// w: its sign weight).  A chunk of codes lies in one quarter and one
+// 16-coordinate unit of the packed layout (a quarter holds dp / 4 codes, a
+// multiple of 16), so its codes come from at most three halfwords; so do a
+// chunk's signs when it starts at a multiple of 8 past d.  Other chunks take
+// the general unpack per entry (with d and m multiples of 8, only the zero
+// padding past d + m).
+__device__ __forceinline__ void decode_chunk(const uint16_t* __restrict__ hw, const RowGeom& g, int c,
+                                             const float* lv, float n16, float w, float (&v)[8]) {
+  const int j0 = 8 * c;
+  if (j0 + 8 <= g.d) {
+    const int qd = g.dp >> 2;
+    const int q = (j0 >= qd) + (j0 >= 2 * qd) + (j0 >= 3 * qd);
+    const int r0 = (j0 - q * qd) >> 2;   // register of entries 0..3; entries 4..7 are in r0 + 1
+    const int i0 = r0 & 3;               // 0 or 2
+    const uint16_t* base = hw + q * g.per_q + (r0 >> 2) * g.bmse;
+    if (g.bmse == 3) {
+      const uint32_t h0 = __ldg(base), h1 = __ldg(base + 1), h2 = __ldg(base + 2);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (i0 == 0) {
+          v[e] = n16 * lv[(h0 >> (4 * e)) & 7u];
+          v[4 + e] = n16 * lv[(h1 >> (4 * e)) & 7u];
+        } else {
+          v[e] = n16 * lv[(h2 >> (4 * e)) & 7u];
+          v[4 + e] = n16 * lv[((h0 >> (4 * e + 3)) & 1u) | (((h1 >> (4 * e + 3)) & 1u) << 1) |
+                              (((h2 >> (4 * e + 3)) & 1u) << 2)];
+        }
+      }
+    } else if (g.bmse == 2) {
+      const uint32_t h = __ldg(base + (i0 >> 1));
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        v[e] = n16 * lv[(h >> (4 * e)) & 3u];
+        v[4 + e] = n16 * lv[(h >> (4 * e + 2)) & 3u];
+      }
+    } else {
+      const uint32_t h = __ldg(base);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        v[e] = n16 * lv[(h >> (4 * e + i0)) & 1u];
+        v[4 + e] = n16 * lv[(h >> (4 * e + i0 + 1)) & 1u];
+      }
+    }
+    return;
+  }
+  const int s0 = j0 - g.d;
+  if (s0 >= 0 && j0 + 8 <= g.d + g.m && (s0 & 7) == 0) {
+    const int qm = g.mp >> 2;
+    const int q = (s0 >= qm) + (s0 >= 2 * qm) + (s0 >= 3 * qm);
+    const int r0 = (s0 - q * qm) >> 2, i0 = r0 & 3;
+    const uint32_t h = __ldg(hw + q * g.per_q + g.bmse * g.uq + (r0 >> 2));
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      v[e] = (h >> (4 * e + i0)) & 1u ? w : -w;
+      v[4 + e] = (h >> (4 * e + i0 + 1)) & 1u ? w : -w;
+    }
+    return;
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const int j = j0 + e;
+    v[e] = j < g.d ? n16 * lv[unpack_code(hw, g, j)] : j < g.d + g.m ? (unpack_sign(hw, g, j - g.d) ? w : -w) : 0.f;
+  }
+}
+
+// One warp per row, the rows taken in a grid-stride loop: Kw in fp16, and the
+// largest code-part norm and sign weight over the rows (reduced in the block,
+// one atomic per block and quantity).
 __global__ void __launch_bounds__(256) decode_rows_kernel(const uint8_t* __restrict__ payload,
                                                           const uint16_t* __restrict__ norms, int64_t n,
                                                           int64_t n_pad, int d, int m, int bmse, int kp,
                                                           CodebookParams cb, __half* __restrict__ kw,
                                                           uint32_t* __restrict__ maxk_bits) {
-  const int lane = threadIdx.x & 31;
-  const int64_t r = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  if (r >= n_pad) return;
+  __shared__ float lv[kMaxLevels];
+  __shared__ float red[2][8];
+  if (threadIdx.x < kMaxLevels) lv[threadIdx.x] = cb.c[threadIdx.x];
+  __syncthreads();
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const RowGeom g = make_geom(d, m, bmse);
-  const bool real = r < n;
-  const uint16_t* hw = reinterpret_cast<const uint16_t*>(payload + (real ? r : 0) * g.row_bytes);
-  const float n16 = real ? half_bits_to_float(norms[2 * r]) : 0.f;
-  const float w = real && m > 0 ? float(kQjlConst) / float(m) * half_bits_to_float(norms[2 * r + 1]) : 0.f;
-  float ss = 0.f;
-  for (int c = lane; c < kp / 8; c += 32) {
-    __align__(16) __half h[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int j = 8 * c + e;
-      float v = 0.f;
-      if (real) {
-        if (j < d)
-          v = n16 * cb.c[unpack_code(hw, g, j)];
-        else if (j < d + m)
-          v = unpack_sign(hw, g, j - d) ? w : -w;
-      }
-      h[e] = __float2half_rn(v);
-      const float hv = __half2float(h[e]);
-      if (j < d) ss = fmaf(hv, hv, ss);
+  const int64_t nwarps = int64_t(gridDim.x) * (blockDim.x >> 5);
+  float mk = 0.f, mw = 0.f;
+  for (int64_t r = int64_t(blockIdx.x) * (blockDim.x >> 5) + wib; r < n_pad; r += nwarps) {
+    __half* out = kw + r * kp;
+    if (r >= n) {   // padding rows
+      for (int c = lane; c < kp / 8; c += 32) *reinterpret_cast<uint4*>(out + 8 * c) = make_uint4(0u, 0u, 0u, 0u);
+      continue;
     }
-    *reinterpret_cast<uint4*>(kw + r * kp + 8 * c) = *reinterpret_cast<const uint4*>(h);
-  }
+    const uint16_t* hw = reinterpret_cast<const uint16_t*>(payload + r * g.row_bytes);
+    const float n16 = half_bits_to_float(__ldg(norms + 2 * r));
+    const float w = m > 0 ? float(kQjlConst) / float(m) * half_bits_to_float(__ldg(norms + 2 * r + 1)) : 0.f;
+    float ss = 0.f;
+    for (int c = lane; c < kp / 8; c += 32) {
+      float v[8];
+      decode_chunk(hw, g, c, lv, n16, w, v);
+      __align__(16) __half h[8];
 #pragma unroll
-  for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
-  if (lane == 0 && real) {
-    atomicMax(maxk_bits, __float_as_uint(sqrtf(ss)));
-    atomicMax(maxk_bits + 1, __float_as_uint(fabsf(__half2float(__float2half_rn(w)))));
+      for (int e = 0; e < 8; ++e) {
+        h[e] = __float2half_rn(v[e]);
+        const float hv = __half2float(h[e]);
+        if (8 * c + e < d) ss = fmaf(hv, hv, ss);
+      }
+      *reinterpret_cast<uint4*>(out + 8 * c) = *reinterpret_cast<const uint4*>(h);
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+    mk = fmaxf(mk, sqrtf(ss));
+    mw = fmaxf(mw, fabsf(__half2float(__float2half_rn(w))));
+  }
+  if (lane == 0) {
+    red[0][wib] = mk;
+    red[1][wib] = mw;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int i = 1; i < int(blockDim.x >> 5); ++i) {
+      mk = fmaxf(mk, red[0][i]);
+      mw = fmaxf(mw, red[1][i]);
+    }
+    if (mk > 0.f) atomicMax(maxk_bits, __float_as_uint(mk));   // non-negative floats order as their bits
+    if (mw > 0.f) atomicMax(maxk_bits + 1, __float_as_uint(mw));
   }
 }
 
@@ -192,33 +276,52 @@ __device__ __forceinline__ float key_float(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
-// Work: unit u = (query tile u / row_tiles, row tile u % row_tiles); CTA b
-// takes the contiguous units [U b / G, U (b + 1) / G) of the U = qtiles x
-// row_tiles, so it keeps one query tile (or two) for long stretches.  (A
-// part-major round-robin order that makes all CTAs stream the same rows at
-// the same time measured slower: 17.0 against 13.7 ms at 10^6 x 10^4.)
+// Work: unit (query tile, row tile).  The grid is cut into groups of G
+// consecutive CTAs and the query tiles into groups of G consecutive tiles.
+// Group g of the NG = ctas / G takes the contiguous units [U g / NG,
+// U (g + 1) / NG) of the U = ceil(qtiles / G) x row_tiles pairs (query-tile
+// group qg, row tile t), qg-major, and its member r works on query tile
+// G qg + r of each: a CTA keeps one query tile (or two) for long stretches,
+// and the G members of a group read the same row tiles in the same order, so
+// that all but the first find each tile in L2 (the row matrix crosses HBM
+// about ceil(qtiles / G) times instead of qtiles times).  A member whose
+// query tile is past the last one skips those units.  (A part-major
+// round-robin order that makes all CTAs stream the same rows at the same
+// time, restarting each query's running k-th best at every part, measured
+// slower: 17.0 against 13.7 ms at 10^6 x 10^4.)
 struct Units {
-  int64_t row_tiles, u, u1;
+  int64_t qtiles, row_tiles, u, u1;
   int64_t qt, t;
-  __device__ Units(int64_t qtiles, int64_t row_tiles_, int64_t cta, int64_t ctas) : row_tiles(row_tiles_) {
-    const int64_t total = qtiles * row_tiles_;
-    u = total * cta / ctas - 1;
-    u1 = total * (cta + 1) / ctas;
+  int64_t G, r;
+  __device__ Units(int64_t qtiles_, int64_t row_tiles_, int64_t cta, int64_t ctas, int64_t G_)
+      : qtiles(qtiles_), row_tiles(row_tiles_), G(G_) {
+    const int64_t ng = ctas / G, g = cta / G;
+    r = cta - g * G;
+    const int64_t total = ((qtiles + G - 1) / G) * row_tiles;
+    u = total * g / ng - 1;
+    u1 = total * (g + 1) / ng;
     qt = t = 0;
   }
   // advance to the next (query tile, row tile); false when done
   __device__ bool next() {
-    if (++u >= u1) return false;
-    qt = u / row_tiles;
-    t = u - qt * row_tiles;
-    return true;
+    while (++u < u1) {
+      const int64_t qg = u / row_tiles;
+      qt = qg * G + r;
+      if (qt >= qtiles) {   // no such tile: skip the rest of this query-tile group
+        u = (qg + 1) * row_tiles - 1;
+        continue;
+      }
+      t = u - qg * row_tiles;
+      return true;
+    }
+    return false;
   }
 };
 
 template <int KB>
 __global__ void __launch_bounds__(kSearchThreads, 1) search_tc_kernel(
     const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap, int64_t nq, int64_t n,
-    int64_t qtiles, int64_t row_tiles, int k, const float* __restrict__ qerr,
+    int64_t qtiles, int64_t row_tiles, int64_t group, int k, const float* __restrict__ qerr,
     uint32_t* __restrict__ gkth, uint32_t* __restrict__ cnt,
     uint2* __restrict__ cand, uint32_t* __restrict__ status) {
   using L = SearchSmem<KB>;
@@ -264,7 +367,7 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_tc_kernel(
       int64_t qt_prev = -1, it = 0;
       int na = 0;
       bool ok = true;
-      Units w(qtiles, row_tiles, blockIdx.x, gridDim.x);
+      Units w(qtiles, row_tiles, blockIdx.x, gridDim.x, group);
       while (ok && w.next()) {
         const int64_t qt = w.qt, t = w.t;
         if (qt != qt_prev) {
@@ -297,7 +400,7 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_tc_kernel(
       int64_t qt_prev = -1, it = 0, j = 0;
       int na = 0;
       bool ok = true;
-      Units w(qtiles, row_tiles, blockIdx.x, gridDim.x);
+      Units w(qtiles, row_tiles, blockIdx.x, gridDim.x, group);
       for (; ok && w.next(); ++j) {
         const int64_t qt = w.qt;
         if (qt != qt_prev) {
@@ -348,7 +451,7 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_tc_kernel(
     // score) and appended with one atomic per tile
     uint2 stage[kRT];
     int64_t j = 0;
-    Units w(qtiles, row_tiles, blockIdx.x, gridDim.x);
+    Units w(qtiles, row_tiles, blockIdx.x, gridDim.x, group);
     for (; w.next(); ++j) {
       const int64_t qt = w.qt, t = w.t;
       if (qt != qt_prev) {
@@ -700,6 +803,18 @@ SearchWs search_ws(const tq_ctx* ctx, int64_t nq, int64_t n, void* base) {
   return w;
 }
 
+// CTAs per group of the schedule above: groups of eight when there are enough
+// query tiles that an idle member (query tile past the end) costs little; the
+// grid is then the largest multiple of the group size that fits the SMs (144
+// of 148).  Measured at 10^6 rows x 10^4 queries (79 query tiles): 12.1 /
+// 13.5 ms (b = 2 / 4) for single CTAs, 11.9 / 13.4 for groups of four, 11.5 /
+// 12.6 for groups of eight.
+int64_t search_group(int64_t qtiles, int sms) {
+  int64_t g = qtiles >= 32 ? 8 : qtiles >= 16 ? 4 : qtiles >= 8 ? 2 : 1;
+  while (g > 1 && sms < g) g >>= 1;
+  return g;
+}
+
 template <int KB>
 cudaError_t launch_search_kernel(const CUtensorMap& qmap, const CUtensorMap& kmap, int64_t nq, int64_t n,
                                  int64_t qtiles, int64_t row_tiles, int k, const SearchWs& w, uint32_t* status,
@@ -711,10 +826,12 @@ cudaError_t launch_search_kernel(const CUtensorMap& qmap, const CUtensorMap& kma
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t units = qtiles * row_tiles;
-  const int grid = int(units < sms ? units : sms);
-  kern<<<grid, kSearchThreads, L::kBytes, st>>>(qmap, kmap, nq, n, qtiles, row_tiles, k, w.qerr, w.gkth, w.cnt,
-                                                w.cand, status);
+  const int64_t group = search_group(qtiles, sms);
+  const int64_t units = ((qtiles + group - 1) / group) * row_tiles;   // per member of a group
+  const int64_t groups = units < sms / group ? units : sms / group;
+  const int grid = int(groups * group);
+  kern<<<grid, kSearchThreads, L::kBytes, st>>>(qmap, kmap, nq, n, qtiles, row_tiles, group, k, w.qerr, w.gkth,
+                                                w.cnt, w.cand, status);
   return cudaGetLastError();
 }
 
@@ -749,8 +866,12 @@ cudaError_t launch_search_tc(const tq_ctx* ctx, const float* q, int64_t nq, cons
   if ((e = cudaMemsetAsync(w.maxk, 0, 8, st)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(w.cnt, 0, size_t(nq_pad) * 4, st)) != cudaSuccess) return e;
   if ((e = cudaMemsetAsync(w.gkth, 0, size_t(nq_pad) * 4, st)) != cudaSuccess) return e;
-  const int64_t warps = n_pad;
-  decode_rows_kernel<<<unsigned((warps * 32 + 255) / 256), 256, 0, st>>>(
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t row_blocks = (n_pad + 7) / 8;   // eight warps (rows) per block and pass
+  const int64_t dec_blocks = row_blocks < int64_t(sms) * 8 ? row_blocks : int64_t(sms) * 8;
+  decode_rows_kernel<<<unsigned(dec_blocks), 256, 0, st>>>(
       payload, norms, n, n_pad, ctx->d, ctx->m, ctx->bmse, kp, ctx->cb, w.kw, w.maxk);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   prep_queries_kernel<<<unsigned(nq), 256, 0, st>>>(q, ctx->dRt, ctx->dPt, ctx->d, ctx->m, kp, w.maxk, w.qw,

@@ -319,7 +319,8 @@ def test_dequantize_full_matches_logits(lib):
 
 
 @pytest.mark.parametrize("d,bits,n,nq,k", [(128, 3, 5000, 16, 10), (128, 4, 3001, 9, 1), (128, 2, 700, 5, 64),
-                                           (128, 3, 100, 3, 10), (200, 2, 3000, 7, 10), (200, 4, 2000, 5, 10)])
+                                           (128, 3, 100, 3, 10), (200, 2, 3000, 7, 10), (200, 4, 2000, 5, 10),
+                                           (104, 3, 3000, 6, 10), (72, 2, 1500, 4, 5)])
 def test_topk_against_oracle(lib, d, bits, n, nq, k):
     ctx = _ctx(lib, d=d, bits=bits, seed=17)
     db = W.search_vectors(n, d, seed=100 + bits, which=0)
@@ -343,12 +344,14 @@ def test_topk_against_oracle(lib, d, bits, n, nq, k):
                                atol=1e-6 * A.max())
 
 
-@pytest.mark.parametrize("d,bits", [(200, 2), (128, 4)])
-def test_topk_many_query_tiles(lib, d, bits):
+@pytest.mark.parametrize("d,bits,n,nq", [(200, 2, 20000, 500), (128, 4, 20000, 500), (200, 4, 12000, 2100)])
+def test_topk_many_query_tiles(lib, d, bits, n, nq):
     """More (query tile, row tile) units than SMs: CTAs switch query tiles
-    inside their range of the tensor-core search."""
+    inside their range of the tensor-core search.  With 2100 queries (17 tiles)
+    the CTAs work in groups of four over the same row tiles, and three members
+    of the last group have no query tile."""
     ctx = _ctx(lib, d=d, bits=bits, seed=19)
-    n, nq, k = 20000, 500, 10
+    k = 10
     db = W.search_vectors(n, d, seed=300 + bits, which=0)
     qs = W.search_vectors(nq, d, seed=300 + bits, which=1)
     payload, norms = lib.tq_quantize(ctx, torch.from_numpy(db).to(DEV))
