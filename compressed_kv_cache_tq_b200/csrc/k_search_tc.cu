@@ -5,16 +5,20 @@
 // is one inner product s = <Kw, Qw> of a per-row weight vector
 //   Kw = [n16 c[idx_0 .. d-1], sqrt(pi/2)/m rho16 sigma_0 .. m-1, 0 ...]
 // and a per-query vector Qw = [Rq, Sq, 0 ...], both KP = round-up(d + m, 64)
-// long.  Four kernels:
+// long.  Five kernels:
 //   1. decode_rows_kernel: packed rows -> Kw in fp16 (one warp per row), and
 //      the largest code-part norm ||Kw_code|| and sign weight |w| over rows.
-//   2. prep_queries_kernel: Qw in fp16 and the per-query error bound E_q.
-//   3. search_tc_kernel: tcgen05 MMA of 128-query tiles (resident in shared
-//      memory) against 256-row tiles (TMA ring), scores in TMEM; the epilogue
+//   2. query_tables_kernel: x = R q and y = P R q = S q in fp64 (kept for the
+//      exact re-scoring).
+//   3. prep_queries_kernel: Qw = [x, y] rounded to fp16 and the per-query
+//      error bound E_q.
+//   4. search_tc_kernel: tcgen05 MMA of 128-query tiles (resident in tensor
+//      memory, the A operand) against 128-row tiles (a twelve-stage TMA ring
+//      of 16 KB K-blocks: shared memory holds only row tiles, so that about
+//      190 KB of them are in flight per SM), scores in TMEM; the epilogue
 //      keeps each query's running k best scores and appends every row whose
 //      score is at least (k-th best - 2 E_q) to the query's candidate list.
-//   4. query_tables_kernel (x = Rq, y = Sq in fp64) and finish_kernel: per
-//      query, the k-th largest approximate score among the candidates (by
+//   5. finish_kernel: per query, the k-th largest approximate score among the candidates (by
 //      bisection), the candidates within 2 E_q of it re-scored exactly in fp64
 //      and ordered by (score descending, id ascending); the first k are the
 //      answer.
@@ -27,9 +31,9 @@
 // largest local A_k published so far (each is at most the global one, so the
 // argument holds for their maximum).  A query whose candidate list
 // overflows is answered by an exact scan of all rows in the finishing kernel.
-// Error bound: Kw and Qw are rounded to fp16 (relative 2^-11 each) after fp32
-// arithmetic (R q and P R q in fp32: relative error below 2e-4 of ||Kw|| ||q||
-// at d <= 256), and the tensor cores accumulate KP <= 512 exact products in
+// Error bound: Kw (from fp32 arithmetic) and Qw (from the fp64 tables) are
+// rounded to fp16 (relative 2^-11 each; the bound below also leaves 2e-4 of
+// ||Kw|| ||q|| for fp32 arithmetic before the rounding), and the tensor cores accumulate KP <= 512 exact products in
 // fp32 (below KP 2^-23 of sum |Kw_j Qw_j|).  With
 //   sum_j |Kw_j Qw_j| <= max ||Kw_code|| ||Rq||_2 + max |w| ||Sq||_1
 // (Cauchy-Schwarz on the code part; the sign part has |sigma_i| = 1),
@@ -50,27 +54,27 @@ namespace {
 using namespace tc;
 
 constexpr int kQT = 128;                 // queries per tile (MMA M)
-constexpr int kRT = 256;                 // database rows per tile (MMA N)
-constexpr int kBStages = 3;              // row-tile K-block ring
+constexpr int kRT = 128;                 // database rows per tile (MMA N)
+constexpr int kBStages = 12;             // row-tile K-block ring (16 KB stages)
 constexpr int kSearchThreads = 192;      // TMA warp, MMA warp, 4 epilogue warps
 constexpr int kMaxK = 32;                // k handled by the epilogue's running top-k
 constexpr int kCap = 2048;               // candidates kept per query
 constexpr float kErrRel = 1.5e-3f;       // relative error bound (see above)
 constexpr float kErrAbs = 0x1p-20f;      // absolute term (fp16 subnormals)
-constexpr uint32_t kIdescSearch = idesc_f16(0, kQT, kRT);   // fp16 x fp16 -> fp32, 128 x 256
+constexpr uint32_t kIdescSearch = idesc_f16(0, kQT, kRT);   // fp16 x fp16 -> fp32, 128 x 128
+// TMEM: the query tile (A operand, K-major, two fp16 per column) in columns
+// 0 .. KP / 2 - 1 (at most 256), two score accumulators of 128 columns above.
+constexpr uint32_t kTmemD = 256;
 
-template <int KB>
 struct SearchSmem {
-  static constexpr uint32_t kOffA = 0;                           // KB blocks of 128 rows x 128 B
-  static constexpr uint32_t kOffB = KB * 16384u;                 // kBStages blocks of 256 rows x 128 B
-  static constexpr uint32_t kOffBar = kOffB + kBStages * 32768u;
+  static constexpr uint32_t kOffB = 0;                           // kBStages blocks of 128 rows x 128 B
+  static constexpr uint32_t kOffBar = kOffB + kBStages * 16384u;
   static constexpr uint32_t kBytes = kOffBar + 256 + 1024;       // + slack for 1024-byte alignment
 };
 
 enum SBar {
-  kSAFull = 0,
-  kSAFree = 1,
-  kSBFull = 2,
+  kSAFull = 0,                 // query tile written to TMEM (128 epilogue arrivals)
+  kSBFull = 1,
   kSBEmpty = kSBFull + kBStages,
   kSDFull = kSBEmpty + kBStages,
   kSDEmpty = kSDFull + 2,
@@ -218,52 +222,34 @@ __global__ void __launch_bounds__(256) decode_rows_kernel(const uint8_t* __restr
   }
 }
 
-// One block per query: Qw = [R q, P R q] in fp16 (the rest of the row was
-// zeroed by the caller) and the error bound E_q (see the top of this file).
-__global__ void __launch_bounds__(256) prep_queries_kernel(const float* __restrict__ q, const float* __restrict__ Rt,
-                                                           const float* __restrict__ Pt, int d, int m, int kp,
-                                                           const uint32_t* __restrict__ maxk_bits,
+// One warp per query: Qw = [R q, P R q] rounded to fp16 from the query's
+// fp64 tables xy = [x, y] (the rest of the row was zeroed by the caller), and
+// the error bound E_q (see the top of this file) from the rounded values.
+__global__ void __launch_bounds__(256) prep_queries_kernel(const double* __restrict__ xy, int64_t nq, int d, int m,
+                                                           int kp, const uint32_t* __restrict__ maxk_bits,
                                                            __half* __restrict__ qw, float* __restrict__ qerr) {
-  __shared__ float sq[256], sx[256];
-  __shared__ float red[8], red1[8];
-  const int qi = blockIdx.x, tid = threadIdx.x;
-  for (int i = tid; i < d; i += blockDim.x) sq[i] = q[size_t(qi) * d + i];
-  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int64_t qi = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (qi >= nq) return;
+  const double* src = xy + qi * (d + m);
   float ss = 0.f, s1 = 0.f;   // ||Rq||_2^2 and ||Sq||_1 of the rounded values
-  for (int j = tid; j < d; j += blockDim.x) {
-    float x = 0.f;
-    for (int i = 0; i < d; ++i) x = fmaf(Rt[i * d + j], sq[i], x);
-    sx[j] = x;
-    const __half h = __float2half_rn(x);
-    qw[size_t(qi) * kp + j] = h;
-    ss = fmaf(__half2float(h), __half2float(h), ss);
-  }
-  __syncthreads();
-  for (int i = tid; i < m; i += blockDim.x) {
-    float y = 0.f;
-    for (int j = 0; j < d; ++j) y = fmaf(Pt[j * m + i], sx[j], y);
-    const __half h = __float2half_rn(y);
-    qw[size_t(qi) * kp + d + i] = h;
-    s1 += fabsf(__half2float(h));
+  for (int i = lane; i < d + m; i += 32) {
+    const __half h = __double2half(src[i]);
+    qw[qi * kp + i] = h;
+    const float hv = __half2float(h);
+    if (i < d)
+      ss = fmaf(hv, hv, ss);
+    else
+      s1 += fabsf(hv);
   }
 #pragma unroll
   for (int o = 16; o; o >>= 1) {
     ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
     s1 += __shfl_xor_sync(0xFFFFFFFFu, s1, o);
   }
-  if ((tid & 31) == 0) {
-    red[tid >> 5] = ss;
-    red1[tid >> 5] = s1;
-  }
-  __syncthreads();
-  if (tid == 0) {
-    float t = 0.f, t1 = 0.f;
-    for (int w = 0; w < int(blockDim.x / 32); ++w) {
-      t += red[w];
-      t1 += red1[w];
-    }
-    const float rq = sqrtf(t), kc = __uint_as_float(maxk_bits[0]), kw1 = __uint_as_float(maxk_bits[1]);
-    qerr[qi] = kErrRel * (kc * rq + kw1 * t1) + kErrAbs * (kc + float(m) * kw1 + rq + t1);
+  if (lane == 0) {
+    const float rq = sqrtf(ss), kc = __uint_as_float(maxk_bits[0]), kw1 = __uint_as_float(maxk_bits[1]);
+    qerr[qi] = kErrRel * (kc * rq + kw1 * s1) + kErrAbs * (kc + float(m) * kw1 + rq + s1);
   }
 }
 
@@ -320,11 +306,12 @@ struct Units {
 
 template <int KB>
 __global__ void __launch_bounds__(kSearchThreads, 1) search_tc_kernel(
-    const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap, int64_t nq, int64_t n,
+    const __grid_constant__ CUtensorMap kmap, const __half* __restrict__ qw, int64_t nq, int64_t n,
     int64_t qtiles, int64_t row_tiles, int64_t group, int k, const float* __restrict__ qerr,
     uint32_t* __restrict__ gkth, uint32_t* __restrict__ cnt,
     uint2* __restrict__ cand, uint32_t* __restrict__ status) {
-  using L = SearchSmem<KB>;
+  using L = SearchSmem;
+  constexpr int kp = 64 * KB;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -336,8 +323,7 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_tc_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(kSAFull), 1);
-    mbar_init(bar(kSAFree), 1);
+    mbar_init(bar(kSAFull), 128);
     for (int s = 0; s < kBStages; ++s) {
       mbar_init(bar(kSBFull + s), 1);
       mbar_init(bar(kSBEmpty + s), 1);
@@ -363,36 +349,26 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_tc_kernel(
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
+    // (row tiles only: the epilogue writes each query tile into TMEM)
     if (lane == 0) {
-      int64_t qt_prev = -1, it = 0;
-      int na = 0;
+      int64_t it = 0;
       bool ok = true;
       Units w(qtiles, row_tiles, blockIdx.x, gridDim.x, group);
       while (ok && w.next()) {
-        const int64_t qt = w.qt, t = w.t;
-        if (qt != qt_prev) {
-          // the MMAs that read the previous query tile have completed
-          if (na > 0 && !swait(bar(kSAFree), uint32_t((na - 1) & 1), abort_flag, status)) break;
-          mbar_expect_tx(bar(kSAFull), KB * 16384u);
-          for (int kb = 0; kb < KB; ++kb)
-            tma_load_2d(base + L::kOffA + 16384u * kb, &qmap, 64 * kb, int(qt * kQT), bar(kSAFull));
-          ++na;
-          qt_prev = qt;
-        }
+        const int64_t t = w.t;
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = int(it % kBStages);
           if (it >= kBStages && !swait(bar(kSBEmpty + s), uint32_t((it / kBStages - 1) & 1), abort_flag, status)) {
             ok = false;
             break;
           }
-          mbar_expect_tx(bar(kSBFull + s), 32768u);
-          tma_load_2d(base + L::kOffB + 32768u * s, &kmap, 64 * kb, int(t * kRT), bar(kSBFull + s));
+          mbar_expect_tx(bar(kSBFull + s), 16384u);
+          tma_load_2d(base + L::kOffB + 16384u * s, &kmap, 64 * kb, int(t * kRT), bar(kSBFull + s));
         }
       }
       // leave no copy in flight
       for (int64_t j = (it >= kBStages ? it - kBStages : 0); j < it; ++j)
         sdrain(bar(kSBFull + int(j % kBStages)), uint32_t((j / kBStages) & 1), abort_flag, status);
-      if (na > 0) sdrain(bar(kSAFull), uint32_t((na - 1) & 1), abort_flag, status);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
@@ -404,7 +380,9 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_tc_kernel(
       for (; ok && w.next(); ++j) {
         const int64_t qt = w.qt;
         if (qt != qt_prev) {
-          if (na > 0) mma_commit(bar(kSAFree));   // tracks every MMA on the previous query tile
+          // the epilogue has written this query tile into TMEM (it does so
+          // only after the scores of every unit of the previous tile, so no
+          // MMA still reads the old one)
           if (!swait(bar(kSAFull), uint32_t(na & 1), abort_flag, status)) break;
           ++na;
           qt_prev = qt;
@@ -412,7 +390,7 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_tc_kernel(
         const int slot = int(j & 1);
         if (j >= 2 && !swait(bar(kSDEmpty + slot), uint32_t(((j >> 1) - 1) & 1), abort_flag, status)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem + 256u * slot;
+        const uint32_t d_tmem = tmem + kTmemD + 128u * slot;
         uint32_t acc = 0;
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const int s = int(it % kBStages);
@@ -422,8 +400,9 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_tc_kernel(
           }
           tc_fence_after();
           for (int ks = 0; ks < 4; ++ks) {
-            mma_f16(d_tmem, smem_desc(base + L::kOffA + 16384u * kb + 32u * ks),
-                    smem_desc(base + L::kOffB + 32768u * s + 32u * ks), kIdescSearch, acc);
+            // query coordinates 64 kb + 16 ks .. +15: TMEM columns 32 kb + 8 ks .. +7
+            mma_f16_ts(d_tmem, tmem + 32u * kb + 8u * ks, smem_desc(base + L::kOffB + 16384u * s + 32u * ks),
+                       kIdescSearch, acc);
             acc = 1;
           }
           mma_commit(bar(kSBEmpty + s));
@@ -458,6 +437,19 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_tc_kernel(
         qt_prev = qt;
         q = qt * kQT + row;
         E2 = q < nq ? 2.f * qerr[q] : 0.f;
+        // this thread's query row (zero past nq) into TMEM lane `row`, columns
+        // 0 .. kp / 2 - 1.  Every MMA on the previous query tile has completed:
+        // the scores of its last unit were waited for above.
+        const uint4* src = reinterpret_cast<const uint4*>(qw + size_t(q) * kp);
+#pragma unroll 4
+        for (int c = 0; c < kp / 16; ++c) {
+          const uint4 lo = __ldg(src + 2 * c), hi = __ldg(src + 2 * c + 1);
+          const uint32_t r[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+          tmem_st8(tmem + lane_base + 8u * c, r);
+        }
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        tc_fence_before();
+        mbar_arrive(bar(kSAFull));
 #pragma unroll 1
         for (int i = 0; i < k; ++i) topv[i] = -INFINITY;
         kth = -INFINITY;
@@ -476,7 +468,7 @@ __global__ void __launch_bounds__(kSearchThreads, 1) search_tc_kernel(
 #pragma unroll 1
       for (int c = 0; c < kRT / 32; ++c) {
         float v[32];
-        tmem_ld32(tmem + lane_base + 256u * slot + 32u * c, v);
+        tmem_ld32(tmem + lane_base + kTmemD + 128u * slot + 32u * c, v);
         tmem_wait32(v);
         if (q >= nq) continue;
         const float thr = fmaxf(kth, gk) - E2;
@@ -540,6 +532,26 @@ __device__ double exact_score(const uint8_t* __restrict__ payload, const uint16_
   double a = 0.0, b = 0.0;
   for (int j = 0; j < g.d; ++j) a += c[unpack_code(hw, g, j)] * x[j];
   for (int i = 0; i < g.m; ++i) b += unpack_sign(hw, g, i) ? y[i] : -y[i];
+  const double n16 = double(half_bits_to_float(norms[2 * row]));
+  const double r16 = double(half_bits_to_float(norms[2 * row + 1]));
+  return n16 * a + qc * r16 * b;
+}
+
+// The same estimate, its terms split over the 32 lanes of a warp (lane `ln`
+// takes coordinates ln, ln + 32, ...) and summed by a butterfly: every lane
+// returns the same value, and equal rows get equal scores.
+__device__ double exact_score_warp(const uint8_t* __restrict__ payload, const uint16_t* __restrict__ norms,
+                                   int64_t row, const RowGeom& g, const double* __restrict__ c, const double* x,
+                                   const double* y, double qc, int ln) {
+  const uint16_t* hw = reinterpret_cast<const uint16_t*>(payload + row * g.row_bytes);
+  double a = 0.0, b = 0.0;
+  for (int j = ln; j < g.d; j += 32) a += c[unpack_code(hw, g, j)] * x[j];
+  for (int i = ln; i < g.m; i += 32) b += unpack_sign(hw, g, i) ? y[i] : -y[i];
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    a += __shfl_xor_sync(0xFFFFFFFFu, a, o);
+    b += __shfl_xor_sync(0xFFFFFFFFu, b, o);
+  }
   const double n16 = double(half_bits_to_float(norms[2 * row]));
   const double r16 = double(half_bits_to_float(norms[2 * row + 1]));
   return n16 * a + qc * r16 * b;
@@ -728,8 +740,11 @@ __global__ void __launch_bounds__(kFinishThreads) finish_kernel(
   }
   __syncthreads();
   const int mc = s_mc;
-  // 3. exact scores, then (score descending, id ascending)
-  for (int i = tid; i < mc; i += nth) ssc[i] = exact_score(payload, norms, sid[i], g, c, sx, sy, qc);
+  // 3. exact scores (one warp per candidate), then (score descending, id ascending)
+  for (int i = tid >> 5; i < mc; i += nth >> 5) {
+    const double sc = exact_score_warp(payload, norms, sid[i], g, c, sx, sy, qc, tid & 31);
+    if ((tid & 31) == 0) ssc[i] = sc;
+  }
   int sp2 = 1;
   while (sp2 < mc) sp2 <<= 1;
   for (int i = mc + tid; i < sp2; i += nth) {
@@ -816,11 +831,13 @@ int64_t search_group(int64_t qtiles, int sms) {
 }
 
 template <int KB>
-cudaError_t launch_search_kernel(const CUtensorMap& qmap, const CUtensorMap& kmap, int64_t nq, int64_t n,
+cudaError_t launch_search_kernel(const CUtensorMap& kmap, const __half* qw, int64_t nq, int64_t n,
                                  int64_t qtiles, int64_t row_tiles, int k, const SearchWs& w, uint32_t* status,
                                  cudaStream_t st) {
-  using L = SearchSmem<KB>;
+  using L = SearchSmem;
   static_assert(L::kBytes <= 232448, "shared memory per block");
+  static_assert(8 * kSNumBars + 8 <= 256, "barrier area");
+  static_assert(32 * KB <= int(kTmemD), "query tile columns");
   auto kern = search_tc_kernel<KB>;
   cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(L::kBytes));
   int dev = 0, sms = 148;
@@ -830,7 +847,7 @@ cudaError_t launch_search_kernel(const CUtensorMap& qmap, const CUtensorMap& kma
   const int64_t units = ((qtiles + group - 1) / group) * row_tiles;   // per member of a group
   const int64_t groups = units < sms / group ? units : sms / group;
   const int grid = int(groups * group);
-  kern<<<grid, kSearchThreads, L::kBytes, st>>>(qmap, kmap, nq, n, qtiles, row_tiles, group, k, w.qerr, w.gkth,
+  kern<<<grid, kSearchThreads, L::kBytes, st>>>(kmap, qw, nq, n, qtiles, row_tiles, group, k, w.qerr, w.gkth,
                                                 w.cnt, w.cand, status);
   return cudaGetLastError();
 }
@@ -869,32 +886,33 @@ cudaError_t launch_search_tc(const tq_ctx* ctx, const float* q, int64_t nq, cons
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int dec_per_sm = 0;   // resident blocks per SM (one wave of the grid-stride loop)
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&dec_per_sm, decode_rows_kernel, 256, 0);
+  if (dec_per_sm < 1) dec_per_sm = 1;
   const int64_t row_blocks = (n_pad + 7) / 8;   // eight warps (rows) per block and pass
-  const int64_t dec_blocks = row_blocks < int64_t(sms) * 8 ? row_blocks : int64_t(sms) * 8;
+  const int64_t dec_blocks = row_blocks < int64_t(sms) * dec_per_sm ? row_blocks : int64_t(sms) * dec_per_sm;
   decode_rows_kernel<<<unsigned(dec_blocks), 256, 0, st>>>(
       payload, norms, n, n_pad, ctx->d, ctx->m, ctx->bmse, kp, ctx->cb, w.kw, w.maxk);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  prep_queries_kernel<<<unsigned(nq), 256, 0, st>>>(q, ctx->dRt, ctx->dPt, ctx->d, ctx->m, kp, w.maxk, w.qw,
-                                                     w.qerr);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  CUtensorMap qmap, kmap;
-  if (!encode_fp16_map(&qmap, w.qw, kp, nq_pad, kQT) || !encode_fp16_map(&kmap, w.kw, kp, n_pad, kRT))
-    return cudaErrorInvalidValue;
-  const int64_t row_tiles = n_pad / kRT, qtiles = nq_pad / kQT;
-  switch (kb) {
-    case 1: e = launch_search_kernel<1>(qmap, kmap, nq, n, qtiles, row_tiles, k, w, ctx->dstatus, st); break;
-    case 2: e = launch_search_kernel<2>(qmap, kmap, nq, n, qtiles, row_tiles, k, w, ctx->dstatus, st); break;
-    case 3: e = launch_search_kernel<3>(qmap, kmap, nq, n, qtiles, row_tiles, k, w, ctx->dstatus, st); break;
-    case 4: e = launch_search_kernel<4>(qmap, kmap, nq, n, qtiles, row_tiles, k, w, ctx->dstatus, st); break;
-    case 5: e = launch_search_kernel<5>(qmap, kmap, nq, n, qtiles, row_tiles, k, w, ctx->dstatus, st); break;
-    case 6: e = launch_search_kernel<6>(qmap, kmap, nq, n, qtiles, row_tiles, k, w, ctx->dstatus, st); break;
-    case 7: e = launch_search_kernel<7>(qmap, kmap, nq, n, qtiles, row_tiles, k, w, ctx->dstatus, st); break;
-    default: e = launch_search_kernel<8>(qmap, kmap, nq, n, qtiles, row_tiles, k, w, ctx->dstatus, st); break;
-  }
-  if (e != cudaSuccess) return e;
   query_tables_kernel<<<unsigned((nq + kTabQueries - 1) / kTabQueries), 256, 0, st>>>(q, nq, ctx->d, ctx->m,
                                                                                        ctx->dR64, ctx->dP64, w.xy);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  prep_queries_kernel<<<unsigned((nq + 7) / 8), 256, 0, st>>>(w.xy, nq, ctx->d, ctx->m, kp, w.maxk, w.qw, w.qerr);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  CUtensorMap kmap;
+  if (!encode_fp16_map(&kmap, w.kw, kp, n_pad, kRT)) return cudaErrorInvalidValue;
+  const int64_t row_tiles = n_pad / kRT, qtiles = nq_pad / kQT;
+  switch (kb) {
+    case 1: e = launch_search_kernel<1>(kmap, w.qw, nq, n, qtiles, row_tiles, k, w, ctx->dstatus, st); break;
+    case 2: e = launch_search_kernel<2>(kmap, w.qw, nq, n, qtiles, row_tiles, k, w, ctx->dstatus, st); break;
+    case 3: e = launch_search_kernel<3>(kmap, w.qw, nq, n, qtiles, row_tiles, k, w, ctx->dstatus, st); break;
+    case 4: e = launch_search_kernel<4>(kmap, w.qw, nq, n, qtiles, row_tiles, k, w, ctx->dstatus, st); break;
+    case 5: e = launch_search_kernel<5>(kmap, w.qw, nq, n, qtiles, row_tiles, k, w, ctx->dstatus, st); break;
+    case 6: e = launch_search_kernel<6>(kmap, w.qw, nq, n, qtiles, row_tiles, k, w, ctx->dstatus, st); break;
+    case 7: e = launch_search_kernel<7>(kmap, w.qw, nq, n, qtiles, row_tiles, k, w, ctx->dstatus, st); break;
+    default: e = launch_search_kernel<8>(kmap, w.qw, nq, n, qtiles, row_tiles, k, w, ctx->dstatus, st); break;
+  }
+  if (e != cudaSuccess) return e;
   const size_t fsmem = size_t(2 * 256 + kCap) * 8 + size_t(kCap) * 8;
   cudaFuncSetAttribute(finish_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(fsmem));
   finish_kernel<<<unsigned(nq), kFinishThreads, fsmem, st>>>(ctx->d, ctx->m, ctx->bmse, k, n, payload, norms, w.xy,
