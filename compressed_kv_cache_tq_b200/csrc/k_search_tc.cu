@@ -44,6 +44,7 @@
 
 #include <algorithm>
 
+#include "search_units.h"
 #include "tc_sm100.cuh"
 #include "tq_device.cuh"
 #include "tq_internal.h"
@@ -261,48 +262,6 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 __device__ __forceinline__ float key_float(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
-
-// Work: unit (query tile, row tile).  The grid is cut into groups of G
-// consecutive CTAs and the query tiles into groups of G consecutive tiles.
-// Group g of the NG = ctas / G takes the contiguous units [U g / NG,
-// U (g + 1) / NG) of the U = ceil(qtiles / G) x row_tiles pairs (query-tile
-// group qg, row tile t), qg-major, and its member r works on query tile
-// G qg + r of each: a CTA keeps one query tile (or two) for long stretches,
-// and the G members of a group read the same row tiles in the same order, so
-// that all but the first find each tile in L2 (the row matrix crosses HBM
-// about ceil(qtiles / G) times instead of qtiles times).  A member whose
-// query tile is past the last one skips those units.  (A part-major
-// round-robin order that makes all CTAs stream the same rows at the same
-// time, restarting each query's running k-th best at every part, measured
-// slower: 17.0 against 13.7 ms at 10^6 x 10^4.)
-struct Units {
-  int64_t qtiles, row_tiles, u, u1;
-  int64_t qt, t;
-  int64_t G, r;
-  __device__ Units(int64_t qtiles_, int64_t row_tiles_, int64_t cta, int64_t ctas, int64_t G_)
-      : qtiles(qtiles_), row_tiles(row_tiles_), G(G_) {
-    const int64_t ng = ctas / G, g = cta / G;
-    r = cta - g * G;
-    const int64_t total = ((qtiles + G - 1) / G) * row_tiles;
-    u = total * g / ng - 1;
-    u1 = total * (g + 1) / ng;
-    qt = t = 0;
-  }
-  // advance to the next (query tile, row tile); false when done
-  __device__ bool next() {
-    while (++u < u1) {
-      const int64_t qg = u / row_tiles;
-      qt = qg * G + r;
-      if (qt >= qtiles) {   // no such tile: skip the rest of this query-tile group
-        u = (qg + 1) * row_tiles - 1;
-        continue;
-      }
-      t = u - qg * row_tiles;
-      return true;
-    }
-    return false;
-  }
-};
 
 template <int KB>
 __global__ void __launch_bounds__(kSearchThreads, 1) search_tc_kernel(
@@ -816,18 +775,6 @@ SearchWs search_ws(const tq_ctx* ctx, int64_t nq, int64_t n, void* base) {
   w.xy = reinterpret_cast<double*>(take(size_t(nq) * (ctx->d + ctx->m) * 8));
   w.total = off;
   return w;
-}
-
-// CTAs per group of the schedule above: groups of eight when there are enough
-// query tiles that an idle member (query tile past the end) costs little; the
-// grid is then the largest multiple of the group size that fits the SMs (144
-// of 148).  Measured at 10^6 rows x 10^4 queries (79 query tiles): 12.1 /
-// 13.5 ms (b = 2 / 4) for single CTAs, 11.9 / 13.4 for groups of four, 11.5 /
-// 12.6 for groups of eight.
-int64_t search_group(int64_t qtiles, int sms) {
-  int64_t g = qtiles >= 32 ? 8 : qtiles >= 16 ? 4 : qtiles >= 8 ? 2 : 1;
-  while (g > 1 && sms < g) g >>= 1;
-  return g;
 }
 
 template <int KB>
