@@ -7,7 +7,7 @@
 //                                64-channel groups (described further down).
 //
 // What it computes per key k (airosetta.com "Google TurboQuant", stage 1 and
-// stage 2; mooersco.com section 1.1 "rotated = key @ rotation"):
+// stage 2; mooersco.com section 1.1, the key multiplied by the rotation):
 //   y = R k                      (tcgen05 MMA: K R_hi^T + K R_lo^T, fp32 in TMEM)
 //   n = ||k||                    (from the key tile in shared memory, fp32)
 //   idx_j = #{i : t_i < y_j / n} (Lloyd-Max cell search in registers)

@@ -552,8 +552,8 @@ def split_dequantize(perm: np.ndarray, qz_hi: Quantized, qz_lo: Quantized, tb_hi
 # ---------------------------------------------------------------------------
 # Packed row layout (the library's documented storage format)
 #
-# The pages fix no storage layout (only "no per-block constants", i.e. the
-# codebook is global).  This is the format the C ABI documents, restated
+# The pages fix no storage layout (they only say that no constants are stored
+# per block, i.e. the codebook is global).  This is the format the C ABI documents, restated
 # here from its definition so that packed bytes can be compared exactly.
 #
 # d and m are multiples of 64.  A row holds one key: four "quarter" chunks
