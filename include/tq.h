@@ -12,8 +12,8 @@
  *         and section "第二階段：QJL" (1-bit sign sketch of the residual,
  *         unbiased inner-product estimator, O(d) per vector).
  *   [p1]  mooersco.com news article, section 1.1 (rotation preserves the L2
- *         norm; pseudocode "rotated = key @ rotation") and 2.2 (4-bit logits on
- *         GPU are memory-bandwidth bound).
+ *         norm; the key is multiplied by the rotation matrix) and 2.2 (4-bit
+ *         logits on GPU are memory-bandwidth bound).
  *   [p5]  zhengruan.com news, "第一步 / 第二步" (precomputed codebook; one bit
  *         for the residual direction combined with the full-precision query).
  *
@@ -77,9 +77,9 @@ typedef enum {
 typedef enum { TQ_F32 = 0, TQ_BF16 = 1 } tq_dtype;
 
 /* Build the data-oblivious parameters of one quantizer and upload them to
- * the current CUDA device ([p2] stage 1: "rotation via QR of a Gaussian
- * matrix", "Lloyd-Max, precomputed codebook"; [p2] stage 2: Gaussian JL
- * matrix).  R (d x d) is the orthogonal factor, with a positive triangular
+ * the current CUDA device ([p2] stage 1: a rotation from the QR factor of a
+ * Gaussian matrix and a precomputed Lloyd-Max codebook; [p2] stage 2: a
+ * Gaussian JL matrix).  R (d x d) is the orthogonal factor, with a positive triangular
  * diagonal, of a d x d Gaussian drawn from Philox4x32-10 stream 0 of `seed`;
  * P (m x d) is drawn from stream 1 and the JL matrix applied to the residual
  * is S = P R; the codebook has 2^(bits-1) Lloyd-Max levels for the law of one
