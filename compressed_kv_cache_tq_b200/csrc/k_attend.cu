@@ -31,6 +31,7 @@
 #include <math.h>
 
 #include "tq_device.cuh"
+#include "attend_plan.h"
 #include "tq_internal.h"
 
 namespace tq {
@@ -665,7 +666,7 @@ __global__ void __launch_bounds__(256) attend_combine_kernel(const float* __rest
   extern __shared__ float sv[];
   float* sa = sv;          // [dp] merged a, then u
   float* sb = sa + g.dp;   // [mp] merged b
-  __shared__ float sf[1024];   // per-split factors exp(m_i - M)
+  __shared__ float sf[kAttMaxSplits];   // per-split factors exp(m_i - M)
   __shared__ float sL;
   const int bh = blockIdx.x, b = bh / Hq, h = bh - b * Hq;
   const int G = Hq / Hkv, hkv = h / G, hl = h - hkv * G;
@@ -731,42 +732,13 @@ __global__ void __launch_bounds__(256) attend_combine_kernel(const float* __rest
                                                                  : sp[0][threadIdx.x];
 }
 
-struct AttPlan {
-  int nsplit;
-  int64_t chunk;
-};
-
-// Key chunks per (batch, KV head).  The time is the number of waves of
-// resident blocks (two per SM) times a block's time, taken as a fixed part
-// plus the chunk length.  The tensor-core kernel's fixed part (ring fill,
-// the merge of its warps' partial sums) was measured at the cost of about
-// 180 keys; the CUDA-core kernel's is charged as a small cost per split.
+// Key chunks per (batch, KV head): att_plan_for in attend_plan.h, with this
+// device's SM count.
 AttPlan att_plan(int B, int Hkv, int64_t S, bool mma) {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t groups = int64_t(B) * Hkv;
-  const int64_t cap = int64_t(sms) * 2;
-  int64_t max_ns = (S + kAttTile - 1) / kAttTile;
-  if (max_ns > 1024) max_ns = 1024;
-  if (max_ns < 1) max_ns = 1;
-  int64_t best = 1;
-  double best_cost = 1e300;
-  for (int64_t ns = 1; ns <= max_ns; ++ns) {
-    const double waves = double((groups * ns + cap - 1) / cap);
-    const double cost = mma ? waves * (180.0 + double(S) / double(ns))
-                            : waves / double(ns) + 0.0002 * double(ns);
-    if (cost < best_cost) {
-      best_cost = cost;
-      best = ns;
-    }
-  }
-  int64_t chunk = (S + best - 1) / best;
-  chunk = (chunk + kAttTile - 1) / kAttTile * kAttTile;
-  if (chunk < kAttTile) chunk = kAttTile;
-  int64_t ns = (S + chunk - 1) / chunk;
-  if (ns < 1) ns = 1;
-  return AttPlan{int(ns), chunk};
+  return att_plan_for(B, Hkv, S, mma, sms, kAttTile);
 }
 
 // The tensor-core kernel serves d = m = 128 (or m = 0) with up to 4 query
